@@ -1,0 +1,426 @@
+#!/usr/bin/env python
+"""Benchmark: GPTQ quantization of one linear layer on B200.
+
+One step = the whole hot path on one layer, inputs resident in HBM:
+  H = 0;  H += 2 X X^T            (gptq_hessian_accumulate, tcgen05 SYRK)
+  dead / act-order / damping / U  (gptq_cholesky_inverse)
+  column sweep + lazy updates     (gptq_quantize_layer)
+  int4 packing                    (gptq_pack_int4)
+  dequantization to bf16          (gptq_dequant)
+The default workload is the Llama-7B q_proj shape: W 4096x4096 bf16, X 4096
+features x 262144 tokens bf16 (128 x 2048) with 8 outlier channels x20,
+4-bit, group 128, act-order.  value = weights quantized per second over the
+whole job (all ranks).  Under torchrun each rank quantizes its own replica
+(the layer does not shard; no collective on the data path).
+
+`--impl reference` times the fp64 CPU oracle instead, on a bounded sample of
+the same workload per step (see cpu_sample()).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "weights quantized/sec (GPTQ 4-bit g128) + Hessian TFLOP/s, % of roofline, 1×B200"
+UNIT = "weights/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="q_proj_7b")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        d["_source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["_source"] = "fallback"
+    return d
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def describe(wl) -> str:
+    s = (f"{wl.name}: W {wl.rows}x{wl.n} {str(wl.w_dtype).split('.')[-1]}, X {wl.n}x{wl.ntok} "
+         f"{str(wl.x_dtype).split('.')[-1]}")
+    if wl.outliers:
+        s += f" ({wl.outliers} outlier channels x{wl.outlier_gain:g})"
+    g = "per-row" if wl.group_size <= 0 else f"g{wl.group_size}"
+    s += f", {wl.bits}-bit {g}{' act-order' if wl.actorder else ''}, damp {wl.percdamp:g}, block {wl.block}"
+    return s
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- oracle sample
+def cpu_sample(wl, W, X, tok_sample: int, row_sample: int):
+    """Time the fp64 oracle on a bounded sample of the workload and scale it
+    to the whole layer: H on `tok_sample` tokens (cost linear in tokens), U
+    in full, sweep + packing on `row_sample` rows (rows are independent once
+    U is known).  Returns (weights/s, description, seconds spent)."""
+    import numpy as np
+    from oracle import gptq_oracle as O
+
+    t_all = time.perf_counter()
+    Xs = X[:, :tok_sample].float().cpu().numpy()
+    Ws = W[:row_sample].float().cpu().numpy().astype(np.float64)
+    t0 = time.perf_counter()
+    Hs = O.hessian(Xs)
+    t_h = (time.perf_counter() - t0) * (wl.ntok / tok_sample)
+    Hfull = Hs * (wl.ntok / tok_sample)          # a stand-in of the right scale for U
+    t0 = time.perf_counter()
+    prep = O.prepare(Hfull, Ws, wl.percdamp, wl.actorder)
+    U = O.upper_cholesky_of_inverse(prep["Hp"])
+    t_u = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    res = O.sweep(prep["Wp"], U, wl.bits, wl.group_size)
+    codes = np.empty_like(res["codes"])
+    codes[:, prep["perm"]] = res["codes"]
+    if wl.bits == 4:
+        packed = O.pack_int4(codes)
+    else:
+        packed = O.pack_int3(codes)
+    O.dequant(packed, wl.bits, wl.n, res["scales"], res["zeros"], wl.group_size)
+    t_s = (time.perf_counter() - t0) * (wl.rows / row_sample)
+    total = t_h + t_u + t_s
+    desc = (f"fp64 NumPy oracle: H on {tok_sample} of {wl.ntok} tokens (time x{wl.ntok / tok_sample:g}), "
+            f"U in full (n={wl.n}), unblocked sweep + pack + dequant on {row_sample} of {wl.rows} rows "
+            f"(time x{wl.rows / row_sample:g}); extrapolated layer time {total:.1f} s")
+    return wl.rows * wl.n / total, desc, time.perf_counter() - t_all
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            return max(i.get("num_threads", 1) for i in info)
+    except Exception:
+        pass
+    return host_cores()
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import post_weight_quantization_25_b200 as G
+    import workloads
+
+    torch.cuda.set_device(local_rank)
+    wl = workloads.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local_rank)
+    W, X = workloads.make_inputs(wl, device=dev)
+    rows, n, N = wl.rows, wl.n, wl.ntok
+    cfg = G.make_config(wl.bits, wl.group_size, wl.percdamp, wl.actorder)
+    G_ = 1 if wl.group_size <= 0 else (n + wl.group_size - 1) // wl.group_size
+
+    H = torch.empty(n, n, dtype=torch.float32, device=dev)
+    U = torch.empty(n, n, dtype=torch.float32, device=dev)
+    perm = torch.empty(n, dtype=torch.int32, device=dev)
+    dead = torch.empty(n, dtype=torch.uint8, device=dev)
+    info = torch.zeros(1, dtype=torch.int32, device=dev)
+    info_h = torch.zeros(1, dtype=torch.int32, device=dev)
+    codes = torch.empty(rows, n, dtype=torch.uint8, device=dev)
+    scales = torch.empty(rows, G_, dtype=torch.float32, device=dev)
+    zeros = torch.empty(rows, G_, dtype=torch.uint8, device=dev)
+    g_idx = torch.empty(n, dtype=torch.int32, device=dev)
+    pack = G.gptq_pack_int4 if wl.bits == 4 else G.gptq_pack_int3
+    packed = torch.empty(rows, n * wl.bits // 32, dtype=torch.int32, device=dev)
+    deq = torch.empty(rows, n, dtype=torch.bfloat16, device=dev)
+    from post_weight_quantization_25_b200._lib import GPTQ_OP_CHOLESKY, GPTQ_OP_HESSIAN, GPTQ_OP_QUANTIZE
+    ws_h = torch.empty(G.gptq_workspace_size(GPTQ_OP_HESSIAN, 0, n, N, X.dtype) + 512,
+                       dtype=torch.uint8, device=dev)
+    ws_c = torch.empty(G.gptq_workspace_size(GPTQ_OP_CHOLESKY, 0, n) + 512, dtype=torch.uint8,
+                       device=dev)
+    ws_q = torch.empty(G.gptq_workspace_size(GPTQ_OP_QUANTIZE, rows, n, 0, torch.bfloat16, cfg)
+                       + 512, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        H.zero_()
+        if ev:
+            ev[0].record(stream)
+        G.gptq_hessian_accumulate(H, X, 2.0, ws=ws_h, info=info_h, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        G.gptq_cholesky_inverse(H, wl.percdamp, wl.actorder, U, perm, dead, info, ws=ws_c,
+                                stream=stream)
+        if ev:
+            ev[2].record(stream)
+        G.gptq_quantize_layer(W, U, perm, dead, cfg, codes, scales, zeros, g_idx, ws=ws_q,
+                              stream=stream)
+        if ev:
+            ev[3].record(stream)
+        pack(codes, packed, stream=stream)
+        if ev:
+            ev[4].record(stream)
+        G.gptq_dequant(packed, wl.bits, n, scales, zeros, wl.group_size, g_idx, torch.bfloat16,
+                       out=deq, stream=stream)
+        if ev:
+            ev[5].record(stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if int(info.item()) != 0 or int(info_h.item()) != 0:
+        raise RuntimeError(f"device status: cholesky info {int(info.item())}, "
+                           f"hessian info {int(info_h.item())}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = G.gptq_launch_count()
+    with ClockSampler(local_rank) as clk:
+        t_start.record(stream)
+        for k in range(args.steps):
+            step(evs[k])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    launches = G.gptq_launch_count() - launches0
+    ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    names = ["hessian", "cholesky_inverse", "sweep", "pack", "dequant"]
+    stage = {nm: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+             for i, nm in enumerate(names)}
+    ms_step = ms / args.steps
+    value = world * rows * n * args.steps / (ms / 1e3)
+    flops = float(n) * (n + 1) * N
+    t_h = stage["hessian"] / 1e3
+    pk = peaks()
+    achieved = flops / t_h / 1e12
+    traffic = None
+    tf_path = os.path.join(ROOT, "profiles", "syrk_traffic.json")
+    if os.path.exists(tf_path):
+        with open(tf_path) as f:
+            tj = json.load(f)
+        if tj.get("workload") == wl.name and tj.get("kernel_rev") == "syrk-v1":
+            traffic = tj.get("bytes_per_launch")
+    roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": traffic,
+            "kernel": "syrk_bf16_kernel (+ mirror) in gptq_hessian_accumulate",
+            "peak_source": f"{pk['_source']} bf16 burst", "algorithmic_flops": flops}
+
+    # end to end through the same C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        Xh = torch.empty_like(X, device="cpu").pin_memory()
+        Xh.copy_(X)
+        Wh = torch.empty_like(W, device="cpu").pin_memory()
+        Wh.copy_(W)
+        outs = [packed, scales, zeros, g_idx]
+        outs_h = [torch.empty_like(t, device="cpu").pin_memory() for t in outs]
+        Xd = torch.empty_like(X)
+        Wd = torch.empty_like(W)
+
+        def e2e_step():
+            Xd.copy_(Xh, non_blocking=True)
+            Wd.copy_(Wh, non_blocking=True)
+            H.zero_()
+            G.gptq_hessian_accumulate(H, Xd, 2.0, ws=ws_h, info=info_h, stream=stream)
+            G.gptq_cholesky_inverse(H, wl.percdamp, wl.actorder, U, perm, dead, info, ws=ws_c,
+                                    stream=stream)
+            G.gptq_quantize_layer(Wd, U, perm, dead, cfg, codes, scales, zeros, g_idx, ws=ws_q,
+                                  stream=stream)
+            pack(codes, packed, stream=stream)
+            G.gptq_dequant(packed, wl.bits, n, scales, zeros, wl.group_size, g_idx,
+                           torch.bfloat16, out=deq, stream=stream)
+            for t, th in zip(outs, outs_h):
+                th.copy_(t, non_blocking=True)
+
+        for _ in range(max(1, min(args.warmup, 2))):
+            e2e_step()
+        barrier()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            ems = float(t.item())
+        h2d = X.numel() * X.element_size() + W.numel() * W.element_size()
+        d2h = sum(t.numel() * t.element_size() for t in outs)
+        e2e = {"value": world * rows * n * args.steps / (ems / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": ems / args.steps}
+        del Xh, Wh, Xd, Wd
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, _ = cpu_sample(wl, W, X, tok_sample=4096, row_sample=64)
+        cpu = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 in / f32", "data": "synthetic",
+            "config": {"workload": describe(wl), "rows": rows, "n": n, "tokens": N,
+                       "bits": wl.bits, "group_size": wl.group_size, "actorder": wl.actorder,
+                       "l2": "inputs larger than L2 (X is %.2f GB)" % (X.numel() * 2 / 1e9),
+                       "parallelism": f"{world} independent replicas"},
+            "hessian_tflops": achieved,
+            "stage_ms": {k: round(v, 4) for k, v in stage.items()},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import torch
+    import workloads
+
+    wl = workloads.WORKLOADS[args.workload]
+    W = workloads.make_weights(wl, "cpu", rows=16)
+    X = workloads.make_calibration(wl, "cpu", ntok=2048)
+    times = []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        v, desc, _ = cpu_sample(wl, W, X, tok_sample=2048, row_sample=16)
+        if i >= args.warmup:
+            times.append(wl.rows * wl.n / v)
+    t = statistics.mean(times)
+    value = wl.rows * wl.n / t
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": describe(wl), "rows": wl.rows, "n": wl.n,
+                       "tokens": wl.ntok, "bits": wl.bits, "group_size": wl.group_size,
+                       "actorder": wl.actorder, "parallelism": "rank 0 only"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,185 @@
+/*
+ * gptq.h -- C ABI of libgptq_b200.so, a GPTQ layer-wise weight quantizer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method is the one described on the web page "GPTQ, with the code open"
+ * (modelfoundations.com/notes/gptq): per linear layer, accumulate the
+ * calibration Hessian H = 2 X X^T; zero dead inputs, optionally reorder the
+ * columns by descending diag(H) ("act-order"), add 1 % of the mean diagonal
+ * ("damping"); take the upper Cholesky factor U of H^-1; sweep the columns
+ * left to right, rounding each to an asymmetric min-max grid ("ruler") and
+ * spreading its rounding error over the columns not yet quantized, with the
+ * repairs past the current block of 128 columns deferred to one product per
+ * block; store tick indices plus a per-row or per-group ruler.
+ *
+ * Conventions shared by every entry point:
+ *  - Every pointer argument is DEVICE memory owned by the caller unless the
+ *    comment says otherwise.  The library allocates nothing that outlives a
+ *    call and keeps no state between calls (apart from the launch counter
+ *    read by gptq_launch_count).
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream).  The returned status covers argument checks and
+ *    kernel launches only.  Numerical failures and device-side wait timeouts
+ *    are written to the caller's device `info` word (0 = no failure).
+ *  - Matrices are row-major and dense: a rows x cols matrix has its element
+ *    (r, c) at offset r*ld + c, with ld = cols unless a leading dimension is
+ *    passed.
+ *  - n (input features, columns of W, size of H) indexes the SWEEP ORDER
+ *    after act-order wherever the comment says "sweep order".
+ */
+#ifndef GPTQ_B200_H
+#define GPTQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GPTQ_OK = 0,
+  GPTQ_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned buffer      */
+  GPTQ_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement    */
+  GPTQ_ERR_WORKSPACE = 3,    /* workspace smaller than gptq_workspace_size()   */
+  GPTQ_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed    */
+  GPTQ_ERR_TIMEOUT = 5       /* (device `info` value) a bounded wait ran out   */
+} gptq_status;
+
+typedef enum { GPTQ_BF16 = 0, GPTQ_F32 = 1 } gptq_dtype;
+
+/* Quantizer settings (page "What is GPTQ", table "Key settings"; page "GPTQ,
+ * with the code open", section "Paper vs. code").
+ *   bits        2..8; the packers handle 3 and 4.
+ *   group_size  -1 = one ruler per row, fitted before the sweep on the
+ *               unrepaired weights; otherwise a new ruler every group_size
+ *               columns of the sweep order, fitted when the sweep reaches the
+ *               group's first column, on the current (repaired) weights.
+ *               Supported: 32, 64, 128 or any multiple of 128.
+ *   percdamp    damping as a fraction of mean(diag H); 0.01 in the pages.
+ *   block       lazy-update block; must be 128.
+ *   actorder    nonzero: sweep columns in order of descending diag(H).
+ *   sym         must be 0 (asymmetric ruler). */
+typedef struct {
+  int bits;
+  int group_size;
+  float percdamp;
+  int block;
+  int actorder;
+  int sym;
+} gptq_config;
+
+typedef enum { GPTQ_OP_HESSIAN = 0, GPTQ_OP_CHOLESKY = 1, GPTQ_OP_QUANTIZE = 2 } gptq_op;
+
+/* Bytes of device workspace `op` needs for these sizes (0 is possible).
+ * rows/n/ntok as in the calls below; xt is the calibration dtype (hessian
+ * only); cfg may be NULL except for GPTQ_OP_QUANTIZE.  Host pointer `bytes`. */
+gptq_status gptq_workspace_size(int op, int64_t rows, int64_t n, int64_t ntok, gptq_dtype xt,
+                                const gptq_config* cfg, size_t* bytes);
+
+/* H += alpha * X X^T     (page "GPTQ, with the code open", section "Measuring
+ * damage where it matters": H = 2 X X^T; section "Paper vs. code": H is built
+ * up over calibration batches -- call once per batch; alpha = 2 gives the sum
+ * form).
+ *   H      n x n fp32.  Must be symmetric on entry (e.g. zeroed); on return
+ *          it is symmetric: the upper triangle is accumulated and mirrored.
+ *   X      n x ntok, features x tokens, row stride ldx elements (ldx >= ntok),
+ *          dtype xt.  bf16: the products are exact in fp32 and summed in fp32
+ *          on the tensor cores.  fp32: each value is split into two bf16
+ *          parts hi + lo and H gets hi hi^T + hi lo^T + lo hi^T.
+ *          Requirements: X 16-byte aligned, ldx * sizeof(element) a multiple
+ *          of 16 bytes; H 16-byte aligned.
+ *   token_major  must be 0.
+ *   ws     workspace of gptq_workspace_size(GPTQ_OP_HESSIAN, 0, n, ntok, xt)
+ *          bytes (0 for bf16).
+ *   info   optional device int32: set to GPTQ_ERR_TIMEOUT if a pipeline wait
+ *          inside the kernel gave up (then H is incomplete).  Not cleared.  */
+gptq_status gptq_hessian_accumulate(float* H, const void* X, gptq_dtype xt, int64_t n,
+                                    int64_t ntok, int64_t ldx, int token_major, float alpha,
+                                    void* ws, size_t ws_bytes, int32_t* info, void* stream);
+
+/* Preparation and the upper Cholesky factor of the damped inverse
+ * (page "GPTQ, with the code open", sections "From one repair to a whole
+ * model" and "Paper vs. code"):
+ *   dead[i]  = diag(H)_i == 0; such diagonal entries are set to 1 (their
+ *              weight columns are zeroed by gptq_quantize_layer);
+ *   perm     = identity, or with actorder a stable sort of the columns by
+ *              descending diag(H) (after the dead fix): perm[k] is the
+ *              original column quantized k-th;
+ *   H'       = H[perm][:, perm] + lambda I, lambda = percdamp * mean(diag H);
+ *   U        n x n fp32, upper triangular (strict lower part written as 0),
+ *              in sweep order, with H'^-1 = U^T U.
+ * H (n x n fp32, symmetric) is read, not modified.
+ * perm may be NULL only when actorder == 0.  dead: uint8[n].
+ * info (device int32, required): 0 on success; k > 0 if H' was found not
+ * positive definite at sweep position k - 1 (the factorisation runs from the
+ * last sweep position towards the first, so this is the highest failing
+ * position); -1 if diag(H) holds a NaN or an infinity.  On failure U is
+ * undefined.  ws: gptq_workspace_size(GPTQ_OP_CHOLESKY, 0, n, 0, .., NULL). */
+gptq_status gptq_cholesky_inverse(const float* H, int64_t n, float percdamp, int actorder,
+                                  float* U, int32_t* perm, uint8_t* dead, int32_t* info,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/* The column sweep with lazy block updates (page "GPTQ, with the code open",
+ * sections "The repair rule", "From one repair to a whole model" and "What
+ * quantization is, and why anyone bothers").  For each column j of the sweep
+ * order, for every row:
+ *   scale = (xmax - xmin) / (2^bits - 1), zero = rint(-xmin / scale) with
+ *   [xmin, xmax] the ruler's range stretched to include 0 ([-1, 1] if flat);
+ *   q = clamp(rint(w / scale) + zero, 0, 2^bits - 1);  w_hat = scale (q - zero);
+ *   err = (w - w_hat) / U[j][j];  W[:, j+1:] -= err * U[j, j+1:]
+ * with the update past the current 128-column block applied once per block.
+ * All arithmetic is fp32 with IEEE division and round-half-to-even.
+ *   W        rows x n in wt (original column order); not modified.
+ *   U, perm, dead  from gptq_cholesky_inverse (perm may be NULL = identity).
+ *   codes    uint8 rows x n, ORIGINAL column order.
+ *   scales   fp32 rows x G, zeros uint8 rows x G, G = ceil(n / group_size)
+ *            (1 for per-row rulers), in sweep order of the groups.
+ *   g_idx    optional int32[n]: group of each original column.
+ *   Wq       optional fp32 rows x n, original order: the dequantized weights.
+ *   row_loss optional fp32[rows]: sum over columns of (w - w_hat)^2 / (2 U_jj^2).
+ *   ws       gptq_workspace_size(GPTQ_OP_QUANTIZE, rows, n, 0, .., cfg). */
+gptq_status gptq_quantize_layer(const void* W, gptq_dtype wt, int64_t rows, int64_t n,
+                                const float* U, const int32_t* perm, const uint8_t* dead,
+                                const gptq_config* cfg, uint8_t* codes, float* scales,
+                                uint8_t* zeros, int32_t* g_idx, float* Wq, float* row_loss,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* Packed storage of tick indices (page "GPTQ, with the code open", section
+ * "What quantization is, and why anyone bothers": store the tick index).  The
+ * bit layout is this library's own:
+ *   int4: column 8i+k of a row -> bits [4k, 4k+4) of uint32 word i of the row
+ *         (n % 8 == 0; out is rows x n/8).
+ *   int3: column 32i+k -> bits [3k, 3k+3) of the 96-bit little-endian word
+ *         formed by uint32 words 3i, 3i+1, 3i+2 of the row (n % 32 == 0; out is
+ *         rows x 3n/32).  Codes are masked to their low 4 (3) bits. */
+gptq_status gptq_pack_int4(const uint8_t* codes, int64_t rows, int64_t n, uint32_t* out,
+                           void* stream);
+gptq_status gptq_pack_int3(const uint8_t* codes, int64_t rows, int64_t n, uint32_t* out,
+                           void* stream);
+
+/* w_hat[r][c] = scale[r][G(c)] * (code[r][c] - zero[r][G(c)])  -- one fp32
+ * multiply (section "What quantization is, and why anyone bothers": turning
+ * an integer back into a number is one multiply); ot = GPTQ_BF16 rounds that
+ * fp32 value to bfloat16, half to even.  G(c) = g_idx[c] if g_idx is given,
+ * else c / group_size, or 0 when group_size <= 0.  packed in the layout of
+ * gptq_pack_int4 / gptq_pack_int3 (bits 4 or 3); scales fp32 and zeros uint8
+ * are rows x G with row stride G = ceil(n / group_size) (1 if per row) --
+ * pass n_groups explicitly when g_idx is used.  out: rows x n of ot. */
+gptq_status gptq_dequant(const uint32_t* packed, int bits, int64_t rows, int64_t n,
+                         const float* scales, const uint8_t* zeros, int group_size,
+                         int64_t n_groups, const int32_t* g_idx, void* out, gptq_dtype ot,
+                         void* stream);
+
+/* Static string for a status code (host). */
+const char* gptq_status_string(int status);
+
+/* Diagnostics (host): number of kernels this library has enqueued in this
+ * process so far.  The one piece of process-wide state the library keeps. */
+int64_t gptq_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ_B200_H */

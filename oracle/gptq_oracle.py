@@ -69,10 +69,24 @@ def hessian(X: np.ndarray, alpha: float = 2.0, token_chunk: int = 8192) -> np.nd
     X = np.asarray(X)
     n, ntok = X.shape
     H = np.zeros((n, n), dtype=np.float64)
+    syrk = _blas_syrk()
     for t0 in range(0, ntok, token_chunk):
         Xc = X[:, t0:t0 + token_chunk].astype(np.float64)
-        H += Xc @ Xc.T
+        if syrk is not None and n >= 512:
+            # the same product through BLAS's symmetric rank-k routine (upper half)
+            Hu = syrk(1.0, np.asfortranarray(Xc))
+            H += np.triu(Hu) + np.triu(Hu, 1).T
+        else:
+            H += Xc @ Xc.T
     return alpha * H
+
+
+def _blas_syrk():
+    try:
+        from scipy.linalg.blas import dsyrk
+    except Exception:  # pragma: no cover - scipy is optional
+        return None
+    return dsyrk
 
 
 def hessian_entry(X: np.ndarray, i: int, j: int, alpha: float = 2.0) -> float:
@@ -124,13 +138,30 @@ def dequantize(q, scale, zero) -> np.ndarray:
 # --------------------------------------------------------------------------
 # Preparation  (§ "Paper vs. code": dead inputs, damping, act-order)
 # --------------------------------------------------------------------------
-def prepare(H: np.ndarray, W: np.ndarray, percdamp: float = 0.01, actorder: bool = False):
+def is_near_tie_order(d: np.ndarray, order, rtol: float) -> bool:
+    """True if ``order`` is a permutation that sorts ``d`` descending except
+    between entries within a relative ``rtol`` of each other."""
+    order = np.asarray(order, dtype=np.int64)
+    n = d.shape[0]
+    if order.shape != (n,) or not np.array_equal(np.sort(order), np.arange(n)):
+        return False
+    a, b = d[order[:-1]], d[order[1:]]
+    return bool(np.all(a >= b - rtol * np.maximum(np.abs(a), np.abs(b))))
+
+
+def prepare(H: np.ndarray, W: np.ndarray, percdamp: float = 0.01, actorder: bool = False,
+            forced_perm=None, perm_rtol: float = 1e-5):
     """Dead inputs -> act-order -> damping.
 
     Returns dict with ``dead`` (bool[n]), ``perm`` (int64[n], perm[k] = the
     original column quantized k-th), ``Hp`` (damped H in sweep order),
     ``W0`` (dead-zeroed W, original order), ``Wp`` (W0 in sweep order) and
     ``lam`` (the damping added to every diagonal entry).
+
+    ``forced_perm`` replays another run's act-order: it is adopted when it
+    orders diag(H) descending up to ties within ``perm_rtol`` (two Hessians
+    summed in different precisions may order such near-equal columns either
+    way); otherwise ValueError.
     """
     H = np.array(H, dtype=np.float64, copy=True)
     W0 = np.array(W, dtype=np.float64, copy=True)
@@ -141,6 +172,10 @@ def prepare(H: np.ndarray, W: np.ndarray, percdamp: float = 0.01, actorder: bool
     W0[:, dead] = 0.0
     if actorder:
         perm = np.argsort(-np.diag(H), kind="stable")
+        if forced_perm is not None:
+            if not is_near_tie_order(np.diag(H), forced_perm, perm_rtol):
+                raise ValueError("forced act-order is not a near-tie reordering of diag(H)")
+            perm = np.asarray(forced_perm, dtype=np.int64)
     else:
         perm = np.arange(n)
     Hp = H[np.ix_(perm, perm)]
@@ -319,15 +354,17 @@ def rtn(Wp: np.ndarray, bits: int, group_size: int = -1):
 # --------------------------------------------------------------------------
 def gptq_layer(W: np.ndarray, H: np.ndarray, bits: int = 4, group_size: int = -1,
                percdamp: float = 0.01, actorder: bool = False,
-               forced_codes=None, forced_zeros=None, tau: float = 1e-3):
+               forced_codes=None, forced_zeros=None, tau: float = 1e-3,
+               forced_perm=None, perm_rtol: float = 1e-5):
     """GPTQ on one linear layer, given its Hessian H (n x n) and weights W.
 
     Returns the sweep's dict plus, in ORIGINAL column order: ``codes_orig``,
     ``Wq_orig`` and ``g_idx`` (group of each original column), and the
     preparation's ``dead``, ``perm``, ``lam``, ``U``, ``W0``.  Forced
-    codes/zeros are given in sweep order.
+    codes/zeros are given in sweep order (see ``sweep``); ``forced_perm`` as
+    in ``prepare``.
     """
-    prep = prepare(H, W, percdamp, actorder)
+    prep = prepare(H, W, percdamp, actorder, forced_perm, perm_rtol)
     U = upper_cholesky_of_inverse(prep["Hp"])
     res = sweep(prep["Wp"], U, bits, group_size, forced_codes, forced_zeros, tau)
     perm = prep["perm"]

@@ -1,0 +1,256 @@
+"""GPTQ layer-wise weight quantizer for NVIDIA B200 -- Python binding.
+
+Every function named ``gptq_*`` here marshals torch tensors into the C entry
+point of the same name in ``libgptq_b200.so`` (declared in include/gptq.h)
+and raises ``GptqError`` on a non-OK status.  All the arithmetic runs in the
+library's CUDA kernels; PyTorch only provides device memory and streams.
+
+``quantize_linear`` chains the calls for one linear layer, the way the page
+"GPTQ, with the code open" describes the method: H from the calibration
+inputs, the Cholesky factor of the damped inverse, the column sweep, packed
+codes.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+
+import torch
+
+from . import _lib
+from ._lib import (GPTQ_BF16, GPTQ_F32, GPTQ_OP_CHOLESKY, GPTQ_OP_HESSIAN, GPTQ_OP_QUANTIZE,
+                   GptqConfig)
+
+__all__ = ["GptqError", "GptqConfig", "gptq_workspace_size", "gptq_hessian_accumulate",
+           "gptq_cholesky_inverse", "gptq_quantize_layer", "gptq_pack_int4", "gptq_pack_int3",
+           "gptq_dequant", "gptq_status_string", "make_config", "QuantizedLinear",
+           "quantize_linear", "library"]
+
+
+class GptqError(RuntimeError):
+    pass
+
+
+def library() -> ctypes.CDLL:
+    return _lib.load()
+
+
+def gptq_status_string(status: int) -> str:
+    return library().gptq_status_string(int(status)).decode()
+
+
+def gptq_launch_count() -> int:
+    """Kernels the library has enqueued in this process so far."""
+    return int(library().gptq_launch_count())
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise GptqError(f"{what}: {gptq_status_string(status)} (status {status})")
+
+
+def _p(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return GPTQ_BF16
+    if dt == torch.float32:
+        return GPTQ_F32
+    raise GptqError(f"unsupported dtype {dt} (bf16 or fp32)")
+
+
+def _need_cuda(*ts) -> None:
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise GptqError("tensors must live on the GPU")
+
+
+def make_config(bits=4, group_size=128, percdamp=0.01, actorder=False, block=128,
+                sym=False) -> GptqConfig:
+    return GptqConfig(int(bits), int(group_size), float(percdamp), int(block), int(bool(actorder)),
+                      int(bool(sym)))
+
+
+def gptq_workspace_size(op: int, rows: int, n: int, ntok: int = 0,
+                        xdtype: torch.dtype = torch.bfloat16, cfg: GptqConfig | None = None) -> int:
+    out = ctypes.c_size_t(0)
+    st = library().gptq_workspace_size(int(op), int(rows), int(n), int(ntok), _dtype_code(xdtype),
+                                       ctypes.byref(cfg) if cfg is not None else None,
+                                       ctypes.byref(out))
+    _check(st, "gptq_workspace_size")
+    return int(out.value)
+
+
+def _workspace(nbytes: int, device, ws):
+    if nbytes == 0:
+        return ws
+    if ws is not None and ws.numel() >= nbytes:
+        return ws
+    return torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+
+
+def _aligned_ptr(ws) -> tuple[int | None, int]:
+    if ws is None:
+        return None, 0
+    p = ws.data_ptr()
+    off = (-p) % 256
+    return p + off, ws.numel() - off
+
+
+def gptq_hessian_accumulate(H: torch.Tensor, X: torch.Tensor, alpha: float = 2.0, ws=None,
+                            info: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """H += alpha * X X^T for X (n features x N tokens, bf16 or fp32); returns H."""
+    _need_cuda(H, X, info)
+    n, ntok = X.shape
+    if H.dtype != torch.float32 or H.shape != (n, n) or not H.is_contiguous():
+        raise GptqError("H must be a contiguous n x n float32 tensor")
+    if X.stride(1) != 1:
+        raise GptqError("X must have contiguous rows (tokens)")
+    need = gptq_workspace_size(GPTQ_OP_HESSIAN, 0, n, ntok, X.dtype)
+    ws = _workspace(need, X.device, ws)
+    wp, wn = _aligned_ptr(ws) if need else (None, 0)
+    st = library().gptq_hessian_accumulate(_p(H), _p(X), _dtype_code(X.dtype), n, ntok,
+                                           X.stride(0), 0, float(alpha), wp, wn, _p(info),
+                                           _stream(stream))
+    _check(st, "gptq_hessian_accumulate")
+    return H
+
+
+def gptq_cholesky_inverse(H: torch.Tensor, percdamp: float = 0.01, actorder: bool = False,
+                          U=None, perm=None, dead=None, info=None, ws=None, stream=None):
+    """Dead inputs, act-order, damping and U (upper, H'^-1 = U^T U).
+    Returns (U, perm, dead, info); info is a device int32 (0 = success)."""
+    _need_cuda(H)
+    n = H.shape[0]
+    dev = H.device
+    U = torch.empty(n, n, dtype=torch.float32, device=dev) if U is None else U
+    perm = torch.empty(n, dtype=torch.int32, device=dev) if perm is None else perm
+    dead = torch.empty(n, dtype=torch.uint8, device=dev) if dead is None else dead
+    info = torch.empty(1, dtype=torch.int32, device=dev) if info is None else info
+    need = gptq_workspace_size(GPTQ_OP_CHOLESKY, 0, n)
+    ws = _workspace(need, dev, ws)
+    wp, wn = _aligned_ptr(ws)
+    st = library().gptq_cholesky_inverse(_p(H), n, float(percdamp), int(bool(actorder)), _p(U),
+                                         _p(perm), _p(dead), _p(info), wp, wn, _stream(stream))
+    _check(st, "gptq_cholesky_inverse")
+    return U, perm, dead, info
+
+
+def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, perm, dead, cfg: GptqConfig,
+                        codes=None, scales=None, zeros=None, g_idx=None, Wq=None, row_loss=None,
+                        want_g_idx: bool = True, want_wq: bool = False, want_loss: bool = False,
+                        ws=None, stream=None) -> dict:
+    """The column sweep.  Returns dict(codes, scales, zeros, g_idx, Wq, row_loss)."""
+    _need_cuda(W, U, perm, dead)
+    rows, n = W.shape
+    if not W.is_contiguous():
+        raise GptqError("W must be contiguous")
+    dev = W.device
+    G = 1 if cfg.group_size <= 0 else (n + cfg.group_size - 1) // cfg.group_size
+    codes = torch.empty(rows, n, dtype=torch.uint8, device=dev) if codes is None else codes
+    scales = torch.empty(rows, G, dtype=torch.float32, device=dev) if scales is None else scales
+    zeros = torch.empty(rows, G, dtype=torch.uint8, device=dev) if zeros is None else zeros
+    if g_idx is None and want_g_idx:
+        g_idx = torch.empty(n, dtype=torch.int32, device=dev)
+    if Wq is None and want_wq:
+        Wq = torch.empty(rows, n, dtype=torch.float32, device=dev)
+    if row_loss is None and want_loss:
+        row_loss = torch.empty(rows, dtype=torch.float32, device=dev)
+    need = gptq_workspace_size(GPTQ_OP_QUANTIZE, rows, n, 0, torch.bfloat16, cfg)
+    ws = _workspace(need, dev, ws)
+    wp, wn = _aligned_ptr(ws)
+    st = library().gptq_quantize_layer(_p(W), _dtype_code(W.dtype), rows, n, _p(U), _p(perm),
+                                       _p(dead), ctypes.byref(cfg), _p(codes), _p(scales),
+                                       _p(zeros), _p(g_idx), _p(Wq), _p(row_loss), wp, wn,
+                                       _stream(stream))
+    _check(st, "gptq_quantize_layer")
+    return {"codes": codes, "scales": scales, "zeros": zeros, "g_idx": g_idx, "Wq": Wq,
+            "row_loss": row_loss}
+
+
+def gptq_pack_int4(codes: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    _need_cuda(codes)
+    rows, n = codes.shape
+    out = torch.empty(rows, n // 8, dtype=torch.int32, device=codes.device) if out is None else out
+    _check(library().gptq_pack_int4(_p(codes), rows, n, _p(out), _stream(stream)),
+           "gptq_pack_int4")
+    return out
+
+
+def gptq_pack_int3(codes: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    _need_cuda(codes)
+    rows, n = codes.shape
+    out = (torch.empty(rows, 3 * n // 32, dtype=torch.int32, device=codes.device)
+           if out is None else out)
+    _check(library().gptq_pack_int3(_p(codes), rows, n, _p(out), _stream(stream)),
+           "gptq_pack_int3")
+    return out
+
+
+def gptq_dequant(packed: torch.Tensor, bits: int, n: int, scales: torch.Tensor,
+                 zeros: torch.Tensor, group_size: int = -1, g_idx=None,
+                 out_dtype: torch.dtype = torch.float32, out=None, stream=None) -> torch.Tensor:
+    _need_cuda(packed, scales, zeros, g_idx)
+    rows = packed.shape[0]
+    out = torch.empty(rows, n, dtype=out_dtype, device=packed.device) if out is None else out
+    st = library().gptq_dequant(_p(packed), int(bits), rows, int(n), _p(scales), _p(zeros),
+                                int(group_size), scales.shape[1], _p(g_idx), _p(out),
+                                _dtype_code(out.dtype), _stream(stream))
+    _check(st, "gptq_dequant")
+    return out
+
+
+@dataclasses.dataclass
+class QuantizedLinear:
+    packed: torch.Tensor
+    scales: torch.Tensor
+    zeros: torch.Tensor
+    g_idx: torch.Tensor | None
+    perm: torch.Tensor
+    bits: int
+    group_size: int
+    n: int
+    codes: torch.Tensor
+    info: torch.Tensor
+    H: torch.Tensor | None = None
+    U: torch.Tensor | None = None
+    Wq: torch.Tensor | None = None
+    row_loss: torch.Tensor | None = None
+
+
+def quantize_linear(W: torch.Tensor, X=None, H: torch.Tensor | None = None, bits: int = 4,
+                    group_size: int = 128, percdamp: float = 0.01, actorder: bool = False,
+                    alpha: float = 2.0, want_wq: bool = False, want_loss: bool = False,
+                    keep_factors: bool = False, stream=None) -> QuantizedLinear:
+    """GPTQ for one linear layer W (rows x n).  X: one calibration tensor
+    (n x N) or an iterable of batches; or pass a ready Hessian H."""
+    _need_cuda(W)
+    rows, n = W.shape
+    if H is None:
+        if X is None:
+            raise GptqError("give calibration inputs X or a Hessian H")
+        H = torch.zeros(n, n, dtype=torch.float32, device=W.device)
+        batches = [X] if isinstance(X, torch.Tensor) else X
+        for xb in batches:
+            gptq_hessian_accumulate(H, xb, alpha, stream=stream)
+    cfg = make_config(bits, group_size, percdamp, actorder)
+    U, perm, dead, info = gptq_cholesky_inverse(H, percdamp, actorder, stream=stream)
+    q = gptq_quantize_layer(W, U, perm, dead, cfg, want_wq=want_wq, want_loss=want_loss,
+                            stream=stream)
+    if bits == 4 and n % 8 == 0:
+        packed = gptq_pack_int4(q["codes"], stream=stream)
+    elif bits == 3 and n % 32 == 0:
+        packed = gptq_pack_int3(q["codes"], stream=stream)
+    else:
+        packed = q["codes"]
+    return QuantizedLinear(packed, q["scales"], q["zeros"], q["g_idx"], perm, bits, group_size, n,
+                           q["codes"], info, H if keep_factors else None,
+                           U if keep_factors else None, q["Wq"], q["row_loss"])

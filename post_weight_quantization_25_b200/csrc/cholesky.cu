@@ -1,0 +1,392 @@
+// Preparation of H and the upper Cholesky factor U of the damped inverse.
+//
+// Page "GPTQ, with the code open":
+//  * section "Paper vs. code": silent inputs (diag(H) == 0) are dead, their
+//    diagonal is set to 1; act-order sorts the columns by descending
+//    diag(H); 1 % of mean(diag H) is added to the diagonal;
+//  * section "From one repair to a whole model": a Cholesky factorisation
+//    whose rows hold every entry of the shrinking inverses [H_F^-1] -- the
+//    upper factor U with H'^-1 = U^T U; U[j][j]^2 = [H_F^-1]_jj for
+//    F = {j, ..., n-1}.
+//
+// Route taken here (one factorisation and one triangular inverse instead of
+// the pages' Cholesky -> inverse -> Cholesky): with J the index reversal,
+// factor J H' J = L L^T (lower L), invert M = L^-1, and U = J M J.  Because
+// H' = (J L J)(J L J)^T with J L J upper, (J L J)^-1 = J M J is the upper
+// factor of H'^-1, and that factor is unique.
+//
+// Both the factorisation and the inverse run right-looking over 128-wide
+// panels p = 0, 1, ...:
+//   (a) factor the diagonal block L_pp                         (1 CTA)
+//   (b) apply L_pp^-1 to every vector that needs it: the panel rows below
+//       (-> L_ip, the triangular solve) and the block row p of the inverse's
+//       right-hand side (-> M_p., forward substitution)       (one warp per vector)
+//   (c) rank-128 updates of the trailing lower matrix and of the remaining
+//       right-hand side rows                                   (fp32 tiles)
+// The inverse is kept transposed (RT = M^T) in U's own buffer, so that every
+// vector in (b) and every operand in (c) is a contiguous row segment; at the
+// end U = J M J = (J RT J)^T is one in-place anti-transpose of that buffer.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+
+#include "gemm_f32.cuh"
+#include "gptq_internal.cuh"
+
+namespace gptq {
+namespace {
+
+constexpr int kPanel = kBlock;  // 128
+constexpr int kPadLD = kPanel + 1;
+
+struct CholWs {
+  float* A;       // n x n, lower part used: J P^T H P J + lambda I
+  float* dprime;  // n: diag(H) with dead entries set to 1
+  double* lam;    // 1: damping
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+CholWs carve(void* ws, int64_t n) {
+  char* p = static_cast<char*>(ws);
+  CholWs w;
+  w.A = reinterpret_cast<float*>(p);
+  p += align_up(sizeof(float) * n * n, 256);
+  w.dprime = reinterpret_cast<float*>(p);
+  p += align_up(sizeof(float) * n, 256);
+  w.lam = reinterpret_cast<double*>(p);
+  return w;
+}
+
+// ---------------------------------------------------------------- preparation
+__global__ void __launch_bounds__(1024) diag_prep_kernel(const float* __restrict__ H, int n,
+                                                         float percdamp, uint8_t* __restrict__ dead,
+                                                         float* __restrict__ dprime,
+                                                         double* __restrict__ lam,
+                                                         int32_t* __restrict__ info) {
+  __shared__ double part[32];
+  double sum = 0.0;
+  bool bad = false;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const float d = H[(int64_t)i * n + i];
+    const bool is_dead = (d == 0.f);
+    const float dd = is_dead ? 1.f : d;
+    bad |= !isfinite(d);
+    dead[i] = is_dead ? 1 : 0;
+    dprime[i] = dd;
+    sum += (double)dd;
+  }
+  if (__syncthreads_or(bad) && threadIdx.x == 0) atomicCAS(info, 0, -1);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = sum;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    double v = (threadIdx.x < (blockDim.x >> 5)) ? part[threadIdx.x] : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (threadIdx.x == 0) *lam = (double)percdamp * (v / (double)n);
+  }
+}
+
+// Stable descending order of dprime: position of i = #{j: d_j > d_i} +
+// #{j < i: d_j == d_i}.  NaN keys rank as -inf so the result is always a
+// permutation (a NaN diagonal is reported through info anyway).
+__device__ __forceinline__ float rank_key(float d) { return isnan(d) ? -INFINITY : d; }
+
+__global__ void __launch_bounds__(256) actorder_rank_kernel(const float* __restrict__ dprime,
+                                                            int n, int32_t* __restrict__ perm) {
+  __shared__ float keys[2048];
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const float ki = (i < n) ? rank_key(dprime[i]) : 0.f;
+  int pos = 0;
+  for (int t0 = 0; t0 < n; t0 += 2048) {
+    const int cnt = min(2048, n - t0);
+    for (int j = threadIdx.x; j < cnt; j += blockDim.x) keys[j] = rank_key(dprime[t0 + j]);
+    __syncthreads();
+    if (i < n) {
+      for (int j = 0; j < cnt; ++j) {
+        const float kj = keys[j];
+        pos += (kj > ki) || (kj == ki && t0 + j < i);
+      }
+    }
+    __syncthreads();
+  }
+  if (i < n) perm[pos] = i;
+}
+
+__global__ void iota_kernel(int32_t* __restrict__ perm, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) perm[i] = i;
+}
+
+// A[a][b] (b <= a) = H[p(n-1-a)][p(n-1-b)] (+ lambda on the diagonal, dead -> 1 + lambda).
+// One CTA per output row; the source row of H is staged in shared memory.
+__global__ void __launch_bounds__(256) gather_reversed_kernel(
+    const float* __restrict__ H, int n, const int32_t* __restrict__ perm,
+    const uint8_t* __restrict__ dead, const double* __restrict__ lam, float* __restrict__ A) {
+  extern __shared__ float hrow[];
+  const int a = blockIdx.x;
+  const int pa = perm ? perm[n - 1 - a] : (n - 1 - a);
+  const float* src = H + (int64_t)pa * n;
+  for (int j = threadIdx.x; j < n; j += blockDim.x) hrow[j] = src[j];
+  __syncthreads();
+  const float lf = (float)(*lam);
+  float* dst = A + (int64_t)a * n;
+  for (int b = threadIdx.x; b <= a; b += blockDim.x) {
+    const int pb = perm ? perm[n - 1 - b] : (n - 1 - b);
+    float v = hrow[pb];
+    if (b == a) v = (dead[pa] ? 1.f : v) + lf;
+    dst[b] = v;
+  }
+}
+
+__global__ void set_diag_one_kernel(float* __restrict__ M, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) M[(int64_t)i * n + i] = 1.f;
+}
+
+// ---------------------------------------------------------------- panel (a)
+// Factor the diagonal block of panel p in place (lower part of A).  Uses the
+// unscaled (LDL^T-like) right-looking form -- one barrier per column -- and
+// scales by 1/sqrt(pivot) at the end.
+__global__ void __launch_bounds__(256) chol_diag_kernel(float* __restrict__ A, int n, int p,
+                                                        int32_t* __restrict__ info) {
+  if (*(volatile int32_t*)info != 0) return;
+  extern __shared__ float dyn_smem[];
+  float(*S)[kPadLD] = reinterpret_cast<float(*)[kPadLD]>(dyn_smem);
+  const int kb = p * kPanel;
+  const int bs = min(kPanel, n - kb);
+  const int tid = threadIdx.x;
+  for (int i = tid; i < kPanel * kPanel; i += blockDim.x) {
+    const int r = i / kPanel, c = i % kPanel;
+    float v = (r == c) ? 1.f : 0.f;
+    if (r < bs && c <= r) v = A[(int64_t)(kb + r) * n + kb + c];
+    S[r][c] = v;
+  }
+  __syncthreads();
+  const int r = tid & (kPanel - 1);
+  const int half = tid >> 7;
+  for (int c = 0; c < bs; ++c) {
+    const float d = S[c][c];
+    if (!(d > 0.f) || !isfinite(d)) {  // same value in every thread: uniform exit
+      if (tid == 0) atomicCAS(info, 0, n - (kb + c));
+      return;
+    }
+    if (r > c && r < bs) {
+      const float lrc = S[r][c] / d;
+      for (int s2 = c + 1 + half; s2 <= r; s2 += 2) S[r][s2] = fmaf(-lrc, S[s2][c], S[r][s2]);
+    }
+    __syncthreads();
+  }
+  for (int i = tid; i < bs * bs; i += blockDim.x) {
+    const int rr = i / bs, c = i % bs;
+    if (c > rr) continue;
+    const float sd = sqrtf(S[c][c]);
+    A[(int64_t)(kb + rr) * n + kb + c] = (rr == c) ? sd : S[rr][c] / sd;
+  }
+}
+
+// ---------------------------------------------------------------- panel (b)
+// v <- L_pp^-1 v for every vector: the rows of A below the panel
+// (restricted to the panel's columns) and rows [0, kb + bs) of RT.  One warp
+// per vector; lane l holds entries l, l+32, l+64, l+96.
+__global__ void __launch_bounds__(256) panel_solve_kernel(float* __restrict__ A,
+                                                          float* __restrict__ RT, int n, int p,
+                                                          const int32_t* __restrict__ info) {
+  if (*(volatile const int32_t*)info != 0) return;
+  extern __shared__ float dyn_smem[];
+  float(*L)[kPadLD] = reinterpret_cast<float(*)[kPadLD]>(dyn_smem);
+  float* rdiag = dyn_smem + kPanel * kPadLD;
+  const int kb = p * kPanel;
+  const int bs = min(kPanel, n - kb);
+  for (int i = threadIdx.x; i < kPanel * kPanel; i += blockDim.x) {
+    const int r = i / kPanel, c = i % kPanel;
+    float v = (r == c) ? 1.f : 0.f;
+    if (r < bs && c <= r) v = A[(int64_t)(kb + r) * n + kb + c];
+    L[r][c] = v;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kPanel; i += blockDim.x) rdiag[i] = 1.f / L[i][i];
+  __syncthreads();
+
+  const int lane = threadIdx.x & 31;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  const int nA = n - kb - bs;
+  const int nvec = nA + kb + bs;
+  for (int v = warp; v < nvec; v += nwarps) {
+    float* vec = (v < nA) ? (A + (int64_t)(kb + bs + v) * n + kb) : (RT + (int64_t)(v - nA) * n + kb);
+    float x[4];
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int col = lane + 32 * s;
+      x[s] = (col < bs) ? vec[col] : 0.f;
+    }
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+#pragma unroll 4
+      for (int l = 0; l < 32; ++l) {
+        const int j = 32 * s + l;
+        if (j >= bs) break;
+        float y = 0.f;
+        if (lane == l) {
+          y = x[s] * rdiag[j];
+          x[s] = y;
+        }
+        y = __shfl_sync(0xffffffffu, y, l);
+#pragma unroll
+        for (int s2 = s; s2 < 4; ++s2) {
+          const int i = lane + 32 * s2;
+          if (i > j) x[s2] = fmaf(-L[i][j], y, x[s2]);
+        }
+      }
+    }
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int col = lane + 32 * s;
+      if (col < bs) vec[col] = x[s];
+    }
+  }
+}
+
+// ---------------------------------------------------------------- panel (c)
+// Tiles [0, T1): lower tiles (rb, sb), p < sb <= rb, of A -= L_p L_p^T.
+// Tiles [T1, T1+T2): RT[cb][rb] -= RT[cb][p] A[rb][p]^T, cb <= p < rb.
+__global__ void __launch_bounds__(256) trailing_kernel(float* __restrict__ A,
+                                                       float* __restrict__ RT, int n, int p,
+                                                       int nblk, const int32_t* __restrict__ info) {
+  if (*(volatile const int32_t*)info != 0) return;
+  __shared__ __align__(16) float sm[kTileSmemFloats];
+  const int m = nblk - p - 1;
+  const int T1 = m * (m + 1) / 2;
+  const int kb = p * kPanel;
+  int t = blockIdx.x;
+  if (t < T1) {
+    int rr = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
+    while ((rr + 1) * (rr + 2) / 2 <= t) ++rr;
+    while (rr * (rr + 1) / 2 > t) --rr;
+    const int ss = t - rr * (rr + 1) / 2;
+    const int rb = p + 1 + rr, sb = p + 1 + ss;
+    float* C = A + (int64_t)rb * kPanel * n + (int64_t)sb * kPanel;
+    const float* P = A + (int64_t)rb * kPanel * n + kb;
+    const float* Q = A + (int64_t)sb * kPanel * n + kb;
+    tile_sub<true>(C, n, P, n, Q, n, min(kPanel, n - rb * kPanel), min(kPanel, n - sb * kPanel),
+                   kPanel, sm);
+  } else {
+    t -= T1;
+    const int cb = t / m, rb = p + 1 + t % m;
+    float* C = RT + (int64_t)cb * kPanel * n + (int64_t)rb * kPanel;
+    const float* P = RT + (int64_t)cb * kPanel * n + kb;
+    const float* Q = A + (int64_t)rb * kPanel * n + kb;
+    tile_sub<true>(C, n, P, n, Q, n, kPanel, min(kPanel, n - rb * kPanel), kPanel, sm);
+  }
+}
+
+// ---------------------------------------------------------------- finish
+// In place: U[i][j] <- U[n-1-j][n-1-i] (an involution; it maps the upper
+// triangle onto itself and the zero lower triangle onto itself).
+// Tiled form for n % 32 == 0: tile (I, J) swaps with (nt-1-J, nt-1-I).
+__global__ void __launch_bounds__(256) anti_transpose_tiles_kernel(float* __restrict__ U, int n) {
+  __shared__ float T0[32][33];
+  __shared__ float T1[32][33];
+  const int nt = n / 32;
+  const int I = blockIdx.y, J = blockIdx.x;
+  if (I > J || I + J > nt - 1) return;
+  const int I2 = nt - 1 - J, J2 = nt - 1 - I;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+  for (int a = ty; a < 32; a += 8) {
+    T0[a][tx] = U[(int64_t)(32 * I + a) * n + 32 * J + tx];
+    T1[a][tx] = U[(int64_t)(32 * I2 + a) * n + 32 * J2 + tx];
+  }
+  __syncthreads();
+  for (int a = ty; a < 32; a += 8) {
+    U[(int64_t)(32 * I + a) * n + 32 * J + tx] = T1[31 - tx][31 - a];
+    U[(int64_t)(32 * I2 + a) * n + 32 * J2 + tx] = T0[31 - tx][31 - a];
+  }
+}
+
+__global__ void anti_transpose_elems_kernel(float* __restrict__ U, int n) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  const int i = blockIdx.y;
+  if (j >= n || i > j || i + j >= n - 1) return;
+  const int64_t a = (int64_t)i * n + j;
+  const int64_t b = (int64_t)(n - 1 - j) * n + (n - 1 - i);
+  const float va = U[a], vb = U[b];
+  U[a] = vb;
+  U[b] = va;
+}
+
+}  // namespace
+
+size_t cholesky_workspace_bytes(int64_t n) {
+  return align_up(sizeof(float) * n * n, 256) + align_up(sizeof(float) * n, 256) + 256;
+}
+
+cudaError_t launch_cholesky_inverse(const float* H, int64_t n64, float percdamp, int actorder,
+                                    float* U, int32_t* perm, uint8_t* dead, int32_t* info,
+                                    void* ws, cudaStream_t s) {
+  const int n = (int)n64;
+  CholWs w = carve(ws, n64);
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(info, 0, sizeof(int32_t), s)) != cudaSuccess) return e;
+  diag_prep_kernel<<<1, 1024, 0, s>>>(H, n, percdamp, dead, w.dprime, w.lam, info);
+  note_launch();
+  int32_t* perm_used = nullptr;
+  if (actorder) {
+    actorder_rank_kernel<<<(n + 255) / 256, 256, 0, s>>>(w.dprime, n, perm);
+    note_launch();
+    perm_used = perm;
+  } else if (perm) {
+    iota_kernel<<<(n + 255) / 256, 256, 0, s>>>(perm, n);
+    note_launch();
+  }
+  const size_t row_smem = sizeof(float) * (size_t)n;
+  if (row_smem > 48 * 1024) {
+    if ((e = cudaFuncSetAttribute(gather_reversed_kernel,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)row_smem)) !=
+        cudaSuccess)
+      return e;
+  }
+  gather_reversed_kernel<<<n, 256, row_smem, s>>>(H, n, perm_used, dead, w.lam, w.A);
+  note_launch();
+  if ((e = cudaMemsetAsync(U, 0, sizeof(float) * (size_t)n * n, s)) != cudaSuccess) return e;
+  set_diag_one_kernel<<<(n + 255) / 256, 256, 0, s>>>(U, n);
+  note_launch();
+
+  const int nblk = (n + kPanel - 1) / kPanel;
+  const int sms = num_sms();
+  const size_t diag_smem = sizeof(float) * kPanel * kPadLD;
+  const size_t solve_smem = diag_smem + sizeof(float) * kPanel;
+  if ((e = cudaFuncSetAttribute(chol_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)diag_smem)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(panel_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)solve_smem)) != cudaSuccess)
+    return e;
+  const int solve_ctas = std::min((n + 7) / 8, 3 * sms);
+  for (int p = 0; p < nblk; ++p) {
+    chol_diag_kernel<<<1, 256, diag_smem, s>>>(w.A, n, p, info);
+    note_launch();
+    panel_solve_kernel<<<solve_ctas, 256, solve_smem, s>>>(w.A, U, n, p, info);
+    note_launch();
+    const int m = nblk - p - 1;
+    const int tiles = m * (m + 1) / 2 + (p + 1) * m;
+    if (tiles > 0) {
+      trailing_kernel<<<tiles, 256, 0, s>>>(w.A, U, n, p, nblk, info);
+      note_launch();
+    }
+  }
+  if (n % 32 == 0) {
+    const int nt = n / 32;
+    anti_transpose_tiles_kernel<<<dim3(nt, (nt + 1) / 2), 256, 0, s>>>(U, n);
+    note_launch();
+  } else {
+    anti_transpose_elems_kernel<<<dim3((n + 255) / 256, n), 256, 0, s>>>(U, n);
+    note_launch();
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace gptq

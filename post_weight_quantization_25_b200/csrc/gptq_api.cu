@@ -1,0 +1,196 @@
+// C ABI of libgptq_b200.so: argument checks, workspace layout, launches.
+// See include/gptq.h for the contract of every entry point.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+
+#include "gptq_internal.cuh"
+
+namespace gptq {
+
+int num_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
+static std::atomic<long long> g_launches{0};
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+}  // namespace gptq
+
+namespace {
+
+constexpr int64_t kMaxN = 57344;       // a row of H / W is staged in shared memory
+constexpr int64_t kMaxRows = 1 << 24;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+gptq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t hessian_ws(int64_t n, int64_t ntok, gptq_dtype xt) {
+  if (xt != GPTQ_F32) return 0;
+  const int64_t ld = (ntok + 7) / 8 * 8;
+  return 2 * align_up(sizeof(uint16_t) * (size_t)n * ld, 256);
+}
+
+gptq_status check_cfg(const gptq_config* cfg) {
+  if (!cfg) return GPTQ_ERR_INVALID_ARG;
+  if (cfg->bits < 2 || cfg->bits > 8) return GPTQ_ERR_INVALID_ARG;
+  if (cfg->sym != 0) return GPTQ_ERR_UNSUPPORTED;
+  if (cfg->block != gptq::kBlock) return GPTQ_ERR_UNSUPPORTED;
+  const int g = cfg->group_size;
+  if (g == 0 || g < -1) return GPTQ_ERR_INVALID_ARG;
+  if (g > 0 && !(g == 32 || g == 64 || g % gptq::kBlock == 0)) return GPTQ_ERR_UNSUPPORTED;
+  return GPTQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t gptq_launch_count(void) { return gptq::g_launches.load(std::memory_order_relaxed); }
+
+const char* gptq_status_string(int status) {
+  switch (status) {
+    case GPTQ_OK: return "ok";
+    case GPTQ_ERR_INVALID_ARG: return "invalid argument";
+    case GPTQ_ERR_UNSUPPORTED: return "unsupported request";
+    case GPTQ_ERR_WORKSPACE: return "workspace too small";
+    case GPTQ_ERR_CUDA: return "CUDA error";
+    case GPTQ_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+gptq_status gptq_workspace_size(int op, int64_t rows, int64_t n, int64_t ntok, gptq_dtype xt,
+                                const gptq_config* cfg, size_t* bytes) {
+  if (!bytes || n <= 0 || n > kMaxN) return GPTQ_ERR_INVALID_ARG;
+  switch (op) {
+    case GPTQ_OP_HESSIAN:
+      if (ntok < 0) return GPTQ_ERR_INVALID_ARG;
+      *bytes = hessian_ws(n, ntok, xt);
+      return GPTQ_OK;
+    case GPTQ_OP_CHOLESKY:
+      *bytes = gptq::cholesky_workspace_bytes(n);
+      return GPTQ_OK;
+    case GPTQ_OP_QUANTIZE: {
+      if (rows < 0 || rows > kMaxRows) return GPTQ_ERR_INVALID_ARG;
+      const gptq_status st = check_cfg(cfg);
+      if (st != GPTQ_OK) return st;
+      *bytes = gptq::quantize_workspace_bytes(rows, n);
+      return GPTQ_OK;
+    }
+    default:
+      return GPTQ_ERR_INVALID_ARG;
+  }
+}
+
+gptq_status gptq_hessian_accumulate(float* H, const void* X, gptq_dtype xt, int64_t n,
+                                    int64_t ntok, int64_t ldx, int token_major, float alpha,
+                                    void* ws, size_t ws_bytes, int32_t* info, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!H || n <= 0 || n > kMaxN || ntok < 0 || ldx < ntok) return GPTQ_ERR_INVALID_ARG;
+  if (xt != GPTQ_BF16 && xt != GPTQ_F32) return GPTQ_ERR_INVALID_ARG;
+  if (token_major) return GPTQ_ERR_UNSUPPORTED;
+  if (!aligned(H, 16)) return GPTQ_ERR_INVALID_ARG;
+  if (ntok == 0) return GPTQ_OK;
+  if (!X) return GPTQ_ERR_INVALID_ARG;
+  cudaError_t e;
+  if (xt == GPTQ_BF16) {
+    if (!aligned(X, 16) || (ldx * 2) % 16 != 0) return GPTQ_ERR_INVALID_ARG;
+    if ((e = gptq::launch_syrk_bf16(H, n, X, X, ntok, ldx, alpha, info, s)) != cudaSuccess)
+      return cuda_status(e);
+  } else {
+    if (!aligned(X, 4)) return GPTQ_ERR_INVALID_ARG;
+    const size_t need = hessian_ws(n, ntok, xt);
+    if (!ws || ws_bytes < need) return GPTQ_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return GPTQ_ERR_INVALID_ARG;
+    const int64_t ld = (ntok + 7) / 8 * 8;
+    char* hi = static_cast<char*>(ws);
+    char* lo = hi + need / 2;
+    if ((e = gptq::launch_split_bf16(static_cast<const float*>(X), n, ntok, ldx, hi, lo, ld, s)) !=
+        cudaSuccess)
+      return cuda_status(e);
+    // hi hi^T + hi lo^T + lo hi^T  (lo lo^T is below fp32 resolution of the sum)
+    if ((e = gptq::launch_syrk_bf16(H, n, hi, hi, ntok, ld, alpha, info, s)) != cudaSuccess ||
+        (e = gptq::launch_syrk_bf16(H, n, hi, lo, ntok, ld, alpha, info, s)) != cudaSuccess ||
+        (e = gptq::launch_syrk_bf16(H, n, lo, hi, ntok, ld, alpha, info, s)) != cudaSuccess)
+      return cuda_status(e);
+  }
+  return cuda_status(gptq::launch_mirror_upper(H, n, s));
+}
+
+gptq_status gptq_cholesky_inverse(const float* H, int64_t n, float percdamp, int actorder,
+                                  float* U, int32_t* perm, uint8_t* dead, int32_t* info,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!H || !U || !dead || !info || n <= 0 || n > kMaxN) return GPTQ_ERR_INVALID_ARG;
+  if (actorder && !perm) return GPTQ_ERR_INVALID_ARG;
+  if (!(percdamp >= 0.f)) return GPTQ_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < gptq::cholesky_workspace_bytes(n)) return GPTQ_ERR_WORKSPACE;
+  if (!aligned(ws, 256) || !aligned(H, 4) || !aligned(U, 16)) return GPTQ_ERR_INVALID_ARG;
+  return cuda_status(gptq::launch_cholesky_inverse(H, n, percdamp, actorder, U, perm, dead, info,
+                                                   ws, s));
+}
+
+gptq_status gptq_quantize_layer(const void* W, gptq_dtype wt, int64_t rows, int64_t n,
+                                const float* U, const int32_t* perm, const uint8_t* dead,
+                                const gptq_config* cfg, uint8_t* codes, float* scales,
+                                uint8_t* zeros, int32_t* g_idx, float* Wq, float* row_loss,
+                                void* ws, size_t ws_bytes, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const gptq_status st = check_cfg(cfg);
+  if (st != GPTQ_OK) return st;
+  if (n <= 0 || n > kMaxN || rows < 0 || rows > kMaxRows) return GPTQ_ERR_INVALID_ARG;
+  if (wt != GPTQ_BF16 && wt != GPTQ_F32) return GPTQ_ERR_INVALID_ARG;
+  if (rows == 0) return GPTQ_OK;
+  if (!W || !U || !dead || !codes || !scales || !zeros) return GPTQ_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < gptq::quantize_workspace_bytes(rows, n)) return GPTQ_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return GPTQ_ERR_INVALID_ARG;
+  return cuda_status(gptq::launch_quantize_layer(W, wt, rows, n, U, perm, dead, cfg->bits,
+                                                 cfg->group_size, codes, scales, zeros, g_idx,
+                                                 Wq, row_loss, ws, s));
+}
+
+gptq_status gptq_pack_int4(const uint8_t* codes, int64_t rows, int64_t n, uint32_t* out,
+                           void* stream) {
+  if (rows < 0 || n <= 0 || n % 8 != 0) return GPTQ_ERR_INVALID_ARG;
+  if (rows == 0) return GPTQ_OK;
+  if (!codes || !out || !aligned(out, 4)) return GPTQ_ERR_INVALID_ARG;
+  return cuda_status(gptq::launch_pack_int4(codes, rows, n, out, static_cast<cudaStream_t>(stream)));
+}
+
+gptq_status gptq_pack_int3(const uint8_t* codes, int64_t rows, int64_t n, uint32_t* out,
+                           void* stream) {
+  if (rows < 0 || n <= 0 || n % 32 != 0) return GPTQ_ERR_INVALID_ARG;
+  if (rows == 0) return GPTQ_OK;
+  if (!codes || !out || !aligned(out, 4)) return GPTQ_ERR_INVALID_ARG;
+  return cuda_status(gptq::launch_pack_int3(codes, rows, n, out, static_cast<cudaStream_t>(stream)));
+}
+
+gptq_status gptq_dequant(const uint32_t* packed, int bits, int64_t rows, int64_t n,
+                         const float* scales, const uint8_t* zeros, int group_size,
+                         int64_t n_groups, const int32_t* g_idx, void* out, gptq_dtype ot,
+                         void* stream) {
+  if (bits != 3 && bits != 4) return GPTQ_ERR_UNSUPPORTED;
+  if (rows < 0 || n <= 0) return GPTQ_ERR_INVALID_ARG;
+  if ((bits == 4 && n % 8) || (bits == 3 && n % 32)) return GPTQ_ERR_INVALID_ARG;
+  if (ot != GPTQ_BF16 && ot != GPTQ_F32) return GPTQ_ERR_INVALID_ARG;
+  const int64_t Gdef = group_size > 0 ? (n + group_size - 1) / group_size : 1;
+  const int64_t G = n_groups > 0 ? n_groups : Gdef;
+  if (!g_idx && G < Gdef) return GPTQ_ERR_INVALID_ARG;
+  if (rows == 0) return GPTQ_OK;
+  if (!packed || !scales || !zeros || !out || !aligned(packed, 4) || !aligned(scales, 4))
+    return GPTQ_ERR_INVALID_ARG;
+  return cuda_status(gptq::launch_dequant(packed, bits, rows, n, scales, zeros, group_size, G,
+                                          g_idx, out, ot == GPTQ_BF16 ? 1 : 0,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,54 @@
+// Internal launch interface between the C-ABI layer (gptq_api.cu) and the
+// kernel files.  Every launcher enqueues on `s` and returns the CUDA error of
+// the launch (cudaSuccess when nothing had to run).
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/gptq.h"
+
+namespace gptq {
+
+constexpr int kBlock = 128;            // lazy-update block of the sweep / Cholesky panel
+constexpr int kGridWaitLimitNs = 1000000000;  // 1 s: upper bound of any in-kernel wait
+
+int num_sms();
+// Counts one kernel enqueued by this library (read by gptq_launch_count).
+void note_launch();
+
+// ---- Hessian (hessian_syrk.cu)
+// H(upper incl. diagonal) += alpha * A_rows * B_rows^T over tokens [0, ntok),
+// A and B are n x ntok bf16 with row stride ld (elements).
+cudaError_t launch_syrk_bf16(float* H, int64_t n, const void* A, const void* B, int64_t ntok,
+                             int64_t ld, float alpha, int32_t* info, cudaStream_t s);
+// fp32 X -> bf16 hi / lo parts (n x ntok, row stride ldo).
+cudaError_t launch_split_bf16(const float* X, int64_t n, int64_t ntok, int64_t ldx, void* hi,
+                              void* lo, int64_t ldo, cudaStream_t s);
+// H[c][r] = H[r][c] for c > r.
+cudaError_t launch_mirror_upper(float* H, int64_t n, cudaStream_t s);
+
+// ---- Cholesky / inverse (cholesky.cu)
+cudaError_t launch_cholesky_inverse(const float* H, int64_t n, float percdamp, int actorder,
+                                    float* U, int32_t* perm, uint8_t* dead, int32_t* info,
+                                    void* ws, cudaStream_t s);
+size_t cholesky_workspace_bytes(int64_t n);
+
+// ---- sweep (sweep.cu)
+cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows, int64_t n, const float* U,
+                                  const int32_t* perm, const uint8_t* dead, int bits,
+                                  int group_size, uint8_t* codes, float* scales, uint8_t* zeros,
+                                  int32_t* g_idx, float* Wq, float* row_loss, void* ws,
+                                  cudaStream_t s);
+size_t quantize_workspace_bytes(int64_t rows, int64_t n);
+
+// ---- storage (pack.cu)
+cudaError_t launch_pack_int4(const uint8_t* codes, int64_t rows, int64_t n, uint32_t* out,
+                             cudaStream_t s);
+cudaError_t launch_pack_int3(const uint8_t* codes, int64_t rows, int64_t n, uint32_t* out,
+                             cudaStream_t s);
+cudaError_t launch_dequant(const uint32_t* packed, int bits, int64_t rows, int64_t n,
+                           const float* scales, const uint8_t* zeros, int group_size,
+                           int64_t n_groups, const int32_t* g_idx, void* out, int out_bf16,
+                           cudaStream_t s);
+
+}  // namespace gptq

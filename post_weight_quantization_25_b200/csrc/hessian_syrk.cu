@@ -1,0 +1,392 @@
+// Calibration Hessian  H += alpha * X X^T  on the tcgen05 tensor cores.
+//
+// Page "GPTQ, with the code open", section "Measuring damage where it
+// matters": H = 2 X X^T prices the layer-output damage exactly; section
+// "Paper vs. code": H is accumulated over calibration batches.
+//
+// Design (sm_100a):
+//  * X is n features x N tokens, token-contiguous, so both GEMM operands are
+//    K-major rows of X.  Only tiles that touch the upper triangle are computed
+//    (128 x 256 output tiles, I <= 2J + 1); the lower triangle is mirrored
+//    afterwards.
+//  * Work unit = (tile, chunk of tokens).  The number of token chunks is
+//    picked so that the units fill whole waves of the SMs; a persistent grid
+//    of one CTA per SM walks the units in token-chunk-major order, so the
+//    CTAs that run together read the same slab of X and it is served from L2.
+//  * Per CTA: warp 0 issues TMA loads (128-byte swizzle, 4-stage ring of
+//    128x64 + 256x64 bf16 tiles), warp 1 issues tcgen05.mma kind::f16
+//    (M=128, N=256, K=16; fp32 accumulators in TMEM, two 256-column buffers
+//    so the epilogue of one unit overlaps the MMAs of the next), warps 2-5
+//    drain TMEM with tcgen05.ld and add alpha * partial into H with vector
+//    atomics (the split-K reduction), masking to the upper triangle.
+//  * No multicast loads.  Every wait is bounded: on timeout the CTA stops,
+//    writes GPTQ_ERR_TIMEOUT to `info`, waits for its own copies and MMAs,
+//    frees TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "gptq_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace gptq {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + 256;
+constexpr uint64_t WAIT_LIMIT_NS = (uint64_t)kGridWaitLimitNs;
+
+struct SyrkArgs {
+  float* H;
+  int n;
+  float alpha;
+  int nkb;          // k-blocks of BK tokens
+  int kb_per_unit;  // k-blocks per unit (last chunk may be shorter)
+  int ntiles;       // tiles touching the upper triangle
+  int nI;           // row blocks of BM
+  int units;        // ntiles * token chunks
+  int vec4;         // H row starts are 16-byte aligned
+  int32_t* info;
+};
+
+// Tile t of the J-major enumeration: column block J holds row blocks 0..min(nI, 2J+2)-1.
+__device__ __forceinline__ void decode_tile(int t, int nI, int& I, int& J) {
+  J = 0;
+  while (true) {
+    const int c = min(nI, 2 * J + 2);
+    if (t < c) {
+      I = t;
+      return;
+    }
+    t -= c;
+    ++J;
+  }
+}
+
+__device__ __forceinline__ void raise_abort(volatile int* abort_flag, int32_t* info) {
+  *abort_flag = 1;
+  if (info) atomicExch(info, (int32_t)GPTQ_ERR_TIMEOUT);
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    syrk_bf16_kernel(const __grid_constant__ CUtensorMap mapA,
+                     const __grid_constant__ CUtensorMap mapB, const SyrkArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* full = bars;                 // [STAGES] TMA landed
+  uint64_t* empty = bars + STAGES;       // [STAGES] MMAs done reading
+  uint64_t* tfull = bars + 2 * STAGES;   // [2] accumulator ready
+  uint64_t* tempty = tfull + 2;          // [2] accumulator drained
+  uint64_t* drain = tempty + 2;          // [1] MMA drain on abort
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(&tfull[a], 1);
+      ptx::mbar_init(&tempty[a], 128);
+    }
+    ptx::mbar_init(drain, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      ptx::prefetch_tmap(&mapA);
+      ptx::prefetch_tmap(&mapB);
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_parity[STAGES];
+      for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
+      bool ok = true;
+      for (int u = blockIdx.x; u < args.units && ok; u += gridDim.x) {
+        int I, J;
+        decode_tile(u % args.ntiles, args.nI, I, J);
+        const int kb0 = (u / args.ntiles) * args.kb_per_unit;
+        const int kb1 = min(kb0 + args.kb_per_unit, args.nkb);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, WAIT_LIMIT_NS)) {
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          ptx::tma_load_2d(sA + stage * A_BYTES, &mapA, &full[stage], kb * BK, I * BM);
+          ptx::tma_load_2d(sB + stage * B_BYTES, &mapB, &full[stage], kb * BK, J * BN);
+          last_parity[stage] = (int)phase;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok || *abort_flag) {
+        raise_abort(abort_flag, args.info);
+        // wait (bounded) for this CTA's own copies still in flight
+        volatile int never = 0;
+        for (int s = 0; s < STAGES; ++s)
+          if (last_parity[s] >= 0)
+            ptx::mbar_wait_bounded(&full[s], (uint32_t)last_parity[s], &never, WAIT_LIMIT_NS);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc = ptx::idesc_bf16_f32(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t aphase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < args.units && ok; u += gridDim.x) {
+        const int kb0 = (u / args.ntiles) * args.kb_per_unit;
+        const int kb1 = min(kb0 + args.kb_per_unit, args.nkb);
+        if (!ptx::mbar_wait_bounded(&tempty[acc], aphase ^ 1, abort_flag, WAIT_LIMIT_NS)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!ptx::mbar_wait_bounded(&full[stage], phase, abort_flag, WAIT_LIMIT_NS)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint64_t adesc = ptx::smem_desc_sw128(ptx::smem_u32(sA + stage * A_BYTES));
+          const uint64_t bdesc = ptx::smem_desc_sw128(ptx::smem_u32(sB + stage * B_BYTES));
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            ptx::mma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc,
+                          (kb > kb0 || k > 0) ? 1u : 0u);
+          ptx::mma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        ptx::mma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) aphase ^= 1;
+      }
+      if (!ok || *abort_flag) {
+        raise_abort(abort_flag, args.info);
+        ptx::mma_commit(drain);  // completes when every MMA issued above is done
+        volatile int never = 0;
+        ptx::mbar_wait_bounded(drain, 0, &never, WAIT_LIMIT_NS);
+      }
+    }
+  } else {
+    // -------------------------------------------------- epilogue (warps 2..5)
+    const int q = warp & 3;  // this warp may read TMEM lanes [32q, 32q + 32)
+    int acc = 0;
+    uint32_t aphase = 0;
+    const int n = args.n;
+    for (int u = blockIdx.x; u < args.units; u += gridDim.x) {
+      int I, J;
+      decode_tile(u % args.ntiles, args.nI, I, J);
+      if (!ptx::mbar_wait_bounded(&tfull[acc], aphase, abort_flag, WAIT_LIMIT_NS)) {
+        raise_abort(abort_flag, args.info);
+        break;
+      }
+      ptx::tc_fence_after();
+      const int row_lo = I * BM + q * 32;
+      const int row = row_lo + lane;
+      float* hrow = args.H + (int64_t)row * n;
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        const int col0 = J * BN + ch * 32;
+        if (col0 >= n) break;
+        if (col0 + 31 < row_lo) continue;  // whole 32x32 piece below the diagonal
+        uint32_t v[32];
+        ptx::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + ch * 32), v);
+        ptx::tmem_ld_wait();
+        if (row < n) {
+#pragma unroll
+          for (int j4 = 0; j4 < 8; ++j4) {
+            const int c = col0 + 4 * j4;
+            const float f0 = args.alpha * __uint_as_float(v[4 * j4 + 0]);
+            const float f1 = args.alpha * __uint_as_float(v[4 * j4 + 1]);
+            const float f2 = args.alpha * __uint_as_float(v[4 * j4 + 2]);
+            const float f3 = args.alpha * __uint_as_float(v[4 * j4 + 3]);
+            if (args.vec4 && c >= row && c + 3 < n) {
+              atomicAdd(reinterpret_cast<float4*>(hrow + c), make_float4(f0, f1, f2, f3));
+            } else {
+              if (c + 0 >= row && c + 0 < n) atomicAdd(hrow + c + 0, f0);
+              if (c + 1 >= row && c + 1 < n) atomicAdd(hrow + c + 1, f1);
+              if (c + 2 >= row && c + 2 < n) atomicAdd(hrow + c + 2, f2);
+              if (c + 3 >= row && c + 3 < n) atomicAdd(hrow + c + 3, f3);
+            }
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) aphase ^= 1;
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// hi = bf16(x) (round to nearest even), lo = bf16(x - hi)
+__global__ void split_bf16_kernel(const float* __restrict__ X, int64_t n, int64_t ntok,
+                                  int64_t ldx, __nv_bfloat16* __restrict__ hi,
+                                  __nv_bfloat16* __restrict__ lo, int64_t ldo) {
+  const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const int64_t r = blockIdx.y;
+  if (t >= ntok) return;
+  const float x = X[r * ldx + t];
+  const __nv_bfloat16 h = __float2bfloat16_rn(x);
+  hi[r * ldo + t] = h;
+  lo[r * ldo + t] = __float2bfloat16_rn(x - __bfloat162float(h));
+}
+
+// H[c][r] = H[r][c] for c > r, 32 x 32 tiles through shared memory.
+__global__ void __launch_bounds__(256) mirror_upper_kernel(float* __restrict__ H, int n) {
+  __shared__ float T[32][33];
+  const int I = blockIdx.y, J = blockIdx.x;
+  if (I > J) return;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int a = ty; a < 32; a += 8) {
+    const int r = 32 * I + a, c = 32 * J + tx;
+    T[a][tx] = (r < n && c < n) ? H[(int64_t)r * n + c] : 0.f;
+  }
+  __syncthreads();
+  for (int a = ty; a < 32; a += 8) {
+    const int r = 32 * J + a, c = 32 * I + tx;  // destination (lower): row r, col c
+    if (r < n && c < n && c < r) H[(int64_t)r * n + c] = T[tx][a];
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t ntok, int64_t ld,
+              uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)ntok, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_syrk_bf16(float* H, int64_t n, const void* A, const void* B, int64_t ntok,
+                             int64_t ld, float alpha, int32_t* info, cudaStream_t s) {
+  if (n <= 0 || ntok <= 0) return cudaSuccess;
+  CUtensorMap mapA, mapB;
+  if (!make_map(&mapA, A, n, ntok, ld, BM) || !make_map(&mapB, B, n, ntok, ld, BN))
+    return cudaErrorInvalidValue;
+  SyrkArgs a;
+  a.H = H;
+  a.n = (int)n;
+  a.alpha = alpha;
+  a.nkb = (int)((ntok + BK - 1) / BK);
+  a.nI = (int)((n + BM - 1) / BM);
+  const int nJ = (int)((n + BN - 1) / BN);
+  a.ntiles = 0;
+  for (int J = 0; J < nJ; ++J) a.ntiles += std::min(a.nI, 2 * J + 2);
+  const int sms = num_sms();
+  // token chunks: the fewest that fill the SMs' waves to >= 97 %, at least 8
+  // k-blocks per unit; else the best fill found.
+  int best_kc = 1;
+  double best_eff = -1.0;
+  const int max_kc = std::max(1, std::min(a.nkb / 8, 512));
+  for (int kc = 1; kc <= max_kc; ++kc) {
+    const long units = (long)a.ntiles * kc;
+    const long waves = (units + sms - 1) / sms;
+    const double eff = (double)units / (double)(waves * sms);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best_kc = kc;
+    }
+    if (eff >= 0.97) break;
+  }
+  a.kb_per_unit = (a.nkb + best_kc - 1) / best_kc;
+  const int kchunks = (a.nkb + a.kb_per_unit - 1) / a.kb_per_unit;
+  a.units = a.ntiles * kchunks;
+  a.vec4 = ((n % 4) == 0 && (reinterpret_cast<uintptr_t>(H) % 16) == 0) ? 1 : 0;
+  a.info = info;
+  cudaError_t e = cudaFuncSetAttribute(syrk_bf16_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int grid = std::min(sms, a.units);
+  syrk_bf16_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(mapA, mapB, a);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_split_bf16(const float* X, int64_t n, int64_t ntok, int64_t ldx, void* hi,
+                              void* lo, int64_t ldo, cudaStream_t s) {
+  if (n <= 0 || ntok <= 0) return cudaSuccess;
+  dim3 grid((unsigned)((ntok + 255) / 256), (unsigned)n);
+  split_bf16_kernel<<<grid, 256, 0, s>>>(X, n, ntok, ldx, static_cast<__nv_bfloat16*>(hi),
+                                         static_cast<__nv_bfloat16*>(lo), ldo);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mirror_upper(float* H, int64_t n, cudaStream_t s) {
+  const unsigned nt = (unsigned)((n + 31) / 32);
+  mirror_upper_kernel<<<dim3(nt, nt), 256, 0, s>>>(H, (int)n);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace gptq

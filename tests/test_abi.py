@@ -1,0 +1,100 @@
+"""The C-ABI library loads and exports every entry point include/gptq.h
+declares; host-side argument checks (no GPU needed, no kernel launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from post_weight_quantization_25_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gptq.h")
+
+
+def _declared():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(gptq_[a-z0-9_]+)\s*\(", txt)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_lib.LIB_PATH):
+        from post_weight_quantization_25_b200 import build
+        build.build()
+    return _lib.load()
+
+
+def test_header_declares_the_expected_entry_points():
+    assert _declared() == sorted(_lib.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    assert lib.gptq_status_string(0) == b"ok"
+    assert lib.gptq_status_string(5) == b"device wait timed out"
+    assert lib.gptq_status_string(99) == b"unknown status"
+
+
+def test_workspace_sizes(lib):
+    out = ctypes.c_size_t(0)
+    cfg = _lib.GptqConfig(4, 128, 0.01, 128, 1, 0)
+    assert lib.gptq_workspace_size(_lib.GPTQ_OP_HESSIAN, 0, 256, 2048, _lib.GPTQ_BF16, None,
+                                   ctypes.byref(out)) == 0
+    assert out.value == 0
+    assert lib.gptq_workspace_size(_lib.GPTQ_OP_HESSIAN, 0, 256, 2048, _lib.GPTQ_F32, None,
+                                   ctypes.byref(out)) == 0
+    assert out.value >= 2 * 256 * 2048 * 2
+    assert lib.gptq_workspace_size(_lib.GPTQ_OP_CHOLESKY, 0, 4096, 0, 0, None,
+                                   ctypes.byref(out)) == 0
+    assert out.value >= 4096 * 4096 * 4
+    assert lib.gptq_workspace_size(_lib.GPTQ_OP_QUANTIZE, 4096, 4096, 0, 0, ctypes.byref(cfg),
+                                   ctypes.byref(out)) == 0
+    assert out.value >= 4096 * 4096 * 5
+    # a symmetric ruler and a block other than 128 are not implemented
+    bad = _lib.GptqConfig(4, 128, 0.01, 128, 1, 1)
+    assert lib.gptq_workspace_size(2, 16, 16, 0, 0, ctypes.byref(bad), ctypes.byref(out)) == 2
+    bad = _lib.GptqConfig(4, 128, 0.01, 64, 1, 0)
+    assert lib.gptq_workspace_size(2, 16, 16, 0, 0, ctypes.byref(bad), ctypes.byref(out)) == 2
+    bad = _lib.GptqConfig(4, 48, 0.01, 128, 1, 0)
+    assert lib.gptq_workspace_size(2, 16, 16, 0, 0, ctypes.byref(bad), ctypes.byref(out)) == 2
+    bad = _lib.GptqConfig(1, 128, 0.01, 128, 1, 0)
+    assert lib.gptq_workspace_size(2, 16, 16, 0, 0, ctypes.byref(bad), ctypes.byref(out)) == 1
+    assert lib.gptq_workspace_size(7, 16, 16, 0, 0, None, ctypes.byref(out)) == 1
+    assert lib.gptq_workspace_size(0, 16, 0, 16, 0, None, ctypes.byref(out)) == 1
+
+
+def test_argument_checks_reject_before_any_launch(lib):
+    # null H / X, bad sizes, token-major layout: rejected on the host
+    assert lib.gptq_hessian_accumulate(None, None, 0, 16, 16, 16, 0, 2.0, None, 0, None,
+                                       None) == 1
+    assert lib.gptq_hessian_accumulate(ctypes.c_void_p(256), ctypes.c_void_p(256), 0, 16, 16, 8,
+                                       0, 2.0, None, 0, None, None) == 1      # ldx < ntok
+    assert lib.gptq_hessian_accumulate(ctypes.c_void_p(256), ctypes.c_void_p(256), 0, 16, 16, 16,
+                                       1, 2.0, None, 0, None, None) == 2      # token-major
+    assert lib.gptq_hessian_accumulate(ctypes.c_void_p(256), ctypes.c_void_p(256), 1, 16, 16, 16,
+                                       0, 2.0, None, 0, None, None) == 3      # fp32 needs ws
+    assert lib.gptq_hessian_accumulate(ctypes.c_void_p(256), ctypes.c_void_p(258), 0, 16, 16, 16,
+                                       0, 2.0, None, 0, None, None) == 1      # misaligned X
+    assert lib.gptq_cholesky_inverse(None, 16, 0.01, 0, None, None, None, None, None, 0,
+                                     None) == 1
+    assert lib.gptq_cholesky_inverse(ctypes.c_void_p(256), 16, 0.01, 1, ctypes.c_void_p(256),
+                                     None, ctypes.c_void_p(256), ctypes.c_void_p(256), None, 0,
+                                     None) == 1                               # act-order, no perm
+    assert lib.gptq_cholesky_inverse(ctypes.c_void_p(256), 16, 0.01, 0, ctypes.c_void_p(256),
+                                     None, ctypes.c_void_p(256), ctypes.c_void_p(256), None, 0,
+                                     None) == 3                               # no workspace
+    cfg = _lib.GptqConfig(4, 128, 0.01, 128, 0, 0)
+    assert lib.gptq_quantize_layer(None, 0, 0, 16, None, None, None, ctypes.byref(cfg), None,
+                                   None, None, None, None, None, None, 0, None) == 0   # empty
+    assert lib.gptq_quantize_layer(None, 0, 4, 16, None, None, None, ctypes.byref(cfg), None,
+                                   None, None, None, None, None, None, 0, None) == 1
+    assert lib.gptq_pack_int4(None, 4, 12, None, None) == 1                   # n % 8
+    assert lib.gptq_pack_int3(None, 4, 40, None, None) == 1                   # n % 32
+    assert lib.gptq_pack_int4(None, 0, 16, None, None) == 0                   # empty
+    assert lib.gptq_dequant(None, 5, 4, 16, None, None, -1, 1, None, None, 0, None) == 2

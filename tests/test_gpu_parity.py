@@ -1,0 +1,204 @@
+"""CUDA path vs the fp64 oracle, element by element, on seeded inputs.
+
+Every call goes through the C ABI (the ctypes binding).  Sizes span several
+128-wide tiles with ragged tails; the tolerances are the agreed ones: H
+relative Frobenius <= 1e-4, codes identical except at rounding ties (replayed
+and counted), objective relative <= 1e-3, per-row scales <= 1e-6, group
+scales <= 1e-4, packing and dequant bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import post_weight_quantization_25_b200 as G
+import workloads
+from oracle import gptq_oracle as O
+
+from gpu_util import compare_layer, device_x, gpu_layer, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+# ------------------------------------------------------------------ storage
+@pytest.mark.parametrize("bits,rows,n,g,use_gidx", [
+    (4, 7, 64, 16, False), (4, 33, 256, 128, True), (4, 5, 24, -1, False),
+    (3, 9, 96, 32, False), (3, 17, 256, 128, True), (3, 3, 32, -1, False)])
+def test_pack_and_dequant_bit_exact(bits, rows, n, g, use_gidx):
+    rng = np.random.default_rng(bits * 1000 + n)
+    codes = rng.integers(0, 2 ** bits, (rows, n))
+    G_ = 1 if g <= 0 else (n + g - 1) // g
+    scales = rng.uniform(1e-4, 0.2, (rows, G_)).astype(np.float32)
+    zeros = rng.integers(0, 2 ** bits, (rows, G_))
+    gidx = rng.integers(0, G_, n) if use_gidx else None
+    cd = torch.from_numpy(codes.astype(np.uint8)).cuda()
+    packed = G.gptq_pack_int4(cd) if bits == 4 else G.gptq_pack_int3(cd)
+    ref = O.pack_int4(codes) if bits == 4 else O.pack_int3(codes)
+    got = packed.cpu().numpy().view(np.uint32)
+    assert np.array_equal(got, ref)
+    sd = torch.from_numpy(scales).cuda()
+    zd = torch.from_numpy(zeros.astype(np.uint8)).cuda()
+    gd = torch.from_numpy(gidx.astype(np.int32)).cuda() if use_gidx else None
+    w32 = G.gptq_dequant(packed, bits, n, sd, zd, g, gd, torch.float32)
+    ref32 = O.dequant(ref, bits, n, scales, zeros, g, gidx)
+    assert np.array_equal(w32.cpu().numpy(), ref32)
+    w16 = G.gptq_dequant(packed, bits, n, sd, zd, g, gd, torch.bfloat16)
+    ref16 = O.dequant(ref, bits, n, scales, zeros, g, gidx, out="bf16")
+    assert np.array_equal(w16.view(torch.int16).cpu().numpy().view(np.uint16), ref16)
+
+
+def test_pack_int4_unaligned_row_length():
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, 16, (6, 40))          # n % 32 != 0: the 8-code path
+    packed = G.gptq_pack_int4(torch.from_numpy(codes.astype(np.uint8)).cuda())
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), O.pack_int4(codes))
+
+
+# ------------------------------------------------------------------ Hessian
+@pytest.mark.parametrize("n,ntok,dtype", [
+    (256, 2048, torch.float32), (6, 100, torch.bfloat16), (130, 1000, torch.bfloat16),
+    (257, 333, torch.bfloat16), (384, 4096, torch.bfloat16), (520, 70, torch.float32),
+    (1000, 3000, torch.bfloat16)])
+def test_hessian_matches_oracle(n, ntok, dtype):
+    _, X = workloads.random_layer(1, n, ntok, seed=n + ntok, dtype=dtype)
+    H = torch.zeros(n, n, dtype=torch.float32, device="cuda")
+    G.gptq_hessian_accumulate(H, device_x(X))
+    Hg = to_np(H).astype(np.float64)
+    Ho = O.hessian(to_np(X))
+    assert np.array_equal(Hg, Hg.T)
+    assert np.linalg.norm(Hg - Ho) / np.linalg.norm(Ho) <= 1e-4
+
+
+def test_hessian_accumulates_over_batches_and_alpha():
+    _, X = workloads.random_layer(1, 192, 1536, seed=3, dtype=torch.bfloat16)
+    H = torch.zeros(192, 192, dtype=torch.float32, device="cuda")
+    Xd = device_x(X)
+    G.gptq_hessian_accumulate(H, Xd[:, :512])
+    G.gptq_hessian_accumulate(H, Xd[:, 512:1024])
+    G.gptq_hessian_accumulate(H, Xd[:, 1024:], alpha=1.0)
+    Xn = to_np(X).astype(np.float64)
+    Ho = 2.0 * Xn[:, :1024] @ Xn[:, :1024].T + Xn[:, 1024:] @ Xn[:, 1024:].T
+    Hg = to_np(H)
+    assert np.linalg.norm(Hg - Ho) / np.linalg.norm(Ho) <= 1e-4
+
+
+def test_hessian_zero_tokens_is_a_no_op():
+    H = torch.full((16, 16), 3.0, device="cuda")
+    X = torch.zeros(16, 8, dtype=torch.bfloat16, device="cuda")
+    G.gptq_hessian_accumulate(H, X[:, :0])
+    assert torch.all(H == 3.0)
+
+
+# ------------------------------------------------------------------ Cholesky
+@pytest.mark.parametrize("n,actorder,dead", [(6, False, ()), (130, True, (7,)),
+                                             (256, False, ()), (300, True, (0, 299)),
+                                             (640, True, ())])
+def test_cholesky_inverse_matches_oracle(n, actorder, dead):
+    _, X = workloads.random_layer(1, n, 3 * n + 50, seed=n, dead=dead, correlated=0.3)
+    Ho32 = O.hessian(to_np(X)).astype(np.float32)          # the oracle's own H, as fp32
+    H = torch.from_numpy(Ho32).cuda()
+    U, perm, dead_d, info = G.gptq_cholesky_inverse(H, 0.01, actorder)
+    torch.cuda.synchronize()
+    assert int(info.item()) == 0
+    W = np.zeros((1, n))
+    prep = O.prepare(Ho32.astype(np.float64), W, 0.01, actorder,
+                     forced_perm=perm.cpu().numpy() if actorder else None)
+    Uo = O.upper_cholesky_of_inverse(prep["Hp"])
+    Ug = to_np(U).astype(np.float64)
+    assert np.all(np.tril(Ug, -1) == 0)
+    assert np.linalg.norm(Ug - Uo) / np.linalg.norm(Uo) <= 1e-4
+    assert np.array_equal(dead_d.cpu().numpy().astype(bool), prep["dead"])
+    if not actorder:
+        assert np.array_equal(perm.cpu().numpy(), np.arange(n))
+
+
+def test_cholesky_reports_failures_in_info():
+    n = 200
+    H = -torch.eye(n, device="cuda")
+    _, _, _, info = G.gptq_cholesky_inverse(H, 0.0, False)
+    assert int(info.item()) > 0            # not positive definite
+    H = torch.eye(n, device="cuda")
+    H[5, 5] = float("nan")
+    _, _, _, info = G.gptq_cholesky_inverse(H, 0.01, True)
+    assert int(info.item()) == -1
+    H = torch.eye(n, device="cuda") * 2.0
+    _, _, _, info = G.gptq_cholesky_inverse(H, 0.01, True)
+    assert int(info.item()) == 0           # the context is still usable
+
+
+def test_scale_equivariance_on_gpu():
+    _, X = workloads.random_layer(1, 256, 900, seed=17, correlated=0.4)
+    Ho32 = O.hessian(to_np(X)).astype(np.float32)
+    W = workloads.random_layer(40, 256, 1, seed=18)[0].cuda()
+    cfg = G.make_config(4, 128, 0.01, True)
+    outs = []
+    for s in (1.0, 4.0):
+        H = torch.from_numpy(Ho32 * np.float32(s)).cuda()
+        U, perm, dead, info = G.gptq_cholesky_inverse(H, 0.01, True)
+        q = G.gptq_quantize_layer(W, U, perm, dead, cfg)
+        outs.append((U.clone(), q["codes"].clone(), perm.clone()))
+    assert torch.equal(outs[0][2], outs[1][2])
+    assert torch.equal(outs[0][0] * 0.5, outs[1][0])
+    assert torch.equal(outs[0][1], outs[1][1])
+
+
+# ------------------------------------------------------------------ whole layer
+LAYERS = [
+    # rows, n, ntok, bits, group, actorder, dtype, dead
+    (256, 256, 2048, 4, -1, False, torch.float32, ()),     # the 256x256 fp32 layer, full size
+    (200, 300, 1000, 4, 128, True, torch.bfloat16, (17,)),
+    (64, 384, 1500, 3, 128, False, torch.bfloat16, ()),
+    (48, 256, 800, 4, 32, True, torch.bfloat16, ()),
+    (48, 256, 800, 4, 64, False, torch.float32, (3,)),
+    (33, 512, 1200, 4, 256, True, torch.bfloat16, ()),
+    (4, 6, 64, 2, -1, False, torch.float32, ()),
+    (1, 130, 300, 4, -1, True, torch.bfloat16, ()),
+    (130, 257, 700, 8, 128, True, torch.bfloat16, ()),
+]
+
+
+@pytest.mark.parametrize("rows,n,ntok,bits,g,act,dtype,dead", LAYERS)
+def test_layer_matches_oracle(rows, n, ntok, bits, g, act, dtype, dead):
+    if (rows, n) == (256, 256):
+        wl = workloads.WORKLOADS["layer256"]
+        W, X = workloads.make_inputs(wl)
+    else:
+        W, X = workloads.random_layer(rows, n, ntok, seed=rows * 7 + n, dtype=dtype, dead=dead,
+                                      correlated=0.3)
+    gpu = gpu_layer(W, X, bits, g, 0.01, act)
+    compare_layer(gpu, W, X, bits, g, 0.01, act)
+
+
+@pytest.mark.parametrize("g,act", [(-1, False), (128, False), (128, True), (32, True)])
+def test_identity_hessian_gives_rtn_on_gpu(g, act):
+    n, rows = 256, 24
+    gains = np.linspace(0.5, 3.0, n)[np.random.default_rng(1).permutation(n)]
+    X = workloads.identity_calibration(n, 4, gains, dtype=torch.bfloat16)
+    W = workloads.random_layer(rows, n, 1, seed=2)[0]
+    gpu = gpu_layer(W, X, 4, g, 0.01, act)
+    Ho = O.hessian(to_np(X))
+    prep = O.prepare(Ho, to_np(W).astype(np.float64), 0.01, act)
+    assert np.array_equal(gpu["perm"], prep["perm"])
+    base = O.rtn(prep["Wp"], 4, g)
+    assert np.array_equal(gpu["codes"][:, prep["perm"]], base["codes"])
+    assert np.array_equal(gpu["zeros"], base["zeros"])
+    assert np.array_equal(gpu["scales"], base["scales"])
+
+
+def test_empty_rows_is_a_no_op():
+    cfg = G.make_config(4, 128, 0.01, False)
+    W = torch.zeros(0, 128, dtype=torch.bfloat16, device="cuda")
+    U = torch.eye(128, device="cuda")
+    perm = torch.arange(128, dtype=torch.int32, device="cuda")
+    dead = torch.zeros(128, dtype=torch.uint8, device="cuda")
+    q = G.gptq_quantize_layer(W, U, perm, dead, cfg)
+    assert q["codes"].shape == (0, 128)
+
+
+def test_quantize_linear_end_to_end():
+    W, X = workloads.random_layer(64, 256, 1024, seed=99, dtype=torch.bfloat16, correlated=0.3)
+    ql = G.quantize_linear(W.cuda(), device_x(X), bits=4, group_size=128, actorder=True,
+                           want_wq=True)
+    torch.cuda.synchronize()
+    assert int(ql.info.item()) == 0
+    w = G.gptq_dequant(ql.packed, 4, 256, ql.scales, ql.zeros, 128, ql.g_idx)
+    assert torch.equal(w, ql.Wq)

@@ -419,3 +419,27 @@ def test_planted_mistakes_are_caught():
     flipped = 2 * np.diag(np.diag(U)) - U                             # sign of the repair
     assert identity_gap(flipped) > 1e-3
     assert identity_gap(U, lam_term=False) > 1e-6                     # dropped term
+
+
+def test_forced_actorder_accepts_only_near_ties():
+    d = np.array([5.0, 3.0, 3.0 + 1e-7, 1.0])
+    H = np.diag(d)
+    W = np.full((1, 4), 0.1)
+    own = O.prepare(H, W, 0.0, True)["perm"]
+    assert list(own) == [0, 2, 1, 3]
+    swapped = O.prepare(H, W, 0.0, True, forced_perm=[0, 1, 2, 3])["perm"]
+    assert list(swapped) == [0, 1, 2, 3]                 # 3 vs 3+1e-7: a near tie
+    with pytest.raises(ValueError):
+        O.prepare(H, W, 0.0, True, forced_perm=[1, 0, 2, 3])   # 5 vs 3: not a tie
+    with pytest.raises(ValueError):
+        O.prepare(H, W, 0.0, True, forced_perm=[0, 0, 2, 3])   # not a permutation
+
+
+def test_hessian_symmetric_blas_route_equals_plain_product():
+    rng = np.random.default_rng(91)
+    X = rng.standard_normal((520, 300)).astype(np.float32)
+    H = O.hessian(X, token_chunk=128)
+    Xd = X.astype(np.float64)
+    ref = 2.0 * Xd @ Xd.T
+    assert np.array_equal(H, H.T)
+    assert np.linalg.norm(H - ref) / np.linalg.norm(ref) < 1e-14
