@@ -19,6 +19,7 @@ the same workload per step (see cpu_sample()).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import json
 import os
@@ -43,6 +44,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="q_proj_7b")
+    p.add_argument("--tokens", type=int, default=0,
+                   help="override the workload's calibration token count (profiling runs)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -189,6 +192,8 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     wl = workloads.WORKLOADS[args.workload]
+    if args.tokens:
+        wl = dataclasses.replace(wl, ntok=args.tokens)
     dev = torch.device("cuda", local_rank)
     W, X = workloads.make_inputs(wl, device=dev)
     rows, n, N = wl.rows, wl.n, wl.ntok
