@@ -120,6 +120,21 @@ gptq_status gptq_cholesky_inverse(const float* H, int64_t n, float percdamp, int
                                   float* U, int32_t* perm, uint8_t* dead, int32_t* info,
                                   void* ws, size_t ws_bytes, void* stream);
 
+/* gptq_cholesky_inverse for callers that cannot allocate device memory.
+ * The pages have no counterpart of this entry point; it exists for host
+ * programs that own all device memory in a fixed pool and forbid allocation
+ * while running, so they can neither call cudaMalloc nor pass a workspace.
+ * Same arguments, results and `info` contract as gptq_cholesky_inverse, minus
+ * the workspace: the scratch is a 16.8 MB array built into the library, so
+ * n must be <= 2048 (larger n returns GPTQ_ERR_WORKSPACE).  The library looks
+ * up that array's device address once per device, in the first call made with
+ * that device current; make that first call before any stream capture.  All
+ * calls share the array: calls that overlap on the GPU race on it, so the
+ * caller must serialise them (e.g. one stream).  No call allocates memory. */
+gptq_status gptq_cholesky_inverse_noalloc(const float* H, int64_t n, float percdamp,
+                                          int actorder, float* U, int32_t* perm, uint8_t* dead,
+                                          int32_t* info, void* stream);
+
 /* The column sweep with lazy block updates (page "GPTQ, with the code open",
  * sections "The repair rule", "From one repair to a whole model" and "What
  * quantization is, and why anyone bothers").  For each column j of the sweep

@@ -144,6 +144,20 @@ def gptq_cholesky_inverse(H: torch.Tensor, percdamp: float = 0.01, actorder: boo
     return U, perm, dead, info
 
 
+def gptq_cholesky_inverse_noalloc(H: torch.Tensor, percdamp: float, actorder: bool, U, perm,
+                                  dead, info, stream=None):
+    """gptq_cholesky_inverse for callers that cannot allocate device memory:
+    every output buffer is the caller's and the scratch is built into the
+    library (n <= 2048).  Nothing is allocated here either."""
+    _need_cuda(H, U, perm, dead, info)
+    n = H.shape[0]
+    st = library().gptq_cholesky_inverse_noalloc(_p(H), n, float(percdamp), int(bool(actorder)),
+                                                 _p(U), _p(perm), _p(dead), _p(info),
+                                                 _stream(stream))
+    _check(st, "gptq_cholesky_inverse_noalloc")
+    return U, perm, dead, info
+
+
 def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, perm, dead, cfg: GptqConfig,
                         codes=None, scales=None, zeros=None, g_idx=None, Wq=None, row_loss=None,
                         want_g_idx: bool = True, want_wq: bool = False, want_loss: bool = False,

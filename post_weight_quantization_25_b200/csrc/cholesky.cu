@@ -390,3 +390,70 @@ cudaError_t launch_cholesky_inverse(const float* H, int64_t n64, float percdamp,
 }
 
 }  // namespace gptq
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of gptq_cholesky_inverse.
+//
+// Some callers cannot allocate device memory at the time they quantize: a
+// host program that hands out all device memory from its own fixed pool and
+// forbids allocation once it is running (a serving process, a plugin inside
+// another runtime) can neither call cudaMalloc nor give this library a
+// workspace.  For them the factorisation's scratch lives in the array below,
+// which is part of the library image: every GPU that loads the library holds
+// these bytes until the process exits.
+//
+// Limit: n <= kNoAllocMaxN (2048), i.e. the scratch of one 2048 x 2048
+// factorisation, 16.8 MB.  Larger n is rejected with GPTQ_ERR_WORKSPACE.
+//
+// The array's name in host code is only a host-side stand-in, not a device
+// address.  The device address is looked up with cudaGetSymbolAddress once
+// per device, with that device current, by the first call made on it; that
+// first call should therefore come before any stream capture.  Every call
+// shares the one array: calls whose kernels overlap on the GPU (on different
+// streams, or from different threads) race on it and must be serialised by
+// the caller.  Nothing in the array has to start at zero: every byte a call
+// reads is written earlier in that same call.
+#include <mutex>
+
+namespace {
+
+constexpr int64_t kNoAllocMaxN = 2048;
+constexpr size_t kNoAllocBytes =
+    ((sizeof(float) * kNoAllocMaxN * kNoAllocMaxN + 255) / 256) * 256 +
+    ((sizeof(float) * kNoAllocMaxN + 255) / 256) * 256 + 256;
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_chol_scratch[kNoAllocBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kNoAllocMaxDevices] = {};
+
+}  // namespace
+
+extern "C" gptq_status gptq_cholesky_inverse_noalloc(const float* H, int64_t n, float percdamp,
+                                                     int actorder, float* U, int32_t* perm,
+                                                     uint8_t* dead, int32_t* info, void* stream) {
+  if (!H || !U || !dead || !info || n <= 0) return GPTQ_ERR_INVALID_ARG;
+  if (actorder && !perm) return GPTQ_ERR_INVALID_ARG;
+  if (!(percdamp >= 0.f)) return GPTQ_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(H) % 4 != 0 || reinterpret_cast<uintptr_t>(U) % 16 != 0)
+    return GPTQ_ERR_INVALID_ARG;
+  if (n > kNoAllocMaxN || gptq::cholesky_workspace_bytes(n) > kNoAllocBytes)
+    return GPTQ_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GPTQ_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return GPTQ_ERR_UNSUPPORTED;
+  void* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_chol_scratch) != cudaSuccess || !p) return GPTQ_ERR_CUDA;
+      g_scratch_addr[dev] = p;
+    }
+    ws = g_scratch_addr[dev];
+  }
+  const cudaError_t e = gptq::launch_cholesky_inverse(H, n, percdamp, actorder, U, perm, dead,
+                                                      info, ws, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
+}
