@@ -114,7 +114,8 @@ gptq_status gptq_hessian_accumulate(float* H, const void* X, gptq_dtype xt, int6
  * info (device int32, required): 0 on success; k > 0 if H' was found not
  * positive definite at sweep position k - 1 (the factorisation runs from the
  * last sweep position towards the first, so this is the highest failing
- * position); -1 if diag(H) holds a NaN or an infinity.  On failure U is
+ * position); -1 if diag(H) holds a NaN or an infinity; -2 if a bounded wait
+ * inside a tensor-core kernel gave up.  On failure U is
  * undefined.  ws: gptq_workspace_size(GPTQ_OP_CHOLESKY, 0, n, 0, .., NULL). */
 gptq_status gptq_cholesky_inverse(const float* H, int64_t n, float percdamp, int actorder,
                                   float* U, int32_t* perm, uint8_t* dead, int32_t* info,
@@ -125,7 +126,7 @@ gptq_status gptq_cholesky_inverse(const float* H, int64_t n, float percdamp, int
  * programs that own all device memory in a fixed pool and forbid allocation
  * while running, so they can neither call cudaMalloc nor pass a workspace.
  * Same arguments, results and `info` contract as gptq_cholesky_inverse, minus
- * the workspace: the scratch is a 16.8 MB array built into the library, so
+ * the workspace: the scratch is an 18.9 MB array built into the library, so
  * n must be <= 2048 (larger n returns GPTQ_ERR_WORKSPACE).  The library looks
  * up that array's device address once per device, in the first call made with
  * that device current; make that first call before any stream capture.  All

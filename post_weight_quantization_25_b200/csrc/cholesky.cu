@@ -32,22 +32,33 @@
 #include <cmath>
 #include <cstdint>
 
-#include "gemm_f32.cuh"
 #include "gptq_internal.cuh"
+#include "panel_gemm.cuh"
+#include "stage.cuh"
 
 namespace gptq {
 namespace {
 
 constexpr int kPanel = kBlock;  // 128
 constexpr int kPadLD = kPanel + 1;
+constexpr int32_t kInfoTimeout = -2;  // `info` value when a device wait gave up
 
 struct CholWs {
   float* A;       // n x n, lower part used: J P^T H P J + lambda I
   float* dprime;  // n: diag(H) with dead entries set to 1
   double* lam;    // 1: damping
+  float* PBh;     // n x 128: the current panel's solved vectors, TF32 part
+  float* PBl;     // n x 128: remainder
 };
 
-size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace bytes for order n (also sizes the built-in scratch of the
+// allocation-free entry point below, hence constexpr).
+constexpr size_t chol_ws_bytes(int64_t n) {
+  return align_up(sizeof(float) * n * n, 256) + align_up(sizeof(float) * n, 256) + 256 +
+         2 * align_up(sizeof(float) * n * kPanel, 256);
+}
 
 CholWs carve(void* ws, int64_t n) {
   char* p = static_cast<char*>(ws);
@@ -57,6 +68,10 @@ CholWs carve(void* ws, int64_t n) {
   w.dprime = reinterpret_cast<float*>(p);
   p += align_up(sizeof(float) * n, 256);
   w.lam = reinterpret_cast<double*>(p);
+  p += 256;
+  w.PBh = reinterpret_cast<float*>(p);
+  p += align_up(sizeof(float) * n * kPanel, 256);
+  w.PBl = reinterpret_cast<float*>(p);
   return w;
 }
 
@@ -149,141 +164,301 @@ __global__ void set_diag_one_kernel(float* __restrict__ M, int n) {
 }
 
 // ---------------------------------------------------------------- panel (a)
-// Factor the diagonal block of panel p in place (lower part of A).  Uses the
-// unscaled (LDL^T-like) right-looking form -- one barrier per column -- and
-// scales by 1/sqrt(pivot) at the end.
+// Factor the diagonal block of panel p in place (lower part of A).
+//
+// Blocked over four 32-column sub-panels, block kept in shared memory:
+//  (1) one warp factors the 32 x 32 diagonal sub-block in registers (lane i
+//      holds row i): per column one shuffle for the pivot, then the column's
+//      entries are shuffled to the lanes that need them -- no barriers;
+//  (2) the rows below it solve against that factor in parallel (one thread
+//      per row, 32 entries in registers, the factor read as broadcasts);
+//  (3) all threads subtract the rank-32 product from the remaining lower
+//      block with 4 x 4 register tiles.
+__device__ __forceinline__ float chol_elem(const float* S, int r, int c) {
+  return S[r * kPadLD + c];
+}
+
 __global__ void __launch_bounds__(256) chol_diag_kernel(float* __restrict__ A, int n, int p,
                                                         int32_t* __restrict__ info) {
   if (*(volatile int32_t*)info != 0) return;
   extern __shared__ float dyn_smem[];
-  float(*S)[kPadLD] = reinterpret_cast<float(*)[kPadLD]>(dyn_smem);
+  float* S = dyn_smem;                     // [128][kPadLD]
+  float* rdiag = dyn_smem + kPanel * kPadLD;  // [128]
+  __shared__ int fail;
   const int kb = p * kPanel;
   const int bs = min(kPanel, n - kb);
-  const int tid = threadIdx.x;
-  for (int i = tid; i < kPanel * kPanel; i += blockDim.x) {
-    const int r = i / kPanel, c = i % kPanel;
-    float v = (r == c) ? 1.f : 0.f;
-    if (r < bs && c <= r) v = A[(int64_t)(kb + r) * n + kb + c];
-    S[r][c] = v;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool vec = (n % 4) == 0;
+  // stage the lower block (identity padding), 8 float4 loads in flight per thread
+  for (int f0 = 0; f0 < kPanel * kPanel / 4; f0 += 8 * 256) {
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int f = f0 + u * 256 + tid;
+      const int r = f >> 5, c = (f & 31) * 4;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < bs && c <= r) {
+        const float* src = A + (int64_t)(kb + r) * n + kb + c;
+        if (vec && c + 3 < bs) {
+          v[u] = *reinterpret_cast<const float4*>(src);
+        } else {
+          v[u].x = src[0];
+          if (c + 1 < bs) v[u].y = src[1];
+          if (c + 2 < bs) v[u].z = src[2];
+          if (c + 3 < bs) v[u].w = src[3];
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int f = f0 + u * 256 + tid;
+      const int r = f >> 5, c = (f & 31) * 4;
+      float* d = S + r * kPadLD + c;
+      d[0] = (r == c) ? (r < bs ? v[u].x : 1.f) : v[u].x;
+      d[1] = (r == c + 1) ? (r < bs ? v[u].y : 1.f) : v[u].y;
+      d[2] = (r == c + 2) ? (r < bs ? v[u].z : 1.f) : v[u].z;
+      d[3] = (r == c + 3) ? (r < bs ? v[u].w : 1.f) : v[u].w;
+    }
   }
+  if (tid == 0) fail = 0;
   __syncthreads();
-  const int r = tid & (kPanel - 1);
-  const int half = tid >> 7;
-  for (int c = 0; c < bs; ++c) {
-    const float d = S[c][c];
-    if (!(d > 0.f) || !isfinite(d)) {  // same value in every thread: uniform exit
-      if (tid == 0) atomicCAS(info, 0, n - (kb + c));
+
+  for (int c0 = 0; c0 < bs; c0 += 32) {
+    // (1) 32 x 32 diagonal sub-block, one warp, registers
+    if (warp == 0) {
+      float a[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) a[k] = (k <= lane) ? chol_elem(S, c0 + lane, c0 + k) : 0.f;
+      bool bad = false;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float d = __shfl_sync(0xffffffffu, a[j], j);
+        if (!bad && (!(d > 0.f) || !isfinite(d))) {  // uniform across the warp
+          bad = true;                                // (results below are discarded)
+          if (lane == 0) fail = c0 + j + 1;
+        }
+        const float sd = sqrtf(d);
+        const float l = (lane == j) ? sd : a[j] / sd;  // L[c0+lane][c0+j]
+        a[j] = (lane >= j) ? l : 0.f;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          if (k > j) {
+            const float lk = __shfl_sync(0xffffffffu, l, k);  // L[c0+k][c0+j]
+            if (lane >= k) a[k] = fmaf(-l, lk, a[k]);
+          }
+        }
+      }
+      if (!bad) {
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          if (k <= lane) S[(c0 + lane) * kPadLD + c0 + k] = a[k];
+        __syncwarp();
+        rdiag[c0 + lane] = 1.f / chol_elem(S, c0 + lane, c0 + lane);
+      }
+    }
+    __syncthreads();
+    if (fail) {
+      if (tid == 0) atomicCAS(info, 0, n - (kb + fail - 1));
       return;
     }
-    if (r > c && r < bs) {
-      const float lrc = S[r][c] / d;
-      for (int s2 = c + 1 + half; s2 <= r; s2 += 2) S[r][s2] = fmaf(-lrc, S[s2][c], S[r][s2]);
+    // (2) rows below the sub-block: x <- x L_sub^-T, one thread per row
+    const int rem = bs - c0 - 32;
+    if (tid < rem) {
+      const int r = c0 + 32 + tid;
+      float x[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) x[k] = chol_elem(S, r, c0 + k);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        x[j] *= rdiag[c0 + j];
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          if (k > j) x[k] = fmaf(-x[j], chol_elem(S, c0 + k, c0 + j), x[k]);
+      }
+#pragma unroll
+      for (int k = 0; k < 32; ++k) S[r * kPadLD + c0 + k] = x[k];
+    }
+    __syncthreads();
+    // (3) trailing lower block [c0+32, bs)^2 -= rank-32 product, 4 x 4 tiles
+    if (rem > 0) {
+      const int mt = (rem + 3) / 4;
+      const int ntiles = mt * (mt + 1) / 2;
+      const int base = c0 + 32;
+      for (int t = tid; t < ntiles; t += blockDim.x) {
+        int ti = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
+        while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
+        while (ti * (ti + 1) / 2 > t) --ti;
+        const int tj = t - ti * (ti + 1) / 2;
+        const int r0 = base + 4 * ti, s0 = base + 4 * tj;
+        float acc[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+          float ra[4], sa[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) ra[i] = chol_elem(S, min(r0 + i, kPanel - 1), c0 + k);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) sa[j] = chol_elem(S, min(s0 + j, kPanel - 1), c0 + k);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(ra[i], sa[j], acc[i][j]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (r0 + i < bs && s0 + j < bs) S[(r0 + i) * kPadLD + s0 + j] -= acc[i][j];
+      }
     }
     __syncthreads();
   }
-  for (int i = tid; i < bs * bs; i += blockDim.x) {
-    const int rr = i / bs, c = i % bs;
-    if (c > rr) continue;
-    const float sd = sqrtf(S[c][c]);
-    A[(int64_t)(kb + rr) * n + kb + c] = (rr == c) ? sd : S[rr][c] / sd;
+  for (int i = tid; i < bs * kPanel; i += blockDim.x) {
+    const int rr = i / kPanel, c = i % kPanel;
+    if (c <= rr) A[(int64_t)(kb + rr) * n + kb + c] = S[rr * kPadLD + c];
   }
 }
 
 // ---------------------------------------------------------------- panel (b)
 // v <- L_pp^-1 v for every vector: the rows of A below the panel
-// (restricted to the panel's columns) and rows [0, kb + bs) of RT.  One warp
-// per vector; lane l holds entries l, l+32, l+64, l+96.
-__global__ void __launch_bounds__(256) panel_solve_kernel(float* __restrict__ A,
-                                                          float* __restrict__ RT, int n, int p,
-                                                          const int32_t* __restrict__ info) {
+// (restricted to the panel's columns) and rows [0, kb + bs) of RT.
+// Four lanes (a quad) per vector, eight vectors per warp; lane q holds
+// entries q, q+4, ..., q+124 (slot s = entry / 4).  Step j: the owner lane
+// (j % 4) scales entry j by 1/L_jj, the quad shares it, and every lane
+// subtracts it times column j of L from its later entries.  Shared memory
+// holds Lq[j][q][s] = L[4 s + q][j] (pitch 36 floats: float4 reads, no bank
+// conflicts); unrolled over j so finished slots cost nothing.
+constexpr int kSolveThreads = 128;
+constexpr int kLqPitch = 36;
+constexpr int kLqRow = 4 * kLqPitch;
+constexpr size_t kSolveSmemBytes = sizeof(float) * (kPanel * kLqRow + kPanel);
+
+// Every solved vector is also written, split into its TF32 part and the
+// remainder, to row `g` of the panel buffer PBh / PBl (g = the vector's row
+// in A or RT), the operand of the tensor-core trailing update.  Rows of A
+// below the panel are not written back: only the trailing update reads them.
+__global__ void __launch_bounds__(kSolveThreads) panel_solve_kernel(
+    float* __restrict__ A, float* __restrict__ RT, int n, int p, float* __restrict__ PBh,
+    float* __restrict__ PBl, const int32_t* __restrict__ info) {
   if (*(volatile const int32_t*)info != 0) return;
-  extern __shared__ float dyn_smem[];
-  float(*L)[kPadLD] = reinterpret_cast<float(*)[kPadLD]>(dyn_smem);
-  float* rdiag = dyn_smem + kPanel * kPadLD;
+  extern __shared__ __align__(16) float dyn_smem[];
+  float* Lq = dyn_smem;
+  float* rdiag = dyn_smem + kPanel * kLqRow;
   const int kb = p * kPanel;
   const int bs = min(kPanel, n - kb);
-  for (int i = threadIdx.x; i < kPanel * kPanel; i += blockDim.x) {
-    const int r = i / kPanel, c = i % kPanel;
-    float v = (r == c) ? 1.f : 0.f;
-    if (r < bs && c <= r) v = A[(int64_t)(kb + r) * n + kb + c];
-    L[r][c] = v;
-  }
+  stage_block_128<kSolveThreads>(
+      A + (int64_t)kb * n + kb, n, bs, bs, /*lower=*/true, (n % 4) == 0,
+      [&](int r, int c, float v) { Lq[c * kLqRow + (r & 3) * kLqPitch + (r >> 2)] = v; },
+      [](int r, int c) { return (r == c) ? 1.f : 0.f; });
   __syncthreads();
-  for (int i = threadIdx.x; i < kPanel; i += blockDim.x) rdiag[i] = 1.f / L[i][i];
+  for (int i = threadIdx.x; i < kPanel; i += blockDim.x)
+    rdiag[i] = 1.f / Lq[i * kLqRow + (i & 3) * kLqPitch + (i >> 2)];
   __syncthreads();
 
+  const int q = threadIdx.x & 3;
   const int lane = threadIdx.x & 31;
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int nwarps = (gridDim.x * blockDim.x) >> 5;
   const int nA = n - kb - bs;
   const int nvec = nA + kb + bs;
-  for (int v = warp; v < nvec; v += nwarps) {
-    float* vec = (v < nA) ? (A + (int64_t)(kb + bs + v) * n + kb) : (RT + (int64_t)(v - nA) * n + kb);
-    float x[4];
+  const int quads = (gridDim.x * blockDim.x) >> 2;
+  const float* lq_lane = Lq + q * kLqPitch;
+  // `base` is the warp's first vector: uniform across the warp, so the whole
+  // warp stays in the loop together (the shuffles need all 32 lanes)
+  for (int base = (blockIdx.x * blockDim.x + (threadIdx.x & ~31)) >> 2; base < nvec;
+       base += quads) {
+    const int v0 = base + (lane >> 2);
+    const bool active = v0 < nvec;
+    float* vec = !active ? nullptr
+                 : (v0 < nA) ? (A + (int64_t)(kb + bs + v0) * n + kb)
+                             : (RT + (int64_t)(v0 - nA) * n + kb);
+    float x[32];
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      const int col = lane + 32 * s;
-      x[s] = (col < bs) ? vec[col] : 0.f;
+    for (int s = 0; s < 32; ++s) {
+      const int c = 4 * s + q;
+      x[s] = (active && c < bs) ? vec[c] : 0.f;
     }
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-#pragma unroll 4
-      for (int l = 0; l < 32; ++l) {
-        const int j = 32 * s + l;
-        if (j >= bs) break;
-        float y = 0.f;
-        if (lane == l) {
-          y = x[s] * rdiag[j];
-          x[s] = y;
-        }
-        y = __shfl_sync(0xffffffffu, y, l);
+    for (int s = 0; s < 32; ++s) {
 #pragma unroll
-        for (int s2 = s; s2 < 4; ++s2) {
-          const int i = lane + 32 * s2;
-          if (i > j) x[s2] = fmaf(-L[i][j], y, x[s2]);
+      for (int k = 0; k < 4; ++k) {
+        const int j = 4 * s + k;
+        if (j >= bs) break;
+        const float yv = x[s] * rdiag[j];
+        const float y = __shfl_sync(0xffffffffu, yv, k, 4);
+        const float* lcol = lq_lane + j * kLqRow;
+#pragma unroll
+        for (int s4 = s >> 2; s4 < 8; ++s4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lcol + 4 * s4);
+          if (4 * s4 + 0 >= s) x[4 * s4 + 0] = fmaf(-l4.x, y, x[4 * s4 + 0]);
+          if (4 * s4 + 1 >= s) x[4 * s4 + 1] = fmaf(-l4.y, y, x[4 * s4 + 1]);
+          if (4 * s4 + 2 >= s) x[4 * s4 + 2] = fmaf(-l4.z, y, x[4 * s4 + 2]);
+          if (4 * s4 + 3 >= s) x[4 * s4 + 3] = fmaf(-l4.w, y, x[4 * s4 + 3]);
         }
+        if (q == k) x[s] = y;
       }
     }
+    if (active) {
+      const bool is_rt = v0 >= nA;
+      const int64_t g = is_rt ? (int64_t)(v0 - nA) : (int64_t)(kb + bs + v0);
+      float* ph = PBh + g * kPanel;
+      float* pl = PBl + g * kPanel;
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      const int col = lane + 32 * s;
-      if (col < bs) vec[col] = x[s];
+      for (int s = 0; s < 32; ++s) {
+        const int c = 4 * s + q;
+        const float xv = (c < bs) ? x[s] : 0.f;
+        if (is_rt && c < bs) vec[c] = xv;
+        float h, l;
+        tf32_split(xv, h, l);
+        ph[c] = h;
+        pl[c] = l;
+      }
     }
   }
 }
 
-// ---------------------------------------------------------------- panel (c)
-// Tiles [0, T1): lower tiles (rb, sb), p < sb <= rb, of A -= L_p L_p^T.
-// Tiles [T1, T1+T2): RT[cb][rb] -= RT[cb][p] A[rb][p]^T, cb <= p < rb.
-__global__ void __launch_bounds__(256) trailing_kernel(float* __restrict__ A,
-                                                       float* __restrict__ RT, int n, int p,
-                                                       int nblk, const int32_t* __restrict__ info) {
-  if (*(volatile const int32_t*)info != 0) return;
-  __shared__ __align__(16) float sm[kTileSmemFloats];
-  const int m = nblk - p - 1;
-  const int T1 = m * (m + 1) / 2;
-  const int kb = p * kPanel;
-  int t = blockIdx.x;
-  if (t < T1) {
-    int rr = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
-    while ((rr + 1) * (rr + 2) / 2 <= t) ++rr;
-    while (rr * (rr + 1) / 2 > t) --rr;
-    const int ss = t - rr * (rr + 1) / 2;
-    const int rb = p + 1 + rr, sb = p + 1 + ss;
-    float* C = A + (int64_t)rb * kPanel * n + (int64_t)sb * kPanel;
-    const float* P = A + (int64_t)rb * kPanel * n + kb;
-    const float* Q = A + (int64_t)sb * kPanel * n + kb;
-    tile_sub<true>(C, n, P, n, Q, n, min(kPanel, n - rb * kPanel), min(kPanel, n - sb * kPanel),
-                   kPanel, sm);
-  } else {
-    t -= T1;
-    const int cb = t / m, rb = p + 1 + t % m;
-    float* C = RT + (int64_t)cb * kPanel * n + (int64_t)rb * kPanel;
-    const float* P = RT + (int64_t)cb * kPanel * n + kb;
-    const float* Q = A + (int64_t)rb * kPanel * n + kb;
-    tile_sub<true>(C, n, P, n, Q, n, kPanel, min(kPanel, n - rb * kPanel), kPanel, sm);
+// The trailing update of panel p as tiles for the tensor-core panel GEMM.
+// Tiles [0, T1): lower tiles (rb, sb), p < sb <= rb, of A -= L_p L_p^T;
+// tiles [T1, T1+T2): RT[cb][rb] -= RT[cb][p] L[rb][p]^T, cb <= p < rb.
+// Both operands are rows of the panel buffer (P = rows of the C tile's row
+// block, Q = rows of its column block).
+struct CholTrailDecoder {
+  float* A;
+  float* RT;
+  int n, p, nblk;
+  __device__ PgTile tile(int bx, int) const {
+    PgTile t;
+    const int m = nblk - p - 1;
+    const int T1 = m * (m + 1) / 2;
+    int idx = bx;
+    t.ldc = n;
+    t.pkx = 0;
+    t.qkx = 0;
+    if (idx < T1) {
+      int rr = (int)((sqrtf(8.f * (float)idx + 1.f) - 1.f) * 0.5f);
+      while ((rr + 1) * (rr + 2) / 2 <= idx) ++rr;
+      while (rr * (rr + 1) / 2 > idx) --rr;
+      const int ss = idx - rr * (rr + 1) / 2;
+      const int rb = p + 1 + rr, sb = p + 1 + ss;
+      t.C = A + (int64_t)rb * kPanel * n + (int64_t)sb * kPanel;
+      t.prow = rb * kPanel;
+      t.qrow = sb * kPanel;
+      t.mext = min(kPanel, n - rb * kPanel);
+      t.cext = min(kPanel, n - sb * kPanel);
+    } else {
+      idx -= T1;
+      const int cb = idx / m, rb = p + 1 + idx % m;
+      t.C = RT + (int64_t)cb * kPanel * n + (int64_t)rb * kPanel;
+      t.prow = cb * kPanel;
+      t.qrow = rb * kPanel;
+      t.mext = kPanel;
+      t.cext = min(kPanel, n - rb * kPanel);
+    }
+    t.valid = 1;
+    return t;
   }
-}
+};
 
 // ---------------------------------------------------------------- finish
 // In place: U[i][j] <- U[n-1-j][n-1-i] (an involution; it maps the upper
@@ -321,9 +496,7 @@ __global__ void anti_transpose_elems_kernel(float* __restrict__ U, int n) {
 
 }  // namespace
 
-size_t cholesky_workspace_bytes(int64_t n) {
-  return align_up(sizeof(float) * n * n, 256) + align_up(sizeof(float) * n, 256) + 256;
-}
+size_t cholesky_workspace_bytes(int64_t n) { return chol_ws_bytes(n); }
 
 cudaError_t launch_cholesky_inverse(const float* H, int64_t n64, float percdamp, int actorder,
                                     float* U, int32_t* perm, uint8_t* dead, int32_t* info,
@@ -358,23 +531,37 @@ cudaError_t launch_cholesky_inverse(const float* H, int64_t n64, float percdamp,
 
   const int nblk = (n + kPanel - 1) / kPanel;
   const int sms = num_sms();
-  const size_t diag_smem = sizeof(float) * kPanel * kPadLD;
-  const size_t solve_smem = diag_smem + sizeof(float) * kPanel;
+  const size_t diag_smem = sizeof(float) * (kPanel * kPadLD + 2 * kPanel);
+  const size_t solve_smem = kSolveSmemBytes;
   if ((e = cudaFuncSetAttribute(chol_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)diag_smem)) != cudaSuccess ||
       (e = cudaFuncSetAttribute(panel_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)solve_smem)) != cudaSuccess)
     return e;
-  const int solve_ctas = std::min((n + 7) / 8, 3 * sms);
+  // one quad per vector (n vectors per panel), capped at 3 resident CTAs per SM
+  const int solve_ctas = std::min((4 * n + kSolveThreads - 1) / kSolveThreads, 3 * sms);
+  CUtensorMap mPh, mPl;
+  if (nblk > 1) {
+    if (!make_tma_2d(&mPh, w.PBh, false, n, kPanel, kPanel, 32, 128) ||
+        !make_tma_2d(&mPl, w.PBl, false, n, kPanel, kPanel, 32, 128))
+      return cudaErrorInvalidValue;
+    if ((e = cudaFuncSetAttribute(panel_gemm_kernel<CholTrailDecoder>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kPgSmemBytes)) != cudaSuccess)
+      return e;
+  }
   for (int p = 0; p < nblk; ++p) {
     chol_diag_kernel<<<1, 256, diag_smem, s>>>(w.A, n, p, info);
     note_launch();
-    panel_solve_kernel<<<solve_ctas, 256, solve_smem, s>>>(w.A, U, n, p, info);
+    panel_solve_kernel<<<solve_ctas, kSolveThreads, solve_smem, s>>>(w.A, U, n, p, w.PBh, w.PBl,
+                                                                      info);
     note_launch();
     const int m = nblk - p - 1;
     const int tiles = m * (m + 1) / 2 + (p + 1) * m;
     if (tiles > 0) {
-      trailing_kernel<<<tiles, 256, 0, s>>>(w.A, U, n, p, nblk, info);
+      const CholTrailDecoder dec{w.A, U, n, p, nblk};
+      panel_gemm_kernel<CholTrailDecoder><<<tiles, kPgThreads, kPgSmemBytes, s>>>(
+          mPh, mPl, mPh, mPl, dec, info, kInfoTimeout, info);
       note_launch();
     }
   }
@@ -403,7 +590,7 @@ cudaError_t launch_cholesky_inverse(const float* H, int64_t n64, float percdamp,
 // these bytes until the process exits.
 //
 // Limit: n <= kNoAllocMaxN (2048), i.e. the scratch of one 2048 x 2048
-// factorisation, 16.8 MB.  Larger n is rejected with GPTQ_ERR_WORKSPACE.
+// factorisation, 18.9 MB.  Larger n is rejected with GPTQ_ERR_WORKSPACE.
 //
 // The array's name in host code is only a host-side stand-in, not a device
 // address.  The device address is looked up with cudaGetSymbolAddress once
@@ -418,9 +605,7 @@ cudaError_t launch_cholesky_inverse(const float* H, int64_t n64, float percdamp,
 namespace {
 
 constexpr int64_t kNoAllocMaxN = 2048;
-constexpr size_t kNoAllocBytes =
-    ((sizeof(float) * kNoAllocMaxN * kNoAllocMaxN + 255) / 256) * 256 +
-    ((sizeof(float) * kNoAllocMaxN + 255) / 256) * 256 + 256;
+constexpr size_t kNoAllocBytes = gptq::chol_ws_bytes(kNoAllocMaxN);
 constexpr int kNoAllocMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_chol_scratch[kNoAllocBytes];

@@ -3,6 +3,7 @@
 // the launch (cudaSuccess when nothing had to run).
 #pragma once
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/gptq.h"
@@ -13,6 +14,11 @@ constexpr int kBlock = 128;            // lazy-update block of the sweep / Chole
 constexpr int kGridWaitLimitNs = 1000000000;  // 1 s: upper bound of any in-kernel wait
 
 int num_sms();
+// 2-D TMA descriptor (128-byte swizzle, zero fill out of bounds) for a
+// row-major rows x cols matrix of bf16 (bf16 = true) or fp32 elements with a
+// row stride of ld elements; boxes of box_cols x box_rows.  Host only.
+bool make_tma_2d(CUtensorMap* map, const void* base, bool bf16, int64_t rows, int64_t cols,
+                 int64_t ld, uint32_t box_cols, uint32_t box_rows);
 // Counts one kernel enqueued by this library (read by gptq_launch_count).
 void note_launch();
 

@@ -28,8 +28,9 @@
 #include <cmath>
 #include <cstdint>
 
-#include "gemm_f32.cuh"
 #include "gptq_internal.cuh"
+#include "panel_gemm.cuh"
+#include "stage.cuh"
 
 namespace gptq {
 namespace {
@@ -38,23 +39,81 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct SweepWs {
   float* Wf;          // rows x n, sweep order; after the sweep holds w_hat
-  float* Err;         // rows x 128
+  float* Err_hi;      // rows x 128: the block's err terms, TF32 part
+  float* Err_lo;      // rows x 128: remainder (err - Err_hi)
   uint8_t* codes_sw;  // rows x n, sweep order
   int32_t* pos;       // n: sweep position of each original column
+  float* UT_hi;       // n x ldut: U^T, TF32 part (the lazy update's K-major operand)
+  float* UT_lo;       // n x ldut: remainder
+  int64_t ldut;
 };
+
+int64_t ut_ld(int64_t n) { return (n + 3) / 4 * 4; }
 
 SweepWs carve(void* ws, int64_t rows, int64_t n) {
   char* p = static_cast<char*>(ws);
   SweepWs w;
   w.Wf = reinterpret_cast<float*>(p);
   p += align_up(sizeof(float) * rows * n, 256);
-  w.Err = reinterpret_cast<float*>(p);
+  w.Err_hi = reinterpret_cast<float*>(p);
+  p += align_up(sizeof(float) * rows * kBlock, 256);
+  w.Err_lo = reinterpret_cast<float*>(p);
   p += align_up(sizeof(float) * rows * kBlock, 256);
   w.codes_sw = reinterpret_cast<uint8_t*>(p);
   p += align_up((size_t)rows * n, 256);
   w.pos = reinterpret_cast<int32_t*>(p);
+  p += align_up(sizeof(int32_t) * n, 256);
+  w.ldut = ut_ld(n);
+  w.UT_hi = reinterpret_cast<float*>(p);
+  p += align_up(sizeof(float) * n * w.ldut, 256);
+  w.UT_lo = reinterpret_cast<float*>(p);
   return w;
 }
+
+// UT[a][b] = U[b][a], split into TF32 part and remainder; columns past n are 0.
+__global__ void __launch_bounds__(256) ut_split_kernel(const float* __restrict__ U, int n,
+                                                       int64_t ldut, float* __restrict__ hi,
+                                                       float* __restrict__ lo) {
+  __shared__ float T[32][33];
+  const int bx = blockIdx.x, by = blockIdx.y;  // output tile: rows 32 by, cols 32 bx
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int i = ty; i < 32; i += 8) {
+    const int r = 32 * bx + i, c = 32 * by + tx;  // source U[r][c]
+    T[i][tx] = (r < n && c < n) ? U[(int64_t)r * n + c] : 0.f;
+  }
+  __syncthreads();
+  for (int i = ty; i < 32; i += 8) {
+    const int a = 32 * by + i, b = 32 * bx + tx;  // destination UT[a][b] = U[b][a]
+    if (a < n && b < ldut) {
+      float h, l;
+      tf32_split(T[tx][i], h, l);
+      hi[(int64_t)a * ldut + b] = h;
+      lo[(int64_t)a * ldut + b] = l;
+    }
+  }
+}
+
+// The lazy update  Wf[:, i2:] -= Err U[i1:i1+128, i2:]  as tiles for the
+// tensor-core panel GEMM: P = Err (rows x 128), Q = U^T rows i2.. (columns
+// i1..i1+128), C = Wf.
+struct SweepTrailDecoder {
+  float* Wf;
+  int rows, n, i1, i2;
+  __device__ PgTile tile(int bx, int by) const {
+    PgTile t;
+    const int c0 = bx * 128, r0 = by * 128;
+    t.C = Wf + (int64_t)r0 * n + i2 + c0;
+    t.ldc = n;
+    t.prow = r0;
+    t.pkx = 0;
+    t.qrow = i2 + c0;
+    t.qkx = i1;
+    t.mext = min(128, rows - r0);
+    t.cext = min(128, n - i2 - c0);
+    t.valid = (t.mext > 0 && t.cext > 0) ? 1 : 0;
+    return t;
+  }
+};
 
 // The ruler for values spanning [mn, mx]: range stretched to include 0
 // ([-1, 1] when flat), scale = (xmax - xmin) / maxq, zero = rint(-xmin / scale).
@@ -77,11 +136,6 @@ __device__ __forceinline__ float warp_min(float v) {
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
 
@@ -133,136 +187,181 @@ __global__ void __launch_bounds__(256) gather_w_kernel(
   if (row_loss && threadIdx.x == 0) row_loss[r] = 0.f;
 }
 
-// One block [i1, i1 + bsz) of the sweep.  One warp per row; lane l holds
-// block columns l, l+32, l+64, l+96.  Column jj is rounded by its owner lane,
-// the error term is broadcast, and every lane repairs its later columns with
-// row jj of U's diagonal block (shared memory).
-//   gmode 0: per-row ruler (already in scales / zeros)
-//   gmode 1: groups of >= 128 columns (a multiple of 128): fitted at a block
-//            start that is a group start, from the current Wf
-//   gmode 2: groups of 32 or 64 columns inside the block
-template <int GMODE>
-__global__ void __launch_bounds__(256) sweep_block_kernel(
+// One block [i1, i1 + bsz) of the sweep.  Four lanes (a "quad") per row,
+// eight rows per warp; lane q of a quad holds block columns q, q+4, ..., q+124
+// (slot s = column / 4).  Column jj is rounded in every lane of the quad, the
+// owner lane's (jj % 4) error term is broadcast inside the quad, and each lane
+// repairs its columns past jj with row jj of U's diagonal block.  The loop
+// over jj is unrolled, so slots left of jj are skipped at compile time.
+// Shared memory holds the block of U as  Uq[jj][q][slot] = U[i1+jj][i1+4 slot+q]
+// (quad-lane-major, row pitch 36 floats: 16-byte float4 reads, no bank
+// conflicts), plus 1/U_jj and 1/(2 U_jj^2).
+//   GS = 0:   per-row ruler (already in scales / zeros)
+//   GS = 128: groups of a multiple of 128 columns, fitted at a block start that
+//             is a group start, from the current Wf
+//   GS = 32, 64: groups inside the block, fitted on the current registers
+constexpr int kSweepThreads = 128;
+constexpr int kUqPitch = 36;                  // floats per (jj, q) row of Uq
+constexpr int kUqRow = 4 * kUqPitch;          // floats per jj
+constexpr size_t kSweepSmemBytes = sizeof(float) * (kBlock * kUqRow + 2 * kBlock);
+
+__device__ __forceinline__ float quad_min(float v) {
+  v = fminf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+  return fminf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+}
+__device__ __forceinline__ float quad_max(float v) {
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+  return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+}
+
+template <int GS>
+__global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
     float* __restrict__ Wf, int rows, int n, const float* __restrict__ U, int i1, int bsz,
-    float maxq, int gsize, int G, float* __restrict__ Err, uint8_t* __restrict__ codes_sw,
-    float* __restrict__ scales, uint8_t* __restrict__ zeros, float* __restrict__ row_loss) {
-  extern __shared__ float Us[];  // [128][128]: U[i1 + a][i1 + b]
-  for (int i = threadIdx.x; i < kBlock * kBlock; i += blockDim.x) {
-    const int a = i / kBlock, b = i % kBlock;
-    Us[i] = (a < bsz && b < bsz) ? U[(int64_t)(i1 + a) * n + i1 + b] : 0.f;
+    float maxq, int gsize, int G, float* __restrict__ Err_hi, float* __restrict__ Err_lo,
+    uint8_t* __restrict__ codes_sw, float* __restrict__ scales, uint8_t* __restrict__ zeros,
+    float* __restrict__ row_loss) {
+  extern __shared__ __align__(16) float smem[];
+  float* Uq = smem;
+  float* rd = smem + kBlock * kUqRow;
+  float* hrd2 = rd + kBlock;
+  stage_block_128<kSweepThreads>(
+      U + (int64_t)i1 * n + i1, n, bsz, bsz, /*lower=*/false, (n % 4) == 0,
+      [&](int a, int b, float v) { Uq[a * kUqRow + (b & 3) * kUqPitch + (b >> 2)] = v; },
+      [](int, int) { return 0.f; });
+  __syncthreads();
+  for (int i = threadIdx.x; i < kBlock; i += blockDim.x) {
+    const float d = (i < bsz) ? Uq[i * kUqRow + (i & 3) * kUqPitch + (i >> 2)] : 1.f;
+    rd[i] = 1.f / d;
+    hrd2[i] = 0.5f / (d * d);
   }
   __syncthreads();
+
   const int lane = threadIdx.x & 31;
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int nwarps = (gridDim.x * blockDim.x) >> 5;
-
-  for (int r = warp; r < rows; r += nwarps) {
-    float* wrow = Wf + (int64_t)r * n + i1;
-    float w[4];
+  const int q = lane & 3;
+  const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 2;
+  const bool active = r < rows;
+  float* wrow = Wf + (int64_t)(active ? r : 0) * n + i1;
+  float w[32];
 #pragma unroll
-    for (int s = 0; s < 4; ++s) w[s] = (lane + 32 * s < bsz) ? wrow[lane + 32 * s] : 0.f;
+  for (int s = 0; s < 32; ++s) {
+    const int c = 4 * s + q;
+    w[s] = (active && c < bsz) ? wrow[c] : 0.f;
+  }
 
-    float scale = 0.f, zf = 0.f;
-    if (GMODE == 0) {
+  float scale = 1.f, zf = 0.f;
+  if (GS == 0) {
+    if (active) {
       scale = scales[r];
       zf = (float)zeros[r];
-    } else if (GMODE == 1) {
-      const int g = i1 / gsize;
-      if (i1 % gsize == 0) {
-        const int end = min(i1 + gsize, n);
-        float mn = INFINITY, mx = -INFINITY;
-        for (int c = i1 + lane; c < end; c += 32) {
+    }
+  } else if (GS == 128) {
+    const int g = i1 / gsize;
+    if (i1 % gsize == 0) {
+      float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+      for (int s = 0; s < 32; ++s)
+        if (4 * s + q < bsz) {
+          mn = fminf(mn, w[s]);
+          mx = fmaxf(mx, w[s]);
+        }
+      const int end = min(i1 + gsize, n);
+      if (active)
+        for (int c = i1 + kBlock + q; c < end; c += 4) {
           const float v = Wf[(int64_t)r * n + c];
           mn = fminf(mn, v);
           mx = fmaxf(mx, v);
         }
-        fit_ruler(warp_min(mn), warp_max(mx), maxq, scale, zf);
-        if (lane == 0) {
-          scales[(int64_t)r * G + g] = scale;
-          zeros[(int64_t)r * G + g] = (uint8_t)zf;
-        }
-      } else {
-        scale = scales[(int64_t)r * G + g];
-        zf = (float)zeros[(int64_t)r * G + g];
+      fit_ruler(quad_min(mn), quad_max(mx), maxq, scale, zf);
+      if (active && q == 0) {
+        scales[(int64_t)r * G + g] = scale;
+        zeros[(int64_t)r * G + g] = (uint8_t)zf;
       }
-    }
-
-    float q_out[4] = {0.f, 0.f, 0.f, 0.f}, wq_out[4] = {0.f, 0.f, 0.f, 0.f},
-          e_out[4] = {0.f, 0.f, 0.f, 0.f};
-    float loss = 0.f;
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      if (32 * s >= bsz) break;
-      if (GMODE == 2 && (32 * s) % gsize == 0) {
-        // group [32 s, 32 s + gsize) of the block, current (repaired) values
-        float mn = INFINITY, mx = -INFINITY;
-#pragma unroll
-        for (int s2 = s; s2 < 4; ++s2) {
-          if (32 * (s2 - s) < gsize && lane + 32 * s2 < bsz) {
-            mn = fminf(mn, w[s2]);
-            mx = fmaxf(mx, w[s2]);
-          }
-        }
-        fit_ruler(warp_min(mn), warp_max(mx), maxq, scale, zf);
-        if (lane == 0) {
-          const int g = (i1 + 32 * s) / gsize;
-          scales[(int64_t)r * G + g] = scale;
-          zeros[(int64_t)r * G + g] = (uint8_t)zf;
-        }
-      }
-#pragma unroll 4
-      for (int l = 0; l < 32; ++l) {
-        const int jj = 32 * s + l;
-        if (jj >= bsz) break;
-        float err = 0.f;
-        if (lane == l) {
-          const float x = w[s];
-          float q = rintf(__fdiv_rn(x, scale)) + zf;
-          q = fminf(fmaxf(q, 0.f), maxq);
-          const float wh = __fmul_rn(scale, q - zf);
-          const float e = x - wh;
-          const float d = Us[jj * kBlock + jj];
-          err = __fdiv_rn(e, d);
-          loss += __fdiv_rn(e * e, 2.f * d * d);
-          q_out[s] = q;
-          wq_out[s] = wh;
-          e_out[s] = err;
-        }
-        err = __shfl_sync(0xffffffffu, err, l);
-        const float* urow = Us + jj * kBlock;
-#pragma unroll
-        for (int s2 = s; s2 < 4; ++s2) w[s2] = fmaf(-err, urow[32 * s2 + lane], w[s2]);
-      }
-    }
-    uint8_t* crow = codes_sw + (int64_t)r * n + i1;
-    float* erow = Err + (int64_t)r * kBlock;
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      const int c = lane + 32 * s;
-      if (c < bsz) {
-        crow[c] = (uint8_t)q_out[s];
-        wrow[c] = wq_out[s];
-      }
-      erow[c] = e_out[s];
-    }
-    if (row_loss) {
-      loss = warp_sum(loss);
-      if (lane == 0) row_loss[r] += loss;
+    } else if (active) {
+      scale = scales[(int64_t)r * G + g];
+      zf = (float)zeros[(int64_t)r * G + g];
     }
   }
-}
 
-// Wf[:, i2:] -= Err(rows x K) * U[i1:i1+K, i2:]   (grid: col tiles x row tiles)
-__global__ void __launch_bounds__(256) sweep_trailing_kernel(float* __restrict__ Wf, int rows,
-                                                             int n, const float* __restrict__ U,
-                                                             const float* __restrict__ Err, int i1,
-                                                             int i2, int K) {
-  __shared__ __align__(16) float sm[kTileSmemFloats];
-  const int c0 = blockIdx.x * kTileM, r0 = blockIdx.y * kTileM;
-  float* C = Wf + (int64_t)r0 * n + i2 + c0;
-  const float* P = Err + (int64_t)r0 * kBlock;
-  const float* Q = U + (int64_t)i1 * n + i2 + c0;
-  tile_sub<false>(C, n, P, kBlock, Q, n, min(kTileM, rows - r0), min(kTileM, n - i2 - c0), K, sm);
+  float e_out[32];
+  uint32_t cw[8];
+#pragma unroll
+  for (int s = 0; s < 32; ++s) e_out[s] = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) cw[k] = 0u;
+  float loss = 0.f;
+  const float* uq_lane = Uq + q * kUqPitch;
+
+#pragma unroll
+  for (int s = 0; s < 32; ++s) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int jj = 4 * s + k;
+    if (jj >= bsz) break;
+    constexpr int kGS = (GS == 32 || GS == 64) ? GS : 1;  // in-block group size
+    if ((GS == 32 || GS == 64) && (jj % kGS) == 0) {
+      // group [jj, jj + GS) of the block, current (repaired) values
+      float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+      for (int s2 = s; s2 < s + GS / 4; ++s2)
+        if (4 * s2 + q < bsz) {
+          mn = fminf(mn, w[s2]);
+          mx = fmaxf(mx, w[s2]);
+        }
+      fit_ruler(quad_min(mn), quad_max(mx), maxq, scale, zf);
+      if (active && q == 0) {
+        const int g = (i1 + jj) / kGS;
+        scales[(int64_t)r * G + g] = scale;
+        zeros[(int64_t)r * G + g] = (uint8_t)zf;
+      }
+    }
+    // every lane rounds its slot s; the owner's (q == jj % 4) result is used
+    const float x = w[s];
+    float qv = rintf(__fdiv_rn(x, scale)) + zf;
+    qv = fminf(fmaxf(qv, 0.f), maxq);
+    const float wh = __fmul_rn(scale, qv - zf);
+    const float e = x - wh;
+    const float ev = e * rd[jj];
+    const float err = __shfl_sync(0xffffffffu, ev, jj & 3, 4);
+    const float* urow = uq_lane + jj * kUqRow;
+#pragma unroll
+    for (int s4 = s >> 2; s4 < 8; ++s4) {
+      const float4 u = *reinterpret_cast<const float4*>(urow + 4 * s4);
+      if (4 * s4 + 0 >= s) w[4 * s4 + 0] = fmaf(-err, u.x, w[4 * s4 + 0]);
+      if (4 * s4 + 1 >= s) w[4 * s4 + 1] = fmaf(-err, u.y, w[4 * s4 + 1]);
+      if (4 * s4 + 2 >= s) w[4 * s4 + 2] = fmaf(-err, u.z, w[4 * s4 + 2]);
+      if (4 * s4 + 3 >= s) w[4 * s4 + 3] = fmaf(-err, u.w, w[4 * s4 + 3]);
+    }
+    if (q == (jj & 3)) {
+      w[s] = wh;
+      e_out[s] = ev;
+      loss = fmaf(e * e, hrd2[jj], loss);
+      cw[s >> 2] |= ((uint32_t)qv) << (8 * (s & 3));
+    }
+  }
+  }
+
+  if (active) {
+    uint8_t* crow = codes_sw + (int64_t)r * n + i1;
+    float* ehi = Err_hi + (int64_t)r * kBlock;
+    float* elo = Err_lo + (int64_t)r * kBlock;
+#pragma unroll
+    for (int s = 0; s < 32; ++s) {
+      const int c = 4 * s + q;
+      if (c < bsz) {
+        crow[c] = (uint8_t)((cw[s >> 2] >> (8 * (s & 3))) & 0xFFu);
+        wrow[c] = w[s];
+      }
+      float h, l;
+      tf32_split(e_out[s], h, l);
+      ehi[c] = h;
+      elo[c] = l;
+    }
+  }
+  if (row_loss) {
+    loss += __shfl_xor_sync(0xffffffffu, loss, 1);
+    loss += __shfl_xor_sync(0xffffffffu, loss, 2);
+    if (active && q == 0) row_loss[r] += loss;
+  }
 }
 
 // One CTA per row: codes[r][c] = codes_sw[r][pos[c]], Wq[r][c] = Wf[r][pos[c]].
@@ -301,8 +400,9 @@ cudaError_t set_smem(F* f, size_t bytes) {
 }  // namespace
 
 size_t quantize_workspace_bytes(int64_t rows, int64_t n) {
-  return align_up(sizeof(float) * rows * n, 256) + align_up(sizeof(float) * rows * kBlock, 256) +
-         align_up((size_t)rows * n, 256) + align_up(sizeof(int32_t) * n, 256);
+  return align_up(sizeof(float) * rows * n, 256) +
+         2 * align_up(sizeof(float) * rows * kBlock, 256) + align_up((size_t)rows * n, 256) +
+         align_up(sizeof(int32_t) * n, 256) + 2 * align_up(sizeof(float) * n * ut_ld(n), 256);
 }
 
 cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t n64,
@@ -335,30 +435,51 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
     note_launch();
   }
 
-  const size_t us_smem = sizeof(float) * kBlock * kBlock;
+  const size_t us_smem = kSweepSmemBytes;
   if ((e = set_smem(sweep_block_kernel<0>, us_smem)) != cudaSuccess) return e;
-  if ((e = set_smem(sweep_block_kernel<1>, us_smem)) != cudaSuccess) return e;
-  if ((e = set_smem(sweep_block_kernel<2>, us_smem)) != cudaSuccess) return e;
-  const int sweep_ctas = std::min((rows + 7) / 8, 3 * num_sms());
+  if ((e = set_smem(sweep_block_kernel<128>, us_smem)) != cudaSuccess) return e;
+  if ((e = set_smem(sweep_block_kernel<32>, us_smem)) != cudaSuccess) return e;
+  if ((e = set_smem(sweep_block_kernel<64>, us_smem)) != cudaSuccess) return e;
+  const int sweep_ctas = (rows * 4 + kSweepThreads - 1) / kSweepThreads;
+
+  // operands of the lazy update on the tensor cores
+  CUtensorMap mEh, mEl, mUh, mUl;
+  if (n > kBlock) {
+    ut_split_kernel<<<dim3((unsigned)((w.ldut + 31) / 32), (unsigned)((n + 31) / 32)), 256, 0, s>>>(
+        U, n, w.ldut, w.UT_hi, w.UT_lo);
+    note_launch();
+    if (!make_tma_2d(&mEh, w.Err_hi, false, rows, kBlock, kBlock, 32, 128) ||
+        !make_tma_2d(&mEl, w.Err_lo, false, rows, kBlock, kBlock, 32, 128) ||
+        !make_tma_2d(&mUh, w.UT_hi, false, n, n, w.ldut, 32, 128) ||
+        !make_tma_2d(&mUl, w.UT_lo, false, n, n, w.ldut, 32, 128))
+      return cudaErrorInvalidValue;
+    if ((e = cudaFuncSetAttribute(panel_gemm_kernel<SweepTrailDecoder>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kPgSmemBytes)) != cudaSuccess)
+      return e;
+  }
   for (int i1 = 0; i1 < n; i1 += kBlock) {
     const int bsz = std::min(kBlock, n - i1);
     const int i2 = i1 + bsz;
+#define GPTQ_SWEEP_LAUNCH(GSV)                                                                 \
+  sweep_block_kernel<GSV><<<sweep_ctas, kSweepThreads, us_smem, s>>>(                          \
+      w.Wf, rows, n, U, i1, bsz, maxq, group_size, G, w.Err_hi, w.Err_lo, w.codes_sw, scales,  \
+      zeros, row_loss)
     if (gmode == 0)
-      sweep_block_kernel<0><<<sweep_ctas, 256, us_smem, s>>>(
-          w.Wf, rows, n, U, i1, bsz, maxq, group_size, G, w.Err, w.codes_sw, scales, zeros,
-          row_loss);
+      GPTQ_SWEEP_LAUNCH(0);
     else if (gmode == 1)
-      sweep_block_kernel<1><<<sweep_ctas, 256, us_smem, s>>>(
-          w.Wf, rows, n, U, i1, bsz, maxq, group_size, G, w.Err, w.codes_sw, scales, zeros,
-          row_loss);
+      GPTQ_SWEEP_LAUNCH(128);
+    else if (group_size == 32)
+      GPTQ_SWEEP_LAUNCH(32);
     else
-      sweep_block_kernel<2><<<sweep_ctas, 256, us_smem, s>>>(
-          w.Wf, rows, n, U, i1, bsz, maxq, group_size, G, w.Err, w.codes_sw, scales, zeros,
-          row_loss);
+      GPTQ_SWEEP_LAUNCH(64);
+#undef GPTQ_SWEEP_LAUNCH
     note_launch();
-    if (i2 < n) {
-      dim3 grid((n - i2 + kTileM - 1) / kTileM, (rows + kTileM - 1) / kTileM);
-      sweep_trailing_kernel<<<grid, 256, 0, s>>>(w.Wf, rows, n, U, w.Err, i1, i2, bsz);
+    if (i2 < n) {  // bsz == 128 here: only the last block is short
+      const SweepTrailDecoder dec{w.Wf, rows, n, i1, i2};
+      dim3 grid((unsigned)((n - i2 + 127) / 128), (unsigned)((rows + 127) / 128));
+      panel_gemm_kernel<SweepTrailDecoder><<<grid, kPgThreads, kPgSmemBytes, s>>>(
+          mEh, mEl, mUh, mUl, dec, nullptr, 0, nullptr);
       note_launch();
     }
   }
