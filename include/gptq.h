@@ -194,6 +194,14 @@ const char* gptq_status_string(int status);
  * process so far.  The one piece of process-wide state the library keeps. */
 int64_t gptq_launch_count(void);
 
+/* Self-test of the division the sweep uses to round w / scale (a
+ * correctly rounded binary32 division by Markstein's FMA method, with the
+ * reciprocal of the divisor computed once per ruler): out[i] = a[i] / b[i]
+ * for b[i] > 0.  Device arrays of `count` floats.  The result must equal
+ * IEEE round-to-nearest division bit for bit; the tests check that. */
+gptq_status gptq_selftest_division(const float* a, const float* b, int64_t count, float* out,
+                                   void* stream);
+
 #ifdef __cplusplus
 }
 #endif

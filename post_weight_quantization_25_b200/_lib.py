@@ -25,7 +25,8 @@ GPTQ_OP_QUANTIZE = 2
 
 EXPORTS = ("gptq_workspace_size", "gptq_hessian_accumulate", "gptq_cholesky_inverse",
            "gptq_quantize_layer", "gptq_pack_int4", "gptq_pack_int3", "gptq_dequant",
-           "gptq_status_string", "gptq_launch_count", "gptq_cholesky_inverse_noalloc")
+           "gptq_status_string", "gptq_launch_count", "gptq_cholesky_inverse_noalloc",
+           "gptq_selftest_division")
 
 
 class GptqConfig(ctypes.Structure):
@@ -55,6 +56,7 @@ _SIGNATURES = {
     "gptq_status_string": (ctypes.c_char_p, [_int]),
     "gptq_launch_count": (_i64, []),
     "gptq_cholesky_inverse_noalloc": (_int, [_vp, _i64, _f, _int, _vp, _vp, _vp, _vp, _vp]),
+    "gptq_selftest_division": (_int, [_vp, _vp, _i64, _vp, _vp]),
 }
 
 _LIB = None

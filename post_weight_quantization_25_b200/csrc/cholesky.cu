@@ -224,36 +224,58 @@ __global__ void __launch_bounds__(256) chol_diag_kernel(float* __restrict__ A, i
   __syncthreads();
 
   for (int c0 = 0; c0 < bs; c0 += 32) {
-    // (1) 32 x 32 diagonal sub-block, one warp, registers
+    // (1) 32 x 32 diagonal sub-block, one warp, registers.  Unscaled
+    // (LDL^T-like) right-looking form: step j publishes column j as it
+    // stands (colj[k] = a_kj) and every lane i > j applies
+    // a_ik -= (a_ij / d_j) a_kj; the column entries are read from shared
+    // memory with independent loads issued ahead of the FMAs, so a step is
+    // one short dependency chain.  Square roots come at the end:
+    // L_ik = a_ik / sqrt(d_k), L_kk = sqrt(d_k).
     if (warp == 0) {
+      float* colj = rdiag + kPanel;  // 32 floats of scratch after rdiag
       float a[32];
 #pragma unroll
       for (int k = 0; k < 32; ++k) a[k] = (k <= lane) ? chol_elem(S, c0 + lane, c0 + k) : 0.f;
       bool bad = false;
+      int first_bad = 0;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        const float d = __shfl_sync(0xffffffffu, a[j], j);
-        if (!bad && (!(d > 0.f) || !isfinite(d))) {  // uniform across the warp
-          bad = true;                                // (results below are discarded)
-          if (lane == 0) fail = c0 + j + 1;
-        }
-        const float sd = sqrtf(d);
-        const float l = (lane == j) ? sd : a[j] / sd;  // L[c0+lane][c0+j]
-        a[j] = (lane >= j) ? l : 0.f;
+        colj[lane] = (lane >= j) ? a[j] : 0.f;
+        __syncwarp();
+        const float d = colj[j];
+        // failure bookkeeping by selects (no branch inside the unrolled loop);
+        // once bad, the results are discarded
+        const bool badj = !(d > 0.f) || !isfinite(d);
+        first_bad = (!bad && badj) ? (c0 + j + 1) : first_bad;
+        bad = bad || badj;
+        float ck[32];
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          if (k > j) {
-            const float lk = __shfl_sync(0xffffffffu, l, k);  // L[c0+k][c0+j]
-            if (lane >= k) a[k] = fmaf(-l, lk, a[k]);
-          }
-        }
-      }
-      if (!bad) {
+        for (int k = 0; k < 32; ++k) ck[k] = (k > j) ? colj[k] : 0.f;
+        // 1/d: hardware estimate plus one Newton step (fp32 accurate to ~1
+        // ulp, which is all a multiplier of the factorisation needs)
+        const float r0 = ptx::rcp_approx(d);
+        const float rd = fmaf(fmaf(-d, r0, 1.f), r0, r0);
+        const float lij = (lane > j) ? a[j] * rd : 0.f;
 #pragma unroll
         for (int k = 0; k < 32; ++k)
-          if (k <= lane) S[(c0 + lane) * kPadLD + c0 + k] = a[k];
+          if (k > j) a[k] = fmaf(-lij, ck[k], a[k]);
         __syncwarp();
-        rdiag[c0 + lane] = 1.f / chol_elem(S, c0 + lane, c0 + lane);
+      }
+      if (bad && lane == 0) fail = first_bad;
+      if (!bad) {
+        // pivots d_k = a_kk; scale row `lane` by 1/sqrt(d_k)
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          if (k == lane) colj[lane] = a[k];
+        __syncwarp();
+        const float rs_own = 1.f / sqrtf(colj[lane]);
+        rdiag[c0 + lane] = rs_own;  // 1 / L_kk for the solve below
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          if (k < lane) S[(c0 + lane) * kPadLD + c0 + k] = a[k] * rdiag[c0 + k];
+          if (k == lane) S[(c0 + lane) * kPadLD + c0 + k] = sqrtf(a[k]);
+        }
       }
     }
     __syncthreads();
@@ -383,8 +405,9 @@ __global__ void __launch_bounds__(kSolveThreads) panel_solve_kernel(
     for (int s = 0; s < 32; ++s) {
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
+        // no early exit for a short panel: entries past bs are 0 and the
+        // padded factor is the identity there, so those steps change nothing
         const int j = 4 * s + k;
-        if (j >= bs) break;
         const float yv = x[s] * rdiag[j];
         const float y = __shfl_sync(0xffffffffu, yv, k, 4);
         const float* lcol = lq_lane + j * kLqRow;
@@ -396,7 +419,7 @@ __global__ void __launch_bounds__(kSolveThreads) panel_solve_kernel(
           if (4 * s4 + 2 >= s) x[4 * s4 + 2] = fmaf(-l4.z, y, x[4 * s4 + 2]);
           if (4 * s4 + 3 >= s) x[4 * s4 + 3] = fmaf(-l4.w, y, x[4 * s4 + 3]);
         }
-        if (q == k) x[s] = y;
+        x[s] = (q == k) ? y : x[s];
       }
     }
     if (active) {

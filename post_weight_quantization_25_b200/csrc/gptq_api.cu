@@ -91,6 +91,15 @@ extern "C" {
 
 int64_t gptq_launch_count(void) { return gptq::g_launches.load(std::memory_order_relaxed); }
 
+gptq_status gptq_selftest_division(const float* a, const float* b, int64_t count, float* out,
+                                   void* stream) {
+  if (count < 0) return GPTQ_ERR_INVALID_ARG;
+  if (count == 0) return GPTQ_OK;
+  if (!a || !b || !out) return GPTQ_ERR_INVALID_ARG;
+  return cuda_status(
+      gptq::launch_selftest_division(a, b, count, out, static_cast<cudaStream_t>(stream)));
+}
+
 const char* gptq_status_string(int status) {
   switch (status) {
     case GPTQ_OK: return "ok";

@@ -46,6 +46,9 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows, int64_t n
                                   int32_t* g_idx, float* Wq, float* row_loss, void* ws,
                                   cudaStream_t s);
 size_t quantize_workspace_bytes(int64_t rows, int64_t n);
+// out[i] = a[i] / b[i] by the sweep's division routine (fdiv.cuh)
+cudaError_t launch_selftest_division(const float* a, const float* b, int64_t count, float* out,
+                                     cudaStream_t s);
 
 // ---- storage (pack.cu)
 cudaError_t launch_pack_int4(const uint8_t* codes, int64_t rows, int64_t n, uint32_t* out,

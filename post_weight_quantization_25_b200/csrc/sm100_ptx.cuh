@@ -131,6 +131,13 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64
       : "memory");
 }
 
+// Hardware reciprocal estimate (PTX rcp.approx.f32, no flush to zero).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 // x rounded to TF32 (nearest, ties away), returned as an fp32 whose low 13
 // mantissa bits are zero; x - tf32_hi(x) is then exact in fp32.
 __device__ __forceinline__ float tf32_hi(float x) {

@@ -30,6 +30,7 @@
 
 #include "gptq_internal.cuh"
 #include "panel_gemm.cuh"
+#include "fdiv.cuh"
 #include "stage.cuh"
 
 namespace gptq {
@@ -96,22 +97,25 @@ __global__ void __launch_bounds__(256) ut_split_kernel(const float* __restrict__
 // The lazy update  Wf[:, i2:] -= Err U[i1:i1+128, i2:]  as tiles for the
 // tensor-core panel GEMM: P = Err (rows x 128), Q = U^T rows i2.. (columns
 // i1..i1+128), C = Wf.
-struct SweepTrailDecoder {
+// Item i = rows [128 i, 128 i + 128) of Wf, with its P block (the err terms)
+// kept resident while the tiles of columns i2, i2 + 128, ... stream by.
+struct SweepTrailItems {
   float* Wf;
   int rows, n, i1, i2;
-  __device__ PgTile tile(int bx, int by) const {
-    PgTile t;
-    const int c0 = bx * 128, r0 = by * 128;
-    t.C = Wf + (int64_t)r0 * n + i2 + c0;
-    t.ldc = n;
-    t.prow = r0;
-    t.pkx = 0;
-    t.qrow = i2 + c0;
-    t.qkx = i1;
-    t.mext = min(128, rows - r0);
-    t.cext = min(128, n - i2 - c0);
-    t.valid = (t.mext > 0 && t.cext > 0) ? 1 : 0;
-    return t;
+  __host__ __device__ int num_items() const { return (rows + 127) / 128; }
+  __host__ __device__ int item_nq(int) const { return (n - i2 + 127) / 128; }
+  __device__ PgItem item(int i) const {
+    PgItem I;
+    I.C0 = Wf + (int64_t)i * 128 * n + i2;
+    I.ldc = n;
+    I.prow = 128 * i;
+    I.pkx = 0;
+    I.qrow0 = i2;
+    I.qkx = i1;
+    I.nq = item_nq(i);
+    I.mext = min(128, rows - 128 * i);
+    I.cext_last = n - i2 - 128 * (I.nq - 1);
+    return I;
   }
 };
 
@@ -282,6 +286,9 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
     }
   }
 
+  // w / scale, correctly rounded, with the reciprocal of the scale computed
+  // once per ruler (Markstein's method, fdiv.cuh)
+  MDiv md = md_prepare(scale);
   float e_out[32];
   uint32_t cw[8];
 #pragma unroll
@@ -295,8 +302,11 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
   for (int s = 0; s < 32; ++s) {
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
+    // No early exit for a short last block: its columns past bsz hold 0 and
+    // its U rows past bsz are 0 (with 1/U_jj = 1), so they round to the zero
+    // point with no error and change nothing; keeping the 128 steps free of
+    // branches lets the compiler overlap consecutive steps.
     const int jj = 4 * s + k;
-    if (jj >= bsz) break;
     constexpr int kGS = (GS == 32 || GS == 64) ? GS : 1;  // in-block group size
     if ((GS == 32 || GS == 64) && (jj % kGS) == 0) {
       // group [jj, jj + GS) of the block, current (repaired) values
@@ -308,7 +318,8 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
           mx = fmaxf(mx, w[s2]);
         }
       fit_ruler(quad_min(mn), quad_max(mx), maxq, scale, zf);
-      if (active && q == 0) {
+      md = md_prepare(scale);
+      if (active && q == 0 && jj < bsz) {  // groups past the last column do not exist
         const int g = (i1 + jj) / kGS;
         scales[(int64_t)r * G + g] = scale;
         zeros[(int64_t)r * G + g] = (uint8_t)zf;
@@ -316,7 +327,7 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
     }
     // every lane rounds its slot s; the owner's (q == jj % 4) result is used
     const float x = w[s];
-    float qv = rintf(__fdiv_rn(x, scale)) + zf;
+    float qv = rintf(md_div(x, md)) + zf;
     qv = fminf(fmaxf(qv, 0.f), maxq);
     const float wh = __fmul_rn(scale, qv - zf);
     const float e = x - wh;
@@ -331,12 +342,11 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
       if (4 * s4 + 2 >= s) w[4 * s4 + 2] = fmaf(-err, u.z, w[4 * s4 + 2]);
       if (4 * s4 + 3 >= s) w[4 * s4 + 3] = fmaf(-err, u.w, w[4 * s4 + 3]);
     }
-    if (q == (jj & 3)) {
-      w[s] = wh;
-      e_out[s] = ev;
-      loss = fmaf(e * e, hrd2[jj], loss);
-      cw[s >> 2] |= ((uint32_t)qv) << (8 * (s & 3));
-    }
+    const bool own = (q == (jj & 3));
+    w[s] = own ? wh : w[s];
+    e_out[s] = own ? ev : e_out[s];
+    loss = own ? fmaf(e * e, hrd2[jj], loss) : loss;
+    cw[s >> 2] |= own ? (((uint32_t)qv) << (8 * (s & 3))) : 0u;
   }
   }
 
@@ -399,6 +409,22 @@ cudaError_t set_smem(F* f, size_t bytes) {
 
 }  // namespace
 
+namespace {
+__global__ void selftest_division_kernel(const float* __restrict__ a, const float* __restrict__ b,
+                                         int64_t count, float* __restrict__ out) {
+  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i < count) out[i] = md_div(a[i], md_prepare(b[i]));
+}
+}  // namespace
+
+cudaError_t launch_selftest_division(const float* a, const float* b, int64_t count, float* out,
+                                     cudaStream_t s) {
+  if (count <= 0) return cudaSuccess;
+  selftest_division_kernel<<<(unsigned)((count + 255) / 256), 256, 0, s>>>(a, b, count, out);
+  note_launch();
+  return cudaGetLastError();
+}
+
 size_t quantize_workspace_bytes(int64_t rows, int64_t n) {
   return align_up(sizeof(float) * rows * n, 256) +
          2 * align_up(sizeof(float) * rows * kBlock, 256) + align_up((size_t)rows * n, 256) +
@@ -441,6 +467,7 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
   if ((e = set_smem(sweep_block_kernel<32>, us_smem)) != cudaSuccess) return e;
   if ((e = set_smem(sweep_block_kernel<64>, us_smem)) != cudaSuccess) return e;
   const int sweep_ctas = (rows * 4 + kSweepThreads - 1) / kSweepThreads;
+  const int sms = num_sms();
 
   // operands of the lazy update on the tensor cores
   CUtensorMap mEh, mEl, mUh, mUl;
@@ -453,9 +480,9 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
         !make_tma_2d(&mUh, w.UT_hi, false, n, n, w.ldut, 32, 128) ||
         !make_tma_2d(&mUl, w.UT_lo, false, n, n, w.ldut, 32, 128))
       return cudaErrorInvalidValue;
-    if ((e = cudaFuncSetAttribute(panel_gemm_kernel<SweepTrailDecoder>,
+    if ((e = cudaFuncSetAttribute(panel_gemm2_kernel<SweepTrailItems>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)kPgSmemBytes)) != cudaSuccess)
+                                  (int)kPg2SmemBytes)) != cudaSuccess)
       return e;
   }
   for (int i1 = 0; i1 < n; i1 += kBlock) {
@@ -476,10 +503,11 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
 #undef GPTQ_SWEEP_LAUNCH
     note_launch();
     if (i2 < n) {  // bsz == 128 here: only the last block is short
-      const SweepTrailDecoder dec{w.Wf, rows, n, i1, i2};
-      dim3 grid((unsigned)((n - i2 + 127) / 128), (unsigned)((rows + 127) / 128));
-      panel_gemm_kernel<SweepTrailDecoder><<<grid, kPgThreads, kPgSmemBytes, s>>>(
-          mEh, mEl, mUh, mUl, dec, nullptr, 0, nullptr);
+      const SweepTrailItems dec{w.Wf, rows, n, i1, i2};
+      int chunk = 1, units = 0;
+      pg2_plan(dec, sms, chunk, units);
+      panel_gemm2_kernel<SweepTrailItems><<<std::min(units, sms), kPg2Threads, kPg2SmemBytes, s>>>(
+          mEh, mEl, mUh, mUl, dec, chunk, units, nullptr, 0, nullptr);
       note_launch();
     }
   }
