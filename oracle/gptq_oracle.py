@@ -149,6 +149,44 @@ def is_near_tie_order(d: np.ndarray, order, rtol: float) -> bool:
     return bool(np.all(a >= b - rtol * np.maximum(np.abs(a), np.abs(b))))
 
 
+def prepare_from_diagonal(d: np.ndarray, percdamp: float = 0.01, actorder: bool = False,
+                          forced_perm=None, perm_rtol: float = 1e-5):
+    """The part of the preparation that diag(H) alone fixes.
+
+    Dead inputs are the zero diagonal entries (their diagonal becomes 1);
+    with act-order the sweep order is a stable sort by descending diagonal;
+    the damping is ``lam = percdamp * mean`` of the (fixed, reordered)
+    diagonal.  Returns dict ``dead``, ``perm``, ``lam`` and ``d`` (the fixed
+    diagonal, original order).  ``forced_perm`` as in ``prepare``.
+    """
+    d = np.array(d, dtype=np.float64, copy=True)
+    n = d.shape[0]
+    dead = d == 0.0
+    d[dead] = 1.0
+    if actorder:
+        perm = np.argsort(-d, kind="stable")
+        if forced_perm is not None:
+            if not is_near_tie_order(d, forced_perm, perm_rtol):
+                raise ValueError("forced act-order is not a near-tie reordering of diag(H)")
+            perm = np.asarray(forced_perm, dtype=np.int64)
+    else:
+        perm = np.arange(n)
+    lam = percdamp * float(np.mean(d[perm]))
+    return {"dead": dead, "perm": perm, "lam": lam, "d": d}
+
+
+def damped_block(H: np.ndarray, prep: dict, k0: int, k1: int) -> np.ndarray:
+    """Rows and columns [k0, k1) (sweep order) of the prepared matrix
+    H' = H[perm][:, perm] + lam I, dead diagonal entries set to 1 first."""
+    idx = np.asarray(prep["perm"])[k0:k1]
+    B = np.array(H[np.ix_(idx, idx)], dtype=np.float64)
+    m = k1 - k0
+    dd = np.asarray(prep["dead"])[idx]
+    B[np.arange(m)[dd], np.arange(m)[dd]] = 1.0
+    B[np.arange(m), np.arange(m)] += prep["lam"]
+    return B
+
+
 def prepare(H: np.ndarray, W: np.ndarray, percdamp: float = 0.01, actorder: bool = False,
             forced_perm=None, perm_rtol: float = 1e-5):
     """Dead inputs -> act-order -> damping.
@@ -163,25 +201,15 @@ def prepare(H: np.ndarray, W: np.ndarray, percdamp: float = 0.01, actorder: bool
     summed in different precisions may order such near-equal columns either
     way); otherwise ValueError.
     """
-    H = np.array(H, dtype=np.float64, copy=True)
+    H = np.asarray(H, dtype=np.float64)
     W0 = np.array(W, dtype=np.float64, copy=True)
     n = H.shape[0]
-    d = np.diag(H).copy()
-    dead = d == 0.0
-    H[dead, dead] = 1.0
-    W0[:, dead] = 0.0
-    if actorder:
-        perm = np.argsort(-np.diag(H), kind="stable")
-        if forced_perm is not None:
-            if not is_near_tie_order(np.diag(H), forced_perm, perm_rtol):
-                raise ValueError("forced act-order is not a near-tie reordering of diag(H)")
-            perm = np.asarray(forced_perm, dtype=np.int64)
-    else:
-        perm = np.arange(n)
-    Hp = H[np.ix_(perm, perm)]
-    lam = percdamp * float(np.mean(np.diag(Hp)))
-    Hp[np.arange(n), np.arange(n)] += lam
-    return {"dead": dead, "perm": perm, "Hp": Hp, "W0": W0, "Wp": W0[:, perm], "lam": lam}
+    prep = prepare_from_diagonal(np.diag(H), percdamp, actorder, forced_perm, perm_rtol)
+    W0[:, prep["dead"]] = 0.0
+    Hp = damped_block(H, prep, 0, n)
+    perm = prep["perm"]
+    return {"dead": prep["dead"], "perm": perm, "Hp": Hp, "W0": W0, "Wp": W0[:, perm],
+            "lam": prep["lam"]}
 
 
 def upper_cholesky_of_inverse(Hp: np.ndarray) -> np.ndarray:
@@ -206,8 +234,14 @@ def _near_half(t, tau: float) -> np.ndarray:
     return np.abs((t - np.floor(t)) - 0.5) < tau
 
 
+def _half_distance(t) -> float:
+    t = float(t)
+    return abs((t - np.floor(t)) - 0.5)
+
+
 def sweep(Wp: np.ndarray, U: np.ndarray, bits: int, group_size: int = -1,
-          forced_codes=None, forced_zeros=None, tau: float = 1e-3, trace=None):
+          forced_codes=None, forced_zeros=None, tau: float = 1e-3, trace=None,
+          adoptions=None):
     """Unblocked GPTQ sweep over the columns of Wp (already in sweep order).
 
     For each column j, left to right, for every row at once:
@@ -223,7 +257,9 @@ def sweep(Wp: np.ndarray, U: np.ndarray, bits: int, group_size: int = -1,
     (a rounding tie that two correct implementations may break either way),
     the forced value is adopted; any other difference is counted as a
     mismatch and this run's own value is kept.  ``trace(j, W)`` is called
-    after column j's repair with the working matrix.
+    after column j's repair with the working matrix.  ``adoptions``, if a
+    list, receives ``(row, column, "code" | "zero", distance of the
+    pre-rounding value from the half-integer, in ticks)`` for each adoption.
 
     Returns a dict: codes (int64 rows x n), scales (float32 rows x G), zeros
     (int64 rows x G), Wq (fp64 rows x n), err (fp64 rows x n, the e/U_jj
@@ -251,8 +287,12 @@ def sweep(Wp: np.ndarray, U: np.ndarray, bits: int, group_size: int = -1,
             if forced_zeros is not None:
                 fz = np.asarray(forced_zeros)[:, j // g].astype(np.int64)
                 diff = fz != zero
-                tie = _near_half(zero_prevalue(blk.min(axis=1), bits, scale), tau)
+                zp = zero_prevalue(blk.min(axis=1), bits, scale)
+                tie = _near_half(zp, tau)
                 adopted += int(np.count_nonzero(diff & tie))
+                if adoptions is not None:
+                    for r in np.nonzero(diff & tie)[0]:
+                        adoptions.append((int(r), j, "zero", _half_distance(zp[r])))
                 mismatched += int(np.count_nonzero(diff & ~tie))
                 zero = np.where(diff & tie, fz, zero)
             scales[:, j // g] = scale
@@ -265,6 +305,9 @@ def sweep(Wp: np.ndarray, U: np.ndarray, bits: int, group_size: int = -1,
             t = w / scale.astype(np.float64)
             tie = _near_half(t, tau)
             adopted += int(np.count_nonzero(diff & tie))
+            if adoptions is not None:
+                for r in np.nonzero(diff & tie)[0]:
+                    adoptions.append((int(r), j, "code", _half_distance(t[r])))
             mismatched += int(np.count_nonzero(diff & ~tie))
             q = np.where(diff & tie, fq, q)
         codes[:, j] = q

@@ -16,9 +16,17 @@
 //  * Per CTA: warp 0 issues TMA loads (128-byte swizzle, 4-stage ring of
 //    128x64 + 256x64 bf16 tiles), warp 1 issues tcgen05.mma kind::f16
 //    (M=128, N=256, K=16; fp32 accumulators in TMEM, two 256-column buffers
-//    so the epilogue of one unit overlaps the MMAs of the next), warps 2-5
-//    drain TMEM with tcgen05.ld and add alpha * partial into H with vector
-//    atomics (the split-K reduction), masking to the upper triangle.
+//    so the epilogue of one piece overlaps the MMAs of the next), warps 2-9
+//    drain TMEM with tcgen05.ld.
+//  * Accuracy: the fp32 sum the tensor cores keep in TMEM loses more than
+//    IEEE round-to-nearest would over a long chain of MMAs; measured on this
+//    kernel, the relative error of H grew in proportion to the number of
+//    MMAs accumulated into one TMEM tile (about 1.2e-7 per K = 16 MMA).  So
+//    a unit's token range is cut into pieces of kSubKb k-blocks (1024
+//    tokens, 64 MMAs); each piece starts a fresh TMEM sum, and the epilogue
+//    adds the pieces into an fp32 register copy of the tile with ordinary
+//    IEEE adds.  At the end of the unit it adds alpha * tile into H with
+//    vector atomics (the split-K reduction), masked to the upper triangle.
 //  * No multicast loads.  Every wait is bounded: on timeout the CTA stops,
 //    writes GPTQ_ERR_TIMEOUT to `info`, waits for its own copies and MMAs,
 //    frees TMEM and exits.
@@ -39,7 +47,8 @@ constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;          // TMA warp, MMA warp, 8 epilogue warps
+constexpr int kSubKb = 16;                // k-blocks per fresh TMEM sum (1024 tokens)
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + 256;
 constexpr uint64_t WAIT_LIMIT_NS = (uint64_t)kGridWaitLimitNs;
@@ -101,7 +110,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(&tfull[a], 1);
-      ptx::mbar_init(&tempty[a], 128);
+      ptx::mbar_init(&tempty[a], 256);
     }
     ptx::mbar_init(drain, 1);
     *abort_flag = 0;
@@ -167,34 +176,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int u = blockIdx.x; u < args.units && ok; u += gridDim.x) {
         const int kb0 = (u / args.ntiles) * args.kb_per_unit;
         const int kb1 = min(kb0 + args.kb_per_unit, args.nkb);
-        if (!ptx::mbar_wait_bounded(&tempty[acc], aphase ^ 1, abort_flag, WAIT_LIMIT_NS)) {
-          ok = false;
-          break;
-        }
-        ptx::tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!ptx::mbar_wait_bounded(&full[stage], phase, abort_flag, WAIT_LIMIT_NS)) {
+        for (int p0 = kb0; p0 < kb1 && ok; p0 += kSubKb) {
+          const int p1 = min(p0 + kSubKb, kb1);
+          if (!ptx::mbar_wait_bounded(&tempty[acc], aphase ^ 1, abort_flag, WAIT_LIMIT_NS)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
-          const uint64_t adesc = ptx::smem_desc_sw128(ptx::smem_u32(sA + stage * A_BYTES));
-          const uint64_t bdesc = ptx::smem_desc_sw128(ptx::smem_u32(sB + stage * B_BYTES));
+          const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+          for (int kb = p0; kb < p1; ++kb) {
+            if (!ptx::mbar_wait_bounded(&full[stage], phase, abort_flag, WAIT_LIMIT_NS)) {
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
+            const uint64_t adesc = ptx::smem_desc_sw128(ptx::smem_u32(sA + stage * A_BYTES));
+            const uint64_t bdesc = ptx::smem_desc_sw128(ptx::smem_u32(sB + stage * B_BYTES));
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            ptx::mma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc,
-                          (kb > kb0 || k > 0) ? 1u : 0u);
-          ptx::mma_commit(&empty[stage]);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1;
+            for (int k = 0; k < BK / 16; ++k)
+              ptx::mma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc,
+                            (kb > p0 || k > 0) ? 1u : 0u);
+            ptx::mma_commit(&empty[stage]);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1;
+            }
           }
+          if (!ok) break;
+          ptx::mma_commit(&tfull[acc]);
+          acc ^= 1;
+          if (acc == 0) aphase ^= 1;
         }
-        if (!ok) break;
-        ptx::mma_commit(&tfull[acc]);
-        acc ^= 1;
-        if (acc == 0) aphase ^= 1;
       }
       if (!ok || *abort_flag) {
         raise_abort(abort_flag, args.info);
@@ -204,53 +216,73 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else {
-    // -------------------------------------------------- epilogue (warps 2..5)
-    const int q = warp & 3;  // this warp may read TMEM lanes [32q, 32q + 32)
+    // -------------------------------------------------- epilogue (warps 2..9)
+    // warp w reads TMEM lanes [32 (w % 4), +32) (rows of the tile) and
+    // columns [128 half, +128) of the accumulator
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     int acc = 0;
     uint32_t aphase = 0;
     const int n = args.n;
-    for (int u = blockIdx.x; u < args.units; u += gridDim.x) {
+    bool stop = false;
+    for (int u = blockIdx.x; u < args.units && !stop; u += gridDim.x) {
       int I, J;
       decode_tile(u % args.ntiles, args.nI, I, J);
-      if (!ptx::mbar_wait_bounded(&tfull[acc], aphase, abort_flag, WAIT_LIMIT_NS)) {
-        raise_abort(abort_flag, args.info);
-        break;
-      }
-      ptx::tc_fence_after();
+      const int kb0 = (u / args.ntiles) * args.kb_per_unit;
+      const int kb1 = min(kb0 + args.kb_per_unit, args.nkb);
       const int row_lo = I * BM + q * 32;
       const int row = row_lo + lane;
-      float* hrow = args.H + (int64_t)row * n;
-#pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
-        const int col0 = J * BN + ch * 32;
-        if (col0 >= n) break;
-        if (col0 + 31 < row_lo) continue;  // whole 32x32 piece below the diagonal
-        uint32_t v[32];
-        ptx::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + ch * 32), v);
-        ptx::tmem_ld_wait();
-        if (row < n) {
+      const int cbase = J * BN + half * 128;
+      float tile[128];
 #pragma unroll
-          for (int j4 = 0; j4 < 8; ++j4) {
-            const int c = col0 + 4 * j4;
-            const float f0 = args.alpha * __uint_as_float(v[4 * j4 + 0]);
-            const float f1 = args.alpha * __uint_as_float(v[4 * j4 + 1]);
-            const float f2 = args.alpha * __uint_as_float(v[4 * j4 + 2]);
-            const float f3 = args.alpha * __uint_as_float(v[4 * j4 + 3]);
-            if (args.vec4 && c >= row && c + 3 < n) {
-              atomicAdd(reinterpret_cast<float4*>(hrow + c), make_float4(f0, f1, f2, f3));
-            } else {
-              if (c + 0 >= row && c + 0 < n) atomicAdd(hrow + c + 0, f0);
-              if (c + 1 >= row && c + 1 < n) atomicAdd(hrow + c + 1, f1);
-              if (c + 2 >= row && c + 2 < n) atomicAdd(hrow + c + 2, f2);
-              if (c + 3 >= row && c + 3 < n) atomicAdd(hrow + c + 3, f3);
-            }
+      for (int j = 0; j < 128; ++j) tile[j] = 0.f;
+      for (int p0 = kb0; p0 < kb1; p0 += kSubKb) {
+        if (!ptx::mbar_wait_bounded(&tfull[acc], aphase, abort_flag, WAIT_LIMIT_NS)) {
+          raise_abort(abort_flag, args.info);
+          stop = true;
+          break;
+        }
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const int col0 = cbase + ch * 32;
+          // warp-uniform: pieces past n or wholly below the diagonal are not needed
+          if (col0 < n && col0 + 31 >= row_lo) {
+            uint32_t v[32];
+            ptx::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) +
+                                        (uint32_t)(acc * BN + half * 128 + ch * 32),
+                                    v);
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) tile[ch * 32 + j] += __uint_as_float(v[j]);
+          }
+        }
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&tempty[acc]);
+        acc ^= 1;
+        if (acc == 0) aphase ^= 1;
+      }
+      if (stop) break;
+      if (row < n) {
+        float* hrow = args.H + (int64_t)row * n;
+#pragma unroll
+        for (int j4 = 0; j4 < 32; ++j4) {
+          const int c = cbase + 4 * j4;
+          if (c + 3 < row || c >= n) continue;
+          const float f0 = args.alpha * tile[4 * j4 + 0];
+          const float f1 = args.alpha * tile[4 * j4 + 1];
+          const float f2 = args.alpha * tile[4 * j4 + 2];
+          const float f3 = args.alpha * tile[4 * j4 + 3];
+          if (args.vec4 && c >= row && c + 3 < n) {
+            atomicAdd(reinterpret_cast<float4*>(hrow + c), make_float4(f0, f1, f2, f3));
+          } else {
+            if (c + 0 >= row && c + 0 < n) atomicAdd(hrow + c + 0, f0);
+            if (c + 1 >= row && c + 1 < n) atomicAdd(hrow + c + 1, f1);
+            if (c + 2 >= row && c + 2 < n) atomicAdd(hrow + c + 2, f2);
+            if (c + 3 >= row && c + 3 < n) atomicAdd(hrow + c + 3, f3);
           }
         }
       }
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&tempty[acc]);
-      acc ^= 1;
-      if (acc == 0) aphase ^= 1;
     }
   }
 

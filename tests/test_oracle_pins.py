@@ -308,6 +308,35 @@ def test_actorder_is_stable_descending():
     assert list(p) == [3, 1, 4, 0, 2]
 
 
+def test_prepared_blocks_come_from_the_diagonal_alone():
+    """dead / act-order / damping read only diag(H): any principal block of
+    the prepared matrix can be built without forming the whole of it (the
+    full-size checks rely on this), and it is the textbook construction
+    H[perm][:, perm] + lam I with dead diagonal entries set to 1."""
+    H, _ = _rand_spd(40, seed=77)
+    for c in (3, 17):
+        H[c, :] = 0.0
+        H[:, c] = 0.0
+    W = np.ones((2, 40))
+    for act in (False, True):
+        full = O.prepare(H, W, 0.01, act)
+        diag_only = O.prepare_from_diagonal(np.diag(H), 0.01, act)
+        assert np.array_equal(full["perm"], diag_only["perm"])
+        assert np.array_equal(full["dead"], diag_only["dead"])
+        d = np.diag(H).copy()
+        d[[3, 17]] = 1.0
+        assert diag_only["lam"] == pytest.approx(0.01 * d.mean(), rel=1e-14)
+        Hd = H.copy()
+        Hd[[3, 17], [3, 17]] = 1.0
+        p = diag_only["perm"]
+        textbook = Hd[p][:, p] + diag_only["lam"] * np.eye(40)
+        assert np.array_equal(full["Hp"], textbook)
+        for k0, k1 in ((0, 40), (10, 25), (33, 40)):
+            assert np.array_equal(O.damped_block(H, diag_only, k0, k1), textbook[k0:k1, k0:k1])
+    # dead channels go last under act-order (their diagonal, 1, is the smallest here)
+    assert set(O.prepare_from_diagonal(np.diag(H), 0.01, True)["perm"][-2:]) == {3, 17}
+
+
 def test_gptq_beats_rtn_on_correlated_inputs():
     W, X = _layer(16, 64, 256, seed=41, corr=0.8)
     H = O.hessian(X)
