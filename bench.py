@@ -81,17 +81,62 @@ def describe(wl) -> str:
 
 
 # ----------------------------------------------------------------- clocks
+REASON_NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+
 class ClockSampler:
+    """SM clock and clock-event reasons sampled DURING the timed region.
+
+    Reads NVML from a background thread every ``period_s`` (read-only
+    queries); if NVML is unavailable, falls back to ``nvidia-smi -lms 200``.
+    Nothing here changes a GPU setting."""
+
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, uuid: str | None = None, period_s: float = 0.01):
         self.gpu = gpu_index
+        self.uuid = uuid
+        self.period = period_s
         self.proc = None
         self.path = None
+        self.thread = None
+        self.samples = []          # (sm_mhz, sm_max_mhz, set of reason names)
+        self._stop = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        if self.uuid:
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _poll(self, nv, h):
+        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+        smax = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        while not self._stop.is_set():
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((sm, smax, {k for k, v in bits.items() if r & v}))
+            except Exception:
+                break
+            self._stop.wait(self.period)
 
     def __enter__(self):
+        import threading
+        try:
+            nv, h = self._nvml_handle()
+            self._stop = threading.Event()
+            self.thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.thread = None
         fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
         os.close(fd)
         try:
@@ -104,6 +149,9 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self._stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -111,29 +159,52 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
+    def _read_smi(self):
         if not self.path or not os.path.exists(self.path):
-            return None
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            return
         with open(self.path) as f:
             for line in f:
                 parts = [x.strip() for x in line.split(",")]
                 if len(parts) < 9:
                     continue
                 try:
-                    sm.append(float(parts[1]))
-                    smax.append(float(parts[2]))
+                    sm, smax = float(parts[1]), float(parts[2])
                 except ValueError:
                     continue
-                for nm, v in zip(names, parts[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(nm)
+                reasons = {nm for nm, v in zip(REASON_NAMES, parts[5:9]) if v.lower() == "active"}
+                self.samples.append((sm, smax, reasons))
         os.unlink(self.path)
-        if not sm:
+
+    def summary(self):
+        self._read_smi()
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        reasons = set()
+        for _, _, r in self.samples:
+            reasons |= r
+        return {"sm_mhz": statistics.median(x[0] for x in self.samples),
+                "sm_max_mhz": max(x[1] for x in self.samples), "reasons": sorted(reasons),
+                "samples": len(self.samples),
+                "source": "nvml" if self.thread is not None else "nvidia-smi"}
+
+
+# ----------------------------------------------------------------- ranks
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest value of ``x`` over all ranks (a device time: the job ends
+    when its slowest rank does)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, units_per_rank: int, steps: int, ms: float) -> float:
+    """Whole-job units per second: every rank processes ``units_per_rank``
+    per step (weak scaling), timed as the slowest rank's ``ms``."""
+    return world * units_per_rank * steps / (ms / 1e3)
 
 
 # ----------------------------------------------------------------- oracle sample
@@ -197,53 +268,13 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     W, X = workloads.make_inputs(wl, device=dev)
     rows, n, N = wl.rows, wl.n, wl.ntok
-    cfg = G.make_config(wl.bits, wl.group_size, wl.percdamp, wl.actorder)
-    G_ = 1 if wl.group_size <= 0 else (n + wl.group_size - 1) // wl.group_size
-
-    H = torch.empty(n, n, dtype=torch.float32, device=dev)
-    U = torch.empty(n, n, dtype=torch.float32, device=dev)
-    perm = torch.empty(n, dtype=torch.int32, device=dev)
-    dead = torch.empty(n, dtype=torch.uint8, device=dev)
-    info = torch.zeros(1, dtype=torch.int32, device=dev)
-    info_h = torch.zeros(1, dtype=torch.int32, device=dev)
-    codes = torch.empty(rows, n, dtype=torch.uint8, device=dev)
-    scales = torch.empty(rows, G_, dtype=torch.float32, device=dev)
-    zeros = torch.empty(rows, G_, dtype=torch.uint8, device=dev)
-    g_idx = torch.empty(n, dtype=torch.int32, device=dev)
-    pack = G.gptq_pack_int4 if wl.bits == 4 else G.gptq_pack_int3
-    packed = torch.empty(rows, n * wl.bits // 32, dtype=torch.int32, device=dev)
-    deq = torch.empty(rows, n, dtype=torch.bfloat16, device=dev)
-    from post_weight_quantization_25_b200._lib import GPTQ_OP_CHOLESKY, GPTQ_OP_HESSIAN, GPTQ_OP_QUANTIZE
-    ws_h = torch.empty(G.gptq_workspace_size(GPTQ_OP_HESSIAN, 0, n, N, X.dtype) + 512,
-                       dtype=torch.uint8, device=dev)
-    ws_c = torch.empty(G.gptq_workspace_size(GPTQ_OP_CHOLESKY, 0, n) + 512, dtype=torch.uint8,
-                       device=dev)
-    ws_q = torch.empty(G.gptq_workspace_size(GPTQ_OP_QUANTIZE, rows, n, 0, torch.bfloat16, cfg)
-                       + 512, dtype=torch.uint8, device=dev)
+    lq = G.LayerQuantizer(rows, n, N, wl.bits, wl.group_size, wl.percdamp, wl.actorder,
+                          x_dtype=X.dtype, w_dtype=W.dtype, out_dtype=torch.bfloat16,
+                          device=dev)
     stream = torch.cuda.current_stream()
 
     def step(ev=None):
-        H.zero_()
-        if ev:
-            ev[0].record(stream)
-        G.gptq_hessian_accumulate(H, X, 2.0, ws=ws_h, info=info_h, stream=stream)
-        if ev:
-            ev[1].record(stream)
-        G.gptq_cholesky_inverse(H, wl.percdamp, wl.actorder, U, perm, dead, info, ws=ws_c,
-                                stream=stream)
-        if ev:
-            ev[2].record(stream)
-        G.gptq_quantize_layer(W, U, perm, dead, cfg, codes, scales, zeros, g_idx, ws=ws_q,
-                              stream=stream)
-        if ev:
-            ev[3].record(stream)
-        pack(codes, packed, stream=stream)
-        if ev:
-            ev[4].record(stream)
-        G.gptq_dequant(packed, wl.bits, n, scales, zeros, wl.group_size, g_idx, torch.bfloat16,
-                       out=deq, stream=stream)
-        if ev:
-            ev[5].record(stream)
+        lq.run(W, X, stream=stream, events=ev)
 
     def barrier():
         if world > 1:
@@ -252,9 +283,7 @@ def run_ours(args, rank, world, local_rank):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    if int(info.item()) != 0 or int(info_h.item()) != 0:
-        raise RuntimeError(f"device status: cholesky info {int(info.item())}, "
-                           f"hessian info {int(info_h.item())}")
+    lq.check_info()
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
@@ -262,7 +291,11 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     torch.cuda.synchronize()
     launches0 = G.gptq_launch_count()
-    with ClockSampler(local_rank) as clk:
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
+    with ClockSampler(local_rank, uuid) as clk:
         t_start.record(stream)
         for k in range(args.steps):
             step(evs[k])
@@ -270,16 +303,12 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
     barrier()
     launches = G.gptq_launch_count() - launches0
-    ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    names = ["hessian", "cholesky_inverse", "sweep", "pack", "dequant"]
+    ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
+    names = list(G.LayerQuantizer.STAGES)
     stage = {nm: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
              for i, nm in enumerate(names)}
     ms_step = ms / args.steps
-    value = world * rows * n * args.steps / (ms / 1e3)
+    value = job_throughput(world, rows * n, args.steps, ms)
     flops = float(n) * (n + 1) * N
     t_h = stage["hessian"] / 1e3
     pk = peaks()
@@ -303,7 +332,7 @@ def run_ours(args, rank, world, local_rank):
         Xh.copy_(X)
         Wh = torch.empty_like(W, device="cpu").pin_memory()
         Wh.copy_(W)
-        outs = [packed, scales, zeros, g_idx]
+        outs = [lq.packed, lq.scales, lq.zeros, lq.g_idx]
         outs_h = [torch.empty_like(t, device="cpu").pin_memory() for t in outs]
         Xd = torch.empty_like(X)
         Wd = torch.empty_like(W)
@@ -311,15 +340,7 @@ def run_ours(args, rank, world, local_rank):
         def e2e_step():
             Xd.copy_(Xh, non_blocking=True)
             Wd.copy_(Wh, non_blocking=True)
-            H.zero_()
-            G.gptq_hessian_accumulate(H, Xd, 2.0, ws=ws_h, info=info_h, stream=stream)
-            G.gptq_cholesky_inverse(H, wl.percdamp, wl.actorder, U, perm, dead, info, ws=ws_c,
-                                    stream=stream)
-            G.gptq_quantize_layer(Wd, U, perm, dead, cfg, codes, scales, zeros, g_idx, ws=ws_q,
-                                  stream=stream)
-            pack(codes, packed, stream=stream)
-            G.gptq_dequant(packed, wl.bits, n, scales, zeros, wl.group_size, g_idx,
-                           torch.bfloat16, out=deq, stream=stream)
+            lq.run(Wd, Xd, stream=stream)
             for t, th in zip(outs, outs_h):
                 th.copy_(t, non_blocking=True)
 
@@ -335,14 +356,10 @@ def run_ours(args, rank, world, local_rank):
         b.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ems = a.elapsed_time(b)
-        if world > 1:
-            t = torch.tensor([ems], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = max_over_ranks(a.elapsed_time(b), world, dev)
         h2d = X.numel() * X.element_size() + W.numel() * W.element_size()
         d2h = sum(t.numel() * t.element_size() for t in outs)
-        e2e = {"value": world * rows * n * args.steps / (ems / 1e3), "unit": UNIT,
+        e2e = {"value": job_throughput(world, rows * n, args.steps, ems), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": ems / args.steps}
         del Xh, Wh, Xd, Wd

@@ -24,7 +24,7 @@ from ._lib import (GPTQ_BF16, GPTQ_F32, GPTQ_OP_CHOLESKY, GPTQ_OP_HESSIAN, GPTQ_
 __all__ = ["GptqError", "GptqConfig", "gptq_workspace_size", "gptq_hessian_accumulate",
            "gptq_cholesky_inverse", "gptq_quantize_layer", "gptq_pack_int4", "gptq_pack_int3",
            "gptq_dequant", "gptq_status_string", "make_config", "QuantizedLinear",
-           "quantize_linear", "library"]
+           "quantize_linear", "LayerQuantizer", "library"]
 
 
 class GptqError(RuntimeError):
@@ -268,3 +268,89 @@ def quantize_linear(W: torch.Tensor, X=None, H: torch.Tensor | None = None, bits
     return QuantizedLinear(packed, q["scales"], q["zeros"], q["g_idx"], perm, bits, group_size, n,
                            q["codes"], info, H if keep_factors else None,
                            U if keep_factors else None, q["Wq"], q["row_loss"])
+
+
+class LayerQuantizer:
+    """Repeated GPTQ of one layer shape with every buffer allocated once.
+
+    ``run(W, X)`` enqueues the whole hot path on one stream, in order:
+    H = 0, H += 2 X X^T, dead inputs / act-order / damping / U, the column
+    sweep, packing, and dequantization to ``out_dtype``.  Outputs stay in the
+    attributes (``H``, ``U``, ``perm``, ``dead``, ``info``, ``codes``,
+    ``scales``, ``zeros``, ``g_idx``, ``packed``, ``deq`` and, if asked for,
+    ``Wq`` and ``row_loss``).  ``events``: six CUDA events recorded around the
+    five stages, for timing.
+    """
+
+    STAGES = ("hessian", "cholesky_inverse", "sweep", "pack", "dequant")
+
+    def __init__(self, rows: int, n: int, ntok: int, bits: int = 4, group_size: int = 128,
+                 percdamp: float = 0.01, actorder: bool = False,
+                 x_dtype: torch.dtype = torch.bfloat16, w_dtype: torch.dtype = torch.bfloat16,
+                 out_dtype: torch.dtype = torch.bfloat16, want_wq: bool = False,
+                 want_loss: bool = False, device=None):
+        if bits == 4 and n % 8:
+            raise GptqError("int4 packing needs n % 8 == 0")
+        if bits == 3 and n % 32:
+            raise GptqError("int3 packing needs n % 32 == 0")
+        if bits not in (3, 4):
+            raise GptqError("packed storage is int3 or int4")
+        dev = torch.device("cuda") if device is None else torch.device(device)
+        self.rows, self.n, self.ntok, self.bits = rows, n, ntok, bits
+        self.group_size, self.percdamp, self.actorder = group_size, percdamp, actorder
+        self.cfg = make_config(bits, group_size, percdamp, actorder)
+        G = 1 if group_size <= 0 else (n + group_size - 1) // group_size
+        f32 = torch.float32
+        self.H = torch.empty(n, n, dtype=f32, device=dev)
+        self.U = torch.empty(n, n, dtype=f32, device=dev)
+        self.perm = torch.empty(n, dtype=torch.int32, device=dev)
+        self.dead = torch.empty(n, dtype=torch.uint8, device=dev)
+        self.info = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.info_h = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.codes = torch.empty(rows, n, dtype=torch.uint8, device=dev)
+        self.scales = torch.empty(rows, G, dtype=f32, device=dev)
+        self.zeros = torch.empty(rows, G, dtype=torch.uint8, device=dev)
+        self.g_idx = torch.empty(n, dtype=torch.int32, device=dev)
+        self.packed = torch.empty(rows, n * bits // 32, dtype=torch.int32, device=dev)
+        self.deq = torch.empty(rows, n, dtype=out_dtype, device=dev)
+        self.Wq = torch.empty(rows, n, dtype=f32, device=dev) if want_wq else None
+        self.row_loss = torch.empty(rows, dtype=f32, device=dev) if want_loss else None
+        self.ws_h = _workspace(gptq_workspace_size(GPTQ_OP_HESSIAN, 0, n, ntok, x_dtype), dev,
+                               None)
+        self.ws_c = _workspace(gptq_workspace_size(GPTQ_OP_CHOLESKY, 0, n), dev, None)
+        self.ws_q = _workspace(gptq_workspace_size(GPTQ_OP_QUANTIZE, rows, n, 0, w_dtype,
+                                                   self.cfg), dev, None)
+        self._pack = gptq_pack_int4 if bits == 4 else gptq_pack_int3
+
+    def run(self, W: torch.Tensor, X: torch.Tensor, stream=None, events=None):
+        s = torch.cuda.current_stream() if stream is None else stream
+        ev = events
+
+        def mark(i):
+            if ev is not None:
+                ev[i].record(s)
+
+        with torch.cuda.stream(s):
+            self.H.zero_()
+        mark(0)
+        gptq_hessian_accumulate(self.H, X, 2.0, ws=self.ws_h, info=self.info_h, stream=s)
+        mark(1)
+        gptq_cholesky_inverse(self.H, self.percdamp, self.actorder, self.U, self.perm, self.dead,
+                              self.info, ws=self.ws_c, stream=s)
+        mark(2)
+        gptq_quantize_layer(W, self.U, self.perm, self.dead, self.cfg, self.codes, self.scales,
+                            self.zeros, self.g_idx, self.Wq, self.row_loss, ws=self.ws_q,
+                            stream=s)
+        mark(3)
+        self._pack(self.codes, self.packed, stream=s)
+        mark(4)
+        gptq_dequant(self.packed, self.bits, self.n, self.scales, self.zeros, self.group_size,
+                     self.g_idx, self.deq.dtype, out=self.deq, stream=s)
+        mark(5)
+        return self
+
+    def check_info(self) -> None:
+        """Raises GptqError if a device status word reports a failure (syncs)."""
+        ci, hi = int(self.info.item()), int(self.info_h.item())
+        if ci != 0 or hi != 0:
+            raise GptqError(f"device status: cholesky info {ci}, hessian info {hi}")
