@@ -1,0 +1,363 @@
+// The two latency-critical steps of one 128-wide Cholesky panel.
+//
+//  chol_diag_kernel    one CTA factors the panel's diagonal block A_pp = L L^T
+//                      and inverts L's four 32 x 32 diagonal leaves.
+//  panel_apply_kernel  every vector of the panel (a row of A below the block,
+//                      or a row of the inverse's right-hand side) is solved,
+//                      x = v L^-T, as four dense 32-column stages:
+//                          x_j = (v_j - sum_{k<j} x_k L_jk^T) Li_jj^T,
+//                      so no vector walks 128 dependent substitution steps.
+//
+// The diagonal block sits in shared memory and is worked in 32 x 32 leaves.
+// For leaf j one warp factors the leaf in registers (right-looking, unscaled
+// LDL^T steps; each step's column is published once in shared memory and
+// read back with 16-byte broadcast loads; square roots at the end), the rows
+// below it are solved against the leaf by substitution (one thread per row),
+// and the remaining lower block takes the rank-32 update from a transposed
+// copy of the solved rows (16-byte loads, 8 x 4 register tiles).  At the end
+// four warps invert the four leaves at once (one lane per column).
+// Every product is an fp32 FMA; no step uses reduced precision.
+#pragma once
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace gptq {
+
+constexpr int kDiagThreads = 256;
+constexpr int kDP = 129;   // row pitch (floats) of the block S
+constexpr int kXP = 132;   // row pitch of XT (transposed solved rows)
+constexpr int kTP = 36;    // row pitch of a transposed 32 x 32 leaf
+// S[128][kDP] | XT[32][kXP] | LTl[32][kTP] | rinv[128] | colb[2][32]
+constexpr size_t kDiagSmemBytes =
+    sizeof(float) * (128 * kDP + 32 * kXP + 32 * kTP + 128 + 64) + 16;
+
+// Outputs of chol_diag_kernel, in the Cholesky workspace:
+//   Lt[k][c]     = L[c][k]           (128 x 128, zero for k > c)
+//   LiT[j][t][c] = (L_jj^-1)[c][t]   (4 leaves of 32 x 32, zero for t > c)
+constexpr int kDiagOutFloats = 128 * 128 + 4 * 32 * 32;
+
+// One warp: factor the 32 x 32 leaf at (c0, c0) of S in place (lower part);
+// writes 1 / L_kk to rinv[c0 + k] and the leaf transposed to LTl[t][m] =
+// L[c0+m][c0+t].  Returns (warp-uniform) the 1-based index of the first
+// non-positive or non-finite pivot within the leaf, or 0.
+__device__ __forceinline__ int leaf_factor(float* S, float* rinv, float* LTl, float* colb,
+                                           int c0, int lane) {
+  float a[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) a[k] = (k <= lane) ? S[(c0 + lane) * kDP + c0 + k] : 0.f;
+  int first_bad = 0;
+  // Column j is published (lane k writes its a[j]) as soon as its last
+  // update is done, so the next step's broadcast overlaps this step's FMAs;
+  // two buffers, so a step's write never meets the previous step's reads.
+  colb[lane] = a[0];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float* cb = colb + (j & 1) * 32;
+    __syncwarp();
+    float col[32];
+#pragma unroll
+    for (int q = j / 4; q < 8; ++q) {
+      const float4 v = reinterpret_cast<const float4*>(cb)[q];
+      col[4 * q] = v.x;
+      col[4 * q + 1] = v.y;
+      col[4 * q + 2] = v.z;
+      col[4 * q + 3] = v.w;
+    }
+    const float d = col[j];
+    const bool badj = !(d > 0.f) || !isfinite(d);
+    first_bad = (first_bad == 0 && badj) ? (j + 1) : first_bad;
+    // 1/d: hardware estimate and one Newton step (a multiplier needs no more)
+    const float r0 = ptx::rcp_approx(d);
+    const float rd = fmaf(fmaf(-d, r0, 1.f), r0, r0);
+    const float m = (lane > j) ? a[j] * rd : 0.f;
+    if (j + 1 < 32) {
+      a[j + 1] = fmaf(-m, col[j + 1], a[j + 1]);
+      colb[((j + 1) & 1) * 32 + lane] = a[j + 1];
+    }
+#pragma unroll
+    for (int k = j + 2; k < 32; ++k) a[k] = fmaf(-m, col[k], a[k]);
+  }
+  if (first_bad) return first_bad;
+  // L_ik = a_ik / sqrt(d_k), L_kk = sqrt(d_k)
+  float dd = 1.f;
+#pragma unroll
+  for (int k = 0; k < 32; ++k)
+    if (k == lane) dd = a[k];
+  const float rs = __frsqrt_rn(dd);
+  rinv[c0 + lane] = rs;
+  const float lkk = __fsqrt_rn(dd);
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const float rk = __shfl_sync(0xffffffffu, rs, k);
+    const float l = (k < lane) ? a[k] * rk : ((k == lane) ? lkk : 0.f);
+    if (k <= lane) S[(c0 + lane) * kDP + c0 + k] = l;
+    LTl[k * kTP + lane] = l;   // zero above the diagonal of the transpose
+  }
+  return 0;
+}
+
+// One warp: column `lane` of the inverse of the 32 x 32 lower leaf at
+// (c0, c0) of S, written as row `lane` of LiT: LiT[lane][m] = Li[m][lane].
+__device__ __forceinline__ void leaf_inverse(const float* S, const float* rinv, float* LiT,
+                                             int c0, int lane) {
+  float x[32];
+#pragma unroll
+  for (int m = 0; m < 32; ++m) x[m] = (m == lane) ? 1.f : 0.f;
+#pragma unroll
+  for (int t = 0; t < 32; ++t) {
+    const float xt = x[t] * rinv[c0 + t];
+    x[t] = xt;
+#pragma unroll
+    for (int m = t + 1; m < 32; ++m) x[m] = fmaf(-S[(c0 + m) * kDP + c0 + t], xt, x[m]);
+  }
+  float4* dst = reinterpret_cast<float4*>(LiT + lane * 32);
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    dst[q] = make_float4(4 * q + 0 >= lane ? x[4 * q + 0] : 0.f, 4 * q + 1 >= lane ? x[4 * q + 1] : 0.f,
+                         4 * q + 2 >= lane ? x[4 * q + 2] : 0.f, 4 * q + 3 >= lane ? x[4 * q + 3] : 0.f);
+}
+
+// Factor the diagonal block of panel p of the n x n lower matrix A and
+// invert its leaves; writes Lt and LiT (layouts above) to `out`.  Rows and
+// columns past a short last panel are identity padding.  On a failed pivot
+// sets *info = n - (global index of the pivot in A), if no failure was
+// recorded before, and returns.
+__global__ void __launch_bounds__(kDiagThreads) chol_diag_kernel(const float* __restrict__ A,
+                                                                 int n, int p,
+                                                                 float* __restrict__ out,
+                                                                 int32_t* __restrict__ info) {
+  if (*(volatile int32_t*)info != 0) return;
+  extern __shared__ __align__(16) float dsm[];
+  float* S = dsm;                    // [128][kDP]  the block, becomes L
+  float* XT = S + 128 * kDP;         // [32][kXP]   XT[k][r] = solved row r, column k of the leaf
+  XT = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(XT) + 15) & ~uintptr_t(15));
+  float* LTl = XT + 32 * kXP;        // [32][kTP]   current leaf, transposed
+  float* rinv = LTl + 32 * kTP;      // [128]       1 / L_kk
+  float* colb = rinv + 128;          // [2][32]     the leaf factor's column buffers
+  __shared__ int fail;
+  const int kb = p * 128;
+  const int bs = min(128, n - kb);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  // stage the lower block (async copies, all in flight at once); rows past
+  // bs are the identity; entries above the diagonal are never read
+  for (int f = tid; f < 128 * 32; f += kDiagThreads) {
+    const int r = f >> 5, c = (f & 31) * 4;
+    if (c > r) continue;
+    if (r >= bs) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) S[r * kDP + c + i] = (r == c + i) ? 1.f : 0.f;
+      continue;
+    }
+    const float* src = A + (int64_t)(kb + r) * n + kb + c;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      ptx::cp_async_4(S + r * kDP + c + i, (c + i < bs) ? src + i : src, (c + i < bs) ? 4 : 0);
+  }
+  ptx::cp_async_wait_all();
+  if (tid == 0) fail = 0;
+  __syncthreads();
+
+  for (int j = 0; j < 4; ++j) {
+    const int c0 = 32 * j;
+    if (warp == 0) {
+      const int fb = leaf_factor(S, rinv, LTl, colb, c0, lane);
+      if (fb && lane == 0) fail = c0 + fb;
+    }
+    __syncthreads();
+    if (fail) {
+      if (tid == 0) atomicCAS(info, 0, n - (kb + fail - 1));
+      return;
+    }
+    const int base = c0 + 32;
+    const int rem = 128 - base;
+    if (rem == 0) break;
+    // rows below the leaf: x <- x L_jj^-T by substitution, one thread per row;
+    // the leaf's columns come from LTl as 16-byte broadcasts
+    if (tid < rem) {
+      const int r = base + tid;
+      float x[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) x[k] = S[r * kDP + c0 + k];
+#pragma unroll
+      for (int t = 0; t < 32; ++t) {
+        const float xt = x[t] * rinv[c0 + t];
+        x[t] = xt;
+        const float4* lt = reinterpret_cast<const float4*>(LTl + t * kTP);
+#pragma unroll
+        for (int q = (t + 1) / 4; q < 8; ++q) {
+          const float4 l4 = lt[q];
+          if (4 * q + 0 > t) x[4 * q + 0] = fmaf(-xt, l4.x, x[4 * q + 0]);
+          if (4 * q + 1 > t) x[4 * q + 1] = fmaf(-xt, l4.y, x[4 * q + 1]);
+          if (4 * q + 2 > t) x[4 * q + 2] = fmaf(-xt, l4.z, x[4 * q + 2]);
+          if (4 * q + 3 > t) x[4 * q + 3] = fmaf(-xt, l4.w, x[4 * q + 3]);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        S[r * kDP + c0 + k] = x[k];
+        XT[k * kXP + (r - base)] = x[k];
+      }
+    }
+    __syncthreads();
+    // rank-32 update of the remaining lower block: 8-row x 4-column tiles
+    // (ti, tj) with 4 tj <= 8 ti + 7; rows past bs are identity padding
+    {
+      const int mt = rem / 8;                 // row tiles
+      const int ntiles = mt * (mt + 1);       // sum over ti of (2 ti + 2)
+      for (int t = tid; t < ntiles; t += kDiagThreads) {
+        int ti = 0;
+        while ((ti + 1) * (ti + 2) <= t) ++ti;
+        const int tj = t - ti * (ti + 1);
+        const int rl = 8 * ti, sl = 4 * tj;   // local to base
+        float acc[8][4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[i][q] = 0.f;
+#pragma unroll 4
+        for (int k = 0; k < 32; ++k) {
+          const float4 r4a = *reinterpret_cast<const float4*>(XT + k * kXP + rl);
+          const float4 r4b = *reinterpret_cast<const float4*>(XT + k * kXP + rl + 4);
+          const float4 s4 = *reinterpret_cast<const float4*>(XT + k * kXP + sl);
+          const float ra[8] = {r4a.x, r4a.y, r4a.z, r4a.w, r4b.x, r4b.y, r4b.z, r4b.w};
+          const float sa[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[i][q] = fmaf(ra[i], sa[q], acc[i][q]);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = base + rl + i;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int s = base + sl + q;
+            if (s <= r && r < bs) S[r * kDP + s] -= acc[i][q];
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---- outputs: L transposed, then the four leaf inverses
+  float* Lt = out;
+  float* LiT = out + 128 * 128;
+  for (int f = tid; f < 128 * 32; f += kDiagThreads) {
+    const int k = f >> 5, c = (f & 31) * 4;
+    float4 o;
+    o.x = (k <= c + 0) ? S[(c + 0) * kDP + k] : 0.f;
+    o.y = (k <= c + 1) ? S[(c + 1) * kDP + k] : 0.f;
+    o.z = (k <= c + 2) ? S[(c + 2) * kDP + k] : 0.f;
+    o.w = (k <= c + 3) ? S[(c + 3) * kDP + k] : 0.f;
+    reinterpret_cast<float4*>(Lt)[f] = o;
+  }
+  if (warp < 4) leaf_inverse(S, rinv, LiT + warp * 32 * 32, 32 * warp, lane);
+}
+
+// x = v L^-T for every vector of panel p: vectors [0, nA) are rows
+// kb+bs+v of A, vectors [nA, nA + kb + bs) are rows v - nA of RT (both
+// restricted to the panel's columns [kb, kb + bs)).  The result goes, split
+// into its TF32 part and remainder, to row g of PBh / PBl (g = the vector's
+// row in A or RT); RT rows also get x written back.
+// 32 vectors per CTA; stage j: thread (v, cq) = (tid / 8, tid % 8) owns
+// columns 32 j + 4 cq .. + 3 of vector v.
+constexpr int kApplyThreads = 256;
+constexpr int kApplyVecs = 32;
+constexpr int kVP = 132;  // row pitch of the vector tile
+constexpr size_t kApplySmemBytes =
+    sizeof(float) * (128 * 128 + 4 * 32 * 32 + 2 * kApplyVecs * kVP);
+
+__global__ void __launch_bounds__(kApplyThreads) panel_apply_kernel(
+    const float* __restrict__ A, float* __restrict__ RT, int n, int p,
+    const float* __restrict__ diag_out, float* __restrict__ PBh, float* __restrict__ PBl,
+    const int32_t* __restrict__ info) {
+  if (*(volatile const int32_t*)info != 0) return;
+  extern __shared__ __align__(16) float asmem[];
+  float* Lt = asmem;                         // [128][128]
+  float* LiT = Lt + 128 * 128;               // [4][32][32]
+  float* X = LiT + 4 * 32 * 32;              // [32][kVP]  vectors, solved in place
+  float* Y = X + kApplyVecs * kVP;           // [32][kVP]  stage scratch
+  const int kb = p * 128;
+  const int bs = min(128, n - kb);
+  const int nA = n - kb - bs;
+  const int nvec = nA + kb + bs;
+  const int v0 = blockIdx.x * kApplyVecs;
+  if (v0 >= nvec) return;
+  const int tid = threadIdx.x;
+  // everything staged with async copies, all in flight at once
+  for (int f = tid; f < kDiagOutFloats / 4; f += kApplyThreads)
+    ptx::cp_async_16(asmem + 4 * f, diag_out + 4 * f);
+  for (int f = tid; f < kApplyVecs * 128; f += kApplyThreads) {
+    const int vi = f >> 7, k = f & 127;
+    const int v = v0 + vi;
+    const bool ok = v < nvec && k < bs;
+    const float* row = (v < nA) ? (A + (int64_t)(kb + bs + v) * n + kb)
+                                : (RT + (int64_t)min(v - nA, n - 1) * n + kb);
+    ptx::cp_async_4(X + vi * kVP + k, ok ? row + k : A, ok ? 4 : 0);
+  }
+  ptx::cp_async_wait_all();
+  __syncthreads();
+  const int vi = tid >> 3, cq = tid & 7;
+  float* xr = X + vi * kVP;
+  for (int j = 0; j < 4; ++j) {
+    const int cb = 32 * j + 4 * cq;
+    // y = v_j - sum_{k < 32 j} x_k L[cb + i][k]
+    float y0 = xr[cb], y1 = xr[cb + 1], y2 = xr[cb + 2], y3 = xr[cb + 3];
+#pragma unroll 8
+    for (int k = 0; k < 32 * j; ++k) {
+      const float xk = xr[k];
+      const float4 l4 = *reinterpret_cast<const float4*>(Lt + k * 128 + cb);
+      y0 = fmaf(-xk, l4.x, y0);
+      y1 = fmaf(-xk, l4.y, y1);
+      y2 = fmaf(-xk, l4.z, y2);
+      y3 = fmaf(-xk, l4.w, y3);
+    }
+    *reinterpret_cast<float4*>(Y + vi * kVP + 4 * cq) = make_float4(y0, y1, y2, y3);
+    __syncthreads();
+    // x_j = y Li_jj^T: x[c] = sum_{t <= c} y[t] Li[c][t] = sum_t y[t] LiT[t][c]
+    const float* yr = Y + vi * kVP;
+    const float* lit = LiT + j * 32 * 32 + 4 * cq;
+    float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
+#pragma unroll 8
+    for (int t = 0; t < 32; ++t) {
+      const float yt = yr[t];
+      const float4 l4 = *reinterpret_cast<const float4*>(lit + t * 32);
+      z0 = fmaf(yt, l4.x, z0);
+      z1 = fmaf(yt, l4.y, z1);
+      z2 = fmaf(yt, l4.z, z2);
+      z3 = fmaf(yt, l4.w, z3);
+    }
+    *reinterpret_cast<float4*>(xr + cb) = make_float4(z0, z1, z2, z3);
+    __syncthreads();
+  }
+  // outputs
+  for (int f = tid; f < kApplyVecs * 32; f += kApplyThreads) {
+    const int vv = f >> 5, c4 = (f & 31) * 4;
+    const int v = v0 + vv;
+    if (v >= nvec) continue;
+    const bool is_rt = v >= nA;
+    const int64_t g = is_rt ? (int64_t)(v - nA) : (int64_t)(kb + bs + v);
+    float4 x4 = *reinterpret_cast<const float4*>(X + vv * kVP + c4);
+    float xv[4] = {x4.x, x4.y, x4.z, x4.w};
+    float hv[4], lv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (c4 + i >= bs) xv[i] = 0.f;
+      hv[i] = ptx::tf32_hi(xv[i]);
+      lv[i] = xv[i] - hv[i];
+    }
+    *reinterpret_cast<float4*>(PBh + g * 128 + c4) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+    *reinterpret_cast<float4*>(PBl + g * 128 + c4) = make_float4(lv[0], lv[1], lv[2], lv[3]);
+    if (is_rt) {
+      float* rt = RT + g * n + kb;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (c4 + i < bs) rt[c4 + i] = xv[i];
+    }
+  }
+}
+
+}  // namespace gptq

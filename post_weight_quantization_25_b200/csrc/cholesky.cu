@@ -17,10 +17,10 @@
 //
 // Both the factorisation and the inverse run right-looking over 128-wide
 // panels p = 0, 1, ...:
-//   (a) factor the diagonal block L_pp                         (1 CTA)
+//   (a) factor the diagonal block L_pp, invert its 32 x 32 leaves  (1 CTA)
 //   (b) apply L_pp^-1 to every vector that needs it: the panel rows below
-//       (-> L_ip, the triangular solve) and the block row p of the inverse's
-//       right-hand side (-> M_p., forward substitution)       (one warp per vector)
+//       (-> L_ip) and the block row p of the inverse's right-hand side
+//       (-> M_p.), in four dense 32-column stages (fp32 FMA)
 //   (c) rank-128 updates of the trailing lower matrix and of the remaining
 //       right-hand side rows                                   (fp32 tiles)
 // The inverse is kept transposed (RT = M^T) in U's own buffer, so that every
@@ -33,14 +33,13 @@
 #include <cstdint>
 
 #include "gptq_internal.cuh"
+#include "chol_diag.cuh"
 #include "panel_gemm.cuh"
-#include "stage.cuh"
 
 namespace gptq {
 namespace {
 
 constexpr int kPanel = kBlock;  // 128
-constexpr int kPadLD = kPanel + 1;
 constexpr int32_t kInfoTimeout = -2;  // `info` value when a device wait gave up
 
 struct CholWs {
@@ -49,6 +48,7 @@ struct CholWs {
   double* lam;    // 1: damping
   float* PBh;     // n x 128: the current panel's solved vectors, TF32 part
   float* PBl;     // n x 128: remainder
+  float* Dout;    // the diagonal step's outputs: L^T of the block, inverted leaves
 };
 
 constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -57,7 +57,7 @@ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // allocation-free entry point below, hence constexpr).
 constexpr size_t chol_ws_bytes(int64_t n) {
   return align_up(sizeof(float) * n * n, 256) + align_up(sizeof(float) * n, 256) + 256 +
-         2 * align_up(sizeof(float) * n * kPanel, 256);
+         2 * align_up(sizeof(float) * n * kPanel, 256) + sizeof(float) * kDiagOutFloats;
 }
 
 CholWs carve(void* ws, int64_t n) {
@@ -72,6 +72,8 @@ CholWs carve(void* ws, int64_t n) {
   w.PBh = reinterpret_cast<float*>(p);
   p += align_up(sizeof(float) * n * kPanel, 256);
   w.PBl = reinterpret_cast<float*>(p);
+  p += align_up(sizeof(float) * n * kPanel, 256);
+  w.Dout = reinterpret_cast<float*>(p);
   return w;
 }
 
@@ -163,323 +165,37 @@ __global__ void set_diag_one_kernel(float* __restrict__ M, int n) {
   if (i < n) M[(int64_t)i * n + i] = 1.f;
 }
 
-// ---------------------------------------------------------------- panel (a)
-// Factor the diagonal block of panel p in place (lower part of A).
-//
-// Blocked over four 32-column sub-panels, block kept in shared memory:
-//  (1) one warp factors the 32 x 32 diagonal sub-block in registers (lane i
-//      holds row i): per column one shuffle for the pivot, then the column's
-//      entries are shuffled to the lanes that need them -- no barriers;
-//  (2) the rows below it solve against that factor in parallel (one thread
-//      per row, 32 entries in registers, the factor read as broadcasts);
-//  (3) all threads subtract the rank-32 product from the remaining lower
-//      block with 4 x 4 register tiles.
-__device__ __forceinline__ float chol_elem(const float* S, int r, int c) {
-  return S[r * kPadLD + c];
-}
+// ---------------------------------------------------------------- panel (a), (b)
+// chol_diag_kernel and panel_apply_kernel (chol_diag.cuh).
 
-__global__ void __launch_bounds__(256) chol_diag_kernel(float* __restrict__ A, int n, int p,
-                                                        int32_t* __restrict__ info) {
-  if (*(volatile int32_t*)info != 0) return;
-  extern __shared__ float dyn_smem[];
-  float* S = dyn_smem;                     // [128][kPadLD]
-  float* rdiag = dyn_smem + kPanel * kPadLD;  // [128]
-  __shared__ int fail;
-  const int kb = p * kPanel;
-  const int bs = min(kPanel, n - kb);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const bool vec = (n % 4) == 0;
-  // stage the lower block (identity padding), 8 float4 loads in flight per thread
-  for (int f0 = 0; f0 < kPanel * kPanel / 4; f0 += 8 * 256) {
-    float4 v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int f = f0 + u * 256 + tid;
-      const int r = f >> 5, c = (f & 31) * 4;
-      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < bs && c <= r) {
-        const float* src = A + (int64_t)(kb + r) * n + kb + c;
-        if (vec && c + 3 < bs) {
-          v[u] = *reinterpret_cast<const float4*>(src);
-        } else {
-          v[u].x = src[0];
-          if (c + 1 < bs) v[u].y = src[1];
-          if (c + 2 < bs) v[u].z = src[2];
-          if (c + 3 < bs) v[u].w = src[3];
-        }
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int f = f0 + u * 256 + tid;
-      const int r = f >> 5, c = (f & 31) * 4;
-      float* d = S + r * kPadLD + c;
-      d[0] = (r == c) ? (r < bs ? v[u].x : 1.f) : v[u].x;
-      d[1] = (r == c + 1) ? (r < bs ? v[u].y : 1.f) : v[u].y;
-      d[2] = (r == c + 2) ? (r < bs ? v[u].z : 1.f) : v[u].z;
-      d[3] = (r == c + 3) ? (r < bs ? v[u].w : 1.f) : v[u].w;
-    }
-  }
-  if (tid == 0) fail = 0;
-  __syncthreads();
-
-  for (int c0 = 0; c0 < bs; c0 += 32) {
-    // (1) 32 x 32 diagonal sub-block, one warp, registers.  Unscaled
-    // (LDL^T-like) right-looking form: step j publishes column j as it
-    // stands (colj[k] = a_kj) and every lane i > j applies
-    // a_ik -= (a_ij / d_j) a_kj; the column entries are read from shared
-    // memory with independent loads issued ahead of the FMAs, so a step is
-    // one short dependency chain.  Square roots come at the end:
-    // L_ik = a_ik / sqrt(d_k), L_kk = sqrt(d_k).
-    if (warp == 0) {
-      float* colj = rdiag + kPanel;  // 32 floats of scratch after rdiag
-      float a[32];
-#pragma unroll
-      for (int k = 0; k < 32; ++k) a[k] = (k <= lane) ? chol_elem(S, c0 + lane, c0 + k) : 0.f;
-      bool bad = false;
-      int first_bad = 0;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        colj[lane] = (lane >= j) ? a[j] : 0.f;
-        __syncwarp();
-        const float d = colj[j];
-        // failure bookkeeping by selects (no branch inside the unrolled loop);
-        // once bad, the results are discarded
-        const bool badj = !(d > 0.f) || !isfinite(d);
-        first_bad = (!bad && badj) ? (c0 + j + 1) : first_bad;
-        bad = bad || badj;
-        float ck[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) ck[k] = (k > j) ? colj[k] : 0.f;
-        // 1/d: hardware estimate plus one Newton step (fp32 accurate to ~1
-        // ulp, which is all a multiplier of the factorisation needs)
-        const float r0 = ptx::rcp_approx(d);
-        const float rd = fmaf(fmaf(-d, r0, 1.f), r0, r0);
-        const float lij = (lane > j) ? a[j] * rd : 0.f;
-#pragma unroll
-        for (int k = 0; k < 32; ++k)
-          if (k > j) a[k] = fmaf(-lij, ck[k], a[k]);
-        __syncwarp();
-      }
-      if (bad && lane == 0) fail = first_bad;
-      if (!bad) {
-        // pivots d_k = a_kk; scale row `lane` by 1/sqrt(d_k)
-#pragma unroll
-        for (int k = 0; k < 32; ++k)
-          if (k == lane) colj[lane] = a[k];
-        __syncwarp();
-        const float rs_own = 1.f / sqrtf(colj[lane]);
-        rdiag[c0 + lane] = rs_own;  // 1 / L_kk for the solve below
-        __syncwarp();
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          if (k < lane) S[(c0 + lane) * kPadLD + c0 + k] = a[k] * rdiag[c0 + k];
-          if (k == lane) S[(c0 + lane) * kPadLD + c0 + k] = sqrtf(a[k]);
-        }
-      }
-    }
-    __syncthreads();
-    if (fail) {
-      if (tid == 0) atomicCAS(info, 0, n - (kb + fail - 1));
-      return;
-    }
-    // (2) rows below the sub-block: x <- x L_sub^-T, one thread per row
-    const int rem = bs - c0 - 32;
-    if (tid < rem) {
-      const int r = c0 + 32 + tid;
-      float x[32];
-#pragma unroll
-      for (int k = 0; k < 32; ++k) x[k] = chol_elem(S, r, c0 + k);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        x[j] *= rdiag[c0 + j];
-#pragma unroll
-        for (int k = 0; k < 32; ++k)
-          if (k > j) x[k] = fmaf(-x[j], chol_elem(S, c0 + k, c0 + j), x[k]);
-      }
-#pragma unroll
-      for (int k = 0; k < 32; ++k) S[r * kPadLD + c0 + k] = x[k];
-    }
-    __syncthreads();
-    // (3) trailing lower block [c0+32, bs)^2 -= rank-32 product, 4 x 4 tiles
-    if (rem > 0) {
-      const int mt = (rem + 3) / 4;
-      const int ntiles = mt * (mt + 1) / 2;
-      const int base = c0 + 32;
-      for (int t = tid; t < ntiles; t += blockDim.x) {
-        int ti = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
-        while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
-        while (ti * (ti + 1) / 2 > t) --ti;
-        const int tj = t - ti * (ti + 1) / 2;
-        const int r0 = base + 4 * ti, s0 = base + 4 * tj;
-        float acc[4][4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll 8
-        for (int k = 0; k < 32; ++k) {
-          float ra[4], sa[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) ra[i] = chol_elem(S, min(r0 + i, kPanel - 1), c0 + k);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) sa[j] = chol_elem(S, min(s0 + j, kPanel - 1), c0 + k);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(ra[i], sa[j], acc[i][j]);
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (r0 + i < bs && s0 + j < bs) S[(r0 + i) * kPadLD + s0 + j] -= acc[i][j];
-      }
-    }
-    __syncthreads();
-  }
-  for (int i = tid; i < bs * kPanel; i += blockDim.x) {
-    const int rr = i / kPanel, c = i % kPanel;
-    if (c <= rr) A[(int64_t)(kb + rr) * n + kb + c] = S[rr * kPadLD + c];
-  }
-}
-
-// ---------------------------------------------------------------- panel (b)
-// v <- L_pp^-1 v for every vector: the rows of A below the panel
-// (restricted to the panel's columns) and rows [0, kb + bs) of RT.
-// Four lanes (a quad) per vector, eight vectors per warp; lane q holds
-// entries q, q+4, ..., q+124 (slot s = entry / 4).  Step j: the owner lane
-// (j % 4) scales entry j by 1/L_jj, the quad shares it, and every lane
-// subtracts it times column j of L from its later entries.  Shared memory
-// holds Lq[j][q][s] = L[4 s + q][j] (pitch 36 floats: float4 reads, no bank
-// conflicts); unrolled over j so finished slots cost nothing.
-constexpr int kSolveThreads = 128;
-constexpr int kLqPitch = 36;
-constexpr int kLqRow = 4 * kLqPitch;
-constexpr size_t kSolveSmemBytes = sizeof(float) * (kPanel * kLqRow + kPanel);
-
-// Every solved vector is also written, split into its TF32 part and the
-// remainder, to row `g` of the panel buffer PBh / PBl (g = the vector's row
-// in A or RT), the operand of the tensor-core trailing update.  Rows of A
-// below the panel are not written back: only the trailing update reads them.
-__global__ void __launch_bounds__(kSolveThreads) panel_solve_kernel(
-    float* __restrict__ A, float* __restrict__ RT, int n, int p, float* __restrict__ PBh,
-    float* __restrict__ PBl, const int32_t* __restrict__ info) {
-  if (*(volatile const int32_t*)info != 0) return;
-  extern __shared__ __align__(16) float dyn_smem[];
-  float* Lq = dyn_smem;
-  float* rdiag = dyn_smem + kPanel * kLqRow;
-  const int kb = p * kPanel;
-  const int bs = min(kPanel, n - kb);
-  stage_block_128<kSolveThreads>(
-      A + (int64_t)kb * n + kb, n, bs, bs, /*lower=*/true, (n % 4) == 0,
-      [&](int r, int c, float v) { Lq[c * kLqRow + (r & 3) * kLqPitch + (r >> 2)] = v; },
-      [](int r, int c) { return (r == c) ? 1.f : 0.f; });
-  __syncthreads();
-  for (int i = threadIdx.x; i < kPanel; i += blockDim.x)
-    rdiag[i] = 1.f / Lq[i * kLqRow + (i & 3) * kLqPitch + (i >> 2)];
-  __syncthreads();
-
-  const int q = threadIdx.x & 3;
-  const int lane = threadIdx.x & 31;
-  const int nA = n - kb - bs;
-  const int nvec = nA + kb + bs;
-  const int quads = (gridDim.x * blockDim.x) >> 2;
-  const float* lq_lane = Lq + q * kLqPitch;
-  // `base` is the warp's first vector: uniform across the warp, so the whole
-  // warp stays in the loop together (the shuffles need all 32 lanes)
-  for (int base = (blockIdx.x * blockDim.x + (threadIdx.x & ~31)) >> 2; base < nvec;
-       base += quads) {
-    const int v0 = base + (lane >> 2);
-    const bool active = v0 < nvec;
-    float* vec = !active ? nullptr
-                 : (v0 < nA) ? (A + (int64_t)(kb + bs + v0) * n + kb)
-                             : (RT + (int64_t)(v0 - nA) * n + kb);
-    float x[32];
-#pragma unroll
-    for (int s = 0; s < 32; ++s) {
-      const int c = 4 * s + q;
-      x[s] = (active && c < bs) ? vec[c] : 0.f;
-    }
-#pragma unroll
-    for (int s = 0; s < 32; ++s) {
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        // no early exit for a short panel: entries past bs are 0 and the
-        // padded factor is the identity there, so those steps change nothing
-        const int j = 4 * s + k;
-        const float yv = x[s] * rdiag[j];
-        const float y = __shfl_sync(0xffffffffu, yv, k, 4);
-        const float* lcol = lq_lane + j * kLqRow;
-#pragma unroll
-        for (int s4 = s >> 2; s4 < 8; ++s4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lcol + 4 * s4);
-          if (4 * s4 + 0 >= s) x[4 * s4 + 0] = fmaf(-l4.x, y, x[4 * s4 + 0]);
-          if (4 * s4 + 1 >= s) x[4 * s4 + 1] = fmaf(-l4.y, y, x[4 * s4 + 1]);
-          if (4 * s4 + 2 >= s) x[4 * s4 + 2] = fmaf(-l4.z, y, x[4 * s4 + 2]);
-          if (4 * s4 + 3 >= s) x[4 * s4 + 3] = fmaf(-l4.w, y, x[4 * s4 + 3]);
-        }
-        x[s] = (q == k) ? y : x[s];
-      }
-    }
-    if (active) {
-      const bool is_rt = v0 >= nA;
-      const int64_t g = is_rt ? (int64_t)(v0 - nA) : (int64_t)(kb + bs + v0);
-      float* ph = PBh + g * kPanel;
-      float* pl = PBl + g * kPanel;
-#pragma unroll
-      for (int s = 0; s < 32; ++s) {
-        const int c = 4 * s + q;
-        const float xv = (c < bs) ? x[s] : 0.f;
-        if (is_rt && c < bs) vec[c] = xv;
-        float h, l;
-        tf32_split(xv, h, l);
-        ph[c] = h;
-        pl[c] = l;
-      }
-    }
-  }
-}
-
-// The trailing update of panel p as tiles for the tensor-core panel GEMM.
-// Tiles [0, T1): lower tiles (rb, sb), p < sb <= rb, of A -= L_p L_p^T;
-// tiles [T1, T1+T2): RT[cb][rb] -= RT[cb][p] L[rb][p]^T, cb <= p < rb.
-// Both operands are rows of the panel buffer (P = rows of the C tile's row
-// block, Q = rows of its column block).
-struct CholTrailDecoder {
+// The trailing update of panel p as items for the tensor-core panel GEMM.
+// Item R (a 128-row block, P = its rows of the panel buffer):
+//   R > p:  lower tiles A[R][S] -= L_Rp L_Sp^T for p < S <= R   (R - p tiles)
+//   R <= p: tiles RT[R][S] -= RT[R][p] L_Sp^T for p < S < nblk  (nblk-1-p tiles)
+// In both cases the Q rows (the panel buffer rows of block S) and the C
+// tiles run over consecutive blocks from S = p + 1.
+struct CholTrailItems {
   float* A;
   float* RT;
   int n, p, nblk;
-  __device__ PgTile tile(int bx, int) const {
-    PgTile t;
-    const int m = nblk - p - 1;
-    const int T1 = m * (m + 1) / 2;
-    int idx = bx;
-    t.ldc = n;
-    t.pkx = 0;
-    t.qkx = 0;
-    if (idx < T1) {
-      int rr = (int)((sqrtf(8.f * (float)idx + 1.f) - 1.f) * 0.5f);
-      while ((rr + 1) * (rr + 2) / 2 <= idx) ++rr;
-      while (rr * (rr + 1) / 2 > idx) --rr;
-      const int ss = idx - rr * (rr + 1) / 2;
-      const int rb = p + 1 + rr, sb = p + 1 + ss;
-      t.C = A + (int64_t)rb * kPanel * n + (int64_t)sb * kPanel;
-      t.prow = rb * kPanel;
-      t.qrow = sb * kPanel;
-      t.mext = min(kPanel, n - rb * kPanel);
-      t.cext = min(kPanel, n - sb * kPanel);
-    } else {
-      idx -= T1;
-      const int cb = idx / m, rb = p + 1 + idx % m;
-      t.C = RT + (int64_t)cb * kPanel * n + (int64_t)rb * kPanel;
-      t.prow = cb * kPanel;
-      t.qrow = rb * kPanel;
-      t.mext = kPanel;
-      t.cext = min(kPanel, n - rb * kPanel);
-    }
-    t.valid = 1;
-    return t;
+  __host__ __device__ int num_items() const { return nblk; }
+  __host__ __device__ int item_nq(int R) const { return R > p ? R - p : nblk - 1 - p; }
+  __device__ PgItem item(int R) const {
+    PgItem I;
+    const int c0 = (p + 1) * kPanel;
+    I.C0 = (R > p ? A : RT) + (int64_t)R * kPanel * n + c0;
+    I.ldc = n;
+    I.cmap = R > p ? 0 : 1;
+    I.cx0 = c0;
+    I.cy0 = R * kPanel;
+    I.prow = R * kPanel;
+    I.pkx = 0;
+    I.qrow0 = c0;
+    I.qkx = 0;
+    I.nq = item_nq(R);
+    I.mext = min(kPanel, n - R * kPanel);
+    I.cext_last = min(kPanel, n - c0 - kPanel * (I.nq - 1));
+    return I;
   }
 };
 
@@ -554,37 +270,54 @@ cudaError_t launch_cholesky_inverse(const float* H, int64_t n64, float percdamp,
 
   const int nblk = (n + kPanel - 1) / kPanel;
   const int sms = num_sms();
-  const size_t diag_smem = sizeof(float) * (kPanel * kPadLD + 2 * kPanel);
-  const size_t solve_smem = kSolveSmemBytes;
-  if ((e = cudaFuncSetAttribute(chol_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)diag_smem)) != cudaSuccess ||
-      (e = cudaFuncSetAttribute(panel_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)solve_smem)) != cudaSuccess)
+  if ((e = cudaFuncSetAttribute(chol_diag_kernel,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kDiagSmemBytes)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(panel_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kApplySmemBytes)) != cudaSuccess)
     return e;
-  // one quad per vector (n vectors per panel), capped at 3 resident CTAs per SM
-  const int solve_ctas = std::min((4 * n + kSolveThreads - 1) / kSolveThreads, 3 * sms);
-  CUtensorMap mPh, mPl;
+  const int apply_ctas = (n + kApplyVecs - 1) / kApplyVecs;  // n vectors per panel
+  // operands of the trailing updates; with a row stride that is a multiple
+  // of 16 bytes the updates land in A and RT by TMA reduce-add
+  CUtensorMap mPh, mPl, mA, mRT;
+  const bool reduce = (n % 4) == 0;
   if (nblk > 1) {
     if (!make_tma_2d(&mPh, w.PBh, false, n, kPanel, kPanel, 32, 128) ||
         !make_tma_2d(&mPl, w.PBl, false, n, kPanel, kPanel, 32, 128))
       return cudaErrorInvalidValue;
-    if ((e = cudaFuncSetAttribute(panel_gemm_kernel<CholTrailDecoder>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)kPgSmemBytes)) != cudaSuccess)
-      return e;
+    if (reduce) {
+      if (!make_tma_2d(&mA, w.A, false, n, n, n, 32, 32) ||
+          !make_tma_2d(&mRT, U, false, n, n, n, 32, 32))
+        return cudaErrorInvalidValue;
+      if ((e = cudaFuncSetAttribute(panel_gemm2_kernel<CholTrailItems, true>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)pg2_smem_bytes(true))) != cudaSuccess)
+        return e;
+    } else {
+      mA = mRT = mPh;  // not read by the read-modify-write epilogue
+      if ((e = cudaFuncSetAttribute(panel_gemm2_kernel<CholTrailItems, false>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)pg2_smem_bytes(false))) != cudaSuccess)
+        return e;
+    }
   }
   for (int p = 0; p < nblk; ++p) {
-    chol_diag_kernel<<<1, 256, diag_smem, s>>>(w.A, n, p, info);
+    chol_diag_kernel<<<1, kDiagThreads, kDiagSmemBytes, s>>>(w.A, n, p, w.Dout, info);
     note_launch();
-    panel_solve_kernel<<<solve_ctas, kSolveThreads, solve_smem, s>>>(w.A, U, n, p, w.PBh, w.PBl,
-                                                                      info);
+    panel_apply_kernel<<<apply_ctas, kApplyThreads, kApplySmemBytes, s>>>(
+        w.A, U, n, p, w.Dout, w.PBh, w.PBl, info);
     note_launch();
-    const int m = nblk - p - 1;
-    const int tiles = m * (m + 1) / 2 + (p + 1) * m;
-    if (tiles > 0) {
-      const CholTrailDecoder dec{w.A, U, n, p, nblk};
-      panel_gemm_kernel<CholTrailDecoder><<<tiles, kPgThreads, kPgSmemBytes, s>>>(
-          mPh, mPl, mPh, mPl, dec, info, kInfoTimeout, info);
+    if (p + 1 < nblk) {
+      const CholTrailItems dec{w.A, U, n, p, nblk};
+      int chunk = 1, units = 0;
+      pg2_plan(dec, sms, chunk, units);
+      const int grid = std::min(units, sms);
+      if (reduce)
+        panel_gemm2_kernel<CholTrailItems, true><<<grid, kPg2Threads, pg2_smem_bytes(true), s>>>(
+            mPh, mPl, mPh, mPl, mA, mRT, dec, chunk, units, info, kInfoTimeout, info);
+      else
+        panel_gemm2_kernel<CholTrailItems, false><<<grid, kPg2Threads, pg2_smem_bytes(false), s>>>(
+            mPh, mPl, mPh, mPl, mA, mRT, dec, chunk, units, info, kInfoTimeout, info);
       note_launch();
     }
   }

@@ -108,6 +108,9 @@ struct SweepTrailItems {
     PgItem I;
     I.C0 = Wf + (int64_t)i * 128 * n + i2;
     I.ldc = n;
+    I.cmap = 0;
+    I.cx0 = i2;
+    I.cy0 = 128 * i;
     I.prow = 128 * i;
     I.pkx = 0;
     I.qrow0 = i2;
@@ -469,8 +472,10 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
   const int sweep_ctas = (rows * 4 + kSweepThreads - 1) / kSweepThreads;
   const int sms = num_sms();
 
-  // operands of the lazy update on the tensor cores
-  CUtensorMap mEh, mEl, mUh, mUl;
+  // operands of the lazy update on the tensor cores; with a row stride that
+  // is a multiple of 16 bytes the update lands in Wf by TMA reduce-add
+  CUtensorMap mEh, mEl, mUh, mUl, mW;
+  const bool reduce = (n % 4) == 0;
   if (n > kBlock) {
     ut_split_kernel<<<dim3((unsigned)((w.ldut + 31) / 32), (unsigned)((n + 31) / 32)), 256, 0, s>>>(
         U, n, w.ldut, w.UT_hi, w.UT_lo);
@@ -480,10 +485,19 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
         !make_tma_2d(&mUh, w.UT_hi, false, n, n, w.ldut, 32, 128) ||
         !make_tma_2d(&mUl, w.UT_lo, false, n, n, w.ldut, 32, 128))
       return cudaErrorInvalidValue;
-    if ((e = cudaFuncSetAttribute(panel_gemm2_kernel<SweepTrailItems>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)kPg2SmemBytes)) != cudaSuccess)
-      return e;
+    if (reduce) {
+      if (!make_tma_2d(&mW, w.Wf, false, rows, n, n, 32, 32)) return cudaErrorInvalidValue;
+      if ((e = cudaFuncSetAttribute(panel_gemm2_kernel<SweepTrailItems, true>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)pg2_smem_bytes(true))) != cudaSuccess)
+        return e;
+    } else {
+      mW = mEh;  // not read by the read-modify-write epilogue
+      if ((e = cudaFuncSetAttribute(panel_gemm2_kernel<SweepTrailItems, false>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)pg2_smem_bytes(false))) != cudaSuccess)
+        return e;
+    }
   }
   for (int i1 = 0; i1 < n; i1 += kBlock) {
     const int bsz = std::min(kBlock, n - i1);
@@ -506,8 +520,13 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
       const SweepTrailItems dec{w.Wf, rows, n, i1, i2};
       int chunk = 1, units = 0;
       pg2_plan(dec, sms, chunk, units);
-      panel_gemm2_kernel<SweepTrailItems><<<std::min(units, sms), kPg2Threads, kPg2SmemBytes, s>>>(
-          mEh, mEl, mUh, mUl, dec, chunk, units, nullptr, 0, nullptr);
+      const int grid = std::min(units, sms);
+      if (reduce)
+        panel_gemm2_kernel<SweepTrailItems, true><<<grid, kPg2Threads, pg2_smem_bytes(true), s>>>(
+            mEh, mEl, mUh, mUl, mW, mW, dec, chunk, units, nullptr, 0, nullptr);
+      else
+        panel_gemm2_kernel<SweepTrailItems, false><<<grid, kPg2Threads, pg2_smem_bytes(false), s>>>(
+            mEh, mEl, mUh, mUl, mW, mW, dec, chunk, units, nullptr, 0, nullptr);
       note_launch();
     }
   }
