@@ -318,7 +318,7 @@ def run_ours(args, rank, world, local_rank):
     if os.path.exists(tf_path):
         with open(tf_path) as f:
             tj = json.load(f)
-        if tj.get("workload") == wl.name and tj.get("kernel_rev") == "syrk-v1":
+        if tj.get("workload") == wl.name and tj.get("kernel_rev") == "syrk-v2":
             traffic = tj.get("bytes_per_launch")
     roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_tflops"],
             "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": traffic,

@@ -26,8 +26,7 @@ Source of every formula: the web page "GPTQ, with the code open"
 The page "What is GPTQ" (queryfeedz.com glossary), table "Key settings",
 lists the bit widths, group sizes and act-order setting exercised here.
 
-Readings where the pages are silent (each is listed with its reason in
-DESIGN.md):
+Readings where the pages are silent:
 
 * Rounding is IEEE round-half-to-even, for the code and for the zero point;
   the code is ``clamp(rint(w / scale) + zero, 0, 2^b - 1)`` with true division.

@@ -346,7 +346,7 @@ cudaError_t launch_cholesky_inverse(const float* H, int64_t n64, float percdamp,
 // these bytes until the process exits.
 //
 // Limit: n <= kNoAllocMaxN (2048), i.e. the scratch of one 2048 x 2048
-// factorisation, 18.9 MB.  Larger n is rejected with GPTQ_ERR_WORKSPACE.
+// factorisation, 19.0 MB.  Larger n is rejected with GPTQ_ERR_WORKSPACE.
 //
 // The array's name in host code is only a host-side stand-in, not a device
 // address.  The device address is looked up with cudaGetSymbolAddress once

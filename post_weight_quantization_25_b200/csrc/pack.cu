@@ -104,15 +104,9 @@ __device__ __forceinline__ int group_of(int64_t c, int group_size, const int32_t
   return group_size > 0 ? (int)(c / group_size) : 0;
 }
 
-template <bool BF16>
-__device__ __forceinline__ void store_out(void* out, int64_t idx, float v) {
-  if (BF16)
-    static_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
-  else
-    static_cast<float*>(out)[idx] = v;
-}
-
-// One thread per packed word (int4: 8 values) or word triple (int3: 32 values).
+// One thread per 8 consecutive values of a row: an int4 word, or a quarter
+// (24 bits) of an int3 word triple, so each thread writes 16 contiguous bytes
+// (bf16) or 32 (fp32) and a warp's stores are coalesced.
 template <int BITS, bool BF16>
 __global__ void dequant_kernel(const uint32_t* __restrict__ packed, int64_t units_per_row,
                                int64_t total, int64_t n, const float* __restrict__ scales,
@@ -120,57 +114,49 @@ __global__ void dequant_kernel(const uint32_t* __restrict__ packed, int64_t unit
                                const int32_t* __restrict__ g_idx, void* __restrict__ out) {
   const int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (g >= total) return;
-  const int64_t r = g / units_per_row, i = g % units_per_row;
+  const int64_t r = g / units_per_row, j = g % units_per_row;  // values [8 j, 8 j + 8)
   const float* srow = scales + r * G;
   const uint8_t* zrow = zeros + r * G;
+  uint32_t bits24;  // 8 codes, code k in bits [BITS k, BITS k + BITS)
   if (BITS == 4) {
-    const uint32_t w = packed[r * units_per_row + i];
-    const int64_t c0 = 8 * i;
-    float v[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int gi = group_of(c0 + k, group_size, g_idx);
-      const float q = (float)((w >> (4 * k)) & 0xFu);
-      v[k] = __fmul_rn(srow[gi], q - (float)zrow[gi]);
+    bits24 = packed[r * units_per_row + j];
+  } else {
+    // column 32 i + k sits in bits [3 k, 3 k + 3) of words 3i..3i+2 (little-endian)
+    const uint32_t* p = packed + r * (3 * (n / 32)) + 3 * (j >> 2);
+    switch (j & 3) {
+      case 0: bits24 = p[0] & 0xFFFFFFu; break;
+      case 1: bits24 = (p[0] >> 24) | ((p[1] & 0xFFFFu) << 8); break;
+      case 2: bits24 = (p[1] >> 16) | ((p[2] & 0xFFu) << 16); break;
+      default: bits24 = p[2] >> 8; break;
     }
-    if (BF16) {
-      __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out) + r * n + c0;
-      if ((reinterpret_cast<uintptr_t>(o) & 15) == 0) {
-        __align__(16) __nv_bfloat16 t[8];
+  }
+  const int64_t c0 = 8 * j;
+  float v[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) t[k] = __float2bfloat16_rn(v[k]);
-        *reinterpret_cast<uint4*>(o) = *reinterpret_cast<const uint4*>(t);
-      } else {
+  for (int k = 0; k < 8; ++k) {
+    const int gi = group_of(c0 + k, group_size, g_idx);
+    const float q = (float)((bits24 >> (BITS * k)) & ((1u << BITS) - 1u));
+    v[k] = __fmul_rn(srow[gi], q - (float)zrow[gi]);
+  }
+  if (BF16) {
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out) + r * n + c0;
+    if ((reinterpret_cast<uintptr_t>(o) & 15) == 0) {
+      __align__(16) __nv_bfloat16 t[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) o[k] = __float2bfloat16_rn(v[k]);
-      }
+      for (int k = 0; k < 8; ++k) t[k] = __float2bfloat16_rn(v[k]);
+      *reinterpret_cast<uint4*>(o) = *reinterpret_cast<const uint4*>(t);
     } else {
-      float* o = static_cast<float*>(out) + r * n + c0;
-      if ((reinterpret_cast<uintptr_t>(o) & 15) == 0) {
-        reinterpret_cast<float4*>(o)[0] = make_float4(v[0], v[1], v[2], v[3]);
-        reinterpret_cast<float4*>(o)[1] = make_float4(v[4], v[5], v[6], v[7]);
-      } else {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) o[k] = v[k];
-      }
+      for (int k = 0; k < 8; ++k) o[k] = __float2bfloat16_rn(v[k]);
     }
   } else {
-    const uint32_t* p = packed + r * (3 * units_per_row) + 3 * i;
-    const uint64_t lo = (uint64_t)p[0] | ((uint64_t)p[1] << 32);
-    const uint32_t hi = p[2];
-    const int64_t c0 = 32 * i;
+    float* o = static_cast<float*>(out) + r * n + c0;
+    if ((reinterpret_cast<uintptr_t>(o) & 15) == 0) {
+      reinterpret_cast<float4*>(o)[0] = make_float4(v[0], v[1], v[2], v[3]);
+      reinterpret_cast<float4*>(o)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    } else {
 #pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      const int bit = 3 * k;
-      uint32_t q;
-      if (bit + 3 <= 64)
-        q = (uint32_t)(lo >> bit) & 7u;
-      else if (bit < 64)
-        q = ((uint32_t)(lo >> bit) | (hi << (64 - bit))) & 7u;
-      else
-        q = (hi >> (bit - 64)) & 7u;
-      const int gi = group_of(c0 + k, group_size, g_idx);
-      store_out<BF16>(out, r * n + c0 + k, __fmul_rn(srow[gi], (float)q - (float)zrow[gi]));
+      for (int k = 0; k < 8; ++k) o[k] = v[k];
     }
   }
 }
@@ -220,7 +206,7 @@ cudaError_t launch_dequant(const uint32_t* packed, int bits, int64_t rows, int64
       dequant_kernel<4, false><<<blocks_for(total, 256), 256, 0, s>>>(
           packed, upr, total, n, scales, zeros, group_size, n_groups, g_idx, out);
   } else {
-    const int64_t upr = n / 32, total = rows * upr;
+    const int64_t upr = n / 8, total = rows * upr;  // n % 32 == 0 for int3
     if (out_bf16)
       dequant_kernel<3, true><<<blocks_for(total, 256), 256, 0, s>>>(
           packed, upr, total, n, scales, zeros, group_size, n_groups, g_idx, out);
