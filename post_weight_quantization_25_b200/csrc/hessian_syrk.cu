@@ -294,6 +294,266 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// ===========================================================================
+// The same SYRK on CTA pairs (clusters of 2): one tcgen05.mma.cta_group::2
+// (M = 256, N = 256, K = 16) covers a 256 x 256 tile of H.  CTA r of the
+// pair loads its own 128 rows of A (tile rows 128 r..) and its own half of
+// B (tile columns 128 r..), 32 KB per 64-token k-block instead of 48 KB per
+// SM, so the operand feed from L2 per unit of MMA work drops by a third.
+//  * Both CTAs' TMA loads count on the leader's (rank 0) `full` barrier; only
+//    the leader's producer posts the expected bytes (both CTAs' share).
+//  * Only the leader issues MMAs; each commit arrives on the `empty` /
+//    `tfull` barrier at the same offset in both CTAs.
+//  * Each CTA drains its own TMEM (its 128 rows x 256 columns); one lane per
+//    epilogue warp arrives on the leader's `tempty` (16 arrivals per piece).
+//  * TMEM is allocated and freed by one warp in each CTA (cta_group::2);
+//    cluster barriers order set-up and tear-down.
+// Tiles (I2, J) with I2 <= J cover the upper triangle in 256 x 256 blocks.
+// Accuracy handling is the single-CTA kernel's: fresh TMEM sums every
+// kSubKb k-blocks, added in an fp32 register tile, split-K atomics per unit.
+// ===========================================================================
+constexpr int P_STAGES = 6;
+constexpr int P_A_BYTES = 128 * BK * 2;   // this CTA's A rows
+constexpr int P_B_BYTES = 128 * BK * 2;   // this CTA's half of B
+constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
+constexpr size_t P_SMEM_BYTES = (size_t)P_STAGES * P_STAGE_BYTES + 1024 + 256;
+
+struct SyrkPairArgs {
+  float* H;
+  int n;
+  float alpha;
+  int nkb;          // k-blocks of BK tokens
+  int kb_per_unit;
+  int ntiles;       // 256 x 256 tiles touching the upper triangle
+  int units;        // ntiles * token chunks
+  int vec4;
+  int32_t* info;
+};
+
+// Tile t of the J-major enumeration: column block J holds row blocks 0..J.
+__device__ __forceinline__ void decode_tile_pair(int t, int& I2, int& J) {
+  J = 0;
+  while ((J + 1) * (J + 2) / 2 <= t) ++J;
+  I2 = t - J * (J + 1) / 2;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    syrk_bf16_pair_kernel(const __grid_constant__ CUtensorMap mapA,
+                          const __grid_constant__ CUtensorMap mapB, const SyrkPairArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + P_STAGES * P_A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P_STAGES * P_STAGE_BYTES);
+  uint64_t* full = bars;                   // [P_STAGES] (the leader's counts both CTAs' loads)
+  uint64_t* empty = bars + P_STAGES;       // [P_STAGES]
+  uint64_t* tfull = bars + 2 * P_STAGES;   // [2]
+  uint64_t* tempty = tfull + 2;            // [2] (the leader's: 16 warp arrivals)
+  uint64_t* drain = tempty + 2;            // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(&tfull[a], 1);
+      ptx::mbar_init(&tempty[a], 16);
+    }
+    ptx::mbar_init(drain, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    ptx::tmem_relinquish_pair();
+  }
+  ptx::tc_fence_before();
+  ptx::cluster_sync();  // barriers and TMEM of both CTAs exist before any cross-CTA use
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer (both CTAs)
+      ptx::prefetch_tmap(&mapA);
+      ptx::prefetch_tmap(&mapB);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = pair; u < args.units && ok; u += npairs) {
+        int I2, J;
+        decode_tile_pair(u % args.ntiles, I2, J);
+        const int kb0 = (u / args.ntiles) * args.kb_per_unit;
+        const int kb1 = min(kb0 + args.kb_per_unit, args.nkb);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, WAIT_LIMIT_NS)) {
+            ok = false;
+            break;
+          }
+          if (leader) ptx::mbar_arrive_expect_tx(&full[stage], 2 * P_STAGE_BYTES);
+          const uint32_t fb = ptx::mapa_shared(&full[stage], 0);
+          ptx::tma_load_2d_pair(sA + stage * P_A_BYTES, &mapA, fb, kb * BK,
+                                I2 * 256 + (int)rank * 128);
+          ptx::tma_load_2d_pair(sB + stage * P_B_BYTES, &mapB, fb, kb * BK,
+                                J * 256 + (int)rank * 128);
+          if (++stage == P_STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok || *abort_flag) {
+        raise_abort(abort_flag, args.info);
+      } else {
+        // tail: every stage is released once more, so the MMA commits'
+        // arrivals on this CTA's `empty` barriers have all landed
+        for (int i = 0; i < P_STAGES; ++i) {
+          if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
+          if (++stage == P_STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------ MMA issuer (leader only)
+      constexpr uint32_t idesc = ptx::idesc_bf16_f32(256, 256);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t aphase = 0;
+      bool ok = true;
+      for (int u = pair; u < args.units && ok; u += npairs) {
+        const int kb0 = (u / args.ntiles) * args.kb_per_unit;
+        const int kb1 = min(kb0 + args.kb_per_unit, args.nkb);
+        for (int p0 = kb0; p0 < kb1 && ok; p0 += kSubKb) {
+          const int p1 = min(p0 + kSubKb, kb1);
+          if (!ptx::mbar_wait_bounded(&tempty[acc], aphase ^ 1, abort_flag, WAIT_LIMIT_NS)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+          for (int kb = p0; kb < p1; ++kb) {
+            if (!ptx::mbar_wait_bounded(&full[stage], phase, abort_flag, WAIT_LIMIT_NS)) {
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
+            const uint64_t adesc = ptx::smem_desc_sw128(ptx::smem_u32(sA + stage * P_A_BYTES));
+            const uint64_t bdesc = ptx::smem_desc_sw128(ptx::smem_u32(sB + stage * P_B_BYTES));
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k)
+              ptx::mma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc,
+                                 (kb > p0 || k > 0) ? 1u : 0u);
+            ptx::mma_commit_pair(&empty[stage], 0x3);
+            if (++stage == P_STAGES) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+          if (!ok) break;
+          ptx::mma_commit_pair(&tfull[acc], 0x3);
+          acc ^= 1;
+          if (acc == 0) aphase ^= 1;
+        }
+      }
+      if (!ok || *abort_flag) raise_abort(abort_flag, args.info);
+      // every MMA issued above is complete before tear-down (bounded)
+      ptx::mma_commit_pair(drain, 0x1);
+      volatile int never = 0;
+      ptx::mbar_wait_bounded(drain, 0, &never, WAIT_LIMIT_NS);
+    }
+  } else {
+    // -------------------------------------------------- epilogue (warps 2..9, both CTAs)
+    const int q = warp & 3;              // TMEM lanes [32q, 32q + 32): rows of this CTA's half
+    const int half = (warp - 2) >> 2;    // accumulator columns [128 half, +128)
+    const uint32_t tempty_leader0 = ptx::mapa_shared(&tempty[0], 0);
+    const uint32_t tempty_leader1 = ptx::mapa_shared(&tempty[1], 0);
+    int acc = 0;
+    uint32_t aphase = 0;
+    const int n = args.n;
+    bool stop = false;
+    for (int u = pair; u < args.units && !stop; u += npairs) {
+      int I2, J;
+      decode_tile_pair(u % args.ntiles, I2, J);
+      const int kb0 = (u / args.ntiles) * args.kb_per_unit;
+      const int kb1 = min(kb0 + args.kb_per_unit, args.nkb);
+      const int row_lo = I2 * 256 + (int)rank * 128 + q * 32;
+      const int row = row_lo + lane;
+      const int cbase = J * 256 + half * 128;
+      float tile[128];
+#pragma unroll
+      for (int j = 0; j < 128; ++j) tile[j] = 0.f;
+      for (int p0 = kb0; p0 < kb1; p0 += kSubKb) {
+        if (!ptx::mbar_wait_bounded(&tfull[acc], aphase, abort_flag, WAIT_LIMIT_NS)) {
+          raise_abort(abort_flag, args.info);
+          stop = true;
+          break;
+        }
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const int col0 = cbase + ch * 32;
+          // warp-uniform: pieces past n or wholly below the diagonal are not needed
+          if (col0 < n && col0 + 31 >= row_lo) {
+            uint32_t v[32];
+            ptx::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) +
+                                        (uint32_t)(acc * BN + half * 128 + ch * 32),
+                                    v);
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) tile[ch * 32 + j] += __uint_as_float(v[j]);
+          }
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+        acc ^= 1;
+        if (acc == 0) aphase ^= 1;
+      }
+      if (stop) break;
+      if (row < n) {
+        float* hrow = args.H + (int64_t)row * n;
+#pragma unroll
+        for (int j4 = 0; j4 < 32; ++j4) {
+          const int c = cbase + 4 * j4;
+          if (c + 3 < row || c >= n) continue;
+          const float f0 = args.alpha * tile[4 * j4 + 0];
+          const float f1 = args.alpha * tile[4 * j4 + 1];
+          const float f2 = args.alpha * tile[4 * j4 + 2];
+          const float f3 = args.alpha * tile[4 * j4 + 3];
+          if (args.vec4 && c >= row && c + 3 < n) {
+            atomicAdd(reinterpret_cast<float4*>(hrow + c), make_float4(f0, f1, f2, f3));
+          } else {
+            if (c + 0 >= row && c + 0 < n) atomicAdd(hrow + c + 0, f0);
+            if (c + 1 >= row && c + 1 < n) atomicAdd(hrow + c + 1, f1);
+            if (c + 2 >= row && c + 2 < n) atomicAdd(hrow + c + 2, f2);
+            if (c + 3 >= row && c + 3 < n) atomicAdd(hrow + c + 3, f3);
+          }
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  ptx::cluster_sync();  // both CTAs done with every load, MMA and TMEM read
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
 // hi = bf16(x) (round to nearest even), lo = bf16(x - hi)
 __global__ void split_bf16_kernel(const float* __restrict__ X, int64_t n, int64_t ntok,
                                   int64_t ldx, __nv_bfloat16* __restrict__ hi,
@@ -331,9 +591,85 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t ntok, in
 
 }  // namespace
 
+namespace {
+
+// Fewest token chunks that fill `slots` parallel workers' waves to >= 97 %
+// (at least 8 k-blocks per unit), else the best fill found.
+int choose_chunks(int ntiles, int nkb, int slots) {
+  int best_kc = 1;
+  double best_eff = -1.0;
+  const int max_kc = std::max(1, std::min(nkb / 8, 512));
+  for (int kc = 1; kc <= max_kc; ++kc) {
+    const long units = (long)ntiles * kc;
+    const long waves = (units + slots - 1) / slots;
+    const double eff = (double)units / (double)(waves * slots);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best_kc = kc;
+    }
+    if (eff >= 0.97) break;
+  }
+  return best_kc;
+}
+
+// Concurrent CTA pairs the pair kernel can have (0 if it cannot launch).
+int pair_slots() {
+  static int cached = -1;
+  if (cached >= 0) return cached;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * 74, 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = P_SMEM_BYTES;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaFuncSetAttribute(syrk_bf16_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)P_SMEM_BYTES) != cudaSuccess ||
+      cudaOccupancyMaxActiveClusters(&clusters, syrk_bf16_pair_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    clusters = 0;
+  }
+  cached = clusters;
+  return cached;
+}
+
+}  // namespace
+
 cudaError_t launch_syrk_bf16(float* H, int64_t n, const void* A, const void* B, int64_t ntok,
                              int64_t ld, float alpha, int32_t* info, cudaStream_t s) {
   if (n <= 0 || ntok <= 0) return cudaSuccess;
+  const int sms = num_sms();
+  const int nkb = (int)((ntok + BK - 1) / BK);
+  const int vec4 = ((n % 4) == 0 && (reinterpret_cast<uintptr_t>(H) % 16) == 0) ? 1 : 0;
+  cudaError_t e;
+  // CTA pairs for layers of at least 256 inputs, when the device can co-schedule them
+  const int slots = n >= 256 ? pair_slots() : 0;
+  if (slots > 0) {
+    CUtensorMap mapA, mapB;
+    if (!make_map(&mapA, A, n, ntok, ld, 128) || !make_map(&mapB, B, n, ntok, ld, 128))
+      return cudaErrorInvalidValue;
+    SyrkPairArgs a;
+    a.H = H;
+    a.n = (int)n;
+    a.alpha = alpha;
+    a.nkb = nkb;
+    const int nJ = (int)((n + 255) / 256);
+    a.ntiles = nJ * (nJ + 1) / 2;
+    const int kc = choose_chunks(a.ntiles, nkb, slots);
+    a.kb_per_unit = (nkb + kc - 1) / kc;
+    a.units = a.ntiles * ((nkb + a.kb_per_unit - 1) / a.kb_per_unit);
+    a.vec4 = vec4;
+    a.info = info;
+    const int pairs = std::min(slots, a.units);
+    syrk_bf16_pair_kernel<<<2 * pairs, NUM_THREADS, P_SMEM_BYTES, s>>>(mapA, mapB, a);
+    note_launch();
+    return cudaGetLastError();
+  }
   CUtensorMap mapA, mapB;
   if (!make_map(&mapA, A, n, ntok, ld, BM) || !make_map(&mapB, B, n, ntok, ld, BN))
     return cudaErrorInvalidValue;
@@ -341,36 +677,20 @@ cudaError_t launch_syrk_bf16(float* H, int64_t n, const void* A, const void* B, 
   a.H = H;
   a.n = (int)n;
   a.alpha = alpha;
-  a.nkb = (int)((ntok + BK - 1) / BK);
+  a.nkb = nkb;
   a.nI = (int)((n + BM - 1) / BM);
   const int nJ = (int)((n + BN - 1) / BN);
   a.ntiles = 0;
   for (int J = 0; J < nJ; ++J) a.ntiles += std::min(a.nI, 2 * J + 2);
-  const int sms = num_sms();
-  // token chunks: the fewest that fill the SMs' waves to >= 97 %, at least 8
-  // k-blocks per unit; else the best fill found.
-  int best_kc = 1;
-  double best_eff = -1.0;
-  const int max_kc = std::max(1, std::min(a.nkb / 8, 512));
-  for (int kc = 1; kc <= max_kc; ++kc) {
-    const long units = (long)a.ntiles * kc;
-    const long waves = (units + sms - 1) / sms;
-    const double eff = (double)units / (double)(waves * sms);
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
-      best_kc = kc;
-    }
-    if (eff >= 0.97) break;
-  }
+  const int best_kc = choose_chunks(a.ntiles, nkb, sms);
   a.kb_per_unit = (a.nkb + best_kc - 1) / best_kc;
   const int kchunks = (a.nkb + a.kb_per_unit - 1) / a.kb_per_unit;
   a.units = a.ntiles * kchunks;
-  a.vec4 = ((n % 4) == 0 && (reinterpret_cast<uintptr_t>(H) % 16) == 0) ? 1 : 0;
+  a.vec4 = vec4;
   a.info = info;
-  cudaError_t e = cudaFuncSetAttribute(syrk_bf16_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)SMEM_BYTES);
-  if (e != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(syrk_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)SMEM_BYTES)) != cudaSuccess)
+    return e;
   const int grid = std::min(sms, a.units);
   syrk_bf16_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(mapA, mapB, a);
   note_launch();
