@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <mutex>
 #include <cstdint>
 
 #include "gptq_internal.cuh"
@@ -52,6 +53,31 @@ bool make_tma_2d(CUtensorMap* map, const void* base, bool bf16, int64_t rows, in
 }
 
 static std::atomic<long long> g_launches{0};
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_side_mu;
+SideStream g_side[kMaxDevices];
+bool g_side_ok[kMaxDevices] = {};
+}  // namespace
+
+std::mutex& side_lock() { return g_side_mu; }
+
+bool side_stream(SideStream* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  if (!g_side_ok[dev]) {
+    SideStream ss{};
+    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess) return false;
+    for (auto& e : ss.ev)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return false;
+    g_side[dev] = ss;
+    g_side_ok[dev] = true;
+  }
+  *out = g_side[dev];
+  return true;
+}
 
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 

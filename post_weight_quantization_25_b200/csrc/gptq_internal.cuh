@@ -3,6 +3,7 @@
 // the launch (cudaSuccess when nothing had to run).
 #pragma once
 #include <cstdint>
+#include <mutex>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -21,6 +22,18 @@ bool make_tma_2d(CUtensorMap* map, const void* base, bool bf16, int64_t rows, in
                  int64_t ld, uint32_t box_cols, uint32_t box_rows);
 // Counts one kernel enqueued by this library (read by gptq_launch_count).
 void note_launch();
+
+// A second stream on the current device for work that overlaps the
+// caller's stream, and two events to order the two; created on first use
+// per device and kept until the process exits.  A launcher that forks onto
+// it holds side_lock() for its whole enqueue sequence and joins back onto
+// the caller's stream before returning.  Returns false if it cannot be had.
+struct SideStream {
+  cudaStream_t s;
+  cudaEvent_t ev[2];
+};
+bool side_stream(SideStream* out);
+std::mutex& side_lock();
 
 // ---- Hessian (hessian_syrk.cu)
 // H(upper incl. diagonal) += alpha * A_rows * B_rows^T over tokens [0, ntok),

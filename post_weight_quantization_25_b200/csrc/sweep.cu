@@ -40,8 +40,8 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct SweepWs {
   float* Wf;          // rows x n, sweep order; after the sweep holds w_hat
-  float* Err_hi;      // rows x 128: the block's err terms, TF32 part
-  float* Err_lo;      // rows x 128: remainder (err - Err_hi)
+  float* Err_hi[2];   // rows x 128: a block's err terms, TF32 part (blocks alternate)
+  float* Err_lo[2];   // rows x 128: remainder (err - Err_hi)
   uint8_t* codes_sw;  // rows x n, sweep order
   int32_t* pos;       // n: sweep position of each original column
   float* UT_hi;       // n x ldut: U^T, TF32 part (the lazy update's K-major operand)
@@ -56,10 +56,12 @@ SweepWs carve(void* ws, int64_t rows, int64_t n) {
   SweepWs w;
   w.Wf = reinterpret_cast<float*>(p);
   p += align_up(sizeof(float) * rows * n, 256);
-  w.Err_hi = reinterpret_cast<float*>(p);
-  p += align_up(sizeof(float) * rows * kBlock, 256);
-  w.Err_lo = reinterpret_cast<float*>(p);
-  p += align_up(sizeof(float) * rows * kBlock, 256);
+  for (int b = 0; b < 2; ++b) {
+    w.Err_hi[b] = reinterpret_cast<float*>(p);
+    p += align_up(sizeof(float) * rows * kBlock, 256);
+    w.Err_lo[b] = reinterpret_cast<float*>(p);
+    p += align_up(sizeof(float) * rows * kBlock, 256);
+  }
   w.codes_sw = reinterpret_cast<uint8_t*>(p);
   p += align_up((size_t)rows * n, 256);
   w.pos = reinterpret_cast<int32_t*>(p);
@@ -94,30 +96,30 @@ __global__ void __launch_bounds__(256) ut_split_kernel(const float* __restrict__
   }
 }
 
-// The lazy update  Wf[:, i2:] -= Err U[i1:i1+128, i2:]  as tiles for the
-// tensor-core panel GEMM: P = Err (rows x 128), Q = U^T rows i2.. (columns
-// i1..i1+128), C = Wf.
-// Item i = rows [128 i, 128 i + 128) of Wf, with its P block (the err terms)
-// kept resident while the tiles of columns i2, i2 + 128, ... stream by.
+// The lazy update  Wf[:, c0:c1] -= Err U[i1:i1+128, c0:c1]  as items for the
+// tensor-core panel GEMM: P = Err (rows x 128), Q = U^T rows c0.. (columns
+// i1..i1+128), C = Wf.  Item i = rows [128 i, 128 i + 128) of Wf, with its P
+// block (the err terms) kept resident while the tiles of columns c0,
+// c0 + 128, ... stream by.
 struct SweepTrailItems {
   float* Wf;
-  int rows, n, i1, i2;
+  int rows, n, i1, c0, c1;
   __host__ __device__ int num_items() const { return (rows + 127) / 128; }
-  __host__ __device__ int item_nq(int) const { return (n - i2 + 127) / 128; }
+  __host__ __device__ int item_nq(int) const { return (c1 - c0 + 127) / 128; }
   __device__ PgItem item(int i) const {
     PgItem I;
-    I.C0 = Wf + (int64_t)i * 128 * n + i2;
+    I.C0 = Wf + (int64_t)i * 128 * n + c0;
     I.ldc = n;
     I.cmap = 0;
-    I.cx0 = i2;
+    I.cx0 = c0;
     I.cy0 = 128 * i;
     I.prow = 128 * i;
     I.pkx = 0;
-    I.qrow0 = i2;
+    I.qrow0 = c0;
     I.qkx = i1;
     I.nq = item_nq(i);
     I.mext = min(128, rows - 128 * i);
-    I.cext_last = n - i2 - 128 * (I.nq - 1);
+    I.cext_last = c1 - c0 - 128 * (I.nq - 1);
     return I;
   }
 };
@@ -430,7 +432,7 @@ cudaError_t launch_selftest_division(const float* a, const float* b, int64_t cou
 
 size_t quantize_workspace_bytes(int64_t rows, int64_t n) {
   return align_up(sizeof(float) * rows * n, 256) +
-         2 * align_up(sizeof(float) * rows * kBlock, 256) + align_up((size_t)rows * n, 256) +
+         4 * align_up(sizeof(float) * rows * kBlock, 256) + align_up((size_t)rows * n, 256) +
          align_up(sizeof(int32_t) * n, 256) + 2 * align_up(sizeof(float) * n * ut_ld(n), 256);
 }
 
@@ -474,15 +476,17 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
 
   // operands of the lazy update on the tensor cores; with a row stride that
   // is a multiple of 16 bytes the update lands in Wf by TMA reduce-add
-  CUtensorMap mEh, mEl, mUh, mUl, mW;
+  CUtensorMap mEh[2], mEl[2], mUh, mUl, mW;
   const bool reduce = (n % 4) == 0;
   if (n > kBlock) {
     ut_split_kernel<<<dim3((unsigned)((w.ldut + 31) / 32), (unsigned)((n + 31) / 32)), 256, 0, s>>>(
         U, n, w.ldut, w.UT_hi, w.UT_lo);
     note_launch();
-    if (!make_tma_2d(&mEh, w.Err_hi, false, rows, kBlock, kBlock, 32, 128) ||
-        !make_tma_2d(&mEl, w.Err_lo, false, rows, kBlock, kBlock, 32, 128) ||
-        !make_tma_2d(&mUh, w.UT_hi, false, n, n, w.ldut, 32, 128) ||
+    for (int b = 0; b < 2; ++b)
+      if (!make_tma_2d(&mEh[b], w.Err_hi[b], false, rows, kBlock, kBlock, 32, 128) ||
+          !make_tma_2d(&mEl[b], w.Err_lo[b], false, rows, kBlock, kBlock, 32, 128))
+        return cudaErrorInvalidValue;
+    if (!make_tma_2d(&mUh, w.UT_hi, false, n, n, w.ldut, 32, 128) ||
         !make_tma_2d(&mUl, w.UT_lo, false, n, n, w.ldut, 32, 128))
       return cudaErrorInvalidValue;
     if (reduce) {
@@ -492,20 +496,56 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
                                     (int)pg2_smem_bytes(true))) != cudaSuccess)
         return e;
     } else {
-      mW = mEh;  // not read by the read-modify-write epilogue
+      mW = mUh;  // not read by the read-modify-write epilogue
       if ((e = cudaFuncSetAttribute(panel_gemm2_kernel<SweepTrailItems, false>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)pg2_smem_bytes(false))) != cudaSuccess)
         return e;
     }
   }
-  for (int i1 = 0; i1 < n; i1 += kBlock) {
+  auto trail = [&](int blk, int i1, int c0, int c1, int max_grid, cudaStream_t st) {
+    const SweepTrailItems dec{w.Wf, rows, n, i1, c0, c1};
+    int chunk = 1, units = 0;
+    pg2_plan(dec, max_grid, chunk, units);
+    const int grid = std::min(units, max_grid);
+    const int eb = blk & 1;
+    if (reduce)
+      panel_gemm2_kernel<SweepTrailItems, true><<<grid, kPg2Threads, pg2_smem_bytes(true), st>>>(
+          mEh[eb], mEl[eb], mUh, mUl, mW, mW, dec, chunk, units, nullptr, 0, nullptr);
+    else
+      panel_gemm2_kernel<SweepTrailItems, false><<<grid, kPg2Threads, pg2_smem_bytes(false), st>>>(
+          mEh[eb], mEl[eb], mUh, mUl, mW, mW, dec, chunk, units, nullptr, 0, nullptr);
+    note_launch();
+  };
+
+  // Look-ahead.  After block b is swept, only block b+1's columns are
+  // updated on the caller's stream (the "near" update, which the next sweep
+  // waits for); the update of every later column ("far") runs on the side
+  // stream, on part of the SMs, while block b+1 is swept.  Each column block
+  // still receives its updates in block order -- far(0), ..., far(c-2),
+  // near(c-1) for block c -- because near(b) waits for far(b-1); the err
+  // terms alternate between two buffers, and sweep(b+2) (after near(b+1),
+  // after far(b)) is the next writer of far(b)'s buffer.
+  SideStream side{};
+  const bool lookahead = n > 2 * kBlock && side_stream(&side);
+  std::unique_lock<std::mutex> side_guard(side_lock(), std::defer_lock);
+  // SMs left to the far update: the sweep's CTAs (up to two per SM) keep the rest
+  const int far_grid = std::max(sms / 4, sms - (sweep_ctas + 1) / 2);
+  if (lookahead) {
+    side_guard.lock();
+    if ((e = cudaEventRecord(side.ev[0], s)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(side.s, side.ev[0], 0)) != cudaSuccess)
+      return e;
+  }
+  bool far_pending = false;  // far(b-1) was issued and near(b) must wait for it
+  for (int i1 = 0, blk = 0; i1 < n; i1 += kBlock, ++blk) {
     const int bsz = std::min(kBlock, n - i1);
     const int i2 = i1 + bsz;
+    const int eb = blk & 1;
 #define GPTQ_SWEEP_LAUNCH(GSV)                                                                 \
   sweep_block_kernel<GSV><<<sweep_ctas, kSweepThreads, us_smem, s>>>(                          \
-      w.Wf, rows, n, U, i1, bsz, maxq, group_size, G, w.Err_hi, w.Err_lo, w.codes_sw, scales,  \
-      zeros, row_loss)
+      w.Wf, rows, n, U, i1, bsz, maxq, group_size, G, w.Err_hi[eb], w.Err_lo[eb], w.codes_sw,  \
+      scales, zeros, row_loss)
     if (gmode == 0)
       GPTQ_SWEEP_LAUNCH(0);
     else if (gmode == 1)
@@ -516,19 +556,32 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
       GPTQ_SWEEP_LAUNCH(64);
 #undef GPTQ_SWEEP_LAUNCH
     note_launch();
-    if (i2 < n) {  // bsz == 128 here: only the last block is short
-      const SweepTrailItems dec{w.Wf, rows, n, i1, i2};
-      int chunk = 1, units = 0;
-      pg2_plan(dec, sms, chunk, units);
-      const int grid = std::min(units, sms);
-      if (reduce)
-        panel_gemm2_kernel<SweepTrailItems, true><<<grid, kPg2Threads, pg2_smem_bytes(true), s>>>(
-            mEh, mEl, mUh, mUl, mW, mW, dec, chunk, units, nullptr, 0, nullptr);
-      else
-        panel_gemm2_kernel<SweepTrailItems, false><<<grid, kPg2Threads, pg2_smem_bytes(false), s>>>(
-            mEh, mEl, mUh, mUl, mW, mW, dec, chunk, units, nullptr, 0, nullptr);
-      note_launch();
+    if (i2 >= n) break;  // bsz == 128 below: only the last block is short
+    if (!lookahead) {
+      trail(blk, i1, i2, n, sms, s);
+      continue;
     }
+    const int near_end = std::min(i2 + kBlock, n);
+    if (near_end < n) {
+      // far(b) needs block b's err terms: fork after the sweep
+      if ((e = cudaEventRecord(side.ev[0], s)) != cudaSuccess ||
+          (e = cudaStreamWaitEvent(side.s, side.ev[0], 0)) != cudaSuccess)
+        return e;
+    }
+    if (far_pending && (e = cudaStreamWaitEvent(s, side.ev[1], 0)) != cudaSuccess) return e;
+    trail(blk, i1, i2, near_end, sms, s);
+    far_pending = false;
+    if (near_end < n) {
+      trail(blk, i1, near_end, n, far_grid, side.s);
+      if ((e = cudaEventRecord(side.ev[1], side.s)) != cudaSuccess) return e;
+      far_pending = true;
+    }
+  }
+  if (lookahead) {  // join: everything on the side stream precedes what follows on s
+    if ((e = cudaEventRecord(side.ev[1], side.s)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(s, side.ev[1], 0)) != cudaSuccess)
+      return e;
+    side_guard.unlock();
   }
   const size_t un_smem = (Wq ? sizeof(float) * (size_t)n : 0) + (size_t)n;
   if ((e = set_smem(unpermute_kernel, un_smem)) != cudaSuccess) return e;
