@@ -59,7 +59,10 @@ typedef enum { GPTQ_BF16 = 0, GPTQ_F32 = 1 } gptq_dtype;
  *   percdamp    damping as a fraction of mean(diag H); 0.01 in the pages.
  *   block       lazy-update block; must be 128.
  *   actorder    nonzero: sweep columns in order of descending diag(H).
- *   sym         must be 0 (asymmetric ruler). */
+ *   sym         0: asymmetric min-max ruler (the default in the pages);
+ *               1: the opt-in symmetric ruler -- range [-m, m] with
+ *               m = max(|min|, |max|), scale = 2m / (2^b - 1), zero point on
+ *               the middle tick 2^(b-1).  Any other value: invalid. */
 typedef struct {
   int bits;
   int group_size;

@@ -97,19 +97,31 @@ def hessian_entry(X: np.ndarray, i: int, j: int, alpha: float = 2.0) -> float:
 # The ruler  (§ "What quantization is, and why anyone bothers"; § "Paper vs.
 # code": asymmetric min-max, range stretched to include zero)
 # --------------------------------------------------------------------------
-def fit_grid(wmin, wmax, bits: int):
+def fit_grid(wmin, wmax, bits: int, sym: bool = False):
     """Ruler for values spanning [wmin, wmax]; arrays broadcast.
 
     Returns ``(scale, zero)``: scale as binary32, zero as int64.  The range is
     first stretched to include 0.  The decisions are binary32 (module notes).
+
+    ``sym``: the opt-in symmetric ruler (page "GPTQ, with the code open",
+    § "Paper vs. code").  The pages give no formula; the reading taken is the
+    plainest one: the range becomes [-m, m] with m = max(|min|, |max|), the
+    same scale formula applies, and the zero point is the middle tick
+    (2^b - 1 + 1) / 2, a whole tick, so 0.0 stays exactly representable.
     """
     maxq = F32(2 ** bits - 1)
     xmin = np.minimum(np.asarray(wmin, dtype=np.float64), 0.0).astype(F32)
     xmax = np.maximum(np.asarray(wmax, dtype=np.float64), 0.0).astype(F32)
+    if sym:
+        m = np.maximum(-xmin, xmax).astype(F32)
+        xmin, xmax = (-m).astype(F32), m
     flat = (xmin == 0) & (xmax == 0)
     xmin = np.where(flat, F32(-1), xmin).astype(F32)
     xmax = np.where(flat, F32(1), xmax).astype(F32)
     scale = ((xmax - xmin).astype(F32) / maxq).astype(F32)
+    if sym:
+        zero = np.full(np.shape(scale), (2 ** bits) // 2, dtype=np.int64)
+        return scale, zero
     zero_pre = ((-xmin).astype(F32) / scale).astype(F32)
     zero = np.rint(zero_pre).astype(np.int64)
     return scale, zero
@@ -240,7 +252,7 @@ def _half_distance(t) -> float:
 
 def sweep(Wp: np.ndarray, U: np.ndarray, bits: int, group_size: int = -1,
           forced_codes=None, forced_zeros=None, tau: float = 1e-3, trace=None,
-          adoptions=None):
+          adoptions=None, sym: bool = False):
     """Unblocked GPTQ sweep over the columns of Wp (already in sweep order).
 
     For each column j, left to right, for every row at once:
@@ -282,8 +294,8 @@ def sweep(Wp: np.ndarray, U: np.ndarray, bits: int, group_size: int = -1,
     for j in range(n):
         if j % g == 0:
             blk = W[:, j:j + g]
-            scale, zero = fit_grid(blk.min(axis=1), blk.max(axis=1), bits)
-            if forced_zeros is not None:
+            scale, zero = fit_grid(blk.min(axis=1), blk.max(axis=1), bits, sym)
+            if forced_zeros is not None and not sym:
                 fz = np.asarray(forced_zeros)[:, j // g].astype(np.int64)
                 diff = fz != zero
                 zp = zero_prevalue(blk.min(axis=1), bits, scale)
@@ -325,7 +337,8 @@ def sweep(Wp: np.ndarray, U: np.ndarray, bits: int, group_size: int = -1,
             "loss": loss, "adopted": adopted, "mismatched": mismatched}
 
 
-def sweep_blocked(Wp: np.ndarray, U: np.ndarray, bits: int, group_size: int, block: int):
+def sweep_blocked(Wp: np.ndarray, U: np.ndarray, bits: int, group_size: int, block: int,
+                  sym: bool = False):
     """The lazy-batch form (§ "From one repair to a whole model"): repairs
     inside the current block of ``block`` columns at once, the repair of every
     later column deferred to one product per block.  Used only to show that
@@ -354,7 +367,7 @@ def sweep_blocked(Wp: np.ndarray, U: np.ndarray, bits: int, group_size: int, blo
                 # (jj == 0): no repair of this block has run yet, and the
                 # columns past the block hold every earlier block's repair
                 grp = np.concatenate([Wb[:, jj:], W[:, i2:j + g]], axis=1)[:, :g]
-                scale, zero = fit_grid(grp.min(axis=1), grp.max(axis=1), bits)
+                scale, zero = fit_grid(grp.min(axis=1), grp.max(axis=1), bits, sym)
                 scales[:, j // g] = scale
                 zeros[:, j // g] = zero
             w = Wb[:, jj]
@@ -373,7 +386,7 @@ def sweep_blocked(Wp: np.ndarray, U: np.ndarray, bits: int, group_size: int, blo
     return {"codes": codes, "scales": scales, "zeros": zeros, "Wq": Wq, "loss": loss}
 
 
-def rtn(Wp: np.ndarray, bits: int, group_size: int = -1):
+def rtn(Wp: np.ndarray, bits: int, group_size: int = -1, sym: bool = False):
     """Round-to-nearest on the same ruler, no repair (§ "The obvious approach,
     and how it fails").  Groups are consecutive columns of Wp's order."""
     W = np.asarray(Wp, dtype=np.float64)
@@ -385,7 +398,7 @@ def rtn(Wp: np.ndarray, bits: int, group_size: int = -1):
     zeros = np.zeros((rows, G), dtype=np.int64)
     for k in range(G):
         blk = W[:, k * g:(k + 1) * g]
-        s, z = fit_grid(blk.min(axis=1), blk.max(axis=1), bits)
+        s, z = fit_grid(blk.min(axis=1), blk.max(axis=1), bits, sym)
         scales[:, k], zeros[:, k] = s, z
         codes[:, k * g:(k + 1) * g] = quantize(blk, s[:, None], z[:, None], bits)
     return {"codes": codes, "scales": scales, "zeros": zeros}
@@ -397,18 +410,18 @@ def rtn(Wp: np.ndarray, bits: int, group_size: int = -1):
 def gptq_layer(W: np.ndarray, H: np.ndarray, bits: int = 4, group_size: int = -1,
                percdamp: float = 0.01, actorder: bool = False,
                forced_codes=None, forced_zeros=None, tau: float = 1e-3,
-               forced_perm=None, perm_rtol: float = 1e-5):
+               forced_perm=None, perm_rtol: float = 1e-5, sym: bool = False):
     """GPTQ on one linear layer, given its Hessian H (n x n) and weights W.
 
     Returns the sweep's dict plus, in ORIGINAL column order: ``codes_orig``,
     ``Wq_orig`` and ``g_idx`` (group of each original column), and the
     preparation's ``dead``, ``perm``, ``lam``, ``U``, ``W0``.  Forced
     codes/zeros are given in sweep order (see ``sweep``); ``forced_perm`` as
-    in ``prepare``.
+    in ``prepare``; ``sym`` selects the symmetric ruler (``fit_grid``).
     """
     prep = prepare(H, W, percdamp, actorder, forced_perm, perm_rtol)
     U = upper_cholesky_of_inverse(prep["Hp"])
-    res = sweep(prep["Wp"], U, bits, group_size, forced_codes, forced_zeros, tau)
+    res = sweep(prep["Wp"], U, bits, group_size, forced_codes, forced_zeros, tau, sym=sym)
     perm = prep["perm"]
     n = perm.shape[0]
     g = group_size if group_size > 0 else n

@@ -243,7 +243,8 @@ class QuantizedLinear:
 def quantize_linear(W: torch.Tensor, X=None, H: torch.Tensor | None = None, bits: int = 4,
                     group_size: int = 128, percdamp: float = 0.01, actorder: bool = False,
                     alpha: float = 2.0, want_wq: bool = False, want_loss: bool = False,
-                    keep_factors: bool = False, stream=None) -> QuantizedLinear:
+                    keep_factors: bool = False, sym: bool = False,
+                    stream=None) -> QuantizedLinear:
     """GPTQ for one linear layer W (rows x n).  X: one calibration tensor
     (n x N) or an iterable of batches; or pass a ready Hessian H."""
     _need_cuda(W)
@@ -255,7 +256,7 @@ def quantize_linear(W: torch.Tensor, X=None, H: torch.Tensor | None = None, bits
         batches = [X] if isinstance(X, torch.Tensor) else X
         for xb in batches:
             gptq_hessian_accumulate(H, xb, alpha, stream=stream)
-    cfg = make_config(bits, group_size, percdamp, actorder)
+    cfg = make_config(bits, group_size, percdamp, actorder, sym=sym)
     U, perm, dead, info = gptq_cholesky_inverse(H, percdamp, actorder, stream=stream)
     q = gptq_quantize_layer(W, U, perm, dead, cfg, want_wq=want_wq, want_loss=want_loss,
                             stream=stream)
@@ -288,7 +289,7 @@ class LayerQuantizer:
                  percdamp: float = 0.01, actorder: bool = False,
                  x_dtype: torch.dtype = torch.bfloat16, w_dtype: torch.dtype = torch.bfloat16,
                  out_dtype: torch.dtype = torch.bfloat16, want_wq: bool = False,
-                 want_loss: bool = False, device=None):
+                 want_loss: bool = False, sym: bool = False, device=None):
         if bits == 4 and n % 8:
             raise GptqError("int4 packing needs n % 8 == 0")
         if bits == 3 and n % 32:
@@ -298,7 +299,7 @@ class LayerQuantizer:
         dev = torch.device("cuda") if device is None else torch.device(device)
         self.rows, self.n, self.ntok, self.bits = rows, n, ntok, bits
         self.group_size, self.percdamp, self.actorder = group_size, percdamp, actorder
-        self.cfg = make_config(bits, group_size, percdamp, actorder)
+        self.cfg = make_config(bits, group_size, percdamp, actorder, sym=sym)
         G = 1 if group_size <= 0 else (n + group_size - 1) // group_size
         f32 = torch.float32
         self.H = torch.empty(n, n, dtype=f32, device=dev)

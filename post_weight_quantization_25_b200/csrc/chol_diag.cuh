@@ -10,8 +10,9 @@
 //
 // The diagonal block sits in shared memory and is worked in 32 x 32 leaves.
 // For leaf j one warp factors the leaf in registers (right-looking, unscaled
-// LDL^T steps; each step's column is published once in shared memory and
-// read back with 16-byte broadcast loads; square roots at the end), the rows
+// LDL^T, four columns per step: each lane runs the 4 x 4 block's recurrence
+// itself, rows exchange 16-byte values through shared memory; square roots
+// at the end), the rows
 // below it are solved against the leaf by substitution (one thread per row),
 // and the remaining lower block takes the rank-32 update from a transposed
 // copy of the solved rows (16-byte loads, 8 x 4 register tiles).  At the end
@@ -28,55 +29,96 @@ constexpr int kDiagThreads = 256;
 constexpr int kDP = 129;   // row pitch (floats) of the block S
 constexpr int kXP = 132;   // row pitch of XT (transposed solved rows)
 constexpr int kTP = 36;    // row pitch of a transposed 32 x 32 leaf
-// S[128][kDP] | XT[32][kXP] | LTl[32][kTP] | rinv[128] | colb[2][32]
+// S[128][kDP] | XT[32][kXP] | LTl[32][kTP] | rinv[128] | yb[32], zb[32] (float4)
 constexpr size_t kDiagSmemBytes =
-    sizeof(float) * (128 * kDP + 32 * kXP + 32 * kTP + 128 + 64) + 16;
+    sizeof(float) * (128 * kDP + 32 * kXP + 32 * kTP + 128 + 256) + 16;
 
 // Outputs of chol_diag_kernel, in the Cholesky workspace:
 //   Lt[k][c]     = L[c][k]           (128 x 128, zero for k > c)
 //   LiT[j][t][c] = (L_jj^-1)[c][t]   (4 leaves of 32 x 32, zero for t > c)
 constexpr int kDiagOutFloats = 128 * 128 + 4 * 32 * 32;
 
+// 1/d: hardware estimate and one Newton step (a multiplier needs no more)
+__device__ __forceinline__ float recip_nr(float d) {
+  const float r0 = ptx::rcp_approx(d);
+  return fmaf(fmaf(-d, r0, 1.f), r0, r0);
+}
+
 // One warp: factor the 32 x 32 leaf at (c0, c0) of S in place (lower part);
 // writes 1 / L_kk to rinv[c0 + k] and the leaf transposed to LTl[t][m] =
 // L[c0+m][c0+t].  Returns (warp-uniform) the 1-based index of the first
 // non-positive or non-finite pivot within the leaf, or 0.
-__device__ __forceinline__ int leaf_factor(float* S, float* rinv, float* LTl, float* colb,
-                                           int c0, int lane) {
+//
+// Right-looking unscaled LDL^T, four columns per step.  Lane i holds row i.
+// For the panel of columns J..J+3 every lane reads the panel's 4 x 4
+// diagonal block (rows J..J+3, published in shared memory) and runs the
+// same short recurrence: pivots d_t and multipliers M_st = z_st / d_t, with
+//     z_i = y_i M^-T:  z_i0 = y_i0,  z_i1 = y_i1 - M10 z_i0,
+//                      z_i2 = y_i2 - M20 z_i0 - M21 z_i1,
+//                      z_i3 = y_i3 - M30 z_i0 - M31 z_i1 - M32 z_i2
+// for its own row's panel entries y_i (z_ss = d_s for the panel rows, so
+// every lane sees the same pivots).  z_i stays in the row (the unscaled L
+// entries), the rows publish z, and the trailing entries take
+//     a_ik -= sum_t (z_it / d_t) z_kt,
+// the panel's next four columns first so they can be published early.
+// Square roots come at the end: L_ik = z_ik / sqrt(d_k), L_kk = sqrt(d_k).
+__device__ __forceinline__ int leaf_factor(float* S, float* rinv, float* LTl, float4* yb,
+                                           float4* zb, int c0, int lane) {
   float a[32];
 #pragma unroll
   for (int k = 0; k < 32; ++k) a[k] = (k <= lane) ? S[(c0 + lane) * kDP + c0 + k] : 0.f;
   int first_bad = 0;
-  // Column j is published (lane k writes its a[j]) as soon as its last
-  // update is done, so the next step's broadcast overlaps this step's FMAs;
-  // two buffers, so a step's write never meets the previous step's reads.
-  colb[lane] = a[0];
+  yb[lane] = make_float4(a[0], a[1], a[2], a[3]);
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const float* cb = colb + (j & 1) * 32;
+  for (int J = 0; J < 32; J += 4) {
     __syncwarp();
-    float col[32];
+    // the panel's diagonal block, then the shared recurrence
+    const float4 r0 = yb[J], r1 = yb[J + 1], r2 = yb[J + 2], r3 = yb[J + 3];
+    const float d0 = r0.x;
+    const float i0 = recip_nr(d0);
+    const float M10 = r1.x * i0, M20 = r2.x * i0, M30 = r3.x * i0;
+    const float d1 = fmaf(-M10, r1.x, r1.y);                 // z_11
+    const float i1 = recip_nr(d1);
+    const float z21 = fmaf(-M10, r2.x, r2.y);
+    const float z31 = fmaf(-M10, r3.x, r3.y);
+    const float M21 = z21 * i1, M31 = z31 * i1;
+    const float d2 = fmaf(-M21, z21, fmaf(-M20, r2.x, r2.z));  // z_22
+    const float i2 = recip_nr(d2);
+    const float z32 = fmaf(-M21, z31, fmaf(-M20, r3.x, r3.z));
+    const float M32 = z32 * i2;
+    const float d3 = fmaf(-M32, z32, fmaf(-M31, z31, fmaf(-M30, r3.x, r3.w)));  // z_33
+    const float i3 = recip_nr(d3);
+    const float dv[4] = {d0, d1, d2, d3};
 #pragma unroll
-    for (int q = j / 4; q < 8; ++q) {
-      const float4 v = reinterpret_cast<const float4*>(cb)[q];
-      col[4 * q] = v.x;
-      col[4 * q + 1] = v.y;
-      col[4 * q + 2] = v.z;
-      col[4 * q + 3] = v.w;
+    for (int t = 0; t < 4; ++t) {
+      const bool badj = !(dv[t] > 0.f) || !isfinite(dv[t]);
+      first_bad = (first_bad == 0 && badj) ? (J + t + 1) : first_bad;
     }
-    const float d = col[j];
-    const bool badj = !(d > 0.f) || !isfinite(d);
-    first_bad = (first_bad == 0 && badj) ? (j + 1) : first_bad;
-    // 1/d: hardware estimate and one Newton step (a multiplier needs no more)
-    const float r0 = ptx::rcp_approx(d);
-    const float rd = fmaf(fmaf(-d, r0, 1.f), r0, r0);
-    const float m = (lane > j) ? a[j] * rd : 0.f;
-    if (j + 1 < 32) {
-      a[j + 1] = fmaf(-m, col[j + 1], a[j + 1]);
-      colb[((j + 1) & 1) * 32 + lane] = a[j + 1];
-    }
+    // this row's z (for the panel rows this reproduces the pivots above)
+    const float z0 = a[J];
+    const float z1 = fmaf(-M10, z0, a[J + 1]);
+    const float z2 = fmaf(-M21, z1, fmaf(-M20, z0, a[J + 2]));
+    const float z3 = fmaf(-M32, z2, fmaf(-M31, z1, fmaf(-M30, z0, a[J + 3])));
+    a[J] = z0;
+    a[J + 1] = z1;
+    a[J + 2] = z2;
+    a[J + 3] = z3;
+    if (J + 4 < 32) {
+      zb[lane] = make_float4(z0, z1, z2, z3);
+      const float m0 = z0 * i0, m1 = z1 * i1, m2 = z2 * i2, m3 = z3 * i3;
+      __syncwarp();
+      float4 zk[32];
 #pragma unroll
-    for (int k = j + 2; k < 32; ++k) a[k] = fmaf(-m, col[k], a[k]);
+      for (int k = J + 4; k < 32; ++k) zk[k] = zb[k];
+      // the next panel's columns first, then publish them
+#pragma unroll
+      for (int k = J + 4; k < J + 8; ++k)
+        a[k] = fmaf(-m3, zk[k].w, fmaf(-m2, zk[k].z, fmaf(-m1, zk[k].y, fmaf(-m0, zk[k].x, a[k]))));
+      yb[lane] = make_float4(a[J + 4], a[J + 5], a[J + 6], a[J + 7]);
+#pragma unroll
+      for (int k = J + 8; k < 32; ++k)
+        a[k] = fmaf(-m3, zk[k].w, fmaf(-m2, zk[k].z, fmaf(-m1, zk[k].y, fmaf(-m0, zk[k].x, a[k]))));
+    }
   }
   if (first_bad) return first_bad;
   // L_ik = a_ik / sqrt(d_k), L_kk = sqrt(d_k)
@@ -134,7 +176,8 @@ __global__ void __launch_bounds__(kDiagThreads) chol_diag_kernel(const float* __
   XT = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(XT) + 15) & ~uintptr_t(15));
   float* LTl = XT + 32 * kXP;        // [32][kTP]   current leaf, transposed
   float* rinv = LTl + 32 * kTP;      // [128]       1 / L_kk
-  float* colb = rinv + 128;          // [2][32]     the leaf factor's column buffers
+  float4* yb = reinterpret_cast<float4*>(rinv + 128);  // [32] leaf panel rows
+  float4* zb = yb + 32;                                 // [32] leaf z values
   __shared__ int fail;
   const int kb = p * 128;
   const int bs = min(128, n - kb);
@@ -162,7 +205,7 @@ __global__ void __launch_bounds__(kDiagThreads) chol_diag_kernel(const float* __
   for (int j = 0; j < 4; ++j) {
     const int c0 = 32 * j;
     if (warp == 0) {
-      const int fb = leaf_factor(S, rinv, LTl, colb, c0, lane);
+      const int fb = leaf_factor(S, rinv, LTl, yb, zb, c0, lane);
       if (fb && lane == 0) fail = c0 + fb;
     }
     __syncthreads();

@@ -103,7 +103,7 @@ size_t hessian_ws(int64_t n, int64_t ntok, gptq_dtype xt) {
 gptq_status check_cfg(const gptq_config* cfg) {
   if (!cfg) return GPTQ_ERR_INVALID_ARG;
   if (cfg->bits < 2 || cfg->bits > 8) return GPTQ_ERR_INVALID_ARG;
-  if (cfg->sym != 0) return GPTQ_ERR_UNSUPPORTED;
+  if (cfg->sym != 0 && cfg->sym != 1) return GPTQ_ERR_INVALID_ARG;
   if (cfg->block != gptq::kBlock) return GPTQ_ERR_UNSUPPORTED;
   const int g = cfg->group_size;
   if (g == 0 || g < -1) return GPTQ_ERR_INVALID_ARG;
@@ -224,8 +224,8 @@ gptq_status gptq_quantize_layer(const void* W, gptq_dtype wt, int64_t rows, int6
   if (!ws || ws_bytes < gptq::quantize_workspace_bytes(rows, n)) return GPTQ_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return GPTQ_ERR_INVALID_ARG;
   return cuda_status(gptq::launch_quantize_layer(W, wt, rows, n, U, perm, dead, cfg->bits,
-                                                 cfg->group_size, codes, scales, zeros, g_idx,
-                                                 Wq, row_loss, ws, s));
+                                                 cfg->group_size, cfg->sym, codes, scales, zeros,
+                                                 g_idx, Wq, row_loss, ws, s));
 }
 
 gptq_status gptq_pack_int4(const uint8_t* codes, int64_t rows, int64_t n, uint32_t* out,

@@ -55,9 +55,9 @@ size_t cholesky_workspace_bytes(int64_t n);
 // ---- sweep (sweep.cu)
 cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows, int64_t n, const float* U,
                                   const int32_t* perm, const uint8_t* dead, int bits,
-                                  int group_size, uint8_t* codes, float* scales, uint8_t* zeros,
-                                  int32_t* g_idx, float* Wq, float* row_loss, void* ws,
-                                  cudaStream_t s);
+                                  int group_size, int sym, uint8_t* codes, float* scales,
+                                  uint8_t* zeros, int32_t* g_idx, float* Wq, float* row_loss,
+                                  void* ws, cudaStream_t s);
 size_t quantize_workspace_bytes(int64_t rows, int64_t n);
 // out[i] = a[i] / b[i] by the sweep's division routine (fdiv.cuh)
 cudaError_t launch_selftest_division(const float* a, const float* b, int64_t count, float* out,

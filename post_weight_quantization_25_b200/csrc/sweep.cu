@@ -126,15 +126,22 @@ struct SweepTrailItems {
 
 // The ruler for values spanning [mn, mx]: range stretched to include 0
 // ([-1, 1] when flat), scale = (xmax - xmin) / maxq, zero = rint(-xmin / scale).
-__device__ __forceinline__ void fit_ruler(float mn, float mx, float maxq, float& scale,
+// Symmetric ruler (opt-in): the range becomes [-m, m], m = max(-xmin, xmax),
+// with the same scale formula and the zero point on the middle tick.
+__device__ __forceinline__ void fit_ruler(float mn, float mx, float maxq, int sym, float& scale,
                                           float& zf) {
   float xmin = fminf(mn, 0.f), xmax = fmaxf(mx, 0.f);
+  if (sym) {
+    const float m = fmaxf(-xmin, xmax);
+    xmin = -m;
+    xmax = m;
+  }
   if (xmin == 0.f && xmax == 0.f) {
     xmin = -1.f;
     xmax = 1.f;
   }
   scale = __fdiv_rn(xmax - xmin, maxq);
-  zf = rintf(__fdiv_rn(-xmin, scale));
+  zf = sym ? 0.5f * (maxq + 1.f) : rintf(__fdiv_rn(-xmin, scale));
 }
 
 __device__ __forceinline__ float warp_min(float v) {
@@ -158,7 +165,7 @@ __global__ void pos_kernel(const int32_t* __restrict__ perm, int n, int32_t* __r
 template <typename T>
 __global__ void __launch_bounds__(256) gather_w_kernel(
     const T* __restrict__ W, int n, const int32_t* __restrict__ perm,
-    const uint8_t* __restrict__ dead, float* __restrict__ Wf, int per_row, float maxq,
+    const uint8_t* __restrict__ dead, float* __restrict__ Wf, int per_row, float maxq, int sym,
     float* __restrict__ scales, uint8_t* __restrict__ zeros, float* __restrict__ row_loss) {
   extern __shared__ float wrow[];
   __shared__ float red[2][8];
@@ -188,7 +195,7 @@ __global__ void __launch_bounds__(256) gather_w_kernel(
         mx = fmaxf(mx, red[1][i]);
       }
       float scale, zf;
-      fit_ruler(mn, mx, maxq, scale, zf);
+      fit_ruler(mn, mx, maxq, sym, scale, zf);
       scales[r] = scale;
       zeros[r] = (uint8_t)zf;
     }
@@ -226,7 +233,7 @@ __device__ __forceinline__ float quad_max(float v) {
 template <int GS>
 __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
     float* __restrict__ Wf, int rows, int n, const float* __restrict__ U, int i1, int bsz,
-    float maxq, int gsize, int G, float* __restrict__ Err_hi, float* __restrict__ Err_lo,
+    float maxq, int sym, int gsize, int G, float* __restrict__ Err_hi, float* __restrict__ Err_lo,
     uint8_t* __restrict__ codes_sw, float* __restrict__ scales, uint8_t* __restrict__ zeros,
     float* __restrict__ row_loss) {
   extern __shared__ __align__(16) float smem[];
@@ -280,7 +287,7 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
           mn = fminf(mn, v);
           mx = fmaxf(mx, v);
         }
-      fit_ruler(quad_min(mn), quad_max(mx), maxq, scale, zf);
+      fit_ruler(quad_min(mn), quad_max(mx), maxq, sym, scale, zf);
       if (active && q == 0) {
         scales[(int64_t)r * G + g] = scale;
         zeros[(int64_t)r * G + g] = (uint8_t)zf;
@@ -322,7 +329,7 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
           mn = fminf(mn, w[s2]);
           mx = fmaxf(mx, w[s2]);
         }
-      fit_ruler(quad_min(mn), quad_max(mx), maxq, scale, zf);
+      fit_ruler(quad_min(mn), quad_max(mx), maxq, sym, scale, zf);
       md = md_prepare(scale);
       if (active && q == 0 && jj < bsz) {  // groups past the last column do not exist
         const int g = (i1 + jj) / kGS;
@@ -438,9 +445,9 @@ size_t quantize_workspace_bytes(int64_t rows, int64_t n) {
 
 cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t n64,
                                   const float* U, const int32_t* perm, const uint8_t* dead,
-                                  int bits, int group_size, uint8_t* codes, float* scales,
-                                  uint8_t* zeros, int32_t* g_idx, float* Wq, float* row_loss,
-                                  void* ws, cudaStream_t s) {
+                                  int bits, int group_size, int sym, uint8_t* codes,
+                                  float* scales, uint8_t* zeros, int32_t* g_idx, float* Wq,
+                                  float* row_loss, void* ws, cudaStream_t s) {
   const int rows = (int)rows64, n = (int)n64;
   SweepWs w = carve(ws, rows64, n64);
   const float maxq = (float)((1 << bits) - 1);
@@ -455,14 +462,14 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
   if (wt == GPTQ_BF16) {
     if ((e = set_smem(gather_w_kernel<__nv_bfloat16>, row_smem)) != cudaSuccess) return e;
     gather_w_kernel<__nv_bfloat16><<<rows, 256, row_smem, s>>>(
-        static_cast<const __nv_bfloat16*>(W), n, perm, dead, w.Wf, per_row, maxq, scales, zeros,
-        row_loss);
+        static_cast<const __nv_bfloat16*>(W), n, perm, dead, w.Wf, per_row, maxq, sym, scales,
+        zeros, row_loss);
     note_launch();
   } else {
     if ((e = set_smem(gather_w_kernel<float>, row_smem)) != cudaSuccess) return e;
     gather_w_kernel<float><<<rows, 256, row_smem, s>>>(static_cast<const float*>(W), n, perm,
-                                                       dead, w.Wf, per_row, maxq, scales, zeros,
-                                                       row_loss);
+                                                       dead, w.Wf, per_row, maxq, sym, scales,
+                                                       zeros, row_loss);
     note_launch();
   }
 
@@ -544,8 +551,8 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
     const int eb = blk & 1;
 #define GPTQ_SWEEP_LAUNCH(GSV)                                                                 \
   sweep_block_kernel<GSV><<<sweep_ctas, kSweepThreads, us_smem, s>>>(                          \
-      w.Wf, rows, n, U, i1, bsz, maxq, group_size, G, w.Err_hi[eb], w.Err_lo[eb], w.codes_sw,  \
-      scales, zeros, row_loss)
+      w.Wf, rows, n, U, i1, bsz, maxq, sym, group_size, G, w.Err_hi[eb], w.Err_lo[eb],         \
+      w.codes_sw, scales, zeros, row_loss)
     if (gmode == 0)
       GPTQ_SWEEP_LAUNCH(0);
     else if (gmode == 1)

@@ -56,9 +56,12 @@ def test_workspace_sizes(lib):
     assert lib.gptq_workspace_size(_lib.GPTQ_OP_QUANTIZE, 4096, 4096, 0, 0, ctypes.byref(cfg),
                                    ctypes.byref(out)) == 0
     assert out.value >= 4096 * 4096 * 5
-    # a symmetric ruler and a block other than 128 are not implemented
-    bad = _lib.GptqConfig(4, 128, 0.01, 128, 1, 1)
-    assert lib.gptq_workspace_size(2, 16, 16, 0, 0, ctypes.byref(bad), ctypes.byref(out)) == 2
+    # the symmetric ruler is accepted; sym must be 0 or 1
+    sym = _lib.GptqConfig(4, 128, 0.01, 128, 1, 1)
+    assert lib.gptq_workspace_size(2, 16, 16, 0, 0, ctypes.byref(sym), ctypes.byref(out)) == 0
+    bad = _lib.GptqConfig(4, 128, 0.01, 128, 1, 2)
+    assert lib.gptq_workspace_size(2, 16, 16, 0, 0, ctypes.byref(bad), ctypes.byref(out)) == 1
+    # a block other than 128 is not implemented
     bad = _lib.GptqConfig(4, 128, 0.01, 64, 1, 0)
     assert lib.gptq_workspace_size(2, 16, 16, 0, 0, ctypes.byref(bad), ctypes.byref(out)) == 2
     bad = _lib.GptqConfig(4, 48, 0.01, 128, 1, 0)

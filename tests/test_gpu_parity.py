@@ -168,6 +168,17 @@ def test_layer_matches_oracle(rows, n, ntok, bits, g, act, dtype, dead):
     compare_layer(gpu, W, X, bits, g, 0.01, act)
 
 
+@pytest.mark.parametrize("rows,n,ntok,bits,g,act,dtype", [
+    (64, 384, 1500, 4, 128, True, torch.bfloat16), (48, 256, 800, 3, -1, False, torch.float32),
+    (40, 200, 700, 4, 32, True, torch.bfloat16)])
+def test_symmetric_ruler_matches_oracle(rows, n, ntok, bits, g, act, dtype):
+    """The opt-in symmetric ruler: zero point on the middle tick, same sweep."""
+    W, X = workloads.random_layer(rows, n, ntok, seed=rows + 3 * n, dtype=dtype, correlated=0.3)
+    gpu = gpu_layer(W, X, bits, g, 0.01, act, sym=True)
+    assert np.all(gpu["zeros"] == 2 ** (bits - 1))
+    compare_layer(gpu, W, X, bits, g, 0.01, act, sym=True)
+
+
 @pytest.mark.parametrize("g,act", [(-1, False), (128, False), (128, True), (32, True)])
 def test_identity_hessian_gives_rtn_on_gpu(g, act):
     n, rows = 256, 24

@@ -56,6 +56,55 @@ def test_grid_range_includes_zero_and_edges():
     assert int(O.quantize(5.0, s, z, 4)) == 15 and int(O.quantize(-5.0, s, z, 4)) == 0
 
 
+def test_symmetric_ruler_closed_form():
+    """The opt-in symmetric ruler (page 'GPTQ, with the code open', section
+    'Paper vs. code'): range [-m, m] with m = max(|min|, |max|), the same
+    step formula, zero point on the middle tick, so 0.0 is exact."""
+    s, z = O.fit_grid(-0.8, 0.4, 4, sym=True)
+    assert int(z) == 8
+    assert float(s) == float(np.float32(np.float32(1.6) / np.float32(15)))
+    ticks = O.dequantize(np.arange(16), s, z)
+    assert ticks[8] == 0.0 and ticks[0] == -8 * float(s) and ticks[15] == 7 * float(s)
+    assert int(O.quantize(0.4, s, z, 4)) == 12            # rint(3.75) + 8
+    assert int(O.quantize(-0.8, s, z, 4)) == 0            # rint(-7.5) = -8 (to even)
+    # all-positive range: stretched to [0, 0.5], then mirrored to [-0.5, 0.5]
+    s2, z2 = O.fit_grid(0.1, 0.5, 4, sym=True)
+    assert int(z2) == 8 and float(s2) == float(np.float32(np.float32(1.0) / np.float32(15)))
+    # 3 bits: middle tick 4; flat range -> [-1, 1]
+    s3, z3 = O.fit_grid(0.0, 0.0, 3, sym=True)
+    assert int(z3) == 4 and float(s3) == float(np.float32(np.float32(2.0) / np.float32(7)))
+    # only |min| and |max| matter: mirrored ranges give the same ruler
+    for a, b in ((0.3, 0.7), (0.7, 0.3), (0.0, 0.2)):
+        assert O.fit_grid(-a, b, 4, sym=True) == O.fit_grid(-b, a, 4, sym=True)
+    # the asymmetric ruler of the same range differs (zero 10, step 0.08)
+    sa, za = O.fit_grid(-0.8, 0.4, 4)
+    assert int(za) == 10 and float(sa) != float(s)
+
+
+def test_symmetric_ruler_in_the_sweep():
+    """Blocked and unblocked sweeps agree with the symmetric ruler, and with
+    H proportional to I the sweep is round-to-nearest on the same ruler."""
+    W, X = _layer(5, 24, 96, seed=808)
+    prep = O.prepare(O.hessian(X), W, 0.01, True)
+    U = O.upper_cholesky_of_inverse(prep["Hp"])
+    for g in (-1, 8):
+        ref = O.sweep(prep["Wp"], U, 4, g, sym=True)
+        assert np.all(ref["zeros"] == 8)
+        for B in (4, 8, 24):
+            if g > 0 and not (B % g == 0 or g % B == 0):
+                continue
+            b = O.sweep_blocked(prep["Wp"], U, 4, g, B, sym=True)
+            assert np.array_equal(b["codes"], ref["codes"])
+            np.testing.assert_allclose(b["Wq"], ref["Wq"], rtol=0, atol=1e-12)
+    n = 16
+    Xi = np.concatenate([np.eye(n)] * 3, axis=1) * 1.5
+    Wn = np.random.default_rng(9).normal(0, 0.02, (4, n))
+    r = O.gptq_layer(Wn, O.hessian(Xi), 3, 8, 0.01, False, sym=True)
+    base = O.rtn(r["W0"], 3, 8, sym=True)
+    assert np.array_equal(r["codes_orig"], base["codes"])
+    assert np.all(r["zeros"] == 4)
+
+
 def test_rounding_is_half_to_even():
     s, z = np.float32(1.0), 0
     assert list(O.quantize(np.array([0.5, 1.5, 2.5, 3.5]), s, z, 4)) == [0, 2, 2, 4]
