@@ -48,6 +48,8 @@ def parse_args():
                    help="override the workload's calibration token count (profiling runs)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-next", action="store_true",
+                   help="skip the measurement of the dequant x activation kernel")
     return p.parse_args()
 
 
@@ -255,6 +257,40 @@ def blas_threads():
     return host_cores()
 
 
+# ----------------------------------------------------------------- dequant x activation
+def measure_dequant_matvec(G, dev, packed, bits, n, scales, zeros, group_size, g_idx, batch=1,
+                           iters=20, label="", perm=None):
+    """Device time of gptq_dequant_matvec on `batch` bf16 activation vectors,
+    L2 flushed (a 256 MiB write) before every launch; bytes = everything the
+    kernel must read or write once."""
+    import torch
+    x = torch.randn(batch, n, device=dev).to(torch.bfloat16)
+    y = torch.empty(batch, packed.shape[0], dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ts = []
+    for i in range(iters + 3):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        G.gptq_dequant_matvec(packed, bits, n, scales, zeros, x, group_size, g_idx, perm=perm,
+                              out=y)
+        b.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            ts.append(a.elapsed_time(b))
+    t = statistics.median(ts) / 1e3
+    nbytes = sum(int(v.numel() * v.element_size()) for v in (packed, scales, zeros, x, y)
+                 if v is not None) + (int(g_idx.numel() * 4) if g_idx is not None else 0) \
+        + (int(perm.numel() * 4) if perm is not None else 0)
+    pk = peaks()
+    gbs = nbytes / t / 1e9
+    return {"shape": label, "order": "sweep (perm)" if perm is not None else "original (g_idx)",
+            "batch": batch, "bits": bits, "us": round(t * 1e6, 2),
+            "bytes": nbytes, "gbs": round(gbs, 1), "peak_gbs": pk["hbm_gbs"],
+            "frac": round(gbs / pk["hbm_gbs"], 4), "l2": "flushed before each launch"}
+
+
 # ----------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -318,12 +354,48 @@ def run_ours(args, rank, world, local_rank):
     if os.path.exists(tf_path):
         with open(tf_path) as f:
             tj = json.load(f)
-        if tj.get("workload") == wl.name and tj.get("kernel_rev") == "syrk-v2":
+        if tj.get("workload") == wl.name and tj.get("kernel_rev") == "syrk-pair-v1":
             traffic = tj.get("bytes_per_launch")
     roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_tflops"],
             "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": traffic,
-            "kernel": "syrk_bf16_kernel (+ mirror) in gptq_hessian_accumulate",
+            "kernel": "syrk_bf16_pair_kernel (+ mirror) in gptq_hessian_accumulate",
             "peak_source": f"{pk['_source']} bf16 burst", "algorithmic_flops": flops}
+
+    # the consumer of the packed codes (fused dequant x activation), outside
+    # the timed step: on this layer's own output, and on the 70B down-proj
+    # shape (8192 x 28672, 4-bit g128, act-order g_idx) with random codes
+    nxt = None
+    if rank == 0 and not args.no_next and wl.bits in (3, 4):
+        import torch
+        torch.cuda.synchronize()
+        mv = [measure_dequant_matvec(G, dev, lq.packed, wl.bits, n, lq.scales, lq.zeros,
+                                     wl.group_size, lq.g_idx, label=f"{rows}x{n} (this layer)")]
+        if wl.actorder:
+            sw = G.gptq_gather_columns_u8(lq.codes, lq.perm)
+            pk_sw = (G.gptq_pack_int4 if wl.bits == 4 else G.gptq_pack_int3)(sw)
+            mv.append(measure_dequant_matvec(G, dev, pk_sw, wl.bits, n, lq.scales, lq.zeros,
+                                             wl.group_size, None, perm=lq.perm,
+                                             label=f"{rows}x{n} (this layer)"))
+            del sw, pk_sw
+        r7, n7 = 8192, 28672
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(77)
+        pk7 = torch.randint(-2 ** 31, 2 ** 31 - 1, (r7, n7 // 8), generator=gen, device=dev,
+                            dtype=torch.int64).to(torch.int32)
+        sc7 = torch.rand(r7, n7 // 128, generator=gen, device=dev) * 0.01 + 1e-4
+        z7 = torch.randint(0, 16, (r7, n7 // 128), generator=gen, device=dev,
+                           dtype=torch.int64).to(torch.uint8)
+        pm7 = torch.randperm(n7, generator=gen, device=dev).to(torch.int32)
+        gi7 = torch.empty_like(pm7)
+        gi7[pm7.long()] = (torch.arange(n7, device=dev, dtype=torch.int32) // 128)
+        label7 = "8192x28672 (70B down-proj shape)"
+        for b in (1, 8):
+            mv.append(measure_dequant_matvec(G, dev, pk7, 4, n7, sc7, z7, 128, gi7, batch=b,
+                                             label=label7))
+            mv.append(measure_dequant_matvec(G, dev, pk7, 4, n7, sc7, z7, 128, None, batch=b,
+                                             label=label7, perm=pm7))
+        nxt = {"dequant_matvec": mv}
+        del pk7, sc7, z7, gi7, pm7
 
     # end to end through the same C ABI with host buffers
     e2e = None
@@ -387,6 +459,7 @@ def run_ours(args, rank, world, local_rank):
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clk.summary(),
+            "next": nxt,
         }
         print(json.dumps(line), flush=True)
 

@@ -190,6 +190,39 @@ gptq_status gptq_dequant(const uint32_t* packed, int bits, int64_t rows, int64_t
                          int64_t n_groups, const int32_t* g_idx, void* out, gptq_dtype ot,
                          void* stream);
 
+/* The consumer of the packed codes: y = x w_hat^T for `batch` activation
+ * vectors, with w_hat dequantized on the fly and never stored (page "GPTQ,
+ * with the code open", section "Claims & evidence": the faster generation
+ * comes from custom kernels at batch size 1, where reading the weights
+ * dominates -- packed codes are 8 / bits times smaller than fp32, 4 / bits
+ * times smaller than bf16).
+ *   packed, scales, zeros, group_size, n_groups, g_idx: exactly as for
+ *          gptq_dequant (same layout, same single-multiply w_hat).
+ *   perm   NULL, or (with g_idx NULL) the sweep order of an act-order layer:
+ *          the packed rows then hold the codes in sweep order (column k is
+ *          original column perm[k], see gptq_gather_columns_u8), so every
+ *          group is a run of group_size consecutive columns, and column k
+ *          multiplies x[b][perm[k]].  Reading rulers per run instead of per
+ *          column is what makes act-order layers fast here.
+ *   x      batch x n activations, row-major, xt = GPTQ_BF16 or GPTQ_F32.
+ *   y      batch x rows fp32 (written), y[b][r] = sum_c w_hat[r][c] x[b][c],
+ *          summed in fp32 (each term w_hat * x rounded once by an FMA).
+ * batch >= 0 (any size; launched in groups of 8, 4, 2, 1).  Errors as for
+ * gptq_dequant; perm together with g_idx is invalid. */
+gptq_status gptq_dequant_matvec(const uint32_t* packed, int bits, int64_t rows, int64_t n,
+                                const float* scales, const uint8_t* zeros, int group_size,
+                                int64_t n_groups, const int32_t* g_idx, const int32_t* perm,
+                                const void* x, gptq_dtype xt, int64_t batch, float* y,
+                                void* stream);
+
+/* dst[r][k] = src[r][perm[k]] for a rows x n byte matrix (device pointers;
+ * perm int32[n], a permutation of 0..n-1).  With the `perm` of
+ * gptq_cholesky_inverse it turns codes in original column order into codes
+ * in sweep order, for packing and gptq_dequant_matvec.  src and dst must not
+ * overlap. */
+gptq_status gptq_gather_columns_u8(const uint8_t* src, int64_t rows, int64_t n,
+                                   const int32_t* perm, uint8_t* dst, void* stream);
+
 /* Static string for a status code (host). */
 const char* gptq_status_string(int status);
 

@@ -535,3 +535,21 @@ def dequant(packed: np.ndarray, bits: int, n: int, scales: np.ndarray, zeros: np
     if out == "bf16":
         return bf16_round(w)
     return w
+
+
+# --------------------------------------------------------------------------
+# Consumer of the packed codes (page "GPTQ, with the code open", section
+# "Claims & evidence": generation at batch size 1 reads the packed weights)
+# --------------------------------------------------------------------------
+def dequant_matvec(packed: np.ndarray, bits: int, n: int, scales: np.ndarray,
+                   zeros: np.ndarray, x, group_size: int = -1, g_idx=None, perm=None):
+    """y = x w_hat^T in fp64 for activations x (batch x n, or n), with w_hat
+    the binary32 dequantized weights of ``dequant``.  With ``perm`` the
+    packed columns are in sweep order: column k pairs with x[:, perm[k]].
+    Returns ``(y, mag)`` where ``mag = |x| |w_hat|^T`` (the sum of |terms|,
+    for error bounds)."""
+    W = dequant(packed, bits, n, scales, zeros, group_size, g_idx).astype(np.float64)
+    X = np.atleast_2d(np.asarray(x, dtype=np.float64))
+    if perm is not None:
+        X = X[:, np.asarray(perm, dtype=np.int64)]
+    return X @ W.T, np.abs(X) @ np.abs(W).T

@@ -23,7 +23,9 @@ from ._lib import (GPTQ_BF16, GPTQ_F32, GPTQ_OP_CHOLESKY, GPTQ_OP_HESSIAN, GPTQ_
 
 __all__ = ["GptqError", "GptqConfig", "gptq_workspace_size", "gptq_hessian_accumulate",
            "gptq_cholesky_inverse", "gptq_quantize_layer", "gptq_pack_int4", "gptq_pack_int3",
-           "gptq_dequant", "gptq_status_string", "make_config", "QuantizedLinear",
+           "gptq_dequant", "gptq_dequant_matvec", "gptq_gather_columns_u8", "gptq_status_string",
+           "make_config",
+           "QuantizedLinear",
            "quantize_linear", "LayerQuantizer", "library"]
 
 
@@ -220,6 +222,39 @@ def gptq_dequant(packed: torch.Tensor, bits: int, n: int, scales: torch.Tensor,
                                 _dtype_code(out.dtype), _stream(stream))
     _check(st, "gptq_dequant")
     return out
+
+
+def gptq_gather_columns_u8(src: torch.Tensor, perm: torch.Tensor, out=None,
+                           stream=None) -> torch.Tensor:
+    """out[r][k] = src[r][perm[k]] (uint8 rows x n): codes into sweep order."""
+    _need_cuda(src, perm)
+    rows, n = src.shape
+    out = torch.empty_like(src) if out is None else out
+    _check(library().gptq_gather_columns_u8(_p(src), rows, n, _p(perm), _p(out), _stream(stream)),
+           "gptq_gather_columns_u8")
+    return out
+
+
+def gptq_dequant_matvec(packed: torch.Tensor, bits: int, n: int, scales: torch.Tensor,
+                        zeros: torch.Tensor, x: torch.Tensor, group_size: int = -1, g_idx=None,
+                        perm=None, out=None, stream=None) -> torch.Tensor:
+    """y = x w_hat^T with w_hat dequantized on the fly from the packed codes.
+    x: (batch, n) or (n,) bf16/fp32 on the GPU; returns (batch, rows) fp32
+    (or (rows,) for a 1-D x).  perm: the codes are packed in sweep order
+    (see gptq_gather_columns_u8) and column k multiplies x[perm[k]]."""
+    _need_cuda(packed, scales, zeros, g_idx, perm, x)
+    rows = packed.shape[0]
+    x2 = x.reshape(1, -1) if x.dim() == 1 else x
+    if x2.shape[1] != n or not x2.is_contiguous():
+        raise GptqError("x must be a contiguous (batch, n) tensor")
+    batch = x2.shape[0]
+    out = torch.empty(batch, rows, dtype=torch.float32, device=packed.device) if out is None else out
+    st = library().gptq_dequant_matvec(_p(packed), int(bits), rows, int(n), _p(scales), _p(zeros),
+                                       int(group_size), scales.shape[1], _p(g_idx), _p(perm),
+                                       _p(x2), _dtype_code(x2.dtype), batch, _p(out),
+                                       _stream(stream))
+    _check(st, "gptq_dequant_matvec")
+    return out.reshape(-1) if x.dim() == 1 else out
 
 
 @dataclasses.dataclass

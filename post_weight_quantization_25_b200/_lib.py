@@ -26,7 +26,7 @@ GPTQ_OP_QUANTIZE = 2
 EXPORTS = ("gptq_workspace_size", "gptq_hessian_accumulate", "gptq_cholesky_inverse",
            "gptq_quantize_layer", "gptq_pack_int4", "gptq_pack_int3", "gptq_dequant",
            "gptq_status_string", "gptq_launch_count", "gptq_cholesky_inverse_noalloc",
-           "gptq_selftest_division")
+           "gptq_selftest_division", "gptq_dequant_matvec", "gptq_gather_columns_u8")
 
 
 class GptqConfig(ctypes.Structure):
@@ -57,6 +57,9 @@ _SIGNATURES = {
     "gptq_launch_count": (_i64, []),
     "gptq_cholesky_inverse_noalloc": (_int, [_vp, _i64, _f, _int, _vp, _vp, _vp, _vp, _vp]),
     "gptq_selftest_division": (_int, [_vp, _vp, _i64, _vp, _vp]),
+    "gptq_dequant_matvec": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _int, _i64, _vp, _vp, _vp,
+                                   _int, _i64, _vp, _vp]),
+    "gptq_gather_columns_u8": (_int, [_vp, _i64, _i64, _vp, _vp, _vp]),
 }
 
 _LIB = None

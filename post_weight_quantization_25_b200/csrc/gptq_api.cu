@@ -263,4 +263,36 @@ gptq_status gptq_dequant(const uint32_t* packed, int bits, int64_t rows, int64_t
                                           static_cast<cudaStream_t>(stream)));
 }
 
+gptq_status gptq_dequant_matvec(const uint32_t* packed, int bits, int64_t rows, int64_t n,
+                                const float* scales, const uint8_t* zeros, int group_size,
+                                int64_t n_groups, const int32_t* g_idx, const int32_t* perm,
+                                const void* x, gptq_dtype xt, int64_t batch, float* y,
+                                void* stream) {
+  if (bits != 3 && bits != 4) return GPTQ_ERR_UNSUPPORTED;
+  if (rows < 0 || n <= 0 || batch < 0) return GPTQ_ERR_INVALID_ARG;
+  if ((bits == 4 && n % 8) || (bits == 3 && n % 32)) return GPTQ_ERR_INVALID_ARG;
+  if (xt != GPTQ_BF16 && xt != GPTQ_F32) return GPTQ_ERR_INVALID_ARG;
+  if (perm && g_idx) return GPTQ_ERR_INVALID_ARG;
+  const int64_t Gdef = group_size > 0 ? (n + group_size - 1) / group_size : 1;
+  const int64_t G = n_groups > 0 ? n_groups : Gdef;
+  if (!g_idx && G < Gdef) return GPTQ_ERR_INVALID_ARG;
+  if (rows == 0 || batch == 0) return GPTQ_OK;
+  if (!packed || !scales || !zeros || !x || !y || !aligned(packed, 4) || !aligned(scales, 4) ||
+      !aligned(y, 4) || !aligned(x, xt == GPTQ_BF16 ? 2 : 4))
+    return GPTQ_ERR_INVALID_ARG;
+  return cuda_status(gptq::launch_dequant_matvec(packed, bits, rows, n, scales, zeros,
+                                                 group_size, G, g_idx, perm, x,
+                                                 xt == GPTQ_BF16 ? 1 : 0, batch, y,
+                                                 static_cast<cudaStream_t>(stream)));
+}
+
+gptq_status gptq_gather_columns_u8(const uint8_t* src, int64_t rows, int64_t n,
+                                   const int32_t* perm, uint8_t* dst, void* stream) {
+  if (rows < 0 || n <= 0 || n > kMaxN) return GPTQ_ERR_INVALID_ARG;
+  if (rows == 0) return GPTQ_OK;
+  if (!src || !perm || !dst || src == dst) return GPTQ_ERR_INVALID_ARG;
+  return cuda_status(gptq::launch_gather_columns_u8(src, rows, n, perm, dst,
+                                                    static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

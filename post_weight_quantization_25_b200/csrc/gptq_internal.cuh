@@ -68,6 +68,16 @@ cudaError_t launch_pack_int4(const uint8_t* codes, int64_t rows, int64_t n, uint
                              cudaStream_t s);
 cudaError_t launch_pack_int3(const uint8_t* codes, int64_t rows, int64_t n, uint32_t* out,
                              cudaStream_t s);
+// y (batch x rows fp32) = x (batch x n, bf16 or fp32) w_hat^T, w_hat dequantized on the fly;
+// with perm, column k of the packed rows multiplies x[perm[k]].
+cudaError_t launch_dequant_matvec(const uint32_t* packed, int bits, int64_t rows, int64_t n,
+                                  const float* scales, const uint8_t* zeros, int group_size,
+                                  int64_t n_groups, const int32_t* g_idx, const int32_t* perm,
+                                  const void* x, int x_bf16, int64_t batch, float* y,
+                                  cudaStream_t s);
+// dst[r][k] = src[r][perm[k]] (rows x n bytes)
+cudaError_t launch_gather_columns_u8(const uint8_t* src, int64_t rows, int64_t n,
+                                     const int32_t* perm, uint8_t* dst, cudaStream_t s);
 cudaError_t launch_dequant(const uint32_t* packed, int bits, int64_t rows, int64_t n,
                            const float* scales, const uint8_t* zeros, int group_size,
                            int64_t n_groups, const int32_t* g_idx, void* out, int out_bf16,

@@ -46,6 +46,65 @@ def test_pack_and_dequant_bit_exact(bits, rows, n, g, use_gidx):
     assert np.array_equal(w16.view(torch.int16).cpu().numpy().view(np.uint16), ref16)
 
 
+@pytest.mark.parametrize("bits,rows,n,g,use_gidx,batch,xdt", [
+    (4, 7, 64, 16, False, 1, torch.float32), (4, 33, 256, 128, True, 3, torch.bfloat16),
+    (4, 130, 1032, -1, False, 8, torch.bfloat16), (3, 9, 96, 32, False, 2, torch.float32),
+    (3, 17, 2080, 128, True, 11, torch.bfloat16), (4, 1, 8, -1, False, 1, torch.float32)])
+def test_dequant_matvec_matches_oracle(bits, rows, n, g, use_gidx, batch, xdt):
+    """y = x w_hat^T with w_hat dequantized on the fly.  Bound: each lane sums
+    n/32 terms in fp32 and five shuffle levels follow, so the error is at
+    most (n/32 + 5) 2^-24 sum|w_hat x| to first order (doubled here)."""
+    rng = np.random.default_rng(bits * 7 + n + batch)
+    codes = rng.integers(0, 2 ** bits, (rows, n))
+    G_ = 1 if g <= 0 else (n + g - 1) // g
+    scales = rng.uniform(1e-4, 0.2, (rows, G_)).astype(np.float32)
+    zeros = rng.integers(0, 2 ** bits, (rows, G_))
+    gidx = rng.integers(0, G_, n) if use_gidx else None
+    cd = torch.from_numpy(codes.astype(np.uint8)).cuda()
+    packed = G.gptq_pack_int4(cd) if bits == 4 else G.gptq_pack_int3(cd)
+    x = torch.randn(batch, n, generator=torch.Generator().manual_seed(n)).to(xdt)
+    y = G.gptq_dequant_matvec(packed, bits, n, torch.from_numpy(scales).cuda(),
+                              torch.from_numpy(zeros.astype(np.uint8)).cuda(), x.cuda(), g,
+                              torch.from_numpy(gidx.astype(np.int32)).cuda() if use_gidx else None)
+    ref_packed = O.pack_int4(codes) if bits == 4 else O.pack_int3(codes)
+    yo, mag = O.dequant_matvec(ref_packed, bits, n, scales, zeros, x.float().numpy(), g, gidx)
+    err = np.abs(y.cpu().numpy().astype(np.float64) - yo)
+    bound = 2 * (n / 32 + 5) * 2.0 ** -24 * mag + 1e-30
+    assert np.all(err <= bound), float(np.max(err / bound))
+
+
+@pytest.mark.parametrize("bits,rows,n,g,batch", [(4, 40, 1024, 128, 1), (3, 33, 2048, 128, 4),
+                                                 (4, 7, 256, 32, 8)])
+def test_dequant_matvec_in_sweep_order(bits, rows, n, g, batch):
+    """Act-order layers: the codes gathered into sweep order (bit exact), packed,
+    and multiplied with x[perm] -- the same y as the original-order product."""
+    rng = np.random.default_rng(bits + rows + n)
+    codes = rng.integers(0, 2 ** bits, (rows, n))
+    perm = rng.permutation(n)
+    G_ = n // g
+    scales = rng.uniform(1e-4, 0.2, (rows, G_)).astype(np.float32)
+    zeros = rng.integers(0, 2 ** bits, (rows, G_))
+    gidx = np.empty(n, dtype=np.int64)
+    gidx[perm] = np.arange(n) // g          # group of original column c
+    cd = torch.from_numpy(codes.astype(np.uint8)).cuda()
+    pd = torch.from_numpy(perm.astype(np.int32)).cuda()
+    csw = G.gptq_gather_columns_u8(cd, pd)
+    assert np.array_equal(csw.cpu().numpy(), codes[:, perm].astype(np.uint8))
+    pk = G.gptq_pack_int4(csw) if bits == 4 else G.gptq_pack_int3(csw)
+    x = torch.randn(batch, n, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    sd = torch.from_numpy(scales).cuda()
+    zd = torch.from_numpy(zeros.astype(np.uint8)).cuda()
+    y = G.gptq_dequant_matvec(pk, bits, n, sd, zd, x.cuda(), g, perm=pd)
+    ref_sw = O.pack_int4(codes[:, perm]) if bits == 4 else O.pack_int3(codes[:, perm])
+    yo, mag = O.dequant_matvec(ref_sw, bits, n, scales, zeros, x.float().numpy(), g, perm=perm)
+    err = np.abs(y.cpu().numpy().astype(np.float64) - yo)
+    assert np.all(err <= 2 * (n / 32 + 5) * 2.0 ** -24 * mag + 1e-30)
+    # the same product in original column order with g_idx
+    ref_o = O.pack_int4(codes) if bits == 4 else O.pack_int3(codes)
+    yo2, _ = O.dequant_matvec(ref_o, bits, n, scales, zeros, x.float().numpy(), g, gidx)
+    np.testing.assert_allclose(yo, yo2, rtol=0, atol=1e-12 * float(np.max(mag)))
+
+
 def test_pack_int4_unaligned_row_length():
     rng = np.random.default_rng(5)
     codes = rng.integers(0, 16, (6, 40))          # n % 32 != 0: the 8-code path

@@ -474,6 +474,36 @@ def test_dequant_single_rounding_and_bf16():
 
 
 # ---------------------------------------------------------------- mutations
+def test_dequant_matvec_columns_and_brute_force():
+    """A unit activation picks one column of w_hat exactly; a small case
+    equals the plain double loop."""
+    rng = np.random.default_rng(21)
+    for bits, n, g in ((4, 64, 16), (3, 96, 32), (4, 40, -1)):
+        rows = 5
+        codes = rng.integers(0, 2 ** bits, (rows, n))
+        G_ = 1 if g <= 0 else (n + g - 1) // g
+        scales = rng.uniform(1e-3, 0.1, (rows, G_)).astype(np.float32)
+        zeros = rng.integers(0, 2 ** bits, (rows, G_))
+        packed = O.pack_int4(codes) if bits == 4 else O.pack_int3(codes)
+        W = O.dequant(packed, bits, n, scales, zeros, g).astype(np.float64)
+        for c in (0, n // 2, n - 1):
+            e = np.zeros(n)
+            e[c] = 1.0
+            y, _ = O.dequant_matvec(packed, bits, n, scales, zeros, e, g)
+            assert np.array_equal(y[0], W[:, c])
+        x = rng.standard_normal((3, n))
+        y, mag = O.dequant_matvec(packed, bits, n, scales, zeros, x, g)
+        for b in range(3):
+            for r in range(rows):
+                ref = 0.0
+                for c in range(n):
+                    gc = (c // g) if g > 0 else 0
+                    # w_hat is the binary32 rounding of scale * (code - zero)
+                    w = float(np.float32(float(scales[r, gc]) * (codes[r, c] - zeros[r, gc])))
+                    ref += w * x[b, c]
+                assert abs(y[b, r] - ref) <= 1e-12 * mag[b, r]
+
+
 def test_planted_mistakes_are_caught():
     """Plant typical mistakes in the oracle's inputs/steps and check the pins
     above would reject them: a transposed U, a flipped repair sign, a dropped
