@@ -261,15 +261,16 @@ def blas_threads():
 def measure_dequant_matvec(G, dev, packed, bits, n, scales, zeros, group_size, g_idx, batch=1,
                            iters=20, label="", perm=None):
     """Device time of gptq_dequant_matvec on `batch` bf16 activation vectors,
-    L2 flushed (a 256 MiB write) before every launch; bytes = everything the
-    kernel must read or write once."""
+    L2 flushed before every launch by reading 256 MiB (a read leaves clean
+    lines; a write would leave dirty ones whose write-back the timed call
+    pays); bytes = everything the call must read or write once."""
     import torch
     x = torch.randn(batch, n, device=dev).to(torch.bfloat16)
     y = torch.empty(batch, packed.shape[0], dtype=torch.float32, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = torch.zeros(64 << 20, dtype=torch.float32, device=dev)
     ts = []
     for i in range(iters + 3):
-        flush.zero_()
+        flush.sum()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record()
@@ -285,10 +286,14 @@ def measure_dequant_matvec(G, dev, packed, bits, n, scales, zeros, group_size, g
         + (int(perm.numel() * 4) if perm is not None else 0)
     pk = peaks()
     gbs = nbytes / t / 1e9
-    return {"shape": label, "order": "sweep (perm)" if perm is not None else "original (g_idx)",
+    mma = (bits == 4 and x.dtype == torch.bfloat16 and g_idx is None and n % 32 == 0
+           and (group_size <= 0 or (group_size >= 32 and group_size & (group_size - 1) == 0)))
+    return {"shape": label, "order": "sweep (perm)" if perm is not None else
+            ("original (g_idx)" if g_idx is not None else "original"),
+            "kernel": "tensor-core (mma.sync)" if mma else "fp32 pipe",
             "batch": batch, "bits": bits, "us": round(t * 1e6, 2),
             "bytes": nbytes, "gbs": round(gbs, 1), "peak_gbs": pk["hbm_gbs"],
-            "frac": round(gbs / pk["hbm_gbs"], 4), "l2": "flushed before each launch"}
+            "frac": round(gbs / pk["hbm_gbs"], 4), "l2": "flushed (256 MiB read) before each launch"}
 
 
 # ----------------------------------------------------------------- our arm
@@ -394,7 +399,26 @@ def run_ours(args, rank, world, local_rank):
                                              label=label7))
             mv.append(measure_dequant_matvec(G, dev, pk7, 4, n7, sc7, z7, 128, None, batch=b,
                                              label=label7, perm=pm7))
-        nxt = {"dequant_matvec": mv}
+        # a plain streaming read of the same code bytes, same flush: what
+        # one pass over 117 MB reaches on this part
+        flush = torch.zeros(64 << 20, dtype=torch.float32, device=dev)
+        ts = []
+        for i in range(13):
+            flush.sum()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            pk7.view(torch.float32).sum()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts.append(a.elapsed_time(b))
+        rd = pk7.numel() * 4 / (statistics.median(ts) / 1e3) / 1e9
+        del flush
+        nxt = {"dequant_matvec": mv,
+               "stream_read_117MB_gbs": round(rd, 1),
+               "stream_read_note": "torch fp32 sum over the bytes of the 8192x28672 int4 codes "
+                                   "(a plain read pass), same L2 flush"}
         del pk7, sc7, z7, gi7, pm7
 
     # end to end through the same C ABI with host buffers

@@ -196,6 +196,15 @@ gptq_status gptq_dequant(const uint32_t* packed, int bits, int64_t rows, int64_t
  * comes from custom kernels at batch size 1, where reading the weights
  * dominates -- packed codes are 8 / bits times smaller than fp32, 4 / bits
  * times smaller than bf16).
+ * Two kernels serve it.  int4 codes with bf16 x, no g_idx, n % 32 == 0,
+ * group_size a power of two >= 32 (or per row), packed 16-byte aligned and
+ * zero points < 128: the tensor-core kernel, which multiplies exact bf16
+ * (q - zero) pairs with x in fp32 MMA accumulators, scales each group's sum
+ * once, and adds the two column halves of every output onto zeros (two
+ * terms, so the result does not depend on their order).  It first writes x
+ * (gathered by perm, if given) into batch x n bf16 of stream-ordered scratch
+ * from a pool private to this library, and zeroes y.  Everything else: the
+ * FP32-pipe kernel, one rounded FMA per term.
  *   packed, scales, zeros, group_size, n_groups, g_idx: exactly as for
  *          gptq_dequant (same layout, same single-multiply w_hat).
  *   perm   NULL, or (with g_idx NULL) the sweep order of an act-order layer:
@@ -206,7 +215,7 @@ gptq_status gptq_dequant(const uint32_t* packed, int bits, int64_t rows, int64_t
  *          column is what makes act-order layers fast here.
  *   x      batch x n activations, row-major, xt = GPTQ_BF16 or GPTQ_F32.
  *   y      batch x rows fp32 (written), y[b][r] = sum_c w_hat[r][c] x[b][c],
- *          summed in fp32 (each term w_hat * x rounded once by an FMA).
+ *          summed in fp32.
  * batch >= 0 (any size; launched in groups of 8, 4, 2, 1).  Errors as for
  * gptq_dequant; perm together with g_idx is invalid. */
 gptq_status gptq_dequant_matvec(const uint32_t* packed, int bits, int64_t rows, int64_t n,

@@ -59,7 +59,31 @@ constexpr int kMaxDevices = 64;
 std::mutex g_side_mu;
 SideStream g_side[kMaxDevices];
 bool g_side_ok[kMaxDevices] = {};
+std::mutex g_pool_mu;
+cudaMemPool_t g_pool[kMaxDevices] = {};
 }  // namespace
+
+bool scratch_pool(cudaMemPool_t* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(g_pool_mu);
+  if (!g_pool[dev]) {
+    cudaMemPoolProps props{};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t p = nullptr;
+    if (cudaMemPoolCreate(&p, &props) != cudaSuccess) return false;
+    uint64_t keep = ~0ull;
+    if (cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
+      cudaMemPoolDestroy(p);
+      return false;
+    }
+    g_pool[dev] = p;
+  }
+  *out = g_pool[dev];
+  return true;
+}
 
 std::mutex& side_lock() { return g_side_mu; }
 

@@ -35,6 +35,12 @@ struct SideStream {
 bool side_stream(SideStream* out);
 std::mutex& side_lock();
 
+// A stream-ordered memory pool of the current device, private to this
+// library, that keeps freed blocks for reuse (no release threshold), so
+// per-call scratch costs no mapping work after the first call.  Created on
+// first use per device.  Returns false if it cannot be had.
+bool scratch_pool(cudaMemPool_t* out);
+
 // ---- Hessian (hessian_syrk.cu)
 // H(upper incl. diagonal) += alpha * A_rows * B_rows^T over tokens [0, ntok),
 // A and B are n x ntok bf16 with row stride ld (elements).

@@ -12,9 +12,11 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 
 #include "gptq_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace gptq {
 namespace {
@@ -389,6 +391,262 @@ __global__ void __launch_bounds__(256) gather_columns_u8_kernel(const uint8_t* _
   for (int64_t k = threadIdx.x; k < n; k += blockDim.x) dst[r * n + k] = srow[perm[k]];
 }
 
+// ---------------------------------------------------------------------------
+// int4 codes x bf16 activations on the tensor cores (mma.sync, register
+// operands).  Decode-size batches (1..8 vectors) make this a skinny product:
+// on the FP32 pipe the dequantize + FMA per weight costs ~3.4 instructions,
+// more issue slots than the 0.5 byte of HBM it reads, and at 8 vectors it is
+// ALU-bound outright.  Here each pair of codes becomes an exact bf16x2 pair
+// (q - zero) with one shift + LOP3 (magic 128.0) and one bf16x2 subtract, and
+// the dot with all 8 vector slots is one m16n8k16 MMA per 256 weights, so
+// every batch size up to 8 costs the same instructions.
+//
+// Exactness: q - zero (|.| < 128) and x (bf16) are exact bf16 operands, so
+// every product is exact in fp32; partial sums are fp32 (tensor-core
+// accumulation), then scaled by the group's scale with one FMA: y = sum over
+// groups of scale * sum (q - zero) x.
+//
+// Work: CTA (tile, h) takes 16 rows (the MMA's M) and half h of the
+// 128-column slices; its warps take slices in turn and their partial sums
+// are added in a fixed order.  Each warp streams its slices' codes through a
+// private ring of kDqStages shared-memory slots with cp.async (each thread
+// copies and later reads back its own 16-byte pieces), so a warp keeps
+// kDqStages - 1 slices of code loads in flight without holding registers.  The two halves meet in y by atomic adds onto
+// zeros: fp32 addition of two terms is commutative, so y is the same
+// whichever half lands first.  Thread (g = lane / 4, t = lane % 4) holds
+// rows g and g + 8; in a slice, MMA pair j (j = 0..3) covers 32-column block
+// bj with the thread contributing word wj of it:
+//   block mode  (group_size a multiple of 128, or per row): bj = t, wj = j --
+//               one 16-byte load per row, the 4 blocks of a slice share a group;
+//   interleaved (group_size 32 or 64): bj = j, wj = t -- four 4-byte loads
+//               per row, each MMA pair stays inside one 32-column block, so a
+//               group's scale applies to its own partial sum.
+// From word w (8 codes, column 8 wj + i of the block in bits 4i..4i+3) the
+// k-slots are paired as (i, i + 4): ((w >> 4i) & 0x000F000F) | 0x43004300 is
+// the bf16 pair (128 + q_i, 128 + q_{i+4}).  A prep kernel writes x once per
+// call in that pairing (and in sweep order when a perm is given), so the MMA
+// B fragments load straight from it, and zeroes y.
+
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two MMAs for one word per row: codes wa (row g) and wb (row g + 8) with
+// their zero pairs za / zb; xp holds the word's 8 activations of vector g in
+// pair order (x0, x4), (x1, x5), (x2, x6), (x3, x7).
+__device__ __forceinline__ void mma_word(float (&c)[4], uint32_t wa, uint32_t wb, uint32_t za,
+                                         uint32_t zb, const uint4& xp) {
+  constexpr uint32_t kMask = 0x000F000Fu, kMagic = 0x43004300u;
+  mma_bf16_16816(c, bf16x2_sub((wa & kMask) | kMagic, za), bf16x2_sub((wb & kMask) | kMagic, zb),
+                 bf16x2_sub(((wa >> 4) & kMask) | kMagic, za),
+                 bf16x2_sub(((wb >> 4) & kMask) | kMagic, zb), xp.x, xp.y);
+  mma_bf16_16816(c, bf16x2_sub(((wa >> 8) & kMask) | kMagic, za),
+                 bf16x2_sub(((wb >> 8) & kMask) | kMagic, zb),
+                 bf16x2_sub(((wa >> 12) & kMask) | kMagic, za),
+                 bf16x2_sub(((wb >> 12) & kMask) | kMagic, zb), xp.z, xp.w);
+}
+
+__device__ __forceinline__ uint32_t zero_pair(uint8_t z) {
+  return 0x43004300u | (uint32_t)z | ((uint32_t)z << 16);
+}
+
+constexpr int kDqWarps = 4;    // warps per CTA
+constexpr int kDqStages = 5;   // code slices a warp keeps in flight (cp.async ring)
+constexpr int kDqMinBlocks = 8;
+constexpr int kDqSplit = 2;    // column halves per row tile (two atomic adds per output)
+// bytes between the 16 code rows of a staged slice: 64 (block mode: each
+// thread reads back its own 16-byte pieces, conflict-free) or 80 (interleaved
+// mode: 4-byte reads of 8 rows x 4 words land on distinct banks)
+template <bool kInterleaved>
+__host__ __device__ constexpr int dq_pitch() { return kInterleaved ? 80 : 64; }
+
+// The non-code operands of one slice for one thread: activations of its
+// block(s) and the rulers of its rows.
+// (block mode: one ruler per row for the slice; interleaved: one per block)
+template <bool kInterleaved>
+struct DqSide {
+  static constexpr int kR = kInterleaved ? 4 : 1;
+  uint4 xq[4];
+  float fa[kR], fb[kR];
+  uint32_t za[kR], zb[kR];
+};
+
+// gshift = log2(group_size), or 31 for one group per row.  kFull: every
+// block of slice s is inside the row (no masking).
+template <bool kInterleaved, bool kFull>
+__device__ __forceinline__ void dq_side(DqSide<kInterleaved>& d, int s, int nblk, int t, int gshift,
+                                        const __nv_bfloat16* xr, const float* sa, const float* sb,
+                                        const uint8_t* za_row, const uint8_t* zb_row) {
+  if constexpr (!kInterleaved) {
+    const int blk = 4 * s + t;
+    const bool ok = kFull || blk < nblk;
+    const uint4* xv = reinterpret_cast<const uint4*>(xr + 32 * blk);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) d.xq[j] = ok ? __ldg(xv + j) : make_uint4(0, 0, 0, 0);
+    const int grp = (128 * s) >> gshift;  // one group for the whole slice
+    d.fa[0] = __ldg(sa + grp);
+    d.fb[0] = __ldg(sb + grp);
+    d.za[0] = zero_pair(__ldg(za_row + grp));
+    d.zb[0] = zero_pair(__ldg(zb_row + grp));
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int blk = 4 * s + j;
+      const bool ok = kFull || blk < nblk;
+      d.xq[j] = ok ? __ldg(reinterpret_cast<const uint4*>(xr + 32 * blk + 8 * t))
+                   : make_uint4(0, 0, 0, 0);
+      const int grp = ok ? (32 * blk) >> gshift : 0;
+      d.fa[j] = __ldg(sa + grp);
+      d.fb[j] = __ldg(sb + grp);
+      d.za[j] = zero_pair(__ldg(za_row + grp));
+      d.zb[j] = zero_pair(__ldg(zb_row + grp));
+    }
+  }
+}
+
+// `st`: this warp's staged slice (16 rows x pitch bytes of codes).
+template <bool kInterleaved>
+__device__ __forceinline__ void dq_slice(float (&Y)[4], const uint8_t* st,
+                                         const DqSide<kInterleaved>& d,
+                                         int g, int t) {
+  constexpr int P = dq_pitch<kInterleaved>();
+  if constexpr (!kInterleaved) {
+    const uint4 qa = *reinterpret_cast<const uint4*>(st + g * P + 16 * t);
+    const uint4 qb = *reinterpret_cast<const uint4*>(st + (g + 8) * P + 16 * t);
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    mma_word(c, qa.x, qb.x, d.za[0], d.zb[0], d.xq[0]);
+    mma_word(c, qa.y, qb.y, d.za[0], d.zb[0], d.xq[1]);
+    mma_word(c, qa.z, qb.z, d.za[0], d.zb[0], d.xq[2]);
+    mma_word(c, qa.w, qb.w, d.za[0], d.zb[0], d.xq[3]);
+    Y[0] = fmaf(d.fa[0], c[0], Y[0]);
+    Y[1] = fmaf(d.fa[0], c[1], Y[1]);
+    Y[2] = fmaf(d.fb[0], c[2], Y[2]);
+    Y[3] = fmaf(d.fb[0], c[3], Y[3]);
+  } else {
+    // blocks past the row end hold zero x, so their terms vanish
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t wa = *reinterpret_cast<const uint32_t*>(st + g * P + 16 * j + 4 * t);
+      const uint32_t wb = *reinterpret_cast<const uint32_t*>(st + (g + 8) * P + 16 * j + 4 * t);
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
+      mma_word(c, wa, wb, d.za[j], d.zb[j], d.xq[j]);
+      Y[0] = fmaf(d.fa[j], c[0], Y[0]);
+      Y[1] = fmaf(d.fa[j], c[1], Y[1]);
+      Y[2] = fmaf(d.fb[j], c[2], Y[2]);
+      Y[3] = fmaf(d.fb[j], c[3], Y[3]);
+    }
+  }
+}
+
+template <bool kInterleaved>
+__global__ void __launch_bounds__(kDqWarps * 32, kDqMinBlocks) dequant_mma_int4_kernel(
+    const uint32_t* __restrict__ packed, int64_t rows, int64_t n,
+    const float* __restrict__ scales, const uint8_t* __restrict__ zeros, int gshift, int64_t G,
+    const __nv_bfloat16* __restrict__ xp, int nb, float* __restrict__ y, int64_t ldy) {
+  constexpr int P = dq_pitch<kInterleaved>();
+  constexpr int kStageBytes = 16 * P;
+  __shared__ __align__(16) uint8_t ring[kDqWarps][kDqStages][kStageBytes];
+  __shared__ float red[kDqWarps][16][9];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int64_t r0 = (int64_t)blockIdx.x * 16;
+  // rows past the end read the last row (valid memory) and are not stored
+  const int64_t ra = min(r0 + g, rows - 1), rb = min(r0 + g + 8, rows - 1);
+  const int64_t wpr = n / 8;
+  const uint32_t* pa = packed + ra * wpr;
+  const uint32_t* pb = packed + rb * wpr;
+  const float* sa = scales + ra * G;
+  const float* sb = scales + rb * G;
+  const uint8_t* za_row = zeros + ra * G;
+  const uint8_t* zb_row = zeros + rb * G;
+  // vector slots past nb repeat a real vector; their outputs are not stored
+  const __nv_bfloat16* xr = xp + (int64_t)(g % nb) * n;
+  const int nblk = (int)(n / 32), nsl = (nblk + 3) / 4, nfull = nblk / 4;
+  const int per = (nsl + kDqSplit - 1) / kDqSplit;
+  const int s_lo = (int)blockIdx.y * per, s_hi = min(nsl, s_lo + per);
+  // this warp's slices: first + k kDqWarps, k = 0 .. K - 1
+  const int first = s_lo + warp;
+  const int K = first < s_hi ? (s_hi - first + kDqWarps - 1) / kDqWarps : 0;
+  uint8_t* myring = &ring[warp][0][0];
+  // each thread stages its own 16 bytes of rows g and g + 8 per slice
+  auto issue = [&](int k) {
+    if (k < K) {
+      const int blk = 4 * (first + k * kDqWarps) + t;
+      if (blk < nblk) {
+        uint8_t* st = myring + (k % kDqStages) * kStageBytes;
+        ptx::cp_async_16(st + g * P + 16 * t, pa + 4 * blk);
+        ptx::cp_async_16(st + (g + 8) * P + 16 * t, pb + 4 * blk);
+      }
+    }
+    ptx::cp_async_commit();
+  };
+  auto side = [&](DqSide<kInterleaved>& d, int k) {
+    const int s = first + k * kDqWarps;
+    if (s < nfull)
+      dq_side<kInterleaved, true>(d, s, nblk, t, gshift, xr, sa, sb, za_row, zb_row);
+    else
+      dq_side<kInterleaved, false>(d, s, nblk, t, gshift, xr, sa, sb, za_row, zb_row);
+  };
+#pragma unroll
+  for (int k = 0; k < kDqStages - 1; ++k) issue(k);
+  float Y[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int k = 0; k < K; ++k) {
+    if (kInterleaved) __syncwarp();  // every lane is done with the slot refilled next
+    issue(k + kDqStages - 1);
+    ptx::cp_async_wait<kDqStages - 1>();  // slice k has landed (this thread's part)
+    if (kInterleaved) __syncwarp();       // ... and every other lane's part
+    DqSide<kInterleaved> cur;
+    side(cur, k);
+    dq_slice<kInterleaved>(Y, myring + (k % kDqStages) * kStageBytes, cur, g, t);
+  }
+  ptx::cp_async_wait<0>();
+  red[warp][g][2 * t] = Y[0];
+  red[warp][g][2 * t + 1] = Y[1];
+  red[warp][g + 8][2 * t] = Y[2];
+  red[warp][g + 8][2 * t + 1] = Y[3];
+  __syncthreads();
+  for (int i = threadIdx.x; i < 128; i += kDqWarps * 32) {
+    const int b = i >> 4, rr = i & 15;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDqWarps; ++w) v += red[w][rr][b];
+    if (b < nb && r0 + rr < rows) atomicAdd(y + (int64_t)b * ldy + r0 + rr, v);
+  }
+}
+
+// xp[b][8w + 2i] = x[b][c(8w + i)], xp[b][8w + 2i + 1] = x[b][c(8w + i + 4)]
+// (i = 0..3) with c(k) = perm[k] (sweep order) or k; and y[0 .. ny) = 0.
+__global__ void dq_prep_kernel(const __nv_bfloat16* __restrict__ x, int64_t n, int64_t nwords,
+                               const int32_t* __restrict__ perm, __nv_bfloat16* __restrict__ xp,
+                               float* __restrict__ y, int64_t ny) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nwords; i += stride) {
+    const int64_t b = i / (n / 8), w = i % (n / 8);
+    const __nv_bfloat16* xb = x + b * n;
+    __align__(16) __nv_bfloat16 o[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int64_t c0 = 8 * w + k, c1 = 8 * w + k + 4;
+      o[2 * k] = xb[perm ? perm[c0] : c0];
+      o[2 * k + 1] = xb[perm ? perm[c1] : c1];
+    }
+    *reinterpret_cast<uint4*>(xp + b * n + 8 * w) = *reinterpret_cast<const uint4*>(o);
+  }
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < ny; i += stride) y[i] = 0.f;
+}
+
 template <int BITS, int B>
 void mv_launch(const uint32_t* packed, int64_t rows, int64_t n, const float* scales,
                const uint8_t* zeros, int group_size, int64_t G, const int32_t* g_idx,
@@ -443,6 +701,47 @@ cudaError_t launch_dequant_matvec(const uint32_t* packed, int bits, int64_t rows
                                   const void* x, int x_bf16, int64_t batch, float* y,
                                   cudaStream_t s) {
   if (rows == 0 || batch == 0) return cudaSuccess;
+  // the tensor-core path: int4, bf16 activations, groups that are runs of
+  // 32 k consecutive columns, 16-byte aligned code rows and activations
+  // group sizes: one per row, or a power of two >= 32 (a shift finds the group)
+  const bool pow2 = group_size >= 32 && (group_size & (group_size - 1)) == 0;
+  const bool mma = bits == 4 && x_bf16 && !g_idx && n % 32 == 0 && (group_size <= 0 || pow2) &&
+                   reinterpret_cast<uintptr_t>(packed) % 16 == 0;
+  if (mma) {
+    // x in MMA pair order (and sweep order under perm) in stream-ordered scratch
+    cudaMemPool_t pool;
+    if (!scratch_pool(&pool)) return cudaErrorMemoryAllocation;
+    __nv_bfloat16* xp = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&xp),
+                                            (size_t)batch * (size_t)n * sizeof(__nv_bfloat16),
+                                            pool, s);
+    if (e != cudaSuccess) return e;
+    const int64_t nwords = batch * (n / 8), ny = batch * rows;
+    const int64_t work = std::max(nwords, ny);
+    const unsigned pgrid = (unsigned)std::min<int64_t>((work + 255) / 256, (int64_t)num_sms() * 8);
+    dq_prep_kernel<<<pgrid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), n, nwords, perm,
+                                         xp, y, ny);
+    note_launch();
+    const bool inter = group_size > 0 && group_size < 128;
+    int gshift = 31;
+    if (group_size > 0)
+      for (gshift = 0; (1 << gshift) < group_size; ++gshift) {
+      }
+    const dim3 grid((unsigned)((rows + 15) / 16), kDqSplit);
+    for (int64_t b0 = 0; b0 < batch; b0 += 8) {
+      const int nb = (int)(batch - b0 < 8 ? batch - b0 : 8);
+      if (inter)
+        dequant_mma_int4_kernel<true><<<grid, kDqWarps * 32, 0, s>>>(
+            packed, rows, n, scales, zeros, gshift, n_groups, xp + b0 * n, nb, y + b0 * rows, rows);
+      else
+        dequant_mma_int4_kernel<false><<<grid, kDqWarps * 32, 0, s>>>(
+            packed, rows, n, scales, zeros, gshift, n_groups, xp + b0 * n, nb, y + b0 * rows, rows);
+      note_launch();
+    }
+    e = cudaGetLastError();
+    const cudaError_t f = cudaFreeAsync(xp, s);
+    return e != cudaSuccess ? e : f;
+  }
   const size_t esz = x_bf16 ? 2 : 4;
   // batches of 8, 4, 2, 1 vectors per launch
   for (int64_t b0 = 0; b0 < batch;) {

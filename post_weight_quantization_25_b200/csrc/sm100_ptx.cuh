@@ -83,6 +83,14 @@ __device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gmem_src,
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// until at most N of this thread's committed cp.async groups are pending
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
@@ -120,6 +128,20 @@ __device__ __forceinline__ void bulk_wait_read0() {
 // until this thread's committed bulk groups have completed
 __device__ __forceinline__ void bulk_wait_all0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Contiguous bulk copy global -> this CTA's shared memory, completing on
+// `bar` (both addresses 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(smem_dst)),
+      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+// barrier `id` (1..15) over `threads` threads of the CTA
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 // generic-proxy writes to shared memory become visible to the async proxy
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -51,9 +51,7 @@ def test_pack_and_dequant_bit_exact(bits, rows, n, g, use_gidx):
     (4, 130, 1032, -1, False, 8, torch.bfloat16), (3, 9, 96, 32, False, 2, torch.float32),
     (3, 17, 2080, 128, True, 11, torch.bfloat16), (4, 1, 8, -1, False, 1, torch.float32)])
 def test_dequant_matvec_matches_oracle(bits, rows, n, g, use_gidx, batch, xdt):
-    """y = x w_hat^T with w_hat dequantized on the fly.  Bound: each lane sums
-    n/32 terms in fp32 and five shuffle levels follow, so the error is at
-    most (n/32 + 5) 2^-24 sum|w_hat x| to first order (doubled here)."""
+    """y = x w_hat^T with w_hat dequantized on the fly, within mv_bound."""
     rng = np.random.default_rng(bits * 7 + n + batch)
     codes = rng.integers(0, 2 ** bits, (rows, n))
     G_ = 1 if g <= 0 else (n + g - 1) // g
@@ -69,7 +67,56 @@ def test_dequant_matvec_matches_oracle(bits, rows, n, g, use_gidx, batch, xdt):
     ref_packed = O.pack_int4(codes) if bits == 4 else O.pack_int3(codes)
     yo, mag = O.dequant_matvec(ref_packed, bits, n, scales, zeros, x.float().numpy(), g, gidx)
     err = np.abs(y.cpu().numpy().astype(np.float64) - yo)
-    bound = 2 * (n / 32 + 5) * 2.0 ** -24 * mag + 1e-30
+    bound = mv_bound(n, mag)
+    assert np.all(err <= bound), float(np.max(err / bound))
+
+
+def mv_bound(n, mag):
+    """Rounding bound of gptq_dequant_matvec against the fp64 product with
+    binary32 w_hat.  FP32-pipe kernel: each lane sums n/32 rounded FMA terms,
+    then five shuffle levels.  Tensor-core kernel (int4, bf16 x): the products
+    (q - zero) x are exact; at most 8 MMA accumulations of 16 products per
+    128-column slice (<= 16 roundings, internal order unknown), one FMA by the
+    scale, n/512 slice sums per warp, 3 levels over 8 warps, plus one rounding
+    for scale (q - zero) versus the binary32 w_hat.  Both depths are below
+    n/32 + 24; the bound doubles that first-order figure."""
+    return 2 * (n / 32 + 24) * 2.0 ** -24 * mag + 1e-30
+
+
+@pytest.mark.parametrize("rows,n,g,batch,use_perm", [
+    (33, 1056, 32, 3, False), (100, 2048, 128, 8, True), (16, 4096, -1, 1, False),
+    (5, 96, 32, 9, True), (47, 640, 64, 2, False), (18, 1024, 256, 5, False),
+    (257, 4224, 128, 1, True)])
+def test_dequant_matvec_tensor_core_path(rows, n, g, batch, use_perm):
+    """int4 codes x bf16 activations with contiguous groups run on the MMA
+    kernel: one prep launch (x in pair / sweep order, y zeroed), then one
+    launch per 8 vectors.
+    Ragged row tiles (rows % 16), partial 128-column slices (n % 128), group
+    sizes 32 / 64 (per-block scales), 128 / 256 / per row (per-slice scales),
+    batches past 8, and extreme codes against extreme zero points."""
+    rng = np.random.default_rng(rows * 31 + n + batch)
+    codes = rng.integers(0, 16, (rows, n))
+    codes[0, : n // 2] = 15
+    codes[-1, : n // 3] = 0
+    G_ = 1 if g <= 0 else n // g
+    scales = rng.uniform(1e-4, 0.2, (rows, G_)).astype(np.float32)
+    zeros = rng.integers(0, 16, (rows, G_))
+    zeros[0, :] = 0
+    zeros[-1, :] = 15
+    perm = rng.permutation(n) if use_perm else None
+    packed = G.gptq_pack_int4(torch.from_numpy(codes.astype(np.uint8)).cuda())
+    x = torch.randn(batch, n, generator=torch.Generator().manual_seed(rows)).to(torch.bfloat16)
+    before = G.gptq_launch_count()
+    y = G.gptq_dequant_matvec(packed, 4, n, torch.from_numpy(scales).cuda(),
+                              torch.from_numpy(zeros.astype(np.uint8)).cuda(), x.cuda(), g,
+                              perm=torch.from_numpy(perm.astype(np.int32)).cuda()
+                              if use_perm else None)
+    torch.cuda.synchronize()
+    assert G.gptq_launch_count() - before == 1 + (batch + 7) // 8  # x prep + one per 8 vectors
+    yo, mag = O.dequant_matvec(O.pack_int4(codes), 4, n, scales, zeros, x.float().numpy(), g,
+                               perm=perm)
+    err = np.abs(y.cpu().numpy().astype(np.float64) - yo)
+    bound = mv_bound(n, mag)
     assert np.all(err <= bound), float(np.max(err / bound))
 
 
@@ -98,7 +145,7 @@ def test_dequant_matvec_in_sweep_order(bits, rows, n, g, batch):
     ref_sw = O.pack_int4(codes[:, perm]) if bits == 4 else O.pack_int3(codes[:, perm])
     yo, mag = O.dequant_matvec(ref_sw, bits, n, scales, zeros, x.float().numpy(), g, perm=perm)
     err = np.abs(y.cpu().numpy().astype(np.float64) - yo)
-    assert np.all(err <= 2 * (n / 32 + 5) * 2.0 ** -24 * mag + 1e-30)
+    assert np.all(err <= mv_bound(n, mag))
     # the same product in original column order with g_idx
     ref_o = O.pack_int4(codes) if bits == 4 else O.pack_int3(codes)
     yo2, _ = O.dequant_matvec(ref_o, bits, n, scales, zeros, x.float().numpy(), g, gidx)
