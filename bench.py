@@ -296,6 +296,57 @@ def measure_dequant_matvec(G, dev, packed, bits, n, scales, zeros, group_size, g
             "frac": round(gbs / pk["hbm_gbs"], 4), "l2": "flushed (256 MiB read) before each launch"}
 
 
+def measure_hadamard(G, dev, iters=10):
+    """Device time of the random-sign Hadamard rotation (blocks of 1024) of
+    the 70B down-proj workload's operands, in place: X 28672 x 16384 tokens
+    and W 8192 x 28672, both bf16 (each larger than L2, so no flush);
+    bytes = one read and one write of every element."""
+    import torch
+    out = []
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5)
+    s = (torch.randint(0, 2, (28672,), generator=gen, device=dev) * 2 - 1).float()
+    for what, shape in (("X (cols)", (28672, 16384)), ("W (rows)", (8192, 28672))):
+        A = torch.randn(*shape, generator=gen, device=dev).to(torch.bfloat16)
+        fn = G.gptq_hadamard_cols if what.startswith("X") else G.gptq_hadamard_rows
+        ts = []
+        for i in range(iters + 3):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn(A, s, 1024, out=A)
+            b.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts.append(a.elapsed_time(b))
+        t = statistics.median(ts) / 1e3
+        nbytes = 2 * A.numel() * 2
+        pk = peaks()
+        line = {"operand": f"{what} {shape[0]}x{shape[1]} bf16, in place", "us": round(t * 1e6, 1),
+                "bytes": nbytes, "gbs": round(nbytes / t / 1e9, 1), "peak_gbs": pk["hbm_gbs"],
+                "frac": round(nbytes / t / 1e9 / pk["hbm_gbs"], 4)}
+        if what.startswith("W"):
+            # the same rotation as fp32 matrix products (28 blocks), for context
+            H = torch.ones(1, 1, device=dev)
+            while H.shape[0] < 1024:
+                H = torch.cat([torch.cat([H, H], 1), torch.cat([H, -H], 1)], 0)
+            H = H / 32
+            Wf = A.float()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            for k in range(28):
+                sl = slice(1024 * k, 1024 * (k + 1))
+                A[:, sl] = ((Wf[:, sl] * s[None, sl]) @ H.T).to(torch.bfloat16)
+            b.record()
+            torch.cuda.synchronize()
+            line["fp32_matmul_us"] = round(a.elapsed_time(b) * 1e3, 1)
+            del Wf, H
+        out.append(line)
+        del A
+    return out
+
+
 # ----------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -415,7 +466,7 @@ def run_ours(args, rank, world, local_rank):
                 ts.append(a.elapsed_time(b))
         rd = pk7.numel() * 4 / (statistics.median(ts) / 1e3) / 1e9
         del flush
-        nxt = {"dequant_matvec": mv,
+        nxt = {"dequant_matvec": mv, "hadamard_rotation": measure_hadamard(G, dev),
                "stream_read_117MB_gbs": round(rd, 1),
                "stream_read_note": "torch fp32 sum over the bytes of the 8192x28672 int4 codes "
                                    "(a plain read pass), same L2 flush"}

@@ -232,6 +232,32 @@ gptq_status gptq_dequant_matvec(const uint32_t* packed, int bits, int64_t rows, 
 gptq_status gptq_gather_columns_u8(const uint8_t* src, int64_t rows, int64_t n,
                                    const int32_t* perm, uint8_t* dst, void* stream);
 
+/* Random-sign blocked Hadamard rotation R = blockdiag(H_b / sqrt(b)) diag(s)
+ * (page "Post-Training Quantization: Calibration, GPTQ and Why Rotations
+ * Help", section "Rotations: making outliers disappear": rotate the
+ * activations, give the weights the inverse rotation, and the layer's product
+ * is unchanged while outliers are spread over all entries).  H_b is
+ * Sylvester's Hadamard matrix, H[i][j] = (-1)^popcount(i & j); block b is a
+ * power of two in [32, 1024] (else GPTQ_ERR_UNSUPPORTED) and divides n;
+ * signs: n floats, +1 or -1 (device).  Computed in fp32 by a fast
+ * Walsh-Hadamard transform (log2 b butterfly stages), rounded once to ot
+ * (bf16: half to even).
+ *
+ * gptq_hadamard_rows: W' = W R^T for W rows x n (row stride ld_in elements):
+ *   out[r][kb + j] = (1/sqrt(b)) sum_i H_b[j][i] s[kb + i] in[r][kb + i].
+ * gptq_hadamard_cols: X' = R X for X n x ntok (row stride ld_in elements):
+ *   out[kb + j][t] = (1/sqrt(b)) sum_i H_b[j][i] s[kb + i] in[kb + i][t].
+ * in / out: device pointers of type it / ot (GPTQ_BF16 or GPTQ_F32), either
+ * the same buffer (same type and stride: in place) or non-overlapping; the
+ * caller owns both.  Strides must cover a row (ld >= n, resp. ntok).  Zero
+ * rows or tokens: nothing is done. */
+gptq_status gptq_hadamard_rows(const void* in, gptq_dtype it, int64_t rows, int64_t n,
+                               int64_t ld_in, const float* signs, int block, void* out,
+                               gptq_dtype ot, int64_t ld_out, void* stream);
+gptq_status gptq_hadamard_cols(const void* in, gptq_dtype it, int64_t n, int64_t ntok,
+                               int64_t ld_in, const float* signs, int block, void* out,
+                               gptq_dtype ot, int64_t ld_out, void* stream);
+
 /* Static string for a status code (host). */
 const char* gptq_status_string(int status);
 

@@ -257,6 +257,38 @@ def gptq_dequant_matvec(packed: torch.Tensor, bits: int, n: int, scales: torch.T
     return out.reshape(-1) if x.dim() == 1 else out
 
 
+def _hadamard(cols: bool, x: torch.Tensor, signs: torch.Tensor, block: int, out, out_dtype,
+              stream):
+    _need_cuda(x, signs)
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise GptqError("x must be a 2-D tensor with contiguous rows")
+    if signs.dtype != torch.float32 or not signs.is_contiguous():
+        raise GptqError("signs must be a contiguous float32 tensor")
+    a, b = x.shape
+    if out is None:
+        out = torch.empty(a, b, dtype=out_dtype or x.dtype, device=x.device)
+    if out.dim() != 2 or out.shape != x.shape or out.stride(1) != 1:
+        raise GptqError("out must match x, with contiguous rows")
+    fn = library().gptq_hadamard_cols if cols else library().gptq_hadamard_rows
+    st = fn(_p(x), _dtype_code(x.dtype), a, b, x.stride(0), _p(signs), int(block), _p(out),
+            _dtype_code(out.dtype), out.stride(0), _stream(stream))
+    _check(st, "gptq_hadamard_cols" if cols else "gptq_hadamard_rows")
+    return out
+
+
+def gptq_hadamard_rows(W: torch.Tensor, signs: torch.Tensor, block: int = 1024, out=None,
+                       out_dtype=None, stream=None) -> torch.Tensor:
+    """W' = W R^T with R = blockdiag(H_b / sqrt(b)) diag(signs), along the rows
+    of W (rows x n).  out may be W itself (in place)."""
+    return _hadamard(False, W, signs, block, out, out_dtype, stream)
+
+
+def gptq_hadamard_cols(X: torch.Tensor, signs: torch.Tensor, block: int = 1024, out=None,
+                       out_dtype=None, stream=None) -> torch.Tensor:
+    """X' = R X along the first axis of X (n x ntok).  out may be X itself."""
+    return _hadamard(True, X, signs, block, out, out_dtype, stream)
+
+
 @dataclasses.dataclass
 class QuantizedLinear:
     packed: torch.Tensor

@@ -26,7 +26,8 @@ GPTQ_OP_QUANTIZE = 2
 EXPORTS = ("gptq_workspace_size", "gptq_hessian_accumulate", "gptq_cholesky_inverse",
            "gptq_quantize_layer", "gptq_pack_int4", "gptq_pack_int3", "gptq_dequant",
            "gptq_status_string", "gptq_launch_count", "gptq_cholesky_inverse_noalloc",
-           "gptq_selftest_division", "gptq_dequant_matvec", "gptq_gather_columns_u8")
+           "gptq_selftest_division", "gptq_dequant_matvec", "gptq_gather_columns_u8",
+           "gptq_hadamard_rows", "gptq_hadamard_cols")
 
 
 class GptqConfig(ctypes.Structure):
@@ -60,6 +61,8 @@ _SIGNATURES = {
     "gptq_dequant_matvec": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _int, _i64, _vp, _vp, _vp,
                                    _int, _i64, _vp, _vp]),
     "gptq_gather_columns_u8": (_int, [_vp, _i64, _i64, _vp, _vp, _vp]),
+    "gptq_hadamard_rows": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _int, _vp, _int, _i64, _vp]),
+    "gptq_hadamard_cols": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _int, _vp, _int, _i64, _vp]),
 }
 
 _LIB = None

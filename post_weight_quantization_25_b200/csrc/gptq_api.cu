@@ -319,4 +319,36 @@ gptq_status gptq_gather_columns_u8(const uint8_t* src, int64_t rows, int64_t n,
                                                     static_cast<cudaStream_t>(stream)));
 }
 
+static gptq_status hadamard_common(bool cols, const void* in, gptq_dtype it, int64_t a,
+                                   int64_t b, int64_t n, int64_t ld_in, const float* signs,
+                                   int block, void* out, gptq_dtype ot, int64_t ld_out,
+                                   void* stream) {
+  if (block < 32 || block > 1024 || (block & (block - 1))) return GPTQ_ERR_UNSUPPORTED;
+  if ((it != GPTQ_BF16 && it != GPTQ_F32) || (ot != GPTQ_BF16 && ot != GPTQ_F32))
+    return GPTQ_ERR_INVALID_ARG;
+  if (a < 0 || b < 0 || n <= 0 || n % block) return GPTQ_ERR_INVALID_ARG;
+  const int64_t inner = cols ? b : n;  // contiguous extent of a row
+  if (ld_in < inner || ld_out < inner) return GPTQ_ERR_INVALID_ARG;
+  if (a == 0 || b == 0) return GPTQ_OK;
+  if (!in || !out || !signs || !aligned(signs, 4) || !aligned(in, it == GPTQ_BF16 ? 2 : 4) ||
+      !aligned(out, ot == GPTQ_BF16 ? 2 : 4))
+    return GPTQ_ERR_INVALID_ARG;
+  if (in == out && (it != ot || ld_in != ld_out)) return GPTQ_ERR_INVALID_ARG;
+  return cuda_status(gptq::launch_hadamard(cols, block, it == GPTQ_BF16, ot == GPTQ_BF16, in,
+                                           ld_in, out, ld_out, a, b, signs,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+gptq_status gptq_hadamard_rows(const void* in, gptq_dtype it, int64_t rows, int64_t n,
+                               int64_t ld_in, const float* signs, int block, void* out,
+                               gptq_dtype ot, int64_t ld_out, void* stream) {
+  return hadamard_common(false, in, it, rows, n, n, ld_in, signs, block, out, ot, ld_out, stream);
+}
+
+gptq_status gptq_hadamard_cols(const void* in, gptq_dtype it, int64_t n, int64_t ntok,
+                               int64_t ld_in, const float* signs, int block, void* out,
+                               gptq_dtype ot, int64_t ld_out, void* stream) {
+  return hadamard_common(true, in, it, n, ntok, n, ld_in, signs, block, out, ot, ld_out, stream);
+}
+
 }  // extern "C"

@@ -84,6 +84,15 @@ cudaError_t launch_dequant_matvec(const uint32_t* packed, int bits, int64_t rows
 // dst[r][k] = src[r][perm[k]] (rows x n bytes)
 cudaError_t launch_gather_columns_u8(const uint8_t* src, int64_t rows, int64_t n,
                                      const int32_t* perm, uint8_t* dst, cudaStream_t s);
+
+// ---- Hadamard rotation (hadamard.cu)
+// cols = false: out[r][c0 + j] = (1/sqrt(b)) sum_i H_b[j][i] s[c0 + i] in[r][c0 + i]
+//               for a = rows, b_ = n (row stride ld_in / ld_out elements);
+// cols = true:  the same along the first axis of an n x ntok matrix (a = n,
+//               b_ = ntok).  block in {32, ..., 1024}, n % block == 0.
+cudaError_t launch_hadamard(bool cols, int block, int in_bf16, int out_bf16, const void* in,
+                            int64_t ld_in, void* out, int64_t ld_out, int64_t a, int64_t b_,
+                            const float* signs, cudaStream_t s);
 cudaError_t launch_dequant(const uint32_t* packed, int bits, int64_t rows, int64_t n,
                            const float* scales, const uint8_t* zeros, int group_size,
                            int64_t n_groups, const int32_t* g_idx, void* out, int out_bf16,

@@ -1,0 +1,189 @@
+// Random-sign blocked Hadamard rotation (fast Walsh-Hadamard transform).
+//
+// Page "Post-Training Quantization: Calibration, GPTQ and Why Rotations Help",
+// section "Rotations: making outliers disappear": a Hadamard matrix scaled to
+// a rotation spreads one large entry over all entries; the activations get
+// the rotation and the weights its inverse, so the layer's product is
+// unchanged.  Here R = blockdiag(H_b / sqrt(b)) diag(s) with Sylvester's H_b
+// (b a power of two, 32 <= b <= 1024) and per-feature signs s: X' = R X acts
+// on the columns of X (features x tokens), W' = W R^T on the rows of W.
+//
+// Both are HBM-bound passes (one read, one write per element); the transform
+// itself is log2(b) butterfly stages in fp32 registers, never a matrix
+// product.  A warp holds one block of b = 32 VPL values, lane l holding
+// elements l + 32 i: the stages over the high index bits (strides 32 .. b/2)
+// run inside each lane, the five over the low bits (strides 1 .. 16) through
+// shfl_xor.  The order of butterfly stages does not change the result's
+// definition (they commute), only the fp32 rounding.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "gptq_internal.cuh"
+
+namespace gptq {
+namespace {
+
+__device__ __forceinline__ float to_f(const float* p) { return *p; }
+__device__ __forceinline__ float to_f(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+__device__ __forceinline__ void from_f(float* p, float v) { *p = v; }
+__device__ __forceinline__ void from_f(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+
+template <int VPL>
+__device__ __forceinline__ void fwht_warp(float (&v)[VPL], int lane) {
+#pragma unroll
+  for (int h = 1; h < VPL; h <<= 1)
+#pragma unroll
+    for (int i = 0; i < VPL; ++i)
+      if ((i & h) == 0) {
+        const float a = v[i], b = v[i + h];
+        v[i] = a + b;
+        v[i + h] = a - b;
+      }
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1)
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const float o = __shfl_xor_sync(0xffffffffu, v[i], m);
+      v[i] = (lane & m) ? o - v[i] : v[i] + o;
+    }
+}
+
+// W' = W R^T: each row's blocks of b contiguous elements, one warp per block
+// (in == out is allowed: a warp reads its whole block before writing it).
+constexpr int kRowsWarps = 8;
+
+// X' = R X: a CTA stages b features x kColsTok tokens in shared memory
+// (pitch kColsTok + 1 floats: the row loads, and the column reads of the
+// warps, each land on distinct banks), then warp w transforms token column w
+// (in == out is allowed: the tile is read in full before it is written).
+constexpr int kColsTok = 16;
+
+template <int VPL, typename TI, typename TO>
+__global__ void __launch_bounds__(kColsTok * 32) hadamard_cols_kernel(
+    const TI* in, int64_t ld_in, TO* out, int64_t ld_out, int64_t ntok,
+    const float* __restrict__ signs, float scale, int vec_in, int vec_out) {
+  constexpr int B = 32 * VPL, P = kColsTok + 1, NT = kColsTok * 32;
+  constexpr int VI = 16 / (int)sizeof(TI), VO = 16 / (int)sizeof(TO);  // per 16 bytes
+  extern __shared__ float tile[];  // B x P
+  const int64_t f0 = (int64_t)blockIdx.y * B, t0 = (int64_t)blockIdx.x * kColsTok;
+  const int tt = (int)(ntok - t0 < kColsTok ? ntok - t0 : kColsTok);
+  const int tid = threadIdx.x;
+  if (vec_in && tt == kColsTok) {
+    // 16-byte loads: thread -> (feature row, vector of VI tokens)
+    constexpr int kPer = kColsTok / VI;
+    for (int idx = tid; idx < B * kPer; idx += NT) {
+      const int f = idx / kPer, c = idx % kPer;
+      const uint4 raw = *reinterpret_cast<const uint4*>(in + (f0 + f) * ld_in + t0 + c * VI);
+      const TI* e = reinterpret_cast<const TI*>(&raw);
+      const float sg = __ldg(signs + f0 + f);
+#pragma unroll
+      for (int j = 0; j < VI; ++j) tile[f * P + c * VI + j] = to_f(e + j) * sg;
+    }
+  } else {
+    const int tc = tid % kColsTok, fr = tid / kColsTok;
+    for (int f = fr; f < B; f += NT / kColsTok) {
+      const float sg = __ldg(signs + f0 + f);
+      tile[f * P + tc] = tc < tt ? to_f(in + (f0 + f) * ld_in + t0 + tc) * sg : 0.f;
+    }
+  }
+  __syncthreads();
+  const int w = tid >> 5, lane = tid & 31;
+  float v[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) v[i] = tile[(lane + 32 * i) * P + w];
+  fwht_warp<VPL>(v, lane);
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) tile[(lane + 32 * i) * P + w] = v[i] * scale;
+  __syncthreads();
+  if (vec_out && tt == kColsTok) {
+    constexpr int kPer = kColsTok / VO;
+    for (int idx = tid; idx < B * kPer; idx += NT) {
+      const int f = idx / kPer, c = idx % kPer;
+      uint4 raw;
+      TO* e = reinterpret_cast<TO*>(&raw);
+#pragma unroll
+      for (int j = 0; j < VO; ++j) from_f(e + j, tile[f * P + c * VO + j]);
+      *reinterpret_cast<uint4*>(out + (f0 + f) * ld_out + t0 + c * VO) = raw;
+    }
+  } else {
+    const int tc = tid % kColsTok, fr = tid / kColsTok;
+    for (int f = fr; f < B; f += NT / kColsTok)
+      if (tc < tt) from_f(out + (f0 + f) * ld_out + t0 + tc, tile[f * P + tc]);
+  }
+}
+
+unsigned cdiv(int64_t a, int64_t b) { return (unsigned)((a + b - 1) / b); }
+
+template <int VPL, typename TI, typename TO>
+cudaError_t rows_launch(const void* in, int64_t ld_in, void* out, int64_t ld_out, int64_t rows,
+                        int64_t n, const float* signs, float scale, cudaStream_t s) {
+  const int64_t nblk = n / (32 * VPL);
+  hadamard_rows_kernel<VPL, TI, TO><<<cdiv(rows * nblk, kRowsWarps), kRowsWarps * 32, 0, s>>>(
+      static_cast<const TI*>(in), ld_in, static_cast<TO*>(out), ld_out, rows, nblk, signs, scale);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <int VPL, typename TI, typename TO>
+cudaError_t cols_launch(const void* in, int64_t ld_in, void* out, int64_t ld_out, int64_t n,
+                        int64_t ntok, const float* signs, float scale, cudaStream_t s) {
+  constexpr int B = 32 * VPL;
+  const size_t smem = (size_t)B * (kColsTok + 1) * sizeof(float);
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(hadamard_cols_kernel<VPL, TI, TO>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  // 16-byte row pieces when every tile's token start is 16-byte aligned
+  const int vec_in = (reinterpret_cast<uintptr_t>(in) % 16 == 0) &&
+                     ((size_t)ld_in * sizeof(TI)) % 16 == 0;
+  const int vec_out = (reinterpret_cast<uintptr_t>(out) % 16 == 0) &&
+                      ((size_t)ld_out * sizeof(TO)) % 16 == 0;
+  const dim3 grid(cdiv(ntok, kColsTok), (unsigned)(n / B));
+  hadamard_cols_kernel<VPL, TI, TO><<<grid, kColsTok * 32, smem, s>>>(
+      static_cast<const TI*>(in), ld_in, static_cast<TO*>(out), ld_out, ntok, signs, scale,
+      vec_in, vec_out);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <int VPL>
+cudaError_t dispatch(bool cols, int in_bf16, int out_bf16, const void* in, int64_t ld_in,
+                     void* out, int64_t ld_out, int64_t a, int64_t b, const float* signs,
+                     float scale, cudaStream_t s) {
+  using BF = __nv_bfloat16;
+  if (cols) {
+    if (in_bf16 && out_bf16) return cols_launch<VPL, BF, BF>(in, ld_in, out, ld_out, a, b, signs, scale, s);
+    if (in_bf16) return cols_launch<VPL, BF, float>(in, ld_in, out, ld_out, a, b, signs, scale, s);
+    if (out_bf16) return cols_launch<VPL, float, BF>(in, ld_in, out, ld_out, a, b, signs, scale, s);
+    return cols_launch<VPL, float, float>(in, ld_in, out, ld_out, a, b, signs, scale, s);
+  }
+  if (in_bf16 && out_bf16) return rows_launch<VPL, BF, BF>(in, ld_in, out, ld_out, a, b, signs, scale, s);
+  if (in_bf16) return rows_launch<VPL, BF, float>(in, ld_in, out, ld_out, a, b, signs, scale, s);
+  if (out_bf16) return rows_launch<VPL, float, BF>(in, ld_in, out, ld_out, a, b, signs, scale, s);
+  return rows_launch<VPL, float, float>(in, ld_in, out, ld_out, a, b, signs, scale, s);
+}
+
+}  // namespace
+
+cudaError_t launch_hadamard(bool cols, int block, int in_bf16, int out_bf16, const void* in,
+                            int64_t ld_in, void* out, int64_t ld_out, int64_t a, int64_t b,
+                            const float* signs, cudaStream_t s) {
+  // 1 / sqrt(block): exact for block = 4^k (a power of two), else rounded
+  const float scale = (float)(1.0 / std::sqrt((double)block));
+  switch (block) {
+    case 32: return dispatch<1>(cols, in_bf16, out_bf16, in, ld_in, out, ld_out, a, b, signs, scale, s);
+    case 64: return dispatch<2>(cols, in_bf16, out_bf16, in, ld_in, out, ld_out, a, b, signs, scale, s);
+    case 128: return dispatch<4>(cols, in_bf16, out_bf16, in, ld_in, out, ld_out, a, b, signs, scale, s);
+    case 256: return dispatch<8>(cols, in_bf16, out_bf16, in, ld_in, out, ld_out, a, b, signs, scale, s);
+    case 512: return dispatch<16>(cols, in_bf16, out_bf16, in, ld_in, out, ld_out, a, b, signs, scale, s);
+    case 1024: return dispatch<32>(cols, in_bf16, out_bf16, in, ld_in, out, ld_out, a, b, signs, scale, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace gptq

@@ -101,3 +101,21 @@ def test_argument_checks_reject_before_any_launch(lib):
     assert lib.gptq_pack_int3(None, 4, 40, None, None) == 1                   # n % 32
     assert lib.gptq_pack_int4(None, 0, 16, None, None) == 0                   # empty
     assert lib.gptq_dequant(None, 5, 4, 16, None, None, -1, 1, None, None, 0, None) == 2
+
+
+def test_hadamard_argument_checks(lib):
+    """Rejected before any device work: block not a power of two in
+    [32, 1024], n not a multiple of the block, strides shorter than a row,
+    in place with a different type; zero rows is a no-op."""
+    p = ctypes.c_void_p(0x1000)
+    UNSUP, INVAL = 2, 1
+    assert lib.gptq_hadamard_rows(p, 0, 4, 1024, 1024, p, 48, p, 0, 1024, None) == UNSUP
+    assert lib.gptq_hadamard_rows(p, 0, 4, 1024, 1024, p, 2048, p, 0, 1024, None) == UNSUP
+    assert lib.gptq_hadamard_rows(p, 0, 4, 1024, 1024, p, 16, p, 0, 1024, None) == UNSUP
+    assert lib.gptq_hadamard_rows(p, 0, 4, 1000, 1000, p, 32, p, 0, 1000, None) == INVAL
+    assert lib.gptq_hadamard_rows(p, 0, 4, 1024, 512, p, 1024, p, 0, 1024, None) == INVAL
+    assert lib.gptq_hadamard_cols(p, 0, 1024, 16, 8, p, 1024, p, 0, 16, None) == INVAL
+    assert lib.gptq_hadamard_cols(p, 0, 1024, 16, 16, p, 1024, p, 1, 16, None) == INVAL
+    assert lib.gptq_hadamard_rows(p, 2, 4, 1024, 1024, p, 1024, p, 0, 1024, None) == INVAL
+    assert lib.gptq_hadamard_rows(p, 0, 0, 1024, 1024, p, 1024, p, 0, 1024, None) == 0
+    assert lib.gptq_hadamard_cols(p, 0, 1024, 0, 0, p, 1024, p, 0, 0, None) == 0
