@@ -55,6 +55,24 @@ __device__ __forceinline__ void fwht_warp(float (&v)[VPL], int lane) {
 // (in == out is allowed: a warp reads its whole block before writing it).
 constexpr int kRowsWarps = 8;
 
+template <int VPL, typename TI, typename TO>
+__global__ void __launch_bounds__(kRowsWarps * 32) hadamard_rows_kernel(
+    const TI* in, int64_t ld_in, TO* out, int64_t ld_out, int64_t rows, int64_t nblk,
+    const float* __restrict__ signs, float scale) {
+  const int lane = threadIdx.x & 31;
+  const int64_t seg = (int64_t)blockIdx.x * kRowsWarps + (threadIdx.x >> 5);
+  if (seg >= rows * nblk) return;  // whole warps
+  const int64_t r = seg / nblk, c0 = (seg % nblk) * (32 * VPL);
+  const TI* p = in + r * ld_in + c0;
+  float v[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) v[i] = to_f(p + lane + 32 * i) * __ldg(signs + c0 + lane + 32 * i);
+  fwht_warp<VPL>(v, lane);
+  TO* q = out + r * ld_out + c0;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) from_f(q + lane + 32 * i, v[i] * scale);
+}
+
 // X' = R X: a CTA stages b features x kColsTok tokens in shared memory
 // (pitch kColsTok + 1 floats: the row loads, and the column reads of the
 // warps, each land on distinct banks), then warp w transforms token column w
