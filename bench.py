@@ -49,7 +49,10 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-next", action="store_true",
-                   help="skip the measurement of the dequant x activation kernel")
+                   help="skip the measurements of the consumer-side kernels")
+    p.add_argument("--only", choices=["dequant_matvec", "hadamard", "pipeline"], default=None,
+                   help="run one consumer-side measurement alone and print its JSON "
+                        "(for profiling; not the benchmark line)")
     return p.parse_args()
 
 
@@ -296,6 +299,60 @@ def measure_dequant_matvec(G, dev, packed, bits, n, scales, zeros, group_size, g
             "frac": round(gbs / pk["hbm_gbs"], 4), "l2": "flushed (256 MiB read) before each launch"}
 
 
+def _codes_70b(dev):
+    """Random int4 codes and rulers of the 70B down-proj shape (8192 x 28672,
+    g128) and a random act-order permutation with its g_idx."""
+    import torch
+    r7, n7 = 8192, 28672
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(77)
+    pk7 = torch.randint(-2 ** 31, 2 ** 31 - 1, (r7, n7 // 8), generator=gen, device=dev,
+                        dtype=torch.int64).to(torch.int32)
+    sc7 = torch.rand(r7, n7 // 128, generator=gen, device=dev) * 0.01 + 1e-4
+    z7 = torch.randint(0, 16, (r7, n7 // 128), generator=gen, device=dev,
+                       dtype=torch.int64).to(torch.uint8)
+    pm7 = torch.randperm(n7, generator=gen, device=dev).to(torch.int32)
+    gi7 = torch.empty_like(pm7)
+    gi7[pm7.long()] = (torch.arange(n7, device=dev, dtype=torch.int32) // 128)
+    return pk7, sc7, z7, pm7, gi7
+
+
+def measure_dequant_70b(G, dev):
+    """The fused dequant x activation on the 70B down-proj shape: codes in
+    original order with g_idx (FP32-pipe kernel) and in sweep order with perm
+    (tensor-core kernel), 1 and 8 activation vectors."""
+    pk7, sc7, z7, pm7, gi7 = _codes_70b(dev)
+    n7 = 28672
+    label7 = "8192x28672 (70B down-proj shape)"
+    out = []
+    for b in (1, 8):
+        out.append(measure_dequant_matvec(G, dev, pk7, 4, n7, sc7, z7, 128, gi7, batch=b,
+                                          label=label7))
+        out.append(measure_dequant_matvec(G, dev, pk7, 4, n7, sc7, z7, 128, None, batch=b,
+                                          label=label7, perm=pm7))
+    return out
+
+
+def stream_read_gbs(dev):
+    """A plain streaming read of the 70B shape's code bytes with the same L2
+    flush: what one pass over 117 MB reaches on this part."""
+    import torch
+    pk7 = _codes_70b(dev)[0]
+    flush = torch.zeros(64 << 20, dtype=torch.float32, device=dev)
+    ts = []
+    for i in range(13):
+        flush.sum()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        pk7.view(torch.float32).sum()
+        b.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            ts.append(a.elapsed_time(b))
+    return round(pk7.numel() * 4 / (statistics.median(ts) / 1e3) / 1e9, 1)
+
+
 def measure_hadamard(G, dev, iters=10):
     """Device time of the random-sign Hadamard rotation (blocks of 1024) of
     the 70B down-proj workload's operands, in place: X 28672 x 16384 tokens
@@ -345,6 +402,44 @@ def measure_hadamard(G, dev, iters=10):
         out.append(line)
         del A
     return out
+
+
+def measure_pipeline(G, dev, reps=3):
+    """One 7B-shaped decoder block (q, k, v, o, gate, up, down; 4-bit g128,
+    65536 tokens per linear, synthetic bf16 inputs resident on the device)
+    quantized linear after linear on one stream, and with the Hessian of
+    linear l + 1 overlapping the rest of linear l.  weights/s over the block."""
+    import torch
+    import workloads
+    shapes = [(r, n) for _, r, n in workloads.STACK_7B_LINEARS]
+    ntok = 65536
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4000)
+    Ws = [(torch.randn(r, n, generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+          for r, n in shapes]
+    Xs = [torch.randn(n, ntok, generator=gen, device=dev).to(torch.bfloat16) for _, n in shapes]
+    pipe = G.LayerPipeline(shapes, ntok, bits=4, group_size=128, device=dev)
+    nw = sum(r * n for r, n in shapes)
+    res = {"block": "7B decoder block: q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008",
+           "tokens_per_linear": ntok, "weights": nw}
+    for mode, ov in (("one_stream", False), ("overlapped", True)):
+        ts = []
+        for i in range(reps + 1):
+            torch.cuda.synchronize()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            pipe.run(Ws, Xs, overlap=ov)
+            b.record()
+            torch.cuda.synchronize()
+            if i >= 1:
+                ts.append(a.elapsed_time(b))
+        pipe.check_info()
+        t = statistics.median(ts)
+        res[mode] = {"ms": round(t, 3), "weights_per_s": round(nw / (t / 1e3), 1)}
+    res["speedup"] = round(res["one_stream"]["ms"] / res["overlapped"]["ms"], 3)
+    del pipe, Ws, Xs
+    return res
 
 
 # ----------------------------------------------------------------- our arm
@@ -433,44 +528,12 @@ def run_ours(args, rank, world, local_rank):
                                              wl.group_size, None, perm=lq.perm,
                                              label=f"{rows}x{n} (this layer)"))
             del sw, pk_sw
-        r7, n7 = 8192, 28672
-        gen = torch.Generator(device=dev)
-        gen.manual_seed(77)
-        pk7 = torch.randint(-2 ** 31, 2 ** 31 - 1, (r7, n7 // 8), generator=gen, device=dev,
-                            dtype=torch.int64).to(torch.int32)
-        sc7 = torch.rand(r7, n7 // 128, generator=gen, device=dev) * 0.01 + 1e-4
-        z7 = torch.randint(0, 16, (r7, n7 // 128), generator=gen, device=dev,
-                           dtype=torch.int64).to(torch.uint8)
-        pm7 = torch.randperm(n7, generator=gen, device=dev).to(torch.int32)
-        gi7 = torch.empty_like(pm7)
-        gi7[pm7.long()] = (torch.arange(n7, device=dev, dtype=torch.int32) // 128)
-        label7 = "8192x28672 (70B down-proj shape)"
-        for b in (1, 8):
-            mv.append(measure_dequant_matvec(G, dev, pk7, 4, n7, sc7, z7, 128, gi7, batch=b,
-                                             label=label7))
-            mv.append(measure_dequant_matvec(G, dev, pk7, 4, n7, sc7, z7, 128, None, batch=b,
-                                             label=label7, perm=pm7))
-        # a plain streaming read of the same code bytes, same flush: what
-        # one pass over 117 MB reaches on this part
-        flush = torch.zeros(64 << 20, dtype=torch.float32, device=dev)
-        ts = []
-        for i in range(13):
-            flush.sum()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record()
-            pk7.view(torch.float32).sum()
-            b.record()
-            torch.cuda.synchronize()
-            if i >= 3:
-                ts.append(a.elapsed_time(b))
-        rd = pk7.numel() * 4 / (statistics.median(ts) / 1e3) / 1e9
-        del flush
-        nxt = {"dequant_matvec": mv, "hadamard_rotation": measure_hadamard(G, dev),
-               "stream_read_117MB_gbs": round(rd, 1),
-               "stream_read_note": "torch fp32 sum over the bytes of the 8192x28672 int4 codes "
-                                   "(a plain read pass), same L2 flush"}
-        del pk7, sc7, z7, gi7, pm7
+        mv += measure_dequant_70b(G, dev)
+        nxt = {"dequant_matvec": mv, "stream_read_117MB_gbs": stream_read_gbs(dev),
+               "stream_read_note": "torch fp32 sum over 8192x28672 int4 codes' bytes "
+                                   "(a plain read pass), same L2 flush",
+               "hadamard_rotation": measure_hadamard(G, dev),
+               "layer_pipeline": measure_pipeline(G, dev)}
 
     # end to end through the same C ABI with host buffers
     e2e = None
@@ -578,6 +641,16 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.only:
+        import torch
+        import post_weight_quantization_25_b200 as G
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        if rank == 0:
+            fn = {"dequant_matvec": measure_dequant_70b, "hadamard": measure_hadamard,
+                  "pipeline": measure_pipeline}[args.only]
+            print(json.dumps({"only": args.only, "result": fn(G, dev)}), flush=True)
         return
     if world > 1:
         import torch

@@ -21,7 +21,8 @@ from . import _lib
 from ._lib import (GPTQ_BF16, GPTQ_F32, GPTQ_OP_CHOLESKY, GPTQ_OP_HESSIAN, GPTQ_OP_QUANTIZE,
                    GptqConfig)
 
-__all__ = ["GptqError", "GptqConfig", "gptq_workspace_size", "gptq_hessian_accumulate",
+__all__ = ["GptqError", "GptqConfig", "LayerPipeline", "gptq_workspace_size",
+           "gptq_hadamard_rows", "gptq_hadamard_cols", "gptq_hessian_accumulate",
            "gptq_cholesky_inverse", "gptq_quantize_layer", "gptq_pack_int4", "gptq_pack_int3",
            "gptq_dequant", "gptq_dequant_matvec", "gptq_gather_columns_u8", "gptq_status_string",
            "make_config",
@@ -390,6 +391,37 @@ class LayerQuantizer:
                                                    self.cfg), dev, None)
         self._pack = gptq_pack_int4 if bits == 4 else gptq_pack_int3
 
+    def hessian(self, X: torch.Tensor, stream, mark=None) -> None:
+        """H = 0, H += 2 X X^T on `stream`; mark(0) / mark(1) around the
+        accumulation."""
+        with torch.cuda.stream(stream):
+            self.H.zero_()
+        if mark:
+            mark(0)
+        gptq_hessian_accumulate(self.H, X, 2.0, ws=self.ws_h, info=self.info_h, stream=stream)
+        if mark:
+            mark(1)
+
+    def finish(self, W: torch.Tensor, stream, mark=None) -> None:
+        """Everything after the Hessian, on `stream`: U, the sweep, packing,
+        dequantization.  mark(i) is called after stage i (2..5)."""
+        gptq_cholesky_inverse(self.H, self.percdamp, self.actorder, self.U, self.perm, self.dead,
+                              self.info, ws=self.ws_c, stream=stream)
+        if mark:
+            mark(2)
+        gptq_quantize_layer(W, self.U, self.perm, self.dead, self.cfg, self.codes, self.scales,
+                            self.zeros, self.g_idx, self.Wq, self.row_loss, ws=self.ws_q,
+                            stream=stream)
+        if mark:
+            mark(3)
+        self._pack(self.codes, self.packed, stream=stream)
+        if mark:
+            mark(4)
+        gptq_dequant(self.packed, self.bits, self.n, self.scales, self.zeros, self.group_size,
+                     self.g_idx, self.deq.dtype, out=self.deq, stream=stream)
+        if mark:
+            mark(5)
+
     def run(self, W: torch.Tensor, X: torch.Tensor, stream=None, events=None):
         s = torch.cuda.current_stream() if stream is None else stream
         ev = events
@@ -398,23 +430,8 @@ class LayerQuantizer:
             if ev is not None:
                 ev[i].record(s)
 
-        with torch.cuda.stream(s):
-            self.H.zero_()
-        mark(0)
-        gptq_hessian_accumulate(self.H, X, 2.0, ws=self.ws_h, info=self.info_h, stream=s)
-        mark(1)
-        gptq_cholesky_inverse(self.H, self.percdamp, self.actorder, self.U, self.perm, self.dead,
-                              self.info, ws=self.ws_c, stream=s)
-        mark(2)
-        gptq_quantize_layer(W, self.U, self.perm, self.dead, self.cfg, self.codes, self.scales,
-                            self.zeros, self.g_idx, self.Wq, self.row_loss, ws=self.ws_q,
-                            stream=s)
-        mark(3)
-        self._pack(self.codes, self.packed, stream=s)
-        mark(4)
-        gptq_dequant(self.packed, self.bits, self.n, self.scales, self.zeros, self.group_size,
-                     self.g_idx, self.deq.dtype, out=self.deq, stream=s)
-        mark(5)
+        self.hessian(X, s, mark)
+        self.finish(W, s, mark)
         return self
 
     def check_info(self) -> None:
@@ -422,3 +439,64 @@ class LayerQuantizer:
         ci, hi = int(self.info.item()), int(self.info_h.item())
         if ci != 0 or hi != 0:
             raise GptqError(f"device status: cholesky info {ci}, hessian info {hi}")
+
+
+class LayerPipeline:
+    """GPTQ of a sequence of linears, one layer at a time (page "GPTQ, with
+    the code open", section "From one repair to a whole model": each layer is
+    repaired from its own inputs and Hessian), with the Hessian of linear
+    l + 1 accumulating on one stream while linear l is factored, swept,
+    packed and dequantized on another.  The Hessian is tensor-core bound and
+    the rest a chain of small dependent launches, so the two overlap on the
+    SMs the chain leaves idle.
+
+    ``shapes``: (rows, n) per linear; every linear sees ``ntok`` tokens.
+    One LayerQuantizer per linear holds that linear's buffers and outputs
+    (``layers[l]``).  ``run(Ws, Xs)`` enqueues everything and makes the
+    caller's stream wait for the last linear."""
+
+    def __init__(self, shapes, ntok: int, bits: int = 4, group_size: int = 128,
+                 percdamp: float = 0.01, actorder: bool = False, sym: bool = False,
+                 x_dtype: torch.dtype = torch.bfloat16, w_dtype: torch.dtype = torch.bfloat16,
+                 out_dtype: torch.dtype = torch.bfloat16, want_wq: bool = False,
+                 want_loss: bool = False, device=None):
+        dev = torch.device("cuda") if device is None else torch.device(device)
+        self.layers = [LayerQuantizer(rows, n, ntok, bits, group_size, percdamp, actorder,
+                                      x_dtype, w_dtype, out_dtype, want_wq, want_loss, sym=sym,
+                                      device=dev)
+                       for rows, n in shapes]
+        self.s_h = torch.cuda.Stream(dev)
+        self.s_q = torch.cuda.Stream(dev)
+        self.ev_h = [torch.cuda.Event() for _ in shapes]
+        self.ev_start = torch.cuda.Event()
+        self.ev_done = torch.cuda.Event()
+
+    def run(self, Ws, Xs, stream=None, overlap: bool = True):
+        """overlap=False runs the same work one linear after another on the
+        caller's stream (the reference order)."""
+        s = torch.cuda.current_stream() if stream is None else stream
+        if len(Ws) != len(self.layers) or len(Xs) != len(self.layers):
+            raise GptqError("one W and one X per linear")
+        if not overlap:
+            for q, W, X in zip(self.layers, Ws, Xs):
+                q.hessian(X, s)
+                q.finish(W, s)
+            return self
+        self.ev_start.record(s)
+        self.s_h.wait_event(self.ev_start)
+        self.s_q.wait_event(self.ev_start)
+        L = len(self.layers)
+        for l in range(L + 1):
+            if l < L:
+                self.layers[l].hessian(Xs[l], self.s_h)
+                self.ev_h[l].record(self.s_h)
+            if l >= 1:
+                self.s_q.wait_event(self.ev_h[l - 1])
+                self.layers[l - 1].finish(Ws[l - 1], self.s_q)
+        self.ev_done.record(self.s_q)
+        s.wait_event(self.ev_done)
+        return self
+
+    def check_info(self) -> None:
+        for q in self.layers:
+            q.check_info()

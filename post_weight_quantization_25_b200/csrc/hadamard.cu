@@ -42,13 +42,14 @@ __device__ __forceinline__ void fwht_warp(float (&v)[VPL], int lane) {
         v[i] = a + b;
         v[i + h] = a - b;
       }
+  // partner lane l ^ m: the lower lane keeps v + o, the upper one o - v,
+  // i.e. o + sgn v with sgn = -1 on the upper lane (one FMA, exact product)
 #pragma unroll
-  for (int m = 1; m < 32; m <<= 1)
+  for (int m = 1; m < 32; m <<= 1) {
+    const float sgn = (lane & m) ? -1.f : 1.f;
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const float o = __shfl_xor_sync(0xffffffffu, v[i], m);
-      v[i] = (lane & m) ? o - v[i] : v[i] + o;
-    }
+    for (int i = 0; i < VPL; ++i) v[i] = fmaf(sgn, v[i], __shfl_xor_sync(0xffffffffu, v[i], m));
+  }
 }
 
 // W' = W R^T: each row's blocks of b contiguous elements, one warp per block

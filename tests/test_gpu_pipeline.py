@@ -1,0 +1,64 @@
+"""The layer pipeline: the Hessian of linear l + 1 overlapping the rest of
+linear l on a second stream gives every linear the same results as the
+oracle (and as the one-stream order) -- the overlap only reorders
+independent work."""
+import numpy as np
+import pytest
+import torch
+
+import post_weight_quantization_25_b200 as G
+import workloads
+from gpu_util import compare_layer, device_x, to_np
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(40, 256), (33, 384), (64, 256), (17, 128)]
+
+
+def _outputs(q):
+    torch.cuda.synchronize()
+    return {"perm": q.perm.cpu().numpy().astype(np.int64),
+            "dead": q.dead.cpu().numpy().astype(bool), "info": int(q.info.item()),
+            "codes": q.codes.cpu().numpy().astype(np.int64), "scales": q.scales.cpu().numpy(),
+            "zeros": q.zeros.cpu().numpy().astype(np.int64),
+            "g_idx": q.g_idx.cpu().numpy().astype(np.int64), "Wq": q.Wq.cpu().numpy(),
+            "row_loss": q.row_loss.cpu().numpy().astype(np.float64)}
+
+
+@pytest.mark.parametrize("overlap", [True, False])
+@pytest.mark.parametrize("actorder", [False, True])
+def test_pipelined_layers_match_the_oracle(overlap, actorder):
+    ntok = 600
+    layers = [workloads.random_layer(r, n, ntok, seed=50 + i, dtype=torch.bfloat16,
+                                     correlated=0.3)
+              for i, (r, n) in enumerate(SHAPES)]
+    Ws = [W.cuda() for W, _ in layers]
+    Xs = [device_x(X) for _, X in layers]
+    pipe = G.LayerPipeline(SHAPES, ntok, bits=4, group_size=64, actorder=actorder,
+                           w_dtype=torch.bfloat16, want_wq=True, want_loss=True)
+    pipe.run(Ws, Xs, overlap=overlap)
+    torch.cuda.synchronize()
+    pipe.check_info()
+    for q, (W, X) in zip(pipe.layers, layers):
+        compare_layer(_outputs(q), W, X, 4, 64, 0.01, actorder)
+        # the packed and dequantized outputs belong to the same codes
+        deq = to_np(q.deq)
+        sc = q.scales.cpu().numpy()[:, q.g_idx.cpu().numpy()]
+        zz = q.zeros.cpu().numpy()[:, q.g_idx.cpu().numpy()].astype(np.float64)
+        wq = (sc.astype(np.float64) * (q.codes.cpu().numpy() - zz)).astype(np.float32)
+        assert np.array_equal(deq, torch.from_numpy(wq).to(torch.bfloat16).float().numpy())
+
+
+def test_pipeline_runs_again_with_new_inputs():
+    """Buffers are reused across runs: a second run on other inputs matches
+    a fresh one-layer quantizer on those inputs."""
+    ntok = 300
+    shapes = SHAPES[:2]
+    pipe = G.LayerPipeline(shapes, ntok, group_size=128, want_wq=True, want_loss=True)
+    for seed in (1, 2):
+        layers = [workloads.random_layer(r, n, ntok, seed=seed * 10 + i, dtype=torch.bfloat16)
+                  for i, (r, n) in enumerate(shapes)]
+        pipe.run([W.cuda() for W, _ in layers], [device_x(X) for _, X in layers])
+        torch.cuda.synchronize()
+        for q, (W, X) in zip(pipe.layers, layers):
+            compare_layer(_outputs(q), W, X, 4, 128, 0.01, False)
