@@ -129,7 +129,7 @@ gptq_status gptq_cholesky_inverse(const float* H, int64_t n, float percdamp, int
  * programs that own all device memory in a fixed pool and forbid allocation
  * while running, so they can neither call cudaMalloc nor pass a workspace.
  * Same arguments, results and `info` contract as gptq_cholesky_inverse, minus
- * the workspace: the scratch is a 19.0 MB array built into the library, so
+ * the workspace: the scratch is a 21.1 MB array built into the library, so
  * n must be <= 2048 (larger n returns GPTQ_ERR_WORKSPACE).  The library looks
  * up that array's device address once per device, in the first call made with
  * that device current; make that first call before any stream capture.  All

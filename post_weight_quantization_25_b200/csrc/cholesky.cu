@@ -32,6 +32,8 @@
 #include <cmath>
 #include <cstdint>
 
+#include <mutex>
+
 #include "gptq_internal.cuh"
 #include "chol_diag.cuh"
 #include "panel_gemm.cuh"
@@ -46,8 +48,8 @@ struct CholWs {
   float* A;       // n x n, lower part used: J P^T H P J + lambda I
   float* dprime;  // n: diag(H) with dead entries set to 1
   double* lam;    // 1: damping
-  float* PBh;     // n x 128: the current panel's solved vectors, TF32 part
-  float* PBl;     // n x 128: remainder
+  float* PBh[2];  // n x 128: a panel's solved vectors, TF32 part (panel p uses [p % 2])
+  float* PBl[2];  // n x 128: remainder
   float* Dout;    // the diagonal step's outputs: L^T of the block, inverted leaves
 };
 
@@ -57,7 +59,7 @@ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // allocation-free entry point below, hence constexpr).
 constexpr size_t chol_ws_bytes(int64_t n) {
   return align_up(sizeof(float) * n * n, 256) + align_up(sizeof(float) * n, 256) + 256 +
-         2 * align_up(sizeof(float) * n * kPanel, 256) + sizeof(float) * kDiagOutFloats;
+         4 * align_up(sizeof(float) * n * kPanel, 256) + sizeof(float) * kDiagOutFloats;
 }
 
 CholWs carve(void* ws, int64_t n) {
@@ -69,10 +71,12 @@ CholWs carve(void* ws, int64_t n) {
   p += align_up(sizeof(float) * n, 256);
   w.lam = reinterpret_cast<double*>(p);
   p += 256;
-  w.PBh = reinterpret_cast<float*>(p);
-  p += align_up(sizeof(float) * n * kPanel, 256);
-  w.PBl = reinterpret_cast<float*>(p);
-  p += align_up(sizeof(float) * n * kPanel, 256);
+  for (int b = 0; b < 2; ++b) {
+    w.PBh[b] = reinterpret_cast<float*>(p);
+    p += align_up(sizeof(float) * n * kPanel, 256);
+    w.PBl[b] = reinterpret_cast<float*>(p);
+    p += align_up(sizeof(float) * n * kPanel, 256);
+  }
   w.Dout = reinterpret_cast<float*>(p);
   return w;
 }
@@ -178,11 +182,22 @@ struct CholTrailItems {
   float* A;
   float* RT;
   int n, p, nblk;
+  int cb_lo, cb_hi;  // column blocks [cb_lo, cb_hi) of this launch
+  // row block R updates column blocks [p + 1, R] of A (R > p) or
+  // [p + 1, nblk) of RT (R <= p), clipped to the window
+  __host__ __device__ int col_lo() const { return cb_lo > p + 1 ? cb_lo : p + 1; }
+  __host__ __device__ int col_hi(int R) const {
+    const int h = R > p ? R + 1 : nblk;
+    return h < cb_hi ? h : cb_hi;
+  }
   __host__ __device__ int num_items() const { return nblk; }
-  __host__ __device__ int item_nq(int R) const { return R > p ? R - p : nblk - 1 - p; }
+  __host__ __device__ int item_nq(int R) const {
+    const int q = col_hi(R) - col_lo();
+    return q > 0 ? q : 0;
+  }
   __device__ PgItem item(int R) const {
     PgItem I;
-    const int c0 = (p + 1) * kPanel;
+    const int c0 = col_lo() * kPanel;
     I.C0 = (R > p ? A : RT) + (int64_t)R * kPanel * n + c0;
     I.ldc = n;
     I.cmap = R > p ? 0 : 1;
@@ -279,12 +294,13 @@ cudaError_t launch_cholesky_inverse(const float* H, int64_t n64, float percdamp,
   const int apply_ctas = (n + kApplyVecs - 1) / kApplyVecs;  // n vectors per panel
   // operands of the trailing updates; with a row stride that is a multiple
   // of 16 bytes the updates land in A and RT by TMA reduce-add
-  CUtensorMap mPh, mPl, mA, mRT;
+  CUtensorMap mPh[2], mPl[2], mA, mRT;
   const bool reduce = (n % 4) == 0;
   if (nblk > 1) {
-    if (!make_tma_2d(&mPh, w.PBh, false, n, kPanel, kPanel, 32, 128) ||
-        !make_tma_2d(&mPl, w.PBl, false, n, kPanel, kPanel, 32, 128))
-      return cudaErrorInvalidValue;
+    for (int b = 0; b < 2; ++b)
+      if (!make_tma_2d(&mPh[b], w.PBh[b], false, n, kPanel, kPanel, 32, 128) ||
+          !make_tma_2d(&mPl[b], w.PBl[b], false, n, kPanel, kPanel, 32, 128))
+        return cudaErrorInvalidValue;
     if (reduce) {
       if (!make_tma_2d(&mA, w.A, false, n, n, n, 32, 32) ||
           !make_tma_2d(&mRT, U, false, n, n, n, 32, 32))
@@ -294,32 +310,66 @@ cudaError_t launch_cholesky_inverse(const float* H, int64_t n64, float percdamp,
                                     (int)pg2_smem_bytes(true))) != cudaSuccess)
         return e;
     } else {
-      mA = mRT = mPh;  // not read by the read-modify-write epilogue
+      mA = mRT = mPh[0];  // not read by the read-modify-write epilogue
       if ((e = cudaFuncSetAttribute(panel_gemm2_kernel<CholTrailItems, false>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)pg2_smem_bytes(false))) != cudaSuccess)
         return e;
     }
   }
+  // Look-ahead: the trailing update of panel p is split into the next
+  // panel's column block (near, on the caller's stream, so panel p + 1 can be
+  // factored at once) and the rest (far, on a side stream, overlapping the
+  // factorisation of panel p + 1).  Every element still receives the panels'
+  // updates in panel order: near(p) waits for far(p - 1), far(p) follows
+  // far(p - 1) on the side stream, and panel p + 1's vectors go to the other
+  // half of the double-buffered PB while far(p) reads its own.
+  SideStream side{};
+  const bool ahead = nblk > 2 && side_stream(&side);
+  std::unique_lock<std::mutex> side_guard;
+  if (ahead) side_guard = std::unique_lock<std::mutex>(side_lock());
+  auto trail = [&](int p, int cb_lo, int cb_hi, cudaStream_t st) -> cudaError_t {
+    const CholTrailItems dec{w.A, U, n, p, nblk, cb_lo, cb_hi};
+    int chunk = 1, units = 0;
+    pg2_plan(dec, sms, chunk, units);
+    if (units == 0) return cudaSuccess;
+    const int grid = std::min(units, sms);
+    const int b = p & 1;
+    if (reduce)
+      panel_gemm2_kernel<CholTrailItems, true><<<grid, kPg2Threads, pg2_smem_bytes(true), st>>>(
+          mPh[b], mPl[b], mPh[b], mPl[b], mA, mRT, dec, chunk, units, info, kInfoTimeout, info);
+    else
+      panel_gemm2_kernel<CholTrailItems, false><<<grid, kPg2Threads, pg2_smem_bytes(false), st>>>(
+          mPh[b], mPl[b], mPh[b], mPl[b], mA, mRT, dec, chunk, units, info, kInfoTimeout, info);
+    note_launch();
+    return cudaGetLastError();
+  };
   for (int p = 0; p < nblk; ++p) {
+    const int b = p & 1;
     chol_diag_kernel<<<1, kDiagThreads, kDiagSmemBytes, s>>>(w.A, n, p, w.Dout, info);
     note_launch();
     panel_apply_kernel<<<apply_ctas, kApplyThreads, kApplySmemBytes, s>>>(
-        w.A, U, n, p, w.Dout, w.PBh, w.PBl, info);
+        w.A, U, n, p, w.Dout, w.PBh[b], w.PBl[b], info);
     note_launch();
-    if (p + 1 < nblk) {
-      const CholTrailItems dec{w.A, U, n, p, nblk};
-      int chunk = 1, units = 0;
-      pg2_plan(dec, sms, chunk, units);
-      const int grid = std::min(units, sms);
-      if (reduce)
-        panel_gemm2_kernel<CholTrailItems, true><<<grid, kPg2Threads, pg2_smem_bytes(true), s>>>(
-            mPh, mPl, mPh, mPl, mA, mRT, dec, chunk, units, info, kInfoTimeout, info);
-      else
-        panel_gemm2_kernel<CholTrailItems, false><<<grid, kPg2Threads, pg2_smem_bytes(false), s>>>(
-            mPh, mPl, mPh, mPl, mA, mRT, dec, chunk, units, info, kInfoTimeout, info);
-      note_launch();
+    if (p + 1 >= nblk) break;
+    if (!ahead) {
+      if ((e = trail(p, 0, nblk, s)) != cudaSuccess) return e;
+      continue;
     }
+    // side: far(p) after apply(p) (and after far(p - 1), in stream order)
+    if ((e = cudaEventRecord(side.ev[0], s)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(side.s, side.ev[0], 0)) != cudaSuccess)
+      return e;
+    // caller's stream: near(p) after far(p - 1) has landed
+    if (p >= 1 && (e = cudaStreamWaitEvent(s, side.ev[2 + ((p - 1) & 1)], 0)) != cudaSuccess)
+      return e;
+    if ((e = trail(p, p + 1, p + 2, s)) != cudaSuccess) return e;
+    if ((e = trail(p, p + 2, nblk, side.s)) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(side.ev[2 + b], side.s)) != cudaSuccess) return e;
+  }
+  if (ahead && nblk >= 2) {
+    // join: the last far update (panel nblk - 2) before the caller's stream goes on
+    if ((e = cudaStreamWaitEvent(s, side.ev[2 + ((nblk - 2) & 1)], 0)) != cudaSuccess) return e;
   }
   if (n % 32 == 0) {
     const int nt = n / 32;
@@ -346,7 +396,7 @@ cudaError_t launch_cholesky_inverse(const float* H, int64_t n64, float percdamp,
 // these bytes until the process exits.
 //
 // Limit: n <= kNoAllocMaxN (2048), i.e. the scratch of one 2048 x 2048
-// factorisation, 19.0 MB.  Larger n is rejected with GPTQ_ERR_WORKSPACE.
+// factorisation, 21.1 MB.  Larger n is rejected with GPTQ_ERR_WORKSPACE.
 //
 // The array's name in host code is only a host-side stand-in, not a device
 // address.  The device address is looked up with cudaGetSymbolAddress once

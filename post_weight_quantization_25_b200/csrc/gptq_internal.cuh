@@ -30,7 +30,7 @@ void note_launch();
 // the caller's stream before returning.  Returns false if it cannot be had.
 struct SideStream {
   cudaStream_t s;
-  cudaEvent_t ev[2];
+  cudaEvent_t ev[4];
 };
 bool side_stream(SideStream* out);
 std::mutex& side_lock();
