@@ -289,7 +289,7 @@ def measure_dequant_matvec(G, dev, packed, bits, n, scales, zeros, group_size, g
         + (int(perm.numel() * 4) if perm is not None else 0)
     pk = peaks()
     gbs = nbytes / t / 1e9
-    mma = (bits == 4 and x.dtype == torch.bfloat16 and g_idx is None and n % 32 == 0
+    mma = (bits in (3, 4) and x.dtype == torch.bfloat16 and g_idx is None and n % 32 == 0
            and (group_size <= 0 or (group_size >= 32 and group_size & (group_size - 1) == 0)))
     return {"shape": label, "order": "sweep (perm)" if perm is not None else
             ("original (g_idx)" if g_idx is not None else "original"),
@@ -330,6 +330,12 @@ def measure_dequant_70b(G, dev):
                                           label=label7))
         out.append(measure_dequant_matvec(G, dev, pk7, 4, n7, sc7, z7, 128, None, batch=b,
                                           label=label7, perm=pm7))
+    # 3-bit codes of the same shape (the first 3/4 of the int4 words' bits as
+    # int3 words, zero points reduced to 3 bits), sweep order, 1 vector
+    pk3 = pk7.view(-1)[: 8192 * 28672 * 3 // 32].view(8192, -1)
+    z3 = z7 & 7
+    out.append(measure_dequant_matvec(G, dev, pk3, 3, n7, sc7, z3, 128, None, batch=1,
+                                      label=label7, perm=pm7))
     return out
 
 

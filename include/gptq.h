@@ -196,9 +196,9 @@ gptq_status gptq_dequant(const uint32_t* packed, int bits, int64_t rows, int64_t
  * comes from custom kernels at batch size 1, where reading the weights
  * dominates -- packed codes are 8 / bits times smaller than fp32, 4 / bits
  * times smaller than bf16).
- * Two kernels serve it.  int4 codes with bf16 x, no g_idx, n % 32 == 0,
- * group_size a power of two >= 32 (or per row), packed 16-byte aligned and
- * zero points < 128: the tensor-core kernel, which multiplies exact bf16
+ * Two kernels serve it.  int4 or int3 codes with bf16 x, no g_idx,
+ * n % 32 == 0, group_size a power of two >= 32 (or per row), packed 16-byte
+ * (int4) or 4-byte (int3) aligned and zero points < 128: the tensor-core kernel, which multiplies exact bf16
  * (q - zero) pairs with x in fp32 MMA accumulators, scales each group's sum
  * once, and adds the two column halves of every output onto zeros (two
  * terms, so the result does not depend on their order).  It first writes x

@@ -443,19 +443,46 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Two MMAs for one word per row: codes wa (row g) and wb (row g + 8) with
-// their zero pairs za / zb; xp holds the word's 8 activations of vector g in
-// pair order (x0, x4), (x1, x5), (x2, x6), (x3, x7).
+// The four bf16 pairs (128 + q_i, 128 + q_{i+4}), i = 0..3, of 8 codes:
+// int4: a 32-bit word, code i in bits 4i..4i+3; int3: 24 bits, code i in
+// bits 3i..3i+2, first spread so that codes i and i + 4 sit 16 bits apart.
+template <int BITS>
+__device__ __forceinline__ uint4 code_pairs(uint32_t w) {
+  constexpr uint32_t kMagic = 0x43004300u;
+  if constexpr (BITS == 4) {
+    constexpr uint32_t kMask = 0x000F000Fu;
+    return make_uint4((w & kMask) | kMagic, ((w >> 4) & kMask) | kMagic,
+                      ((w >> 8) & kMask) | kMagic, ((w >> 12) & kMask) | kMagic);
+  } else {
+    constexpr uint32_t kMask = 0x00070007u;
+    const uint32_t sp = (w & 0xFFFu) | ((w >> 12) << 16);  // codes 4..7 -> bits 16..27
+    return make_uint4((sp & kMask) | kMagic, ((sp >> 3) & kMask) | kMagic,
+                      ((sp >> 6) & kMask) | kMagic, ((sp >> 9) & kMask) | kMagic);
+  }
+}
+
+// Two MMAs for 8 codes per row: codes wa (row g) and wb (row g + 8) with
+// their zero pairs za / zb; xp holds the 8 activations of vector g in pair
+// order (x0, x4), (x1, x5), (x2, x6), (x3, x7).
+template <int BITS>
 __device__ __forceinline__ void mma_word(float (&c)[4], uint32_t wa, uint32_t wb, uint32_t za,
                                          uint32_t zb, const uint4& xp) {
-  constexpr uint32_t kMask = 0x000F000Fu, kMagic = 0x43004300u;
-  mma_bf16_16816(c, bf16x2_sub((wa & kMask) | kMagic, za), bf16x2_sub((wb & kMask) | kMagic, zb),
-                 bf16x2_sub(((wa >> 4) & kMask) | kMagic, za),
-                 bf16x2_sub(((wb >> 4) & kMask) | kMagic, zb), xp.x, xp.y);
-  mma_bf16_16816(c, bf16x2_sub(((wa >> 8) & kMask) | kMagic, za),
-                 bf16x2_sub(((wb >> 8) & kMask) | kMagic, zb),
-                 bf16x2_sub(((wa >> 12) & kMask) | kMagic, za),
-                 bf16x2_sub(((wb >> 12) & kMask) | kMagic, zb), xp.z, xp.w);
+  const uint4 a = code_pairs<BITS>(wa), b = code_pairs<BITS>(wb);
+  mma_bf16_16816(c, bf16x2_sub(a.x, za), bf16x2_sub(b.x, zb), bf16x2_sub(a.y, za),
+                 bf16x2_sub(b.y, zb), xp.x, xp.y);
+  mma_bf16_16816(c, bf16x2_sub(a.z, za), bf16x2_sub(b.z, zb), bf16x2_sub(a.w, za),
+                 bf16x2_sub(b.w, zb), xp.z, xp.w);
+}
+
+// int3: quarter q (codes 8q .. 8q + 7) of a 32-code block stored in words
+// w0, w1, w2 (little-endian 96 bits); bits above the quarter are ignored.
+__device__ __forceinline__ uint32_t int3_quarter(uint32_t w0, uint32_t w1, uint32_t w2, int q) {
+  switch (q) {
+    case 0: return w0;
+    case 1: return __funnelshift_r(w0, w1, 24);
+    case 2: return __funnelshift_r(w1, w2, 16);
+    default: return w2 >> 8;
+  }
 }
 
 __device__ __forceinline__ uint32_t zero_pair(uint8_t z) {
@@ -466,11 +493,11 @@ constexpr int kDqWarps = 4;    // warps per CTA
 constexpr int kDqStages = 5;   // code slices a warp keeps in flight (cp.async ring)
 constexpr int kDqMinBlocks = 8;
 constexpr int kDqSplit = 2;    // column halves per row tile (two atomic adds per output)
-// bytes between the 16 code rows of a staged slice: 64 (block mode: each
-// thread reads back its own 16-byte pieces, conflict-free) or 80 (interleaved
-// mode: 4-byte reads of 8 rows x 4 words land on distinct banks)
-template <bool kInterleaved>
-__host__ __device__ constexpr int dq_pitch() { return kInterleaved ? 80 : 64; }
+// bytes between the 16 code rows of a staged slice: 64 (int4 block mode: each
+// thread reads back its own 16-byte pieces, conflict-free) or 80 (the 4-byte
+// reads of the other modes: 8 rows x 4 words land on distinct banks)
+template <int BITS, bool kInterleaved>
+__host__ __device__ constexpr int dq_pitch() { return BITS == 4 && !kInterleaved ? 64 : 80; }
 
 // The non-code operands of one slice for one thread: activations of its
 // block(s) and the rulers of its rows.
@@ -516,20 +543,34 @@ __device__ __forceinline__ void dq_side(DqSide<kInterleaved>& d, int s, int nblk
   }
 }
 
-// `st`: this warp's staged slice (16 rows x pitch bytes of codes).
-template <bool kInterleaved>
+// `st`: this warp's staged slice (16 rows x pitch bytes of codes): int4,
+// 16 words per row (block b = words 4b .. 4b + 3); int3, 12 words per row
+// (block b = words 3b .. 3b + 2).
+template <int BITS, bool kInterleaved>
 __device__ __forceinline__ void dq_slice(float (&Y)[4], const uint8_t* st,
-                                         const DqSide<kInterleaved>& d,
-                                         int g, int t) {
-  constexpr int P = dq_pitch<kInterleaved>();
+                                         const DqSide<kInterleaved>& d, int g, int t) {
+  constexpr int P = dq_pitch<BITS, kInterleaved>();
+  const uint32_t* ra = reinterpret_cast<const uint32_t*>(st + g * P);
+  const uint32_t* rb = reinterpret_cast<const uint32_t*>(st + (g + 8) * P);
   if constexpr (!kInterleaved) {
-    const uint4 qa = *reinterpret_cast<const uint4*>(st + g * P + 16 * t);
-    const uint4 qb = *reinterpret_cast<const uint4*>(st + (g + 8) * P + 16 * t);
+    uint32_t wa[4], wb[4];
+    if constexpr (BITS == 4) {
+      const uint4 qa = *reinterpret_cast<const uint4*>(ra + 4 * t);
+      const uint4 qb = *reinterpret_cast<const uint4*>(rb + 4 * t);
+      wa[0] = qa.x; wa[1] = qa.y; wa[2] = qa.z; wa[3] = qa.w;
+      wb[0] = qb.x; wb[1] = qb.y; wb[2] = qb.z; wb[3] = qb.w;
+    } else {
+      const uint32_t a0 = ra[3 * t], a1 = ra[3 * t + 1], a2 = ra[3 * t + 2];
+      const uint32_t b0 = rb[3 * t], b1 = rb[3 * t + 1], b2 = rb[3 * t + 2];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        wa[q] = int3_quarter(a0, a1, a2, q);
+        wb[q] = int3_quarter(b0, b1, b2, q);
+      }
+    }
     float c[4] = {0.f, 0.f, 0.f, 0.f};
-    mma_word(c, qa.x, qb.x, d.za[0], d.zb[0], d.xq[0]);
-    mma_word(c, qa.y, qb.y, d.za[0], d.zb[0], d.xq[1]);
-    mma_word(c, qa.z, qb.z, d.za[0], d.zb[0], d.xq[2]);
-    mma_word(c, qa.w, qb.w, d.za[0], d.zb[0], d.xq[3]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) mma_word<BITS>(c, wa[j], wb[j], d.za[0], d.zb[0], d.xq[j]);
     Y[0] = fmaf(d.fa[0], c[0], Y[0]);
     Y[1] = fmaf(d.fa[0], c[1], Y[1]);
     Y[2] = fmaf(d.fb[0], c[2], Y[2]);
@@ -538,10 +579,23 @@ __device__ __forceinline__ void dq_slice(float (&Y)[4], const uint8_t* st,
     // blocks past the row end hold zero x, so their terms vanish
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint32_t wa = *reinterpret_cast<const uint32_t*>(st + g * P + 16 * j + 4 * t);
-      const uint32_t wb = *reinterpret_cast<const uint32_t*>(st + (g + 8) * P + 16 * j + 4 * t);
+      uint32_t wa, wb;
+      if constexpr (BITS == 4) {
+        wa = ra[4 * j + t];
+        wb = rb[4 * j + t];
+      } else {
+        // quarter t of block j: words 3j + (3t) / 4 and the next
+        const int w0 = 3 * j + (3 * t) / 4;
+        const uint32_t a_lo = ra[w0], b_lo = rb[w0];
+        const uint32_t a_hi = t == 1 || t == 2 ? ra[w0 + 1] : 0u;
+        const uint32_t b_hi = t == 1 || t == 2 ? rb[w0 + 1] : 0u;
+        wa = t == 0 ? a_lo : t == 1 ? __funnelshift_r(a_lo, a_hi, 24)
+                           : t == 2 ? __funnelshift_r(a_lo, a_hi, 16) : a_lo >> 8;
+        wb = t == 0 ? b_lo : t == 1 ? __funnelshift_r(b_lo, b_hi, 24)
+                           : t == 2 ? __funnelshift_r(b_lo, b_hi, 16) : b_lo >> 8;
+      }
       float c[4] = {0.f, 0.f, 0.f, 0.f};
-      mma_word(c, wa, wb, d.za[j], d.zb[j], d.xq[j]);
+      mma_word<BITS>(c, wa, wb, d.za[j], d.zb[j], d.xq[j]);
       Y[0] = fmaf(d.fa[j], c[0], Y[0]);
       Y[1] = fmaf(d.fa[j], c[1], Y[1]);
       Y[2] = fmaf(d.fb[j], c[2], Y[2]);
@@ -550,12 +604,14 @@ __device__ __forceinline__ void dq_slice(float (&Y)[4], const uint8_t* st,
   }
 }
 
-template <bool kInterleaved>
-__global__ void __launch_bounds__(kDqWarps * 32, kDqMinBlocks) dequant_mma_int4_kernel(
+template <int BITS, bool kInterleaved>
+__global__ void __launch_bounds__(kDqWarps * 32, kDqMinBlocks) dequant_mma_kernel(
     const uint32_t* __restrict__ packed, int64_t rows, int64_t n,
     const float* __restrict__ scales, const uint8_t* __restrict__ zeros, int gshift, int64_t G,
     const __nv_bfloat16* __restrict__ xp, int nb, float* __restrict__ y, int64_t ldy) {
-  constexpr int P = dq_pitch<kInterleaved>();
+  constexpr int P = dq_pitch<BITS, kInterleaved>();
+  // int3 pieces are read by other lanes than the ones that stage them
+  constexpr bool kShared = kInterleaved || BITS == 3;
   constexpr int kStageBytes = 16 * P;
   __shared__ __align__(16) uint8_t ring[kDqWarps][kDqStages][kStageBytes];
   __shared__ float red[kDqWarps][16][9];
@@ -564,7 +620,7 @@ __global__ void __launch_bounds__(kDqWarps * 32, kDqMinBlocks) dequant_mma_int4_
   const int64_t r0 = (int64_t)blockIdx.x * 16;
   // rows past the end read the last row (valid memory) and are not stored
   const int64_t ra = min(r0 + g, rows - 1), rb = min(r0 + g + 8, rows - 1);
-  const int64_t wpr = n / 8;
+  const int64_t wpr = n * BITS / 32;  // words per row
   const uint32_t* pa = packed + ra * wpr;
   const uint32_t* pb = packed + rb * wpr;
   const float* sa = scales + ra * G;
@@ -580,14 +636,29 @@ __global__ void __launch_bounds__(kDqWarps * 32, kDqMinBlocks) dequant_mma_int4_
   const int first = s_lo + warp;
   const int K = first < s_hi ? (s_hi - first + kDqWarps - 1) / kDqWarps : 0;
   uint8_t* myring = &ring[warp][0][0];
-  // each thread stages its own 16 bytes of rows g and g + 8 per slice
+  // int4: each thread stages 16 bytes (its block) of rows g and g + 8 per
+  // slice; int3: 4-byte words t, t + 4, t + 8 of the slice's 12 per row (rows
+  // are only 4-byte aligned), words past the row's end not copied
   auto issue = [&](int k) {
     if (k < K) {
-      const int blk = 4 * (first + k * kDqWarps) + t;
-      if (blk < nblk) {
-        uint8_t* st = myring + (k % kDqStages) * kStageBytes;
-        ptx::cp_async_16(st + g * P + 16 * t, pa + 4 * blk);
-        ptx::cp_async_16(st + (g + 8) * P + 16 * t, pb + 4 * blk);
+      const int sl = first + k * kDqWarps;
+      uint8_t* st = myring + (k % kDqStages) * kStageBytes;
+      if constexpr (BITS == 4) {
+        const int blk = 4 * sl + t;
+        if (blk < nblk) {
+          ptx::cp_async_16(st + g * P + 16 * t, pa + 4 * blk);
+          ptx::cp_async_16(st + (g + 8) * P + 16 * t, pb + 4 * blk);
+        }
+      } else {
+        const int nw = 3 * min(4, nblk - 4 * sl);  // words of this slice in a row
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+          const int wdx = t + 4 * i;
+          if (wdx < nw) {
+            ptx::cp_async_4(st + g * P + 4 * wdx, pa + 12 * sl + wdx, 4);
+            ptx::cp_async_4(st + (g + 8) * P + 4 * wdx, pb + 12 * sl + wdx, 4);
+          }
+        }
       }
     }
     ptx::cp_async_commit();
@@ -603,13 +674,13 @@ __global__ void __launch_bounds__(kDqWarps * 32, kDqMinBlocks) dequant_mma_int4_
   for (int k = 0; k < kDqStages - 1; ++k) issue(k);
   float Y[4] = {0.f, 0.f, 0.f, 0.f};
   for (int k = 0; k < K; ++k) {
-    if (kInterleaved) __syncwarp();  // every lane is done with the slot refilled next
+    if (kShared) __syncwarp();  // every lane is done with the slot refilled next
     issue(k + kDqStages - 1);
     ptx::cp_async_wait<kDqStages - 1>();  // slice k has landed (this thread's part)
-    if (kInterleaved) __syncwarp();       // ... and every other lane's part
+    if (kShared) __syncwarp();            // ... and every other lane's part
     DqSide<kInterleaved> cur;
     side(cur, k);
-    dq_slice<kInterleaved>(Y, myring + (k % kDqStages) * kStageBytes, cur, g, t);
+    dq_slice<BITS, kInterleaved>(Y, myring + (k % kDqStages) * kStageBytes, cur, g, t);
   }
   ptx::cp_async_wait<0>();
   red[warp][g][2 * t] = Y[0];
@@ -701,12 +772,12 @@ cudaError_t launch_dequant_matvec(const uint32_t* packed, int bits, int64_t rows
                                   const void* x, int x_bf16, int64_t batch, float* y,
                                   cudaStream_t s) {
   if (rows == 0 || batch == 0) return cudaSuccess;
-  // the tensor-core path: int4, bf16 activations, groups that are runs of
+  // the tensor-core path: int4 / int3, bf16 activations, groups that are runs of
   // 32 k consecutive columns, 16-byte aligned code rows and activations
   // group sizes: one per row, or a power of two >= 32 (a shift finds the group)
   const bool pow2 = group_size >= 32 && (group_size & (group_size - 1)) == 0;
-  const bool mma = bits == 4 && x_bf16 && !g_idx && n % 32 == 0 && (group_size <= 0 || pow2) &&
-                   reinterpret_cast<uintptr_t>(packed) % 16 == 0;
+  const bool mma = x_bf16 && !g_idx && n % 32 == 0 && (group_size <= 0 || pow2) &&
+                   reinterpret_cast<uintptr_t>(packed) % (bits == 4 ? 16 : 4) == 0;
   if (mma) {
     // x in MMA pair order (and sweep order under perm) in stream-ordered scratch
     cudaMemPool_t pool;
@@ -730,12 +801,20 @@ cudaError_t launch_dequant_matvec(const uint32_t* packed, int bits, int64_t rows
     const dim3 grid((unsigned)((rows + 15) / 16), kDqSplit);
     for (int64_t b0 = 0; b0 < batch; b0 += 8) {
       const int nb = (int)(batch - b0 < 8 ? batch - b0 : 8);
-      if (inter)
-        dequant_mma_int4_kernel<true><<<grid, kDqWarps * 32, 0, s>>>(
-            packed, rows, n, scales, zeros, gshift, n_groups, xp + b0 * n, nb, y + b0 * rows, rows);
+      const __nv_bfloat16* xb = xp + b0 * n;
+      float* yb = y + b0 * rows;
+      if (bits == 4 && inter)
+        dequant_mma_kernel<4, true><<<grid, kDqWarps * 32, 0, s>>>(
+            packed, rows, n, scales, zeros, gshift, n_groups, xb, nb, yb, rows);
+      else if (bits == 4)
+        dequant_mma_kernel<4, false><<<grid, kDqWarps * 32, 0, s>>>(
+            packed, rows, n, scales, zeros, gshift, n_groups, xb, nb, yb, rows);
+      else if (inter)
+        dequant_mma_kernel<3, true><<<grid, kDqWarps * 32, 0, s>>>(
+            packed, rows, n, scales, zeros, gshift, n_groups, xb, nb, yb, rows);
       else
-        dequant_mma_int4_kernel<false><<<grid, kDqWarps * 32, 0, s>>>(
-            packed, rows, n, scales, zeros, gshift, n_groups, xp + b0 * n, nb, y + b0 * rows, rows);
+        dequant_mma_kernel<3, false><<<grid, kDqWarps * 32, 0, s>>>(
+            packed, rows, n, scales, zeros, gshift, n_groups, xb, nb, yb, rows);
       note_launch();
     }
     e = cudaGetLastError();

@@ -83,37 +83,41 @@ def mv_bound(n, mag):
     return 2 * (n / 32 + 24) * 2.0 ** -24 * mag + 1e-30
 
 
+@pytest.mark.parametrize("bits", [4, 3])
 @pytest.mark.parametrize("rows,n,g,batch,use_perm", [
     (33, 1056, 32, 3, False), (100, 2048, 128, 8, True), (16, 4096, -1, 1, False),
     (5, 96, 32, 9, True), (47, 640, 64, 2, False), (18, 1024, 256, 5, False),
-    (257, 4224, 128, 1, True)])
-def test_dequant_matvec_tensor_core_path(rows, n, g, batch, use_perm):
-    """int4 codes x bf16 activations with contiguous groups run on the MMA
-    kernel: one prep launch (x in pair / sweep order, y zeroed), then one
+    (257, 4224, 128, 1, True), (9, 160, 32, 2, False)])
+def test_dequant_matvec_tensor_core_path(bits, rows, n, g, batch, use_perm):
+    """int4 / int3 codes x bf16 activations with contiguous groups run on the
+    MMA kernel: one prep launch (x in pair / sweep order, y zeroed), then one
     launch per 8 vectors.
     Ragged row tiles (rows % 16), partial 128-column slices (n % 128), group
     sizes 32 / 64 (per-block scales), 128 / 256 / per row (per-slice scales),
     batches past 8, and extreme codes against extreme zero points."""
-    rng = np.random.default_rng(rows * 31 + n + batch)
-    codes = rng.integers(0, 16, (rows, n))
-    codes[0, : n // 2] = 15
+    rng = np.random.default_rng(rows * 31 + n + batch + bits)
+    top = 2 ** bits - 1
+    codes = rng.integers(0, top + 1, (rows, n))
+    codes[0, : n // 2] = top
     codes[-1, : n // 3] = 0
     G_ = 1 if g <= 0 else n // g
     scales = rng.uniform(1e-4, 0.2, (rows, G_)).astype(np.float32)
-    zeros = rng.integers(0, 16, (rows, G_))
+    zeros = rng.integers(0, top + 1, (rows, G_))
     zeros[0, :] = 0
-    zeros[-1, :] = 15
+    zeros[-1, :] = top
     perm = rng.permutation(n) if use_perm else None
-    packed = G.gptq_pack_int4(torch.from_numpy(codes.astype(np.uint8)).cuda())
+    pack = G.gptq_pack_int4 if bits == 4 else G.gptq_pack_int3
+    packed = pack(torch.from_numpy(codes.astype(np.uint8)).cuda())
     x = torch.randn(batch, n, generator=torch.Generator().manual_seed(rows)).to(torch.bfloat16)
     before = G.gptq_launch_count()
-    y = G.gptq_dequant_matvec(packed, 4, n, torch.from_numpy(scales).cuda(),
+    y = G.gptq_dequant_matvec(packed, bits, n, torch.from_numpy(scales).cuda(),
                               torch.from_numpy(zeros.astype(np.uint8)).cuda(), x.cuda(), g,
                               perm=torch.from_numpy(perm.astype(np.int32)).cuda()
                               if use_perm else None)
     torch.cuda.synchronize()
     assert G.gptq_launch_count() - before == 1 + (batch + 7) // 8  # x prep + one per 8 vectors
-    yo, mag = O.dequant_matvec(O.pack_int4(codes), 4, n, scales, zeros, x.float().numpy(), g,
+    ref_packed = O.pack_int4(codes) if bits == 4 else O.pack_int3(codes)
+    yo, mag = O.dequant_matvec(ref_packed, bits, n, scales, zeros, x.float().numpy(), g,
                                perm=perm)
     err = np.abs(y.cpu().numpy().astype(np.float64) - yo)
     bound = mv_bound(n, mag)
