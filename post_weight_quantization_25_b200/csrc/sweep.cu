@@ -203,31 +203,41 @@ __global__ void __launch_bounds__(256) gather_w_kernel(
   if (row_loss && threadIdx.x == 0) row_loss[r] = 0.f;
 }
 
-// One block [i1, i1 + bsz) of the sweep.  Four lanes (a "quad") per row,
-// eight rows per warp; lane q of a quad holds block columns q, q+4, ..., q+124
-// (slot s = column / 4).  Column jj is rounded in every lane of the quad, the
-// owner lane's (jj % 4) error term is broadcast inside the quad, and each lane
-// repairs its columns past jj with row jj of U's diagonal block.  The loop
-// over jj is unrolled, so slots left of jj are skipped at compile time.
-// Shared memory holds the block of U as  Uq[jj][q][slot] = U[i1+jj][i1+4 slot+q]
-// (quad-lane-major, row pitch 36 floats: 16-byte float4 reads, no bank
-// conflicts), plus 1/U_jj and 1/(2 U_jj^2).
+// One block [i1, i1 + bsz) of the sweep.  kSweepLanes lanes per row (a
+// "team"); lane q of a team holds block columns q, q + L, ..., q + 128 - L
+// (slot s = column / L, L = kSweepLanes).  Column jj is rounded in every lane
+// of the team, the owner lane's (jj % L) error term is broadcast inside the
+// team, and each lane repairs its columns past jj with row jj of U's diagonal
+// block.  The loop over jj is unrolled, so slots left of jj are skipped at
+// compile time.  4 lanes per row is the measured choice at 4096 rows; 16
+// lanes (8 slots each, 80 registers, twice the CTAs) computes the same
+// results but was slower there (2.15 ms against 1.52 ms per layer at 4096 x
+// 4096), its CTAs crowding out the concurrent far update.
+// Shared memory holds the block of U as  Uq[jj][q][slot] = U[i1+jj][i1+L slot+q]
+// (team-lane-major; row pitch kUqPitch floats per lane, chosen so the 16-byte
+// float4 reads of the 8 lanes of a phase hit distinct banks), plus 1/U_jj and
+// 1/(2 U_jj^2).
 //   GS = 0:   per-row ruler (already in scales / zeros)
 //   GS = 128: groups of a multiple of 128 columns, fitted at a block start that
 //             is a group start, from the current Wf
 //   GS = 32, 64: groups inside the block, fitted on the current registers
-constexpr int kSweepThreads = 128;
-constexpr int kUqPitch = 36;                  // floats per (jj, q) row of Uq
-constexpr int kUqRow = 4 * kUqPitch;          // floats per jj
+constexpr int kSweepLanes = 4;                           // lanes per row (4 or 16)
+constexpr int kSweepSlots = kBlock / kSweepLanes;        // columns per lane
+constexpr int kSweepThreads = kSweepLanes == 4 ? 128 : 256;
+constexpr int kUqPitch = kSweepLanes == 4 ? 36 : 12;     // floats per (jj, q)
+constexpr int kUqRow = kSweepLanes * kUqPitch;           // floats per jj
 constexpr size_t kSweepSmemBytes = sizeof(float) * (kBlock * kUqRow + 2 * kBlock);
+static_assert(kSweepSlots % 4 == 0 && kUqPitch >= kSweepSlots, "sweep team layout");
 
-__device__ __forceinline__ float quad_min(float v) {
-  v = fminf(v, __shfl_xor_sync(0xffffffffu, v, 1));
-  return fminf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+__device__ __forceinline__ float team_min(float v) {
+#pragma unroll
+  for (int o = 1; o < kSweepLanes; o <<= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
 }
-__device__ __forceinline__ float quad_max(float v) {
-  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
-  return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+__device__ __forceinline__ float team_max(float v) {
+#pragma unroll
+  for (int o = 1; o < kSweepLanes; o <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
 }
 
 template <int GS>
@@ -236,31 +246,32 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
     float maxq, int sym, int gsize, int G, float* __restrict__ Err_hi, float* __restrict__ Err_lo,
     uint8_t* __restrict__ codes_sw, float* __restrict__ scales, uint8_t* __restrict__ zeros,
     float* __restrict__ row_loss) {
+  constexpr int L = kSweepLanes, NS = kSweepSlots;
   extern __shared__ __align__(16) float smem[];
   float* Uq = smem;
   float* rd = smem + kBlock * kUqRow;
   float* hrd2 = rd + kBlock;
   stage_block_128<kSweepThreads>(
       U + (int64_t)i1 * n + i1, n, bsz, bsz, /*lower=*/false, (n % 4) == 0,
-      [&](int a, int b, float v) { Uq[a * kUqRow + (b & 3) * kUqPitch + (b >> 2)] = v; },
+      [&](int a, int b, float v) { Uq[a * kUqRow + (b % L) * kUqPitch + (b / L)] = v; },
       [](int, int) { return 0.f; });
   __syncthreads();
   for (int i = threadIdx.x; i < kBlock; i += blockDim.x) {
-    const float d = (i < bsz) ? Uq[i * kUqRow + (i & 3) * kUqPitch + (i >> 2)] : 1.f;
+    const float d = (i < bsz) ? Uq[i * kUqRow + (i % L) * kUqPitch + (i / L)] : 1.f;
     rd[i] = 1.f / d;
     hrd2[i] = 0.5f / (d * d);
   }
   __syncthreads();
 
   const int lane = threadIdx.x & 31;
-  const int q = lane & 3;
-  const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 2;
+  const int q = lane % L;
+  const int r = (blockIdx.x * blockDim.x + threadIdx.x) / L;
   const bool active = r < rows;
   float* wrow = Wf + (int64_t)(active ? r : 0) * n + i1;
-  float w[32];
+  float w[NS];
 #pragma unroll
-  for (int s = 0; s < 32; ++s) {
-    const int c = 4 * s + q;
+  for (int s = 0; s < NS; ++s) {
+    const int c = L * s + q;
     w[s] = (active && c < bsz) ? wrow[c] : 0.f;
   }
 
@@ -275,19 +286,19 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
     if (i1 % gsize == 0) {
       float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
-      for (int s = 0; s < 32; ++s)
-        if (4 * s + q < bsz) {
+      for (int s = 0; s < NS; ++s)
+        if (L * s + q < bsz) {
           mn = fminf(mn, w[s]);
           mx = fmaxf(mx, w[s]);
         }
       const int end = min(i1 + gsize, n);
       if (active)
-        for (int c = i1 + kBlock + q; c < end; c += 4) {
+        for (int c = i1 + kBlock + q; c < end; c += L) {
           const float v = Wf[(int64_t)r * n + c];
           mn = fminf(mn, v);
           mx = fmaxf(mx, v);
         }
-      fit_ruler(quad_min(mn), quad_max(mx), maxq, sym, scale, zf);
+      fit_ruler(team_min(mn), team_max(mx), maxq, sym, scale, zf);
       if (active && q == 0) {
         scales[(int64_t)r * G + g] = scale;
         zeros[(int64_t)r * G + g] = (uint8_t)zf;
@@ -301,35 +312,35 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
   // w / scale, correctly rounded, with the reciprocal of the scale computed
   // once per ruler (Markstein's method, fdiv.cuh)
   MDiv md = md_prepare(scale);
-  float e_out[32];
-  uint32_t cw[8];
+  float e_out[NS];
+  uint32_t cw[NS / 4];
 #pragma unroll
-  for (int s = 0; s < 32; ++s) e_out[s] = 0.f;
+  for (int s = 0; s < NS; ++s) e_out[s] = 0.f;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) cw[k] = 0u;
+  for (int k = 0; k < NS / 4; ++k) cw[k] = 0u;
   float loss = 0.f;
   const float* uq_lane = Uq + q * kUqPitch;
 
 #pragma unroll
-  for (int s = 0; s < 32; ++s) {
+  for (int s = 0; s < NS; ++s) {
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
+  for (int k = 0; k < L; ++k) {
     // No early exit for a short last block: its columns past bsz hold 0 and
     // its U rows past bsz are 0 (with 1/U_jj = 1), so they round to the zero
     // point with no error and change nothing; keeping the 128 steps free of
     // branches lets the compiler overlap consecutive steps.
-    const int jj = 4 * s + k;
-    constexpr int kGS = (GS == 32 || GS == 64) ? GS : 1;  // in-block group size
+    const int jj = L * s + k;
+    constexpr int kGS = (GS == 32 || GS == 64) ? GS : L;  // in-block group size
     if ((GS == 32 || GS == 64) && (jj % kGS) == 0) {
       // group [jj, jj + GS) of the block, current (repaired) values
       float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
-      for (int s2 = s; s2 < s + GS / 4; ++s2)
-        if (4 * s2 + q < bsz) {
+      for (int s2 = s; s2 < s + kGS / L; ++s2)
+        if (L * s2 + q < bsz) {
           mn = fminf(mn, w[s2]);
           mx = fmaxf(mx, w[s2]);
         }
-      fit_ruler(quad_min(mn), quad_max(mx), maxq, sym, scale, zf);
+      fit_ruler(team_min(mn), team_max(mx), maxq, sym, scale, zf);
       md = md_prepare(scale);
       if (active && q == 0 && jj < bsz) {  // groups past the last column do not exist
         const int g = (i1 + jj) / kGS;
@@ -337,24 +348,24 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
         zeros[(int64_t)r * G + g] = (uint8_t)zf;
       }
     }
-    // every lane rounds its slot s; the owner's (q == jj % 4) result is used
+    // every lane rounds its slot s; the owner's (q == jj % L) result is used
     const float x = w[s];
     float qv = rintf(md_div(x, md)) + zf;
     qv = fminf(fmaxf(qv, 0.f), maxq);
     const float wh = __fmul_rn(scale, qv - zf);
     const float e = x - wh;
     const float ev = e * rd[jj];
-    const float err = __shfl_sync(0xffffffffu, ev, jj & 3, 4);
+    const float err = __shfl_sync(0xffffffffu, ev, k, L);
     const float* urow = uq_lane + jj * kUqRow;
 #pragma unroll
-    for (int s4 = s >> 2; s4 < 8; ++s4) {
+    for (int s4 = s >> 2; s4 < NS / 4; ++s4) {
       const float4 u = *reinterpret_cast<const float4*>(urow + 4 * s4);
       if (4 * s4 + 0 >= s) w[4 * s4 + 0] = fmaf(-err, u.x, w[4 * s4 + 0]);
       if (4 * s4 + 1 >= s) w[4 * s4 + 1] = fmaf(-err, u.y, w[4 * s4 + 1]);
       if (4 * s4 + 2 >= s) w[4 * s4 + 2] = fmaf(-err, u.z, w[4 * s4 + 2]);
       if (4 * s4 + 3 >= s) w[4 * s4 + 3] = fmaf(-err, u.w, w[4 * s4 + 3]);
     }
-    const bool own = (q == (jj & 3));
+    const bool own = (q == k);
     w[s] = own ? wh : w[s];
     e_out[s] = own ? ev : e_out[s];
     loss = own ? fmaf(e * e, hrd2[jj], loss) : loss;
@@ -367,8 +378,8 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
     float* ehi = Err_hi + (int64_t)r * kBlock;
     float* elo = Err_lo + (int64_t)r * kBlock;
 #pragma unroll
-    for (int s = 0; s < 32; ++s) {
-      const int c = 4 * s + q;
+    for (int s = 0; s < NS; ++s) {
+      const int c = L * s + q;
       if (c < bsz) {
         crow[c] = (uint8_t)((cw[s >> 2] >> (8 * (s & 3))) & 0xFFu);
         wrow[c] = w[s];
@@ -380,8 +391,8 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
     }
   }
   if (row_loss) {
-    loss += __shfl_xor_sync(0xffffffffu, loss, 1);
-    loss += __shfl_xor_sync(0xffffffffu, loss, 2);
+#pragma unroll
+    for (int o = 1; o < L; o <<= 1) loss += __shfl_xor_sync(0xffffffffu, loss, o);
     if (active && q == 0) row_loss[r] += loss;
   }
 }
@@ -478,7 +489,7 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
   if ((e = set_smem(sweep_block_kernel<128>, us_smem)) != cudaSuccess) return e;
   if ((e = set_smem(sweep_block_kernel<32>, us_smem)) != cudaSuccess) return e;
   if ((e = set_smem(sweep_block_kernel<64>, us_smem)) != cudaSuccess) return e;
-  const int sweep_ctas = (rows * 4 + kSweepThreads - 1) / kSweepThreads;
+  const int sweep_ctas = (rows * kSweepLanes + kSweepThreads - 1) / kSweepThreads;
   const int sms = num_sms();
 
   // operands of the lazy update on the tensor cores; with a row stride that
