@@ -453,7 +453,13 @@ class LayerPipeline:
     ``shapes``: (rows, n) per linear; every linear sees ``ntok`` tokens.
     One LayerQuantizer per linear holds that linear's buffers and outputs
     (``layers[l]``).  ``run(Ws, Xs)`` enqueues everything and makes the
-    caller's stream wait for the last linear."""
+    caller's stream wait for the last linear.
+
+    Measured on a 7B decoder block (7 linears, 65536 tokens each) the overlap
+    gains nothing (0.97 to 1.00 of the one-stream time): each linear's
+    factorization and sweep take about four times its Hessian, and the
+    Hessian's persistent grid holds every SM.  ``run(..., overlap=False)``
+    gives the one-stream order."""
 
     def __init__(self, shapes, ntok: int, bits: int = 4, group_size: int = 128,
                  percdamp: float = 0.01, actorder: bool = False, sym: bool = False,
