@@ -1,4 +1,5 @@
-// Packed storage of tick indices and dequantization.
+// Packed storage of tick indices, dequantization, and the consumer of the
+// packed codes (dequant x activation).
 //
 // Page "GPTQ, with the code open", section "What quantization is, and why
 // anyone bothers": a weight is stored as the index of its tick plus, once per
@@ -7,8 +8,10 @@
 //   int4: column 8i+k  -> bits [4k, 4k+4) of 32-bit word i of the row
 //   int3: column 32i+k -> bits [3k, 3k+3) of the 96-bit little-endian word
 //         made of 32-bit words 3i, 3i+1, 3i+2 of the row.
-// All kernels are HBM-bound streaming passes: each thread owns one 32-code
-// group (128-bit loads of codes, 128-bit stores of int4 words).
+// Packing and dequantization are HBM-bound streaming passes (a thread owns a
+// 32-code group or 8 values: 128-bit loads and stores).  The dequant x
+// activation kernels follow further down: one on the FP32 pipe, one on the
+// tensor cores (mma.sync with exact bf16 (q - zero) operands).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
