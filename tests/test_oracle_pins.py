@@ -551,3 +551,28 @@ def test_hessian_symmetric_blas_route_equals_plain_product():
     ref = 2.0 * Xd @ Xd.T
     assert np.array_equal(H, H.T)
     assert np.linalg.norm(H - ref) / np.linalg.norm(ref) < 1e-14
+
+
+def test_dequant_matvec_sweep_order_equals_original_order():
+    """An act-order layer served in sweep order (codes gathered by perm,
+    contiguous groups, x gathered by the same perm) gives the same y as the
+    original order with g_idx (g_idx[c] = position of c in the sweep / g):
+    the same products, summed in another order."""
+    rng = np.random.default_rng(33)
+    for bits, rows, n, g in ((4, 6, 128, 32), (3, 5, 96, 32), (4, 4, 256, 64)):
+        codes = rng.integers(0, 2 ** bits, (rows, n))
+        perm = rng.permutation(n)
+        G_ = n // g
+        scales = rng.uniform(1e-3, 0.1, (rows, G_)).astype(np.float32)
+        zeros = rng.integers(0, 2 ** bits, (rows, G_))
+        g_idx = np.empty(n, dtype=np.int64)
+        g_idx[perm] = np.arange(n) // g
+        pack = O.pack_int4 if bits == 4 else O.pack_int3
+        x = rng.standard_normal((3, n))
+        y_sw, mag = O.dequant_matvec(pack(codes[:, perm]), bits, n, scales, zeros, x, g,
+                                     perm=perm)
+        y_or, _ = O.dequant_matvec(pack(codes), bits, n, scales, zeros, x, g, g_idx)
+        np.testing.assert_allclose(y_sw, y_or, rtol=0, atol=1e-13 * float(np.max(mag)))
+        # a planted mistake: x not gathered -- caught
+        y_bad, _ = O.dequant_matvec(pack(codes[:, perm]), bits, n, scales, zeros, x, g)
+        assert not np.allclose(y_bad, y_or)
