@@ -52,6 +52,21 @@ __device__ __forceinline__ void fwht_warp(float (&v)[VPL], int lane) {
   }
 }
 
+// Butterflies over the index bits of i inside one lane (v[i] holds element
+// base + stride * i of the block, for any base and stride).
+template <int N>
+__device__ __forceinline__ void fwht_lane(float (&v)[N]) {
+#pragma unroll
+  for (int h = 1; h < N; h <<= 1)
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      if ((i & h) == 0) {
+        const float a = v[i], b = v[i + h];
+        v[i] = a + b;
+        v[i + h] = a - b;
+      }
+}
+
 // W' = W R^T: each row's blocks of b contiguous elements, one warp per block
 // (in == out is allowed: a warp reads its whole block before writing it).
 constexpr int kRowsWarps = 8;
@@ -87,6 +102,13 @@ __global__ void __launch_bounds__(kColsTok * 32) hadamard_cols_kernel(
   constexpr int B = 32 * VPL, P = kColsTok + 1, NT = kColsTok * 32;
   constexpr int VI = 16 / (int)sizeof(TI), VO = 16 / (int)sizeof(TO);  // per 16 bytes
   extern __shared__ float tile[];  // B x P
+  // element (f, t) of the tile; for b = 1024 the token index is XOR-swizzled
+  // by the feature's 32-block, so that both column passes below (lane l on
+  // features l + 32 i, then on 32 l + i) read their 32 values from distinct
+  // banks (at most two-way in the second)
+  auto at = [](int f, int t) {
+    return VPL == 32 ? f * P + (t ^ ((f >> 5) & (kColsTok - 1))) : f * P + t;
+  };
   const int64_t f0 = (int64_t)blockIdx.y * B, t0 = (int64_t)blockIdx.x * kColsTok;
   const int tt = (int)(ntok - t0 < kColsTok ? ntok - t0 : kColsTok);
   const int tid = threadIdx.x;
@@ -99,23 +121,39 @@ __global__ void __launch_bounds__(kColsTok * 32) hadamard_cols_kernel(
       const TI* e = reinterpret_cast<const TI*>(&raw);
       const float sg = __ldg(signs + f0 + f);
 #pragma unroll
-      for (int j = 0; j < VI; ++j) tile[f * P + c * VI + j] = to_f(e + j) * sg;
+      for (int j = 0; j < VI; ++j) tile[at(f, c * VI + j)] = to_f(e + j) * sg;
     }
   } else {
     const int tc = tid % kColsTok, fr = tid / kColsTok;
     for (int f = fr; f < B; f += NT / kColsTok) {
       const float sg = __ldg(signs + f0 + f);
-      tile[f * P + tc] = tc < tt ? to_f(in + (f0 + f) * ld_in + t0 + tc) * sg : 0.f;
+      tile[at(f, tc)] = tc < tt ? to_f(in + (f0 + f) * ld_in + t0 + tc) * sg : 0.f;
     }
   }
   __syncthreads();
   const int w = tid >> 5, lane = tid & 31;
   float v[VPL];
+  if constexpr (VPL == 32) {
+    // no shuffles: the high index bits in registers (lane l: features
+    // l + 32 i), back to the tile, then the low bits (lane l: 32 l + i)
 #pragma unroll
-  for (int i = 0; i < VPL; ++i) v[i] = tile[(lane + 32 * i) * P + w];
-  fwht_warp<VPL>(v, lane);
+    for (int i = 0; i < 32; ++i) v[i] = tile[at(lane + 32 * i, w)];
+    fwht_lane<32>(v);
 #pragma unroll
-  for (int i = 0; i < VPL; ++i) tile[(lane + 32 * i) * P + w] = v[i] * scale;
+    for (int i = 0; i < 32; ++i) tile[at(lane + 32 * i, w)] = v[i];
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = tile[at(32 * lane + i, w)];
+    fwht_lane<32>(v);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) tile[at(32 * lane + i, w)] = v[i] * scale;
+  } else {
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) v[i] = tile[at(lane + 32 * i, w)];
+    fwht_warp<VPL>(v, lane);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) tile[at(lane + 32 * i, w)] = v[i] * scale;
+  }
   __syncthreads();
   if (vec_out && tt == kColsTok) {
     constexpr int kPer = kColsTok / VO;
@@ -124,13 +162,13 @@ __global__ void __launch_bounds__(kColsTok * 32) hadamard_cols_kernel(
       uint4 raw;
       TO* e = reinterpret_cast<TO*>(&raw);
 #pragma unroll
-      for (int j = 0; j < VO; ++j) from_f(e + j, tile[f * P + c * VO + j]);
+      for (int j = 0; j < VO; ++j) from_f(e + j, tile[at(f, c * VO + j)]);
       *reinterpret_cast<uint4*>(out + (f0 + f) * ld_out + t0 + c * VO) = raw;
     }
   } else {
     const int tc = tid % kColsTok, fr = tid / kColsTok;
     for (int f = fr; f < B; f += NT / kColsTok)
-      if (tc < tt) from_f(out + (f0 + f) * ld_out + t0 + tc, tile[f * P + tc]);
+      if (tc < tt) from_f(out + (f0 + f) * ld_out + t0 + tc, tile[at(f, tc)]);
   }
 }
 
