@@ -13,8 +13,10 @@
 // product.  A warp holds one block of b = 32 VPL values, lane l holding
 // elements l + 32 i: the stages over the high index bits (strides 32 .. b/2)
 // run inside each lane, the five over the low bits (strides 1 .. 16) through
-// shfl_xor.  The order of butterfly stages does not change the result's
-// definition (they commute), only the fp32 rounding.
+// shfl_xor -- or, in the column kernel for b = 1024, inside each lane again
+// after the warp re-reads its column from shared memory as elements 32 l + i.
+// The order of butterfly stages does not change the result's definition
+// (they commute), only the fp32 rounding.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -90,8 +92,9 @@ __global__ void __launch_bounds__(kRowsWarps * 32) hadamard_rows_kernel(
 }
 
 // X' = R X: a CTA stages b features x kColsTok tokens in shared memory
-// (pitch kColsTok + 1 floats: the row loads, and the column reads of the
-// warps, each land on distinct banks), then warp w transforms token column w
+// (pitch kColsTok + 1 floats, token index XOR-swizzled for b = 1024: the row
+// loads and the column passes of the warps land on distinct banks, at most
+// two-way in the second pass), then warp w transforms token column w
 // (in == out is allowed: the tile is read in full before it is written).
 constexpr int kColsTok = 16;
 
