@@ -119,3 +119,26 @@ def test_hadamard_argument_checks(lib):
     assert lib.gptq_hadamard_rows(p, 2, 4, 1024, 1024, p, 1024, p, 0, 1024, None) == INVAL
     assert lib.gptq_hadamard_rows(p, 0, 0, 1024, 1024, p, 1024, p, 0, 1024, None) == 0
     assert lib.gptq_hadamard_cols(p, 0, 1024, 0, 0, p, 1024, p, 0, 0, None) == 0
+
+
+def test_consumer_calls_with_nothing_to_do_or_bad_arguments(lib):
+    """Zero rows or zero vectors are no-ops (no pointer is touched); bad
+    widths, odd n, perm with g_idx and bad dtypes are rejected before any
+    launch."""
+    p = ctypes.c_void_p(0x1000)
+    # gptq_dequant_matvec(packed, bits, rows, n, scales, zeros, gsize, ngroups,
+    #                     g_idx, perm, x, xt, batch, y, stream)
+    assert lib.gptq_dequant_matvec(None, 4, 0, 64, None, None, 32, 2, None, None, None, 0, 1,
+                                   None, None) == 0
+    assert lib.gptq_dequant_matvec(None, 4, 8, 64, None, None, 32, 2, None, None, None, 0, 0,
+                                   None, None) == 0
+    assert lib.gptq_dequant_matvec(p, 5, 8, 64, p, p, 32, 2, None, None, p, 0, 1, p, None) == 2
+    assert lib.gptq_dequant_matvec(p, 4, 8, 60, p, p, 32, 2, None, None, p, 0, 1, p, None) == 1
+    assert lib.gptq_dequant_matvec(p, 3, 8, 48, p, p, 16, 3, None, None, p, 0, 1, p, None) == 1
+    assert lib.gptq_dequant_matvec(p, 4, 8, 64, p, p, 32, 2, p, p, p, 0, 1, p, None) == 1
+    assert lib.gptq_dequant_matvec(p, 4, 8, 64, p, p, 32, 2, None, None, p, 7, 1, p, None) == 1
+    assert lib.gptq_dequant_matvec(p, 4, 8, 64, p, p, 32, 1, None, None, p, 0, 1, p, None) == 1
+    # gptq_gather_columns_u8(src, rows, n, perm, dst, stream)
+    assert lib.gptq_gather_columns_u8(None, 0, 64, None, None, None) == 0
+    assert lib.gptq_gather_columns_u8(p, 4, 64, p, p, None) == 1  # src == dst
+    assert lib.gptq_gather_columns_u8(p, 4, 0, p, ctypes.c_void_p(0x2000), None) == 1
