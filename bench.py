@@ -516,7 +516,11 @@ def run_ours(args, rank, world, local_rank):
     roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_tflops"],
             "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": traffic,
             "kernel": "syrk_bf16_pair_kernel (+ mirror) in gptq_hessian_accumulate",
-            "peak_source": f"{pk['_source']} bf16 burst", "algorithmic_flops": flops}
+            "peak_source": f"{pk['_source']} bf16 burst", "algorithmic_flops": flops,
+            "frac_of_sustained_peak": round(
+                achieved / pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]),
+                4),
+            "gemm_equivalent_tflops": round(2.0 * n * n * N / t_h / 1e12, 2)}
 
     # the consumer of the packed codes (fused dequant x activation), outside
     # the timed step: on this layer's own output, and on the 70B down-proj
