@@ -1,0 +1,52 @@
+"""Repeatability of the kernels whose design claims it.
+
+- gptq_cholesky_inverse: the look-ahead splits each panel's trailing update
+  into a near part (caller's stream) and a far part (side stream), but every
+  element still receives the panels' updates in panel order, each once per
+  launch.  So the same H gives the same U, bit for bit, however the two
+  streams interleave.
+- gptq_dequant_matvec (tensor cores): the two column halves of every output
+  meet by two atomic adds onto zero; fp32 addition of two terms commutes, so y
+  is the same whichever half lands first.
+"""
+import numpy as np
+import pytest
+import torch
+
+import post_weight_quantization_25_b200 as G
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("n,actorder", [(1024, True), (1000, False), (4096, True)])
+def test_cholesky_inverse_is_repeatable(n, actorder):
+    g = torch.Generator(device="cuda").manual_seed(n)
+    X = torch.randn(n, 3 * n, generator=g, device="cuda").to(torch.bfloat16)
+    H = torch.zeros(n, n, device="cuda")
+    G.gptq_hessian_accumulate(H, X)
+    outs = []
+    for _ in range(3):
+        U, perm, dead, info = G.gptq_cholesky_inverse(H, 0.01, actorder)
+        torch.cuda.synchronize()
+        assert int(info.item()) == 0
+        outs.append((U.clone(), perm.clone()))
+    for U, perm in outs[1:]:
+        assert torch.equal(perm, outs[0][1])
+        assert torch.equal(U, outs[0][0])
+
+
+@pytest.mark.parametrize("bits,rows,n,g,batch", [(4, 8192, 4096, 128, 1), (4, 1000, 2048, 32, 8),
+                                                 (3, 4096, 4096, 128, 3)])
+def test_dequant_matvec_is_repeatable(bits, rows, n, g, batch):
+    rng = np.random.default_rng(rows + n)
+    codes = torch.from_numpy(rng.integers(0, 2 ** bits, (rows, n)).astype(np.uint8)).cuda()
+    packed = G.gptq_pack_int4(codes) if bits == 4 else G.gptq_pack_int3(codes)
+    scales = torch.rand(rows, n // g, device="cuda") * 0.01 + 1e-4
+    zeros = torch.randint(0, 2 ** bits, (rows, n // g), device="cuda", dtype=torch.uint8)
+    perm = torch.randperm(n, device="cuda").to(torch.int32)
+    x = torch.randn(batch, n, device="cuda").to(torch.bfloat16)
+    ys = [G.gptq_dequant_matvec(packed, bits, n, scales, zeros, x, g, perm=perm)
+          for _ in range(4)]
+    torch.cuda.synchronize()
+    for y in ys[1:]:
+        assert torch.equal(y, ys[0])
