@@ -186,12 +186,22 @@ def prepare_from_diagonal(d: np.ndarray, percdamp: float = 0.01, actorder: bool 
     return {"dead": dead, "perm": perm, "lam": lam, "d": d}
 
 
-def damped_block(H: np.ndarray, prep: dict, k0: int, k1: int) -> np.ndarray:
+def damped_block(H: np.ndarray, prep: dict, k0: int, k1: int,
+                 row_chunk: int | None = None) -> np.ndarray:
     """Rows and columns [k0, k1) (sweep order) of the prepared matrix
-    H' = H[perm][:, perm] + lam I, dead diagonal entries set to 1 first."""
+    H' = H[perm][:, perm] + lam I, dead diagonal entries set to 1 first.
+
+    ``row_chunk``: gather that many rows at a time into the fp64 result, so
+    no full-size temporary of H's own dtype is made (for n in the tens of
+    thousands); the values are the same."""
     idx = np.asarray(prep["perm"])[k0:k1]
-    B = np.array(H[np.ix_(idx, idx)], dtype=np.float64)
     m = k1 - k0
+    if row_chunk is None:
+        B = np.array(H[np.ix_(idx, idx)], dtype=np.float64)
+    else:
+        B = np.empty((m, m), dtype=np.float64)
+        for r0 in range(0, m, row_chunk):
+            B[r0:r0 + row_chunk] = H[idx[r0:r0 + row_chunk]][:, idx]
     dd = np.asarray(prep["dead"])[idx]
     B[np.arange(m)[dd], np.arange(m)[dd]] = 1.0
     B[np.arange(m), np.arange(m)] += prep["lam"]
@@ -235,6 +245,47 @@ def upper_cholesky_of_inverse(Hp: np.ndarray) -> np.ndarray:
     Hinv = Linv.T @ Linv                       # Hp^-1
     Hinv = 0.5 * (Hinv + Hinv.T)
     return np.linalg.cholesky(Hinv).T          # Hinv = U^T U
+
+
+def upper_cholesky_of_inverse_inplace(Hp: np.ndarray) -> np.ndarray:
+    """The same U as ``upper_cholesky_of_inverse``, by the same route, for
+    orders where a general inverse and a full product are too slow (n in the
+    tens of thousands): every step is the LAPACK routine for it, on one fp64
+    buffer that is overwritten (``Hp`` must be C-contiguous fp64; it becomes
+    U).  Steps, in the page's order (§ "From one repair to a whole model"):
+      Cholesky           Hp = L L^T                     (dpotrf)
+      inverse of L       Linv = L^-1, triangular        (dtrtri)
+      the inverse        Hp^-1 = Linv^T Linv            (dlauum)
+      Cholesky again     Hp^-1 = L2 L2^T, and U = L2^T  (dpotrf)
+    U is upper with Hp^-1 = U^T U; that factor is unique, so this equals the
+    general-inverse form.  Raises numpy.linalg.LinAlgError if a step fails.
+
+    The buffer is handed to LAPACK as its transpose (a Fortran-ordered view
+    of the same memory), so no copy is made: the lower triangle of that view
+    is the upper triangle of ``Hp``.
+    """
+    from scipy.linalg import lapack
+
+    if Hp.dtype != np.float64 or not Hp.flags.c_contiguous:
+        raise ValueError("Hp must be a C-contiguous float64 array")
+    F = Hp.T                                   # Fortran view; F == Hp (symmetric)
+    for name, fn, kw in (("dpotrf", lapack.dpotrf, {"lower": 1, "overwrite_a": 1, "clean": 0}),
+                         ("dtrtri", lapack.dtrtri, {"lower": 1, "overwrite_c": 1}),
+                         ("dlauum", lapack.dlauum, {"lower": 1, "overwrite_c": 1}),
+                         ("dpotrf", lapack.dpotrf, {"lower": 1, "overwrite_a": 1, "clean": 0})):
+        out, info = fn(F, **kw)
+        if info != 0:
+            raise np.linalg.LinAlgError(f"{name} failed, info={info}")
+        if not np.shares_memory(out, Hp):
+            raise RuntimeError(f"{name} did not work in place")
+    # U = L2^T: the lower triangle of F is the upper triangle of Hp; clear the rest
+    n = Hp.shape[0]
+    for r0 in range(0, n, 1024):
+        r1 = min(n, r0 + 1024)
+        blk = Hp[r0:r1]
+        rr = np.arange(r0, r1)[:, None]
+        blk[np.arange(n)[None, :] < rr] = 0.0
+    return Hp
 
 
 # --------------------------------------------------------------------------

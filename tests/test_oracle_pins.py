@@ -182,6 +182,33 @@ def test_sub_inverse_relation():
             assert U[j, j] ** 2 == pytest.approx(Fi[0, 0], rel=1e-10)
 
 
+def test_inplace_lapack_route_matches_definition():
+    """The in-place LAPACK form of the route (used at n = 28672) gives the
+    factor the definition fixes: upper, positive diagonal, U^T U H = I, rows
+    equal to the scaled shrinking inverses; it overwrites its input and
+    rejects a matrix that is not positive definite."""
+    for n, seed in ((7, 3), (12, 4), (301, 5)):
+        H, _ = _rand_spd(n, seed)
+        B = np.ascontiguousarray(H.copy())
+        U = O.upper_cholesky_of_inverse_inplace(B)
+        assert U is B
+        assert np.all(np.tril(U, -1) == 0.0)
+        assert np.all(np.diag(U) > 0)
+        np.testing.assert_allclose(U.T @ U @ H, np.eye(n), atol=1e-8)
+        if n <= 12:
+            for j in range(n):
+                Fi = np.linalg.inv(H[j:, j:])
+                np.testing.assert_allclose(U[j, j:], Fi[0] / np.sqrt(Fi[0, 0]), rtol=1e-9,
+                                           atol=1e-12)
+        ref = O.upper_cholesky_of_inverse(H)
+        assert np.linalg.norm(U - ref) / np.linalg.norm(ref) < 1e-11
+    bad = np.ascontiguousarray(np.diag([1.0, -1.0, 2.0]))
+    with pytest.raises(np.linalg.LinAlgError):
+        O.upper_cholesky_of_inverse_inplace(bad)
+    with pytest.raises(ValueError):
+        O.upper_cholesky_of_inverse_inplace(np.eye(3, dtype=np.float32))
+
+
 # ---------------------------------------------------------------- the sweep
 def _layer(rows, n, ntok, seed, corr=0.5, dead=()):
     W, X = workloads.random_layer(rows, n, ntok, seed, correlated=corr, dead=dead)
