@@ -14,9 +14,13 @@
  *
  * Conventions shared by every entry point:
  *  - Every pointer argument is DEVICE memory owned by the caller unless the
- *    comment says otherwise.  The library allocates nothing that outlives a
- *    call and keeps no state between calls (apart from the launch counter
- *    read by gptq_launch_count).
+ *    comment says otherwise.  The library allocates no device memory (every
+ *    scratch buffer is a caller workspace sized by gptq_workspace_size),
+ *    creates no stream, and keeps no state between calls apart from the
+ *    launch counter read by gptq_launch_count, the calling thread's wait
+ *    gate (gptq_set_wait_gate, a test hook) and a per-device cache of one
+ *    occupancy query.  A call given a side stream creates four CUDA events
+ *    for its enqueue and destroys them before it returns.
  *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
  *    legacy default stream).  The returned status covers argument checks and
  *    kernel launches only.  Numerical failures and device-side wait timeouts
@@ -72,11 +76,19 @@ typedef struct {
   int sym;
 } gptq_config;
 
-typedef enum { GPTQ_OP_HESSIAN = 0, GPTQ_OP_CHOLESKY = 1, GPTQ_OP_QUANTIZE = 2 } gptq_op;
+typedef enum {
+  GPTQ_OP_HESSIAN = 0,
+  GPTQ_OP_CHOLESKY = 1,
+  GPTQ_OP_QUANTIZE = 2,
+  GPTQ_OP_DEQUANT_MATVEC = 3
+} gptq_op;
 
 /* Bytes of device workspace `op` needs for these sizes (0 is possible).
- * rows/n/ntok as in the calls below; xt is the calibration dtype (hessian
- * only); cfg may be NULL except for GPTQ_OP_QUANTIZE.  Host pointer `bytes`. */
+ * rows/n/ntok as in the calls below (for GPTQ_OP_DEQUANT_MATVEC, rows is the
+ * number of activation vectors, `batch`); xt is the calibration dtype
+ * (hessian only); cfg may be NULL except for GPTQ_OP_QUANTIZE.  Host
+ * pointer `bytes`.  Workspaces are 256-byte aligned; their contents on entry
+ * do not matter. */
 gptq_status gptq_workspace_size(int op, int64_t rows, int64_t n, int64_t ntok, gptq_dtype xt,
                                 const gptq_config* cfg, size_t* bytes);
 
@@ -94,9 +106,14 @@ gptq_status gptq_workspace_size(int op, int64_t rows, int64_t n, int64_t ntok, g
  *          of 16 bytes; H 16-byte aligned.
  *   token_major  must be 0.
  *   ws     workspace of gptq_workspace_size(GPTQ_OP_HESSIAN, 0, n, ntok, xt)
- *          bytes (0 for bf16).
+ *          bytes: counters of the ordered reduction (below), and for fp32 X
+ *          the bf16 parts.
  *   info   optional device int32: set to GPTQ_ERR_TIMEOUT if a pipeline wait
- *          inside the kernel gave up (then H is incomplete).  Not cleared.  */
+ *          inside the kernel gave up (then H is incomplete).  Not cleared.
+ * The result is reproducible bit for bit: the tokens are cut into chunks
+ * (for parallelism) and the chunks of each output tile are added into H in
+ * chunk order, never by atomics.  Calls that overlap on the GPU must not
+ * share a workspace or an H. */
 gptq_status gptq_hessian_accumulate(float* H, const void* X, gptq_dtype xt, int64_t n,
                                     int64_t ntok, int64_t ldx, int token_major, float alpha,
                                     void* ws, size_t ws_bytes, int32_t* info, void* stream);
@@ -119,22 +136,31 @@ gptq_status gptq_hessian_accumulate(float* H, const void* X, gptq_dtype xt, int6
  * last sweep position towards the first, so this is the highest failing
  * position); -1 if diag(H) holds a NaN or an infinity; -2 if a bounded wait
  * inside a tensor-core kernel gave up.  On failure U is
- * undefined.  ws: gptq_workspace_size(GPTQ_OP_CHOLESKY, 0, n, 0, .., NULL). */
+ * undefined.  ws: gptq_workspace_size(GPTQ_OP_CHOLESKY, 0, n, 0, .., NULL).
+ * side_stream: NULL (or equal to stream) runs everything on `stream`.
+ * Otherwise a second stream of the caller's, used for look-ahead: the part
+ * of each panel's trailing update that the next panel does not need runs
+ * there, overlapping the next panel's factorisation; the call leaves
+ * `stream` ordered after all of it.  The caller must not use side_stream for
+ * anything that may run between the call's enqueue and the completion of
+ * its work on `stream`; results are identical either way. */
 gptq_status gptq_cholesky_inverse(const float* H, int64_t n, float percdamp, int actorder,
                                   float* U, int32_t* perm, uint8_t* dead, int32_t* info,
-                                  void* ws, size_t ws_bytes, void* stream);
+                                  void* ws, size_t ws_bytes, void* stream, void* side_stream);
 
 /* gptq_cholesky_inverse for callers that cannot allocate device memory.
  * The pages have no counterpart of this entry point; it exists for host
  * programs that own all device memory in a fixed pool and forbid allocation
  * while running, so they can neither call cudaMalloc nor pass a workspace.
  * Same arguments, results and `info` contract as gptq_cholesky_inverse, minus
- * the workspace: the scratch is a 21.1 MB array built into the library, so
- * n must be <= 2048 (larger n returns GPTQ_ERR_WORKSPACE).  The library looks
+ * the workspace and the side stream: the scratch is a 21.1 MB array built
+ * into the library, so n must be <= 2048 (larger n returns
+ * GPTQ_ERR_WORKSPACE), and everything runs on `stream`.  The library looks
  * up that array's device address once per device, in the first call made with
  * that device current; make that first call before any stream capture.  All
  * calls share the array: calls that overlap on the GPU race on it, so the
- * caller must serialise them (e.g. one stream).  No call allocates memory. */
+ * caller must serialise them (e.g. one stream).  No call allocates device
+ * memory or creates a stream or an event. */
 gptq_status gptq_cholesky_inverse_noalloc(const float* H, int64_t n, float percdamp,
                                           int actorder, float* U, int32_t* perm, uint8_t* dead,
                                           int32_t* info, void* stream);
@@ -148,7 +174,8 @@ gptq_status gptq_cholesky_inverse_noalloc(const float* H, int64_t n, float percd
  *   q = clamp(rint(w / scale) + zero, 0, 2^bits - 1);  w_hat = scale (q - zero);
  *   err = (w - w_hat) / U[j][j];  W[:, j+1:] -= err * U[j, j+1:]
  * with the update past the current 128-column block applied once per block.
- * All arithmetic is fp32 with IEEE division and round-half-to-even.
+ * All arithmetic is fp32 with IEEE division and round-half-to-even.  The
+ * result is reproducible bit for bit.
  *   W        rows x n in wt (original column order); not modified.
  *   U, perm, dead  from gptq_cholesky_inverse (perm may be NULL = identity).
  *   codes    uint8 rows x n, ORIGINAL column order.
@@ -157,12 +184,19 @@ gptq_status gptq_cholesky_inverse_noalloc(const float* H, int64_t n, float percd
  *   g_idx    optional int32[n]: group of each original column.
  *   Wq       optional fp32 rows x n, original order: the dequantized weights.
  *   row_loss optional fp32[rows]: sum over columns of (w - w_hat)^2 / (2 U_jj^2).
- *   ws       gptq_workspace_size(GPTQ_OP_QUANTIZE, rows, n, 0, .., cfg). */
+ *   ws       gptq_workspace_size(GPTQ_OP_QUANTIZE, rows, n, 0, .., cfg).
+ *   info     optional device int32, set to 0 by the call, then to -2 if a
+ *            bounded wait inside a tensor-core kernel gave up (the outputs
+ *            are then undefined).
+ *   side_stream  as for gptq_cholesky_inverse: NULL runs everything on
+ *            `stream`; a second stream lets the lazy update of the columns
+ *            past the next block overlap the next block's sweep. */
 gptq_status gptq_quantize_layer(const void* W, gptq_dtype wt, int64_t rows, int64_t n,
                                 const float* U, const int32_t* perm, const uint8_t* dead,
                                 const gptq_config* cfg, uint8_t* codes, float* scales,
                                 uint8_t* zeros, int32_t* g_idx, float* Wq, float* row_loss,
-                                void* ws, size_t ws_bytes, void* stream);
+                                void* ws, size_t ws_bytes, int32_t* info, void* stream,
+                                void* side_stream);
 
 /* Packed storage of tick indices (page "GPTQ, with the code open", section
  * "What quantization is, and why anyone bothers": store the tick index).  The
@@ -202,9 +236,8 @@ gptq_status gptq_dequant(const uint32_t* packed, int bits, int64_t rows, int64_t
  * (q - zero) pairs with x in fp32 MMA accumulators, scales each group's sum
  * once, and adds the two column halves of every output onto zeros (two
  * terms, so the result does not depend on their order).  It first writes x
- * (gathered by perm, if given) into batch x n bf16 of stream-ordered scratch
- * from a pool private to this library, and zeroes y.  Everything else: the
- * FP32-pipe kernel, one rounded FMA per term.
+ * (gathered by perm, if given) into the workspace as batch x n bf16, and
+ * zeroes y.  Everything else: the FP32-pipe kernel, one rounded FMA per term.
  *   packed, scales, zeros, group_size, n_groups, g_idx: exactly as for
  *          gptq_dequant (same layout, same single-multiply w_hat).
  *   perm   NULL, or (with g_idx NULL) the sweep order of an act-order layer:
@@ -216,13 +249,14 @@ gptq_status gptq_dequant(const uint32_t* packed, int bits, int64_t rows, int64_t
  *   x      batch x n activations, row-major, xt = GPTQ_BF16 or GPTQ_F32.
  *   y      batch x rows fp32 (written), y[b][r] = sum_c w_hat[r][c] x[b][c],
  *          summed in fp32.
+ *   ws     gptq_workspace_size(GPTQ_OP_DEQUANT_MATVEC, batch, n, ...) bytes.
  * batch >= 0 (any size; launched in groups of 8, 4, 2, 1).  Errors as for
  * gptq_dequant; perm together with g_idx is invalid. */
 gptq_status gptq_dequant_matvec(const uint32_t* packed, int bits, int64_t rows, int64_t n,
                                 const float* scales, const uint8_t* zeros, int group_size,
                                 int64_t n_groups, const int32_t* g_idx, const int32_t* perm,
                                 const void* x, gptq_dtype xt, int64_t batch, float* y,
-                                void* stream);
+                                void* ws, size_t ws_bytes, void* stream);
 
 /* dst[r][k] = src[r][perm[k]] for a rows x n byte matrix (device pointers;
  * perm int32[n], a permutation of 0..n-1).  With the `perm` of
@@ -262,8 +296,21 @@ gptq_status gptq_hadamard_cols(const void* in, gptq_dtype it, int64_t n, int64_t
 const char* gptq_status_string(int status);
 
 /* Diagnostics (host): number of kernels this library has enqueued in this
- * process so far.  The one piece of process-wide state the library keeps. */
+ * process so far. */
 int64_t gptq_launch_count(void);
+
+/* Test hook for the bounded waits (host).  Every wait inside the library's
+ * tensor-core kernels (gptq_hessian_accumulate, the trailing updates of
+ * gptq_cholesky_inverse and gptq_quantize_layer) gives up after 1 s and
+ * reports through the call's `info` word instead of hanging.  To exercise
+ * that path, a test passes a device int32 `gate` that holds 0 and a short
+ * limit_ns (1..1e9): every such kernel that the calling host thread enqueues
+ * afterwards first waits for *gate != 0 with nothing in flight, gives up
+ * after limit_ns, and the call reports its timeout as documented.  gate =
+ * NULL restores the normal behaviour (limit_ns ignored).  The setting
+ * belongs to the calling host thread only.  Returns GPTQ_ERR_INVALID_ARG for
+ * a limit out of range. */
+gptq_status gptq_set_wait_gate(const int32_t* gate, int64_t limit_ns);
 
 /* Self-test of the division the sweep uses to round w / scale (a
  * correctly rounded binary32 division by Markstein's FMA method, with the

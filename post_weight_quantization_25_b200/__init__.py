@@ -18,14 +18,14 @@ import dataclasses
 import torch
 
 from . import _lib
-from ._lib import (GPTQ_BF16, GPTQ_F32, GPTQ_OP_CHOLESKY, GPTQ_OP_HESSIAN, GPTQ_OP_QUANTIZE,
-                   GptqConfig)
+from ._lib import (GPTQ_BF16, GPTQ_F32, GPTQ_OP_CHOLESKY, GPTQ_OP_DEQUANT_MATVEC, GPTQ_OP_HESSIAN,
+                   GPTQ_OP_QUANTIZE, GptqConfig)
 
 __all__ = ["GptqError", "GptqConfig", "LayerPipeline", "gptq_workspace_size",
            "gptq_hadamard_rows", "gptq_hadamard_cols", "gptq_hessian_accumulate",
            "gptq_cholesky_inverse", "gptq_quantize_layer", "gptq_pack_int4", "gptq_pack_int3",
            "gptq_dequant", "gptq_dequant_matvec", "gptq_gather_columns_u8", "gptq_status_string",
-           "make_config",
+           "make_config", "gptq_set_wait_gate", "gptq_launch_count",
            "QuantizedLinear",
            "quantize_linear", "LayerQuantizer", "library"]
 
@@ -47,6 +47,18 @@ def gptq_launch_count() -> int:
     return int(library().gptq_launch_count())
 
 
+def gptq_set_wait_gate(gate: torch.Tensor | None, limit_ns: int = 1_000_000_000) -> None:
+    """Test hook of the bounded device waits (see include/gptq.h): with a
+    device int32 ``gate`` holding 0, the tensor-core kernels this thread
+    enqueues next wait for it and give up after ``limit_ns``; None restores
+    the normal behaviour."""
+    if gate is not None:
+        _need_cuda(gate)
+        if gate.dtype != torch.int32:
+            raise GptqError("gate must be a device int32 tensor")
+    _check(library().gptq_set_wait_gate(_p(gate), int(limit_ns)), "gptq_set_wait_gate")
+
+
 def _check(status: int, what: str) -> None:
     if status != 0:
         raise GptqError(f"{what}: {gptq_status_string(status)} (status {status})")
@@ -60,6 +72,11 @@ def _stream(stream) -> int | None:
     if stream is None:
         stream = torch.cuda.current_stream()
     return stream.cuda_stream
+
+
+def _side(side_stream) -> int | None:
+    """A second stream for look-ahead, or None (one stream)."""
+    return None if side_stream is None else side_stream.cuda_stream
 
 
 def _dtype_code(dt: torch.dtype) -> int:
@@ -119,7 +136,7 @@ def gptq_hessian_accumulate(H: torch.Tensor, X: torch.Tensor, alpha: float = 2.0
         raise GptqError("X must have contiguous rows (tokens)")
     need = gptq_workspace_size(GPTQ_OP_HESSIAN, 0, n, ntok, X.dtype)
     ws = _workspace(need, X.device, ws)
-    wp, wn = _aligned_ptr(ws) if need else (None, 0)
+    wp, wn = _aligned_ptr(ws)
     st = library().gptq_hessian_accumulate(_p(H), _p(X), _dtype_code(X.dtype), n, ntok,
                                            X.stride(0), 0, float(alpha), wp, wn, _p(info),
                                            _stream(stream))
@@ -128,9 +145,11 @@ def gptq_hessian_accumulate(H: torch.Tensor, X: torch.Tensor, alpha: float = 2.0
 
 
 def gptq_cholesky_inverse(H: torch.Tensor, percdamp: float = 0.01, actorder: bool = False,
-                          U=None, perm=None, dead=None, info=None, ws=None, stream=None):
+                          U=None, perm=None, dead=None, info=None, ws=None, stream=None,
+                          side_stream=None):
     """Dead inputs, act-order, damping and U (upper, H'^-1 = U^T U).
-    Returns (U, perm, dead, info); info is a device int32 (0 = success)."""
+    Returns (U, perm, dead, info); info is a device int32 (0 = success).
+    side_stream: a second torch.cuda.Stream for the look-ahead (same result)."""
     _need_cuda(H)
     n = H.shape[0]
     dev = H.device
@@ -142,7 +161,8 @@ def gptq_cholesky_inverse(H: torch.Tensor, percdamp: float = 0.01, actorder: boo
     ws = _workspace(need, dev, ws)
     wp, wn = _aligned_ptr(ws)
     st = library().gptq_cholesky_inverse(_p(H), n, float(percdamp), int(bool(actorder)), _p(U),
-                                         _p(perm), _p(dead), _p(info), wp, wn, _stream(stream))
+                                         _p(perm), _p(dead), _p(info), wp, wn, _stream(stream),
+                                         _side(side_stream))
     _check(st, "gptq_cholesky_inverse")
     return U, perm, dead, info
 
@@ -164,8 +184,10 @@ def gptq_cholesky_inverse_noalloc(H: torch.Tensor, percdamp: float, actorder: bo
 def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, perm, dead, cfg: GptqConfig,
                         codes=None, scales=None, zeros=None, g_idx=None, Wq=None, row_loss=None,
                         want_g_idx: bool = True, want_wq: bool = False, want_loss: bool = False,
-                        ws=None, stream=None) -> dict:
-    """The column sweep.  Returns dict(codes, scales, zeros, g_idx, Wq, row_loss)."""
+                        ws=None, info=None, stream=None, side_stream=None) -> dict:
+    """The column sweep.  Returns dict(codes, scales, zeros, g_idx, Wq, row_loss).
+    info: optional device int32 (set to 0, or -2 if a device wait gave up);
+    side_stream: a second torch.cuda.Stream for the look-ahead (same result)."""
     _need_cuda(W, U, perm, dead)
     rows, n = W.shape
     if not W.is_contiguous():
@@ -187,7 +209,7 @@ def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, perm, dead, cfg: GptqC
     st = library().gptq_quantize_layer(_p(W), _dtype_code(W.dtype), rows, n, _p(U), _p(perm),
                                        _p(dead), ctypes.byref(cfg), _p(codes), _p(scales),
                                        _p(zeros), _p(g_idx), _p(Wq), _p(row_loss), wp, wn,
-                                       _stream(stream))
+                                       _p(info), _stream(stream), _side(side_stream))
     _check(st, "gptq_quantize_layer")
     return {"codes": codes, "scales": scales, "zeros": zeros, "g_idx": g_idx, "Wq": Wq,
             "row_loss": row_loss}
@@ -238,7 +260,7 @@ def gptq_gather_columns_u8(src: torch.Tensor, perm: torch.Tensor, out=None,
 
 def gptq_dequant_matvec(packed: torch.Tensor, bits: int, n: int, scales: torch.Tensor,
                         zeros: torch.Tensor, x: torch.Tensor, group_size: int = -1, g_idx=None,
-                        perm=None, out=None, stream=None) -> torch.Tensor:
+                        perm=None, out=None, ws=None, stream=None) -> torch.Tensor:
     """y = x w_hat^T with w_hat dequantized on the fly from the packed codes.
     x: (batch, n) or (n,) bf16/fp32 on the GPU; returns (batch, rows) fp32
     (or (rows,) for a 1-D x).  perm: the codes are packed in sweep order
@@ -250,9 +272,12 @@ def gptq_dequant_matvec(packed: torch.Tensor, bits: int, n: int, scales: torch.T
         raise GptqError("x must be a contiguous (batch, n) tensor")
     batch = x2.shape[0]
     out = torch.empty(batch, rows, dtype=torch.float32, device=packed.device) if out is None else out
+    need = gptq_workspace_size(GPTQ_OP_DEQUANT_MATVEC, batch, n)
+    ws = _workspace(need, packed.device, ws)
+    wp, wn = _aligned_ptr(ws)
     st = library().gptq_dequant_matvec(_p(packed), int(bits), rows, int(n), _p(scales), _p(zeros),
                                        int(group_size), scales.shape[1], _p(g_idx), _p(perm),
-                                       _p(x2), _dtype_code(x2.dtype), batch, _p(out),
+                                       _p(x2), _dtype_code(x2.dtype), batch, _p(out), wp, wn,
                                        _stream(stream))
     _check(st, "gptq_dequant_matvec")
     return out.reshape(-1) if x.dim() == 1 else out
@@ -348,7 +373,9 @@ class LayerQuantizer:
     attributes (``H``, ``U``, ``perm``, ``dead``, ``info``, ``codes``,
     ``scales``, ``zeros``, ``g_idx``, ``packed``, ``deq`` and, if asked for,
     ``Wq`` and ``row_loss``).  ``events``: six CUDA events recorded around the
-    five stages, for timing.
+    five stages, for timing.  ``side``: the quantizer's own second stream,
+    given to the factorisation and the sweep for their look-ahead
+    (``lookahead=False``: everything on the caller's stream; same results).
     """
 
     STAGES = ("hessian", "cholesky_inverse", "sweep", "pack", "dequant")
@@ -357,7 +384,8 @@ class LayerQuantizer:
                  percdamp: float = 0.01, actorder: bool = False,
                  x_dtype: torch.dtype = torch.bfloat16, w_dtype: torch.dtype = torch.bfloat16,
                  out_dtype: torch.dtype = torch.bfloat16, want_wq: bool = False,
-                 want_loss: bool = False, sym: bool = False, device=None):
+                 want_loss: bool = False, sym: bool = False, device=None,
+                 lookahead: bool = True):
         if bits == 4 and n % 8:
             raise GptqError("int4 packing needs n % 8 == 0")
         if bits == 3 and n % 32:
@@ -376,6 +404,8 @@ class LayerQuantizer:
         self.dead = torch.empty(n, dtype=torch.uint8, device=dev)
         self.info = torch.zeros(1, dtype=torch.int32, device=dev)
         self.info_h = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.info_q = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.side = torch.cuda.Stream(dev) if lookahead else None
         self.codes = torch.empty(rows, n, dtype=torch.uint8, device=dev)
         self.scales = torch.empty(rows, G, dtype=f32, device=dev)
         self.zeros = torch.empty(rows, G, dtype=torch.uint8, device=dev)
@@ -406,12 +436,12 @@ class LayerQuantizer:
         """Everything after the Hessian, on `stream`: U, the sweep, packing,
         dequantization.  mark(i) is called after stage i (2..5)."""
         gptq_cholesky_inverse(self.H, self.percdamp, self.actorder, self.U, self.perm, self.dead,
-                              self.info, ws=self.ws_c, stream=stream)
+                              self.info, ws=self.ws_c, stream=stream, side_stream=self.side)
         if mark:
             mark(2)
         gptq_quantize_layer(W, self.U, self.perm, self.dead, self.cfg, self.codes, self.scales,
                             self.zeros, self.g_idx, self.Wq, self.row_loss, ws=self.ws_q,
-                            stream=stream)
+                            info=self.info_q, stream=stream, side_stream=self.side)
         if mark:
             mark(3)
         self._pack(self.codes, self.packed, stream=stream)
@@ -436,9 +466,10 @@ class LayerQuantizer:
 
     def check_info(self) -> None:
         """Raises GptqError if a device status word reports a failure (syncs)."""
-        ci, hi = int(self.info.item()), int(self.info_h.item())
-        if ci != 0 or hi != 0:
-            raise GptqError(f"device status: cholesky info {ci}, hessian info {hi}")
+        ci, hi, qi = int(self.info.item()), int(self.info_h.item()), int(self.info_q.item())
+        if ci != 0 or hi != 0 or qi != 0:
+            raise GptqError(f"device status: cholesky info {ci}, hessian info {hi}, "
+                            f"sweep info {qi}")
 
 
 class LayerPipeline:
@@ -456,10 +487,11 @@ class LayerPipeline:
     caller's stream wait for the last linear.
 
     Measured on a 7B decoder block (7 linears, 65536 tokens each) the overlap
-    gains nothing (0.97 to 1.00 of the one-stream time): each linear's
-    factorization and sweep take about four times its Hessian, and the
-    Hessian's persistent grid holds every SM.  ``run(..., overlap=False)``
-    gives the one-stream order."""
+    gains nothing (0.96 to 1.00 of the one-stream time): the Hessian's
+    persistent grid holds every SM, so the factorisation's and the sweep's
+    kernels only get SMs when it ends.  So ``run`` uses the one-stream order
+    unless ``overlap=True`` is asked for.
+    """
 
     def __init__(self, shapes, ntok: int, bits: int = 4, group_size: int = 128,
                  percdamp: float = 0.01, actorder: bool = False, sym: bool = False,
@@ -477,9 +509,10 @@ class LayerPipeline:
         self.ev_start = torch.cuda.Event()
         self.ev_done = torch.cuda.Event()
 
-    def run(self, Ws, Xs, stream=None, overlap: bool = True):
-        """overlap=False runs the same work one linear after another on the
-        caller's stream (the reference order)."""
+    def run(self, Ws, Xs, stream=None, overlap: bool = False):
+        """overlap=False (the default) runs the work one linear after another
+        on the caller's stream; overlap=True puts each next Hessian on a
+        second stream (same results)."""
         s = torch.cuda.current_stream() if stream is None else stream
         if len(Ws) != len(self.layers) or len(Xs) != len(self.layers):
             raise GptqError("one W and one X per linear")

@@ -22,12 +22,13 @@ GPTQ_F32 = 1
 GPTQ_OP_HESSIAN = 0
 GPTQ_OP_CHOLESKY = 1
 GPTQ_OP_QUANTIZE = 2
+GPTQ_OP_DEQUANT_MATVEC = 3
 
 EXPORTS = ("gptq_workspace_size", "gptq_hessian_accumulate", "gptq_cholesky_inverse",
            "gptq_quantize_layer", "gptq_pack_int4", "gptq_pack_int3", "gptq_dequant",
            "gptq_status_string", "gptq_launch_count", "gptq_cholesky_inverse_noalloc",
            "gptq_selftest_division", "gptq_dequant_matvec", "gptq_gather_columns_u8",
-           "gptq_hadamard_rows", "gptq_hadamard_cols")
+           "gptq_hadamard_rows", "gptq_hadamard_cols", "gptq_set_wait_gate")
 
 
 class GptqConfig(ctypes.Structure):
@@ -47,10 +48,11 @@ _SIGNATURES = {
                                    ctypes.POINTER(_sz)]),
     "gptq_hessian_accumulate": (_int, [_vp, _vp, _int, _i64, _i64, _i64, _int, _f, _vp, _sz,
                                        _vp, _vp]),
-    "gptq_cholesky_inverse": (_int, [_vp, _i64, _f, _int, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "gptq_cholesky_inverse": (_int, [_vp, _i64, _f, _int, _vp, _vp, _vp, _vp, _vp, _sz, _vp,
+                                     _vp]),
     "gptq_quantize_layer": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _vp,
                                    ctypes.POINTER(GptqConfig), _vp, _vp, _vp, _vp, _vp, _vp,
-                                   _vp, _sz, _vp]),
+                                   _vp, _sz, _vp, _vp, _vp]),
     "gptq_pack_int4": (_int, [_vp, _i64, _i64, _vp, _vp]),
     "gptq_pack_int3": (_int, [_vp, _i64, _i64, _vp, _vp]),
     "gptq_dequant": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _int, _i64, _vp, _vp, _int, _vp]),
@@ -59,10 +61,11 @@ _SIGNATURES = {
     "gptq_cholesky_inverse_noalloc": (_int, [_vp, _i64, _f, _int, _vp, _vp, _vp, _vp, _vp]),
     "gptq_selftest_division": (_int, [_vp, _vp, _i64, _vp, _vp]),
     "gptq_dequant_matvec": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _int, _i64, _vp, _vp, _vp,
-                                   _int, _i64, _vp, _vp]),
+                                   _int, _i64, _vp, _vp, _sz, _vp]),
     "gptq_gather_columns_u8": (_int, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "gptq_hadamard_rows": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _int, _vp, _int, _i64, _vp]),
     "gptq_hadamard_cols": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _int, _vp, _int, _i64, _vp]),
+    "gptq_set_wait_gate": (_int, [_vp, _i64]),
 }
 
 _LIB = None

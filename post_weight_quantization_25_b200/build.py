@@ -32,17 +32,32 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
 
 
+def _flags(verbose: bool) -> list[str]:
+    f = ["-O3", "-lineinfo", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
+         "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
+    return (["-Xptxas=-v"] + f) if verbose else f
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every source to an object file in parallel (the files share
+    no device symbols), then link the shared library."""
     if not force and not _stale():
         return LIB
-    cmd = [_nvcc(), "-O3", "-lineinfo", "-std=c++17",
-           "-gencode", "arch=compute_100a,code=sm_100a",
-           "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr",
-           "-I", os.path.join(ROOT, "include"),
-           "-o", LIB + ".tmp"] + [os.path.join(CSRC, f) for f in SOURCES]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-        print(" ".join(cmd), file=sys.stderr)
+    from concurrent.futures import ThreadPoolExecutor
+    objdir = os.path.join(PKG, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    objs = [os.path.join(objdir, os.path.splitext(f)[0] + ".o") for f in SOURCES]
+
+    def compile_one(i: int) -> None:
+        cmd = [_nvcc()] + _flags(verbose) + ["-c", os.path.join(CSRC, SOURCES[i]), "-o", objs[i]]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        subprocess.run(cmd, check=True)
+
+    with ThreadPoolExecutor(max_workers=min(len(SOURCES), os.cpu_count() or 1)) as ex:
+        list(ex.map(compile_one, range(len(SOURCES))))
+    cmd = [_nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o",
+           LIB + ".tmp"] + objs
     subprocess.run(cmd, check=True)
     os.replace(LIB + ".tmp", LIB)
     return LIB

@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(kDiagThreads) chol_diag_kernel(const float* __
 // x = v L^-T for every vector of panel p: vectors [0, nA) are rows
 // kb+bs+v of A, vectors [nA, nA + kb + bs) are rows v - nA of RT (both
 // restricted to the panel's columns [kb, kb + bs)).  The result goes, split
-// into its TF32 part and remainder, to row g of PBh / PBl (g = the vector's
+// into its TF32 part and remainder, to row g (row pitch ldpb) of PBh / PBl (g = the vector's
 // row in A or RT); RT rows also get x written back.
 // 32 vectors per CTA; stage j: thread (v, cq) = (tid / 8, tid % 8) owns
 // columns 32 j + 4 cq .. + 3 of vector v.
@@ -315,7 +315,7 @@ constexpr size_t kApplySmemBytes =
 
 __global__ void __launch_bounds__(kApplyThreads) panel_apply_kernel(
     const float* __restrict__ A, float* __restrict__ RT, int n, int p,
-    const float* __restrict__ diag_out, float* __restrict__ PBh, float* __restrict__ PBl,
+    const float* __restrict__ diag_out, float* __restrict__ PBh, float* __restrict__ PBl, int ldpb,
     const int32_t* __restrict__ info) {
   if (*(volatile const int32_t*)info != 0) return;
   extern __shared__ __align__(16) float asmem[];
@@ -392,8 +392,8 @@ __global__ void __launch_bounds__(kApplyThreads) panel_apply_kernel(
       hv[i] = ptx::tf32_hi(xv[i]);
       lv[i] = xv[i] - hv[i];
     }
-    *reinterpret_cast<float4*>(PBh + g * 128 + c4) = make_float4(hv[0], hv[1], hv[2], hv[3]);
-    *reinterpret_cast<float4*>(PBl + g * 128 + c4) = make_float4(lv[0], lv[1], lv[2], lv[3]);
+    *reinterpret_cast<float4*>(PBh + g * ldpb + c4) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+    *reinterpret_cast<float4*>(PBl + g * ldpb + c4) = make_float4(lv[0], lv[1], lv[2], lv[3]);
     if (is_rt) {
       float* rt = RT + g * n + kb;
 #pragma unroll

@@ -32,8 +32,6 @@
 #include <cmath>
 #include <cstdint>
 
-#include <mutex>
-
 #include "gptq_internal.cuh"
 #include "chol_diag.cuh"
 #include "panel_gemm.cuh"
@@ -44,12 +42,24 @@ namespace {
 constexpr int kPanel = kBlock;  // 128
 constexpr int32_t kInfoTimeout = -2;  // `info` value when a device wait gave up
 
+// Two-level blocking for large n: inside a super-panel of kSuperPanelCols
+// columns the trailing updates are rank-128 (one per panel) and stop at the
+// super-panel's end; the columns past it are updated once per super-panel
+// with all its panels' vectors (K up to kSuperPanelCols), so the trailing
+// matrix is read and written once per super-panel instead of once per panel.
+// Smaller n uses one level (the super-panel is the panel).
+constexpr int kSuperPanelCols = 1024;
+constexpr int64_t kTwoLevelMinN = 8192;
+constexpr int64_t super_panel_cols(int64_t n) {
+  return n >= kTwoLevelMinN ? kSuperPanelCols : kPanel;
+}
+
 struct CholWs {
   float* A;       // n x n, lower part used: J P^T H P J + lambda I
   float* dprime;  // n: diag(H) with dead entries set to 1
   double* lam;    // 1: damping
-  float* PBh[2];  // n x 128: a panel's solved vectors, TF32 part (panel p uses [p % 2])
-  float* PBl[2];  // n x 128: remainder
+  float* PBh[2];  // n x SP: a super-panel's solved vectors, TF32 part (super-panels alternate)
+  float* PBl[2];  // n x SP: remainder
   float* Dout;    // the diagonal step's outputs: L^T of the block, inverted leaves
 };
 
@@ -59,7 +69,8 @@ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // allocation-free entry point below, hence constexpr).
 constexpr size_t chol_ws_bytes(int64_t n) {
   return align_up(sizeof(float) * n * n, 256) + align_up(sizeof(float) * n, 256) + 256 +
-         4 * align_up(sizeof(float) * n * kPanel, 256) + sizeof(float) * kDiagOutFloats;
+         4 * align_up(sizeof(float) * n * super_panel_cols(n), 256) +
+         sizeof(float) * kDiagOutFloats;
 }
 
 CholWs carve(void* ws, int64_t n) {
@@ -71,11 +82,12 @@ CholWs carve(void* ws, int64_t n) {
   p += align_up(sizeof(float) * n, 256);
   w.lam = reinterpret_cast<double*>(p);
   p += 256;
+  const int64_t sp = super_panel_cols(n);
   for (int b = 0; b < 2; ++b) {
     w.PBh[b] = reinterpret_cast<float*>(p);
-    p += align_up(sizeof(float) * n * kPanel, 256);
+    p += align_up(sizeof(float) * n * sp, 256);
     w.PBl[b] = reinterpret_cast<float*>(p);
-    p += align_up(sizeof(float) * n * kPanel, 256);
+    p += align_up(sizeof(float) * n * sp, 256);
   }
   w.Dout = reinterpret_cast<float*>(p);
   return w;
@@ -183,6 +195,7 @@ struct CholTrailItems {
   float* RT;
   int n, p, nblk;
   int cb_lo, cb_hi;  // column blocks [cb_lo, cb_hi) of this launch
+  int pk;            // column of panel p's vectors in the super-panel buffer
   // row block R updates column blocks [p + 1, R] of A (R > p) or
   // [p + 1, nblk) of RT (R <= p), clipped to the window
   __host__ __device__ int col_lo() const { return cb_lo > p + 1 ? cb_lo : p + 1; }
@@ -204,12 +217,56 @@ struct CholTrailItems {
     I.cx0 = c0;
     I.cy0 = R * kPanel;
     I.prow = R * kPanel;
-    I.pkx = 0;
+    I.pkx = pk;
     I.qrow0 = c0;
-    I.qkx = 0;
+    I.qkx = pk;
     I.nq = item_nq(R);
     I.mext = min(kPanel, n - R * kPanel);
     I.cext_last = min(kPanel, n - c0 - kPanel * (I.nq - 1));
+    I.nkb = kPanel / 32;
+    return I;
+  }
+};
+
+// The update past a finished super-panel [P0, P1) (panels), for the column
+// blocks [cb_lo, cb_hi) at or past P1, with all its panels' vectors at once
+// (stream_gemm_kernel):
+//   R >= P1: lower tiles A[R][S] -= sum_{P0 <= p < P1} L_Rp L_Sp^T, P1 <= S <= R
+//   R <  P1: tiles RT[R][S] -= sum_{max(P0, R) <= p < P1} RT[R][p] L_Sp^T, S >= P1
+// (a row block inside the super-panel is a right-hand-side row only for the
+// panels at or after it, so its K range starts there).
+struct CholSuperItems {
+  float* A;
+  float* RT;
+  int n, P0, P1, nblk;
+  int cb_lo, cb_hi;
+  __host__ __device__ int col_lo() const { return cb_lo > P1 ? cb_lo : P1; }
+  __host__ __device__ int col_hi(int R) const {
+    const int h = R >= P1 ? R + 1 : nblk;
+    return h < cb_hi ? h : cb_hi;
+  }
+  __host__ __device__ int num_items() const { return nblk; }
+  __host__ __device__ int item_nq(int R) const {
+    const int q = col_hi(R) - col_lo();
+    return q > 0 ? q : 0;
+  }
+  __device__ PgItem item(int R) const {
+    PgItem I;
+    const int c0 = col_lo() * kPanel;
+    const int kp0 = R >= P1 ? P0 : (R > P0 ? R : P0);  // first panel that reaches row block R
+    I.C0 = (R >= P1 ? A : RT) + (int64_t)R * kPanel * n + c0;
+    I.ldc = n;
+    I.cmap = R >= P1 ? 0 : 1;
+    I.cx0 = c0;
+    I.cy0 = R * kPanel;
+    I.prow = R * kPanel;
+    I.pkx = (kp0 - P0) * kPanel;
+    I.qrow0 = c0;
+    I.qkx = I.pkx;
+    I.nq = item_nq(R);
+    I.mext = min(kPanel, n - R * kPanel);
+    I.cext_last = min(kPanel, n - c0 - kPanel * (I.nq - 1));
+    I.nkb = (P1 - kp0) * (kPanel / 32);
     return I;
   }
 };
@@ -254,7 +311,7 @@ size_t cholesky_workspace_bytes(int64_t n) { return chol_ws_bytes(n); }
 
 cudaError_t launch_cholesky_inverse(const float* H, int64_t n64, float percdamp, int actorder,
                                     float* U, int32_t* perm, uint8_t* dead, int32_t* info,
-                                    void* ws, cudaStream_t s) {
+                                    void* ws, cudaStream_t s, cudaStream_t side_s) {
   const int n = (int)n64;
   CholWs w = carve(ws, n64);
   cudaError_t e;
@@ -292,84 +349,139 @@ cudaError_t launch_cholesky_inverse(const float* H, int64_t n64, float percdamp,
                                 (int)kApplySmemBytes)) != cudaSuccess)
     return e;
   const int apply_ctas = (n + kApplyVecs - 1) / kApplyVecs;  // n vectors per panel
+  const int SPW = (int)super_panel_cols(n);  // super-panel columns (kPanel: one level)
+  const int npan = SPW / kPanel;             // panels per super-panel
   // operands of the trailing updates; with a row stride that is a multiple
   // of 16 bytes the updates land in A and RT by TMA reduce-add
   CUtensorMap mPh[2], mPl[2], mA, mRT;
   const bool reduce = (n % 4) == 0;
   if (nblk > 1) {
     for (int b = 0; b < 2; ++b)
-      if (!make_tma_2d(&mPh[b], w.PBh[b], false, n, kPanel, kPanel, 32, 128) ||
-          !make_tma_2d(&mPl[b], w.PBl[b], false, n, kPanel, kPanel, 32, 128))
+      if (!make_tma_2d(&mPh[b], w.PBh[b], false, n, SPW, SPW, 32, 128) ||
+          !make_tma_2d(&mPl[b], w.PBl[b], false, n, SPW, SPW, 32, 128))
         return cudaErrorInvalidValue;
     if (reduce) {
       if (!make_tma_2d(&mA, w.A, false, n, n, n, 32, 32) ||
           !make_tma_2d(&mRT, U, false, n, n, n, 32, 32))
         return cudaErrorInvalidValue;
-      if ((e = cudaFuncSetAttribute(panel_gemm2_kernel<CholTrailItems, true>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)pg2_smem_bytes(true))) != cudaSuccess)
-        return e;
     } else {
       mA = mRT = mPh[0];  // not read by the read-modify-write epilogue
-      if ((e = cudaFuncSetAttribute(panel_gemm2_kernel<CholTrailItems, false>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)pg2_smem_bytes(false))) != cudaSuccess)
-        return e;
     }
+    if ((e = cudaFuncSetAttribute(reduce ? (const void*)panel_gemm2_kernel<CholTrailItems, true>
+                                         : (const void*)panel_gemm2_kernel<CholTrailItems, false>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)pg2_smem_bytes(reduce))) != cudaSuccess)
+      return e;
+    if (npan > 1 &&
+        (e = cudaFuncSetAttribute(reduce ? (const void*)stream_gemm_kernel<CholSuperItems, true>
+                                         : (const void*)stream_gemm_kernel<CholSuperItems, false>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)sg_smem_bytes(reduce))) != cudaSuccess)
+      return e;
   }
-  // Look-ahead: the trailing update of panel p is split into the next
-  // panel's column block (near, on the caller's stream, so panel p + 1 can be
-  // factored at once) and the rest (far, on a side stream, overlapping the
-  // factorisation of panel p + 1).  Every element still receives the panels'
-  // updates in panel order: near(p) waits for far(p - 1), far(p) follows
-  // far(p - 1) on the side stream, and panel p + 1's vectors go to the other
-  // half of the double-buffered PB while far(p) reads its own.
-  SideStream side{};
-  const bool ahead = nblk > 2 && side_stream(&side);
-  std::unique_lock<std::mutex> side_guard;
-  if (ahead) side_guard = std::unique_lock<std::mutex>(side_lock());
-  auto trail = [&](int p, int cb_lo, int cb_hi, cudaStream_t st) -> cudaError_t {
-    const CholTrailItems dec{w.A, U, n, p, nblk, cb_lo, cb_hi};
+  const WaitGate wg = current_wait_gate();
+  // rank-128 update by panel p (buffer b, column pk) of column blocks [cb_lo, cb_hi)
+  auto trail = [&](int b, int p, int pk, int cb_lo, int cb_hi, cudaStream_t st) -> cudaError_t {
+    const CholTrailItems dec{w.A, U, n, p, nblk, cb_lo, cb_hi, pk};
     int chunk = 1, units = 0;
     pg2_plan(dec, sms, chunk, units);
     if (units == 0) return cudaSuccess;
     const int grid = std::min(units, sms);
-    const int b = p & 1;
     if (reduce)
       panel_gemm2_kernel<CholTrailItems, true><<<grid, kPg2Threads, pg2_smem_bytes(true), st>>>(
-          mPh[b], mPl[b], mPh[b], mPl[b], mA, mRT, dec, chunk, units, info, kInfoTimeout, info);
+          mPh[b], mPl[b], mPh[b], mPl[b], mA, mRT, dec, chunk, units, info, kInfoTimeout, info,
+          wg.gate, wg.limit_ns);
     else
       panel_gemm2_kernel<CholTrailItems, false><<<grid, kPg2Threads, pg2_smem_bytes(false), st>>>(
-          mPh[b], mPl[b], mPh[b], mPl[b], mA, mRT, dec, chunk, units, info, kInfoTimeout, info);
+          mPh[b], mPl[b], mPh[b], mPl[b], mA, mRT, dec, chunk, units, info, kInfoTimeout, info,
+          wg.gate, wg.limit_ns);
     note_launch();
     return cudaGetLastError();
   };
-  for (int p = 0; p < nblk; ++p) {
-    const int b = p & 1;
-    chol_diag_kernel<<<1, kDiagThreads, kDiagSmemBytes, s>>>(w.A, n, p, w.Dout, info);
+  // the update past the super-panel [P0, P1) of column blocks [cb_lo, cb_hi)
+  auto past = [&](int b, int P0, int P1, int cb_lo, int cb_hi, cudaStream_t st) -> cudaError_t {
+    if (npan == 1) return trail(b, P0, 0, cb_lo, cb_hi, st);
+    const CholSuperItems dec{w.A, U, n, P0, P1, nblk, cb_lo, cb_hi};
+    const int units = sg_units(dec);
+    if (units == 0) return cudaSuccess;
+    const int grid = std::min(units, sms);
+    if (reduce)
+      stream_gemm_kernel<CholSuperItems, true><<<grid, kPg2Threads, sg_smem_bytes(true), st>>>(
+          mPh[b], mPl[b], mPh[b], mPl[b], mA, mRT, dec, units, info, kInfoTimeout, info, wg.gate,
+          wg.limit_ns);
+    else
+      stream_gemm_kernel<CholSuperItems, false><<<grid, kPg2Threads, sg_smem_bytes(false), st>>>(
+          mPh[b], mPl[b], mPh[b], mPl[b], mA, mRT, dec, units, info, kInfoTimeout, info, wg.gate,
+          wg.limit_ns);
     note_launch();
-    panel_apply_kernel<<<apply_ctas, kApplyThreads, kApplySmemBytes, s>>>(
-        w.A, U, n, p, w.Dout, w.PBh[b], w.PBl[b], info);
-    note_launch();
-    if (p + 1 >= nblk) break;
-    if (!ahead) {
-      if ((e = trail(p, 0, nblk, s)) != cudaSuccess) return e;
-      continue;
+    return cudaGetLastError();
+  };
+  // Look-ahead (when the caller gives a side stream): the trailing update of
+  // panel p is split into the next panel's column block (near, on the
+  // caller's stream, so panel p + 1 can be factored at once) and the rest
+  // (far, on the side stream, overlapping the factorisation of panel p + 1).
+  // Inside a super-panel the updates stop at its end; after its last panel
+  // the update past it is split the same way.  Every element still receives
+  // its updates in a fixed order: each near update waits for the far update
+  // issued before it.  Super-panels alternate between the two halves of the
+  // panel-vector buffer; the next writer of a half (the first panel two
+  // super-panels on) runs after the caller's stream has waited for the last
+  // far update that reads it.  Without a side stream everything runs on s.
+  SideEvents side;
+  const bool ahead = nblk > 2 && side_s != nullptr && side_s != s;
+  if (ahead && !side.create()) return cudaErrorMemoryAllocation;
+  bool far_pending = false, past_pending = false;
+  for (int P0 = 0, sp = 0; P0 < nblk; P0 += npan, ++sp) {
+    const int P1 = std::min(P0 + npan, nblk);
+    const int b = sp & 1;
+    for (int p = P0; p < P1; ++p) {
+      const int pk = (p - P0) * kPanel;
+      chol_diag_kernel<<<1, kDiagThreads, kDiagSmemBytes, s>>>(w.A, n, p, w.Dout, info);
+      note_launch();
+      panel_apply_kernel<<<apply_ctas, kApplyThreads, kApplySmemBytes, s>>>(
+          w.A, U, n, p, w.Dout, w.PBh[b] + pk, w.PBl[b] + pk, SPW, info);
+      note_launch();
+      if (p + 1 >= nblk) break;
+      const bool inside = p + 1 < P1;      // more panels of this super-panel follow
+      const int end = inside ? P1 : nblk;  // column blocks this panel's update reaches
+      if (!ahead) {
+        if ((e = inside ? trail(b, p, pk, p + 1, end, s) : past(b, P0, P1, p + 1, end, s)) !=
+            cudaSuccess)
+          return e;
+        continue;
+      }
+      if (p + 2 < end) {
+        // side: far(p) after apply(p) (and after the earlier far updates, in stream order)
+        if ((e = cudaEventRecord(side.ev[0], s)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(side_s, side.ev[0], 0)) != cudaSuccess)
+          return e;
+      }
+      // caller's stream: near(p) after the far update issued before it has landed
+      if (far_pending) {
+        if ((e = cudaStreamWaitEvent(s, side.ev[1], 0)) != cudaSuccess) return e;
+        far_pending = false;
+      }
+      if (past_pending) {
+        if ((e = cudaStreamWaitEvent(s, side.ev[2], 0)) != cudaSuccess) return e;
+        past_pending = false;
+      }
+      if ((e = inside ? trail(b, p, pk, p + 1, p + 2, s) : past(b, P0, P1, p + 1, p + 2, s)) !=
+          cudaSuccess)
+        return e;
+      if (p + 2 < end) {
+        if ((e = inside ? trail(b, p, pk, p + 2, end, side_s)
+                        : past(b, P0, P1, p + 2, end, side_s)) != cudaSuccess)
+          return e;
+        if ((e = cudaEventRecord(side.ev[inside ? 1 : 2], side_s)) != cudaSuccess) return e;
+        (inside ? far_pending : past_pending) = true;
+      }
     }
-    // side: far(p) after apply(p) (and after far(p - 1), in stream order)
-    if ((e = cudaEventRecord(side.ev[0], s)) != cudaSuccess ||
-        (e = cudaStreamWaitEvent(side.s, side.ev[0], 0)) != cudaSuccess)
-      return e;
-    // caller's stream: near(p) after far(p - 1) has landed
-    if (p >= 1 && (e = cudaStreamWaitEvent(s, side.ev[2 + ((p - 1) & 1)], 0)) != cudaSuccess)
-      return e;
-    if ((e = trail(p, p + 1, p + 2, s)) != cudaSuccess) return e;
-    if ((e = trail(p, p + 2, nblk, side.s)) != cudaSuccess) return e;
-    if ((e = cudaEventRecord(side.ev[2 + b], side.s)) != cudaSuccess) return e;
   }
-  if (ahead && nblk >= 2) {
-    // join: the last far update (panel nblk - 2) before the caller's stream goes on
-    if ((e = cudaStreamWaitEvent(s, side.ev[2 + ((nblk - 2) & 1)], 0)) != cudaSuccess) return e;
+  if (ahead) {
+    // join: every far update before the caller's stream goes on
+    if ((e = cudaEventRecord(side.ev[1], side_s)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(s, side.ev[1], 0)) != cudaSuccess)
+      return e;
   }
   if (n % 32 == 0) {
     const int nt = n / 32;
@@ -445,6 +557,7 @@ extern "C" gptq_status gptq_cholesky_inverse_noalloc(const float* H, int64_t n, 
     ws = g_scratch_addr[dev];
   }
   const cudaError_t e = gptq::launch_cholesky_inverse(H, n, percdamp, actorder, U, perm, dead,
-                                                      info, ws, static_cast<cudaStream_t>(stream));
+                                                      info, ws, static_cast<cudaStream_t>(stream),
+                                                      nullptr);
   return e == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
 }

@@ -3,7 +3,6 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
-#include <mutex>
 #include <cstdint>
 
 #include "gptq_internal.cuh"
@@ -54,53 +53,29 @@ bool make_tma_2d(CUtensorMap* map, const void* base, bool bf16, int64_t rows, in
 
 static std::atomic<long long> g_launches{0};
 
-namespace {
-constexpr int kMaxDevices = 64;
-std::mutex g_side_mu;
-SideStream g_side[kMaxDevices];
-bool g_side_ok[kMaxDevices] = {};
-std::mutex g_pool_mu;
-cudaMemPool_t g_pool[kMaxDevices] = {};
-}  // namespace
-
-bool scratch_pool(cudaMemPool_t* out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
-  std::lock_guard<std::mutex> lock(g_pool_mu);
-  if (!g_pool[dev]) {
-    cudaMemPoolProps props{};
-    props.allocType = cudaMemAllocationTypePinned;
-    props.location.type = cudaMemLocationTypeDevice;
-    props.location.id = dev;
-    cudaMemPool_t p = nullptr;
-    if (cudaMemPoolCreate(&p, &props) != cudaSuccess) return false;
-    uint64_t keep = ~0ull;
-    if (cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
-      cudaMemPoolDestroy(p);
+bool SideEvents::create() {
+  for (auto& e : ev)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      e = nullptr;
       return false;
     }
-    g_pool[dev] = p;
-  }
-  *out = g_pool[dev];
   return true;
 }
 
-std::mutex& side_lock() { return g_side_mu; }
+SideEvents::~SideEvents() {
+  for (auto& e : ev)
+    if (e) cudaEventDestroy(e);
+}
 
-bool side_stream(SideStream* out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
-  std::lock_guard<std::mutex> lock(g_side_mu);
-  if (!g_side_ok[dev]) {
-    SideStream ss{};
-    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess) return false;
-    for (auto& e : ss.ev)
-      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return false;
-    g_side[dev] = ss;
-    g_side_ok[dev] = true;
-  }
-  *out = g_side[dev];
-  return true;
+namespace {
+thread_local WaitGate t_gate = {nullptr, (uint64_t)kGridWaitLimitNs};
+}  // namespace
+
+WaitGate current_wait_gate() { return t_gate; }
+
+void set_wait_gate(const int32_t* gate, uint64_t limit_ns) {
+  t_gate.gate = gate;
+  t_gate.limit_ns = gate ? limit_ns : (uint64_t)kGridWaitLimitNs;
 }
 
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
@@ -118,10 +93,16 @@ gptq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GPTQ_OK : GPT
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-size_t hessian_ws(int64_t n, int64_t ntok, gptq_dtype xt) {
-  if (xt != GPTQ_F32) return 0;
+// [split-K turnstile flags | fp32 input only: bf16 hi part | bf16 lo part]
+size_t hessian_flags_bytes(int64_t n) { return align_up(gptq::syrk_flag_bytes(n), 256); }
+
+size_t hessian_split_bytes(int64_t n, int64_t ntok) {
   const int64_t ld = (ntok + 7) / 8 * 8;
-  return 2 * align_up(sizeof(uint16_t) * (size_t)n * ld, 256);
+  return align_up(sizeof(uint16_t) * (size_t)n * ld, 256);
+}
+
+size_t hessian_ws(int64_t n, int64_t ntok, gptq_dtype xt) {
+  return hessian_flags_bytes(n) + (xt == GPTQ_F32 ? 2 * hessian_split_bytes(n, ntok) : 0);
 }
 
 gptq_status check_cfg(const gptq_config* cfg) {
@@ -140,6 +121,12 @@ gptq_status check_cfg(const gptq_config* cfg) {
 extern "C" {
 
 int64_t gptq_launch_count(void) { return gptq::g_launches.load(std::memory_order_relaxed); }
+
+gptq_status gptq_set_wait_gate(const int32_t* gate, int64_t limit_ns) {
+  if (gate && (limit_ns <= 0 || limit_ns > gptq::kGridWaitLimitNs)) return GPTQ_ERR_INVALID_ARG;
+  gptq::set_wait_gate(gate, (uint64_t)limit_ns);
+  return GPTQ_OK;
+}
 
 gptq_status gptq_selftest_division(const float* a, const float* b, int64_t count, float* out,
                                    void* stream) {
@@ -180,6 +167,10 @@ gptq_status gptq_workspace_size(int op, int64_t rows, int64_t n, int64_t ntok, g
       *bytes = gptq::quantize_workspace_bytes(rows, n);
       return GPTQ_OK;
     }
+    case GPTQ_OP_DEQUANT_MATVEC:
+      if (rows < 0) return GPTQ_ERR_INVALID_ARG;
+      *bytes = gptq::dequant_matvec_workspace_bytes(rows, n);
+      return GPTQ_OK;
     default:
       return GPTQ_ERR_INVALID_ARG;
   }
@@ -195,26 +186,31 @@ gptq_status gptq_hessian_accumulate(float* H, const void* X, gptq_dtype xt, int6
   if (!aligned(H, 16)) return GPTQ_ERR_INVALID_ARG;
   if (ntok == 0) return GPTQ_OK;
   if (!X) return GPTQ_ERR_INVALID_ARG;
+  const size_t need = hessian_ws(n, ntok, xt);
+  if (!ws || ws_bytes < need) return GPTQ_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return GPTQ_ERR_INVALID_ARG;
+  void* flags = ws;
   cudaError_t e;
   if (xt == GPTQ_BF16) {
     if (!aligned(X, 16) || (ldx * 2) % 16 != 0) return GPTQ_ERR_INVALID_ARG;
-    if ((e = gptq::launch_syrk_bf16(H, n, X, X, ntok, ldx, alpha, info, s)) != cudaSuccess)
+    if ((e = gptq::launch_syrk_bf16(H, n, X, X, ntok, ldx, alpha, info, flags, s)) !=
+        cudaSuccess)
       return cuda_status(e);
   } else {
     if (!aligned(X, 4)) return GPTQ_ERR_INVALID_ARG;
-    const size_t need = hessian_ws(n, ntok, xt);
-    if (!ws || ws_bytes < need) return GPTQ_ERR_WORKSPACE;
-    if (!aligned(ws, 256)) return GPTQ_ERR_INVALID_ARG;
     const int64_t ld = (ntok + 7) / 8 * 8;
-    char* hi = static_cast<char*>(ws);
-    char* lo = hi + need / 2;
+    char* hi = static_cast<char*>(ws) + hessian_flags_bytes(n);
+    char* lo = hi + hessian_split_bytes(n, ntok);
     if ((e = gptq::launch_split_bf16(static_cast<const float*>(X), n, ntok, ldx, hi, lo, ld, s)) !=
         cudaSuccess)
       return cuda_status(e);
     // hi hi^T + hi lo^T + lo hi^T  (lo lo^T is below fp32 resolution of the sum)
-    if ((e = gptq::launch_syrk_bf16(H, n, hi, hi, ntok, ld, alpha, info, s)) != cudaSuccess ||
-        (e = gptq::launch_syrk_bf16(H, n, hi, lo, ntok, ld, alpha, info, s)) != cudaSuccess ||
-        (e = gptq::launch_syrk_bf16(H, n, lo, hi, ntok, ld, alpha, info, s)) != cudaSuccess)
+    if ((e = gptq::launch_syrk_bf16(H, n, hi, hi, ntok, ld, alpha, info, flags, s)) !=
+            cudaSuccess ||
+        (e = gptq::launch_syrk_bf16(H, n, hi, lo, ntok, ld, alpha, info, flags, s)) !=
+            cudaSuccess ||
+        (e = gptq::launch_syrk_bf16(H, n, lo, hi, ntok, ld, alpha, info, flags, s)) !=
+            cudaSuccess)
       return cuda_status(e);
   }
   return cuda_status(gptq::launch_mirror_upper(H, n, s));
@@ -222,7 +218,7 @@ gptq_status gptq_hessian_accumulate(float* H, const void* X, gptq_dtype xt, int6
 
 gptq_status gptq_cholesky_inverse(const float* H, int64_t n, float percdamp, int actorder,
                                   float* U, int32_t* perm, uint8_t* dead, int32_t* info,
-                                  void* ws, size_t ws_bytes, void* stream) {
+                                  void* ws, size_t ws_bytes, void* stream, void* side_stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!H || !U || !dead || !info || n <= 0 || n > kMaxN) return GPTQ_ERR_INVALID_ARG;
   if (actorder && !perm) return GPTQ_ERR_INVALID_ARG;
@@ -230,14 +226,15 @@ gptq_status gptq_cholesky_inverse(const float* H, int64_t n, float percdamp, int
   if (!ws || ws_bytes < gptq::cholesky_workspace_bytes(n)) return GPTQ_ERR_WORKSPACE;
   if (!aligned(ws, 256) || !aligned(H, 4) || !aligned(U, 16)) return GPTQ_ERR_INVALID_ARG;
   return cuda_status(gptq::launch_cholesky_inverse(H, n, percdamp, actorder, U, perm, dead, info,
-                                                   ws, s));
+                                                   ws, s, static_cast<cudaStream_t>(side_stream)));
 }
 
 gptq_status gptq_quantize_layer(const void* W, gptq_dtype wt, int64_t rows, int64_t n,
                                 const float* U, const int32_t* perm, const uint8_t* dead,
                                 const gptq_config* cfg, uint8_t* codes, float* scales,
                                 uint8_t* zeros, int32_t* g_idx, float* Wq, float* row_loss,
-                                void* ws, size_t ws_bytes, void* stream) {
+                                void* ws, size_t ws_bytes, int32_t* info, void* stream,
+                                void* side_stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const gptq_status st = check_cfg(cfg);
   if (st != GPTQ_OK) return st;
@@ -249,7 +246,8 @@ gptq_status gptq_quantize_layer(const void* W, gptq_dtype wt, int64_t rows, int6
   if (!aligned(ws, 256)) return GPTQ_ERR_INVALID_ARG;
   return cuda_status(gptq::launch_quantize_layer(W, wt, rows, n, U, perm, dead, cfg->bits,
                                                  cfg->group_size, cfg->sym, codes, scales, zeros,
-                                                 g_idx, Wq, row_loss, ws, s));
+                                                 g_idx, Wq, row_loss, ws, info, s,
+                                                 static_cast<cudaStream_t>(side_stream)));
 }
 
 gptq_status gptq_pack_int4(const uint8_t* codes, int64_t rows, int64_t n, uint32_t* out,
@@ -291,7 +289,7 @@ gptq_status gptq_dequant_matvec(const uint32_t* packed, int bits, int64_t rows, 
                                 const float* scales, const uint8_t* zeros, int group_size,
                                 int64_t n_groups, const int32_t* g_idx, const int32_t* perm,
                                 const void* x, gptq_dtype xt, int64_t batch, float* y,
-                                void* stream) {
+                                void* ws, size_t ws_bytes, void* stream) {
   if (bits != 3 && bits != 4) return GPTQ_ERR_UNSUPPORTED;
   if (rows < 0 || n <= 0 || batch < 0) return GPTQ_ERR_INVALID_ARG;
   if ((bits == 4 && n % 8) || (bits == 3 && n % 32)) return GPTQ_ERR_INVALID_ARG;
@@ -304,9 +302,12 @@ gptq_status gptq_dequant_matvec(const uint32_t* packed, int bits, int64_t rows, 
   if (!packed || !scales || !zeros || !x || !y || !aligned(packed, 4) || !aligned(scales, 4) ||
       !aligned(y, 4) || !aligned(x, xt == GPTQ_BF16 ? 2 : 4))
     return GPTQ_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < gptq::dequant_matvec_workspace_bytes(batch, n))
+    return GPTQ_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return GPTQ_ERR_INVALID_ARG;
   return cuda_status(gptq::launch_dequant_matvec(packed, bits, rows, n, scales, zeros,
                                                  group_size, G, g_idx, perm, x,
-                                                 xt == GPTQ_BF16 ? 1 : 0, batch, y,
+                                                 xt == GPTQ_BF16 ? 1 : 0, batch, y, ws,
                                                  static_cast<cudaStream_t>(stream)));
 }
 

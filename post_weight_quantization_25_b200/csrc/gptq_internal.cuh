@@ -23,29 +23,36 @@ bool make_tma_2d(CUtensorMap* map, const void* base, bool bf16, int64_t rows, in
 // Counts one kernel enqueued by this library (read by gptq_launch_count).
 void note_launch();
 
-// A second stream on the current device for work that overlaps the
-// caller's stream, and two events to order the two; created on first use
-// per device and kept until the process exits.  A launcher that forks onto
-// it holds side_lock() for its whole enqueue sequence and joins back onto
-// the caller's stream before returning.  Returns false if it cannot be had.
-struct SideStream {
-  cudaStream_t s;
-  cudaEvent_t ev[4];
+// Events that order a caller-given side stream against the caller's stream
+// for the duration of one call's enqueue: created by create(), destroyed by
+// the destructor (CUDA frees an event whose recorded work is still pending
+// once that work completes, so destroying right after the enqueue is safe).
+// The library keeps no stream or event between calls.
+struct SideEvents {
+  cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
+  bool create();
+  ~SideEvents();
 };
-bool side_stream(SideStream* out);
-std::mutex& side_lock();
 
-// A stream-ordered memory pool of the current device, private to this
-// library, that keeps freed blocks for reuse (no release threshold), so
-// per-call scratch costs no mapping work after the first call.  Created on
-// first use per device.  Returns false if it cannot be had.
-bool scratch_pool(cudaMemPool_t* out);
+// Test hook for the bounded waits (see gptq_set_wait_gate in gptq.h): the
+// producer of every tensor-core kernel enqueued afterwards by the calling
+// host thread first waits for *gate != 0, giving up after limit_ns.  With no
+// gate set (the default) gate is null and limit_ns = kGridWaitLimitNs.
+struct WaitGate {
+  const int32_t* gate;
+  uint64_t limit_ns;
+};
+WaitGate current_wait_gate();
 
 // ---- Hessian (hessian_syrk.cu)
 // H(upper incl. diagonal) += alpha * A_rows * B_rows^T over tokens [0, ntok),
-// A and B are n x ntok bf16 with row stride ld (elements).
+// A and B are n x ntok bf16 with row stride ld (elements).  `flags`: device
+// scratch of syrk_flag_bytes(n) bytes (256-byte aligned) for the ordered
+// split-K reduction; zeroed by the launcher.
 cudaError_t launch_syrk_bf16(float* H, int64_t n, const void* A, const void* B, int64_t ntok,
-                             int64_t ld, float alpha, int32_t* info, cudaStream_t s);
+                             int64_t ld, float alpha, int32_t* info, void* flags,
+                             cudaStream_t s);
+size_t syrk_flag_bytes(int64_t n);
 // fp32 X -> bf16 hi / lo parts (n x ntok, row stride ldo).
 cudaError_t launch_split_bf16(const float* X, int64_t n, int64_t ntok, int64_t ldx, void* hi,
                               void* lo, int64_t ldo, cudaStream_t s);
@@ -53,9 +60,10 @@ cudaError_t launch_split_bf16(const float* X, int64_t n, int64_t ntok, int64_t l
 cudaError_t launch_mirror_upper(float* H, int64_t n, cudaStream_t s);
 
 // ---- Cholesky / inverse (cholesky.cu)
+// side: a second stream for the look-ahead, or null (everything on s).
 cudaError_t launch_cholesky_inverse(const float* H, int64_t n, float percdamp, int actorder,
                                     float* U, int32_t* perm, uint8_t* dead, int32_t* info,
-                                    void* ws, cudaStream_t s);
+                                    void* ws, cudaStream_t s, cudaStream_t side);
 size_t cholesky_workspace_bytes(int64_t n);
 
 // ---- sweep (sweep.cu)
@@ -63,7 +71,7 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows, int64_t n
                                   const int32_t* perm, const uint8_t* dead, int bits,
                                   int group_size, int sym, uint8_t* codes, float* scales,
                                   uint8_t* zeros, int32_t* g_idx, float* Wq, float* row_loss,
-                                  void* ws, cudaStream_t s);
+                                  void* ws, int32_t* info, cudaStream_t s, cudaStream_t side);
 size_t quantize_workspace_bytes(int64_t rows, int64_t n);
 // out[i] = a[i] / b[i] by the sweep's division routine (fdiv.cuh)
 cudaError_t launch_selftest_division(const float* a, const float* b, int64_t count, float* out,
@@ -80,7 +88,9 @@ cudaError_t launch_dequant_matvec(const uint32_t* packed, int bits, int64_t rows
                                   const float* scales, const uint8_t* zeros, int group_size,
                                   int64_t n_groups, const int32_t* g_idx, const int32_t* perm,
                                   const void* x, int x_bf16, int64_t batch, float* y,
-                                  cudaStream_t s);
+                                  void* ws, cudaStream_t s);
+// scratch of launch_dequant_matvec: x re-laid out as batch x n bf16
+size_t dequant_matvec_workspace_bytes(int64_t batch, int64_t n);
 // dst[r][k] = src[r][perm[k]] (rows x n bytes)
 cudaError_t launch_gather_columns_u8(const uint8_t* src, int64_t rows, int64_t n,
                                      const int32_t* perm, uint8_t* dst, cudaStream_t s);

@@ -25,8 +25,16 @@
 //    a unit's token range is cut into pieces of kSubKb k-blocks (1024
 //    tokens, 64 MMAs); each piece starts a fresh TMEM sum, and the epilogue
 //    adds the pieces into an fp32 register copy of the tile with ordinary
-//    IEEE adds.  At the end of the unit it adds alpha * tile into H with
-//    vector atomics (the split-K reduction), masked to the upper triangle.
+//    IEEE adds.  At the end of the unit it adds alpha * tile into H, masked
+//    to the upper triangle (the split-K reduction).
+//  * Ordered split-K reduction: the token chunks of a tile are added into H
+//    in chunk order, not by atomics.  A per-tile counter in global memory
+//    (a turnstile) holds how many chunks have been added; the unit of chunk
+//    c waits (acquire) until it reads c, adds its tile with plain loads and
+//    stores through L2, and publishes c + 1 (release).  So H is the same bit
+//    for bit from run to run.  Units are walked in chunk-major order by a
+//    persistent grid whose CTAs are all resident, so chunk c - 1 of a tile is
+//    always taken before chunk c and the wait ends.
 //  * No multicast loads.  Every wait is bounded: on timeout the CTA stops,
 //    writes GPTQ_ERR_TIMEOUT to `info`, waits for its own copies and MMAs,
 //    frees TMEM and exits.
@@ -36,6 +44,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <mutex>
 
 #include "gptq_internal.cuh"
 #include "sm100_ptx.cuh"
@@ -64,6 +73,9 @@ struct SyrkArgs {
   int units;        // ntiles * token chunks
   int vec4;         // H row starts are 16-byte aligned
   int32_t* info;
+  uint32_t* flags;  // [ntiles] chunks of each tile added so far
+  const int32_t* gate;  // test gate of the bounded waits (null: none)
+  uint64_t limit_ns;    // limit of every pipeline wait
 };
 
 // Tile t of the J-major enumeration: column block J holds row blocks 0..min(nI, 2J+2)-1.
@@ -83,6 +95,59 @@ __device__ __forceinline__ void decode_tile(int t, int nI, int& I, int& J) {
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int32_t* info) {
   *abort_flag = 1;
   if (info) atomicExch(info, (int32_t)GPTQ_ERR_TIMEOUT);
+}
+
+constexpr int kEpiBar = 1;                 // named barrier of the 8 epilogue warps
+constexpr int kEpiThreads = NUM_THREADS - 64;
+
+// The ordered add of one unit's tile (this thread's row, 128 columns from
+// cbase) into H: wait for the turnstile to show `chunk`, add, publish
+// chunk + 1.  Called by all epilogue threads together; returns false (for
+// all of them) if the wait gave up.
+__device__ __forceinline__ bool ordered_add(float* H, int n, int row, int cbase, float alpha,
+                                            int vec4, const float (&tile)[128], uint32_t* flag,
+                                            uint32_t chunk, volatile int* abort_flag,
+                                            int32_t* info, uint64_t limit_ns, bool waiter) {
+  bool ok = true;
+  if (waiter) {
+    ok = ptx::flag_wait_bounded(flag, chunk, abort_flag, limit_ns);
+    if (!ok) raise_abort(abort_flag, info);
+  }
+  ok = ptx::named_bar_and(kEpiBar, kEpiThreads, ok);
+  if (!ok) return false;
+  if (row < n) {
+    float* hrow = H + (int64_t)row * n;
+#pragma unroll
+    for (int j4 = 0; j4 < 32; ++j4) {
+      const int c = cbase + 4 * j4;
+      if (c + 3 < row || c >= n) continue;
+      const float f0 = alpha * tile[4 * j4 + 0];
+      const float f1 = alpha * tile[4 * j4 + 1];
+      const float f2 = alpha * tile[4 * j4 + 2];
+      const float f3 = alpha * tile[4 * j4 + 3];
+      if (vec4 && c >= row && c + 3 < n) {
+        float4* p = reinterpret_cast<float4*>(hrow + c);
+        float4 h = __ldcg(p);
+        h.x += f0;
+        h.y += f1;
+        h.z += f2;
+        h.w += f3;
+        __stcg(p, h);
+      } else {
+        const float fv[4] = {f0, f1, f2, f3};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (c + i >= row && c + i < n) __stcg(hrow + c + i, __ldcg(hrow + c + i) + fv[i]);
+      }
+    }
+  }
+  // every thread's stores are done before the next chunk may start
+  ptx::named_bar_sync(kEpiBar, kEpiThreads);
+  if (waiter) {
+    __threadfence();
+    ptx::st_release_gpu(flag, chunk + 1);
+  }
+  return true;
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -134,14 +199,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       int last_parity[STAGES];
       for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
-      bool ok = true;
+      bool ok = ptx::gate_wait_bounded(args.gate, args.limit_ns);
       for (int u = blockIdx.x; u < args.units && ok; u += gridDim.x) {
         int I, J;
         decode_tile(u % args.ntiles, args.nI, I, J);
         const int kb0 = (u / args.ntiles) * args.kb_per_unit;
         const int kb1 = min(kb0 + args.kb_per_unit, args.nkb);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, WAIT_LIMIT_NS)) {
+          if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, args.limit_ns)) {
             ok = false;
             break;
           }
@@ -178,14 +243,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int kb1 = min(kb0 + args.kb_per_unit, args.nkb);
         for (int p0 = kb0; p0 < kb1 && ok; p0 += kSubKb) {
           const int p1 = min(p0 + kSubKb, kb1);
-          if (!ptx::mbar_wait_bounded(&tempty[acc], aphase ^ 1, abort_flag, WAIT_LIMIT_NS)) {
+          if (!ptx::mbar_wait_bounded(&tempty[acc], aphase ^ 1, abort_flag, args.limit_ns)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
           const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
           for (int kb = p0; kb < p1; ++kb) {
-            if (!ptx::mbar_wait_bounded(&full[stage], phase, abort_flag, WAIT_LIMIT_NS)) {
+            if (!ptx::mbar_wait_bounded(&full[stage], phase, abort_flag, args.limit_ns)) {
               ok = false;
               break;
             }
@@ -218,14 +283,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // -------------------------------------------------- epilogue (warps 2..9)
     // warp w reads TMEM lanes [32 (w % 4), +32) (rows of the tile) and
-    // columns [128 half, +128) of the accumulator
+    // columns [128 half, +128) of the accumulator.  Every decision to stop is
+    // taken by all 256 epilogue threads together (named barrier with AND).
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     int acc = 0;
     uint32_t aphase = 0;
     const int n = args.n;
-    bool stop = false;
-    for (int u = blockIdx.x; u < args.units && !stop; u += gridDim.x) {
+    for (int u = blockIdx.x; u < args.units; u += gridDim.x) {
       int I, J;
       decode_tile(u % args.ntiles, args.nI, I, J);
       const int kb0 = (u / args.ntiles) * args.kb_per_unit;
@@ -236,10 +301,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       float tile[128];
 #pragma unroll
       for (int j = 0; j < 128; ++j) tile[j] = 0.f;
+      bool ok = true;
       for (int p0 = kb0; p0 < kb1; p0 += kSubKb) {
-        if (!ptx::mbar_wait_bounded(&tfull[acc], aphase, abort_flag, WAIT_LIMIT_NS)) {
-          raise_abort(abort_flag, args.info);
-          stop = true;
+        bool ready = ptx::mbar_wait_bounded(&tfull[acc], aphase, abort_flag, args.limit_ns);
+        if (!ready) raise_abort(abort_flag, args.info);
+        if (!ptx::named_bar_and(kEpiBar, kEpiThreads, ready)) {
+          ok = false;
           break;
         }
         ptx::tc_fence_after();
@@ -262,27 +329,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         acc ^= 1;
         if (acc == 0) aphase ^= 1;
       }
-      if (stop) break;
-      if (row < n) {
-        float* hrow = args.H + (int64_t)row * n;
-#pragma unroll
-        for (int j4 = 0; j4 < 32; ++j4) {
-          const int c = cbase + 4 * j4;
-          if (c + 3 < row || c >= n) continue;
-          const float f0 = args.alpha * tile[4 * j4 + 0];
-          const float f1 = args.alpha * tile[4 * j4 + 1];
-          const float f2 = args.alpha * tile[4 * j4 + 2];
-          const float f3 = args.alpha * tile[4 * j4 + 3];
-          if (args.vec4 && c >= row && c + 3 < n) {
-            atomicAdd(reinterpret_cast<float4*>(hrow + c), make_float4(f0, f1, f2, f3));
-          } else {
-            if (c + 0 >= row && c + 0 < n) atomicAdd(hrow + c + 0, f0);
-            if (c + 1 >= row && c + 1 < n) atomicAdd(hrow + c + 1, f1);
-            if (c + 2 >= row && c + 2 < n) atomicAdd(hrow + c + 2, f2);
-            if (c + 3 >= row && c + 3 < n) atomicAdd(hrow + c + 3, f3);
-          }
-        }
-      }
+      if (!ok) break;
+      const int t = u % args.ntiles;
+      if (!ordered_add(args.H, n, row, cbase, args.alpha, args.vec4, tile, args.flags + t,
+                       (uint32_t)(u / args.ntiles), abort_flag, args.info, args.limit_ns,
+                       warp == 2 && lane == 0))
+        break;
     }
   }
 
@@ -328,6 +380,9 @@ struct SyrkPairArgs {
   int units;        // ntiles * token chunks
   int vec4;
   int32_t* info;
+  uint32_t* flags;  // [2][ntiles] chunks of each tile half (CTA rank) added so far
+  const int32_t* gate;
+  uint64_t limit_ns;
 };
 
 // Tile t of the J-major enumeration: column block J holds row blocks 0..J.
@@ -387,18 +442,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       ptx::prefetch_tmap(&mapB);
       int stage = 0;
       uint32_t phase = 0;
-      bool ok = true;
+      int last_parity[P_STAGES];  // leader: last phase of full[s] it armed
+      for (int s = 0; s < P_STAGES; ++s) last_parity[s] = -1;
+      bool ok = ptx::gate_wait_bounded(args.gate, args.limit_ns);
       for (int u = pair; u < args.units && ok; u += npairs) {
         int I2, J;
         decode_tile_pair(u % args.ntiles, I2, J);
         const int kb0 = (u / args.ntiles) * args.kb_per_unit;
         const int kb1 = min(kb0 + args.kb_per_unit, args.nkb);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, WAIT_LIMIT_NS)) {
+          if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, args.limit_ns)) {
             ok = false;
             break;
           }
-          if (leader) ptx::mbar_arrive_expect_tx(&full[stage], 2 * P_STAGE_BYTES);
+          if (leader) {
+            ptx::mbar_arrive_expect_tx(&full[stage], 2 * P_STAGE_BYTES);
+            last_parity[stage] = (int)phase;
+          }
           const uint32_t fb = ptx::mapa_shared(&full[stage], 0);
           ptx::tma_load_2d_pair(sA + stage * P_A_BYTES, &mapA, fb, kb * BK,
                                 I2 * 256 + (int)rank * 128);
@@ -412,11 +472,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       }
       if (!ok || *abort_flag) {
         raise_abort(abort_flag, args.info);
+        // Loads still in flight must land before the pair tears down.  Both
+        // CTAs' loads of a stage complete on the leader's full[] barrier, so
+        // the leader waits (bounded) for the last phase it armed on each
+        // stage; the other CTA is held by the final cluster barrier until
+        // the leader gets there.
+        if (leader) {
+          volatile int never = 0;
+          for (int s = 0; s < P_STAGES; ++s)
+            if (last_parity[s] >= 0)
+              ptx::mbar_wait_bounded(&full[s], (uint32_t)last_parity[s], &never, WAIT_LIMIT_NS);
+        }
       } else {
         // tail: every stage is released once more, so the MMA commits'
         // arrivals on this CTA's `empty` barriers have all landed
         for (int i = 0; i < P_STAGES; ++i) {
-          if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
+          if (!ptx::mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, args.limit_ns)) break;
           if (++stage == P_STAGES) {
             stage = 0;
             phase ^= 1;
@@ -438,14 +509,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const int kb1 = min(kb0 + args.kb_per_unit, args.nkb);
         for (int p0 = kb0; p0 < kb1 && ok; p0 += kSubKb) {
           const int p1 = min(p0 + kSubKb, kb1);
-          if (!ptx::mbar_wait_bounded(&tempty[acc], aphase ^ 1, abort_flag, WAIT_LIMIT_NS)) {
+          if (!ptx::mbar_wait_bounded(&tempty[acc], aphase ^ 1, abort_flag, args.limit_ns)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
           const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
           for (int kb = p0; kb < p1; ++kb) {
-            if (!ptx::mbar_wait_bounded(&full[stage], phase, abort_flag, WAIT_LIMIT_NS)) {
+            if (!ptx::mbar_wait_bounded(&full[stage], phase, abort_flag, args.limit_ns)) {
               ok = false;
               break;
             }
@@ -483,8 +554,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     int acc = 0;
     uint32_t aphase = 0;
     const int n = args.n;
-    bool stop = false;
-    for (int u = pair; u < args.units && !stop; u += npairs) {
+    for (int u = pair; u < args.units; u += npairs) {
       int I2, J;
       decode_tile_pair(u % args.ntiles, I2, J);
       const int kb0 = (u / args.ntiles) * args.kb_per_unit;
@@ -495,10 +565,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       float tile[128];
 #pragma unroll
       for (int j = 0; j < 128; ++j) tile[j] = 0.f;
+      bool ok = true;
       for (int p0 = kb0; p0 < kb1; p0 += kSubKb) {
-        if (!ptx::mbar_wait_bounded(&tfull[acc], aphase, abort_flag, WAIT_LIMIT_NS)) {
-          raise_abort(abort_flag, args.info);
-          stop = true;
+        bool ready = ptx::mbar_wait_bounded(&tfull[acc], aphase, abort_flag, args.limit_ns);
+        if (!ready) raise_abort(abort_flag, args.info);
+        if (!ptx::named_bar_and(kEpiBar, kEpiThreads, ready)) {
+          ok = false;
           break;
         }
         ptx::tc_fence_after();
@@ -522,27 +594,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         acc ^= 1;
         if (acc == 0) aphase ^= 1;
       }
-      if (stop) break;
-      if (row < n) {
-        float* hrow = args.H + (int64_t)row * n;
-#pragma unroll
-        for (int j4 = 0; j4 < 32; ++j4) {
-          const int c = cbase + 4 * j4;
-          if (c + 3 < row || c >= n) continue;
-          const float f0 = args.alpha * tile[4 * j4 + 0];
-          const float f1 = args.alpha * tile[4 * j4 + 1];
-          const float f2 = args.alpha * tile[4 * j4 + 2];
-          const float f3 = args.alpha * tile[4 * j4 + 3];
-          if (args.vec4 && c >= row && c + 3 < n) {
-            atomicAdd(reinterpret_cast<float4*>(hrow + c), make_float4(f0, f1, f2, f3));
-          } else {
-            if (c + 0 >= row && c + 0 < n) atomicAdd(hrow + c + 0, f0);
-            if (c + 1 >= row && c + 1 < n) atomicAdd(hrow + c + 1, f1);
-            if (c + 2 >= row && c + 2 < n) atomicAdd(hrow + c + 2, f2);
-            if (c + 3 >= row && c + 3 < n) atomicAdd(hrow + c + 3, f3);
-          }
-        }
-      }
+      if (!ok) break;
+      const int t = u % args.ntiles;
+      if (!ordered_add(args.H, n, row, cbase, args.alpha, args.vec4, tile,
+                       args.flags + (int)rank * args.ntiles + t, (uint32_t)(u / args.ntiles),
+                       abort_flag, args.info, args.limit_ns, warp == 2 && lane == 0))
+        break;
     }
   }
 
@@ -612,10 +669,18 @@ int choose_chunks(int ntiles, int nkb, int slots) {
   return best_kc;
 }
 
-// Concurrent CTA pairs the pair kernel can have (0 if it cannot launch).
+// Concurrent CTA pairs the pair kernel can have on the current device (0 if
+// it cannot launch there).  A property of the device and the kernel, so it is
+// looked up once per device and kept (under a lock).
 int pair_slots() {
-  static int cached = -1;
-  if (cached >= 0) return cached;
+  constexpr int kMaxDev = 64;
+  static std::mutex mu;
+  static int cached[kMaxDev];
+  static bool have[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (have[dev]) return cached[dev];
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * 74, 1, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -634,19 +699,40 @@ int pair_slots() {
     cudaGetLastError();
     clusters = 0;
   }
-  cached = clusters;
-  return cached;
+  cached[dev] = clusters;
+  have[dev] = true;
+  return clusters;
+}
+
+int pair_tiles(int64_t n) {
+  const int nJ = (int)((n + 255) / 256);
+  return nJ * (nJ + 1) / 2;
+}
+
+int single_tiles(int64_t n) {
+  const int nI = (int)((n + BM - 1) / BM), nJ = (int)((n + BN - 1) / BN);
+  int t = 0;
+  for (int J = 0; J < nJ; ++J) t += std::min(nI, 2 * J + 2);
+  return t;
 }
 
 }  // namespace
 
+size_t syrk_flag_bytes(int64_t n) {
+  return sizeof(uint32_t) * (size_t)std::max(2 * pair_tiles(n), single_tiles(n));
+}
+
 cudaError_t launch_syrk_bf16(float* H, int64_t n, const void* A, const void* B, int64_t ntok,
-                             int64_t ld, float alpha, int32_t* info, cudaStream_t s) {
+                             int64_t ld, float alpha, int32_t* info, void* flags,
+                             cudaStream_t s) {
   if (n <= 0 || ntok <= 0) return cudaSuccess;
   const int sms = num_sms();
   const int nkb = (int)((ntok + BK - 1) / BK);
   const int vec4 = ((n % 4) == 0 && (reinterpret_cast<uintptr_t>(H) % 16) == 0) ? 1 : 0;
+  const WaitGate wg = current_wait_gate();
   cudaError_t e;
+  // the turnstile counts start at zero for every launch
+  if ((e = cudaMemsetAsync(flags, 0, syrk_flag_bytes(n), s)) != cudaSuccess) return e;
   // CTA pairs for layers of at least 256 inputs, when the device can co-schedule them
   const int slots = n >= 256 ? pair_slots() : 0;
   if (slots > 0) {
@@ -658,14 +744,22 @@ cudaError_t launch_syrk_bf16(float* H, int64_t n, const void* A, const void* B, 
     a.n = (int)n;
     a.alpha = alpha;
     a.nkb = nkb;
-    const int nJ = (int)((n + 255) / 256);
-    a.ntiles = nJ * (nJ + 1) / 2;
+    a.ntiles = pair_tiles(n);
     const int kc = choose_chunks(a.ntiles, nkb, slots);
     a.kb_per_unit = (nkb + kc - 1) / kc;
     a.units = a.ntiles * ((nkb + a.kb_per_unit - 1) / a.kb_per_unit);
     a.vec4 = vec4;
     a.info = info;
+    a.flags = static_cast<uint32_t*>(flags);
+    a.gate = wg.gate;
+    a.limit_ns = wg.limit_ns;
+    // every pair of the persistent grid must be resident at once (the
+    // turnstile waits on units of other pairs): no more pairs than slots
     const int pairs = std::min(slots, a.units);
+    if ((e = cudaFuncSetAttribute(syrk_bf16_pair_kernel,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)P_SMEM_BYTES)) != cudaSuccess)
+      return e;
     syrk_bf16_pair_kernel<<<2 * pairs, NUM_THREADS, P_SMEM_BYTES, s>>>(mapA, mapB, a);
     note_launch();
     return cudaGetLastError();
@@ -679,15 +773,16 @@ cudaError_t launch_syrk_bf16(float* H, int64_t n, const void* A, const void* B, 
   a.alpha = alpha;
   a.nkb = nkb;
   a.nI = (int)((n + BM - 1) / BM);
-  const int nJ = (int)((n + BN - 1) / BN);
-  a.ntiles = 0;
-  for (int J = 0; J < nJ; ++J) a.ntiles += std::min(a.nI, 2 * J + 2);
+  a.ntiles = single_tiles(n);
   const int best_kc = choose_chunks(a.ntiles, nkb, sms);
   a.kb_per_unit = (a.nkb + best_kc - 1) / best_kc;
   const int kchunks = (a.nkb + a.kb_per_unit - 1) / a.kb_per_unit;
   a.units = a.ntiles * kchunks;
   a.vec4 = vec4;
   a.info = info;
+  a.flags = static_cast<uint32_t*>(flags);
+  a.gate = wg.gate;
+  a.limit_ns = wg.limit_ns;
   if ((e = cudaFuncSetAttribute(syrk_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)SMEM_BYTES)) != cudaSuccess)
     return e;

@@ -769,11 +769,15 @@ cudaError_t launch_gather_columns_u8(const uint8_t* src, int64_t rows, int64_t n
   return cudaGetLastError();
 }
 
+size_t dequant_matvec_workspace_bytes(int64_t batch, int64_t n) {
+  return ((size_t)batch * (size_t)n * sizeof(__nv_bfloat16) + 255) / 256 * 256;
+}
+
 cudaError_t launch_dequant_matvec(const uint32_t* packed, int bits, int64_t rows, int64_t n,
                                   const float* scales, const uint8_t* zeros, int group_size,
                                   int64_t n_groups, const int32_t* g_idx, const int32_t* perm,
                                   const void* x, int x_bf16, int64_t batch, float* y,
-                                  cudaStream_t s) {
+                                  void* ws, cudaStream_t s) {
   if (rows == 0 || batch == 0) return cudaSuccess;
   // the tensor-core path: int4 / int3, bf16 activations, groups that are runs of
   // 32 k consecutive columns, 16-byte aligned code rows and activations
@@ -782,14 +786,8 @@ cudaError_t launch_dequant_matvec(const uint32_t* packed, int bits, int64_t rows
   const bool mma = x_bf16 && !g_idx && n % 32 == 0 && (group_size <= 0 || pow2) &&
                    reinterpret_cast<uintptr_t>(packed) % (bits == 4 ? 16 : 4) == 0;
   if (mma) {
-    // x in MMA pair order (and sweep order under perm) in stream-ordered scratch
-    cudaMemPool_t pool;
-    if (!scratch_pool(&pool)) return cudaErrorMemoryAllocation;
-    __nv_bfloat16* xp = nullptr;
-    cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&xp),
-                                            (size_t)batch * (size_t)n * sizeof(__nv_bfloat16),
-                                            pool, s);
-    if (e != cudaSuccess) return e;
+    // x in MMA pair order (and sweep order under perm), in the caller's workspace
+    __nv_bfloat16* xp = static_cast<__nv_bfloat16*>(ws);
     const int64_t nwords = batch * (n / 8), ny = batch * rows;
     const int64_t work = std::max(nwords, ny);
     const unsigned pgrid = (unsigned)std::min<int64_t>((work + 255) / 256, (int64_t)num_sms() * 8);
@@ -820,9 +818,7 @@ cudaError_t launch_dequant_matvec(const uint32_t* packed, int bits, int64_t rows
             packed, rows, n, scales, zeros, gshift, n_groups, xb, nb, yb, rows);
       note_launch();
     }
-    e = cudaGetLastError();
-    const cudaError_t f = cudaFreeAsync(xp, s);
-    return e != cudaSuccess ? e : f;
+    return cudaGetLastError();
   }
   const size_t esz = x_bf16 ? 2 : 4;
   // batches of 8, 4, 2, 1 vectors per launch

@@ -74,6 +74,13 @@ __device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gmem_src
                "l"(gmem_src)
                : "memory");
 }
+// 16 bytes global -> shared with zero fill: src_bytes = 0 reads nothing and
+// stores zeros (the source address must still be a valid 16-byte aligned one).
+__device__ __forceinline__ void cp_async_16z(void* smem_dst, const void* gmem_src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src), "r"(src_bytes)
+               : "memory");
+}
 // 4 bytes global -> shared; with src_bytes = 0 nothing is read and 0 is stored.
 __device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gmem_src, int src_bytes) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(smem_dst)),
@@ -142,6 +149,59 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, 
 // barrier `id` (1..15) over `threads` threads of the CTA
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+// the same barrier, returning the AND of `pred` over the participating threads
+__device__ __forceinline__ bool named_bar_and(int id, int threads, bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %3, 0;\n\t"
+      "bar.red.and.pred q, %1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"(id), "r"(threads), "r"((uint32_t)pred)
+      : "memory");
+  return out != 0;
+}
+
+// ---------------------------------------------------------------- flags in global memory
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Waits until *flag >= target (acquire).  Returns false if `*abort` becomes
+// nonzero or `limit_ns` nanoseconds pass first.
+__device__ __forceinline__ bool flag_wait_bounded(const uint32_t* flag, uint32_t target,
+                                                  const volatile int* abort,
+                                                  uint64_t limit_ns) {
+  if (ld_acquire_gpu(flag) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i) {
+      __nanosleep(32);
+      if (ld_acquire_gpu(flag) >= target) return true;
+    }
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// Test gate of the bounded waits: waits until *gate != 0 (no gate: returns
+// true at once).  Returns false if `limit_ns` nanoseconds pass first.
+__device__ __forceinline__ bool gate_wait_bounded(const int32_t* gate, uint64_t limit_ns) {
+  if (!gate) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (*(const volatile int32_t*)gate == 0) {
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+    __nanosleep(256);
+  }
+  return true;
 }
 // generic-proxy writes to shared memory become visible to the async proxy
 __device__ __forceinline__ void fence_proxy_async_smem() {

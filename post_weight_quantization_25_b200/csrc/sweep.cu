@@ -38,10 +38,22 @@ namespace {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+constexpr int32_t kSweepInfoTimeout = -2;  // `info` value when a device wait gave up
+
+// Two-level blocking for wide layers: the lazy update inside a super-block of
+// kSuperCols columns is applied per 128-column block (K = 128), the update of
+// the columns past the super-block once per super-block (K = kSuperCols), so
+// those columns are read and written once per super-block instead of once
+// per block.  Narrower layers use one level (the super-block is the block).
+constexpr int kSuperCols = 1024;
+constexpr int64_t kTwoLevelMinN = 8192;
+int64_t super_cols(int64_t n) { return n >= kTwoLevelMinN ? kSuperCols : kBlock; }
+
 struct SweepWs {
   float* Wf;          // rows x n, sweep order; after the sweep holds w_hat
-  float* Err_hi[2];   // rows x 128: a block's err terms, TF32 part (blocks alternate)
-  float* Err_lo[2];   // rows x 128: remainder (err - Err_hi)
+  float* Err_hi[2];   // rows x S: a super-block's err terms, TF32 part (super-blocks alternate)
+  float* Err_lo[2];   // rows x S: remainder (err - Err_hi)
+  int64_t lde;        // S = super_cols(n)
   uint8_t* codes_sw;  // rows x n, sweep order
   int32_t* pos;       // n: sweep position of each original column
   float* UT_hi;       // n x ldut: U^T, TF32 part (the lazy update's K-major operand)
@@ -56,11 +68,12 @@ SweepWs carve(void* ws, int64_t rows, int64_t n) {
   SweepWs w;
   w.Wf = reinterpret_cast<float*>(p);
   p += align_up(sizeof(float) * rows * n, 256);
+  w.lde = super_cols(n);
   for (int b = 0; b < 2; ++b) {
     w.Err_hi[b] = reinterpret_cast<float*>(p);
-    p += align_up(sizeof(float) * rows * kBlock, 256);
+    p += align_up(sizeof(float) * rows * w.lde, 256);
     w.Err_lo[b] = reinterpret_cast<float*>(p);
-    p += align_up(sizeof(float) * rows * kBlock, 256);
+    p += align_up(sizeof(float) * rows * w.lde, 256);
   }
   w.codes_sw = reinterpret_cast<uint8_t*>(p);
   p += align_up((size_t)rows * n, 256);
@@ -104,6 +117,34 @@ __global__ void __launch_bounds__(256) ut_split_kernel(const float* __restrict__
 struct SweepTrailItems {
   float* Wf;
   int rows, n, i1, c0, c1;
+  int pk;  // column of the block's err terms in the super-block buffer
+  __host__ __device__ int num_items() const { return (rows + 127) / 128; }
+  __host__ __device__ int item_nq(int) const { return (c1 - c0 + 127) / 128; }
+  __device__ PgItem item(int i) const {
+    PgItem I;
+    I.C0 = Wf + (int64_t)i * 128 * n + c0;
+    I.ldc = n;
+    I.cmap = 0;
+    I.cx0 = c0;
+    I.cy0 = 128 * i;
+    I.prow = 128 * i;
+    I.pkx = pk;
+    I.qrow0 = c0;
+    I.qkx = i1;
+    I.nq = item_nq(i);
+    I.mext = min(128, rows - 128 * i);
+    I.cext_last = c1 - c0 - 128 * (I.nq - 1);
+    I.nkb = kBlock / 32;
+    return I;
+  }
+};
+
+// The update past a finished super-block [s1, s1 + S):
+//   Wf[:, c0:c1] -= Err_S U[s1:s1+S, c0:c1]   (K = S, stream_gemm_kernel)
+// Item i = rows [128 i, 128 i + 128) of Wf; its tiles run over the columns.
+struct SweepSuperItems {
+  float* Wf;
+  int rows, n, s1, S, c0, c1;
   __host__ __device__ int num_items() const { return (rows + 127) / 128; }
   __host__ __device__ int item_nq(int) const { return (c1 - c0 + 127) / 128; }
   __device__ PgItem item(int i) const {
@@ -116,10 +157,11 @@ struct SweepTrailItems {
     I.prow = 128 * i;
     I.pkx = 0;
     I.qrow0 = c0;
-    I.qkx = i1;
+    I.qkx = s1;
     I.nq = item_nq(i);
     I.mext = min(128, rows - 128 * i);
     I.cext_last = c1 - c0 - 128 * (I.nq - 1);
+    I.nkb = S / 32;
     return I;
   }
 };
@@ -203,31 +245,36 @@ __global__ void __launch_bounds__(256) gather_w_kernel(
   if (row_loss && threadIdx.x == 0) row_loss[r] = 0.f;
 }
 
-// One block [i1, i1 + bsz) of the sweep.  kSweepLanes lanes per row (a
-// "team"); lane q of a team holds block columns q, q + L, ..., q + 128 - L
-// (slot s = column / L, L = kSweepLanes).  Column jj is rounded in every lane
-// of the team, the owner lane's (jj % L) error term is broadcast inside the
-// team, and each lane repairs its columns past jj with row jj of U's diagonal
-// block.  The loop over jj is unrolled, so slots left of jj are skipped at
-// compile time.  4 lanes per row is the measured choice at 4096 rows; 16
-// lanes (8 slots each, 80 registers, twice the CTAs) computes the same
-// results but was slower there (2.15 ms against 1.52 ms per layer at 4096 x
-// 4096), its CTAs crowding out the concurrent far update.
-// Shared memory holds the block of U as  Uq[jj][q][slot] = U[i1+jj][i1+L slot+q]
-// (team-lane-major; row pitch kUqPitch floats per lane, chosen so the 16-byte
-// float4 reads of the 8 lanes of a phase hit distinct banks), plus 1/U_jj and
-// 1/(2 U_jj^2).
+// One block [i1, i1 + bsz) of the sweep.  A team of kSweepLanes = 4 lanes
+// works one row; a CTA of 128 threads holds 32 rows.
+//
+// The CTA stages U's 128 x 128 diagonal block and its rows' 128 columns of
+// Wf in shared memory.  The block is swept in sub-blocks of kSub = 16
+// columns: lane q of a team loads columns q, q + 4, q + 8, q + 12 of the
+// sub-block into registers, and the 16 column steps run fully unrolled:
+// every lane rounds its own value of the step's slot, the owner of the
+// column (lane k % 4) is broadcast inside the team, and each lane repairs
+// its later columns of the sub-block.  Then the sub-block's 16 error terms
+// (all lanes hold them) update the rest of the block in shared memory, lane
+// q taking the 4-column chunks q, q + 4, ... (a rolled rank-16 update).
+// Every column receives fmaf(-err_j, U[j][c], w) for j = 0, 1, ... in column
+// order, the same operations in the same order as one repair per column
+// step.  The sub-block loop is rolled, so the code stays small enough for
+// the instruction caches (a fully unrolled 128-step sweep does not fit them).
 //   GS = 0:   per-row ruler (already in scales / zeros)
 //   GS = 128: groups of a multiple of 128 columns, fitted at a block start that
 //             is a group start, from the current Wf
-//   GS = 32, 64: groups inside the block, fitted on the current registers
-constexpr int kSweepLanes = 4;                           // lanes per row (4 or 16)
-constexpr int kSweepSlots = kBlock / kSweepLanes;        // columns per lane
-constexpr int kSweepThreads = kSweepLanes == 4 ? 128 : 256;
-constexpr int kUqPitch = kSweepLanes == 4 ? 36 : 12;     // floats per (jj, q)
-constexpr int kUqRow = kSweepLanes * kUqPitch;           // floats per jj
-constexpr size_t kSweepSmemBytes = sizeof(float) * (kBlock * kUqRow + 2 * kBlock);
-static_assert(kSweepSlots % 4 == 0 && kUqPitch >= kSweepSlots, "sweep team layout");
+//   GS = 32, 64: groups inside the block, fitted on the current values
+// Columns past bsz (a short last block) hold 0 and their U rows are 0 with
+// 1/U_jj = 1: they round to the zero point with no error and change nothing.
+constexpr int kSweepLanes = 4;                          // lanes per row (a team)
+constexpr int kSweepThreads = 128;
+constexpr int kSweepRows = kSweepThreads / kSweepLanes; // rows per CTA
+constexpr int kSub = 16;                                // columns per unrolled sub-block
+constexpr int kSubSlots = kSub / kSweepLanes;           // columns per lane in a sub-block
+constexpr int kWbPitch = 132;                           // floats per row of the staged W block
+constexpr size_t kSweepSmemBytes =
+    sizeof(float) * (kBlock * kBlock + kSweepRows * kWbPitch + 2 * kBlock);
 
 __device__ __forceinline__ float team_min(float v) {
 #pragma unroll
@@ -244,37 +291,55 @@ template <int GS>
 __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
     float* __restrict__ Wf, int rows, int n, const float* __restrict__ U, int i1, int bsz,
     float maxq, int sym, int gsize, int G, float* __restrict__ Err_hi, float* __restrict__ Err_lo,
-    uint8_t* __restrict__ codes_sw, float* __restrict__ scales, uint8_t* __restrict__ zeros,
-    float* __restrict__ row_loss) {
-  constexpr int L = kSweepLanes, NS = kSweepSlots;
+    int lde, uint8_t* __restrict__ codes_sw, float* __restrict__ scales,
+    uint8_t* __restrict__ zeros, float* __restrict__ row_loss) {
+  constexpr int L = kSweepLanes, NS = kSubSlots;
   extern __shared__ __align__(16) float smem[];
-  float* Uq = smem;
-  float* rd = smem + kBlock * kUqRow;
-  float* hrd2 = rd + kBlock;
-  stage_block_128<kSweepThreads>(
-      U + (int64_t)i1 * n + i1, n, bsz, bsz, /*lower=*/false, (n % 4) == 0,
-      [&](int a, int b, float v) { Uq[a * kUqRow + (b % L) * kUqPitch + (b / L)] = v; },
-      [](int, int) { return 0.f; });
+  float* Ud = smem;                       // [128][128]  U[i1 + a][i1 + b], 0 past bsz
+  float* Wb = Ud + kBlock * kBlock;       // [32][kWbPitch]  this CTA's rows of the block
+  float* rd = Wb + kSweepRows * kWbPitch; // [128]  1 / U_jj
+  float* hrd2 = rd + kBlock;              // [128]  1 / (2 U_jj^2)
+  const int tid = threadIdx.x;
+  const int r0 = blockIdx.x * kSweepRows;
+  const int vr = min(kSweepRows, rows - r0);
+  if ((n % 4) == 0) {
+    // 16-byte async copies, all in flight at once; bsz is a multiple of 4 here
+    const float* us = U + (int64_t)i1 * n + i1;
+    const float* ws = Wf + (int64_t)r0 * n + i1;
+    for (int f = tid; f < kBlock * kBlock / 4; f += kSweepThreads) {
+      const int a = f >> 5, c = (f & 31) * 4;
+      const bool ok = a < bsz && c < bsz;
+      ptx::cp_async_16z(Ud + a * kBlock + c, ok ? us + (int64_t)a * n + c : us, ok ? 16 : 0);
+    }
+    for (int f = tid; f < kSweepRows * kBlock / 4; f += kSweepThreads) {
+      const int a = f >> 5, c = (f & 31) * 4;
+      const bool ok = a < vr && c < bsz;
+      ptx::cp_async_16z(Wb + a * kWbPitch + c, ok ? ws + (int64_t)a * n + c : ws, ok ? 16 : 0);
+    }
+    ptx::cp_async_wait_all();
+  } else {
+    stage_block_128<kSweepThreads>(
+        U + (int64_t)i1 * n + i1, n, bsz, bsz, /*lower=*/false, false,
+        [&](int a, int b, float v) { Ud[a * kBlock + b] = v; }, [](int, int) { return 0.f; });
+    for (int f = tid; f < kSweepRows * kBlock; f += kSweepThreads) {
+      const int a = f >> 7, c = f & 127;
+      Wb[a * kWbPitch + c] = (a < vr && c < bsz) ? Wf[(int64_t)(r0 + a) * n + i1 + c] : 0.f;
+    }
+  }
   __syncthreads();
-  for (int i = threadIdx.x; i < kBlock; i += blockDim.x) {
-    const float d = (i < bsz) ? Uq[i * kUqRow + (i % L) * kUqPitch + (i / L)] : 1.f;
+  for (int i = tid; i < kBlock; i += kSweepThreads) {
+    const float d = (i < bsz) ? Ud[i * kBlock + i] : 1.f;
     rd[i] = 1.f / d;
     hrd2[i] = 0.5f / (d * d);
   }
   __syncthreads();
 
-  const int lane = threadIdx.x & 31;
-  const int q = lane % L;
-  const int r = (blockIdx.x * blockDim.x + threadIdx.x) / L;
-  const bool active = r < rows;
-  float* wrow = Wf + (int64_t)(active ? r : 0) * n + i1;
-  float w[NS];
-#pragma unroll
-  for (int s = 0; s < NS; ++s) {
-    const int c = L * s + q;
-    w[s] = (active && c < bsz) ? wrow[c] : 0.f;
-  }
-
+  const int lane = tid & 31;
+  const int q = lane % L;                 // lane within the team
+  const int rl = tid / L;                 // row within the CTA
+  const int r = r0 + rl;
+  const bool active = rl < vr;
+  float* wrow = Wb + rl * kWbPitch;
   float scale = 1.f, zf = 0.f;
   if (GS == 0) {
     if (active) {
@@ -285,12 +350,10 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
     const int g = i1 / gsize;
     if (i1 % gsize == 0) {
       float mn = INFINITY, mx = -INFINITY;
-#pragma unroll
-      for (int s = 0; s < NS; ++s)
-        if (L * s + q < bsz) {
-          mn = fminf(mn, w[s]);
-          mx = fmaxf(mx, w[s]);
-        }
+      for (int c = q; c < kBlock; c += L) {
+        mn = fminf(mn, wrow[c]);
+        mx = fmaxf(mx, wrow[c]);
+      }
       const int end = min(i1 + gsize, n);
       if (active)
         for (int c = i1 + kBlock + q; c < end; c += L) {
@@ -308,87 +371,101 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
       zf = (float)zeros[(int64_t)r * G + g];
     }
   }
-
   // w / scale, correctly rounded, with the reciprocal of the scale computed
   // once per ruler (Markstein's method, fdiv.cuh)
   MDiv md = md_prepare(scale);
-  float e_out[NS];
-  uint32_t cw[NS / 4];
-#pragma unroll
-  for (int s = 0; s < NS; ++s) e_out[s] = 0.f;
-#pragma unroll
-  for (int k = 0; k < NS / 4; ++k) cw[k] = 0u;
   float loss = 0.f;
-  const float* uq_lane = Uq + q * kUqPitch;
+  float* wg = Wf + (int64_t)(active ? r : 0) * n + i1;
+  uint8_t* cg = codes_sw + (int64_t)(active ? r : 0) * n + i1;
+  float* ehi = Err_hi + (int64_t)(active ? r : 0) * lde;
+  float* elo = Err_lo + (int64_t)(active ? r : 0) * lde;
 
+#pragma unroll 1
+  for (int c0 = 0; c0 < kBlock; c0 += kSub) {
+    // this lane's columns c0 + L s + q of the sub-block
+    float cur[NS];
 #pragma unroll
-  for (int s = 0; s < NS; ++s) {
-#pragma unroll
-  for (int k = 0; k < L; ++k) {
-    // No early exit for a short last block: its columns past bsz hold 0 and
-    // its U rows past bsz are 0 (with 1/U_jj = 1), so they round to the zero
-    // point with no error and change nothing; keeping the 128 steps free of
-    // branches lets the compiler overlap consecutive steps.
-    const int jj = L * s + k;
-    constexpr int kGS = (GS == 32 || GS == 64) ? GS : L;  // in-block group size
-    if ((GS == 32 || GS == 64) && (jj % kGS) == 0) {
-      // group [jj, jj + GS) of the block, current (repaired) values
+    for (int s = 0; s < NS; ++s) cur[s] = wrow[c0 + L * s + q];
+    constexpr int kGS = (GS == 32 || GS == 64) ? GS : kBlock;  // in-block group size
+    if ((GS == 32 || GS == 64) && (c0 % kGS) == 0) {
+      // the group [c0, c0 + GS) of the block, current (repaired) values
       float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
-      for (int s2 = s; s2 < s + kGS / L; ++s2)
-        if (L * s2 + q < bsz) {
-          mn = fminf(mn, w[s2]);
-          mx = fmaxf(mx, w[s2]);
-        }
+      for (int s = 0; s < NS; ++s) {
+        mn = fminf(mn, cur[s]);
+        mx = fmaxf(mx, cur[s]);
+      }
+      for (int c = c0 + kSub + q; c < c0 + kGS; c += L) {
+        mn = fminf(mn, wrow[c]);
+        mx = fmaxf(mx, wrow[c]);
+      }
       fit_ruler(team_min(mn), team_max(mx), maxq, sym, scale, zf);
       md = md_prepare(scale);
-      if (active && q == 0 && jj < bsz) {  // groups past the last column do not exist
-        const int g = (i1 + jj) / kGS;
+      if (active && q == 0 && c0 < bsz) {  // groups past the last column do not exist
+        const int g = (i1 + c0) / kGS;
         scales[(int64_t)r * G + g] = scale;
         zeros[(int64_t)r * G + g] = (uint8_t)zf;
       }
     }
-    // every lane rounds its slot s; the owner's (q == jj % L) result is used
-    const float x = w[s];
-    float qv = rintf(md_div(x, md)) + zf;
-    qv = fminf(fmaxf(qv, 0.f), maxq);
-    const float wh = __fmul_rn(scale, qv - zf);
-    const float e = x - wh;
-    const float ev = e * rd[jj];
-    const float err = __shfl_sync(0xffffffffu, ev, k, L);
-    const float* urow = uq_lane + jj * kUqRow;
+    float ev_sub[kSub];   // the sub-block's error terms (every lane of the team)
+    float e_own[NS];      // this lane's own columns' error terms
+    uint32_t cw = 0u;     // this lane's own columns' codes, one byte each
 #pragma unroll
-    for (int s4 = s >> 2; s4 < NS / 4; ++s4) {
-      const float4 u = *reinterpret_cast<const float4*>(urow + 4 * s4);
-      if (4 * s4 + 0 >= s) w[4 * s4 + 0] = fmaf(-err, u.x, w[4 * s4 + 0]);
-      if (4 * s4 + 1 >= s) w[4 * s4 + 1] = fmaf(-err, u.y, w[4 * s4 + 1]);
-      if (4 * s4 + 2 >= s) w[4 * s4 + 2] = fmaf(-err, u.z, w[4 * s4 + 2]);
-      if (4 * s4 + 3 >= s) w[4 * s4 + 3] = fmaf(-err, u.w, w[4 * s4 + 3]);
+    for (int k = 0; k < kSub; ++k) {
+      const int jj = c0 + k;
+      const int s = k / L, ko = k % L;   // the step's slot, and its owner lane
+      // every lane rounds its own value of slot s; the owner's is used
+      const float x = cur[s];
+      float qv = rintf(md_div(x, md)) + zf;
+      qv = fminf(fmaxf(qv, 0.f), maxq);
+      const float wh = __fmul_rn(scale, qv - zf);
+      const float e = x - wh;
+      const float ev = e * rd[jj];
+      const float err = __shfl_sync(0xffffffffu, ev, ko, L);
+      ev_sub[k] = err;
+      const bool own = (q == ko);
+      loss = own ? fmaf(e * e, hrd2[jj], loss) : loss;
+      cur[s] = own ? wh : cur[s];
+      e_own[s] = own ? ev : e_own[s];
+      cw |= own ? (((uint32_t)qv) << (8 * s)) : 0u;
+      // repair this lane's later columns of the sub-block
+      const float* urow = Ud + jj * kBlock + c0;
+#pragma unroll
+      for (int s2 = s; s2 < NS; ++s2)
+        if (s2 > s || q > ko) cur[s2] = fmaf(-err, urow[L * s2 + q], cur[s2]);
     }
-    const bool own = (q == k);
-    w[s] = own ? wh : w[s];
-    e_out[s] = own ? ev : e_out[s];
-    loss = own ? fmaf(e * e, hrd2[jj], loss) : loss;
-    cw[s >> 2] |= own ? (((uint32_t)qv) << (8 * (s & 3))) : 0u;
-  }
-  }
-
-  if (active) {
-    uint8_t* crow = codes_sw + (int64_t)r * n + i1;
-    float* ehi = Err_hi + (int64_t)r * kBlock;
-    float* elo = Err_lo + (int64_t)r * kBlock;
+    // the sub-block's results: w_hat into Wf, codes, error terms (TF32 split)
+    if (active) {
 #pragma unroll
-    for (int s = 0; s < NS; ++s) {
-      const int c = L * s + q;
-      if (c < bsz) {
-        crow[c] = (uint8_t)((cw[s >> 2] >> (8 * (s & 3))) & 0xFFu);
-        wrow[c] = w[s];
+      for (int s = 0; s < NS; ++s) {
+        const int c = c0 + L * s + q;
+        if (c < bsz) {
+          wg[c] = cur[s];
+          cg[c] = (uint8_t)((cw >> (8 * s)) & 0xFFu);
+        }
+        float h, l;
+        tf32_split(e_own[s], h, l);
+        ehi[c] = h;
+        elo[c] = l;
       }
-      float h, l;
-      tf32_split(e_out[s], h, l);
-      ehi[c] = h;
-      elo[c] = l;
     }
+    // rank-16 update of the block's later columns (shared memory), lane q
+    // taking the 4-column chunks q, q + L, ...
+#pragma unroll 1
+    for (int c = c0 + kSub + 4 * q; c < kBlock; c += 4 * L) {
+      float4 w4 = *reinterpret_cast<const float4*>(wrow + c);
+      const float* ucol = Ud + c0 * kBlock + c;
+#pragma unroll
+      for (int j = 0; j < kSub; ++j) {
+        const float4 u = *reinterpret_cast<const float4*>(ucol + j * kBlock);
+        w4.x = fmaf(-ev_sub[j], u.x, w4.x);
+        w4.y = fmaf(-ev_sub[j], u.y, w4.y);
+        w4.z = fmaf(-ev_sub[j], u.z, w4.z);
+        w4.w = fmaf(-ev_sub[j], u.w, w4.w);
+      }
+      *reinterpret_cast<float4*>(wrow + c) = w4;
+    }
+    __syncwarp();  // the team's chunk writes land before the next sub-block's loads
   }
   if (row_loss) {
 #pragma unroll
@@ -450,7 +527,7 @@ cudaError_t launch_selftest_division(const float* a, const float* b, int64_t cou
 
 size_t quantize_workspace_bytes(int64_t rows, int64_t n) {
   return align_up(sizeof(float) * rows * n, 256) +
-         4 * align_up(sizeof(float) * rows * kBlock, 256) + align_up((size_t)rows * n, 256) +
+         4 * align_up(sizeof(float) * rows * super_cols(n), 256) + align_up((size_t)rows * n, 256) +
          align_up(sizeof(int32_t) * n, 256) + 2 * align_up(sizeof(float) * n * ut_ld(n), 256);
 }
 
@@ -458,7 +535,8 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
                                   const float* U, const int32_t* perm, const uint8_t* dead,
                                   int bits, int group_size, int sym, uint8_t* codes,
                                   float* scales, uint8_t* zeros, int32_t* g_idx, float* Wq,
-                                  float* row_loss, void* ws, cudaStream_t s) {
+                                  float* row_loss, void* ws, int32_t* info, cudaStream_t s,
+                                  cudaStream_t side_s) {
   const int rows = (int)rows64, n = (int)n64;
   SweepWs w = carve(ws, rows64, n64);
   const float maxq = (float)((1 << bits) - 1);
@@ -467,6 +545,7 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
   const int gmode = per_row ? 0 : (group_size >= kBlock ? 1 : 2);
   cudaError_t e;
 
+  if (info && (e = cudaMemsetAsync(info, 0, sizeof(int32_t), s)) != cudaSuccess) return e;
   pos_kernel<<<(n + 255) / 256, 256, 0, s>>>(perm, n, w.pos);
   note_launch();
   const size_t row_smem = sizeof(float) * (size_t)n;
@@ -489,11 +568,12 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
   if ((e = set_smem(sweep_block_kernel<128>, us_smem)) != cudaSuccess) return e;
   if ((e = set_smem(sweep_block_kernel<32>, us_smem)) != cudaSuccess) return e;
   if ((e = set_smem(sweep_block_kernel<64>, us_smem)) != cudaSuccess) return e;
-  const int sweep_ctas = (rows * kSweepLanes + kSweepThreads - 1) / kSweepThreads;
+  const int sweep_ctas = (rows + kSweepRows - 1) / kSweepRows;
   const int sms = num_sms();
 
   // operands of the lazy update on the tensor cores; with a row stride that
   // is a multiple of 16 bytes the update lands in Wf by TMA reduce-add
+  const int S = (int)w.lde;  // super-block columns (kBlock: one level)
   CUtensorMap mEh[2], mEl[2], mUh, mUl, mW;
   const bool reduce = (n % 4) == 0;
   if (n > kBlock) {
@@ -501,105 +581,160 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
         U, n, w.ldut, w.UT_hi, w.UT_lo);
     note_launch();
     for (int b = 0; b < 2; ++b)
-      if (!make_tma_2d(&mEh[b], w.Err_hi[b], false, rows, kBlock, kBlock, 32, 128) ||
-          !make_tma_2d(&mEl[b], w.Err_lo[b], false, rows, kBlock, kBlock, 32, 128))
+      if (!make_tma_2d(&mEh[b], w.Err_hi[b], false, rows, S, S, 32, 128) ||
+          !make_tma_2d(&mEl[b], w.Err_lo[b], false, rows, S, S, 32, 128))
         return cudaErrorInvalidValue;
     if (!make_tma_2d(&mUh, w.UT_hi, false, n, n, w.ldut, 32, 128) ||
         !make_tma_2d(&mUl, w.UT_lo, false, n, n, w.ldut, 32, 128))
       return cudaErrorInvalidValue;
     if (reduce) {
       if (!make_tma_2d(&mW, w.Wf, false, rows, n, n, 32, 32)) return cudaErrorInvalidValue;
-      if ((e = cudaFuncSetAttribute(panel_gemm2_kernel<SweepTrailItems, true>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)pg2_smem_bytes(true))) != cudaSuccess)
-        return e;
     } else {
       mW = mUh;  // not read by the read-modify-write epilogue
-      if ((e = cudaFuncSetAttribute(panel_gemm2_kernel<SweepTrailItems, false>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)pg2_smem_bytes(false))) != cudaSuccess)
-        return e;
     }
+    if ((e = cudaFuncSetAttribute(reduce ? (const void*)panel_gemm2_kernel<SweepTrailItems, true>
+                                         : (const void*)panel_gemm2_kernel<SweepTrailItems, false>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)pg2_smem_bytes(reduce))) != cudaSuccess)
+      return e;
+    if (S > kBlock &&
+        (e = cudaFuncSetAttribute(reduce ? (const void*)stream_gemm_kernel<SweepSuperItems, true>
+                                         : (const void*)stream_gemm_kernel<SweepSuperItems, false>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)sg_smem_bytes(reduce))) != cudaSuccess)
+      return e;
   }
-  auto trail = [&](int blk, int i1, int c0, int c1, int max_grid, cudaStream_t st) {
-    const SweepTrailItems dec{w.Wf, rows, n, i1, c0, c1};
+  const WaitGate wg = current_wait_gate();
+  // rank-128 update by block i1's err terms (column pk of buffer eb): columns [c0, c1)
+  auto trail = [&](int eb, int i1, int pk, int c0, int c1, int max_grid, cudaStream_t st) {
+    const SweepTrailItems dec{w.Wf, rows, n, i1, c0, c1, pk};
     int chunk = 1, units = 0;
     pg2_plan(dec, max_grid, chunk, units);
     const int grid = std::min(units, max_grid);
-    const int eb = blk & 1;
     if (reduce)
       panel_gemm2_kernel<SweepTrailItems, true><<<grid, kPg2Threads, pg2_smem_bytes(true), st>>>(
-          mEh[eb], mEl[eb], mUh, mUl, mW, mW, dec, chunk, units, nullptr, 0, nullptr);
+          mEh[eb], mEl[eb], mUh, mUl, mW, mW, dec, chunk, units, info, kSweepInfoTimeout,
+          nullptr, wg.gate, wg.limit_ns);
     else
       panel_gemm2_kernel<SweepTrailItems, false><<<grid, kPg2Threads, pg2_smem_bytes(false), st>>>(
-          mEh[eb], mEl[eb], mUh, mUl, mW, mW, dec, chunk, units, nullptr, 0, nullptr);
+          mEh[eb], mEl[eb], mUh, mUl, mW, mW, dec, chunk, units, info, kSweepInfoTimeout,
+          nullptr, wg.gate, wg.limit_ns);
+    note_launch();
+  };
+  // the update past the super-block [s1, s1 + S) (all its err terms): columns [c0, c1)
+  auto past = [&](int eb, int s1, int c0, int c1, int max_grid, cudaStream_t st) {
+    if (S == kBlock) {
+      trail(eb, s1, 0, c0, c1, max_grid, st);
+      return;
+    }
+    const SweepSuperItems dec{w.Wf, rows, n, s1, S, c0, c1};
+    const int units = sg_units(dec);
+    const int grid = std::min(units, max_grid);
+    if (reduce)
+      stream_gemm_kernel<SweepSuperItems, true><<<grid, kPg2Threads, sg_smem_bytes(true), st>>>(
+          mEh[eb], mEl[eb], mUh, mUl, mW, mW, dec, units, info, kSweepInfoTimeout, nullptr,
+          wg.gate, wg.limit_ns);
+    else
+      stream_gemm_kernel<SweepSuperItems, false><<<grid, kPg2Threads, sg_smem_bytes(false), st>>>(
+          mEh[eb], mEl[eb], mUh, mUl, mW, mW, dec, units, info, kSweepInfoTimeout, nullptr,
+          wg.gate, wg.limit_ns);
     note_launch();
   };
 
-  // Look-ahead.  After block b is swept, only block b+1's columns are
-  // updated on the caller's stream (the "near" update, which the next sweep
-  // waits for); the update of every later column ("far") runs on the side
-  // stream, on part of the SMs, while block b+1 is swept.  Each column block
-  // still receives its updates in block order -- far(0), ..., far(c-2),
-  // near(c-1) for block c -- because near(b) waits for far(b-1); the err
-  // terms alternate between two buffers, and sweep(b+2) (after near(b+1),
-  // after far(b)) is the next writer of far(b)'s buffer.
-  SideStream side{};
-  const bool lookahead = n > 2 * kBlock && side_stream(&side);
-  std::unique_lock<std::mutex> side_guard(side_lock(), std::defer_lock);
-  // SMs left to the far update: the sweep's CTAs (up to two per SM) keep the rest
-  const int far_grid = std::max(sms / 4, sms - (sweep_ctas + 1) / 2);
-  if (lookahead) {
-    side_guard.lock();
-    if ((e = cudaEventRecord(side.ev[0], s)) != cudaSuccess ||
-        (e = cudaStreamWaitEvent(side.s, side.ev[0], 0)) != cudaSuccess)
-      return e;
-  }
-  bool far_pending = false;  // far(b-1) was issued and near(b) must wait for it
-  for (int i1 = 0, blk = 0; i1 < n; i1 += kBlock, ++blk) {
-    const int bsz = std::min(kBlock, n - i1);
-    const int i2 = i1 + bsz;
-    const int eb = blk & 1;
+  // Look-ahead (with a side stream).  After block b is swept, only the next
+  // block's columns are updated on the caller's stream (the "near" update,
+  // which the next sweep waits for); the update of every later column
+  // ("far") runs on the side stream, on part of the SMs, while the next
+  // block is swept.  Inside a super-block the updates are rank-128 and stop
+  // at the super-block's end; after its last block, the update past it (all
+  // its err terms at once) is split the same way.  Every column still
+  // receives its updates in a fixed order -- each near update waits for the
+  // far update issued before it -- so the result does not depend on how the
+  // streams interleave.  The err terms of consecutive super-blocks go to two
+  // buffers; the next writer of a buffer (the first sweep two super-blocks
+  // on) runs after the caller's stream has waited for the last far update
+  // that reads it.
+  SideEvents side;
+  const bool lookahead = n > 2 * kBlock && side_s != nullptr && side_s != s;
+  if (lookahead && !side.create()) return cudaErrorMemoryAllocation;
+  // SMs for the far updates, which run beside the next blocks' sweeps: what
+  // one wave of the sweep's CTAs (two per SM) leaves, but at least half of
+  // them -- on tall layers the far updates past a super-block are most of
+  // the work, and a sweep that takes two waves costs less than starving them
+  const int far_grid = std::max(sms / 2, sms - (sweep_ctas + 1) / 2);
+  auto fork = [&]() -> cudaError_t {
+    cudaError_t r = cudaEventRecord(side.ev[0], s);
+    return r != cudaSuccess ? r : cudaStreamWaitEvent(side_s, side.ev[0], 0);
+  };
+  if (lookahead && (e = fork()) != cudaSuccess) return e;
+  bool far_pending = false;   // a far update inside the super-block (ev[1]) is unwaited
+  bool past_pending = false;  // a far update past a super-block (ev[2]) is unwaited
+  bool last = false;
+  for (int s1 = 0, sb = 0; s1 < n && !last; s1 += S, ++sb) {
+    const int s2 = std::min(s1 + S, n);
+    const int eb = sb & 1;
+    for (int i1 = s1; i1 < s2; i1 += kBlock) {
+      const int bsz = std::min(kBlock, n - i1);
+      const int i2 = i1 + bsz;
+      const int pk = i1 - s1;
 #define GPTQ_SWEEP_LAUNCH(GSV)                                                                 \
   sweep_block_kernel<GSV><<<sweep_ctas, kSweepThreads, us_smem, s>>>(                          \
-      w.Wf, rows, n, U, i1, bsz, maxq, sym, group_size, G, w.Err_hi[eb], w.Err_lo[eb],         \
-      w.codes_sw, scales, zeros, row_loss)
-    if (gmode == 0)
-      GPTQ_SWEEP_LAUNCH(0);
-    else if (gmode == 1)
-      GPTQ_SWEEP_LAUNCH(128);
-    else if (group_size == 32)
-      GPTQ_SWEEP_LAUNCH(32);
-    else
-      GPTQ_SWEEP_LAUNCH(64);
+      w.Wf, rows, n, U, i1, bsz, maxq, sym, group_size, G, w.Err_hi[eb] + pk,                  \
+      w.Err_lo[eb] + pk, S, w.codes_sw, scales, zeros, row_loss)
+      if (gmode == 0)
+        GPTQ_SWEEP_LAUNCH(0);
+      else if (gmode == 1)
+        GPTQ_SWEEP_LAUNCH(128);
+      else if (group_size == 32)
+        GPTQ_SWEEP_LAUNCH(32);
+      else
+        GPTQ_SWEEP_LAUNCH(64);
 #undef GPTQ_SWEEP_LAUNCH
-    note_launch();
-    if (i2 >= n) break;  // bsz == 128 below: only the last block is short
-    if (!lookahead) {
-      trail(blk, i1, i2, n, sms, s);
-      continue;
-    }
-    const int near_end = std::min(i2 + kBlock, n);
-    if (near_end < n) {
-      // far(b) needs block b's err terms: fork after the sweep
-      if ((e = cudaEventRecord(side.ev[0], s)) != cudaSuccess ||
-          (e = cudaStreamWaitEvent(side.s, side.ev[0], 0)) != cudaSuccess)
-        return e;
-    }
-    if (far_pending && (e = cudaStreamWaitEvent(s, side.ev[1], 0)) != cudaSuccess) return e;
-    trail(blk, i1, i2, near_end, sms, s);
-    far_pending = false;
-    if (near_end < n) {
-      trail(blk, i1, near_end, n, far_grid, side.s);
-      if ((e = cudaEventRecord(side.ev[1], side.s)) != cudaSuccess) return e;
-      far_pending = true;
+      note_launch();
+      if (i2 >= n) {  // bsz == 128 below: only the last block is short
+        last = true;
+        break;
+      }
+      const bool inside = i2 < s2;        // more blocks of this super-block follow
+      const int end = inside ? s2 : n;    // the columns this block's update reaches
+      if (!lookahead) {
+        if (inside)
+          trail(eb, i1, pk, i2, end, sms, s);
+        else
+          past(eb, s1, i2, end, sms, s);
+        continue;
+      }
+      const int near_end = std::min(i2 + kBlock, end);
+      if (near_end < end && (e = fork()) != cudaSuccess) return e;
+      if (far_pending) {
+        if ((e = cudaStreamWaitEvent(s, side.ev[1], 0)) != cudaSuccess) return e;
+        far_pending = false;
+      }
+      if (past_pending) {
+        if ((e = cudaStreamWaitEvent(s, side.ev[2], 0)) != cudaSuccess) return e;
+        past_pending = false;
+      }
+      if (inside)
+        trail(eb, i1, pk, i2, near_end, sms, s);
+      else
+        past(eb, s1, i2, near_end, sms, s);
+      if (near_end < end) {
+        if (inside) {
+          trail(eb, i1, pk, near_end, end, far_grid, side_s);
+          if ((e = cudaEventRecord(side.ev[1], side_s)) != cudaSuccess) return e;
+          far_pending = true;
+        } else {
+          past(eb, s1, near_end, end, far_grid, side_s);
+          if ((e = cudaEventRecord(side.ev[2], side_s)) != cudaSuccess) return e;
+          past_pending = true;
+        }
+      }
     }
   }
   if (lookahead) {  // join: everything on the side stream precedes what follows on s
-    if ((e = cudaEventRecord(side.ev[1], side.s)) != cudaSuccess ||
+    if ((e = cudaEventRecord(side.ev[1], side_s)) != cudaSuccess ||
         (e = cudaStreamWaitEvent(s, side.ev[1], 0)) != cudaSuccess)
       return e;
-    side_guard.unlock();
   }
   const size_t un_smem = (Wq ? sizeof(float) * (size_t)n : 0) + (size_t)n;
   if ((e = set_smem(unpermute_kernel, un_smem)) != cudaSuccess) return e;

@@ -44,12 +44,19 @@ def test_status_strings(lib):
 def test_workspace_sizes(lib):
     out = ctypes.c_size_t(0)
     cfg = _lib.GptqConfig(4, 128, 0.01, 128, 1, 0)
+    # bf16: the turnstile counters of the ordered split-K reduction only
     assert lib.gptq_workspace_size(_lib.GPTQ_OP_HESSIAN, 0, 256, 2048, _lib.GPTQ_BF16, None,
                                    ctypes.byref(out)) == 0
-    assert out.value == 0
+    assert 0 < out.value <= 4096
+    flags = out.value
     assert lib.gptq_workspace_size(_lib.GPTQ_OP_HESSIAN, 0, 256, 2048, _lib.GPTQ_F32, None,
                                    ctypes.byref(out)) == 0
-    assert out.value >= 2 * 256 * 2048 * 2
+    assert out.value >= flags + 2 * 256 * 2048 * 2
+    assert lib.gptq_workspace_size(_lib.GPTQ_OP_DEQUANT_MATVEC, 8, 4096, 0, 0, None,
+                                   ctypes.byref(out)) == 0
+    assert out.value >= 8 * 4096 * 2
+    assert lib.gptq_workspace_size(_lib.GPTQ_OP_DEQUANT_MATVEC, -1, 4096, 0, 0, None,
+                                   ctypes.byref(out)) == 1
     assert lib.gptq_workspace_size(_lib.GPTQ_OP_CHOLESKY, 0, 4096, 0, 0, None,
                                    ctypes.byref(out)) == 0
     assert out.value >= 4096 * 4096 * 4
@@ -82,21 +89,33 @@ def test_argument_checks_reject_before_any_launch(lib):
                                        1, 2.0, None, 0, None, None) == 2      # token-major
     assert lib.gptq_hessian_accumulate(ctypes.c_void_p(256), ctypes.c_void_p(256), 1, 16, 16, 16,
                                        0, 2.0, None, 0, None, None) == 3      # fp32 needs ws
+    assert lib.gptq_hessian_accumulate(ctypes.c_void_p(256), ctypes.c_void_p(256), 0, 16, 16, 16,
+                                       0, 2.0, None, 0, None, None) == 3      # bf16 too
     assert lib.gptq_hessian_accumulate(ctypes.c_void_p(256), ctypes.c_void_p(258), 0, 16, 16, 16,
-                                       0, 2.0, None, 0, None, None) == 1      # misaligned X
+                                       0, 2.0, ctypes.c_void_p(512), 4096, None,
+                                       None) == 1                             # misaligned X
+    assert lib.gptq_hessian_accumulate(ctypes.c_void_p(256), ctypes.c_void_p(256), 0, 16, 16, 16,
+                                       0, 2.0, ctypes.c_void_p(520), 4096, None,
+                                       None) == 1                             # misaligned ws
     assert lib.gptq_cholesky_inverse(None, 16, 0.01, 0, None, None, None, None, None, 0,
-                                     None) == 1
+                                     None, None) == 1
     assert lib.gptq_cholesky_inverse(ctypes.c_void_p(256), 16, 0.01, 1, ctypes.c_void_p(256),
                                      None, ctypes.c_void_p(256), ctypes.c_void_p(256), None, 0,
-                                     None) == 1                               # act-order, no perm
+                                     None, None) == 1                         # act-order, no perm
     assert lib.gptq_cholesky_inverse(ctypes.c_void_p(256), 16, 0.01, 0, ctypes.c_void_p(256),
                                      None, ctypes.c_void_p(256), ctypes.c_void_p(256), None, 0,
-                                     None) == 3                               # no workspace
+                                     None, None) == 3                         # no workspace
     cfg = _lib.GptqConfig(4, 128, 0.01, 128, 0, 0)
     assert lib.gptq_quantize_layer(None, 0, 0, 16, None, None, None, ctypes.byref(cfg), None,
-                                   None, None, None, None, None, None, 0, None) == 0   # empty
+                                   None, None, None, None, None, None, 0, None, None,
+                                   None) == 0                                 # empty
     assert lib.gptq_quantize_layer(None, 0, 4, 16, None, None, None, ctypes.byref(cfg), None,
-                                   None, None, None, None, None, None, 0, None) == 1
+                                   None, None, None, None, None, None, 0, None, None,
+                                   None) == 1
+    # the wait gate: a limit out of range is rejected; clearing always works
+    assert lib.gptq_set_wait_gate(ctypes.c_void_p(256), 0) == 1
+    assert lib.gptq_set_wait_gate(ctypes.c_void_p(256), 2_000_000_000) == 1
+    assert lib.gptq_set_wait_gate(None, 0) == 0
     assert lib.gptq_pack_int4(None, 4, 12, None, None) == 1                   # n % 8
     assert lib.gptq_pack_int3(None, 4, 40, None, None) == 1                   # n % 32
     assert lib.gptq_pack_int4(None, 0, 16, None, None) == 0                   # empty
@@ -127,17 +146,28 @@ def test_consumer_calls_with_nothing_to_do_or_bad_arguments(lib):
     launch."""
     p = ctypes.c_void_p(0x1000)
     # gptq_dequant_matvec(packed, bits, rows, n, scales, zeros, gsize, ngroups,
-    #                     g_idx, perm, x, xt, batch, y, stream)
+    #                     g_idx, perm, x, xt, batch, y, ws, ws_bytes, stream)
     assert lib.gptq_dequant_matvec(None, 4, 0, 64, None, None, 32, 2, None, None, None, 0, 1,
-                                   None, None) == 0
+                                   None, None, 0, None) == 0
     assert lib.gptq_dequant_matvec(None, 4, 8, 64, None, None, 32, 2, None, None, None, 0, 0,
-                                   None, None) == 0
-    assert lib.gptq_dequant_matvec(p, 5, 8, 64, p, p, 32, 2, None, None, p, 0, 1, p, None) == 2
-    assert lib.gptq_dequant_matvec(p, 4, 8, 60, p, p, 32, 2, None, None, p, 0, 1, p, None) == 1
-    assert lib.gptq_dequant_matvec(p, 3, 8, 48, p, p, 16, 3, None, None, p, 0, 1, p, None) == 1
-    assert lib.gptq_dequant_matvec(p, 4, 8, 64, p, p, 32, 2, p, p, p, 0, 1, p, None) == 1
-    assert lib.gptq_dequant_matvec(p, 4, 8, 64, p, p, 32, 2, None, None, p, 7, 1, p, None) == 1
-    assert lib.gptq_dequant_matvec(p, 4, 8, 64, p, p, 32, 1, None, None, p, 0, 1, p, None) == 1
+                                   None, None, 0, None) == 0
+    assert lib.gptq_dequant_matvec(p, 5, 8, 64, p, p, 32, 2, None, None, p, 0, 1, p, p, 256,
+                                   None) == 2
+    assert lib.gptq_dequant_matvec(p, 4, 8, 60, p, p, 32, 2, None, None, p, 0, 1, p, p, 256,
+                                   None) == 1
+    assert lib.gptq_dequant_matvec(p, 3, 8, 48, p, p, 16, 3, None, None, p, 0, 1, p, p, 256,
+                                   None) == 1
+    assert lib.gptq_dequant_matvec(p, 4, 8, 64, p, p, 32, 2, p, p, p, 0, 1, p, p, 256,
+                                   None) == 1
+    assert lib.gptq_dequant_matvec(p, 4, 8, 64, p, p, 32, 2, None, None, p, 7, 1, p, p, 256,
+                                   None) == 1
+    assert lib.gptq_dequant_matvec(p, 4, 8, 64, p, p, 32, 1, None, None, p, 0, 1, p, p, 256,
+                                   None) == 1
+    # a workspace too small for the x staging, or none
+    assert lib.gptq_dequant_matvec(p, 4, 8, 64, p, p, 32, 2, None, None, p, 0, 4, p, p, 256,
+                                   None) == 3
+    assert lib.gptq_dequant_matvec(p, 4, 8, 64, p, p, 32, 2, None, None, p, 0, 1, p, None, 0,
+                                   None) == 3
     # gptq_gather_columns_u8(src, rows, n, perm, dst, stream)
     assert lib.gptq_gather_columns_u8(None, 0, 64, None, None, None) == 0
     assert lib.gptq_gather_columns_u8(p, 4, 64, p, p, None) == 1  # src == dst

@@ -1,5 +1,7 @@
 """Repeatability of the kernels whose design claims it.
 
+- gptq_hessian_accumulate: the token chunks of each output tile are added in
+  chunk order (a turnstile), not by atomics, so H repeats bit for bit.
 - gptq_cholesky_inverse: the look-ahead splits each panel's trailing update
   into a near part (caller's stream) and a far part (side stream), but every
   element still receives the panels' updates in panel order, each once per
@@ -25,8 +27,11 @@ def test_cholesky_inverse_is_repeatable(n, actorder):
     H = torch.zeros(n, n, device="cuda")
     G.gptq_hessian_accumulate(H, X)
     outs = []
-    for _ in range(3):
-        U, perm, dead, info = G.gptq_cholesky_inverse(H, 0.01, actorder)
+    side = torch.cuda.Stream()
+    for k in range(4):
+        # three runs with the look-ahead on a side stream, one without
+        U, perm, dead, info = G.gptq_cholesky_inverse(H, 0.01, actorder,
+                                                      side_stream=side if k < 3 else None)
         torch.cuda.synchronize()
         assert int(info.item()) == 0
         outs.append((U.clone(), perm.clone()))
@@ -50,3 +55,47 @@ def test_dequant_matvec_is_repeatable(bits, rows, n, g, batch):
     torch.cuda.synchronize()
     for y in ys[1:]:
         assert torch.equal(y, ys[0])
+
+
+@pytest.mark.parametrize("n,ntok", [(512, 65536), (200, 20000), (2048, 32768)])
+def test_hessian_is_repeatable_with_split_tokens(n, ntok):
+    """The tokens are cut into chunks (several units per output tile); the
+    chunks of a tile are added into H in chunk order, so H repeats bit for
+    bit.  fp32 X (three products per launch) as well."""
+    g = torch.Generator(device="cuda").manual_seed(n + ntok)
+    X = torch.randn(n, ntok, generator=g, device="cuda").to(torch.bfloat16)
+    Hs = []
+    for _ in range(3):
+        H = torch.zeros(n, n, device="cuda")
+        G.gptq_hessian_accumulate(H, X)
+        Hs.append(H)
+    Xf = torch.randn(n, 4096, generator=g, device="cuda")
+    for _ in range(2):
+        H = torch.zeros(n, n, device="cuda")
+        G.gptq_hessian_accumulate(H, Xf)
+        Hs.append(H)
+    torch.cuda.synchronize()
+    assert torch.equal(Hs[1], Hs[0]) and torch.equal(Hs[2], Hs[0])
+    assert torch.equal(Hs[4], Hs[3])
+
+
+def test_whole_layer_is_repeatable():
+    """LayerQuantizer.run three times on the bench layer's shape (smaller
+    token count): H, U, codes, rulers and the packed words are identical,
+    with and without the look-ahead streams."""
+    rows, n, ntok = 4096, 4096, 32768
+    g = torch.Generator(device="cuda").manual_seed(11)
+    X = torch.randn(n, ntok, generator=g, device="cuda").to(torch.bfloat16)
+    W = (torch.randn(rows, n, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    outs = []
+    for look in (True, True, True, False):
+        lq = G.LayerQuantizer(rows, n, ntok, 4, 128, 0.01, True, lookahead=look)
+        lq.run(W, X)
+        torch.cuda.synchronize()
+        lq.check_info()
+        outs.append({k: getattr(lq, k).clone() for k in
+                     ("H", "U", "perm", "codes", "scales", "zeros", "packed")})
+        del lq
+    for o in outs[1:]:
+        for k, v in o.items():
+            assert torch.equal(v, outs[0][k]), k
