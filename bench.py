@@ -32,6 +32,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+SYRK_REV = "syrk-pair-v2-ordered"   # the SYRK kernel the committed traffic figure belongs to
 METRIC = "weights quantized/sec (GPTQ 4-bit g128) + Hessian TFLOP/s, % of roofline, 1×B200"
 UNIT = "weights/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -50,6 +51,10 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-next", action="store_true",
                    help="skip the measurements of the consumer-side kernels")
+    p.add_argument("--no-extra", action="store_true",
+                   help="skip the short runs of the other large workloads")
+    p.add_argument("--no-lookahead", action="store_true",
+                   help="run the factorisation and the sweep on one stream")
     p.add_argument("--only", choices=["dequant_matvec", "hadamard", "pipeline"], default=None,
                    help="run one consumer-side measurement alone and print its JSON "
                         "(for profiling; not the benchmark line)")
@@ -448,6 +453,125 @@ def measure_pipeline(G, dev, reps=3):
     return res
 
 
+# ----------------------------------------------------------------- per-stage rooflines
+def fp32_accurate_peak(pk) -> float:
+    """TFLOP/s of fp32-accurate products on the tensor cores: the measured
+    bf16 dense rate halved (TF32 runs at half the bf16 rate) and divided by
+    the three TF32 products of the hi/lo split."""
+    return pk["bf16_tflops"] / 2.0 / 3.0
+
+
+def stage_rooflines(wl, stage_ms: dict, pk) -> dict:
+    """Roofline of every stage after the Hessian, from its CUDA-event time.
+
+    S3 (Cholesky + triangular inverse): n^3/3 + n^3/3 flops against the
+    fp32-accurate tensor peak.  S5-S6 (sweep + lazy updates): rows n^2 flops
+    against the same peak, and its bytes (W read as stored, the upper half of
+    U, the packed codes and the rulers) against HBM; the bound is the larger
+    of the two times.  S7 (pack) and S8 (dequant): bytes against HBM."""
+    rows, n, b = wl.rows, wl.n, wl.bits
+    G = 1 if wl.group_size <= 0 else -(-n // wl.group_size)
+    wbytes = 2 if str(wl.w_dtype).endswith("bfloat16") else 4
+    pf = fp32_accurate_peak(pk) * 1e12
+    hbm = pk["hbm_gbs"] * 1e9
+    out = {"fp32_accurate_peak_tflops": round(pf / 1e12, 1),
+           "fp32_accurate_peak_source": f"{pk['_source']} bf16 burst / 2 (TF32) / 3 (products)"}
+    f3 = 2.0 * n ** 3 / 3.0
+    t3 = stage_ms["cholesky_inverse"] / 1e3
+    out["cholesky_inverse"] = {"bound": "tensor", "algorithmic_flops": f3,
+                               "achieved_tflops": round(f3 / t3 / 1e12, 2),
+                               "frac": round((f3 / pf) / t3, 4), "ms": round(t3 * 1e3, 4)}
+    f56 = float(rows) * n * n
+    b56 = rows * n * wbytes + 2.0 * n * n + rows * n * b / 8.0 + rows * G * 5.0
+    t56 = stage_ms["sweep"] / 1e3
+    tf, tb = f56 / pf, b56 / hbm
+    out["sweep"] = {"bound": "tensor" if tf >= tb else "hbm", "algorithmic_flops": f56,
+                    "algorithmic_bytes": b56, "achieved_tflops": round(f56 / t56 / 1e12, 2),
+                    "achieved_gbs": round(b56 / t56 / 1e9, 1),
+                    "frac": round(max(tf, tb) / t56, 4), "ms": round(t56 * 1e3, 4)}
+    b7 = rows * n * (1 + b / 8.0)
+    t7 = stage_ms["pack"] / 1e3
+    out["pack"] = {"bound": "hbm", "algorithmic_bytes": b7, "achieved_gbs": round(b7 / t7 / 1e9, 1),
+                   "frac": round((b7 / hbm) / t7, 4), "ms": round(t7 * 1e3, 4)}
+    b8 = rows * n * (b / 8.0 + 2) + rows * G * 5.0
+    t8 = stage_ms["dequant"] / 1e3
+    out["dequant"] = {"bound": "hbm", "algorithmic_bytes": b8,
+                      "achieved_gbs": round(b8 / t8 / 1e9, 1),
+                      "frac": round((b8 / hbm) / t8, 4), "ms": round(t8 * 1e3, 4)}
+    return out
+
+
+def measure_layer(G, wl, dev, steps, warmup, stream, lookahead=True, clock=None, world=1,
+                  barrier=None):
+    """The timed loop of one workload: `warmup` untimed steps, then `steps`
+    steps bracketed by CUDA events on `stream`, per-stage events inside every
+    step.  Returns (LayerQuantizer, W, X, dict of timings)."""
+    import torch
+    import workloads
+    W, X = workloads.make_inputs(wl, device=dev)
+    lq = G.LayerQuantizer(wl.rows, wl.n, wl.ntok, wl.bits, wl.group_size, wl.percdamp,
+                          wl.actorder, x_dtype=X.dtype, w_dtype=W.dtype,
+                          out_dtype=torch.bfloat16, device=dev, lookahead=lookahead)
+    for _ in range(warmup):
+        lq.run(W, X, stream=stream)
+    torch.cuda.synchronize()
+    lq.check_info()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    launches0 = G.gptq_launch_count()
+    import contextlib
+    with (clock if clock is not None else contextlib.nullcontext()):
+        t0.record(stream)
+        for k in range(steps):
+            lq.run(W, X, stream=stream, events=evs[k])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    lq.check_info()
+    launches = G.gptq_launch_count() - launches0
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    names = list(G.LayerQuantizer.STAGES)
+    stage = {nm: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+             for i, nm in enumerate(names)}
+    return lq, W, X, {"ms": ms, "stage_ms": stage, "launches": launches}
+
+
+def extra_workload(G, name, dev, stream, steps=3, warmup=2):
+    """A short driver-observed run of another large workload: weights/s,
+    Hessian TFLOP/s against the measured bf16 peak, per-stage times and
+    rooflines."""
+    import torch
+    import workloads
+    wl = workloads.WORKLOADS[name]
+    torch.cuda.empty_cache()
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    clk = ClockSampler(dev.index or 0, uuid)
+    lq, W, X, t = measure_layer(G, wl, dev, steps, warmup, stream, clock=clk)
+    pk = peaks()
+    flops = float(wl.n) * (wl.n + 1) * wl.ntok
+    th = t["stage_ms"]["hessian"] / 1e3
+    res = {"workload": describe(wl), "steps": steps, "warmup": warmup,
+           "ms_per_step": round(t["ms"] / steps, 3),
+           "weights_per_s": wl.rows * wl.n * steps / (t["ms"] / 1e3),
+           "hessian_tflops": round(flops / th / 1e12, 1),
+           "hessian_frac_of_bf16_peak": round(flops / th / 1e12 / pk["bf16_tflops"], 4),
+           "stage_ms": {k: round(v, 4) for k, v in t["stage_ms"].items()},
+           "roofline_stages": stage_rooflines(wl, t["stage_ms"], pk),
+           "gpu_launches": t["launches"], "clocks": clk.summary()}
+    del lq, W, X
+    torch.cuda.empty_cache()
+    return res
+
+
 # ----------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -459,47 +583,23 @@ def run_ours(args, rank, world, local_rank):
     if args.tokens:
         wl = dataclasses.replace(wl, ntok=args.tokens)
     dev = torch.device("cuda", local_rank)
-    W, X = workloads.make_inputs(wl, device=dev)
     rows, n, N = wl.rows, wl.n, wl.ntok
-    lq = G.LayerQuantizer(rows, n, N, wl.bits, wl.group_size, wl.percdamp, wl.actorder,
-                          x_dtype=X.dtype, w_dtype=W.dtype, out_dtype=torch.bfloat16,
-                          device=dev)
     stream = torch.cuda.current_stream()
-
-    def step(ev=None):
-        lq.run(W, X, stream=stream, events=ev)
 
     def barrier():
         if world > 1:
             torch.distributed.barrier()
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    lq.check_info()
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    launches0 = G.gptq_launch_count()
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:
         uuid = None
-    with ClockSampler(local_rank, uuid) as clk:
-        t_start.record(stream)
-        for k in range(args.steps):
-            step(evs[k])
-        t_end.record(stream)
-        torch.cuda.synchronize()
-    barrier()
-    launches = G.gptq_launch_count() - launches0
-    ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
-    names = list(G.LayerQuantizer.STAGES)
-    stage = {nm: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
-             for i, nm in enumerate(names)}
+    clk = ClockSampler(local_rank, uuid)
+    lq, W, X, t = measure_layer(G, wl, dev, args.steps, args.warmup, stream,
+                                lookahead=not args.no_lookahead, clock=clk, world=world,
+                                barrier=barrier)
+    ms, stage, launches = t["ms"], t["stage_ms"], t["launches"]
+    x_gb = X.numel() * X.element_size() / 1e9
     ms_step = ms / args.steps
     value = job_throughput(world, rows * n, args.steps, ms)
     flops = float(n) * (n + 1) * N
@@ -511,7 +611,7 @@ def run_ours(args, rank, world, local_rank):
     if os.path.exists(tf_path):
         with open(tf_path) as f:
             tj = json.load(f)
-        if tj.get("workload") == wl.name and tj.get("kernel_rev") == "syrk-pair-v1":
+        if tj.get("workload") == wl.name and tj.get("kernel_rev") == SYRK_REV:
             traffic = tj.get("bytes_per_launch")
     roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_tflops"],
             "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": traffic,
@@ -519,8 +619,8 @@ def run_ours(args, rank, world, local_rank):
             "peak_source": f"{pk['_source']} bf16 burst", "algorithmic_flops": flops,
             "frac_of_sustained_peak": round(
                 achieved / pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]),
-                4),
-            "gemm_equivalent_tflops": round(2.0 * n * n * N / t_h / 1e12, 2)}
+                4)}
+    roof_stages = stage_rooflines(wl, stage, pk)
 
     # the consumer of the packed codes (fused dequant x activation), outside
     # the timed step: on this layer's own output, and on the 70B down-proj
@@ -584,9 +684,21 @@ def run_ours(args, rank, world, local_rank):
                "ms_per_step": ems / args.steps}
         del Xh, Wh, Xd, Wd
 
+    # short driver-observed runs of the other large workloads (3-bit 7B
+    # down-proj; the rotated 70B down-proj), after this layer's buffers are freed
+    extra = None
+    if rank == 0 and world == 1 and not args.no_extra and args.workload == "q_proj_7b" \
+            and not args.tokens:
+        Wc, Xc = W.cpu(), X[:, :8192].cpu()  # what the CPU baseline below reads
+        del lq, W, X
+        torch.cuda.empty_cache()
+        extra = {name: extra_workload(G, name, dev, stream)
+                 for name in ("down_proj_7b", "down_proj_70b")}
+        W, X = Wc, Xc
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, desc, _ = cpu_sample(wl, W, X, tok_sample=4096, row_sample=64)
+        v, desc, _ = cpu_sample(wl, W, X, **CPU_SAMPLE)
         cpu = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                "sample": desc}
 
@@ -598,40 +710,52 @@ def run_ours(args, rank, world, local_rank):
             "dtype": "bf16 in / f32", "data": "synthetic",
             "config": {"workload": describe(wl), "rows": rows, "n": n, "tokens": N,
                        "bits": wl.bits, "group_size": wl.group_size, "actorder": wl.actorder,
-                       "l2": "inputs larger than L2 (X is %.2f GB)" % (X.numel() * 2 / 1e9),
+                       "l2": "inputs larger than L2 (X is %.2f GB)" % x_gb,
                        "parallelism": f"{world} independent replicas"},
             "hessian_tflops": achieved,
             "stage_ms": {k: round(v, 4) for k, v in stage.items()},
             "roofline": roof,
+            "roofline_stages": roof_stages,
+            "extra_workloads": extra,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clk.summary(),
+            "lookahead": not args.no_lookahead,
             "next": nxt,
         }
         print(json.dumps(line), flush=True)
 
 
 # ----------------------------------------------------------------- reference arm
+CPU_SAMPLE = {"tok_sample": 4096, "row_sample": 64}   # both CPU legs time this sample
+
+
 def run_reference(args, rank, world):
+    """The fp64 oracle on the host cores, one bounded sample of the workload
+    per step (cpu_sample); value = the layer's weights over the layer time
+    extrapolated from the sample, ms_per_step = the measured time of one
+    sample (what the driver's clock sees)."""
     if rank != 0:
         return
-    import torch
     import workloads
 
     wl = workloads.WORKLOADS[args.workload]
-    W = workloads.make_weights(wl, "cpu", rows=16)
-    X = workloads.make_calibration(wl, "cpu", ntok=2048)
-    times = []
+    W = workloads.make_weights(wl, "cpu", rows=CPU_SAMPLE["row_sample"])
+    X = workloads.make_calibration(wl, "cpu", ntok=CPU_SAMPLE["tok_sample"])
+    layer_s, wall_s = [], []
     desc = ""
     for i in range(args.warmup + args.steps):
-        v, desc, _ = cpu_sample(wl, W, X, tok_sample=2048, row_sample=16)
+        v, desc, spent = cpu_sample(wl, W, X, **CPU_SAMPLE)
         if i >= args.warmup:
-            times.append(wl.rows * wl.n / v)
-    t = statistics.mean(times)
-    value = wl.rows * wl.n / t
+            layer_s.append(wl.rows * wl.n / v)
+            wall_s.append(spent)
+    t_layer = statistics.mean(layer_s)
+    value = wl.rows * wl.n / t_layer
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": statistics.mean(wall_s) * 1e3,
+            "extrapolated_layer_s": t_layer,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
             "config": {"workload": describe(wl), "rows": wl.rows, "n": wl.n,
