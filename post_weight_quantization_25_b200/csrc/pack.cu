@@ -426,7 +426,11 @@ __global__ void __launch_bounds__(256) gather_columns_u8_kernel(const uint8_t* _
 //               group's scale applies to its own partial sum.
 // From word w (8 codes, column 8 wj + i of the block in bits 4i..4i+3) the
 // k-slots are paired as (i, i + 4): ((w >> 4i) & 0x000F000F) | 0x43004300 is
-// the bf16 pair (128 + q_i, 128 + q_{i+4}).  A prep kernel writes x once per
+// the bf16 pair (128 + q_i, 128 + q_{i+4}): OR-ing a small integer into the
+// mantissa of a power of two and subtracting that power is the classic
+// "magic number" integer-to-float conversion (for int4 / int8 weights on GPUs
+// it is described in Kim et al., "Who Says Elephants Can't Run: Bringing Large
+// Scale MoE Models into Cloud Scale Production", 2022).  A prep kernel writes x once per
 // call in that pairing (and in sweep order when a perm is given), so the MMA
 // B fragments load straight from it, and zeroes y.
 

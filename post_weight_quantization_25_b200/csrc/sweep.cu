@@ -63,18 +63,53 @@ struct SweepWs {
 
 int64_t ut_ld(int64_t n) { return (n + 3) / 4 * 4; }
 
-SweepWs carve(void* ws, int64_t rows, int64_t n) {
+// Layers narrower than the two-level width, with rows 16-byte aligned, are
+// swept by the persistent kernel, which keeps every block's err terms.
+bool use_persistent(int64_t n) { return n > kBlock && n < kTwoLevelMinN && n % 4 == 0; }
+int64_t persist_lde(int64_t n) { return (n + kBlock - 1) / kBlock * kBlock; }
+size_t persist_ctr_bytes(int64_t rows, int64_t n) {
+  const int64_t RB = (rows + kBlock - 1) / kBlock, nb = persist_lde(n) / kBlock;
+  return align_up(sizeof(uint32_t) * (size_t)(1 + RB + RB * nb), 256);
+}
+// bytes of the err-term region: two super-blocks (hi and lo) or, for the
+// persistent sweep, every block (hi and lo)
+size_t err_region_bytes(int64_t rows, int64_t n) {
+  const size_t two = 4 * align_up(sizeof(float) * rows * super_cols(n), 256);
+  const size_t all = use_persistent(n) ? 2 * align_up(sizeof(float) * rows * persist_lde(n), 256)
+                                       : 0;
+  return std::max(two, all);
+}
+
+struct SweepWsExtra {
+  uint32_t* ctr;  // counters of the persistent sweep
+};
+
+// S: the super-block width in use (at most super_cols(n), which sizes the
+// workspace); persist: the err terms of every block instead of two super-blocks
+SweepWs carve(void* ws, int64_t rows, int64_t n, int64_t S, bool persist = false,
+              SweepWsExtra* extra = nullptr) {
   char* p = static_cast<char*>(ws);
   SweepWs w;
   w.Wf = reinterpret_cast<float*>(p);
   p += align_up(sizeof(float) * rows * n, 256);
-  w.lde = super_cols(n);
-  for (int b = 0; b < 2; ++b) {
-    w.Err_hi[b] = reinterpret_cast<float*>(p);
-    p += align_up(sizeof(float) * rows * w.lde, 256);
-    w.Err_lo[b] = reinterpret_cast<float*>(p);
-    p += align_up(sizeof(float) * rows * w.lde, 256);
+  char* err = p;
+  if (persist) {
+    w.lde = persist_lde(n);
+    w.Err_hi[0] = w.Err_hi[1] = reinterpret_cast<float*>(err);
+    w.Err_lo[0] = w.Err_lo[1] =
+        reinterpret_cast<float*>(err + align_up(sizeof(float) * rows * w.lde, 256));
+  } else {
+    w.lde = S;
+    for (int b = 0; b < 2; ++b) {
+      w.Err_hi[b] = reinterpret_cast<float*>(p);
+      p += align_up(sizeof(float) * rows * w.lde, 256);
+      w.Err_lo[b] = reinterpret_cast<float*>(p);
+      p += align_up(sizeof(float) * rows * w.lde, 256);
+    }
   }
+  p = err + err_region_bytes(rows, n);
+  if (extra) extra->ctr = reinterpret_cast<uint32_t*>(p);
+  p += use_persistent(n) ? persist_ctr_bytes(rows, n) : 0;
   w.codes_sw = reinterpret_cast<uint8_t*>(p);
   p += align_up((size_t)rows * n, 256);
   w.pos = reinterpret_cast<int32_t*>(p);
@@ -273,8 +308,11 @@ constexpr int kSweepRows = kSweepThreads / kSweepLanes; // rows per CTA
 constexpr int kSub = 16;                                // columns per unrolled sub-block
 constexpr int kSubSlots = kSub / kSweepLanes;           // columns per lane in a sub-block
 constexpr int kWbPitch = 132;                           // floats per row of the staged W block
+constexpr int kCbPitch = kBlock + 16;                   // bytes per row of the staged codes
+// Ud [128][128] | Wb, Eb [32][kWbPitch] | rd, hrd2 [128] | Cb [32][kCbPitch] (bytes)
 constexpr size_t kSweepSmemBytes =
-    sizeof(float) * (kBlock * kBlock + kSweepRows * kWbPitch + 2 * kBlock);
+    sizeof(float) * (kBlock * kBlock + 2 * kSweepRows * kWbPitch + 2 * kBlock) +
+    kSweepRows * kCbPitch;
 
 __device__ __forceinline__ float team_min(float v) {
 #pragma unroll
@@ -287,30 +325,49 @@ __device__ __forceinline__ float team_max(float v) {
   return v;
 }
 
+// Issues (does not wait for) the 16-byte async copies of U's diagonal block
+// [i1, i1 + 128)^2 into the body's Ud (n a multiple of 4; 0 past bsz).
+__device__ __forceinline__ void sweep_stage_u(float* smem, int tid, const float* __restrict__ U,
+                                              int n, int i1, int bsz) {
+  const float* us = U + (int64_t)i1 * n + i1;
+  for (int f = tid; f < kBlock * kBlock / 4; f += kSweepThreads) {
+    const int a = f >> 5, c = (f & 31) * 4;
+    const bool ok = a < bsz && c < bsz;
+    ptx::cp_async_16z(smem + a * kBlock + c, ok ? us + (int64_t)a * n + c : us, ok ? 16 : 0);
+  }
+}
+
+// The sweep of one block by threads 0 .. kSweepThreads - 1 of a CTA, for
+// rows [r0, r0 + kSweepRows): `smem` holds kSweepSmemBytes, `bar` is the
+// barrier they synchronise on (0: __syncthreads, else a named barrier of
+// kSweepThreads threads).  Shared by the one-block kernel and the persistent
+// sweep; the latter issues the copies of U's block itself (u_issued, n a
+// multiple of 4) before it waits for the block's columns to be up to date.
 template <int GS>
-__global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
-    float* __restrict__ Wf, int rows, int n, const float* __restrict__ U, int i1, int bsz,
-    float maxq, int sym, int gsize, int G, float* __restrict__ Err_hi, float* __restrict__ Err_lo,
-    int lde, uint8_t* __restrict__ codes_sw, float* __restrict__ scales,
-    uint8_t* __restrict__ zeros, float* __restrict__ row_loss) {
+__device__ __forceinline__ void sweep_block_body(
+    float* smem, int tid, int r0, int bar, float* __restrict__ Wf, int rows, int n,
+    const float* __restrict__ U, int i1, int bsz, float maxq, int sym, int gsize, int G,
+    float* __restrict__ Err_hi, float* __restrict__ Err_lo, int lde,
+    uint8_t* __restrict__ codes_sw, float* __restrict__ scales, uint8_t* __restrict__ zeros,
+    float* __restrict__ row_loss, bool u_issued = false) {
   constexpr int L = kSweepLanes, NS = kSubSlots;
-  extern __shared__ __align__(16) float smem[];
+  auto sync = [bar]() {
+    if (bar == 0)
+      __syncthreads();
+    else
+      ptx::named_bar_sync(bar, kSweepThreads);
+  };
   float* Ud = smem;                       // [128][128]  U[i1 + a][i1 + b], 0 past bsz
-  float* Wb = Ud + kBlock * kBlock;       // [32][kWbPitch]  this CTA's rows of the block
-  float* rd = Wb + kSweepRows * kWbPitch; // [128]  1 / U_jj
+  float* Wb = Ud + kBlock * kBlock;       // [32][kWbPitch]  this CTA's rows of the block; w_hat
+  float* Eb = Wb + kSweepRows * kWbPitch; // [32][kWbPitch]  their error terms
+  float* rd = Eb + kSweepRows * kWbPitch; // [128]  1 / U_jj
   float* hrd2 = rd + kBlock;              // [128]  1 / (2 U_jj^2)
-  const int tid = threadIdx.x;
-  const int r0 = blockIdx.x * kSweepRows;
+  uint8_t* Cb = reinterpret_cast<uint8_t*>(hrd2 + kBlock);  // [32][kCbPitch]  their codes
   const int vr = min(kSweepRows, rows - r0);
   if ((n % 4) == 0) {
     // 16-byte async copies, all in flight at once; bsz is a multiple of 4 here
-    const float* us = U + (int64_t)i1 * n + i1;
     const float* ws = Wf + (int64_t)r0 * n + i1;
-    for (int f = tid; f < kBlock * kBlock / 4; f += kSweepThreads) {
-      const int a = f >> 5, c = (f & 31) * 4;
-      const bool ok = a < bsz && c < bsz;
-      ptx::cp_async_16z(Ud + a * kBlock + c, ok ? us + (int64_t)a * n + c : us, ok ? 16 : 0);
-    }
+    if (!u_issued) sweep_stage_u(smem, tid, U, n, i1, bsz);
     for (int f = tid; f < kSweepRows * kBlock / 4; f += kSweepThreads) {
       const int a = f >> 5, c = (f & 31) * 4;
       const bool ok = a < vr && c < bsz;
@@ -326,13 +383,13 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
       Wb[a * kWbPitch + c] = (a < vr && c < bsz) ? Wf[(int64_t)(r0 + a) * n + i1 + c] : 0.f;
     }
   }
-  __syncthreads();
+  sync();
   for (int i = tid; i < kBlock; i += kSweepThreads) {
     const float d = (i < bsz) ? Ud[i * kBlock + i] : 1.f;
     rd[i] = 1.f / d;
     hrd2[i] = 0.5f / (d * d);
   }
-  __syncthreads();
+  sync();
 
   const int lane = tid & 31;
   const int q = lane % L;                 // lane within the team
@@ -375,10 +432,8 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
   // once per ruler (Markstein's method, fdiv.cuh)
   MDiv md = md_prepare(scale);
   float loss = 0.f;
-  float* wg = Wf + (int64_t)(active ? r : 0) * n + i1;
-  uint8_t* cg = codes_sw + (int64_t)(active ? r : 0) * n + i1;
-  float* ehi = Err_hi + (int64_t)(active ? r : 0) * lde;
-  float* elo = Err_lo + (int64_t)(active ? r : 0) * lde;
+  float* erow = Eb + rl * kWbPitch;
+  uint8_t* crow = Cb + rl * kCbPitch;
 
 #pragma unroll 1
   for (int c0 = 0; c0 < kBlock; c0 += kSub) {
@@ -434,43 +489,526 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
       for (int s2 = s; s2 < NS; ++s2)
         if (s2 > s || q > ko) cur[s2] = fmaf(-err, urow[L * s2 + q], cur[s2]);
     }
-    // the sub-block's results: w_hat into Wf, codes, error terms (TF32 split)
-    if (active) {
+    // the sub-block's results, staged for the block's coalesced write-out:
+    // w_hat in place of the columns just swept (no later step reads them),
+    // the error terms and the codes
 #pragma unroll
-      for (int s = 0; s < NS; ++s) {
-        const int c = c0 + L * s + q;
-        if (c < bsz) {
-          wg[c] = cur[s];
-          cg[c] = (uint8_t)((cw >> (8 * s)) & 0xFFu);
-        }
-        float h, l;
-        tf32_split(e_own[s], h, l);
-        ehi[c] = h;
-        elo[c] = l;
-      }
+    for (int s = 0; s < NS; ++s) {
+      const int c = c0 + L * s + q;
+      wrow[c] = cur[s];
+      erow[c] = e_own[s];
+      crow[c] = (uint8_t)((cw >> (8 * s)) & 0xFFu);
     }
     // rank-16 update of the block's later columns (shared memory), lane q
-    // taking the 4-column chunks q, q + L, ...
-#pragma unroll 1
-    for (int c = c0 + kSub + 4 * q; c < kBlock; c += 4 * L) {
-      float4 w4 = *reinterpret_cast<const float4*>(wrow + c);
-      const float* ucol = Ud + c0 * kBlock + c;
+    // taking the 4-column chunks q, q + L, ...; all of a lane's chunks are
+    // held in registers and updated together, step j by step j, so their
+    // FMA chains run side by side
+    constexpr int kMaxChunks = (kBlock - kSub) / (4 * L);
+    const int nch = (kBlock - c0 - kSub) / (4 * L);   // the same for every lane
+    float* wch = wrow + c0 + kSub + 4 * q;
+    float4 w4[kMaxChunks];
 #pragma unroll
-      for (int j = 0; j < kSub; ++j) {
-        const float4 u = *reinterpret_cast<const float4*>(ucol + j * kBlock);
-        w4.x = fmaf(-ev_sub[j], u.x, w4.x);
-        w4.y = fmaf(-ev_sub[j], u.y, w4.y);
-        w4.z = fmaf(-ev_sub[j], u.z, w4.z);
-        w4.w = fmaf(-ev_sub[j], u.w, w4.w);
+    for (int i = 0; i < kMaxChunks; ++i)
+      if (i < nch) w4[i] = *reinterpret_cast<const float4*>(wch + 4 * L * i);
+#pragma unroll
+    for (int j = 0; j < kSub; ++j) {
+      const float ne = -ev_sub[j];
+      const float* urow = Ud + (c0 + j) * kBlock + c0 + kSub + 4 * q;
+#pragma unroll
+      for (int i = 0; i < kMaxChunks; ++i) {
+        if (i < nch) {
+          const float4 u = *reinterpret_cast<const float4*>(urow + 4 * L * i);
+          w4[i].x = fmaf(ne, u.x, w4[i].x);
+          w4[i].y = fmaf(ne, u.y, w4[i].y);
+          w4[i].z = fmaf(ne, u.z, w4[i].z);
+          w4[i].w = fmaf(ne, u.w, w4[i].w);
+        }
       }
-      *reinterpret_cast<float4*>(wrow + c) = w4;
     }
+#pragma unroll
+    for (int i = 0; i < kMaxChunks; ++i)
+      if (i < nch) *reinterpret_cast<float4*>(wch + 4 * L * i) = w4[i];
     __syncwarp();  // the team's chunk writes land before the next sub-block's loads
   }
   if (row_loss) {
 #pragma unroll
     for (int o = 1; o < L; o <<= 1) loss += __shfl_xor_sync(0xffffffffu, loss, o);
     if (active && q == 0) row_loss[r] += loss;
+  }
+  // write-out, whole row segments at a time: w_hat into Wf and the codes
+  // (columns < bsz), the error terms split into TF32 part and remainder
+  // (all 128 columns; those past bsz are 0)
+  sync();
+  for (int f = tid; f < kSweepRows * (kBlock / 4); f += kSweepThreads) {
+    const int a = f / (kBlock / 4), c = (f % (kBlock / 4)) * 4;
+    if (a >= vr) continue;
+    const float4 e4 = *reinterpret_cast<const float4*>(Eb + a * kWbPitch + c);
+    float4 h4, l4;
+    tf32_split(e4.x, h4.x, l4.x);
+    tf32_split(e4.y, h4.y, l4.y);
+    tf32_split(e4.z, h4.z, l4.z);
+    tf32_split(e4.w, h4.w, l4.w);
+    *reinterpret_cast<float4*>(Err_hi + (int64_t)(r0 + a) * lde + c) = h4;
+    *reinterpret_cast<float4*>(Err_lo + (int64_t)(r0 + a) * lde + c) = l4;
+    const float* wsrc = Wb + a * kWbPitch + c;
+    float* wdst = Wf + (int64_t)(r0 + a) * n + i1 + c;
+    if ((n % 4) == 0 && c + 4 <= bsz) {
+      *reinterpret_cast<float4*>(wdst) = *reinterpret_cast<const float4*>(wsrc);
+    } else {
+      for (int i = 0; i < 4 && c + i < bsz; ++i) wdst[i] = wsrc[i];
+    }
+  }
+  for (int f = tid; f < kSweepRows * (kBlock / 16); f += kSweepThreads) {
+    const int a = f / (kBlock / 16), c = (f % (kBlock / 16)) * 16;
+    if (a >= vr) continue;
+    const uint8_t* csrc = Cb + a * kCbPitch + c;
+    uint8_t* cdst = codes_sw + (int64_t)(r0 + a) * n + i1 + c;
+    if ((n % 16) == 0 && c + 16 <= bsz) {
+      *reinterpret_cast<uint4*>(cdst) = *reinterpret_cast<const uint4*>(csrc);
+    } else {
+      for (int i = 0; i < 16 && c + i < bsz; ++i) cdst[i] = csrc[i];
+    }
+  }
+}
+
+template <int GS>
+__global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(
+    float* __restrict__ Wf, int rows, int n, const float* __restrict__ U, int i1, int bsz,
+    float maxq, int sym, int gsize, int G, float* __restrict__ Err_hi, float* __restrict__ Err_lo,
+    int lde, uint8_t* __restrict__ codes_sw, float* __restrict__ scales,
+    uint8_t* __restrict__ zeros, float* __restrict__ row_loss) {
+  extern __shared__ __align__(16) float smem[];
+  sweep_block_body<GS>(smem, threadIdx.x, blockIdx.x * kSweepRows, 0, Wf, rows, n, U, i1, bsz,
+                       maxq, sym, gsize, G, Err_hi, Err_lo, lde, codes_sw, scales, zeros,
+                       row_loss);
+}
+
+// ===========================================================================
+// The persistent sweep (layers narrower than the two-level width): one
+// launch runs every block's sweep and every lazy update of a layer.
+//
+// The columns of block b's err terms go to the later 128-column tiles in two
+// parts: the "near" tiles [b + 1, b + 1 + nw(b)) -- the next block, or the
+// whole next group when a group ruler wider than a block starts there -- and
+// the "far" tiles past them.  One CTA per SM takes tasks from a global
+// counter in a fixed order in which every task comes after the tasks it
+// depends on (so a CTA that waits, waits for a task some running CTA has
+// already taken, and the waits end).  For each block s:
+//   S(R, h, s)   the sweep of block s for 64 rows (half h of 128-row block R),
+//                two 32-row slices at once on the CTA's first 256 threads
+//   F(s - 1)     the far update by block s - 1 (chunks of up to kSpChunk
+//                tiles), which runs on the SMs the sweep leaves free
+//   N(s)         the near update by block s
+// A 128-row block R keeps two kinds of counters in global memory: sweep
+// tasks done (kSpSlices per block) and, per tile, blocks applied.  S(R, ., s)
+// waits until tile s (and, at the start of a group wider than a block, every
+// tile of the group) has received blocks 0 .. s - 1; an update by block b of
+// tile c waits until block b is swept for all of R's rows and tile c has
+// received blocks 0 .. b - 1.  So every tile gets its updates in block order
+// and the result is the same bit for bit as the launch-by-launch form.
+// Updates are the panel GEMM's rank-128 step on the tensor cores (P = the
+// block's err terms, Q = U^T, C = Wf by TMA reduce-add).  All waits are
+// bounded; writes are published with release stores after the proxy and
+// memory fences, and read after acquire loads and a proxy fence.
+// ===========================================================================
+constexpr int kSpGroups = 2;                    // 32-row slices a sweep task runs at once
+constexpr int kSpSlices = kBlock / (kSweepRows * kSpGroups);  // sweep tasks per row block, block
+constexpr int kSpChunk = 4;                     // tiles per update task at most
+static_assert(kSweepSmemBytes % 16 == 0 &&
+                  kSpGroups * kSweepSmemBytes <= pg2_smem_bytes(true) - 1024 - 256,
+              "a sweep task's slices reuse the update's shared memory");
+static_assert(kSpGroups * kSweepThreads <= kPg2Threads, "one 128-thread group per slice");
+
+struct SweepPersistArgs {
+  float* Wf;
+  int rows, n;
+  const float* U;
+  float maxq;
+  int sym, gsize, G;
+  int gw;     // tiles of a group ruler wider than a block (else 1)
+  float* Eh;  // rows x lde: every block's err terms, TF32 part
+  float* El;  // remainder
+  int lde;
+  uint8_t* codes_sw;
+  float* scales;
+  uint8_t* zeros;
+  float* row_loss;
+  uint32_t* ctr;  // [0] next task, [1 + R] sweep tasks done, [1 + RB + R nb + c] blocks applied
+  int RB, nb;
+  int32_t* info;
+  const int32_t* gate;
+  uint64_t limit_ns;
+};
+
+struct SpTask {
+  int kind;  // 0 sweep, 1 update
+  int R, s;  // row block; block (sweep) or the err terms' block (update)
+  int slice;
+  int c0, c1;  // update: tiles [c0, c1)
+};
+
+// near tiles of block b: [b + 1, b + 1 + sp_near(a, b))
+__host__ __device__ inline int sp_near(const SweepPersistArgs& a, int b) {
+  const int w = (a.gw > 1 && (b + 1) % a.gw == 0) ? a.gw : 1;
+  return max(0, min(w, a.nb - b - 1));
+}
+
+struct SpStep {
+  int nS, nF, nN;  // tasks per 128-row block of each kind
+  int fs;          // first far tile of block s - 1
+  int nwt;         // near tiles of block s
+};
+
+__host__ __device__ inline SpStep sp_step(const SweepPersistArgs& a, int s) {
+  SpStep st;
+  st.nS = kSpSlices;
+  st.nwt = sp_near(a, s);
+  st.nN = (st.nwt + kSpChunk - 1) / kSpChunk;
+  st.fs = a.nb;
+  st.nF = 0;
+  if (s >= 1) {
+    st.fs = s + sp_near(a, s - 1);
+    st.nF = (max(0, a.nb - st.fs) + kSpChunk - 1) / kSpChunk;
+  }
+  return st;
+}
+
+__host__ __device__ inline int sp_total(const SweepPersistArgs& a) {
+  int t = 0;
+  for (int s = 0; s < a.nb; ++s) {
+    const SpStep st = sp_step(a, s);
+    t += a.RB * (st.nS + st.nF + st.nN);
+  }
+  return t;
+}
+
+__host__ __device__ inline SpTask sp_decode(const SweepPersistArgs& a, int t) {
+  SpTask k;
+  k.slice = 0;
+  k.c0 = k.c1 = 0;
+  for (int s = 0;; ++s) {
+    const SpStep st = sp_step(a, s);
+    const int nS = a.RB * st.nS, nF = a.RB * st.nF, nN = a.RB * st.nN;
+    if (t < nS) {
+      k.kind = 0;
+      k.s = s;
+      k.R = t / kSpSlices;
+      k.slice = t % kSpSlices;
+      return k;
+    }
+    t -= nS;
+    if (t < nF + nN) {
+      int chunk, base, end;
+      k.kind = 1;
+      if (t < nF) {   // the far chunks nearest to the sweep first
+        k.R = t % a.RB;
+        chunk = t / a.RB;
+        k.s = s - 1;
+        base = st.fs;
+        end = a.nb;
+      } else {
+        t -= nF;
+        k.R = t % a.RB;
+        chunk = t / a.RB;
+        k.s = s;
+        base = s + 1;
+        end = s + 1 + st.nwt;
+      }
+      k.c0 = base + chunk * kSpChunk;
+      k.c1 = min(k.c0 + kSpChunk, end);
+      return k;
+    }
+    t -= nF + nN;
+  }
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+template <int GS>
+__global__ void __launch_bounds__(kPg2Threads, 1)
+    sweep_persist_kernel(const __grid_constant__ CUtensorMap mEh,
+                         const __grid_constant__ CUtensorMap mEl,
+                         const __grid_constant__ CUtensorMap mUh,
+                         const __grid_constant__ CUtensorMap mUl,
+                         const __grid_constant__ CUtensorMap mW, const SweepPersistArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sP = smem;
+  uint8_t* sQ = smem + kPg2PBytes;
+  uint8_t* sOut = sQ + kPg2QStages * kPg2QStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + 8 * kPg2StageOut);
+  uint64_t* pfull = bars;
+  uint64_t* pempty = bars + 1;
+  uint64_t* qfull = bars + 2;
+  uint64_t* qempty = qfull + kPg2QStages;
+  uint64_t* tfull = qempty + kPg2QStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* task_slot = abort_flag + 1;
+  constexpr uint64_t kDrainLimit = (uint64_t)kGridWaitLimitNs;
+  const uint64_t kLimit = a.limit_ns;
+  constexpr int32_t kTimeout = -2;
+  uint32_t* swept = a.ctr + 1;
+  uint32_t* applied = a.ctr + 1 + a.RB;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    ptx::mbar_init(pfull, 1);
+    ptx::mbar_init(pempty, 1);
+    for (int q = 0; q < kPg2QStages; ++q) {
+      ptx::mbar_init(&qfull[q], 1);
+      ptx::mbar_init(&qempty[q], 1);
+    }
+    for (int c = 0; c < 2; ++c) {
+      ptx::mbar_init(&tfull[c], 1);
+      ptx::mbar_init(&tempty[c], 256);
+    }
+    ptx::mbar_init(drain, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, kPg2TmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  if (tid == 0 && !ptx::gate_wait_bounded(a.gate, kLimit)) pg_abort(abort_flag, a.info, kTimeout);
+
+  // pipeline state of the update tasks, kept by the thread of each role
+  int p_loads = 0;              // producer: P blocks loaded; MMA: P blocks consumed
+  int qst = 0;                  // producer / MMA: Q ring stage
+  uint32_t qph = 0;
+  int acc = 0;                  // MMA / epilogue: TMEM accumulator
+  uint32_t aph = 0;
+  int q_last_parity[kPg2QStages] = {-1, -1};
+  int last_pempty = -1;         // MMA: parity of its last commit on pempty
+  const int total = sp_total(a);
+
+  while (true) {
+    if (tid == 0) *task_slot = (int)atomicAdd(a.ctr, 1u);
+    __syncthreads();
+    const int t = *task_slot;
+    const bool stop = *abort_flag != 0;
+    __syncthreads();
+    if (t >= total || stop) break;
+    const SpTask k = sp_decode(a, t);
+    if (k.kind == 0) {
+      // ---------------------------------------------------------------- sweep task
+      const int i1 = k.s * kBlock;
+      const int bsz = min(kBlock, a.n - i1);
+      const int grp = tid / kSweepThreads;   // slice of the task this thread sweeps
+      const int r0 = k.R * kBlock + (k.slice * kSpGroups + grp) * kSweepRows;
+      const bool mine = grp < kSpGroups && r0 < a.rows;
+      float* gsm = reinterpret_cast<float*>(smem + grp * kSweepSmemBytes);
+      // U's block does not depend on the wait: its copies go out first
+      if (mine) sweep_stage_u(gsm, tid % kSweepThreads, a.U, a.n, i1, bsz);
+      if (tid == 0) {
+        // tile s has every earlier block's update; a group wider than a
+        // block needs its other tiles as well
+        int c_hi = k.s + 1;
+        if (GS == 128 && a.gw > 1 && k.s % a.gw == 0) c_hi = min(a.nb, k.s + a.gw);
+        bool ok = true;
+        for (int c = k.s; c < c_hi && ok; ++c)
+          ok = ptx::flag_wait_bounded(&applied[k.R * a.nb + c], (uint32_t)k.s, abort_flag, kLimit);
+        if (!ok) pg_abort(abort_flag, a.info, kTimeout);
+        fence_proxy_async_global();
+      }
+      __syncthreads();
+      if (*abort_flag) {
+        ptx::cp_async_wait_all();   // this thread's copies land before the CTA leaves
+        continue;
+      }
+      if (mine) {
+        sweep_block_body<GS>(gsm, tid % kSweepThreads, r0, 1 + grp, a.Wf, a.rows, a.n, a.U, i1,
+                             bsz, a.maxq, a.sym, a.gsize, a.G, a.Eh + i1, a.El + i1, a.lde,
+                             a.codes_sw, a.scales, a.zeros, a.row_loss, /*u_issued=*/true);
+        // this thread's writes (shared memory the next task's TMA loads
+        // overwrite; Wf and the err terms other CTAs read by TMA) are ordered
+        // before the async proxy's accesses
+        asm volatile("fence.proxy.async;" ::: "memory");
+      }
+      __syncthreads();
+      if (tid == 0) {
+        __threadfence();
+        atomicAdd(&swept[k.R], 1u);
+      }
+      continue;
+    }
+    // ------------------------------------------------------------------ update task
+    PgItem I;
+    I.C0 = a.Wf + (int64_t)k.R * kBlock * a.n + (int64_t)k.c0 * kBlock;
+    I.ldc = a.n;
+    I.cmap = 0;
+    I.cx0 = k.c0 * kBlock;
+    I.cy0 = k.R * kBlock;
+    I.prow = k.R * kBlock;
+    I.pkx = k.s * kBlock;
+    I.qrow0 = k.c0 * kBlock;
+    I.qkx = k.s * kBlock;
+    I.nq = k.c1 - k.c0;
+    I.mext = min(kBlock, a.rows - k.R * kBlock);
+    I.cext_last = min(kBlock, a.n - (k.c1 - 1) * kBlock);
+    I.nkb = kPgKBlocks;
+    if (tid == 0) {
+      // block s is swept for all of R's rows, and each tile has blocks 0 .. s - 1
+      bool ok = ptx::flag_wait_bounded(&swept[k.R], (uint32_t)(kSpSlices * (k.s + 1)),
+                                       abort_flag, kLimit);
+      for (int c = k.c0; c < k.c1 && ok; ++c)
+        ok = ptx::flag_wait_bounded(&applied[k.R * a.nb + c], (uint32_t)k.s, abort_flag, kLimit);
+      if (!ok) pg_abort(abort_flag, a.info, kTimeout);
+      fence_proxy_async_global();
+    }
+    __syncthreads();
+    if (*abort_flag) continue;
+    if (warp == 0) {
+      if (lane == 0) {
+        // producer: the block's err terms (all of K = 128), then Q per tile
+        bool ok = p_loads == 0 ||
+                  ptx::mbar_wait_bounded(pempty, (uint32_t)((p_loads - 1) & 1), abort_flag, kLimit);
+        if (ok) {
+          ptx::mbar_arrive_expect_tx(pfull, kPg2PBytes);
+          for (int kb = 0; kb < kPgKBlocks; ++kb) {
+            ptx::tma_load_2d(sP + kb * 2 * kPgTileBytes, &mEh, pfull, I.pkx + 32 * kb, I.prow);
+            ptx::tma_load_2d(sP + kb * 2 * kPgTileBytes + kPgTileBytes, &mEl, pfull,
+                             I.pkx + 32 * kb, I.prow);
+          }
+          ++p_loads;
+          for (int q = 0; q < I.nq && ok; ++q)
+            for (int kb = 0; kb < kPgKBlocks; ++kb) {
+              if (!ptx::mbar_wait_bounded(&qempty[qst], qph ^ 1, abort_flag, kLimit)) {
+                ok = false;
+                break;
+              }
+              uint8_t* sb = sQ + qst * kPg2QStageBytes;
+              ptx::mbar_arrive_expect_tx(&qfull[qst], kPg2QStageBytes);
+              ptx::tma_load_2d(sb, &mUh, &qfull[qst], I.qkx + 32 * kb, I.qrow0 + 128 * q);
+              ptx::tma_load_2d(sb + kPgTileBytes, &mUl, &qfull[qst], I.qkx + 32 * kb,
+                               I.qrow0 + 128 * q);
+              q_last_parity[qst] = (int)qph;
+              if (++qst == kPg2QStages) {
+                qst = 0;
+                qph ^= 1;
+              }
+            }
+        }
+        if (!ok) {
+          pg_abort(abort_flag, a.info, kTimeout);
+          volatile int never = 0;  // this CTA's own copies in flight
+          ptx::mbar_wait_bounded(pfull, (uint32_t)((p_loads - 1) & 1), &never, kDrainLimit);
+          for (int q = 0; q < kPg2QStages; ++q)
+            if (q_last_parity[q] >= 0)
+              ptx::mbar_wait_bounded(&qfull[q], (uint32_t)q_last_parity[q], &never, kDrainLimit);
+        }
+      }
+    } else if (warp == 1) {
+      if (lane == 0) {
+        // MMA issuer
+        constexpr uint32_t idesc = ptx::idesc_tf32_f32(128, 128);
+        bool ok = ptx::mbar_wait_bounded(pfull, (uint32_t)(p_loads & 1), abort_flag, kLimit);
+        if (ok) {
+          ptx::tc_fence_after();
+          for (int q = 0; q < I.nq && ok; ++q) {
+            if (!ptx::mbar_wait_bounded(&tempty[acc], aph ^ 1, abort_flag, kLimit)) {
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t d = tmem_base + (uint32_t)(acc * 128);
+            for (int kb = 0; kb < kPgKBlocks; ++kb) {
+              if (!ptx::mbar_wait_bounded(&qfull[qst], qph, abort_flag, kLimit)) {
+                ok = false;
+                break;
+              }
+              ptx::tc_fence_after();
+              const uint32_t pb = ptx::smem_u32(sP + kb * 2 * kPgTileBytes);
+              const uint32_t qb = ptx::smem_u32(sQ + qst * kPg2QStageBytes);
+              const uint64_t ph = ptx::smem_desc_sw128(pb);
+              const uint64_t pl = ptx::smem_desc_sw128(pb + kPgTileBytes);
+              const uint64_t qh = ptx::smem_desc_sw128(qb);
+              const uint64_t ql = ptx::smem_desc_sw128(qb + kPgTileBytes);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                ptx::mma_tf32(d, ph + 2 * kk, qh + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                ptx::mma_tf32(d, ph + 2 * kk, ql + 2 * kk, idesc, 1u);
+                ptx::mma_tf32(d, pl + 2 * kk, qh + 2 * kk, idesc, 1u);
+              }
+              ptx::mma_commit(&qempty[qst]);
+              if (++qst == kPg2QStages) {
+                qst = 0;
+                qph ^= 1;
+              }
+            }
+            if (!ok) break;
+            ptx::mma_commit(&tfull[acc]);
+            acc ^= 1;
+            if (acc == 0) aph ^= 1;
+          }
+          if (ok) {
+            ptx::mma_commit(pempty);
+            last_pempty = p_loads & 1;
+          }
+        }
+        ++p_loads;  // the MMA thread counts the P blocks it consumed
+        if (!ok) {
+          pg_abort(abort_flag, a.info, kTimeout);
+          ptx::mma_commit(drain);
+          volatile int never = 0;
+          ptx::mbar_wait_bounded(drain, 0, &never, kDrainLimit);
+        }
+      }
+    } else {
+      // epilogue: warps 2 .. 9
+      const int quarter = warp & 3;
+      const int half = (warp - 2) >> 2;
+      float* stage = reinterpret_cast<float*>(sOut + (warp - 2) * kPg2StageOut);
+      for (int q = 0; q < I.nq; ++q) {
+        const bool ready = ptx::mbar_wait_bounded(&tfull[acc], aph, abort_flag, kLimit);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, ready && !*abort_flag)) {
+          if (!ready) pg_abort(abort_flag, a.info, kTimeout);
+          break;
+        }
+        ptx::tc_fence_after();
+        pg_tile_epilogue<true>(I, q, tmem_base + (uint32_t)(acc * 128), quarter, half, lane,
+                               stage, mW, mW);
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&tempty[acc]);
+        acc ^= 1;
+        if (acc == 0) aph ^= 1;
+      }
+      // every reduce this warp issued has landed (and is ordered before the
+      // generic proxy's accesses) before the tiles are published
+      if (lane == 0) {
+        ptx::bulk_wait_all0();
+        fence_proxy_async_global();
+      }
+      __syncwarp();
+    }
+    __syncthreads();
+    if (tid == 0 && !*abort_flag) {
+      __threadfence();
+      for (int c = k.c0; c < k.c1; ++c)
+        ptx::st_release_gpu(&applied[k.R * a.nb + c], (uint32_t)(k.s + 1));
+    }
+  }
+  // the last commit on pempty has landed before the CTA tears down (bounded)
+  if (warp == 1 && lane == 0 && last_pempty >= 0) {
+    volatile int never = 0;
+    ptx::mbar_wait_bounded(pempty, (uint32_t)last_pempty, &never, kDrainLimit);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, kPg2TmemCols);
   }
 }
 
@@ -526,8 +1064,8 @@ cudaError_t launch_selftest_division(const float* a, const float* b, int64_t cou
 }
 
 size_t quantize_workspace_bytes(int64_t rows, int64_t n) {
-  return align_up(sizeof(float) * rows * n, 256) +
-         4 * align_up(sizeof(float) * rows * super_cols(n), 256) + align_up((size_t)rows * n, 256) +
+  return align_up(sizeof(float) * rows * n, 256) + err_region_bytes(rows, n) +
+         (use_persistent(n) ? persist_ctr_bytes(rows, n) : 0) + align_up((size_t)rows * n, 256) +
          align_up(sizeof(int32_t) * n, 256) + 2 * align_up(sizeof(float) * n * ut_ld(n), 256);
 }
 
@@ -538,7 +1076,16 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
                                   float* row_loss, void* ws, int32_t* info, cudaStream_t s,
                                   cudaStream_t side_s) {
   const int rows = (int)rows64, n = (int)n64;
-  SweepWs w = carve(ws, rows64, n64);
+  // A group ruler wider than a block is fitted on all of the group's current
+  // columns, so a group must not cross a super-block's end (the columns past
+  // it get the super-block's updates only at its end): other group sizes use
+  // one level.
+  int64_t S64 = super_cols(n64);
+  if (S64 > kBlock && group_size > kBlock && S64 % group_size != 0 && group_size % S64 != 0)
+    S64 = kBlock;
+  const bool persist = use_persistent(n64);
+  SweepWsExtra extra{};
+  SweepWs w = carve(ws, rows64, n64, S64, persist, &extra);
   const float maxq = (float)((1 << bits) - 1);
   const int per_row = group_size <= 0;
   const int G = per_row ? 1 : (n + group_size - 1) / group_size;
@@ -571,6 +1118,65 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
   const int sweep_ctas = (rows + kSweepRows - 1) / kSweepRows;
   const int sms = num_sms();
 
+  if (persist) {
+    // one launch for every block's sweep and every lazy update (the side
+    // stream is not needed)
+    ut_split_kernel<<<dim3((unsigned)((w.ldut + 31) / 32), (unsigned)((n + 31) / 32)), 256, 0, s>>>(
+        U, n, w.ldut, w.UT_hi, w.UT_lo);
+    note_launch();
+    CUtensorMap pEh, pEl, pUh, pUl, pW;
+    if (!make_tma_2d(&pEh, w.Err_hi[0], false, rows, w.lde, w.lde, 32, 128) ||
+        !make_tma_2d(&pEl, w.Err_lo[0], false, rows, w.lde, w.lde, 32, 128) ||
+        !make_tma_2d(&pUh, w.UT_hi, false, n, n, w.ldut, 32, 128) ||
+        !make_tma_2d(&pUl, w.UT_lo, false, n, n, w.ldut, 32, 128) ||
+        !make_tma_2d(&pW, w.Wf, false, rows, n, n, 32, 32))
+      return cudaErrorInvalidValue;
+    if ((e = cudaMemsetAsync(extra.ctr, 0, persist_ctr_bytes(rows64, n64), s)) != cudaSuccess)
+      return e;
+    const WaitGate pg = current_wait_gate();
+    SweepPersistArgs a;
+    a.Wf = w.Wf;
+    a.rows = rows;
+    a.n = n;
+    a.U = U;
+    a.maxq = maxq;
+    a.sym = sym;
+    a.gsize = group_size;
+    a.G = G;
+    a.gw = gmode == 1 ? group_size / kBlock : 1;
+    a.Eh = w.Err_hi[0];
+    a.El = w.Err_lo[0];
+    a.lde = (int)w.lde;
+    a.codes_sw = w.codes_sw;
+    a.scales = scales;
+    a.zeros = zeros;
+    a.row_loss = row_loss;
+    a.ctr = extra.ctr;
+    a.RB = (rows + kBlock - 1) / kBlock;
+    a.nb = (int)(w.lde / kBlock);
+    a.info = info;
+    a.gate = pg.gate;
+    a.limit_ns = pg.limit_ns;
+    const int grid = std::min(sms, sp_total(a));
+    const size_t smem = pg2_smem_bytes(true);
+#define GPTQ_PERSIST_LAUNCH(GSV)                                                             \
+  if ((e = cudaFuncSetAttribute(sweep_persist_kernel<GSV>,                                  \
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != \
+      cudaSuccess)                                                                          \
+    return e;                                                                               \
+  sweep_persist_kernel<GSV><<<grid, kPg2Threads, smem, s>>>(pEh, pEl, pUh, pUl, pW, a)
+    if (gmode == 0) {
+      GPTQ_PERSIST_LAUNCH(0);
+    } else if (gmode == 1) {
+      GPTQ_PERSIST_LAUNCH(128);
+    } else if (group_size == 32) {
+      GPTQ_PERSIST_LAUNCH(32);
+    } else {
+      GPTQ_PERSIST_LAUNCH(64);
+    }
+#undef GPTQ_PERSIST_LAUNCH
+    note_launch();
+  } else {
   // operands of the lazy update on the tensor cores; with a row stride that
   // is a multiple of 16 bytes the update lands in Wf by TMA reduce-add
   const int S = (int)w.lde;  // super-block columns (kBlock: one level)
@@ -704,7 +1310,11 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
           past(eb, s1, i2, end, sms, s);
         continue;
       }
-      const int near_end = std::min(i2 + kBlock, end);
+      // the near part is what the next sweep reads: the next block, or, when
+      // the next block starts a group wider than a block, the whole group
+      // (its ruler is fitted on all of the group's current columns)
+      const int near_w = (gmode == 1 && i2 % group_size == 0) ? group_size : kBlock;
+      const int near_end = std::min(i2 + near_w, end);
       if (near_end < end && (e = fork()) != cudaSuccess) return e;
       if (far_pending) {
         if ((e = cudaStreamWaitEvent(s, side.ev[1], 0)) != cudaSuccess) return e;
@@ -736,6 +1346,7 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
         (e = cudaStreamWaitEvent(s, side.ev[1], 0)) != cudaSuccess)
       return e;
   }
+  }  // one-block launches
   const size_t un_smem = (Wq ? sizeof(float) * (size_t)n : 0) + (size_t)n;
   if ((e = set_smem(unpermute_kernel, un_smem)) != cudaSuccess) return e;
   unpermute_kernel<<<rows, 256, un_smem, s>>>(w.codes_sw, w.Wf, n, w.pos, codes, Wq);

@@ -323,3 +323,29 @@ def test_quantize_linear_end_to_end():
     assert int(ql.info.item()) == 0
     w = G.gptq_dequant(ql.packed, 4, 256, ql.scales, ql.zeros, 128, ql.g_idx)
     assert torch.equal(w, ql.Wq)
+
+
+@pytest.mark.parametrize("g,actorder", [(256, True), (512, False), (256, False)])
+def test_groups_wider_than_a_block_with_lookahead(g, actorder):
+    """A group of 256 or 512 columns is fitted, when the sweep reaches its
+    first column, on all of its current columns -- several blocks.  With the
+    look-ahead stream the update that reaches those columns must land before
+    the fit: the result equals the one-stream result bit for bit and the
+    oracle's up to rounding ties."""
+    W, X = workloads.random_layer(192, 1024, 4096, seed=g + actorder, dtype=torch.bfloat16,
+                                  correlated=0.4)
+    Wd, Xd = W.cuda(), device_x(X)
+    H = torch.zeros(1024, 1024, device="cuda")
+    G.gptq_hessian_accumulate(H, Xd)
+    cfg = G.make_config(4, g, 0.01, actorder)
+    outs = []
+    for side in (torch.cuda.Stream(), None):
+        U, perm, dead, info = G.gptq_cholesky_inverse(H, 0.01, actorder, side_stream=side)
+        q = G.gptq_quantize_layer(Wd, U, perm, dead, cfg, want_wq=True, side_stream=side)
+        torch.cuda.synchronize()
+        assert int(info.item()) == 0
+        outs.append(q)
+    for k in ("codes", "scales", "zeros", "Wq"):
+        assert torch.equal(outs[0][k], outs[1][k]), k
+    gpu = gpu_layer(W, X, 4, g, 0.01, actorder, H=H)
+    compare_layer(gpu, W, X, 4, g, 0.01, actorder)

@@ -38,8 +38,10 @@ def _run(W, X, actorder, g, side):
     return H, U, perm, dead, q
 
 
-@pytest.mark.parametrize("actorder,g", [(True, 128), (False, 64)])
+@pytest.mark.parametrize("actorder,g", [(True, 128), (False, 64), (False, 384)])
 def test_two_level_blocking_matches_oracle(actorder, g):
+    # g = 384 does not divide a 1024-column super-block: that layer is swept
+    # with one level (the factorisation keeps two)
     rows, n, ntok = 200, 8192, 12288
     Wc, Xc = workloads.random_layer(rows, n, ntok, seed=8192 + g, dtype=torch.bfloat16,
                                     correlated=0.3, dead=(17, 4000))
@@ -80,7 +82,13 @@ def test_two_level_blocking_matches_oracle(actorder, g):
                     + "\n")
     assert rep["mismatched"] == 0, rep["mismatched"]
     assert np.array_equal(rep["codes"], codes_sw)
-    assert all(a[3] <= 1e-5 for a in adoptions), adoptions
+    # a tie is a code whose pre-rounding value lies within 1e-3 tick of a
+    # half-integer; the GPU's values sit much closer to the oracle's than
+    # that: within 1e-5 tick on the two-level path, and within 3e-5 on the
+    # one-level path, whose last columns take 64 separately rounded rank-128
+    # updates instead of 8 of K = 1024
+    bound = 1e-5 if g != 384 else 3e-5
+    assert all(a[3] <= bound for a in adoptions), adoptions
     tie_rows = {a[0] for a in adoptions}
     clean = np.array([r not in tie_rows for r in range(rows)])
     assert float(np.mean(own["codes"][clean] == codes_sw[clean])) >= 0.999
