@@ -12,7 +12,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libgptq_b200.so")
 SOURCES = ["gptq_api.cu", "hessian_syrk.cu", "cholesky.cu", "sweep.cu", "pack.cu", "hadamard.cu"]
-HEADERS = ["gptq_internal.cuh", "sm100_ptx.cuh", "panel_gemm.cuh", "stage.cuh", "chol_diag.cuh",
+HEADERS = ["gptq_internal.cuh", "sm100_ptx.cuh", "panel_gemm.cuh", "persist.cuh", "stage.cuh", "chol_diag.cuh",
            "fdiv.cuh"]
 ROOT = os.path.dirname(PKG)
 

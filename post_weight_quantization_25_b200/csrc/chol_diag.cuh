@@ -29,9 +29,9 @@ constexpr int kDiagThreads = 256;
 constexpr int kDP = 129;   // row pitch (floats) of the block S
 constexpr int kXP = 132;   // row pitch of XT (transposed solved rows)
 constexpr int kTP = 36;    // row pitch of a transposed 32 x 32 leaf
-// S[128][kDP] | XT[32][kXP] | LTl[32][kTP] | rinv[128] | yb[32], zb[32] (float4)
+// S[128][kDP] | XT[32][kXP] | LTl[32][kTP] | rinv[128] | yb[64], zb[64] (float4) | fail
 constexpr size_t kDiagSmemBytes =
-    sizeof(float) * (128 * kDP + 32 * kXP + 32 * kTP + 128 + 256) + 16;
+    sizeof(float) * (128 * kDP + 32 * kXP + 32 * kTP + 128 + 512) + 16 + 16;  // + the fail flag
 
 // Outputs of chol_diag_kernel, in the Cholesky workspace:
 //   Lt[k][c]     = L[c][k]           (128 x 128, zero for k > c)
@@ -139,6 +139,108 @@ __device__ __forceinline__ int leaf_factor(float* S, float* rinv, float* LTl, fl
   return 0;
 }
 
+// The same leaf factor with eight columns per step (four steps per leaf): the
+// per-step costs that do not grow with the panel width (publishing and
+// reading the panel's rows, the warp syncs) are paid half as often, and the
+// eight pivots' recurrence is one dependent chain.  yb and zb hold two
+// float4 per row.  For the panel of columns J..J+7 with diagonal block y:
+//     z_st = y_st - sum_{u<t} M_tu z_su   (t <= s),  d_s = z_ss,
+//     M_st = z_st / d_t   (t < s),
+// each row i takes z_it = y_it - sum_{u<t} M_tu z_iu, and the trailing
+// entries take a_ik -= sum_t (z_it / d_t) z_kt.
+// one eight-column step of leaf_factor8 (J a compile-time constant, so the
+// row stays in registers)
+template <int J>
+__device__ __forceinline__ void leaf_step8(float (&a)[32], float4* yb, float4* zb, int lane,
+                                           int& first_bad) {
+  __syncwarp();
+  // the panel's diagonal block and its recurrence (every lane)
+  float z[8][8], M[8][8], iv[8];
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const float4 lo = yb[2 * (J + s)], hi = yb[2 * (J + s) + 1];
+    const float ys[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+    for (int t = 0; t <= s; ++t) {
+      float v = ys[t];
+#pragma unroll
+      for (int u = 0; u < t; ++u) v = fmaf(-M[t][u], z[s][u], v);
+      z[s][t] = v;
+      if (t < s) M[s][t] = v * iv[t];
+    }
+    iv[s] = recip_nr(z[s][s]);
+  }
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    const float d = z[t][t];
+    const bool badj = !(d > 0.f) || !isfinite(d);
+    first_bad = (first_bad == 0 && badj) ? (J + t + 1) : first_bad;
+  }
+  // this row's z (for the panel rows this reproduces the block's values)
+  float zi[8];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    float v = a[J + t];
+#pragma unroll
+    for (int u = 0; u < t; ++u) v = fmaf(-M[t][u], zi[u], v);
+    zi[t] = v;
+    a[J + t] = v;
+  }
+  if constexpr (J + 8 < 32) {
+    zb[2 * lane] = make_float4(zi[0], zi[1], zi[2], zi[3]);
+    zb[2 * lane + 1] = make_float4(zi[4], zi[5], zi[6], zi[7]);
+    float m[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) m[t] = zi[t] * iv[t];
+    __syncwarp();
+    // the next panel's columns first, then publish them
+#pragma unroll
+    for (int k = J + 8; k < 32; ++k) {
+      const float4 lo = zb[2 * k], hi = zb[2 * k + 1];
+      const float zk[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+      float v = a[k];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) v = fmaf(-m[t], zk[t], v);
+      a[k] = v;
+      if (k == J + 15) {
+        yb[2 * lane] = make_float4(a[J + 8], a[J + 9], a[J + 10], a[J + 11]);
+        yb[2 * lane + 1] = make_float4(a[J + 12], a[J + 13], a[J + 14], a[J + 15]);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ int leaf_factor8(float* S, float* rinv, float* LTl, float4* yb,
+                                            float4* zb, int c0, int lane) {
+  float a[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) a[k] = (k <= lane) ? S[(c0 + lane) * kDP + c0 + k] : 0.f;
+  int first_bad = 0;
+  yb[2 * lane] = make_float4(a[0], a[1], a[2], a[3]);
+  yb[2 * lane + 1] = make_float4(a[4], a[5], a[6], a[7]);
+  leaf_step8<0>(a, yb, zb, lane, first_bad);
+  leaf_step8<8>(a, yb, zb, lane, first_bad);
+  leaf_step8<16>(a, yb, zb, lane, first_bad);
+  leaf_step8<24>(a, yb, zb, lane, first_bad);
+  if (first_bad) return first_bad;
+  // L_ik = a_ik / sqrt(d_k), L_kk = sqrt(d_k)
+  float dd = 1.f;
+#pragma unroll
+  for (int k = 0; k < 32; ++k)
+    if (k == lane) dd = a[k];
+  const float rs = __frsqrt_rn(dd);
+  rinv[c0 + lane] = rs;
+  const float lkk = __fsqrt_rn(dd);
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const float rk = __shfl_sync(0xffffffffu, rs, k);
+    const float l = (k < lane) ? a[k] * rk : ((k == lane) ? lkk : 0.f);
+    if (k <= lane) S[(c0 + lane) * kDP + c0 + k] = l;
+    LTl[k * kTP + lane] = l;   // zero above the diagonal of the transpose
+  }
+  return 0;
+}
+
 // One warp: column `lane` of the inverse of the 32 x 32 lower leaf at
 // (c0, c0) of S, written as row `lane` of LiT: LiT[lane][m] = Li[m][lane].
 __device__ __forceinline__ void leaf_inverse(const float* S, const float* rinv, float* LiT,
@@ -160,57 +262,95 @@ __device__ __forceinline__ void leaf_inverse(const float* S, const float* rinv, 
                          4 * q + 2 >= lane ? x[4 * q + 2] : 0.f, 4 * q + 3 >= lane ? x[4 * q + 3] : 0.f);
 }
 
+// Threads 0 .. kDiagThreads - 1 synchronise on barrier `bar` (0:
+// __syncthreads, else a named barrier of kDiagThreads threads).
+__device__ __forceinline__ void diag_sync(int bar) {
+  if (bar == 0)
+    __syncthreads();
+  else
+    ptx::named_bar_sync(bar, kDiagThreads);
+}
+
 // Factor the diagonal block of panel p of the n x n lower matrix A and
 // invert its leaves; writes Lt and LiT (layouts above) to `out`.  Rows and
 // columns past a short last panel are identity padding.  On a failed pivot
 // sets *info = n - (global index of the pivot in A), if no failure was
-// recorded before, and returns.
-__global__ void __launch_bounds__(kDiagThreads) chol_diag_kernel(const float* __restrict__ A,
-                                                                 int n, int p,
-                                                                 float* __restrict__ out,
-                                                                 int32_t* __restrict__ info) {
-  if (*(volatile int32_t*)info != 0) return;
-  extern __shared__ __align__(16) float dsm[];
+// recorded before, and returns.  Run by threads 0 .. kDiagThreads - 1 (tid)
+// with kDiagSmemBytes of shared memory at dsm.
+__device__ __forceinline__ void chol_diag_body(const float* __restrict__ A, int n, int p,
+                                               float* __restrict__ out,
+                                               int32_t* __restrict__ info, float* dsm, int tid,
+                                               int bar) {
   float* S = dsm;                    // [128][kDP]  the block, becomes L
   float* XT = S + 128 * kDP;         // [32][kXP]   XT[k][r] = solved row r, column k of the leaf
   XT = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(XT) + 15) & ~uintptr_t(15));
   float* LTl = XT + 32 * kXP;        // [32][kTP]   current leaf, transposed
   float* rinv = LTl + 32 * kTP;      // [128]       1 / L_kk
-  float4* yb = reinterpret_cast<float4*>(rinv + 128);  // [32] leaf panel rows
-  float4* zb = yb + 32;                                 // [32] leaf z values
-  __shared__ int fail;
+  float4* yb = reinterpret_cast<float4*>(rinv + 128);  // [64] leaf panel rows
+  float4* zb = yb + 64;                                 // [64] leaf z values
+  volatile int* fail = reinterpret_cast<volatile int*>(zb + 64);
   const int kb = p * 128;
   const int bs = min(128, n - kb);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int lane = tid & 31, warp = tid >> 5;
 
   // stage the lower block (async copies, all in flight at once); rows past
   // bs are the identity; entries above the diagonal are never read
-  for (int f = tid; f < 128 * 32; f += kDiagThreads) {
-    const int r = f >> 5, c = (f & 31) * 4;
-    if (c > r) continue;
-    if (r >= bs) {
+  if ((n % 4) == 0) {
+    // 16-byte loads (rows start 16-byte aligned, bs is a multiple of 4), four
+    // in flight per thread before their stores into the odd-pitched block
+    constexpr int kIt = 128 * 32 / kDiagThreads;
+#pragma unroll 1
+    for (int i0 = 0; i0 < kIt; i0 += 4) {
+      float4 v[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) S[r * kDP + c + i] = (r == c + i) ? 1.f : 0.f;
-      continue;
+      for (int i = 0; i < 4; ++i) {
+        const int f = tid + kDiagThreads * (i0 + i);
+        const int r = f >> 5, c = (f & 31) * 4;
+        v[i] = (c <= r && r < bs)
+                   ? __ldcg(reinterpret_cast<const float4*>(A + (int64_t)(kb + r) * n + kb + c))
+                   : make_float4(r == c, r == c + 1, r == c + 2, r == c + 3);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int f = tid + kDiagThreads * (i0 + i);
+        const int r = f >> 5, c = (f & 31) * 4;
+        if (c > r) continue;
+        float* d = S + r * kDP + c;
+        d[0] = v[i].x;
+        d[1] = v[i].y;
+        d[2] = v[i].z;
+        d[3] = v[i].w;
+      }
     }
-    const float* src = A + (int64_t)(kb + r) * n + kb + c;
+  } else {
+    for (int f = tid; f < 128 * 32; f += kDiagThreads) {
+      const int r = f >> 5, c = (f & 31) * 4;
+      if (c > r) continue;
+      if (r >= bs) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      ptx::cp_async_4(S + r * kDP + c + i, (c + i < bs) ? src + i : src, (c + i < bs) ? 4 : 0);
+        for (int i = 0; i < 4; ++i) S[r * kDP + c + i] = (r == c + i) ? 1.f : 0.f;
+        continue;
+      }
+      const float* src = A + (int64_t)(kb + r) * n + kb + c;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        ptx::cp_async_4(S + r * kDP + c + i, (c + i < bs) ? src + i : src, (c + i < bs) ? 4 : 0);
+    }
+    ptx::cp_async_wait_all();
   }
-  ptx::cp_async_wait_all();
-  if (tid == 0) fail = 0;
-  __syncthreads();
+  if (tid == 0) *fail = 0;
+  diag_sync(bar);
 
   for (int j = 0; j < 4; ++j) {
     const int c0 = 32 * j;
     if (warp == 0) {
       const int fb = leaf_factor(S, rinv, LTl, yb, zb, c0, lane);
-      if (fb && lane == 0) fail = c0 + fb;
+      if (fb && lane == 0) *fail = c0 + fb;
     }
-    __syncthreads();
-    if (fail) {
-      if (tid == 0) atomicCAS(info, 0, n - (kb + fail - 1));
+    diag_sync(bar);
+    const int fl = *fail;
+    if (fl) {
+      if (tid == 0) atomicCAS(info, 0, n - (kb + fl - 1));
       return;
     }
     const int base = c0 + 32;
@@ -243,7 +383,7 @@ __global__ void __launch_bounds__(kDiagThreads) chol_diag_kernel(const float* __
         XT[k * kXP + (r - base)] = x[k];
       }
     }
-    __syncthreads();
+    diag_sync(bar);
     // rank-32 update of the remaining lower block: 8-row x 4-column tiles
     // (ti, tj) with 4 tj <= 8 ti + 7; rows past bs are identity padding
     {
@@ -282,7 +422,7 @@ __global__ void __launch_bounds__(kDiagThreads) chol_diag_kernel(const float* __
         }
       }
     }
-    __syncthreads();
+    diag_sync(bar);
   }
 
   // ---- outputs: L transposed, then the four leaf inverses
@@ -300,6 +440,15 @@ __global__ void __launch_bounds__(kDiagThreads) chol_diag_kernel(const float* __
   if (warp < 4) leaf_inverse(S, rinv, LiT + warp * 32 * 32, 32 * warp, lane);
 }
 
+__global__ void __launch_bounds__(kDiagThreads) chol_diag_kernel(const float* __restrict__ A,
+                                                                 int n, int p,
+                                                                 float* __restrict__ out,
+                                                                 int32_t* __restrict__ info) {
+  if (*(volatile int32_t*)info != 0) return;
+  extern __shared__ __align__(16) float dsm[];
+  chol_diag_body(A, n, p, out, info, dsm, threadIdx.x, 0);
+}
+
 // x = v L^-T for every vector of panel p: vectors [0, nA) are rows
 // kb+bs+v of A, vectors [nA, nA + kb + bs) are rows v - nA of RT (both
 // restricted to the panel's columns [kb, kb + bs)).  The result goes, split
@@ -313,12 +462,13 @@ constexpr int kVP = 132;  // row pitch of the vector tile
 constexpr size_t kApplySmemBytes =
     sizeof(float) * (128 * 128 + 4 * 32 * 32 + 2 * kApplyVecs * kVP);
 
-__global__ void __launch_bounds__(kApplyThreads) panel_apply_kernel(
+// Vectors [v0, v0 + kApplyVecs) of panel p, by threads 0 .. kApplyThreads - 1
+// (tid) with kApplySmemBytes of shared memory at asmem; barrier as diag_sync.
+__device__ __forceinline__ void panel_apply_body(
     const float* __restrict__ A, float* __restrict__ RT, int n, int p,
     const float* __restrict__ diag_out, float* __restrict__ PBh, float* __restrict__ PBl, int ldpb,
-    const int32_t* __restrict__ info) {
-  if (*(volatile const int32_t*)info != 0) return;
-  extern __shared__ __align__(16) float asmem[];
+    float* asmem, int tid, int v0, int bar) {
+  static_assert(kApplyThreads == kDiagThreads, "the apply shares the diagonal step's barrier");
   float* Lt = asmem;                         // [128][128]
   float* LiT = Lt + 128 * 128;               // [4][32][32]
   float* X = LiT + 4 * 32 * 32;              // [32][kVP]  vectors, solved in place
@@ -327,54 +477,80 @@ __global__ void __launch_bounds__(kApplyThreads) panel_apply_kernel(
   const int bs = min(128, n - kb);
   const int nA = n - kb - bs;
   const int nvec = nA + kb + bs;
-  const int v0 = blockIdx.x * kApplyVecs;
   if (v0 >= nvec) return;
-  const int tid = threadIdx.x;
   // everything staged with async copies, all in flight at once
   for (int f = tid; f < kDiagOutFloats / 4; f += kApplyThreads)
     ptx::cp_async_16(asmem + 4 * f, diag_out + 4 * f);
-  for (int f = tid; f < kApplyVecs * 128; f += kApplyThreads) {
-    const int vi = f >> 7, k = f & 127;
-    const int v = v0 + vi;
-    const bool ok = v < nvec && k < bs;
-    const float* row = (v < nA) ? (A + (int64_t)(kb + bs + v) * n + kb)
-                                : (RT + (int64_t)min(v - nA, n - 1) * n + kb);
-    ptx::cp_async_4(X + vi * kVP + k, ok ? row + k : A, ok ? 4 : 0);
+  if ((n % 4) == 0) {
+    // rows start 16-byte aligned and bs is a multiple of 4: 16-byte copies
+    for (int f = tid; f < kApplyVecs * 32; f += kApplyThreads) {
+      const int vi = f >> 5, k = (f & 31) * 4;
+      const int v = v0 + vi;
+      const bool ok = v < nvec && k < bs;
+      const float* row = (v < nA) ? (A + (int64_t)(kb + bs + v) * n + kb)
+                                  : (RT + (int64_t)min(v - nA, n - 1) * n + kb);
+      ptx::cp_async_16z(X + vi * kVP + k, ok ? row + k : A, ok ? 16 : 0);
+    }
+  } else {
+    for (int f = tid; f < kApplyVecs * 128; f += kApplyThreads) {
+      const int vi = f >> 7, k = f & 127;
+      const int v = v0 + vi;
+      const bool ok = v < nvec && k < bs;
+      const float* row = (v < nA) ? (A + (int64_t)(kb + bs + v) * n + kb)
+                                  : (RT + (int64_t)min(v - nA, n - 1) * n + kb);
+      ptx::cp_async_4(X + vi * kVP + k, ok ? row + k : A, ok ? 4 : 0);
+    }
   }
   ptx::cp_async_wait_all();
-  __syncthreads();
+  diag_sync(bar);
   const int vi = tid >> 3, cq = tid & 7;
   float* xr = X + vi * kVP;
   for (int j = 0; j < 4; ++j) {
     const int cb = 32 * j + 4 * cq;
     // y = v_j - sum_{k < 32 j} x_k L[cb + i][k]
     float y0 = xr[cb], y1 = xr[cb + 1], y2 = xr[cb + 2], y3 = xr[cb + 3];
-#pragma unroll 8
-    for (int k = 0; k < 32 * j; ++k) {
-      const float xk = xr[k];
-      const float4 l4 = *reinterpret_cast<const float4*>(Lt + k * 128 + cb);
-      y0 = fmaf(-xk, l4.x, y0);
-      y1 = fmaf(-xk, l4.y, y1);
-      y2 = fmaf(-xk, l4.z, y2);
-      y3 = fmaf(-xk, l4.w, y3);
+    // eight k at a time: their loads are issued together, then the FMAs
+    // (still in k order)
+#pragma unroll 1
+    for (int k0 = 0; k0 < 32 * j; k0 += 8) {
+      const float4 xa = *reinterpret_cast<const float4*>(xr + k0);
+      const float4 xb = *reinterpret_cast<const float4*>(xr + k0 + 4);
+      const float xk[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+      float4 l4[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) l4[i] = *reinterpret_cast<const float4*>(Lt + (k0 + i) * 128 + cb);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        y0 = fmaf(-xk[i], l4[i].x, y0);
+        y1 = fmaf(-xk[i], l4[i].y, y1);
+        y2 = fmaf(-xk[i], l4[i].z, y2);
+        y3 = fmaf(-xk[i], l4[i].w, y3);
+      }
     }
     *reinterpret_cast<float4*>(Y + vi * kVP + 4 * cq) = make_float4(y0, y1, y2, y3);
-    __syncthreads();
+    diag_sync(bar);
     // x_j = y Li_jj^T: x[c] = sum_{t <= c} y[t] Li[c][t] = sum_t y[t] LiT[t][c]
     const float* yr = Y + vi * kVP;
     const float* lit = LiT + j * 32 * 32 + 4 * cq;
     float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
-#pragma unroll 8
-    for (int t = 0; t < 32; ++t) {
-      const float yt = yr[t];
-      const float4 l4 = *reinterpret_cast<const float4*>(lit + t * 32);
-      z0 = fmaf(yt, l4.x, z0);
-      z1 = fmaf(yt, l4.y, z1);
-      z2 = fmaf(yt, l4.z, z2);
-      z3 = fmaf(yt, l4.w, z3);
+#pragma unroll
+    for (int t0 = 0; t0 < 32; t0 += 8) {
+      const float4 ya = *reinterpret_cast<const float4*>(yr + t0);
+      const float4 yb = *reinterpret_cast<const float4*>(yr + t0 + 4);
+      const float yt[8] = {ya.x, ya.y, ya.z, ya.w, yb.x, yb.y, yb.z, yb.w};
+      float4 l4[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) l4[i] = *reinterpret_cast<const float4*>(lit + (t0 + i) * 32);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        z0 = fmaf(yt[i], l4[i].x, z0);
+        z1 = fmaf(yt[i], l4[i].y, z1);
+        z2 = fmaf(yt[i], l4[i].z, z2);
+        z3 = fmaf(yt[i], l4[i].w, z3);
+      }
     }
     *reinterpret_cast<float4*>(xr + cb) = make_float4(z0, z1, z2, z3);
-    __syncthreads();
+    diag_sync(bar);
   }
   // outputs
   for (int f = tid; f < kApplyVecs * 32; f += kApplyThreads) {
@@ -401,6 +577,16 @@ __global__ void __launch_bounds__(kApplyThreads) panel_apply_kernel(
         if (c4 + i < bs) rt[c4 + i] = xv[i];
     }
   }
+}
+
+__global__ void __launch_bounds__(kApplyThreads) panel_apply_kernel(
+    const float* __restrict__ A, float* __restrict__ RT, int n, int p,
+    const float* __restrict__ diag_out, float* __restrict__ PBh, float* __restrict__ PBl, int ldpb,
+    const int32_t* __restrict__ info) {
+  if (*(volatile const int32_t*)info != 0) return;
+  extern __shared__ __align__(16) float asmem[];
+  panel_apply_body(A, RT, n, p, diag_out, PBh, PBl, ldpb, asmem, threadIdx.x,
+                   blockIdx.x * kApplyVecs, 0);
 }
 
 }  // namespace gptq

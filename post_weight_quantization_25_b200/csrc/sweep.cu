@@ -30,6 +30,7 @@
 
 #include "gptq_internal.cuh"
 #include "panel_gemm.cuh"
+#include "persist.cuh"
 #include "fdiv.cuh"
 #include "stage.cuh"
 
@@ -722,10 +723,6 @@ __host__ __device__ inline SpTask sp_decode(const SweepPersistArgs& a, int t) {
   }
 }
 
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
 template <int GS>
 __global__ void __launch_bounds__(kPg2Threads, 1)
     sweep_persist_kernel(const __grid_constant__ CUtensorMap mEh,
@@ -734,71 +731,21 @@ __global__ void __launch_bounds__(kPg2Threads, 1)
                          const __grid_constant__ CUtensorMap mUl,
                          const __grid_constant__ CUtensorMap mW, const SweepPersistArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* sP = smem;
-  uint8_t* sQ = smem + kPg2PBytes;
-  uint8_t* sOut = sQ + kPg2QStages * kPg2QStageBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + 8 * kPg2StageOut);
-  uint64_t* pfull = bars;
-  uint64_t* pempty = bars + 1;
-  uint64_t* qfull = bars + 2;
-  uint64_t* qempty = qfull + kPg2QStages;
-  uint64_t* tfull = qempty + kPg2QStages;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* task_slot = abort_flag + 1;
-  constexpr uint64_t kDrainLimit = (uint64_t)kGridWaitLimitNs;
-  const uint64_t kLimit = a.limit_ns;
   constexpr int32_t kTimeout = -2;
+  PersistCta cta;
+  cta.init(smem_raw, a.limit_ns);
+  uint8_t* smem = cta.smem;
+  volatile int* abort_flag = cta.abort_flag;
+  const uint64_t kLimit = a.limit_ns;
   uint32_t* swept = a.ctr + 1;
   uint32_t* applied = a.ctr + 1 + a.RB;
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (tid == 0) {
-    ptx::mbar_init(pfull, 1);
-    ptx::mbar_init(pempty, 1);
-    for (int q = 0; q < kPg2QStages; ++q) {
-      ptx::mbar_init(&qfull[q], 1);
-      ptx::mbar_init(&qempty[q], 1);
-    }
-    for (int c = 0; c < 2; ++c) {
-      ptx::mbar_init(&tfull[c], 1);
-      ptx::mbar_init(&tempty[c], 256);
-    }
-    ptx::mbar_init(drain, 1);
-    *abort_flag = 0;
-    ptx::fence_mbar_init();
-  }
-  if (warp == 1) {
-    ptx::tmem_alloc(tmem_slot, kPg2TmemCols);
-    ptx::tmem_relinquish();
-  }
-  ptx::tc_fence_before();
-  __syncthreads();
-  ptx::tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  if (tid == 0 && !ptx::gate_wait_bounded(a.gate, kLimit)) pg_abort(abort_flag, a.info, kTimeout);
-
-  // pipeline state of the update tasks, kept by the thread of each role
-  int p_loads = 0;              // producer: P blocks loaded; MMA: P blocks consumed
-  int qst = 0;                  // producer / MMA: Q ring stage
-  uint32_t qph = 0;
-  int acc = 0;                  // MMA / epilogue: TMEM accumulator
-  uint32_t aph = 0;
-  int q_last_parity[kPg2QStages] = {-1, -1};
-  int last_pempty = -1;         // MMA: parity of its last commit on pempty
+  const int tid = threadIdx.x;
+  if (tid == 0 && !ptx::gate_wait_bounded(a.gate, kLimit)) persist_abort(abort_flag, a.info, kTimeout);
   const int total = sp_total(a);
 
   while (true) {
-    if (tid == 0) *task_slot = (int)atomicAdd(a.ctr, 1u);
-    __syncthreads();
-    const int t = *task_slot;
-    const bool stop = *abort_flag != 0;
-    __syncthreads();
-    if (t >= total || stop) break;
+    const int t = cta.next_task(a.ctr, total);
+    if (t < 0) break;
     const SpTask k = sp_decode(a, t);
     if (k.kind == 0) {
       // ---------------------------------------------------------------- sweep task
@@ -818,7 +765,7 @@ __global__ void __launch_bounds__(kPg2Threads, 1)
         bool ok = true;
         for (int c = k.s; c < c_hi && ok; ++c)
           ok = ptx::flag_wait_bounded(&applied[k.R * a.nb + c], (uint32_t)k.s, abort_flag, kLimit);
-        if (!ok) pg_abort(abort_flag, a.info, kTimeout);
+        if (!ok) persist_abort(abort_flag, a.info, kTimeout);
         fence_proxy_async_global();
       }
       __syncthreads();
@@ -863,135 +810,12 @@ __global__ void __launch_bounds__(kPg2Threads, 1)
                                        abort_flag, kLimit);
       for (int c = k.c0; c < k.c1 && ok; ++c)
         ok = ptx::flag_wait_bounded(&applied[k.R * a.nb + c], (uint32_t)k.s, abort_flag, kLimit);
-      if (!ok) pg_abort(abort_flag, a.info, kTimeout);
+      if (!ok) persist_abort(abort_flag, a.info, kTimeout);
       fence_proxy_async_global();
     }
     __syncthreads();
     if (*abort_flag) continue;
-    if (warp == 0) {
-      if (lane == 0) {
-        // producer: the block's err terms (all of K = 128), then Q per tile
-        bool ok = p_loads == 0 ||
-                  ptx::mbar_wait_bounded(pempty, (uint32_t)((p_loads - 1) & 1), abort_flag, kLimit);
-        if (ok) {
-          ptx::mbar_arrive_expect_tx(pfull, kPg2PBytes);
-          for (int kb = 0; kb < kPgKBlocks; ++kb) {
-            ptx::tma_load_2d(sP + kb * 2 * kPgTileBytes, &mEh, pfull, I.pkx + 32 * kb, I.prow);
-            ptx::tma_load_2d(sP + kb * 2 * kPgTileBytes + kPgTileBytes, &mEl, pfull,
-                             I.pkx + 32 * kb, I.prow);
-          }
-          ++p_loads;
-          for (int q = 0; q < I.nq && ok; ++q)
-            for (int kb = 0; kb < kPgKBlocks; ++kb) {
-              if (!ptx::mbar_wait_bounded(&qempty[qst], qph ^ 1, abort_flag, kLimit)) {
-                ok = false;
-                break;
-              }
-              uint8_t* sb = sQ + qst * kPg2QStageBytes;
-              ptx::mbar_arrive_expect_tx(&qfull[qst], kPg2QStageBytes);
-              ptx::tma_load_2d(sb, &mUh, &qfull[qst], I.qkx + 32 * kb, I.qrow0 + 128 * q);
-              ptx::tma_load_2d(sb + kPgTileBytes, &mUl, &qfull[qst], I.qkx + 32 * kb,
-                               I.qrow0 + 128 * q);
-              q_last_parity[qst] = (int)qph;
-              if (++qst == kPg2QStages) {
-                qst = 0;
-                qph ^= 1;
-              }
-            }
-        }
-        if (!ok) {
-          pg_abort(abort_flag, a.info, kTimeout);
-          volatile int never = 0;  // this CTA's own copies in flight
-          ptx::mbar_wait_bounded(pfull, (uint32_t)((p_loads - 1) & 1), &never, kDrainLimit);
-          for (int q = 0; q < kPg2QStages; ++q)
-            if (q_last_parity[q] >= 0)
-              ptx::mbar_wait_bounded(&qfull[q], (uint32_t)q_last_parity[q], &never, kDrainLimit);
-        }
-      }
-    } else if (warp == 1) {
-      if (lane == 0) {
-        // MMA issuer
-        constexpr uint32_t idesc = ptx::idesc_tf32_f32(128, 128);
-        bool ok = ptx::mbar_wait_bounded(pfull, (uint32_t)(p_loads & 1), abort_flag, kLimit);
-        if (ok) {
-          ptx::tc_fence_after();
-          for (int q = 0; q < I.nq && ok; ++q) {
-            if (!ptx::mbar_wait_bounded(&tempty[acc], aph ^ 1, abort_flag, kLimit)) {
-              ok = false;
-              break;
-            }
-            ptx::tc_fence_after();
-            const uint32_t d = tmem_base + (uint32_t)(acc * 128);
-            for (int kb = 0; kb < kPgKBlocks; ++kb) {
-              if (!ptx::mbar_wait_bounded(&qfull[qst], qph, abort_flag, kLimit)) {
-                ok = false;
-                break;
-              }
-              ptx::tc_fence_after();
-              const uint32_t pb = ptx::smem_u32(sP + kb * 2 * kPgTileBytes);
-              const uint32_t qb = ptx::smem_u32(sQ + qst * kPg2QStageBytes);
-              const uint64_t ph = ptx::smem_desc_sw128(pb);
-              const uint64_t pl = ptx::smem_desc_sw128(pb + kPgTileBytes);
-              const uint64_t qh = ptx::smem_desc_sw128(qb);
-              const uint64_t ql = ptx::smem_desc_sw128(qb + kPgTileBytes);
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                ptx::mma_tf32(d, ph + 2 * kk, qh + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-                ptx::mma_tf32(d, ph + 2 * kk, ql + 2 * kk, idesc, 1u);
-                ptx::mma_tf32(d, pl + 2 * kk, qh + 2 * kk, idesc, 1u);
-              }
-              ptx::mma_commit(&qempty[qst]);
-              if (++qst == kPg2QStages) {
-                qst = 0;
-                qph ^= 1;
-              }
-            }
-            if (!ok) break;
-            ptx::mma_commit(&tfull[acc]);
-            acc ^= 1;
-            if (acc == 0) aph ^= 1;
-          }
-          if (ok) {
-            ptx::mma_commit(pempty);
-            last_pempty = p_loads & 1;
-          }
-        }
-        ++p_loads;  // the MMA thread counts the P blocks it consumed
-        if (!ok) {
-          pg_abort(abort_flag, a.info, kTimeout);
-          ptx::mma_commit(drain);
-          volatile int never = 0;
-          ptx::mbar_wait_bounded(drain, 0, &never, kDrainLimit);
-        }
-      }
-    } else {
-      // epilogue: warps 2 .. 9
-      const int quarter = warp & 3;
-      const int half = (warp - 2) >> 2;
-      float* stage = reinterpret_cast<float*>(sOut + (warp - 2) * kPg2StageOut);
-      for (int q = 0; q < I.nq; ++q) {
-        const bool ready = ptx::mbar_wait_bounded(&tfull[acc], aph, abort_flag, kLimit);
-        __syncwarp();
-        if (!__all_sync(0xffffffffu, ready && !*abort_flag)) {
-          if (!ready) pg_abort(abort_flag, a.info, kTimeout);
-          break;
-        }
-        ptx::tc_fence_after();
-        pg_tile_epilogue<true>(I, q, tmem_base + (uint32_t)(acc * 128), quarter, half, lane,
-                               stage, mW, mW);
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(&tempty[acc]);
-        acc ^= 1;
-        if (acc == 0) aph ^= 1;
-      }
-      // every reduce this warp issued has landed (and is ordered before the
-      // generic proxy's accesses) before the tiles are published
-      if (lane == 0) {
-        ptx::bulk_wait_all0();
-        fence_proxy_async_global();
-      }
-      __syncwarp();
-    }
+    cta.update(I, mEh, mEl, mUh, mUl, mW, mW, a.info, kTimeout);
     __syncthreads();
     if (tid == 0 && !*abort_flag) {
       __threadfence();
@@ -999,17 +823,7 @@ __global__ void __launch_bounds__(kPg2Threads, 1)
         ptx::st_release_gpu(&applied[k.R * a.nb + c], (uint32_t)(k.s + 1));
     }
   }
-  // the last commit on pempty has landed before the CTA tears down (bounded)
-  if (warp == 1 && lane == 0 && last_pempty >= 0) {
-    volatile int never = 0;
-    ptx::mbar_wait_bounded(pempty, (uint32_t)last_pempty, &never, kDrainLimit);
-  }
-  ptx::tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, kPg2TmemCols);
-  }
+  cta.teardown();
 }
 
 // One CTA per row: codes[r][c] = codes_sw[r][pos[c]], Wq[r][c] = Wf[r][pos[c]].

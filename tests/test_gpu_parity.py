@@ -199,9 +199,12 @@ def test_hessian_zero_tokens_is_a_no_op():
 
 
 # ------------------------------------------------------------------ Cholesky
+# widths that are a multiple of 128 with at least 3 panels (384, 640, 1024,
+# 2048) take the persistent factorisation; the others launch panel by panel
 @pytest.mark.parametrize("n,actorder,dead", [(6, False, ()), (130, True, (7,)),
                                              (256, False, ()), (300, True, (0, 299)),
-                                             (640, True, ())])
+                                             (384, True, ()), (640, True, ()),
+                                             (1024, False, (3, 1000)), (2048, True, ())])
 def test_cholesky_inverse_matches_oracle(n, actorder, dead):
     _, X = workloads.random_layer(1, n, 3 * n + 50, seed=n, dead=dead, correlated=0.3)
     Ho32 = O.hessian(to_np(X)).astype(np.float32)          # the oracle's own H, as fp32
@@ -221,8 +224,8 @@ def test_cholesky_inverse_matches_oracle(n, actorder, dead):
         assert np.array_equal(perm.cpu().numpy(), np.arange(n))
 
 
-def test_cholesky_reports_failures_in_info():
-    n = 200
+@pytest.mark.parametrize("n", [200, 512])
+def test_cholesky_reports_failures_in_info(n):
     H = -torch.eye(n, device="cuda")
     _, _, _, info = G.gptq_cholesky_inverse(H, 0.0, False)
     assert int(info.item()) > 0            # not positive definite
@@ -230,6 +233,14 @@ def test_cholesky_reports_failures_in_info():
     H[5, 5] = float("nan")
     _, _, _, info = G.gptq_cholesky_inverse(H, 0.01, True)
     assert int(info.item()) == -1
+    # a negative pivot at column j of a diagonal H: the factorisation runs from
+    # the last column to the first, so it is found at step n - 1 - j and
+    # reported as j + 1 (a later panel than the first on both paths)
+    j = 100
+    H = torch.eye(n, device="cuda") * 2.0
+    H[j, j] = -1.0
+    _, _, _, info = G.gptq_cholesky_inverse(H, 0.0, False)
+    assert int(info.item()) == j + 1
     H = torch.eye(n, device="cuda") * 2.0
     _, _, _, info = G.gptq_cholesky_inverse(H, 0.01, True)
     assert int(info.item()) == 0           # the context is still usable
