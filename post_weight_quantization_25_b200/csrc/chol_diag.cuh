@@ -29,9 +29,9 @@ constexpr int kDiagThreads = 256;
 constexpr int kDP = 129;   // row pitch (floats) of the block S
 constexpr int kXP = 132;   // row pitch of XT (transposed solved rows)
 constexpr int kTP = 36;    // row pitch of a transposed 32 x 32 leaf
-// S[128][kDP] | XT[32][kXP] | LTl[32][kTP] | rinv[128] | yb[64], zb[64] (float4) | fail
+// S[128][kDP] | XT[32][kXP] | LTl[32][kTP] | rinv[128] | yb[32], zb[32] (float4) | fail
 constexpr size_t kDiagSmemBytes =
-    sizeof(float) * (128 * kDP + 32 * kXP + 32 * kTP + 128 + 512) + 16 + 16;  // + the fail flag
+    sizeof(float) * (128 * kDP + 32 * kXP + 32 * kTP + 128 + 256) + 16 + 16;  // + the fail flag
 
 // Outputs of chol_diag_kernel, in the Cholesky workspace:
 //   Lt[k][c]     = L[c][k]           (128 x 128, zero for k > c)
@@ -139,108 +139,6 @@ __device__ __forceinline__ int leaf_factor(float* S, float* rinv, float* LTl, fl
   return 0;
 }
 
-// The same leaf factor with eight columns per step (four steps per leaf): the
-// per-step costs that do not grow with the panel width (publishing and
-// reading the panel's rows, the warp syncs) are paid half as often, and the
-// eight pivots' recurrence is one dependent chain.  yb and zb hold two
-// float4 per row.  For the panel of columns J..J+7 with diagonal block y:
-//     z_st = y_st - sum_{u<t} M_tu z_su   (t <= s),  d_s = z_ss,
-//     M_st = z_st / d_t   (t < s),
-// each row i takes z_it = y_it - sum_{u<t} M_tu z_iu, and the trailing
-// entries take a_ik -= sum_t (z_it / d_t) z_kt.
-// one eight-column step of leaf_factor8 (J a compile-time constant, so the
-// row stays in registers)
-template <int J>
-__device__ __forceinline__ void leaf_step8(float (&a)[32], float4* yb, float4* zb, int lane,
-                                           int& first_bad) {
-  __syncwarp();
-  // the panel's diagonal block and its recurrence (every lane)
-  float z[8][8], M[8][8], iv[8];
-#pragma unroll
-  for (int s = 0; s < 8; ++s) {
-    const float4 lo = yb[2 * (J + s)], hi = yb[2 * (J + s) + 1];
-    const float ys[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-#pragma unroll
-    for (int t = 0; t <= s; ++t) {
-      float v = ys[t];
-#pragma unroll
-      for (int u = 0; u < t; ++u) v = fmaf(-M[t][u], z[s][u], v);
-      z[s][t] = v;
-      if (t < s) M[s][t] = v * iv[t];
-    }
-    iv[s] = recip_nr(z[s][s]);
-  }
-#pragma unroll
-  for (int t = 0; t < 8; ++t) {
-    const float d = z[t][t];
-    const bool badj = !(d > 0.f) || !isfinite(d);
-    first_bad = (first_bad == 0 && badj) ? (J + t + 1) : first_bad;
-  }
-  // this row's z (for the panel rows this reproduces the block's values)
-  float zi[8];
-#pragma unroll
-  for (int t = 0; t < 8; ++t) {
-    float v = a[J + t];
-#pragma unroll
-    for (int u = 0; u < t; ++u) v = fmaf(-M[t][u], zi[u], v);
-    zi[t] = v;
-    a[J + t] = v;
-  }
-  if constexpr (J + 8 < 32) {
-    zb[2 * lane] = make_float4(zi[0], zi[1], zi[2], zi[3]);
-    zb[2 * lane + 1] = make_float4(zi[4], zi[5], zi[6], zi[7]);
-    float m[8];
-#pragma unroll
-    for (int t = 0; t < 8; ++t) m[t] = zi[t] * iv[t];
-    __syncwarp();
-    // the next panel's columns first, then publish them
-#pragma unroll
-    for (int k = J + 8; k < 32; ++k) {
-      const float4 lo = zb[2 * k], hi = zb[2 * k + 1];
-      const float zk[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-      float v = a[k];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) v = fmaf(-m[t], zk[t], v);
-      a[k] = v;
-      if (k == J + 15) {
-        yb[2 * lane] = make_float4(a[J + 8], a[J + 9], a[J + 10], a[J + 11]);
-        yb[2 * lane + 1] = make_float4(a[J + 12], a[J + 13], a[J + 14], a[J + 15]);
-      }
-    }
-  }
-}
-
-__device__ __forceinline__ int leaf_factor8(float* S, float* rinv, float* LTl, float4* yb,
-                                            float4* zb, int c0, int lane) {
-  float a[32];
-#pragma unroll
-  for (int k = 0; k < 32; ++k) a[k] = (k <= lane) ? S[(c0 + lane) * kDP + c0 + k] : 0.f;
-  int first_bad = 0;
-  yb[2 * lane] = make_float4(a[0], a[1], a[2], a[3]);
-  yb[2 * lane + 1] = make_float4(a[4], a[5], a[6], a[7]);
-  leaf_step8<0>(a, yb, zb, lane, first_bad);
-  leaf_step8<8>(a, yb, zb, lane, first_bad);
-  leaf_step8<16>(a, yb, zb, lane, first_bad);
-  leaf_step8<24>(a, yb, zb, lane, first_bad);
-  if (first_bad) return first_bad;
-  // L_ik = a_ik / sqrt(d_k), L_kk = sqrt(d_k)
-  float dd = 1.f;
-#pragma unroll
-  for (int k = 0; k < 32; ++k)
-    if (k == lane) dd = a[k];
-  const float rs = __frsqrt_rn(dd);
-  rinv[c0 + lane] = rs;
-  const float lkk = __fsqrt_rn(dd);
-#pragma unroll
-  for (int k = 0; k < 32; ++k) {
-    const float rk = __shfl_sync(0xffffffffu, rs, k);
-    const float l = (k < lane) ? a[k] * rk : ((k == lane) ? lkk : 0.f);
-    if (k <= lane) S[(c0 + lane) * kDP + c0 + k] = l;
-    LTl[k * kTP + lane] = l;   // zero above the diagonal of the transpose
-  }
-  return 0;
-}
-
 // One warp: column `lane` of the inverse of the 32 x 32 lower leaf at
 // (c0, c0) of S, written as row `lane` of LiT: LiT[lane][m] = Li[m][lane].
 __device__ __forceinline__ void leaf_inverse(const float* S, const float* rinv, float* LiT,
@@ -286,9 +184,9 @@ __device__ __forceinline__ void chol_diag_body(const float* __restrict__ A, int 
   XT = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(XT) + 15) & ~uintptr_t(15));
   float* LTl = XT + 32 * kXP;        // [32][kTP]   current leaf, transposed
   float* rinv = LTl + 32 * kTP;      // [128]       1 / L_kk
-  float4* yb = reinterpret_cast<float4*>(rinv + 128);  // [64] leaf panel rows
-  float4* zb = yb + 64;                                 // [64] leaf z values
-  volatile int* fail = reinterpret_cast<volatile int*>(zb + 64);
+  float4* yb = reinterpret_cast<float4*>(rinv + 128);  // [32] leaf panel rows
+  float4* zb = yb + 32;                                 // [32] leaf z values
+  volatile int* fail = reinterpret_cast<volatile int*>(zb + 32);
   const int kb = p * 128;
   const int bs = min(128, n - kb);
   const int lane = tid & 31, warp = tid >> 5;
