@@ -434,8 +434,8 @@ __global__ void __launch_bounds__(kPg2Threads, 1)
   constexpr int32_t kTimeout = kInfoTimeout;
   PersistCta cta;
   cta.init(smem_raw, a.limit_ns);
-  volatile int* abort_flag = cta.abort_flag;
-  volatile int* skip_flag = cta.task_slot + 1;
+  volatile int* abort_flag = cta.abort_flag();
+  volatile int* skip_flag = cta.skip_slot();
   const uint64_t kLimit = a.limit_ns;
   const int nblk = a.nblk, n = a.n;
   uint32_t* tile = a.ctr + 1;
@@ -662,13 +662,11 @@ cudaError_t launch_cholesky_inverse(const float* H, int64_t n64, float percdamp,
                                   (int)sg_smem_bytes(reduce))) != cudaSuccess)
       return e;
   }
-  // Widths that are a multiple of 128 below the two-level width, called
-  // without a side stream: one persistent launch.  With a side stream the
-  // launch-by-launch form with its look-ahead is used: at n = 4096 it
-  // measured 1.88 ms against 1.96 ms for the persistent form (and 2.03 ms
-  // for the launch-by-launch form without the side stream).
-  const bool ahead_possible = nblk > 2 && side_s != nullptr && side_s != s;
-  const bool persist = reduce && n % kPanel == 0 && nblk >= 3 && npan == 1 && !ahead_possible;
+  // Widths that are a multiple of 128 below the two-level width: one
+  // persistent launch, with or without a side stream (at n = 4096 it measured
+  // 1.856 ms against 1.898 ms for the launch-by-launch form with its
+  // look-ahead stream); other widths launch panel by panel.
+  const bool persist = reduce && n % kPanel == 0 && nblk >= 3 && npan == 1;
   if (persist) {
     if ((e = cudaMemsetAsync(w.ctr, 0, chol_ctr_bytes(n64), s)) != cudaSuccess) return e;
     const WaitGate pg = current_wait_gate();

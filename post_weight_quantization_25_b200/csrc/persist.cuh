@@ -32,84 +32,101 @@ __device__ __forceinline__ void persist_abort(volatile int* abort_flag, int32_t*
 
 static_assert(kPg2QStages == 2, "the Q ring's last-load parities are two scalars");
 
+// The update pipeline's state, kept in shared memory between tasks so that it
+// holds no registers while a CTA runs other kinds of task.
+struct PgPipeState {
+  int p_loads;        // P blocks loaded (= consumed: the producer and the MMA agree after a task)
+  int qst;            // Q ring stage
+  uint32_t qph;
+  int acc;            // TMEM accumulator
+  uint32_t aph;
+  int q_last0, q_last1;  // parity of the last load into Q stage 0 / 1 (-1: none yet)
+  int last_pempty;    // parity of the last commit on pempty (-1: none yet)
+};
+
 struct PersistCta {
   uint8_t* smem;  // 1024-aligned; the update's buffers, free between tasks
-  uint8_t* sP;
-  uint8_t* sQ;
-  uint8_t* sOut;
-  uint64_t *pfull, *pempty, *qfull, *qempty, *tfull, *tempty, *drain;
   uint32_t tmem_base;
-  volatile int* abort_flag;
-  volatile int* task_slot;
   uint64_t limit;
-  // pipeline state, each field kept by the thread of its role
-  int p_loads;       // producer: P blocks loaded; MMA: P blocks consumed
-  int qst;           // producer / MMA: Q ring stage
-  uint32_t qph;
-  int acc;           // MMA / epilogue: TMEM accumulator
-  uint32_t aph;
-  int q_last0, q_last1;  // producer: parity of the last load into Q stage 0 / 1
-  int last_pempty;   // MMA: parity of its last commit on pempty
+
+  // the regions and barriers (fixed offsets from smem)
+  __device__ __forceinline__ uint8_t* sP() const { return smem; }
+  __device__ __forceinline__ uint8_t* sQ() const { return smem + kPg2PBytes; }
+  __device__ __forceinline__ uint8_t* sOut() const {
+    return smem + kPg2PBytes + kPg2QStages * kPg2QStageBytes;
+  }
+  __device__ __forceinline__ uint64_t* bars() const {
+    return reinterpret_cast<uint64_t*>(sOut() + 8 * kPg2StageOut);
+  }
+  __device__ __forceinline__ uint64_t* pfull() const { return bars(); }
+  __device__ __forceinline__ uint64_t* pempty() const { return bars() + 1; }
+  __device__ __forceinline__ uint64_t* qfull(int q) const { return bars() + 2 + q; }
+  __device__ __forceinline__ uint64_t* qempty(int q) const { return bars() + 2 + kPg2QStages + q; }
+  __device__ __forceinline__ uint64_t* tfull(int c) const { return bars() + 2 + 2 * kPg2QStages + c; }
+  __device__ __forceinline__ uint64_t* tempty(int c) const {
+    return bars() + 4 + 2 * kPg2QStages + c;
+  }
+  __device__ __forceinline__ uint64_t* drain() const { return bars() + 6 + 2 * kPg2QStages; }
+  __device__ __forceinline__ uint32_t* tmem_slot() const {
+    return reinterpret_cast<uint32_t*>(bars() + 7 + 2 * kPg2QStages);
+  }
+  __device__ __forceinline__ volatile int* abort_flag() const {
+    return reinterpret_cast<volatile int*>(tmem_slot() + 1);
+  }
+  // two words the kernels use to broadcast thread 0's decisions
+  __device__ __forceinline__ volatile int* task_slot() const { return abort_flag() + 1; }
+  __device__ __forceinline__ volatile int* skip_slot() const { return abort_flag() + 2; }
+  __device__ __forceinline__ PgPipeState* state() const {
+    return reinterpret_cast<PgPipeState*>(sOut() + 8 * kPg2StageOut + 128);
+  }
 
   // Every thread: carve shared memory, initialise the barriers, allocate TMEM.
   __device__ __forceinline__ void init(uint8_t* smem_raw, uint64_t limit_ns) {
+    static_assert(sizeof(PgPipeState) <= 128, "the pipeline state fits its slot");
     smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                       ~static_cast<uintptr_t>(1023));
-    sP = smem;
-    sQ = smem + kPg2PBytes;
-    sOut = sQ + kPg2QStages * kPg2QStageBytes;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + 8 * kPg2StageOut);
-    pfull = bars;
-    pempty = bars + 1;
-    qfull = bars + 2;
-    qempty = qfull + kPg2QStages;
-    tfull = qempty + kPg2QStages;
-    tempty = tfull + 2;
-    drain = tempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-    abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    task_slot = abort_flag + 1;
     limit = limit_ns;
-    p_loads = 0;
-    qst = 0;
-    qph = 0;
-    acc = 0;
-    aph = 0;
-    q_last0 = q_last1 = -1;
-    last_pempty = -1;
     const int tid = threadIdx.x, warp = tid >> 5;
     if (tid == 0) {
-      ptx::mbar_init(pfull, 1);
-      ptx::mbar_init(pempty, 1);
+      ptx::mbar_init(pfull(), 1);
+      ptx::mbar_init(pempty(), 1);
       for (int q = 0; q < kPg2QStages; ++q) {
-        ptx::mbar_init(&qfull[q], 1);
-        ptx::mbar_init(&qempty[q], 1);
+        ptx::mbar_init(qfull(q), 1);
+        ptx::mbar_init(qempty(q), 1);
       }
       for (int c = 0; c < 2; ++c) {
-        ptx::mbar_init(&tfull[c], 1);
-        ptx::mbar_init(&tempty[c], 256);
+        ptx::mbar_init(tfull(c), 1);
+        ptx::mbar_init(tempty(c), 256);
       }
-      ptx::mbar_init(drain, 1);
-      *abort_flag = 0;
+      ptx::mbar_init(drain(), 1);
+      *abort_flag() = 0;
+      PgPipeState* st = state();
+      st->p_loads = 0;
+      st->qst = 0;
+      st->qph = 0;
+      st->acc = 0;
+      st->aph = 0;
+      st->q_last0 = st->q_last1 = -1;
+      st->last_pempty = -1;
       ptx::fence_mbar_init();
     }
     if (warp == 1) {
-      ptx::tmem_alloc(tmem_slot, kPg2TmemCols);
+      ptx::tmem_alloc(tmem_slot(), kPg2TmemCols);
       ptx::tmem_relinquish();
     }
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    tmem_base = *tmem_slot;
+    tmem_base = *tmem_slot();
   }
 
   // Every thread: the next task index (taken by thread 0), or -1 once the
   // CTA should stop (no task left, or an abort).
   __device__ __forceinline__ int next_task(uint32_t* counter, int total) {
-    if (threadIdx.x == 0) *task_slot = (int)atomicAdd(counter, 1u);
+    if (threadIdx.x == 0) *task_slot() = (int)atomicAdd(counter, 1u);
     __syncthreads();
-    const int t = *task_slot;
-    const bool stop = *abort_flag != 0;
+    const int t = *task_slot();
+    const bool stop = *abort_flag() != 0;
     __syncthreads();
     return (t >= total || stop) ? -1 : t;
   }
@@ -124,6 +141,21 @@ struct PersistCta {
                                          int32_t timeout_code) {
     constexpr uint64_t kDrainLimit = (uint64_t)kGridWaitLimitNs;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    volatile int* abort_flag = this->abort_flag();
+    uint8_t* sP = this->sP();
+    uint8_t* sQ = this->sQ();
+    uint8_t* sOut = this->sOut();
+    uint64_t* pfull = this->pfull();
+    uint64_t* pempty = this->pempty();
+    uint64_t* qfull = this->qfull(0);
+    uint64_t* qempty = this->qempty(0);
+    uint64_t* tfull = this->tfull(0);
+    uint64_t* tempty = this->tempty(0);
+    uint64_t* drain = this->drain();
+    PgPipeState* stp = state();
+    int p_loads = stp->p_loads, qst = stp->qst, acc = stp->acc;
+    uint32_t qph = stp->qph, aph = stp->aph;
+    int q_last0 = stp->q_last0, q_last1 = stp->q_last1, last_pempty = stp->last_pempty;
     if (warp == 0) {
       if (lane == 0) {
         // producer: P (all of K = 128), then Q per tile
@@ -165,6 +197,8 @@ struct PersistCta {
           if (q_last0 >= 0) ptx::mbar_wait_bounded(&qfull[0], (uint32_t)q_last0, &never, kDrainLimit);
           if (q_last1 >= 0) ptx::mbar_wait_bounded(&qfull[1], (uint32_t)q_last1, &never, kDrainLimit);
         }
+        stp->q_last0 = q_last0;
+        stp->q_last1 = q_last1;
       }
     } else if (warp == 1) {
       if (lane == 0) {
@@ -221,6 +255,13 @@ struct PersistCta {
           volatile int never = 0;
           ptx::mbar_wait_bounded(drain, 0, &never, kDrainLimit);
         }
+        // the state after the task (the producer's ring and P counts agree)
+        stp->p_loads = p_loads;
+        stp->qst = qst;
+        stp->qph = qph;
+        stp->acc = acc;
+        stp->aph = aph;
+        stp->last_pempty = last_pempty;
       }
     } else {
       // epilogue: warps 2 .. 9
@@ -257,9 +298,10 @@ struct PersistCta {
   __device__ __forceinline__ void teardown() {
     constexpr uint64_t kDrainLimit = (uint64_t)kGridWaitLimitNs;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int last_pempty = state()->last_pempty;
     if (warp == 1 && lane == 0 && last_pempty >= 0) {
       volatile int never = 0;
-      ptx::mbar_wait_bounded(pempty, (uint32_t)last_pempty, &never, kDrainLimit);
+      ptx::mbar_wait_bounded(pempty(), (uint32_t)last_pempty, &never, kDrainLimit);
     }
     ptx::tc_fence_before();
     __syncthreads();

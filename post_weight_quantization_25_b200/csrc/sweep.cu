@@ -735,7 +735,7 @@ __global__ void __launch_bounds__(kPg2Threads, 1)
   PersistCta cta;
   cta.init(smem_raw, a.limit_ns);
   uint8_t* smem = cta.smem;
-  volatile int* abort_flag = cta.abort_flag;
+  volatile int* abort_flag = cta.abort_flag();
   const uint64_t kLimit = a.limit_ns;
   uint32_t* swept = a.ctr + 1;
   uint32_t* applied = a.ctr + 1 + a.RB;
