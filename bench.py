@@ -32,7 +32,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-SYRK_REV = "syrk-pair-v2-ordered"   # the SYRK kernel the committed traffic figure belongs to
+SYRK_REV = "syrk-pair-v3-ordered-red"   # the SYRK kernel the committed traffic figure belongs to
 METRIC = "weights quantized/sec (GPTQ 4-bit g128) + Hessian TFLOP/s, % of roofline, 1×B200"
 UNIT = "weights/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}

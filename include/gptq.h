@@ -112,7 +112,7 @@ gptq_status gptq_workspace_size(int op, int64_t rows, int64_t n, int64_t ntok, g
  *          inside the kernel gave up (then H is incomplete).  Not cleared.
  * The result is reproducible bit for bit: the tokens are cut into chunks
  * (for parallelism) and the chunks of each output tile are added into H in
- * chunk order, never by atomics.  Calls that overlap on the GPU must not
+ * chunk order, one chunk at a time.  Calls that overlap on the GPU must not
  * share a workspace or an H. */
 gptq_status gptq_hessian_accumulate(float* H, const void* X, gptq_dtype xt, int64_t n,
                                     int64_t ntok, int64_t ldx, int token_major, float alpha,

@@ -28,11 +28,13 @@
 //    IEEE adds.  At the end of the unit it adds alpha * tile into H, masked
 //    to the upper triangle (the split-K reduction).
 //  * Ordered split-K reduction: the token chunks of a tile are added into H
-//    in chunk order, not by atomics.  A per-tile counter in global memory
-//    (a turnstile) holds how many chunks have been added; the unit of chunk
-//    c waits (acquire) until it reads c, adds its tile with plain loads and
-//    stores through L2, and publishes c + 1 (release).  So H is the same bit
-//    for bit from run to run.  Units are walked in chunk-major order by a
+//    in chunk order.  A per-tile counter in global memory (a turnstile) holds
+//    how many chunks have been added; the unit of chunk c waits (acquire)
+//    until it reads c, adds its tile by reductions in L2 (red.add, which
+//    return nothing, so the epilogue does not wait on L2 round trips), makes
+//    them visible (fence) and publishes c + 1 (release).  Only one chunk adds
+//    into a tile at a time, so every element takes its adds in chunk order
+//    and H is the same bit for bit from run to run.  Units are walked in chunk-major order by a
 //    persistent grid whose CTAs are all resident, so chunk c - 1 of a tile is
 //    always taken before chunk c and the wait ends.
 //  * No multicast loads.  Every wait is bounded: on timeout the CTA stops,
@@ -116,6 +118,10 @@ __device__ __forceinline__ bool ordered_add(float* H, int n, int row, int cbase,
   ok = ptx::named_bar_and(kEpiBar, kEpiThreads, ok);
   if (!ok) return false;
   if (row < n) {
+    // reductions in L2 (no value comes back, so nothing waits on a round
+    // trip); the turnstile lets one unit at a time add into the tile, so each
+    // element still takes its chunks' adds one after another in chunk order,
+    // each an IEEE round-to-nearest fp32 add
     float* hrow = H + (int64_t)row * n;
 #pragma unroll
     for (int j4 = 0; j4 < 32; ++j4) {
@@ -126,20 +132,15 @@ __device__ __forceinline__ bool ordered_add(float* H, int n, int row, int cbase,
       const float f2 = alpha * tile[4 * j4 + 2];
       const float f3 = alpha * tile[4 * j4 + 3];
       if (vec4 && c >= row && c + 3 < n) {
-        float4* p = reinterpret_cast<float4*>(hrow + c);
-        float4 h = __ldcg(p);
-        h.x += f0;
-        h.y += f1;
-        h.z += f2;
-        h.w += f3;
-        __stcg(p, h);
+        atomicAdd(reinterpret_cast<float4*>(hrow + c), make_float4(f0, f1, f2, f3));
       } else {
         const float fv[4] = {f0, f1, f2, f3};
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          if (c + i >= row && c + i < n) __stcg(hrow + c + i, __ldcg(hrow + c + i) + fv[i]);
+          if (c + i >= row && c + i < n) atomicAdd(hrow + c + i, fv[i]);
       }
     }
+    __threadfence();   // this thread's reductions are performed before the release below
   }
   // every thread's stores are done before the next chunk may start
   ptx::named_bar_sync(kEpiBar, kEpiThreads);
@@ -362,7 +363,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 //    cluster barriers order set-up and tear-down.
 // Tiles (I2, J) with I2 <= J cover the upper triangle in 256 x 256 blocks.
 // Accuracy handling is the single-CTA kernel's: fresh TMEM sums every
-// kSubKb k-blocks, added in an fp32 register tile, split-K atomics per unit.
+// kSubKb k-blocks, added in an fp32 register tile, the ordered split-K add per unit.
 // ===========================================================================
 constexpr int P_STAGES = 6;
 constexpr int P_A_BYTES = 128 * BK * 2;   // this CTA's A rows
