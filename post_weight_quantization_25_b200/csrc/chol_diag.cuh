@@ -34,7 +34,9 @@ constexpr size_t kDiagSmemBytes =
     sizeof(float) * (128 * kDP + 32 * kXP + 32 * kTP + 128 + 256) + 16 + 16;  // + the fail flag
 
 // Outputs of chol_diag_kernel, in the Cholesky workspace:
-//   Lt[k][c]     = L[c][k]           (128 x 128, zero for k > c)
+//   Lt[k][c]     = L[c][k]           (128 x 128; only the 32 x 32 blocks with
+//                                     block(k) < block(c) are written, the
+//                                     ones the apply reads)
 //   LiT[j][t][c] = (L_jj^-1)[c][t]   (4 leaves of 32 x 32, zero for t > c)
 constexpr int kDiagOutFloats = 128 * 128 + 4 * 32 * 32;
 
@@ -323,19 +325,28 @@ __device__ __forceinline__ void chol_diag_body(const float* __restrict__ A, int 
     diag_sync(bar);
   }
 
-  // ---- outputs: L transposed, then the four leaf inverses
+  // ---- outputs: the four leaf inverses (warps 0-3) beside the blocks of
+  // L transposed that the apply reads (warps 4-7): the six 32 x 32 blocks
+  // (kb, jb), kb < jb, of Lt (rows k of block kb, columns c of block jb);
+  // the rest of Lt is never read and is not written
   float* Lt = out;
   float* LiT = out + 128 * 128;
-  for (int f = tid; f < 128 * 32; f += kDiagThreads) {
-    const int k = f >> 5, c = (f & 31) * 4;
-    float4 o;
-    o.x = (k <= c + 0) ? S[(c + 0) * kDP + k] : 0.f;
-    o.y = (k <= c + 1) ? S[(c + 1) * kDP + k] : 0.f;
-    o.z = (k <= c + 2) ? S[(c + 2) * kDP + k] : 0.f;
-    o.w = (k <= c + 3) ? S[(c + 3) * kDP + k] : 0.f;
-    reinterpret_cast<float4*>(Lt)[f] = o;
+  if (warp < 4) {
+    leaf_inverse(S, rinv, LiT + warp * 32 * 32, 32 * warp, lane);
+  } else {
+    for (int f = tid - 128; f < 6 * 32 * 8; f += kDiagThreads - 128) {
+      const int b = f >> 8, r = (f >> 3) & 31, q = f & 7;
+      const int kb = b < 3 ? 0 : (b < 5 ? 1 : 2);
+      const int jb = b < 3 ? b + 1 : (b < 5 ? b - 1 : 3);
+      const int k = 32 * kb + r, c = 32 * jb + 4 * q;   // k < c: below the diagonal of L
+      float4 o;
+      o.x = S[(c + 0) * kDP + k];
+      o.y = S[(c + 1) * kDP + k];
+      o.z = S[(c + 2) * kDP + k];
+      o.w = S[(c + 3) * kDP + k];
+      *reinterpret_cast<float4*>(Lt + k * 128 + c) = o;
+    }
   }
-  if (warp < 4) leaf_inverse(S, rinv, LiT + warp * 32 * 32, 32 * warp, lane);
 }
 
 __global__ void __launch_bounds__(kDiagThreads) chol_diag_kernel(const float* __restrict__ A,
@@ -376,9 +387,18 @@ __device__ __forceinline__ void panel_apply_body(
   const int nA = n - kb - bs;
   const int nvec = nA + kb + bs;
   if (v0 >= nvec) return;
-  // everything staged with async copies, all in flight at once
-  for (int f = tid; f < kDiagOutFloats / 4; f += kApplyThreads)
-    ptx::cp_async_16(asmem + 4 * f, diag_out + 4 * f);
+  // everything staged with async copies, all in flight at once.  Of L^T only
+  // the six 32 x 32 blocks (kb, jb), kb < jb, are read (stage jb takes rows
+  // k < 32 jb of its columns); the inverted leaves in full
+  for (int f = tid; f < 6 * 32 * 8; f += kApplyThreads) {
+    const int b = f >> 8, r = (f >> 3) & 31, q = f & 7;
+    const int kb = b < 3 ? 0 : (b < 5 ? 1 : 2);
+    const int jb = b < 3 ? b + 1 : (b < 5 ? b - 1 : 3);
+    const int off = (32 * kb + r) * 128 + 32 * jb + 4 * q;
+    ptx::cp_async_16(asmem + off, diag_out + off);
+  }
+  for (int f = tid; f < 4 * 32 * 32 / 4; f += kApplyThreads)
+    ptx::cp_async_16(LiT + 4 * f, diag_out + 128 * 128 + 4 * f);
   if ((n % 4) == 0) {
     // rows start 16-byte aligned and bs is a multiple of 4: 16-byte copies
     for (int f = tid; f < kApplyVecs * 32; f += kApplyThreads) {
