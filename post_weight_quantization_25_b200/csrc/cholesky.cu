@@ -856,6 +856,7 @@ void* g_scratch_addr[kNoAllocMaxDevices] = {};
 extern "C" gptq_status gptq_cholesky_inverse_noalloc(const float* H, int64_t n, float percdamp,
                                                      int actorder, float* U, int32_t* perm,
                                                      uint8_t* dead, int32_t* info, void* stream) {
+  const gptq::NvtxScope nvtx("gptq_cholesky_inverse_noalloc");
   if (!H || !U || !dead || !info || n <= 0) return GPTQ_ERR_INVALID_ARG;
   if (actorder && !perm) return GPTQ_ERR_INVALID_ARG;
   if (!(percdamp >= 0.f)) return GPTQ_ERR_INVALID_ARG;

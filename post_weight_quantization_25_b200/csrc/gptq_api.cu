@@ -179,6 +179,7 @@ gptq_status gptq_workspace_size(int op, int64_t rows, int64_t n, int64_t ntok, g
 gptq_status gptq_hessian_accumulate(float* H, const void* X, gptq_dtype xt, int64_t n,
                                     int64_t ntok, int64_t ldx, int token_major, float alpha,
                                     void* ws, size_t ws_bytes, int32_t* info, void* stream) {
+  const gptq::NvtxScope nvtx("gptq_hessian_accumulate");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!H || n <= 0 || n > kMaxN || ntok < 0 || ldx < ntok) return GPTQ_ERR_INVALID_ARG;
   if (xt != GPTQ_BF16 && xt != GPTQ_F32) return GPTQ_ERR_INVALID_ARG;
@@ -219,6 +220,7 @@ gptq_status gptq_hessian_accumulate(float* H, const void* X, gptq_dtype xt, int6
 gptq_status gptq_cholesky_inverse(const float* H, int64_t n, float percdamp, int actorder,
                                   float* U, int32_t* perm, uint8_t* dead, int32_t* info,
                                   void* ws, size_t ws_bytes, void* stream, void* side_stream) {
+  const gptq::NvtxScope nvtx("gptq_cholesky_inverse");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!H || !U || !dead || !info || n <= 0 || n > kMaxN) return GPTQ_ERR_INVALID_ARG;
   if (actorder && !perm) return GPTQ_ERR_INVALID_ARG;
@@ -235,6 +237,7 @@ gptq_status gptq_quantize_layer(const void* W, gptq_dtype wt, int64_t rows, int6
                                 uint8_t* zeros, int32_t* g_idx, float* Wq, float* row_loss,
                                 void* ws, size_t ws_bytes, int32_t* info, void* stream,
                                 void* side_stream) {
+  const gptq::NvtxScope nvtx("gptq_quantize_layer");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const gptq_status st = check_cfg(cfg);
   if (st != GPTQ_OK) return st;
@@ -252,6 +255,7 @@ gptq_status gptq_quantize_layer(const void* W, gptq_dtype wt, int64_t rows, int6
 
 gptq_status gptq_pack_int4(const uint8_t* codes, int64_t rows, int64_t n, uint32_t* out,
                            void* stream) {
+  const gptq::NvtxScope nvtx("gptq_pack_int4");
   if (rows < 0 || n <= 0 || n % 8 != 0) return GPTQ_ERR_INVALID_ARG;
   if (rows == 0) return GPTQ_OK;
   if (!codes || !out || !aligned(out, 4)) return GPTQ_ERR_INVALID_ARG;
@@ -260,6 +264,7 @@ gptq_status gptq_pack_int4(const uint8_t* codes, int64_t rows, int64_t n, uint32
 
 gptq_status gptq_pack_int3(const uint8_t* codes, int64_t rows, int64_t n, uint32_t* out,
                            void* stream) {
+  const gptq::NvtxScope nvtx("gptq_pack_int3");
   if (rows < 0 || n <= 0 || n % 32 != 0) return GPTQ_ERR_INVALID_ARG;
   if (rows == 0) return GPTQ_OK;
   if (!codes || !out || !aligned(out, 4)) return GPTQ_ERR_INVALID_ARG;
@@ -270,6 +275,7 @@ gptq_status gptq_dequant(const uint32_t* packed, int bits, int64_t rows, int64_t
                          const float* scales, const uint8_t* zeros, int group_size,
                          int64_t n_groups, const int32_t* g_idx, void* out, gptq_dtype ot,
                          void* stream) {
+  const gptq::NvtxScope nvtx("gptq_dequant");
   if (bits != 3 && bits != 4) return GPTQ_ERR_UNSUPPORTED;
   if (rows < 0 || n <= 0) return GPTQ_ERR_INVALID_ARG;
   if ((bits == 4 && n % 8) || (bits == 3 && n % 32)) return GPTQ_ERR_INVALID_ARG;
@@ -290,6 +296,7 @@ gptq_status gptq_dequant_matvec(const uint32_t* packed, int bits, int64_t rows, 
                                 int64_t n_groups, const int32_t* g_idx, const int32_t* perm,
                                 const void* x, gptq_dtype xt, int64_t batch, float* y,
                                 void* ws, size_t ws_bytes, void* stream) {
+  const gptq::NvtxScope nvtx("gptq_dequant_matvec");
   if (bits != 3 && bits != 4) return GPTQ_ERR_UNSUPPORTED;
   if (rows < 0 || n <= 0 || batch < 0) return GPTQ_ERR_INVALID_ARG;
   if ((bits == 4 && n % 8) || (bits == 3 && n % 32)) return GPTQ_ERR_INVALID_ARG;
@@ -313,6 +320,7 @@ gptq_status gptq_dequant_matvec(const uint32_t* packed, int bits, int64_t rows, 
 
 gptq_status gptq_gather_columns_u8(const uint8_t* src, int64_t rows, int64_t n,
                                    const int32_t* perm, uint8_t* dst, void* stream) {
+  const gptq::NvtxScope nvtx("gptq_gather_columns_u8");
   if (rows < 0 || n <= 0 || n > kMaxN) return GPTQ_ERR_INVALID_ARG;
   if (rows == 0) return GPTQ_OK;
   if (!src || !perm || !dst || src == dst) return GPTQ_ERR_INVALID_ARG;
@@ -343,12 +351,14 @@ static gptq_status hadamard_common(bool cols, const void* in, gptq_dtype it, int
 gptq_status gptq_hadamard_rows(const void* in, gptq_dtype it, int64_t rows, int64_t n,
                                int64_t ld_in, const float* signs, int block, void* out,
                                gptq_dtype ot, int64_t ld_out, void* stream) {
+  const gptq::NvtxScope nvtx("gptq_hadamard_rows");
   return hadamard_common(false, in, it, rows, n, n, ld_in, signs, block, out, ot, ld_out, stream);
 }
 
 gptq_status gptq_hadamard_cols(const void* in, gptq_dtype it, int64_t n, int64_t ntok,
                                int64_t ld_in, const float* signs, int block, void* out,
                                gptq_dtype ot, int64_t ld_out, void* stream) {
+  const gptq::NvtxScope nvtx("gptq_hadamard_cols");
   return hadamard_common(true, in, it, n, ntok, n, ld_in, signs, block, out, ot, ld_out, stream);
 }
 

@@ -6,6 +6,7 @@
 #include <mutex>
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/gptq.h"
 
@@ -13,6 +14,17 @@ namespace gptq {
 
 constexpr int kBlock = 128;            // lazy-update block of the sweep / Cholesky panel
 constexpr int kGridWaitLimitNs = 1000000000;  // 1 s: upper bound of any in-kernel wait
+
+// NVTX range around one C-ABI call (host side: the call's argument checks
+// and enqueue; the kernels it enqueues show up under it in a profiler's
+// timeline).  NVTX is header-only; without a tool attached a push or pop is a
+// check of a null hook and costs a few nanoseconds.
+struct NvtxScope {
+  explicit NvtxScope(const char* name) { nvtxRangePushA(name); }
+  ~NvtxScope() { nvtxRangePop(); }
+  NvtxScope(const NvtxScope&) = delete;
+  NvtxScope& operator=(const NvtxScope&) = delete;
+};
 
 int num_sms();
 // 2-D TMA descriptor (128-byte swizzle, zero fill out of bounds) for a
