@@ -539,3 +539,60 @@ class LayerPipeline:
     def check_info(self) -> None:
         for q in self.layers:
             q.check_info()
+
+
+# ----------------------------------------------------------------- checkpoint / resume
+# Page "GPTQ, with the code open", section "From one repair to a whole model":
+# a model is quantized one layer at a time, each from its own inputs.  For a
+# long run over many linears, each finished linear's stored result is written
+# to its own file, and a restarted run skips the linears whose files exist.
+
+STORED_KEYS = ("packed", "scales", "zeros", "g_idx", "perm")
+
+
+def save_quantized(path: str, outputs: dict, meta: dict) -> None:
+    """Write one linear's stored result (host copies of ``STORED_KEYS`` and
+    ``meta``) to ``path``.  The file appears only once it is complete: it is
+    written under a temporary name and renamed, so an interrupted run leaves
+    no partial result that a resumed run would take for a finished one."""
+    import os
+    blob = {k: outputs[k].detach().cpu() for k in STORED_KEYS if outputs.get(k) is not None}
+    blob["meta"] = dict(meta)
+    tmp = path + ".partial"
+    torch.save(blob, tmp)
+    os.replace(tmp, path)
+
+
+def load_quantized(path: str) -> dict:
+    return torch.load(path, map_location="cpu", weights_only=True)
+
+
+def quantize_linears(names, quantize, out_dir: str, resume: bool = True) -> list:
+    """Quantize the linears ``names`` in order with ``quantize(name) ->
+    (outputs, meta)`` (``outputs`` holds at least ``packed``, ``scales`` and
+    ``zeros`` of that linear), storing each under ``out_dir/<name>.pt``.  With
+    ``resume``, a linear whose file already exists is not quantized again.
+    Returns the names quantized by this call."""
+    import os
+    os.makedirs(out_dir, exist_ok=True)
+    done = []
+    for name in names:
+        path = os.path.join(out_dir, f"{name}.pt")
+        if resume and os.path.exists(path):
+            continue
+        outputs, meta = quantize(name)
+        save_quantized(path, outputs, meta)
+        done.append(name)
+    return done
+
+
+def layer_quantizer_outputs(lq: "LayerQuantizer") -> tuple:
+    """(outputs, meta) of a LayerQuantizer after ``run``, for
+    quantize_linears: checks ``info`` first (a failed linear is not stored)."""
+    lq.check_info()
+    outputs = {"packed": lq.packed, "scales": lq.scales, "zeros": lq.zeros,
+               "g_idx": lq.g_idx if lq.actorder else None,
+               "perm": lq.perm if lq.actorder else None}
+    meta = {"rows": lq.rows, "n": lq.n, "bits": lq.bits, "group_size": lq.group_size,
+            "actorder": bool(lq.actorder), "percdamp": lq.percdamp}
+    return outputs, meta
