@@ -55,7 +55,7 @@ def parse_args():
                    help="skip the short runs of the other large workloads")
     p.add_argument("--no-lookahead", action="store_true",
                    help="run the factorisation and the sweep on one stream")
-    p.add_argument("--only", choices=["dequant_matvec", "hadamard", "pipeline"], default=None,
+    p.add_argument("--only", choices=["dequant_matvec", "hadamard", "pipeline", "stack"], default=None,
                    help="run one consumer-side measurement alone and print its JSON "
                         "(for profiling; not the benchmark line)")
     return p.parse_args()
@@ -298,7 +298,9 @@ def measure_dequant_matvec(G, dev, packed, bits, n, scales, zeros, group_size, g
            and (group_size <= 0 or (group_size >= 32 and group_size & (group_size - 1) == 0)))
     return {"shape": label, "order": "sweep (perm)" if perm is not None else
             ("original (g_idx)" if g_idx is not None else "original"),
-            "kernel": "tensor-core (mma.sync)" if mma else "fp32 pipe",
+            "kernel": "tensor-core (mma.sync)" if mma else (
+                "row-per-lane fp32 pipe (g_idx)"
+                if g_idx is not None and n % (32 if bits == 4 else 128) == 0 else "fp32 pipe"),
             "batch": batch, "bits": bits, "us": round(t * 1e6, 2),
             "bytes": nbytes, "gbs": round(gbs, 1), "peak_gbs": pk["hbm_gbs"],
             "frac": round(gbs / pk["hbm_gbs"], 4), "l2": "flushed (256 MiB read) before each launch"}
@@ -324,7 +326,7 @@ def _codes_70b(dev):
 
 def measure_dequant_70b(G, dev):
     """The fused dequant x activation on the 70B down-proj shape: codes in
-    original order with g_idx (FP32-pipe kernel) and in sweep order with perm
+    original order with g_idx (row-per-lane FP32-pipe kernel) and in sweep order with perm
     (tensor-core kernel), 1 and 8 activation vectors."""
     pk7, sc7, z7, pm7, gi7 = _codes_70b(dev)
     n7 = 28672
@@ -451,6 +453,57 @@ def measure_pipeline(G, dev, reps=3):
     res["speedup"] = round(res["one_stream"]["ms"] / res["overlapped"]["ms"], 3)
     del pipe, Ws, Xs
     return res
+
+
+def measure_stack(G, dev, blocks=32):
+    """The 7B-shaped decoder stack: 32 blocks x 7 linears (q, k, v, o
+    4096x4096; gate, up 11008x4096; down 4096x11008), bf16 N(0, 0.02^2)
+    weights, one seeded X of 65536 tokens N(0,1) per linear, 4-bit g128,
+    quantized linear after linear on one stream.  Each block's inputs are
+    drawn on the device before its timed run (drawing is not timed); the
+    stack's time is the sum of the 32 blocks' CUDA-event times.  Block 0 runs
+    once untimed first (warm-up)."""
+    import torch
+    import workloads
+    shapes = [(r, n) for _, r, n in workloads.STACK_7B_LINEARS]
+    ntok = 65536
+    pipe = G.LayerPipeline(shapes, ntok, bits=4, group_size=128, device=dev)
+
+    def inputs(b):
+        wls = [workloads.stack_7b_workload(b, l, ntok) for l in range(len(shapes))]
+        return ([workloads.make_weights(wl, dev) for wl in wls],
+                [workloads.make_calibration(wl, dev) for wl in wls])
+
+    Ws, Xs = inputs(0)
+    pipe.run(Ws, Xs)
+    torch.cuda.synchronize()
+    ts = []
+    for b in range(blocks):
+        del Ws, Xs
+        Ws, Xs = inputs(b)
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        a.record()
+        pipe.run(Ws, Xs)
+        e.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(e))
+    pipe.check_info()
+    del Ws, Xs, pipe
+    torch.cuda.empty_cache()
+    nw = blocks * sum(r * n for r, n in shapes)
+    flops = blocks * sum(float(n) * (n + 1) * ntok for _, n in shapes)
+    total = sum(ts)
+    return {"workload": "stack_7b: %d blocks x 7 linears (q,k,v,o 4096x4096; gate,up "
+                        "11008x4096; down 4096x11008) bf16, X 65536 tokens per linear, "
+                        "4-bit g128, one stream" % blocks,
+            "linears": blocks * len(shapes), "weights": nw, "ms_total": round(total, 2),
+            "weights_per_s": nw / (total / 1e3),
+            "block_ms": {"min": round(min(ts), 3), "median": round(statistics.median(ts), 3),
+                         "max": round(max(ts), 3)},
+            "hessian_flops_total": flops,
+            "note": "sum of per-block CUDA-event times; inputs drawn between blocks, untimed"}
 
 
 # ----------------------------------------------------------------- per-stage rooflines
@@ -694,6 +747,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.empty_cache()
         extra = {name: extra_workload(G, name, dev, stream)
                  for name in ("down_proj_7b", "down_proj_70b")}
+        extra["stack_7b"] = measure_stack(G, dev)
         W, X = Wc, Xc
 
     cpu = None
@@ -783,7 +837,7 @@ def main():
         torch.cuda.set_device(dev)
         if rank == 0:
             fn = {"dequant_matvec": measure_dequant_70b, "hadamard": measure_hadamard,
-                  "pipeline": measure_pipeline}[args.only]
+                  "pipeline": measure_pipeline, "stack": measure_stack}[args.only]
             print(json.dumps({"only": args.only, "result": fn(G, dev)}), flush=True)
         return
     if world > 1:

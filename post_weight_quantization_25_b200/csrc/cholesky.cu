@@ -142,10 +142,15 @@ __global__ void __launch_bounds__(1024) diag_prep_kernel(const float* __restrict
 // permutation (a NaN diagonal is reported through info anyway).
 __device__ __forceinline__ float rank_key(float d) { return isnan(d) ? -INFINITY : d; }
 
+// Eight threads (consecutive lanes) count for each key, over every eighth
+// other key, and their counts are summed: a CTA of 256 threads ranks 32 keys.
+constexpr int kRankSplit = 8;
+constexpr int kRankKeysPerCta = 256 / kRankSplit;
 __global__ void __launch_bounds__(256) actorder_rank_kernel(const float* __restrict__ dprime,
                                                             int n, int32_t* __restrict__ perm) {
   __shared__ float keys[2048];
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const int i = blockIdx.x * kRankKeysPerCta + threadIdx.x / kRankSplit;
+  const int sub = threadIdx.x % kRankSplit;
   const float ki = (i < n) ? rank_key(dprime[i]) : 0.f;
   int pos = 0;
   for (int t0 = 0; t0 < n; t0 += 2048) {
@@ -153,14 +158,16 @@ __global__ void __launch_bounds__(256) actorder_rank_kernel(const float* __restr
     for (int j = threadIdx.x; j < cnt; j += blockDim.x) keys[j] = rank_key(dprime[t0 + j]);
     __syncthreads();
     if (i < n) {
-      for (int j = 0; j < cnt; ++j) {
+      for (int j = sub; j < cnt; j += kRankSplit) {
         const float kj = keys[j];
         pos += (kj > ki) || (kj == ki && t0 + j < i);
       }
     }
     __syncthreads();
   }
-  if (i < n) perm[pos] = i;
+#pragma unroll
+  for (int o = 1; o < kRankSplit; o <<= 1) pos += __shfl_xor_sync(0xffffffffu, pos, o);
+  if (i < n && sub == 0) perm[pos] = i;
 }
 
 __global__ void iota_kernel(int32_t* __restrict__ perm, int n) {
@@ -603,7 +610,8 @@ cudaError_t launch_cholesky_inverse(const float* H, int64_t n64, float percdamp,
   note_launch();
   int32_t* perm_used = nullptr;
   if (actorder) {
-    actorder_rank_kernel<<<(n + 255) / 256, 256, 0, s>>>(w.dprime, n, perm);
+    actorder_rank_kernel<<<(n + kRankKeysPerCta - 1) / kRankKeysPerCta, 256, 0, s>>>(w.dprime, n,
+                                                                                   perm);
     note_launch();
     perm_used = perm;
   } else if (perm) {

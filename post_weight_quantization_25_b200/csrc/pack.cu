@@ -321,6 +321,265 @@ __global__ void __launch_bounds__(kMvThreads) dequant_matvec_kernel(
   }
 }
 
+// ---------------------------------------------------------------------------
+// The same product for codes in the ORIGINAL column order with a per-column
+// group index g_idx (act-order layers stored without re-ordering).  Here the
+// 8 columns of a code word belong to unrelated groups, so every weight needs
+// its own (scale, zero) and the per-group factoring of the tensor-core
+// kernel does not apply.  The cost is then the ruler lookup, and the layout
+// below makes it one conflict-free shared-memory read per weight:
+//   * lane = row: a warp owns 32 rows and walks columns; the column (hence
+//     its group g_idx[c] and its activations) is the same for every lane, so
+//     those reads are broadcasts, and lane l reads the ruler of row l,
+//     group g at rul[l * rpitch + g] with an odd pitch (distinct banks);
+//   * a CTA is 8 warps on the same 32 rows, each warp taking 128 of every
+//     1024-column chunk; each warp stages its 32 x 128 codes with coalesced
+//     16-byte cp.async copies, double-buffered (the next chunk's codes load
+//     while this one's are used); piece k of row l sits in slot
+//     k ^ ((l >> 1) & 3) of the row's four 16-byte slots, so that the lanes'
+//     16-byte reads of their own rows do not conflict;
+//   * w_hat = scale * (q - zero) as one fp32 multiply of the exact q - zero,
+//     formed as (2^23 + q) - (2^23 + zero) from the code's bits;
+//   * each lane keeps 4 interleaved partial sums per vector (column k of a
+//     code word goes to sum k % 4), the 8 warps' sums meet in shared memory
+//     in a fixed order: y is the same from run to run.
+// Requires packed 16-byte aligned, n % 32 == 0 (int4) or n % 128 == 0
+// (int3), so that every staged piece is a whole, aligned 16 bytes.
+constexpr int kGxWarps = 8;
+constexpr int kGxChunk = 1024;
+constexpr int kGxSlice = kGxChunk / kGxWarps;     // 128 columns per warp per chunk
+constexpr int kGxPitchW = 16;                     // code tile row pitch in words (64 B)
+constexpr int kGxTileWords = 32 * kGxPitchW;
+constexpr int64_t kGxMaxRulerBytes = 112 * 1024;  // staged rulers per CTA; past that, L1
+
+template <int B>
+__host__ __device__ constexpr size_t gx_fixed_bytes() {
+  return sizeof(uint32_t) * kGxWarps * 2 * kGxTileWords + 2 * sizeof(float) * B * kGxChunk +
+         2 * sizeof(int) * kGxChunk + sizeof(float) * kGxWarps * B * 32;
+}
+constexpr int kGxPer = kGxChunk / (kGxWarps * 32);  // columns of a chunk each thread stages
+
+template <int BITS, int B, bool XBF16, bool STAGED>
+__global__ void __launch_bounds__(kGxWarps * 32) dequant_matvec_gidx_kernel(
+    const uint32_t* __restrict__ packed, int64_t rows, int64_t n,
+    const float* __restrict__ scales, const uint8_t* __restrict__ zeros, int64_t G, int rpitch,
+    const int32_t* __restrict__ g_idx, const void* __restrict__ x, int64_t ldx,
+    float* __restrict__ y, int64_t ldy) {
+  extern __shared__ __align__(16) uint32_t gx_smem[];
+  uint32_t* tiles = gx_smem;                                               // [warp][2][32][pitch]
+  float* xs2 = reinterpret_cast<float*>(tiles + kGxWarps * 2 * kGxTileWords);  // [2][B][chunk]
+  int* gs2 = reinterpret_cast<int*>(xs2 + 2 * B * kGxChunk);              // [2][chunk]
+  float* red = reinterpret_cast<float*>(gs2 + 2 * kGxChunk);              // [warp][B][32]
+  float2* rul = reinterpret_cast<float2*>(red + kGxWarps * B * 32);      // [32][rpitch]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row0 = (int64_t)blockIdx.x * 32;
+  const int64_t r = row0 + lane;
+  const int64_t wpr = n * BITS / 32;  // packed words per row
+  constexpr int kWords = kGxSlice * BITS / 32;   // words of a row per slice: 16 or 12
+  constexpr int kPieces = kWords / 4;            // 16-byte pieces per row: 4 or 3
+  constexpr float kMagic = 8388608.f;            // 2^23
+  if (STAGED) {
+    // the CTA's rows' rulers are contiguous in scales / zeros: element i of
+    // that range is (row i / G, group i % G); four loads in flight per thread
+    const int Gi = (int)G, tot = 32 * Gi;
+    const int64_t live = (min(rows - row0, (int64_t)32)) * G;
+    const float* sbase = scales + row0 * G;
+    const uint8_t* zbase = zeros + row0 * G;
+    for (int i0 = threadIdx.x; i0 < tot; i0 += 4 * kGxWarps * 32) {
+      float sv[4], zv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * kGxWarps * 32;
+        const bool ok = i < live;
+        sv[u] = ok ? __ldg(sbase + i) : 0.f;
+        zv[u] = ok ? (float)__ldg(zbase + i) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * kGxWarps * 32;
+        if (i < tot) {
+          const int rr = i / Gi;
+          rul[rr * rpitch + (i - rr * Gi)] = make_float2(sv[u], kMagic + zv[u]);
+        }
+      }
+    }
+  }
+  const float* srow = scales + min(r, rows - 1) * G;
+  const uint8_t* zrow = zeros + min(r, rows - 1) * G;
+  // stage this warp's slice of chunk c0 into buffer buf
+  auto stage_codes = [&](int64_t c0, int buf) {
+    uint32_t* t = tiles + (warp * 2 + buf) * kGxTileWords;
+    const int64_t col = c0 + (int64_t)warp * kGxSlice;
+#pragma unroll
+    for (int k = 0; k < kPieces; ++k) {
+      const int i = lane + 32 * k;
+      const int rr = i / kPieces, part = i % kPieces;
+      const int64_t pc = col + (int64_t)part * (128 / kPieces);  // first column of the piece
+      const bool ok = row0 + rr < rows && pc < n;
+      const uint32_t* src = ok ? packed + (row0 + rr) * wpr + col * BITS / 32 + 4 * part : packed;
+      ptx::cp_async_16z(t + rr * kGxPitchW + 4 * (part ^ ((rr >> 1) & 3)), src, ok ? 16 : 0);
+    }
+  };
+  // this thread's columns i = tid + 256 j of a chunk: activations and groups
+  // are loaded into registers one chunk ahead and stored after the chunk's
+  // work, so their load latency hides behind it
+  float xr[kGxPer][B];
+  int gr[kGxPer];
+  auto load_side = [&](int64_t c0) {
+#pragma unroll
+    for (int j = 0; j < kGxPer; ++j) {
+      const int64_t c = c0 + threadIdx.x + kGxWarps * 32 * j;
+      const bool ok = c < n;
+      gr[j] = ok ? __ldg(g_idx + c) : 0;
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        const int64_t xi = (int64_t)b * ldx + (ok ? c : 0);
+        xr[j][b] = !ok ? 0.f
+                 : XBF16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(x)[xi])
+                         : __ldg(static_cast<const float*>(x) + xi);
+      }
+    }
+  };
+  auto store_side = [&](int sb) {
+#pragma unroll
+    for (int j = 0; j < kGxPer; ++j) {
+      const int i = threadIdx.x + kGxWarps * 32 * j;
+      gs2[sb * kGxChunk + i] = gr[j];
+#pragma unroll
+      for (int b = 0; b < B; ++b) xs2[(sb * B + b) * kGxChunk + i] = xr[j][b];
+    }
+  };
+  float acc[B][4];
+#pragma unroll
+  for (int b = 0; b < B; ++b)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[b][k] = 0.f;
+  stage_codes(0, 0);
+  ptx::cp_async_commit();
+  load_side(0);
+  store_side(0);
+  int buf = 0;
+  for (int64_t c0 = 0; c0 < n; c0 += kGxChunk, buf ^= 1) {
+    const int cn = (int)min((int64_t)kGxChunk, n - c0);
+    const bool more = c0 + kGxChunk < n;
+    __syncwarp();  // every lane is done reading the tile the next copies overwrite
+    if (more) {
+      stage_codes(c0 + kGxChunk, buf ^ 1);
+      load_side(c0 + kGxChunk);
+    }
+    ptx::cp_async_commit();
+    ptx::cp_async_wait<1>();  // this thread's pieces of chunk c0 have landed
+    __syncthreads();          // ... and every other thread's, with chunk c0's xs and gs
+    const float* xs = xs2 + buf * B * kGxChunk;
+    const int* gs = gs2 + buf * kGxChunk;
+    const uint32_t* t = tiles + (warp * 2 + buf) * kGxTileWords + lane * kGxPitchW;
+    uint32_t w[kWords];
+#pragma unroll
+    for (int k = 0; k < kPieces; ++k) {
+      const uint4 v = *reinterpret_cast<const uint4*>(t + 4 * (k ^ ((lane >> 1) & 3)));
+      w[4 * k] = v.x;
+      w[4 * k + 1] = v.y;
+      w[4 * k + 2] = v.z;
+      w[4 * k + 3] = v.w;
+    }
+    const int cb0 = warp * kGxSlice;
+    const float2* rrow = rul + lane * rpitch;
+#pragma unroll
+    for (int u = 0; u < kGxSlice / 8; ++u) {
+      const int cb = cb0 + 8 * u;
+      if (cb >= cn) break;  // warp-uniform (n % 32 == 0: whole units)
+      uint32_t bits24;
+      if (BITS == 4) {
+        bits24 = w[u];
+      } else {
+        const int j = u >> 2;
+        bits24 = (u & 3) == 0 ? w[3 * j]
+               : (u & 3) == 1 ? __funnelshift_r(w[3 * j], w[3 * j + 1], 24)
+               : (u & 3) == 2 ? __funnelshift_r(w[3 * j + 1], w[3 * j + 2], 16)
+                              : (w[3 * j + 2] >> 8);
+      }
+      const int4 ga = *reinterpret_cast<const int4*>(gs + cb);
+      const int4 gb = *reinterpret_cast<const int4*>(gs + cb + 4);
+      const int gi[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+      float wq[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float2 sz = STAGED ? rrow[gi[k]] : make_float2(__ldg(srow + gi[k]),
+                                                             kMagic + (float)__ldg(zrow + gi[k]));
+        const float q = __uint_as_float(0x4B000000u | ((bits24 >> (BITS * k)) & ((1u << BITS) - 1u)));
+        wq[k] = __fmul_rn(sz.x, q - sz.y);
+      }
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        const float4 xa = *reinterpret_cast<const float4*>(xs + b * kGxChunk + cb);
+        const float4 xb = *reinterpret_cast<const float4*>(xs + b * kGxChunk + cb + 4);
+        acc[b][0] = fmaf(wq[0], xa.x, acc[b][0]);
+        acc[b][1] = fmaf(wq[1], xa.y, acc[b][1]);
+        acc[b][2] = fmaf(wq[2], xa.z, acc[b][2]);
+        acc[b][3] = fmaf(wq[3], xa.w, acc[b][3]);
+        acc[b][0] = fmaf(wq[4], xb.x, acc[b][0]);
+        acc[b][1] = fmaf(wq[5], xb.y, acc[b][1]);
+        acc[b][2] = fmaf(wq[6], xb.z, acc[b][2]);
+        acc[b][3] = fmaf(wq[7], xb.w, acc[b][3]);
+      }
+    }
+    // the next chunk's side buffer: last read during the previous chunk, which
+    // every thread finished before this chunk's barrier
+    if (more) store_side(buf ^ 1);
+  }
+  ptx::cp_async_wait_all();
+#pragma unroll
+  for (int b = 0; b < B; ++b)
+    red[(warp * B + b) * 32 + lane] = (acc[b][0] + acc[b][1]) + (acc[b][2] + acc[b][3]);
+  __syncthreads();
+  // fixed-order sum over the 8 warps: thread (b, l) for b < B
+  if (threadIdx.x < B * 32) {
+    const int b = threadIdx.x >> 5, l = threadIdx.x & 31;
+    float v[kGxWarps];
+#pragma unroll
+    for (int k = 0; k < kGxWarps; ++k) v[k] = red[(k * B + b) * 32 + l];
+    const float s = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+    if (row0 + l < rows) y[(int64_t)b * ldy + row0 + l] = s;
+  }
+}
+
+template <int BITS, int B>
+void gx_launch(const uint32_t* packed, int64_t rows, int64_t n, const float* scales,
+               const uint8_t* zeros, int64_t G, const int32_t* g_idx, const void* x, int x_bf16,
+               int64_t ldx, float* y, int64_t ldy, cudaStream_t s) {
+  static_assert(kGxWarps == 8, "the fixed-order sum is written for 8 warps");
+  const unsigned grid = (unsigned)((rows + 31) / 32);
+  const int rpitch = (int)(G | 1);
+  const int64_t rb = (int64_t)32 * rpitch * 8;
+  const bool staged = rb <= kGxMaxRulerBytes;
+  const size_t dyn = gx_fixed_bytes<B>() + (staged ? (size_t)rb : 0);
+#define GX_GO(XB, ST)                                                                          \
+  {                                                                                            \
+    auto k = dequant_matvec_gidx_kernel<BITS, B, XB, ST>;                                      \
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);           \
+    k<<<grid, kGxWarps * 32, dyn, s>>>(packed, rows, n, scales, zeros, G, rpitch, g_idx, x, ldx, \
+                                       y, ldy);                                                \
+  }
+  if (x_bf16) {
+    if (staged) GX_GO(true, true) else GX_GO(true, false)
+  } else {
+    if (staged) GX_GO(false, true) else GX_GO(false, false)
+  }
+#undef GX_GO
+  note_launch();
+}
+template <int BITS>
+void gx_batch(int b, const uint32_t* packed, int64_t rows, int64_t n, const float* scales,
+              const uint8_t* zeros, int64_t G, const int32_t* g_idx, const void* x, int x_bf16,
+              int64_t ldx, float* y, int64_t ldy, cudaStream_t s) {
+  switch (b) {
+    case 8: gx_launch<BITS, 8>(packed, rows, n, scales, zeros, G, g_idx, x, x_bf16, ldx, y, ldy, s); break;
+    case 4: gx_launch<BITS, 4>(packed, rows, n, scales, zeros, G, g_idx, x, x_bf16, ldx, y, ldy, s); break;
+    case 2: gx_launch<BITS, 2>(packed, rows, n, scales, zeros, G, g_idx, x, x_bf16, ldx, y, ldy, s); break;
+    default: gx_launch<BITS, 1>(packed, rows, n, scales, zeros, G, g_idx, x, x_bf16, ldx, y, ldy, s); break;
+  }
+}
+
 unsigned blocks_for(int64_t total, int threads) { return (unsigned)((total + threads - 1) / threads); }
 
 }  // namespace
@@ -825,13 +1084,21 @@ cudaError_t launch_dequant_matvec(const uint32_t* packed, int bits, int64_t rows
     return cudaGetLastError();
   }
   const size_t esz = x_bf16 ? 2 : 4;
+  // original column order with g_idx: the row-per-lane kernel, where its
+  // 16-byte staging applies
+  const bool gx = g_idx && reinterpret_cast<uintptr_t>(packed) % 16 == 0 &&
+                  (bits == 4 ? n % 32 == 0 : n % 128 == 0);
   // batches of 8, 4, 2, 1 vectors per launch
   for (int64_t b0 = 0; b0 < batch;) {
     const int64_t left = batch - b0;
     const int b = left >= 8 ? 8 : left >= 4 ? 4 : left >= 2 ? 2 : 1;
     const void* xb = static_cast<const char*>(x) + (size_t)b0 * (size_t)n * esz;
     float* yb = y + b0 * rows;
-    if (bits == 4)
+    if (gx && bits == 4)
+      gx_batch<4>(b, packed, rows, n, scales, zeros, n_groups, g_idx, xb, x_bf16, n, yb, rows, s);
+    else if (gx)
+      gx_batch<3>(b, packed, rows, n, scales, zeros, n_groups, g_idx, xb, x_bf16, n, yb, rows, s);
+    else if (bits == 4)
       mv_batch<4>(b, packed, rows, n, scales, zeros, group_size, n_groups, g_idx, perm, xb,
                   x_bf16, n, yb, rows, s);
     else

@@ -9,7 +9,8 @@
   streams interleave.
 - gptq_dequant_matvec (tensor cores): the two column halves of every output
   meet by two atomic adds onto zero; fp32 addition of two terms commutes, so y
-  is the same whichever half lands first.
+  is the same whichever half lands first.  The g_idx (original order) kernel
+  sums each output's partial sums over its warps in a fixed order.
 """
 import numpy as np
 import pytest
@@ -52,6 +53,14 @@ def test_dequant_matvec_is_repeatable(bits, rows, n, g, batch):
     x = torch.randn(batch, n, device="cuda").to(torch.bfloat16)
     ys = [G.gptq_dequant_matvec(packed, bits, n, scales, zeros, x, g, perm=perm)
           for _ in range(4)]
+    # the same codes in original order with a g_idx (row-per-lane kernel)
+    gidx = torch.randint(0, n // g, (n,), device="cuda", dtype=torch.int32)
+    ys += [G.gptq_dequant_matvec(packed, bits, n, scales, zeros, x, g, g_idx=gidx)
+           for _ in range(3)]
+    torch.cuda.synchronize()
+    for y in ys[5:]:
+        assert torch.equal(y, ys[4])
+    ys = ys[:4]
     torch.cuda.synchronize()
     for y in ys[1:]:
         assert torch.equal(y, ys[0])

@@ -49,7 +49,12 @@ def test_pack_and_dequant_bit_exact(bits, rows, n, g, use_gidx):
 @pytest.mark.parametrize("bits,rows,n,g,use_gidx,batch,xdt", [
     (4, 7, 64, 16, False, 1, torch.float32), (4, 33, 256, 128, True, 3, torch.bfloat16),
     (4, 130, 1032, -1, False, 8, torch.bfloat16), (3, 9, 96, 32, False, 2, torch.float32),
-    (3, 17, 2080, 128, True, 11, torch.bfloat16), (4, 1, 8, -1, False, 1, torch.float32)])
+    (3, 17, 2080, 128, True, 11, torch.bfloat16), (4, 1, 8, -1, False, 1, torch.float32),
+    # original order with g_idx on the row-per-lane kernel: several 1024-column
+    # chunks with a ragged last one, rows past a 32-row tile, fp32 and bf16 x,
+    # int3 (n % 128 == 0), and 512 groups (rulers read through L1, not staged)
+    (4, 70, 1056, 32, True, 8, torch.float32), (3, 45, 2176, 64, True, 5, torch.bfloat16),
+    (4, 40, 2048, 4, True, 2, torch.bfloat16), (4, 33, 3072, 128, True, 1, torch.bfloat16)])
 def test_dequant_matvec_matches_oracle(bits, rows, n, g, use_gidx, batch, xdt):
     """y = x w_hat^T with w_hat dequantized on the fly, within mv_bound."""
     rng = np.random.default_rng(bits * 7 + n + batch)
@@ -74,7 +79,9 @@ def test_dequant_matvec_matches_oracle(bits, rows, n, g, use_gidx, batch, xdt):
 def mv_bound(n, mag):
     """Rounding bound of gptq_dequant_matvec against the fp64 product with
     binary32 w_hat.  FP32-pipe kernel: each lane sums n/32 rounded FMA terms,
-    then five shuffle levels.  Tensor-core kernel (int4, bf16 x): the products
+    then five shuffle levels.  Row-per-lane g_idx kernel: each of a lane's
+    four partial sums takes n/32 rounded FMA terms (8 warps share the
+    columns), then two levels over the four sums and three over the warps.  Tensor-core kernel (int4, bf16 x): the products
     (q - zero) x are exact; at most 8 MMA accumulations of 16 products per
     128-column slice (<= 16 roundings, internal order unknown), one FMA by the
     scale, n/512 slice sums per warp, 3 levels over 8 warps, plus one rounding

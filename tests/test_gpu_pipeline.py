@@ -62,3 +62,30 @@ def test_pipeline_runs_again_with_new_inputs():
         torch.cuda.synchronize()
         for q, (W, X) in zip(pipe.layers, layers):
             compare_layer(_outputs(q), W, X, 4, 128, 0.01, False)
+
+
+def test_stack_run_stores_each_linear_and_resumes(tmp_path):
+    """quantize_linears with LayerQuantizer: each stored file holds exactly the
+    device outputs of its linear, and a second call quantizes nothing."""
+    ntok = 512
+    shapes = {"l0": (40, 256), "l1": (33, 384)}
+    inputs = {name: workloads.random_layer(r, n, ntok, seed=70 + i, dtype=torch.bfloat16)
+              for i, (name, (r, n)) in enumerate(shapes.items())}
+    kept = {}
+
+    def quantize(name):
+        r, n = shapes[name]
+        q = G.LayerQuantizer(r, n, ntok, bits=4, group_size=128, actorder=True)
+        W, X = inputs[name]
+        q.run(W.cuda(), device_x(X))
+        torch.cuda.synchronize()
+        kept[name] = q
+        return G.layer_quantizer_outputs(q)
+
+    assert G.quantize_linears(list(shapes), quantize, str(tmp_path)) == list(shapes)
+    for name, q in kept.items():
+        blob = G.load_quantized(str(tmp_path / f"{name}.pt"))
+        for k in ("packed", "scales", "zeros", "g_idx", "perm"):
+            assert torch.equal(blob[k], getattr(q, k).cpu())
+        assert blob["meta"]["rows"] == shapes[name][0] and blob["meta"]["actorder"]
+    assert G.quantize_linears(list(shapes), quantize, str(tmp_path)) == []
