@@ -249,15 +249,42 @@ __global__ void __launch_bounds__(256) gather_w_kernel(
   __shared__ float red[2][8];
   const int r = blockIdx.x;
   const T* src = W + (int64_t)r * n;
-  for (int j = threadIdx.x; j < n; j += blockDim.x) wrow[j] = dead[j] ? 0.f : (float)src[j];
+  // 16-byte loads of W (with the matching dead flags) and 4-column outputs
+  // when the rows allow it (the same values either way)
+  constexpr int VI = 16 / (int)sizeof(T);
+  const bool vin = n % VI == 0 && reinterpret_cast<uintptr_t>(src) % 16 == 0 &&
+                   reinterpret_cast<uintptr_t>(dead) % VI == 0;
+  if (vin) {
+    for (int j = threadIdx.x; j < n / VI; j += blockDim.x) {
+      const uint4 raw = reinterpret_cast<const uint4*>(src)[j];
+      const T* e = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+      for (int i = 0; i < VI; ++i) wrow[VI * j + i] = dead[VI * j + i] ? 0.f : (float)e[i];
+    }
+  } else {
+    for (int j = threadIdx.x; j < n; j += blockDim.x) wrow[j] = dead[j] ? 0.f : (float)src[j];
+  }
   __syncthreads();
   float mn = INFINITY, mx = -INFINITY;
   float* dst = Wf + (int64_t)r * n;
-  for (int k = threadIdx.x; k < n; k += blockDim.x) {
-    const float v = wrow[perm ? perm[k] : k];
-    dst[k] = v;
-    mn = fminf(mn, v);
-    mx = fmaxf(mx, v);
+  const bool vout = n % 4 == 0 && reinterpret_cast<uintptr_t>(dst) % 16 == 0 &&
+                    (!perm || reinterpret_cast<uintptr_t>(perm) % 16 == 0);
+  if (vout) {
+    for (int k4 = threadIdx.x; k4 < n / 4; k4 += blockDim.x) {
+      const int4 k = perm ? reinterpret_cast<const int4*>(perm)[k4]
+                          : make_int4(4 * k4, 4 * k4 + 1, 4 * k4 + 2, 4 * k4 + 3);
+      const float4 v = make_float4(wrow[k.x], wrow[k.y], wrow[k.z], wrow[k.w]);
+      reinterpret_cast<float4*>(dst)[k4] = v;
+      mn = fminf(fminf(mn, fminf(v.x, v.y)), fminf(v.z, v.w));
+      mx = fmaxf(fmaxf(mx, fmaxf(v.x, v.y)), fmaxf(v.z, v.w));
+    }
+  } else {
+    for (int k = threadIdx.x; k < n; k += blockDim.x) {
+      const float v = wrow[perm ? perm[k] : k];
+      dst[k] = v;
+      mn = fminf(mn, v);
+      mx = fmaxf(mx, v);
+    }
   }
   if (per_row) {
     mn = warp_min(mn);
@@ -835,15 +862,45 @@ __global__ void __launch_bounds__(256) unpermute_kernel(const uint8_t* __restric
   extern __shared__ float srow[];
   uint8_t* crow = reinterpret_cast<uint8_t*>(srow + (Wq ? n : 0));
   const int r = blockIdx.x;
-  for (int j = threadIdx.x; j < n; j += blockDim.x) {
-    crow[j] = codes_sw[(int64_t)r * n + j];
-    if (Wq) srow[j] = Wf[(int64_t)r * n + j];
+  const uint8_t* csrc = codes_sw + (int64_t)r * n;
+  uint8_t* cdst = codes + (int64_t)r * n;
+  float* wdst = Wq ? Wq + (int64_t)r * n : nullptr;
+  // 16-byte staging and 4-column outputs when the rows allow it (same bytes)
+  const bool vin = n % 16 == 0 && reinterpret_cast<uintptr_t>(csrc) % 16 == 0 &&
+                   (!Wq || reinterpret_cast<uintptr_t>(Wf) % 16 == 0);
+  const bool vout = n % 4 == 0 && reinterpret_cast<uintptr_t>(cdst) % 4 == 0 &&
+                    reinterpret_cast<uintptr_t>(pos) % 16 == 0 &&
+                    (!Wq || reinterpret_cast<uintptr_t>(wdst) % 16 == 0);
+  if (vin) {
+    for (int j = threadIdx.x; j < n / 16; j += blockDim.x) {
+      reinterpret_cast<uint4*>(crow)[j] = reinterpret_cast<const uint4*>(csrc)[j];
+      if (Wq)
+        for (int q = 0; q < 4; ++q)
+          reinterpret_cast<float4*>(srow)[4 * j + q] =
+              reinterpret_cast<const float4*>(Wf + (int64_t)r * n)[4 * j + q];
+    }
+  } else {
+    for (int j = threadIdx.x; j < n; j += blockDim.x) {
+      crow[j] = csrc[j];
+      if (Wq) srow[j] = Wf[(int64_t)r * n + j];
+    }
   }
   __syncthreads();
-  for (int c = threadIdx.x; c < n; c += blockDim.x) {
-    const int k = pos[c];
-    codes[(int64_t)r * n + c] = crow[k];
-    if (Wq) Wq[(int64_t)r * n + c] = srow[k];
+  if (vout) {
+    for (int c4 = threadIdx.x; c4 < n / 4; c4 += blockDim.x) {
+      const int4 k = reinterpret_cast<const int4*>(pos)[c4];
+      reinterpret_cast<uint32_t*>(cdst)[c4] = (uint32_t)crow[k.x] | ((uint32_t)crow[k.y] << 8) |
+                                              ((uint32_t)crow[k.z] << 16) |
+                                              ((uint32_t)crow[k.w] << 24);
+      if (Wq)
+        reinterpret_cast<float4*>(wdst)[c4] = make_float4(srow[k.x], srow[k.y], srow[k.z], srow[k.w]);
+    }
+  } else {
+    for (int c = threadIdx.x; c < n; c += blockDim.x) {
+      const int k = pos[c];
+      cdst[c] = crow[k];
+      if (Wq) wdst[c] = srow[k];
+    }
   }
 }
 
