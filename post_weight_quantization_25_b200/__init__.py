@@ -420,6 +420,8 @@ class LayerQuantizer:
         self.ws_q = _workspace(gptq_workspace_size(GPTQ_OP_QUANTIZE, rows, n, 0, w_dtype,
                                                    self.cfg), dev, None)
         self._pack = gptq_pack_int4 if bits == 4 else gptq_pack_int3
+        self.x_dtype, self.w_dtype = x_dtype, w_dtype
+        self._stage = None        # run_streamed: two device staging buffers, device W, events
 
     def hessian(self, X: torch.Tensor, stream, mark=None) -> None:
         """H = 0, H += 2 X X^T on `stream`; mark(0) / mark(1) around the
@@ -451,6 +453,64 @@ class LayerQuantizer:
                      self.g_idx, self.deq.dtype, out=self.deq, stream=stream)
         if mark:
             mark(5)
+
+    def run_streamed(self, W_host: torch.Tensor, X_batches, stream=None):
+        """The whole layer from inputs in (pinned) host memory: W and the
+        calibration batches X_b (each n x N_b, contiguous) are copied in on a
+        copy stream while H accumulates batch by batch on ``stream`` (page
+        "GPTQ, with the code open", section "Paper vs. code": H is a sum over
+        calibration batches), so the host-to-device copies overlap the
+        Hessian.  Two device staging buffers of the largest batch take turns;
+        a buffer is refilled only after the accumulation that read it.  The
+        result equals ``run`` on the concatenated X up to the fp32 order of
+        the Hessian's sums."""
+        s = torch.cuda.current_stream() if stream is None else stream
+        dev = self.H.device
+        if len(X_batches) == 0:
+            raise GptqError("no calibration batch")
+        for Xb in X_batches:
+            if Xb.dim() != 2 or Xb.shape[0] != self.n or not Xb.is_contiguous() \
+                    or Xb.dtype != self.x_dtype:
+                raise GptqError("each batch must be a contiguous n x N_b tensor of the layer's "
+                                "input dtype")
+        if W_host.shape != (self.rows, self.n) or W_host.dtype != self.w_dtype:
+            raise GptqError("W must be rows x n in the layer's weight dtype")
+        nb = max(int(Xb.shape[1]) for Xb in X_batches)
+        st = self._stage
+        if st is None or st["cap"] < nb:
+            st = {"cap": nb,
+                  "buf": [torch.empty(self.n * nb, dtype=self.x_dtype, device=dev)
+                          for _ in range(2)],
+                  "W": torch.empty(self.rows, self.n, dtype=self.w_dtype, device=dev),
+                  "copy": torch.cuda.Stream(dev),
+                  "ev_start": torch.cuda.Event(), "ev_w": torch.cuda.Event(),
+                  "ev_copied": [torch.cuda.Event(), torch.cuda.Event()],
+                  "ev_used": [torch.cuda.Event(), torch.cuda.Event()]}
+            self._stage = st
+        cs = st["copy"]
+        # the copy stream starts after everything already queued on s (the
+        # previous run's reads of the staging buffers and of W among it)
+        st["ev_start"].record(s)
+        cs.wait_event(st["ev_start"])
+        with torch.cuda.stream(cs):
+            st["W"].copy_(W_host, non_blocking=True)
+        st["ev_w"].record(cs)
+        with torch.cuda.stream(s):
+            self.H.zero_()
+        for i, Xb in enumerate(X_batches):
+            slot = i % 2
+            if i >= 2:
+                cs.wait_event(st["ev_used"][slot])
+            dst = st["buf"][slot][: self.n * Xb.shape[1]].view(self.n, Xb.shape[1])
+            with torch.cuda.stream(cs):
+                dst.copy_(Xb, non_blocking=True)
+            st["ev_copied"][slot].record(cs)
+            s.wait_event(st["ev_copied"][slot])
+            gptq_hessian_accumulate(self.H, dst, 2.0, ws=self.ws_h, info=self.info_h, stream=s)
+            st["ev_used"][slot].record(s)
+        s.wait_event(st["ev_w"])
+        self.finish(st["W"], s)
+        return self
 
     def run(self, W: torch.Tensor, X: torch.Tensor, stream=None, events=None):
         s = torch.cuda.current_stream() if stream is None else stream
