@@ -705,7 +705,7 @@ def run_ours(args, rank, world, local_rank):
         # sequences (32768 tokens), each a contiguous pinned n x 32768 tensor;
         # run_streamed copies them in on a copy stream while H accumulates
         nbatch = max(1, N // 32768)
-        bt = (N + nbatch - 1) // nbatch
+        bt = ((N + nbatch - 1) // nbatch + 7) // 8 * 8   # rows 16-byte aligned
         Xh = [torch.empty(n, min(bt, N - a), dtype=X.dtype).pin_memory()
               for a in range(0, N, bt)]
         for i, xb in enumerate(Xh):
