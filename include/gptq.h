@@ -237,7 +237,12 @@ gptq_status gptq_dequant(const uint32_t* packed, int bits, int64_t rows, int64_t
  * once, and adds the two column halves of every output onto zeros (two
  * terms, so the result does not depend on their order).  It first writes x
  * (gathered by perm, if given) into the workspace as batch x n bf16, and
- * zeroes y.  Everything else: the FP32-pipe kernel, one rounded FMA per term.
+ * zeroes y.  Codes in original order with g_idx (int4 with n % 32 == 0, or
+ * int3 with n % 128 == 0, packed 16-byte aligned): a kernel with one row
+ * per lane, each weight's own (scale, zero) read from shared memory, four
+ * partial sums per lane and vector added over the warps in a fixed order.
+ * Everything else: the FP32-pipe kernel, one rounded FMA per term.  Every
+ * path gives the same y from run to run.
  *   packed, scales, zeros, group_size, n_groups, g_idx: exactly as for
  *          gptq_dequant (same layout, same single-multiply w_hat).
  *   perm   NULL, or (with g_idx NULL) the sweep order of an act-order layer:

@@ -463,7 +463,14 @@ class LayerQuantizer:
         Hessian.  Two device staging buffers of the largest batch take turns;
         a buffer is refilled only after the accumulation that read it.  The
         result equals ``run`` on the concatenated X up to the fp32 order of
-        the Hessian's sums."""
+        the Hessian's sums.
+
+        Consecutive calls overlap: a call's copies wait only for the last
+        reads of the buffers they overwrite (a staging buffer's previous
+        accumulation, the device W's previous sweep), so they can run while
+        the previous call's factorisation and sweep finish.  The host
+        tensors must stay alive and unchanged until the copies are done (for
+        example until ``stream`` has reached this call's end)."""
         s = torch.cuda.current_stream() if stream is None else stream
         dev = self.H.device
         if len(X_batches) == 0:
@@ -483,15 +490,20 @@ class LayerQuantizer:
                           for _ in range(2)],
                   "W": torch.empty(self.rows, self.n, dtype=self.w_dtype, device=dev),
                   "copy": torch.cuda.Stream(dev),
-                  "ev_start": torch.cuda.Event(), "ev_w": torch.cuda.Event(),
+                  "ev_w": torch.cuda.Event(), "ev_w_free": torch.cuda.Event(),
                   "ev_copied": [torch.cuda.Event(), torch.cuda.Event()],
                   "ev_used": [torch.cuda.Event(), torch.cuda.Event()]}
+            if self._stage is not None:
+                # new buffers: the old ones may still be read on s
+                ev = torch.cuda.Event()
+                ev.record(s)
+                st["copy"].wait_event(ev)
             self._stage = st
         cs = st["copy"]
-        # the copy stream starts after everything already queued on s (the
-        # previous run's reads of the staging buffers and of W among it)
-        st["ev_start"].record(s)
-        cs.wait_event(st["ev_start"])
+        # W is overwritten once the previous call's sweep has read it; each
+        # staging buffer once the accumulation that read it last is done
+        # (events never recorded yet make these waits no-ops)
+        cs.wait_event(st["ev_w_free"])
         with torch.cuda.stream(cs):
             st["W"].copy_(W_host, non_blocking=True)
         st["ev_w"].record(cs)
@@ -499,8 +511,7 @@ class LayerQuantizer:
             self.H.zero_()
         for i, Xb in enumerate(X_batches):
             slot = i % 2
-            if i >= 2:
-                cs.wait_event(st["ev_used"][slot])
+            cs.wait_event(st["ev_used"][slot])
             dst = st["buf"][slot][: self.n * Xb.shape[1]].view(self.n, Xb.shape[1])
             with torch.cuda.stream(cs):
                 dst.copy_(Xb, non_blocking=True)
@@ -510,6 +521,7 @@ class LayerQuantizer:
             st["ev_used"][slot].record(s)
         s.wait_event(st["ev_w"])
         self.finish(st["W"], s)
+        st["ev_w_free"].record(s)
         return self
 
     def run(self, W: torch.Tensor, X: torch.Tensor, stream=None, events=None):

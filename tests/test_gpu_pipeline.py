@@ -94,19 +94,31 @@ def test_stack_run_stores_each_linear_and_resumes(tmp_path):
 def test_streamed_host_batches_match_the_oracle():
     """LayerQuantizer.run_streamed: W and the calibration batches come from
     pinned host memory, the copies overlap the batch-by-batch Hessian; the
-    layer matches the oracle on the concatenated X, on a first call and on
-    a second call with other inputs (staging buffers reused, more batches
-    than buffers)."""
+    layer matches the oracle on the concatenated X.  Then two calls back to
+    back with no synchronisation between them (the second call's copies
+    overlap the first call's factorisation and sweep; staging buffers
+    reused, more batches than buffers): the last call's results match the
+    oracle on its own inputs."""
     r, n = 40, 256
-    for seed, sizes in ((91, [512, 512, 304]), (92, [256, 128, 384, 64])):
+
+    def inputs(seed, sizes):
         W, X = workloads.random_layer(r, n, sum(sizes), seed=seed, dtype=torch.bfloat16,
                                       correlated=0.3)
         cut = np.cumsum([0] + sizes)
         batches = [X[:, a:b].contiguous().pin_memory() for a, b in zip(cut[:-1], cut[1:])]
-        if seed == 91:
-            q = G.LayerQuantizer(r, n, sum(sizes), bits=4, group_size=64, actorder=True,
-                                 want_wq=True, want_loss=True)
-        q.run_streamed(W.pin_memory(), batches)
-        torch.cuda.synchronize()
-        q.check_info()
-        compare_layer(_outputs(q), W, X, 4, 64, 0.01, True)
+        return W, X, W.pin_memory(), batches
+
+    Wa, Xa, Wah, Ba = inputs(91, [512, 512, 304])
+    Wb, Xb, Wbh, Bb = inputs(92, [256, 128, 384, 64])
+    q = G.LayerQuantizer(r, n, 1328, bits=4, group_size=64, actorder=True, want_wq=True,
+                         want_loss=True)
+    q.run_streamed(Wah, Ba)
+    torch.cuda.synchronize()
+    q.check_info()
+    compare_layer(_outputs(q), Wa, Xa, 4, 64, 0.01, True)
+    q.run_streamed(Wbh, Bb)
+    q.run_streamed(Wah, Ba)
+    q.run_streamed(Wbh, Bb)
+    torch.cuda.synchronize()
+    q.check_info()
+    compare_layer(_outputs(q), Wb, Xb, 4, 64, 0.01, True)
