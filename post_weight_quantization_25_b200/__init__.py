@@ -500,15 +500,14 @@ class LayerQuantizer:
                 st["copy"].wait_event(ev)
             self._stage = st
         cs = st["copy"]
-        # W is overwritten once the previous call's sweep has read it; each
-        # staging buffer once the accumulation that read it last is done
-        # (events never recorded yet make these waits no-ops)
-        cs.wait_event(st["ev_w_free"])
-        with torch.cuda.stream(cs):
-            st["W"].copy_(W_host, non_blocking=True)
-        st["ev_w"].record(cs)
+        # each staging buffer is overwritten once the accumulation that read
+        # it last is done, W once the previous call's sweep has read it
+        # (events never recorded yet make these waits no-ops).  W goes after
+        # the first two batches, so that the copy stream does not hold those
+        # behind the previous call's sweep.
         with torch.cuda.stream(s):
             self.H.zero_()
+        w_after = min(1, len(X_batches) - 1)
         for i, Xb in enumerate(X_batches):
             slot = i % 2
             cs.wait_event(st["ev_used"][slot])
@@ -516,6 +515,11 @@ class LayerQuantizer:
             with torch.cuda.stream(cs):
                 dst.copy_(Xb, non_blocking=True)
             st["ev_copied"][slot].record(cs)
+            if i == w_after:
+                cs.wait_event(st["ev_w_free"])
+                with torch.cuda.stream(cs):
+                    st["W"].copy_(W_host, non_blocking=True)
+                st["ev_w"].record(cs)
             s.wait_event(st["ev_copied"][slot])
             gptq_hessian_accumulate(self.H, dst, 2.0, ws=self.ws_h, info=self.info_h, stream=s)
             st["ev_used"][slot].record(s)
