@@ -206,12 +206,14 @@ def test_hessian_zero_tokens_is_a_no_op():
 
 
 # ------------------------------------------------------------------ Cholesky
-# widths that are a multiple of 128 with at least 3 panels (384, 640, 1024,
-# 2048) take the persistent factorisation; the others launch panel by panel
+# widths that are a multiple of 128 with at least 3 panels below 8192 (384,
+# 640, 1024, 2048, 8064) take the persistent factorisation; the others launch
+# panel by panel
 @pytest.mark.parametrize("n,actorder,dead", [(6, False, ()), (130, True, (7,)),
                                              (256, False, ()), (300, True, (0, 299)),
                                              (384, True, ()), (640, True, ()),
-                                             (1024, False, (3, 1000)), (2048, True, ())])
+                                             (1024, False, (3, 1000)), (2048, True, ()),
+                                             (8064, True, (5,))])
 def test_cholesky_inverse_matches_oracle(n, actorder, dead):
     _, X = workloads.random_layer(1, n, 3 * n + 50, seed=n, dead=dead, correlated=0.3)
     Ho32 = O.hessian(to_np(X)).astype(np.float32)          # the oracle's own H, as fp32
@@ -281,6 +283,8 @@ LAYERS = [
     (4, 6, 64, 2, -1, False, torch.float32, ()),
     (1, 130, 300, 4, -1, True, torch.bfloat16, ()),
     (130, 257, 700, 8, 128, True, torch.bfloat16, ()),
+    # the widest layer the persistent factorisation and sweep take (63 panels)
+    (48, 8064, 9000, 4, 128, True, torch.bfloat16, (5,)),
 ]
 
 
