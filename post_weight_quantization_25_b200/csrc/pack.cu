@@ -166,6 +166,71 @@ __global__ void dequant_kernel(const uint32_t* __restrict__ packed, int64_t unit
   }
 }
 
+// The same dequantization with one CTA per row: the row's rulers are staged
+// once in shared memory as (scale, zero) pairs, so each value costs one
+// shared-memory read for its ruler instead of two global ones, and the
+// group index of 8 columns comes in two 16-byte loads.  Same arithmetic and
+// bytes out as dequant_kernel.
+constexpr int kDqRowThreads = 128;
+constexpr int kDqRowMaxG = 2048;   // rulers per row staged (16 KB of shared memory)
+
+template <int BITS, bool BF16>
+__global__ void __launch_bounds__(kDqRowThreads) dequant_row_kernel(
+    const uint32_t* __restrict__ packed, int64_t n, const float* __restrict__ scales,
+    const uint8_t* __restrict__ zeros, int group_size, int64_t G,
+    const int32_t* __restrict__ g_idx, void* __restrict__ out) {
+  __shared__ float2 rul[kDqRowMaxG];
+  const int64_t r = blockIdx.x;
+  for (int64_t g = threadIdx.x; g < G; g += kDqRowThreads)
+    rul[g] = make_float2(scales[r * G + g], (float)zeros[r * G + g]);
+  __syncthreads();
+  const int64_t upr = n / 8;
+  const uint32_t* prow = packed + r * (n * BITS / 32);
+  for (int64_t j = threadIdx.x; j < upr; j += kDqRowThreads) {
+    uint32_t bits24;
+    if (BITS == 4) {
+      bits24 = prow[j];
+    } else {
+      const uint32_t* p = prow + 3 * (j >> 2);
+      switch (j & 3) {
+        case 0: bits24 = p[0] & 0xFFFFFFu; break;
+        case 1: bits24 = (p[0] >> 24) | ((p[1] & 0xFFFFu) << 8); break;
+        case 2: bits24 = (p[1] >> 16) | ((p[2] & 0xFFu) << 16); break;
+        default: bits24 = p[2] >> 8; break;
+      }
+    }
+    const int64_t c0 = 8 * j;
+    int gi[8];
+    if (g_idx) {
+      const int4 ga = __ldg(reinterpret_cast<const int4*>(g_idx + c0));
+      const int4 gb = __ldg(reinterpret_cast<const int4*>(g_idx + c0) + 1);
+      gi[0] = ga.x; gi[1] = ga.y; gi[2] = ga.z; gi[3] = ga.w;
+      gi[4] = gb.x; gi[5] = gb.y; gi[6] = gb.z; gi[7] = gb.w;
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) gi[k] = group_size > 0 ? (int)((c0 + k) / group_size) : 0;
+    }
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float2 sz = rul[gi[k]];
+      const float q = (float)((bits24 >> (BITS * k)) & ((1u << BITS) - 1u));
+      v[k] = __fmul_rn(sz.x, q - sz.y);
+    }
+    if (BF16) {
+      __align__(16) __nv_bfloat16 t[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) t[k] = __float2bfloat16_rn(v[k]);
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + r * n + c0) =
+          *reinterpret_cast<const uint4*>(t);
+    } else {
+      float* o = static_cast<float*>(out) + r * n + c0;
+      reinterpret_cast<float4*>(o)[0] = make_float4(v[0], v[1], v[2], v[3]);
+      reinterpret_cast<float4*>(o)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+  }
+}
+
 // 8 codes of row `prow` starting at column 8 j (int4: word j; int3: the
 // quarter j % 4 of word triple j / 4), code k in bits [BITS k, BITS k + BITS).
 template <int BITS>
@@ -616,6 +681,29 @@ cudaError_t launch_dequant(const uint32_t* packed, int bits, int64_t rows, int64
                            int64_t n_groups, const int32_t* g_idx, void* out, int out_bf16,
                            cudaStream_t s) {
   if (rows == 0) return cudaSuccess;
+  // one CTA per row when the rulers fit its shared memory and every row's
+  // output starts 16-byte aligned (and g_idx, if given, is 16-byte aligned)
+  const bool row_form = n_groups <= kDqRowMaxG && (n * (out_bf16 ? 2 : 4)) % 16 == 0 &&
+                        reinterpret_cast<uintptr_t>(out) % 16 == 0 &&
+                        (!g_idx || reinterpret_cast<uintptr_t>(g_idx) % 16 == 0) &&
+                        rows <= 0x7fffffff;
+  if (row_form) {
+    const unsigned grid = (unsigned)rows;
+    if (bits == 4 && out_bf16)
+      dequant_row_kernel<4, true><<<grid, kDqRowThreads, 0, s>>>(packed, n, scales, zeros,
+                                                                  group_size, n_groups, g_idx, out);
+    else if (bits == 4)
+      dequant_row_kernel<4, false><<<grid, kDqRowThreads, 0, s>>>(packed, n, scales, zeros,
+                                                                   group_size, n_groups, g_idx, out);
+    else if (out_bf16)
+      dequant_row_kernel<3, true><<<grid, kDqRowThreads, 0, s>>>(packed, n, scales, zeros,
+                                                                  group_size, n_groups, g_idx, out);
+    else
+      dequant_row_kernel<3, false><<<grid, kDqRowThreads, 0, s>>>(packed, n, scales, zeros,
+                                                                   group_size, n_groups, g_idx, out);
+    note_launch();
+    return cudaGetLastError();
+  }
   if (bits == 4) {
     const int64_t upr = n / 8, total = rows * upr;
     if (out_bf16)
