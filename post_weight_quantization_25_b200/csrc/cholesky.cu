@@ -184,14 +184,37 @@ __global__ void __launch_bounds__(256) gather_reversed_kernel(
   const int a = blockIdx.x;
   const int pa = perm ? perm[n - 1 - a] : (n - 1 - a);
   const float* src = H + (int64_t)pa * n;
-  for (int j = threadIdx.x; j < n; j += blockDim.x) hrow[j] = src[j];
+  float* dst = A + (int64_t)a * n;
+  // 16-byte row loads and four-column outputs where the rows allow it
+  const bool v4 = (n % 4) == 0 && reinterpret_cast<uintptr_t>(H) % 16 == 0 &&
+                  reinterpret_cast<uintptr_t>(A) % 16 == 0 &&
+                  (!perm || reinterpret_cast<uintptr_t>(perm) % 16 == 0);
+  if (v4) {
+    for (int j = threadIdx.x; j < n / 4; j += blockDim.x)
+      reinterpret_cast<float4*>(hrow)[j] = reinterpret_cast<const float4*>(src)[j];
+  } else {
+    for (int j = threadIdx.x; j < n; j += blockDim.x) hrow[j] = src[j];
+  }
   __syncthreads();
   const float lf = (float)(*lam);
-  float* dst = A + (int64_t)a * n;
-  for (int b = threadIdx.x; b <= a; b += blockDim.x) {
+  const float diag = dead[pa] ? 1.f : hrow[pa];
+  // columns [0, 4 nv) four at a time: column b + i takes perm[n - 1 - b - i],
+  // i.e. the 16-byte group perm[n - 4 - b .. n - 1 - b] read backwards
+  const int nv = v4 ? (a + 1) / 4 : 0;
+  for (int b4 = threadIdx.x; b4 < nv; b4 += blockDim.x) {
+    const int b = 4 * b4;
+    int4 q;
+    if (perm)
+      q = *reinterpret_cast<const int4*>(perm + (n - 4 - b));
+    else
+      q = make_int4(n - 4 - b, n - 3 - b, n - 2 - b, n - 1 - b);
+    float4 v = make_float4(hrow[q.w], hrow[q.z], hrow[q.y], hrow[q.x]);
+    if (b + 3 == a) v.w = diag + lf;
+    *reinterpret_cast<float4*>(dst + b) = v;
+  }
+  for (int b = 4 * nv + threadIdx.x; b <= a; b += blockDim.x) {
     const int pb = perm ? perm[n - 1 - b] : (n - 1 - b);
-    float v = hrow[pb];
-    if (b == a) v = (dead[pa] ? 1.f : v) + lf;
+    const float v = (b == a) ? diag + lf : hrow[pb];
     dst[b] = v;
   }
 }
