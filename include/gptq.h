@@ -317,6 +317,22 @@ int64_t gptq_launch_count(void);
  * a limit out of range. */
 gptq_status gptq_set_wait_gate(const int32_t* gate, int64_t limit_ns);
 
+/* Debug builds only (host; no counterpart in the pages).  The library can be
+ * built a second time as libgptq_b200_debug.so with device-side index checks
+ * (python -m post_weight_quantization_25_b200.build --debug): every kernel
+ * that indexes with a caller-supplied group index (g_idx of gptq_dequant,
+ * gptq_dequant_matvec) or permutation (perm of gptq_quantize_layer,
+ * gptq_gather_columns_u8, gptq_dequant_matvec) tests each index against its
+ * range first, does not use one that is out of range (the value it would
+ * have produced is left 0, so those outputs are undefined), and records the
+ * kind of check that failed.  gptq_device_checks waits for the device
+ * (cudaDeviceSynchronize), writes the recorded kinds to *flags (host) as a
+ * bit set -- 1: a group index out of [0, n_groups), 2: a permutation entry
+ * out of [0, n) -- and clears them.  Release builds do no such checks (those
+ * indices are the caller's to keep in range) and return GPTQ_ERR_UNSUPPORTED;
+ * a debug build returns GPTQ_ERR_INVALID_ARG for flags = NULL. */
+gptq_status gptq_device_checks(uint32_t* flags);
+
 /* Self-test of the division the sweep uses to round w / scale (a
  * correctly rounded binary32 division by Markstein's FMA method, with the
  * reciprocal of the divisor computed once per ruler): out[i] = a[i] / b[i]

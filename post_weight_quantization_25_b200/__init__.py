@@ -38,6 +38,22 @@ def library() -> ctypes.CDLL:
     return _lib.load()
 
 
+def debug_library() -> ctypes.CDLL:
+    """libgptq_b200_debug.so: the same entry points with device-side checks
+    of caller-supplied indices (build it with ``build(debug=True)``)."""
+    return _lib.load(_lib.DEBUG_LIB_PATH)
+
+
+def gptq_device_checks(lib: ctypes.CDLL | None = None) -> int:
+    """The index checks that failed since the last read, as a bit set (1: a
+    group index out of range, 2: a permutation entry out of range), then
+    cleared; waits for the device.  Debug library only."""
+    lib = debug_library() if lib is None else lib
+    flags = ctypes.c_uint32(0)
+    _check(lib.gptq_device_checks(ctypes.byref(flags)), "gptq_device_checks")
+    return int(flags.value)
+
+
 def gptq_status_string(status: int) -> str:
     return library().gptq_status_string(int(status)).decode()
 

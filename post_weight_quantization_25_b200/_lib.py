@@ -8,6 +8,8 @@ import ctypes
 import os
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgptq_b200.so")
+# the same library built with device-side index checks (gptq_device_checks)
+DEBUG_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgptq_b200_debug.so")
 
 GPTQ_OK = 0
 GPTQ_ERR_INVALID_ARG = 1
@@ -28,7 +30,8 @@ EXPORTS = ("gptq_workspace_size", "gptq_hessian_accumulate", "gptq_cholesky_inve
            "gptq_quantize_layer", "gptq_pack_int4", "gptq_pack_int3", "gptq_dequant",
            "gptq_status_string", "gptq_launch_count", "gptq_cholesky_inverse_noalloc",
            "gptq_selftest_division", "gptq_dequant_matvec", "gptq_gather_columns_u8",
-           "gptq_hadamard_rows", "gptq_hadamard_cols", "gptq_set_wait_gate")
+           "gptq_hadamard_rows", "gptq_hadamard_cols", "gptq_set_wait_gate",
+           "gptq_device_checks")
 
 
 class GptqConfig(ctypes.Structure):
@@ -66,6 +69,7 @@ _SIGNATURES = {
     "gptq_hadamard_rows": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _int, _vp, _int, _i64, _vp]),
     "gptq_hadamard_cols": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _int, _vp, _int, _i64, _vp]),
     "gptq_set_wait_gate": (_int, [_vp, _i64]),
+    "gptq_device_checks": (_int, [ctypes.POINTER(ctypes.c_uint32)]),
 }
 
 _LIB = None

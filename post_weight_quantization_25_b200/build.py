@@ -1,6 +1,9 @@
 """Build libgptq_b200.so in place with nvcc for sm_100a.
 
-Usage: python -m post_weight_quantization_25_b200.build   (or build() from Python)
+Usage: python -m post_weight_quantization_25_b200.build [--force] [--debug]
+(or build() from Python).  --debug builds libgptq_b200_debug.so instead: the
+same sources with device-side index checks (-DGPTQ_DEVICE_CHECKS, read back
+by gptq_device_checks).
 """
 from __future__ import annotations
 
@@ -11,6 +14,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libgptq_b200.so")
+DEBUG_LIB = os.path.join(PKG, "libgptq_b200_debug.so")
 SOURCES = ["gptq_api.cu", "hessian_syrk.cu", "cholesky.cu", "sweep.cu", "pack.cu", "hadamard.cu"]
 HEADERS = ["gptq_internal.cuh", "sm100_ptx.cuh", "panel_gemm.cuh", "persist.cuh", "stage.cuh", "chol_diag.cuh",
            "fdiv.cuh"]
@@ -23,10 +27,10 @@ def _nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
     deps.append(os.path.join(ROOT, "include", "gptq.h"))
     return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
@@ -38,18 +42,21 @@ def _flags(verbose: bool) -> list[str]:
     return (["-Xptxas=-v"] + f) if verbose else f
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
     """Compile every source to an object file in parallel (the files share
-    no device symbols), then link the shared library."""
-    if not force and not _stale():
-        return LIB
+    no device symbols), then link the shared library (the checked one with
+    debug=True)."""
+    lib = DEBUG_LIB if debug else LIB
+    if not force and not _stale(lib):
+        return lib
     from concurrent.futures import ThreadPoolExecutor
-    objdir = os.path.join(PKG, "_build")
+    objdir = os.path.join(PKG, "_build_debug" if debug else "_build")
     os.makedirs(objdir, exist_ok=True)
     objs = [os.path.join(objdir, os.path.splitext(f)[0] + ".o") for f in SOURCES]
 
     def compile_one(i: int) -> None:
-        cmd = [_nvcc()] + _flags(verbose) + ["-c", os.path.join(CSRC, SOURCES[i]), "-o", objs[i]]
+        cmd = [_nvcc()] + _flags(verbose) + (["-DGPTQ_DEVICE_CHECKS"] if debug else []) + \
+            ["-c", os.path.join(CSRC, SOURCES[i]), "-o", objs[i]]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
         subprocess.run(cmd, check=True)
@@ -57,12 +64,11 @@ def build(force: bool = False, verbose: bool = False) -> str:
     with ThreadPoolExecutor(max_workers=min(len(SOURCES), os.cpu_count() or 1)) as ex:
         list(ex.map(compile_one, range(len(SOURCES))))
     cmd = [_nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o",
-           LIB + ".tmp"] + objs
+           lib + ".tmp"] + objs
     subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug="--debug" in sys.argv))

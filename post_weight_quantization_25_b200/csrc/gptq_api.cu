@@ -137,6 +137,20 @@ gptq_status gptq_selftest_division(const float* a, const float* b, int64_t count
       gptq::launch_selftest_division(a, b, count, out, static_cast<cudaStream_t>(stream)));
 }
 
+gptq_status gptq_device_checks(uint32_t* flags) {
+#ifdef GPTQ_DEVICE_CHECKS
+  if (!flags) return GPTQ_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return GPTQ_ERR_CUDA;
+  const uint32_t v = gptq::take_device_checks_pack() | gptq::take_device_checks_sweep();
+  if (v == ~0u) return GPTQ_ERR_CUDA;
+  *flags = v;
+  return GPTQ_OK;
+#else
+  (void)flags;
+  return GPTQ_ERR_UNSUPPORTED;
+#endif
+}
+
 const char* gptq_status_string(int status) {
   switch (status) {
     case GPTQ_OK: return "ok";

@@ -26,6 +26,46 @@ struct NvtxScope {
   NvtxScope& operator=(const NvtxScope&) = delete;
 };
 
+// ---- device-side index checks (debug builds)
+// Built with -DGPTQ_DEVICE_CHECKS (libgptq_b200_debug.so), the kernels that
+// index with caller-supplied arrays (a group index g_idx, a permutation)
+// test every such index before they use it; an index out of range is not
+// used (the value it would have produced is left 0) and its kind is OR-ed
+// into a per-translation-unit device word that gptq_device_checks reads.
+// In release builds index_ok is a constant true and costs nothing.
+enum : uint32_t { kCheckGroupIndex = 1u, kCheckPermutation = 2u };
+namespace {
+#ifdef GPTQ_DEVICE_CHECKS
+__device__ uint32_t g_dev_checks;
+#endif
+__device__ __forceinline__ bool index_ok(int64_t i, int64_t lim, uint32_t what) {
+#ifdef GPTQ_DEVICE_CHECKS
+  if (i >= 0 && i < lim) return true;
+  atomicOr(&g_dev_checks, what);
+  return false;
+#else
+  (void)i;
+  (void)lim;
+  (void)what;
+  return true;
+#endif
+}
+// Host: this translation unit's recorded checks, then cleared (0 in release
+// builds).  Synchronous.
+inline uint32_t take_unit_device_checks() {
+#ifdef GPTQ_DEVICE_CHECKS
+  uint32_t v = 0, z = 0;
+  if (cudaMemcpyFromSymbol(&v, g_dev_checks, sizeof(v)) != cudaSuccess) return ~0u;
+  if (cudaMemcpyToSymbol(g_dev_checks, &z, sizeof(z)) != cudaSuccess) return ~0u;
+  return v;
+#else
+  return 0u;
+#endif
+}
+}  // namespace
+uint32_t take_device_checks_pack();
+uint32_t take_device_checks_sweep();
+
 int num_sms();
 // 2-D TMA descriptor (128-byte swizzle, zero fill out of bounds) for a
 // row-major rows x cols matrix of bf16 (bf16 = true) or fp32 elements with a

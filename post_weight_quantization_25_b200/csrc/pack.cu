@@ -141,7 +141,7 @@ __global__ void dequant_kernel(const uint32_t* __restrict__ packed, int64_t unit
   for (int k = 0; k < 8; ++k) {
     const int gi = group_of(c0 + k, group_size, g_idx);
     const float q = (float)((bits24 >> (BITS * k)) & ((1u << BITS) - 1u));
-    v[k] = __fmul_rn(srow[gi], q - (float)zrow[gi]);
+    v[k] = index_ok(gi, G, kCheckGroupIndex) ? __fmul_rn(srow[gi], q - (float)zrow[gi]) : 0.f;
   }
   if (BF16) {
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out) + r * n + c0;
@@ -213,9 +213,13 @@ __global__ void __launch_bounds__(kDqRowThreads) dequant_row_kernel(
     float v[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const float2 sz = rul[gi[k]];
       const float q = (float)((bits24 >> (BITS * k)) & ((1u << BITS) - 1u));
-      v[k] = __fmul_rn(sz.x, q - sz.y);
+      if (index_ok(gi[k], G, kCheckGroupIndex)) {
+        const float2 sz = rul[gi[k]];
+        v[k] = __fmul_rn(sz.x, q - sz.y);
+      } else {
+        v[k] = 0.f;
+      }
     }
     if (BF16) {
       __align__(16) __nv_bfloat16 t[8];
@@ -292,14 +296,16 @@ __global__ void __launch_bounds__(kMvThreads) dequant_matvec_kernel(
     for (int i = threadIdx.x; i < cn; i += kMvThreads) {
       // column c0 + i of the packed row multiplies x[perm[c0 + i]] (codes in
       // sweep order) or x[c0 + i] (original order)
-      const int64_t xc = perm ? (int64_t)perm[c0 + i] : c0 + i;
+      int64_t xc = perm ? (int64_t)perm[c0 + i] : c0 + i;
+      if (!index_ok(xc, n, kCheckPermutation)) xc = 0;
 #pragma unroll
       for (int b = 0; b < B; ++b) {
         const int64_t xi = (int64_t)b * ldx + xc;
         xs[b][i] = XBF16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(x)[xi])
                          : static_cast<const float*>(x)[xi];
       }
-      gs[i] = group_of(c0 + i, group_size, g_idx);
+      const int gsel = group_of(c0 + i, group_size, g_idx);
+      gs[i] = index_ok(gsel, G, kCheckGroupIndex) ? gsel : 0;
     }
     __syncthreads();
     const int units = cn / 8;  // n % 8 == 0 (int4) or n % 32 == 0 (int3)
@@ -496,6 +502,7 @@ __global__ void __launch_bounds__(kGxWarps * 32) dequant_matvec_gidx_kernel(
       const int64_t c = c0 + threadIdx.x + kGxWarps * 32 * j;
       const bool ok = c < n;
       gr[j] = ok ? __ldg(g_idx + c) : 0;
+      if (!index_ok(gr[j], G, kCheckGroupIndex)) gr[j] = 0;
 #pragma unroll
       for (int b = 0; b < B; ++b) {
         const int64_t xi = (int64_t)b * ldx + (ok ? c : 0);
@@ -738,7 +745,10 @@ __global__ void __launch_bounds__(256) gather_columns_u8_kernel(const uint8_t* _
   const int64_t r = blockIdx.x;
   for (int64_t c = threadIdx.x; c < n; c += blockDim.x) srow[c] = src[r * n + c];
   __syncthreads();
-  for (int64_t k = threadIdx.x; k < n; k += blockDim.x) dst[r * n + k] = srow[perm[k]];
+  for (int64_t k = threadIdx.x; k < n; k += blockDim.x) {
+    const int32_t pk = perm[k];
+    dst[r * n + k] = index_ok(pk, n, kCheckPermutation) ? srow[pk] : 0;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -1064,8 +1074,11 @@ __global__ void dq_prep_kernel(const __nv_bfloat16* __restrict__ x, int64_t n, i
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int64_t c0 = 8 * w + k, c1 = 8 * w + k + 4;
-      o[2 * k] = xb[perm ? perm[c0] : c0];
-      o[2 * k + 1] = xb[perm ? perm[c1] : c1];
+      int64_t s0 = perm ? perm[c0] : c0, s1 = perm ? perm[c1] : c1;
+      if (!index_ok(s0, n, kCheckPermutation)) s0 = 0;
+      if (!index_ok(s1, n, kCheckPermutation)) s1 = 0;
+      o[2 * k] = xb[s0];
+      o[2 * k + 1] = xb[s1];
     }
     *reinterpret_cast<uint4*>(xp + b * n + 8 * w) = *reinterpret_cast<const uint4*>(o);
   }
@@ -1196,5 +1209,7 @@ cudaError_t launch_dequant_matvec(const uint32_t* packed, int bits, int64_t rows
   }
   return cudaGetLastError();
 }
+
+uint32_t take_device_checks_pack() { return take_unit_device_checks(); }
 
 }  // namespace gptq

@@ -235,7 +235,9 @@ __device__ __forceinline__ float warp_max(float v) {
 
 __global__ void pos_kernel(const int32_t* __restrict__ perm, int n, int32_t* __restrict__ pos) {
   const int k = blockIdx.x * blockDim.x + threadIdx.x;
-  if (k < n) pos[perm ? perm[k] : k] = k;
+  if (k >= n) return;
+  const int pk = perm ? perm[k] : k;
+  if (index_ok(pk, n, kCheckPermutation)) pos[pk] = k;
 }
 
 // One CTA per row: Wf[r][k] = dead[perm[k]] ? 0 : W[r][perm[k]]; per-row ruler
@@ -273,14 +275,18 @@ __global__ void __launch_bounds__(256) gather_w_kernel(
     for (int k4 = threadIdx.x; k4 < n / 4; k4 += blockDim.x) {
       const int4 k = perm ? reinterpret_cast<const int4*>(perm)[k4]
                           : make_int4(4 * k4, 4 * k4 + 1, 4 * k4 + 2, 4 * k4 + 3);
-      const float4 v = make_float4(wrow[k.x], wrow[k.y], wrow[k.z], wrow[k.w]);
+      const float4 v = make_float4(index_ok(k.x, n, kCheckPermutation) ? wrow[k.x] : 0.f,
+                                   index_ok(k.y, n, kCheckPermutation) ? wrow[k.y] : 0.f,
+                                   index_ok(k.z, n, kCheckPermutation) ? wrow[k.z] : 0.f,
+                                   index_ok(k.w, n, kCheckPermutation) ? wrow[k.w] : 0.f);
       reinterpret_cast<float4*>(dst)[k4] = v;
       mn = fminf(fminf(mn, fminf(v.x, v.y)), fminf(v.z, v.w));
       mx = fmaxf(fmaxf(mx, fmaxf(v.x, v.y)), fmaxf(v.z, v.w));
     }
   } else {
     for (int k = threadIdx.x; k < n; k += blockDim.x) {
-      const float v = wrow[perm ? perm[k] : k];
+      const int pk = perm ? perm[k] : k;
+      const float v = index_ok(pk, n, kCheckPermutation) ? wrow[pk] : 0.f;
       dst[k] = v;
       mn = fminf(mn, v);
       mx = fmaxf(mx, v);
@@ -888,7 +894,12 @@ __global__ void __launch_bounds__(256) unpermute_kernel(const uint8_t* __restric
   __syncthreads();
   if (vout) {
     for (int c4 = threadIdx.x; c4 < n / 4; c4 += blockDim.x) {
-      const int4 k = reinterpret_cast<const int4*>(pos)[c4];
+      int4 k = reinterpret_cast<const int4*>(pos)[c4];
+      // positions come from the caller's permutation (checked in debug builds)
+      if (!index_ok(k.x, n, kCheckPermutation)) k.x = 0;
+      if (!index_ok(k.y, n, kCheckPermutation)) k.y = 0;
+      if (!index_ok(k.z, n, kCheckPermutation)) k.z = 0;
+      if (!index_ok(k.w, n, kCheckPermutation)) k.w = 0;
       reinterpret_cast<uint32_t*>(cdst)[c4] = (uint32_t)crow[k.x] | ((uint32_t)crow[k.y] << 8) |
                                               ((uint32_t)crow[k.z] << 16) |
                                               ((uint32_t)crow[k.w] << 24);
@@ -897,7 +908,8 @@ __global__ void __launch_bounds__(256) unpermute_kernel(const uint8_t* __restric
     }
   } else {
     for (int c = threadIdx.x; c < n; c += blockDim.x) {
-      const int k = pos[c];
+      int k = pos[c];
+      if (!index_ok(k, n, kCheckPermutation)) k = 0;
       cdst[c] = crow[k];
       if (Wq) wdst[c] = srow[k];
     }
@@ -1228,5 +1240,7 @@ cudaError_t launch_quantize_layer(const void* W, int wt, int64_t rows64, int64_t
   }
   return cudaGetLastError();
 }
+
+uint32_t take_device_checks_sweep() { return take_unit_device_checks(); }
 
 }  // namespace gptq

@@ -172,3 +172,25 @@ def test_consumer_calls_with_nothing_to_do_or_bad_arguments(lib):
     assert lib.gptq_gather_columns_u8(None, 0, 64, None, None, None) == 0
     assert lib.gptq_gather_columns_u8(p, 4, 64, p, p, None) == 1  # src == dst
     assert lib.gptq_gather_columns_u8(p, 4, 0, p, ctypes.c_void_p(0x2000), None) == 1
+
+
+@pytest.fixture(scope="module")
+def debug_lib():
+    if not os.path.exists(_lib.DEBUG_LIB_PATH):
+        from post_weight_quantization_25_b200 import build
+        build.build(debug=True)
+    return _lib.load(_lib.DEBUG_LIB_PATH)
+
+
+def test_debug_library_exports_every_declared_symbol(debug_lib):
+    for name in _declared():
+        assert hasattr(debug_lib, name), name
+
+
+def test_device_checks_only_in_the_debug_build(lib, debug_lib):
+    flags = ctypes.c_uint32(7)
+    # release: no checks compiled in (nothing touches the device)
+    assert lib.gptq_device_checks(ctypes.byref(flags)) == _lib.GPTQ_ERR_UNSUPPORTED
+    assert flags.value == 7
+    # debug: argument check before any device call
+    assert debug_lib.gptq_device_checks(None) == _lib.GPTQ_ERR_INVALID_ARG
