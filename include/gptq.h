@@ -18,8 +18,9 @@
  *    scratch buffer is a caller workspace sized by gptq_workspace_size),
  *    creates no stream, and keeps no state between calls apart from the
  *    launch counter read by gptq_launch_count, the calling thread's wait
- *    gate (gptq_set_wait_gate, a test hook) and a per-device cache of one
- *    occupancy query.  A call given a side stream creates four CUDA events
+ *    gate (gptq_set_wait_gate, a test hook), a per-device cache of one
+ *    occupancy query and, in the debug build only, the words of failed
+ *    index checks (gptq_device_checks).  A call given a side stream creates four CUDA events
  *    for its enqueue and destroys them before it returns.
  *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
  *    legacy default stream).  The returned status covers argument checks and
