@@ -96,7 +96,10 @@ __global__ void __launch_bounds__(kRowsWarps * 32) hadamard_rows_kernel(
 // loads and the column passes of the warps land on distinct banks, at most
 // two-way in the second pass), then warp w transforms token column w
 // (in == out is allowed: the tile is read in full before it is written).
-constexpr int kColsTok = 16;
+// 32 tokens per tile: each feature row is read and written as 64-byte
+// pieces of bf16 (measured 0.90 against 0.97 ms with 16-token tiles on the
+// 28672 x 16384 rotation, same results)
+constexpr int kColsTok = 32;
 
 template <int VPL, typename TI, typename TO>
 __global__ void __launch_bounds__(kColsTok * 32) hadamard_cols_kernel(
