@@ -22,6 +22,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <type_traits>
 
 #include "gptq_internal.cuh"
 
@@ -178,6 +179,93 @@ __global__ void __launch_bounds__(kColsTok * 32) hadamard_cols_kernel(
   }
 }
 
+// R X for blocks of 1024 features with bf16 input and output, 64 tokens per
+// CTA: the tile is staged as bf16 token pairs (one 32-bit word per feature
+// and pair), so each feature row moves as one 128-byte piece; the fp32
+// values between the two passes go through a per-warp scratch instead of the
+// tile.  Warp w transforms token pairs w and w + 16, one token at a time,
+// with the same operations in the same order as hadamard_cols_kernel<32>
+// (signs, high index bits, low index bits, scale, one rounding to bf16), so
+// the results are the same bit for bit.  Full 64-token tiles only.
+constexpr int kC64Tok = 64;
+constexpr int kC64Warps = 16;
+constexpr int kC64WP = 33;                 // words per tile row (32 pairs + 1: no bank conflicts)
+constexpr size_t kC64Smem =
+    sizeof(uint32_t) * 1024 * kC64WP + sizeof(float) * kC64Warps * 32 * 33 + sizeof(float) * 1024;
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__global__ void __launch_bounds__(kC64Warps * 32) hadamard_cols1024_bf16_kernel(
+    const __nv_bfloat16* in, int64_t ld_in, __nv_bfloat16* out, int64_t ld_out,
+    const float* __restrict__ signs, float scale) {
+  extern __shared__ __align__(16) uint32_t c64_smem[];
+  uint32_t* tile = c64_smem;                                       // [1024][kC64WP]
+  float* scr_all = reinterpret_cast<float*>(tile + 1024 * kC64WP); // [warp][32][33]
+  float* sgn = scr_all + kC64Warps * 32 * 33;                      // [1024]
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int64_t f0 = (int64_t)blockIdx.y * 1024, t0 = (int64_t)blockIdx.x * kC64Tok;
+  for (int f = tid; f < 1024; f += kC64Warps * 32) sgn[f] = __ldg(signs + f0 + f);
+  // load: piece p = (row p / 8, 8 tokens 8 (p % 8) ..): 16 bytes from global,
+  // four words into the row (a warp covers 4 rows x 128 bytes)
+#pragma unroll 4
+  for (int j = 0; j < 1024 * 8 / (kC64Warps * 32); ++j) {
+    const int p = tid + kC64Warps * 32 * j;
+    const int f = p >> 3, c = p & 7;
+    const uint4 v = *reinterpret_cast<const uint4*>(in + (f0 + f) * ld_in + t0 + 8 * c);
+    uint32_t* d = tile + f * kC64WP + 4 * c;
+    d[0] = v.x;
+    d[1] = v.y;
+    d[2] = v.z;
+    d[3] = v.w;
+  }
+  __syncthreads();
+  float* scr = scr_all + w * 32 * 33;
+  for (int kp = 0; kp < 2; ++kp) {
+    const int k = w + kC64Warps * kp;   // token pair 2k, 2k + 1
+    float res[2][32];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float v[32];
+      // pass one: lane l holds features l + 32 i (high index bits in registers)
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const uint32_t word = tile[(lane + 32 * i) * kC64WP + k];
+        v[i] = (half ? bf16_hi(word) : bf16_lo(word)) * sgn[lane + 32 * i];
+      }
+      fwht_lane<32>(v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) scr[i * 33 + lane] = v[i];
+      __syncwarp();
+      // pass two: lane l holds features 32 l + i (low index bits)
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = scr[lane * 33 + i];
+      fwht_lane<32>(v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) scr[lane * 33 + i] = v[i] * scale;
+      __syncwarp();
+      // back to lane l holding features l + 32 i
+#pragma unroll
+      for (int i = 0; i < 32; ++i) res[half][i] = scr[i * 33 + lane];
+      __syncwarp();
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const uint32_t lo = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(res[0][i]));
+      const uint32_t hi = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(res[1][i]));
+      tile[(lane + 32 * i) * kC64WP + k] = lo | (hi << 16);
+    }
+  }
+  __syncthreads();
+#pragma unroll 4
+  for (int j = 0; j < 1024 * 8 / (kC64Warps * 32); ++j) {
+    const int p = tid + kC64Warps * 32 * j;
+    const int f = p >> 3, c = p & 7;
+    const uint32_t* s = tile + f * kC64WP + 4 * c;
+    *reinterpret_cast<uint4*>(out + (f0 + f) * ld_out + t0 + 8 * c) = make_uint4(s[0], s[1], s[2], s[3]);
+  }
+}
+
 unsigned cdiv(int64_t a, int64_t b) { return (unsigned)((a + b - 1) / b); }
 
 template <int VPL, typename TI, typename TO>
@@ -194,6 +282,29 @@ template <int VPL, typename TI, typename TO>
 cudaError_t cols_launch(const void* in, int64_t ld_in, void* out, int64_t ld_out, int64_t n,
                         int64_t ntok, const float* signs, float scale, cudaStream_t s) {
   constexpr int B = 32 * VPL;
+  if constexpr (VPL == 32 && std::is_same<TI, __nv_bfloat16>::value &&
+                std::is_same<TO, __nv_bfloat16>::value) {
+    // whole 64-token tiles by the bf16-tile kernel, the rest (if any) below
+    const int64_t nfull = ntok / kC64Tok * kC64Tok;
+    const bool ok = nfull > 0 && reinterpret_cast<uintptr_t>(in) % 16 == 0 &&
+                    reinterpret_cast<uintptr_t>(out) % 16 == 0 && (ld_in * 2) % 16 == 0 &&
+                    (ld_out * 2) % 16 == 0;
+    if (ok) {
+      cudaError_t e = cudaFuncSetAttribute(hadamard_cols1024_bf16_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)kC64Smem);
+      if (e != cudaSuccess) return e;
+      const dim3 grid((unsigned)(nfull / kC64Tok), (unsigned)(n / 1024));
+      hadamard_cols1024_bf16_kernel<<<grid, kC64Warps * 32, kC64Smem, s>>>(
+          static_cast<const __nv_bfloat16*>(in), ld_in, static_cast<__nv_bfloat16*>(out), ld_out,
+          signs, scale);
+      note_launch();
+      if ((e = cudaGetLastError()) != cudaSuccess || nfull == ntok) return e;
+      in = static_cast<const __nv_bfloat16*>(in) + nfull;
+      out = static_cast<__nv_bfloat16*>(out) + nfull;
+      ntok -= nfull;
+    }
+  }
   const size_t smem = (size_t)B * (kColsTok + 1) * sizeof(float);
   if (smem > 48 * 1024) {
     const cudaError_t e = cudaFuncSetAttribute(hadamard_cols_kernel<VPL, TI, TO>,

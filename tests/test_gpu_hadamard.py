@@ -60,7 +60,9 @@ def test_rows_match_oracle(rows, n, b, it, ot):
 @pytest.mark.parametrize("n,ntok,b,it,ot", [
     (1024, 37, 1024, torch.bfloat16, torch.bfloat16), (2048, 16, 1024, torch.float32, torch.float32),
     (96, 1, 32, torch.float32, torch.float32), (512, 100, 256, torch.bfloat16, torch.float32),
-    (3072, 33, 512, torch.float32, torch.bfloat16), (128, 64, 64, torch.bfloat16, torch.bfloat16)])
+    (3072, 33, 512, torch.float32, torch.bfloat16), (128, 64, 64, torch.bfloat16, torch.bfloat16),
+    # bf16 blocks of 1024: whole 64-token tiles on the bf16-tile kernel, then a ragged tail
+    (2048, 150, 1024, torch.bfloat16, torch.bfloat16), (1024, 128, 1024, torch.bfloat16, torch.bfloat16)])
 def test_cols_match_oracle(n, ntok, b, it, ot):
     g = torch.Generator().manual_seed(n + ntok + b)
     X = torch.randn(n, ntok, generator=g).to(it)
@@ -74,11 +76,13 @@ def test_cols_match_oracle(n, ntok, b, it, ot):
     assert np.all(err <= bound), float(np.max(err / bound))
 
 
-def test_strided_and_in_place():
+@pytest.mark.parametrize("ntok", [40, 200])
+def test_strided_and_in_place(ntok):
     """Row strides wider than a row (views into a larger buffer) and in-place
-    rotation give the same values as the contiguous out-of-place call."""
+    rotation give the same values as the contiguous out-of-place call (200
+    tokens: three whole 64-token tiles and a tail)."""
     g = torch.Generator().manual_seed(5)
-    n, ntok, b = 2048, 40, 1024
+    n, b = 2048, 1024
     s = _signs(n, 9).cuda()
     big = torch.randn(n, ntok + 24, generator=g).to(torch.bfloat16).cuda()
     X = big[:, 8:8 + ntok]
