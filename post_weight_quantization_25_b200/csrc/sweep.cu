@@ -499,29 +499,38 @@ __device__ __forceinline__ void sweep_block_body(
     float ev_sub[kSub];   // the sub-block's error terms (every lane of the team)
     float e_own[NS];      // this lane's own columns' error terms
     uint32_t cw = 0u;     // this lane's own columns' codes, one byte each
+    // Every lane of the team rounds the step's column itself, so the error
+    // term needs no exchange: xk is column jj's current value, and xn is
+    // column jj + 1's value before step jj's repair, which its owner sends
+    // one step ahead (the send is off the chain of dependent steps).  Both
+    // are the owner's register values bit for bit.
+    float xk = wrow[c0];
+    float xn = wrow[c0 + 1];
 #pragma unroll
     for (int k = 0; k < kSub; ++k) {
       const int jj = c0 + k;
       const int s = k / L, ko = k % L;   // the step's slot, and its owner lane
-      // every lane rounds its own value of slot s; the owner's is used
-      const float x = cur[s];
+      const float x = xk;
       float qv = rintf(md_div(x, md)) + zf;
       qv = fminf(fmaxf(qv, 0.f), maxq);
       const float wh = __fmul_rn(scale, qv - zf);
       const float e = x - wh;
       const float ev = e * rd[jj];
-      const float err = __shfl_sync(0xffffffffu, ev, ko, L);
-      ev_sub[k] = err;
+      ev_sub[k] = ev;
       const bool own = (q == ko);
       loss = own ? fmaf(e * e, hrd2[jj], loss) : loss;
       cur[s] = own ? wh : cur[s];
       e_own[s] = own ? ev : e_own[s];
       cw |= own ? (((uint32_t)qv) << (8 * s)) : 0u;
-      // repair this lane's later columns of the sub-block
       const float* urow = Ud + jj * kBlock + c0;
+      // the next column, repaired by this step: the chain to the next step
+      if (k + 1 < kSub) xk = fmaf(-ev, urow[k + 1], xn);
+      // repair this lane's later columns of the sub-block
 #pragma unroll
       for (int s2 = s; s2 < NS; ++s2)
-        if (s2 > s || q > ko) cur[s2] = fmaf(-err, urow[L * s2 + q], cur[s2]);
+        if (s2 > s || q > ko) cur[s2] = fmaf(-ev, urow[L * s2 + q], cur[s2]);
+      // column jj + 2 after this step's repair, from its owner
+      if (k + 2 < kSub) xn = __shfl_sync(0xffffffffu, cur[(k + 2) / L], (k + 2) % L, L);
     }
     // the sub-block's results, staged for the block's coalesced write-out:
     // w_hat in place of the columns just swept (no later step reads them),
