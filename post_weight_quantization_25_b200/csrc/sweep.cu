@@ -321,9 +321,10 @@ __global__ void __launch_bounds__(256) gather_w_kernel(
 // Wf in shared memory.  The block is swept in sub-blocks of kSub = 16
 // columns: lane q of a team loads columns q, q + 4, q + 8, q + 12 of the
 // sub-block into registers, and the 16 column steps run fully unrolled:
-// every lane rounds its own value of the step's slot, the owner of the
-// column (lane k % 4) is broadcast inside the team, and each lane repairs
-// its later columns of the sub-block.  Then the sub-block's 16 error terms
+// every lane of the team rounds the step's column itself (its value is
+// carried from step to step; the owner of the column after next sends it
+// one step ahead), and each lane repairs its later columns of the
+// sub-block.  Then the sub-block's 16 error terms
 // (all lanes hold them) update the rest of the block in shared memory, lane
 // q taking the 4-column chunks q, q + 4, ... (a rolled rank-16 update).
 // Every column receives fmaf(-err_j, U[j][c], w) for j = 0, 1, ... in column
