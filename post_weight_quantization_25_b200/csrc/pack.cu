@@ -166,39 +166,30 @@ __global__ void dequant_kernel(const uint32_t* __restrict__ packed, int64_t unit
   }
 }
 
-// The same dequantization with one CTA per row: the row's rulers are staged
-// once in shared memory as (scale, zero) pairs, so each value costs one
-// shared-memory read for its ruler instead of two global ones, and the
-// group index of 8 columns comes in two 16-byte loads.  Same arithmetic and
-// bytes out as dequant_kernel.
+// The same dequantization with one CTA per RPC rows: the rows' rulers are
+// staged once in shared memory as (scale, zero) pairs, so each value costs
+// one shared-memory read for its ruler instead of two global ones, and the
+// group index of 8 columns comes in two 16-byte loads that serve all RPC
+// rows (g_idx is read once per RPC rows, not once per row).  Same
+// arithmetic and bytes out as dequant_kernel.
 constexpr int kDqRowThreads = 128;
-constexpr int kDqRowMaxG = 2048;   // rulers per row staged (16 KB of shared memory)
+constexpr int kDqRowMaxG = 2048;   // rulers staged per CTA (16 KB of shared memory)
+constexpr int kDqRowsPerCta = 4;   // RPC when RPC x G rulers fit
 
-template <int BITS, bool BF16>
+template <int BITS, bool BF16, int RPC>
 __global__ void __launch_bounds__(kDqRowThreads) dequant_row_kernel(
-    const uint32_t* __restrict__ packed, int64_t n, const float* __restrict__ scales,
+    const uint32_t* __restrict__ packed, int64_t rows, int64_t n, const float* __restrict__ scales,
     const uint8_t* __restrict__ zeros, int group_size, int64_t G,
     const int32_t* __restrict__ g_idx, void* __restrict__ out) {
-  __shared__ float2 rul[kDqRowMaxG];
-  const int64_t r = blockIdx.x;
-  for (int64_t g = threadIdx.x; g < G; g += kDqRowThreads)
-    rul[g] = make_float2(scales[r * G + g], (float)zeros[r * G + g]);
+  __shared__ float2 rul[kDqRowMaxG];   // [RPC][G]
+  const int64_t r0 = (int64_t)blockIdx.x * RPC;
+  const int nr = (int)(rows - r0 < RPC ? rows - r0 : RPC);
+  // the rows r0 .. r0 + nr - 1 are contiguous in scales and zeros
+  for (int64_t e = threadIdx.x; e < nr * G; e += kDqRowThreads)
+    rul[e] = make_float2(scales[r0 * G + e], (float)zeros[r0 * G + e]);
   __syncthreads();
   const int64_t upr = n / 8;
-  const uint32_t* prow = packed + r * (n * BITS / 32);
   for (int64_t j = threadIdx.x; j < upr; j += kDqRowThreads) {
-    uint32_t bits24;
-    if (BITS == 4) {
-      bits24 = prow[j];
-    } else {
-      const uint32_t* p = prow + 3 * (j >> 2);
-      switch (j & 3) {
-        case 0: bits24 = p[0] & 0xFFFFFFu; break;
-        case 1: bits24 = (p[0] >> 24) | ((p[1] & 0xFFFFu) << 8); break;
-        case 2: bits24 = (p[1] >> 16) | ((p[2] & 0xFFu) << 16); break;
-        default: bits24 = p[2] >> 8; break;
-      }
-    }
     const int64_t c0 = 8 * j;
     int gi[8];
     if (g_idx) {
@@ -210,27 +201,46 @@ __global__ void __launch_bounds__(kDqRowThreads) dequant_row_kernel(
 #pragma unroll
       for (int k = 0; k < 8; ++k) gi[k] = group_size > 0 ? (int)((c0 + k) / group_size) : 0;
     }
-    float v[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float q = (float)((bits24 >> (BITS * k)) & ((1u << BITS) - 1u));
-      if (index_ok(gi[k], G, kCheckGroupIndex)) {
-        const float2 sz = rul[gi[k]];
-        v[k] = __fmul_rn(sz.x, q - sz.y);
+    for (int rho = 0; rho < RPC; ++rho) {
+      if (rho >= nr) break;
+      const int64_t r = r0 + rho;
+      const uint32_t* prow = packed + r * (n * BITS / 32);
+      uint32_t bits24;
+      if (BITS == 4) {
+        bits24 = prow[j];
       } else {
-        v[k] = 0.f;
+        const uint32_t* p = prow + 3 * (j >> 2);
+        switch (j & 3) {
+          case 0: bits24 = p[0] & 0xFFFFFFu; break;
+          case 1: bits24 = (p[0] >> 24) | ((p[1] & 0xFFFFu) << 8); break;
+          case 2: bits24 = (p[1] >> 16) | ((p[2] & 0xFFu) << 16); break;
+          default: bits24 = p[2] >> 8; break;
+        }
       }
-    }
-    if (BF16) {
-      __align__(16) __nv_bfloat16 t[8];
+      const float2* rr = rul + rho * G;
+      float v[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) t[k] = __float2bfloat16_rn(v[k]);
-      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + r * n + c0) =
-          *reinterpret_cast<const uint4*>(t);
-    } else {
-      float* o = static_cast<float*>(out) + r * n + c0;
-      reinterpret_cast<float4*>(o)[0] = make_float4(v[0], v[1], v[2], v[3]);
-      reinterpret_cast<float4*>(o)[1] = make_float4(v[4], v[5], v[6], v[7]);
+      for (int k = 0; k < 8; ++k) {
+        const float q = (float)((bits24 >> (BITS * k)) & ((1u << BITS) - 1u));
+        if (index_ok(gi[k], G, kCheckGroupIndex)) {
+          const float2 sz = rr[gi[k]];
+          v[k] = __fmul_rn(sz.x, q - sz.y);
+        } else {
+          v[k] = 0.f;
+        }
+      }
+      if (BF16) {
+        __align__(16) __nv_bfloat16 t[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) t[k] = __float2bfloat16_rn(v[k]);
+        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + r * n + c0) =
+            *reinterpret_cast<const uint4*>(t);
+      } else {
+        float* o = static_cast<float*>(out) + r * n + c0;
+        reinterpret_cast<float4*>(o)[0] = make_float4(v[0], v[1], v[2], v[3]);
+        reinterpret_cast<float4*>(o)[1] = make_float4(v[4], v[5], v[6], v[7]);
+      }
     }
   }
 }
@@ -695,19 +705,23 @@ cudaError_t launch_dequant(const uint32_t* packed, int bits, int64_t rows, int64
                         (!g_idx || reinterpret_cast<uintptr_t>(g_idx) % 16 == 0) &&
                         rows <= 0x7fffffff;
   if (row_form) {
-    const unsigned grid = (unsigned)rows;
-    if (bits == 4 && out_bf16)
-      dequant_row_kernel<4, true><<<grid, kDqRowThreads, 0, s>>>(packed, n, scales, zeros,
-                                                                  group_size, n_groups, g_idx, out);
-    else if (bits == 4)
-      dequant_row_kernel<4, false><<<grid, kDqRowThreads, 0, s>>>(packed, n, scales, zeros,
-                                                                   group_size, n_groups, g_idx, out);
-    else if (out_bf16)
-      dequant_row_kernel<3, true><<<grid, kDqRowThreads, 0, s>>>(packed, n, scales, zeros,
-                                                                  group_size, n_groups, g_idx, out);
-    else
-      dequant_row_kernel<3, false><<<grid, kDqRowThreads, 0, s>>>(packed, n, scales, zeros,
-                                                                   group_size, n_groups, g_idx, out);
+    // RPC rows per CTA when their rulers fit the staged table
+    const bool multi = n_groups * kDqRowsPerCta <= kDqRowMaxG;
+    const int rpc = multi ? kDqRowsPerCta : 1;
+    const unsigned grid = (unsigned)((rows + rpc - 1) / rpc);
+#define GPTQ_DQ_ROW(B, F, R)                                                              \
+  dequant_row_kernel<B, F, R><<<grid, kDqRowThreads, 0, s>>>(packed, rows, n, scales, zeros, \
+                                                             group_size, n_groups, g_idx, out)
+    if (bits == 4 && out_bf16) {
+      if (multi) GPTQ_DQ_ROW(4, true, kDqRowsPerCta); else GPTQ_DQ_ROW(4, true, 1);
+    } else if (bits == 4) {
+      if (multi) GPTQ_DQ_ROW(4, false, kDqRowsPerCta); else GPTQ_DQ_ROW(4, false, 1);
+    } else if (out_bf16) {
+      if (multi) GPTQ_DQ_ROW(3, true, kDqRowsPerCta); else GPTQ_DQ_ROW(3, true, 1);
+    } else {
+      if (multi) GPTQ_DQ_ROW(3, false, kDqRowsPerCta); else GPTQ_DQ_ROW(3, false, 1);
+    }
+#undef GPTQ_DQ_ROW
     note_launch();
     return cudaGetLastError();
   }
