@@ -227,6 +227,9 @@ def cpu_sample(wl, W, X, tok_sample: int, row_sample: int):
     from oracle import gptq_oracle as O
 
     t_all = time.perf_counter()
+    # a sample never larger than the workload (nor than the inputs drawn for it)
+    tok_sample = min(tok_sample, wl.ntok, X.shape[1])
+    row_sample = min(row_sample, wl.rows, W.shape[0])
     Xs = X[:, :tok_sample].float().cpu().numpy()
     Ws = W[:row_sample].float().cpu().numpy().astype(np.float64)
     t0 = time.perf_counter()

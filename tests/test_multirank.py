@@ -74,3 +74,30 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
 
     bench.run_reference(A(), rank=1, world=2)
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_on_rank_zero(capsys):
+    """The oracle arm's JSON line: the contract's keys, the host-only e2e leg
+    (no copies) and a sample no larger than the workload."""
+    sys.path.insert(0, ROOT)
+    import json
+    import bench
+
+    class A:
+        steps, warmup, workload, tokens = 1, 0, "layer256", 0
+
+    bench.run_reference(A(), rank=0, world=1)
+    lines = capsys.readouterr().out.strip().splitlines()
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "impl", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1
+    assert "H on 2048 of 2048 tokens (time x1)" in cb["sample"]
+    assert "64 of 256 rows (time x4)" in cb["sample"]
